@@ -1,0 +1,341 @@
+"""Benchmark: WKV fwd+bwd channel-tokens/s and achieved HBM GB/s on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libwkv|reference]
+                [--workload rwkv169m|rwkv1b5_bf16|longctx|decode14b]
+
+A step is one pass of the whole hot path over one batch of the workload:
+``wkv_forward`` (writing the checkpoints) followed by ``wkv_backward`` on the
+same inputs, through the C ABI, inputs resident in HBM.  The default
+workload is the RWKV-4 169M-shaped layer (B8 T1024 C768 fp32, seeded
+synthetic inputs).  L2 is flushed (a 2x-L2 buffer is written) before every
+timed step, outside the timed events; each step is bracketed by CUDA events
+on the launching stream and the per-step times are summed.
+
+Multi-GPU (torchrun): every rank runs an independent replica of the workload
+on its own GPU (the operator has no cross-sequence exchange; weak scaling);
+ranks are timed on the device and the maximum over ranks is reported.
+
+``--impl reference`` times the float64 CPU oracle (the only reference this
+operator has) on a bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rwkv_linear_rnn_b200 import workloads  # noqa: E402
+
+# algorithmic bytes per channel-token (per channel-step for the decode step)
+ALG_BYTES = {("fwd", "f32"): 12, ("fwd", "bf16"): 6, ("bwd", "f32"): 20, ("bwd", "bf16"): 10,
+             ("step", "f32"): 36}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def cpu_baseline(wl_name: str, min_seconds: float = 10.0):
+    """Time the oracle (float64 recurrence fwd + reverse bwd) on the host."""
+    import oracle
+    wl = workloads.WORKLOADS[wl_name]
+    if wl_name == "rwkv169m":
+        inp = workloads.generate(wl)
+        sample = "full rwkv169m workload (B8 T1024 C768) fwd+bwd, repeated"
+    else:  # a channel slice of the big workloads keeps the sample bounded
+        C = 256
+        inp = workloads.generate(wl, C=C, T=min(wl.T, 4096), grad=True)
+        sample = f"{wl_name} with C={C}, T={inp['T']} fwd+bwd, repeated"
+    args = [np.asarray(inp[n], np.float64) for n in ("w", "u", "k", "v", "gy")]
+    units = inp["B"] * inp["T"] * inp["C"]
+    times = []
+    t_end = time.perf_counter() + min_seconds
+    while time.perf_counter() < t_end or len(times) < 3:
+        t0 = time.perf_counter()
+        oracle.fwd_recur(*args[:4], want_y=True)
+        oracle.bwd_recur(*args)
+        times.append(time.perf_counter() - t0)
+    med = statistics.median(times)
+    return {"value": units / med, "unit": "channel-tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{sample} x{len(times)}, median"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    cb = cpu_baseline(args.workload, min_seconds=max(1.0, 2.0 * args.steps))
+    wl = workloads.WORKLOADS[args.workload]
+    line = {"metric": "WKV fwd+bwd channel-tokens/s (HBM GB/s and % of roofline alongside)",
+            "value": cb["value"], "unit": "channel-tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": wl.channel_tokens / cb["value"] * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "impl": "reference",
+            "config": {"workload": args.workload, "B": wl.B, "T": wl.T, "C": wl.C},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "channel-tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_libwkv(args):
+    import torch
+    import rwkv_linear_rnn_b200 as W
+    from rwkv_linear_rnn_b200 import abi
+
+    ws_n, rank, local = dist_env()
+    dist = None
+    if ws_n > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = workloads.WORKLOADS[args.workload]
+    if "bwd" not in wl.ops:
+        raise SystemExit(f"workload {args.workload} has no backward; pick a fwd+bwd workload")
+    inp = workloads.generate(wl, seed=wl.seed + 1000 * rank)
+    B, T, C = inp["B"], inp["T"], inp["C"]
+    dt = W.WKV_BF16 if inp["dtype"] == "bf16" else W.WKV_F32
+    tdt = torch.bfloat16 if dt == W.WKV_BF16 else torch.float32
+
+    def to_dev(name):
+        if dt == W.WKV_BF16 and name in ("k", "v", "gy"):
+            return torch.from_numpy(inp[name + "_bits"].view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(inp[name]).to(dev)
+
+    w, u, k, v, gy = (to_dev(n) for n in ("w", "u", "k", "v", "gy"))
+    y = torch.empty_like(k)
+    gk = torch.empty_like(k)
+    gv = torch.empty_like(v)
+    gw = torch.empty(C, device=dev)
+    gu = torch.empty(C, device=dev)
+    ckpt = torch.empty(W.wkv_ckpt_size(B, T, C) // 4, device=dev)
+    nws = W.wkv_workspace_size(W.WKV_OP_BACKWARD, B, T, C, dt)
+    wsb = torch.zeros(nws, dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_w = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        # write 2x L2 (evicts everything), then read another 2x L2 so the
+        # lines left behind are clean: the timed kernels neither hit their
+        # inputs in L2 nor pay for write-backs of the flush
+        flush_w.zero_()
+        flush_r.sum()
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    P = lambda t: t.data_ptr()
+
+    def fwd():
+        abi.check(abi.wkv_forward(B, T, C, dt, P(w), P(u), P(k), P(v), 0, P(y), 0, P(ckpt),
+                                  P(wsb), nws, sp))
+
+    def bwd():
+        abi.check(abi.wkv_backward(B, T, C, dt, P(w), P(u), P(k), P(v), P(gy), 0, P(ckpt),
+                                   P(gw), P(gu), P(gk), P(gv), P(wsb), nws, sp))
+
+    for _ in range(args.warmup):
+        flush_l2()
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    if abi.wkv_get_status(P(wsb), sp) != 0:
+        raise SystemExit("device-side status error during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(K):
+        flush_l2()
+        ev[i][0].record(stream)
+        fwd()
+        ev[i][1].record(stream)
+        bwd()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist:
+        dist.barrier()
+    t_fwd = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    t_bwd = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    total_ms = sum(t_fwd) + sum(t_bwd)
+    if dist:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    status = abi.wkv_get_status(P(wsb), sp)
+
+    # e2e: host buffers (pinned), copies in the timed region, through the same ABI
+    e2e = None
+    if not args.no_e2e:
+        hk = k.cpu().pin_memory(); hv = v.cpu().pin_memory(); hg = gy.cpu().pin_memory()
+        hy = torch.empty_like(hk).pin_memory(); hgk = torch.empty_like(hk).pin_memory()
+        hgv = torch.empty_like(hk).pin_memory()
+        hgw = torch.empty(C).pin_memory(); hgu = torch.empty(C).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hg))
+        d2h = sum(t.numel() * t.element_size() for t in (hy, hgk, hgv, hgw, hgu))
+        ee = []
+        n_e2e = max(3, min(K, 10))
+        for i in range(n_e2e + 1):
+            e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+            gy.copy_(hg, non_blocking=True)
+            fwd(); bwd()
+            hy.copy_(y, non_blocking=True); hgk.copy_(gk, non_blocking=True)
+            hgv.copy_(gv, non_blocking=True); hgw.copy_(gw, non_blocking=True)
+            hgu.copy_(gu, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i > 0:
+                ee.append(e0.elapsed_time(e1))
+        e2e_ms = statistics.median(ee)
+        if dist:
+            tt = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": ws_n * B * T * C / (e2e_ms * 1e-3), "unit": "channel-tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if rank == 0:
+        units = B * T * C
+        hbm, peak_kind = peaks()
+        fwd_ms = statistics.mean(t_fwd)
+        bwd_ms = statistics.mean(t_bwd)
+        fb = ALG_BYTES[("fwd", inp["dtype"])] * units
+        bb = ALG_BYTES[("bwd", inp["dtype"])] * units
+        bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9
+        fwd_gbs = fb / (fwd_ms * 1e-3) / 1e9
+        step_ms = total_ms / K
+        line = {
+            "metric": "WKV fwd+bwd channel-tokens/s (HBM GB/s and % of roofline alongside)",
+            "value": ws_n * units / (step_ms * 1e-3), "unit": "channel-tokens/s",
+            "n_gpus": ws_n, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": inp["dtype"], "data": "synthetic (seeded, BASELINE distributions)",
+            "config": {"workload": args.workload, "B": B, "T": T, "C": C,
+                       "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
+                       "l2": "flushed before every timed step (2x L2 write + 2x L2 read, outside events)"},
+            "roofline": {"bound": "hbm", "kernel": "wkv_backward (bwd_chunked + reduce_wu)",
+                         "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": bwd_gbs / hbm, "traffic": None, "peak_kind": peak_kind},
+            "fwd": {"ms": fwd_ms, "gbs": fwd_gbs, "frac": fwd_gbs / hbm,
+                    "channel_tokens_per_s": units / (fwd_ms * 1e-3)},
+            "bwd": {"ms": bwd_ms, "gbs": bwd_gbs, "frac": bwd_gbs / hbm},
+            "fwd_bwd_gbs": (fb + bb) / (step_ms * 1e-3) / 1e9,
+            "clocks": clocks, "gpu_launches": 3 * K, "device_status": status,
+        }
+        if e2e:
+            line["e2e"] = e2e
+        if not args.no_cpu_baseline and ws_n == 1:
+            line["cpu_baseline"] = cpu_baseline(args.workload, min_seconds=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="libwkv", choices=["libwkv", "reference"])
+    ap.add_argument("--workload", default="rwkv169m")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_libwkv(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,217 @@
+/*
+ * wkv.h -- C ABI of libwkv, the RWKV-4 WKV time-mixing operator on NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operator (RWKV paper review, "[논문 리뷰] Reinvention RNNs for the
+ * Transformer Era: RWKV", section "WKV 연산자", eq. wkv_t; 0-based t, decay
+ * written as the signed per-step log-decay w, normally w = -exp(time_decay)):
+ *
+ *   y_t = ( sum_{i<t} e^{(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
+ *       / ( sum_{i<t} e^{(t-1-i) w + k_i}     + e^{u + k_t}     )
+ *
+ * independently for every batch row b and channel c (w, u are per channel).
+ * Its RNN form (same review, section "RNN-유사추론", eq. WKV_t) keeps per
+ * channel the hidden sums A_t = sum_{i<t} e^{(t-1-i) w + k_i} v_i and
+ * B_t = sum_{i<t} e^{(t-1-i) w + k_i}, so y_t = (A_t + e^{u+k_t} v_t) /
+ * (B_t + e^{u+k_t}) and A_{t+1} = e^w A_t + e^{k_t} v_t (same for B).
+ *
+ * Three calls follow the review's two execution modes:
+ *   wkv_forward   time-parallel mode ("Transformer-유사학습": the whole
+ *                 sequence at once, WKV evaluated as a scan over time);
+ *   wkv_backward  gradients of a scalar loss for the same mode;
+ *   wkv_step      RNN mode ("RNN-유사추론" / "자기 회귀 디코딩" steps 4 and 7):
+ *                 one token per sequence against a stored state.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *   allocates and frees nothing and keeps no global state; scratch lives in a
+ *   caller-provided workspace.
+ * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *   NULL = legacy default stream).  The return value covers host-side
+ *   argument checks and the launch itself; conditions detected on the device
+ *   (a bounded wait that gave up) are read later with wkv_get_status().
+ *   A call that returns an error has launched nothing, except WKV_ERR_CUDA,
+ *   which reports a failed launch.
+ * - Layout: k, v, y, grad_y, grad_k, grad_v are [B, T, C] row-major with C
+ *   fastest (the (B, T, d) layout of the sequence model); w, u, grad_w,
+ *   grad_u are [C] float32.
+ * - Element type of k, v, y, grad_y, grad_k, grad_v: WKV_F32 or WKV_BF16
+ *   (bfloat16 storage, float32 arithmetic, round-to-nearest-even stores).
+ *   w, u, states, checkpoints and parameter gradients are always float32.
+ * - State: three float32 planes [3][B][C] holding (a, b, p) per (b, c), with
+ *   A = a * e^p and B = b * e^p.  The form is not unique; any (a, b, p) with
+ *   b >= 0 is accepted.  The empty state is (0, 0, -inf); p = -inf is
+ *   accepted as input.  State outputs are normalised so that p is the
+ *   largest exponent seen (b >= 1 after at least one token).
+ * - w and u must be finite.  NaN or Inf in k, v, grad_y propagate to the
+ *   outputs; they are not checked.
+ * - Alignment: every tensor pointer must be aligned to its element size;
+ *   misaligned pointers give WKV_ERR_UNSUPPORTED.  Any C >= 1 is accepted.
+ * - Sizes: B, C >= 1 and T >= 0 (N >= 1 for wkv_step); B*T*C < 2^62;
+ *   T < 2^31.  T = 0 copies state_in to state_out (if given).
+ * - Not thread-safe per workspace: calls that share a workspace must be
+ *   ordered on one stream.
+ */
+#ifndef LIBWKV_WKV_H
+#define LIBWKV_WKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WKV_VERSION 100 /* 1.0.0 */
+
+/* Element type of the [B, T, C] tensors. */
+typedef enum { WKV_F32 = 0, WKV_BF16 = 1 } wkv_dtype;
+
+/* Return codes. */
+typedef enum {
+  WKV_OK = 0,
+  WKV_ERR_INVALID_ARG = -1, /* required pointer NULL, size out of range, bad dtype/op */
+  WKV_ERR_UNSUPPORTED = -2, /* misaligned pointer or unsupported aliasing */
+  WKV_ERR_WORKSPACE = -3,   /* workspace NULL, misaligned or smaller than required */
+  WKV_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+  WKV_ERR_TIMEOUT = -5      /* device side: a bounded cross-block wait gave up */
+} wkv_status;
+
+/* Operation selector for wkv_workspace_size. */
+enum { WKV_OP_FORWARD = 0, WKV_OP_BACKWARD = 1, WKV_OP_STEP = 2 };
+
+/* Kernel selector (wkv_options.kernel). */
+enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2 };
+
+/*
+ * Optional knobs for the *_ex calls.  A NULL options pointer, or all fields
+ * zero, means the defaults.  None of them changes the result beyond
+ * floating-point rounding order.
+ *   kernel      WKV_KERNEL_AUTO picks by problem shape; SEQUENTIAL runs one
+ *               thread per (b, c) chain over all of T; CHUNKED splits T into
+ *               chunks joined by a single-pass decoupled look-back scan.
+ *   spin_limit  polls a block makes on one predecessor's flag before it gives
+ *               up with WKV_ERR_TIMEOUT (0 = default, about one second).
+ *   test_hold_first_chunk
+ *               test hook: blocks of the first chunk in scan order never
+ *               publish their results, so the blocks that depend on them must
+ *               run out their wait limit.  Results are then invalid and
+ *               wkv_get_status() returns WKV_ERR_TIMEOUT.
+ */
+typedef struct {
+  int kernel;
+  int test_hold_first_chunk;
+  int64_t spin_limit;
+} wkv_options;
+
+/*
+ * Bytes of workspace the given operation needs (0 for WKV_OP_STEP, which
+ * needs none).  The workspace is any device buffer of at least that size,
+ * aligned to 256 bytes, ZERO-FILLED ONCE before its first use (cudaMemset or
+ * wkv_workspace_init); the library keeps it consistent from then on.  One
+ * workspace sized for the largest call may serve forward and backward calls
+ * of any shape, as long as those calls are ordered on one stream.
+ * Returns 0 for invalid arguments.
+ */
+size_t wkv_workspace_size(int op, int64_t B, int64_t T, int64_t C, int dtype);
+
+/* Zero-fills a workspace on `stream` (asynchronous). */
+int wkv_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Bytes of the forward checkpoint buffer: the state at every 64th token,
+ * float32 [ceil(T/64)][3][B][C].  Its contents are private to the library
+ * (the exponent is stored in base 2); it only carries the forward's
+ * per-chunk states to wkv_backward so the backward does not rescan.
+ */
+size_t wkv_ckpt_size(int64_t B, int64_t T, int64_t C);
+
+/*
+ * wkv_forward -- time-parallel forward.
+ *   B, T, C    batch, sequence length, channels.
+ *   dtype      element type of k, v, y.
+ *   w, u       [C] float32 decay (per-step log-decay, normally < 0) and bonus.
+ *   k, v       [B, T, C] inputs.
+ *   state_in   [3][B][C] state before token 0, or NULL for the empty state.
+ *   y          [B, T, C] output; must not overlap k or v.
+ *   state_out  [3][B][C] state after token T-1, or NULL.  May equal state_in.
+ *   ckpt       wkv_ckpt_size() bytes to receive the checkpoints for
+ *              wkv_backward, or NULL.
+ *   ws         workspace of wkv_workspace_size(WKV_OP_FORWARD, ...) bytes.
+ * Errors: INVALID_ARG (NULL w/u/k/v/y, bad sizes or dtype), UNSUPPORTED
+ * (misaligned, y overlapping k/v), WORKSPACE, CUDA.
+ */
+int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                const float *u, const void *k, const void *v, const float *state_in,
+                void *y, float *state_out, float *ckpt, void *ws, size_t ws_bytes,
+                void *stream);
+
+int wkv_forward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                   const float *u, const void *k, const void *v,
+                   const float *state_in, void *y, float *state_out, float *ckpt,
+                   void *ws, size_t ws_bytes, void *stream, const wkv_options *opt);
+
+/*
+ * wkv_backward -- gradients of a scalar loss L given grad_y = dL/dy.
+ *   state_in   the state the forward started from, or NULL (empty).
+ *   ckpt       the checkpoints the forward wrote for the same inputs, or NULL
+ *              to have them recomputed here (one extra read of k and v).
+ *   grad_w     [C] float32, receives dL/dw summed over the batch (overwritten).
+ *              A caller holding time_decay (w = -exp(time_decay)) gets
+ *              dL/dtime_decay = grad_w * w.
+ *   grad_u     [C] float32, receives dL/du summed over the batch (overwritten).
+ *   grad_k, grad_v  [B, T, C] outputs (element type dtype); must not overlap
+ *              the inputs.
+ *   ws         workspace of wkv_workspace_size(WKV_OP_BACKWARD, ...) bytes.
+ * The state after the last token receives no gradient, and state_in gets
+ * none.  gw and gu are reduced in a fixed order, so repeated calls give
+ * bit-identical results.
+ * Errors: as wkv_forward (NULL grad_y/grad_w/grad_u/grad_k/grad_v is
+ * INVALID_ARG).
+ */
+int wkv_backward(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                 const float *u, const void *k, const void *v, const void *grad_y,
+                 const float *state_in, const float *ckpt, float *grad_w,
+                 float *grad_u, void *grad_k, void *grad_v, void *ws,
+                 size_t ws_bytes, void *stream);
+
+int wkv_backward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                    const float *u, const void *k, const void *v,
+                    const void *grad_y, const float *state_in, const float *ckpt,
+                    float *grad_w, float *grad_u, void *grad_k, void *grad_v,
+                    void *ws, size_t ws_bytes, void *stream, const wkv_options *opt);
+
+/*
+ * wkv_step -- one RNN-mode token for N independent sequences (float32).
+ *   k_t, v_t   [N, C] inputs of this token.
+ *   state_in   [3][N][C] state before the token (required).
+ *   y_t        [N, C] output.
+ *   state_out  [3][N][C] state after the token; may equal state_in (update in
+ *              place); must not partly overlap it.
+ * Equivalent to wkv_forward with T = 1.  Needs no workspace.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+int wkv_step(int64_t N, int64_t C, const float *w, const float *u,
+             const float *k_t, const float *v_t, const float *state_in, float *y_t,
+             float *state_out, void *stream);
+
+/*
+ * Waits for `stream`, then returns and clears the device-side status word of
+ * the workspace: WKV_OK, or WKV_ERR_TIMEOUT if a bounded wait of an earlier
+ * call on it gave up (its results are then invalid).  WKV_ERR_CUDA if the
+ * synchronisation or the copy failed, WKV_ERR_WORKSPACE for a NULL ws.
+ */
+int wkv_get_status(void *ws, void *stream);
+
+/* Static string for a return code ("unknown status" otherwise). */
+const char *wkv_strerror(int status);
+
+/* WKV_VERSION of the built library. */
+int wkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBWKV_WKV_H */

@@ -1,0 +1,201 @@
+"""libwkv: the RWKV-4 WKV time-mixing operator on NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/wkv.h``.  The functions in
+``abi`` carry the C names and take raw device pointers (ints) -- argument
+marshalling only.  The tensor helpers below (``forward``, ``backward``,
+``step``, ``WKV``) take torch CUDA tensors, allocate outputs with torch, and
+call the same entry points; PyTorch provides memory and streams only, every
+step of the operator runs in the library's CUDA kernels.
+
+The library is required: importing this package fails loudly if
+``libwkv.so`` is missing (build it with ``python -m rwkv_linear_rnn_b200.build``).
+There is no CPU or PyTorch fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from . import abi
+from .abi import (WKV_BF16, WKV_F32, WKV_KERNEL_AUTO, WKV_KERNEL_CHUNKED, WKV_KERNEL_SEQUENTIAL,
+                  WKV_OP_BACKWARD, WKV_OP_FORWARD, WKV_OP_STEP, WKVError, wkv_ckpt_size,
+                  wkv_strerror, wkv_version, wkv_workspace_size)
+
+__all__ = [
+    "abi", "WKVError", "WKV_F32", "WKV_BF16", "WKV_OP_FORWARD", "WKV_OP_BACKWARD", "WKV_OP_STEP",
+    "WKV_KERNEL_AUTO", "WKV_KERNEL_SEQUENTIAL", "WKV_KERNEL_CHUNKED", "Workspace", "forward",
+    "backward", "step", "WKV", "wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror",
+    "wkv_version", "library_path",
+]
+
+
+def library_path() -> str:
+    return abi.LIB_PATH
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return WKV_F32
+    if t.dtype == torch.bfloat16:
+        return WKV_BF16
+    raise TypeError(f"k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return 0 if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must be on a CUDA device")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+class Workspace:
+    """A zero-initialised device workspace that grows on demand.
+
+    One workspace may serve forward and backward calls of any shape, as long
+    as they are ordered on one stream.
+    """
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf = None
+
+    def get(self, op, B, T, C, dtype):
+        torch = _torch()
+        need = wkv_workspace_size(op, B, T, C, dtype)
+        if need == 0:
+            return None, 0
+        if self.buf is None or self.buf.numel() < need:
+            # zero-filled: the library requires a zeroed workspace before first use
+            self.buf = torch.zeros(need + 256, dtype=torch.uint8, device=self.device or "cuda")
+        return self.buf, self.buf.numel()
+
+    def status(self, stream=None) -> int:
+        """Device-side status of earlier calls (waits for the stream); clears it."""
+        if self.buf is None:
+            return 0
+        return abi.wkv_get_status(self.buf.data_ptr(), _stream(stream))
+
+
+_default_ws = {}
+
+
+def _ws_for(device, ws):
+    if ws is not None:
+        return ws
+    key = str(device)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def forward(w, u, k, v, state_in=None, *, want_state=False, want_ckpt=False, y=None,
+            workspace=None, stream=None, kernel=WKV_KERNEL_AUTO):
+    """y = WKV(w, u, k, v) for k, v [B, T, C]; optionally the final state and
+    the checkpoints for ``backward``.  Returns (y, state_out, ckpt)."""
+    torch = _torch()
+    _check_cuda(w, u, k, v, state_in, y)
+    B, T, C = k.shape
+    dt = _dtype_code(k)
+    if y is None:
+        y = torch.empty_like(k)
+    state_out = torch.empty((3, B, C), dtype=torch.float32, device=k.device) if want_state else None
+    ckpt = None
+    if want_ckpt:
+        n = wkv_ckpt_size(B, T, C) // 4
+        ckpt = torch.empty(max(n, 1), dtype=torch.float32, device=k.device)
+    ws = _ws_for(k.device, workspace)
+    buf, nbytes = ws.get(WKV_OP_FORWARD, B, T, C, dt)
+    opts = abi.Options(kernel=kernel)
+    abi.check(abi.wkv_forward_ex(B, T, C, dt, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(state_in),
+                                 _ptr(y), _ptr(state_out), _ptr(ckpt), _ptr(buf), nbytes,
+                                 _stream(stream), opts))
+    return y, state_out, ckpt
+
+
+def backward(w, u, k, v, grad_y, state_in=None, ckpt=None, *, workspace=None, stream=None,
+             kernel=WKV_KERNEL_AUTO):
+    """Gradients (grad_w [C], grad_u [C], grad_k, grad_v) of L given grad_y."""
+    torch = _torch()
+    _check_cuda(w, u, k, v, grad_y, state_in, ckpt)
+    B, T, C = k.shape
+    dt = _dtype_code(k)
+    gw = torch.empty(C, dtype=torch.float32, device=k.device)
+    gu = torch.empty(C, dtype=torch.float32, device=k.device)
+    gk = torch.empty_like(k)
+    gv = torch.empty_like(v)
+    ws = _ws_for(k.device, workspace)
+    buf, nbytes = ws.get(WKV_OP_BACKWARD, B, T, C, dt)
+    opts = abi.Options(kernel=kernel)
+    abi.check(abi.wkv_backward_ex(B, T, C, dt, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(grad_y),
+                                  _ptr(state_in), _ptr(ckpt), _ptr(gw), _ptr(gu), _ptr(gk),
+                                  _ptr(gv), _ptr(buf), nbytes, _stream(stream), opts))
+    return gw, gu, gk, gv
+
+
+def step(w, u, k_t, v_t, state, *, y=None, state_out=None, stream=None):
+    """One RNN-mode token for N sequences.  ``state_out`` defaults to updating
+    ``state`` in place.  Returns (y_t, state_out)."""
+    torch = _torch()
+    _check_cuda(w, u, k_t, v_t, state, y, state_out)
+    N, C = k_t.shape
+    if y is None:
+        y = torch.empty_like(k_t)
+    if state_out is None:
+        state_out = state
+    abi.check(abi.wkv_step(N, C, _ptr(w), _ptr(u), _ptr(k_t), _ptr(v_t), _ptr(state), _ptr(y),
+                           _ptr(state_out), _stream(stream)))
+    return y, state_out
+
+
+class WKV:
+    """torch.autograd.Function wrapper: y = WKV.apply(w, u, k, v)."""
+
+    _fn = None
+
+    @classmethod
+    def apply(cls, w, u, k, v):
+        if cls._fn is None:
+            torch = _torch()
+
+            class _F(torch.autograd.Function):
+                @staticmethod
+                def forward(ctx, w, u, k, v):
+                    w, u, k, v = (t.contiguous() for t in (w, u, k, v))
+                    y, _, ck = forward(w, u, k, v, want_ckpt=True)
+                    ctx.save_for_backward(w, u, k, v, ck)
+                    return y
+
+                @staticmethod
+                def backward(ctx, gy):
+                    w, u, k, v, ck = ctx.saved_tensors
+                    gw, gu, gk, gv = backward(w, u, k, v, gy.contiguous(), ckpt=ck)
+                    return gw, gu, gk, gv
+
+            cls._fn = _F
+        return cls._fn.apply(w, u, k, v)
+
+
+def wkv(w, u, k, v):
+    """Differentiable WKV: y [B, T, C] from w, u [C] and k, v [B, T, C]."""
+    return WKV.apply(w, u, k, v)

@@ -1,0 +1,128 @@
+"""ctypes declarations of the libwkv C ABI (``include/wkv.h``).
+
+Each function keeps its C name and signature; pointers are passed as Python
+ints (device addresses), streams as ``cudaStream_t`` ints.  Loading fails
+loudly if ``libwkv.so`` has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwkv.so")
+
+WKV_F32, WKV_BF16 = 0, 1
+WKV_OK, WKV_ERR_INVALID_ARG, WKV_ERR_UNSUPPORTED, WKV_ERR_WORKSPACE, WKV_ERR_CUDA, \
+    WKV_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+WKV_OP_FORWARD, WKV_OP_BACKWARD, WKV_OP_STEP = 0, 1, 2
+WKV_KERNEL_AUTO, WKV_KERNEL_SEQUENTIAL, WKV_KERNEL_CHUNKED = 0, 1, 2
+
+# Every symbol the header declares, in declaration order.
+EXPORTS = (
+    "wkv_workspace_size", "wkv_workspace_init", "wkv_ckpt_size", "wkv_forward", "wkv_forward_ex",
+    "wkv_backward", "wkv_backward_ex", "wkv_step", "wkv_get_status", "wkv_strerror",
+    "wkv_version",
+)
+
+
+class Options(ctypes.Structure):
+    """wkv_options: kernel selector, test hook, look-back wait limit."""
+    _fields_ = [("kernel", ctypes.c_int), ("test_hold_first_chunk", ctypes.c_int),
+                ("spin_limit", ctypes.c_int64)]
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libwkv.so not found at {LIB_PATH}; build it with "
+                      "`python -m rwkv_linear_rnn_b200.build` (nvcc, sm_100a)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_i64, _int, _sz, _p = ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+_opt = ctypes.POINTER(Options)
+
+_SIGS = {
+    "wkv_workspace_size": (_sz, [_int, _i64, _i64, _i64, _int]),
+    "wkv_workspace_init": (_int, [_p, _sz, _p]),
+    "wkv_ckpt_size": (_sz, [_i64, _i64, _i64]),
+    "wkv_forward": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "wkv_forward_ex": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p,
+                              _opt]),
+    "wkv_backward": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
+                            _p, _sz, _p]),
+    "wkv_backward_ex": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
+                               _p, _p, _sz, _p, _opt]),
+    "wkv_step": (_int, [_i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "wkv_get_status": (_int, [_p, _p]),
+    "wkv_strerror": (ctypes.c_char_p, [_int]),
+    "wkv_version": (_int, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class WKVError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        super().__init__(f"libwkv error {status}: {wkv_strerror(status)}")
+
+
+def _opts(o):
+    return None if o is None else ctypes.byref(o)
+
+
+def wkv_workspace_size(op, B, T, C, dtype):
+    return lib.wkv_workspace_size(op, B, T, C, dtype)
+
+
+def wkv_workspace_init(ws, ws_bytes, stream):
+    return lib.wkv_workspace_init(ws, ws_bytes, stream)
+
+
+def wkv_ckpt_size(B, T, C):
+    return lib.wkv_ckpt_size(B, T, C)
+
+
+def wkv_forward(B, T, C, dtype, w, u, k, v, state_in, y, state_out, ckpt, ws, ws_bytes, stream):
+    return lib.wkv_forward(B, T, C, dtype, w, u, k, v, state_in, y, state_out, ckpt, ws, ws_bytes,
+                           stream)
+
+
+def wkv_forward_ex(B, T, C, dtype, w, u, k, v, state_in, y, state_out, ckpt, ws, ws_bytes, stream,
+                   opt=None):
+    return lib.wkv_forward_ex(B, T, C, dtype, w, u, k, v, state_in, y, state_out, ckpt, ws,
+                              ws_bytes, stream, _opts(opt))
+
+
+def wkv_backward(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u, grad_k,
+                 grad_v, ws, ws_bytes, stream):
+    return lib.wkv_backward(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u,
+                            grad_k, grad_v, ws, ws_bytes, stream)
+
+
+def wkv_backward_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u, grad_k,
+                    grad_v, ws, ws_bytes, stream, opt=None):
+    return lib.wkv_backward_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u,
+                               grad_k, grad_v, ws, ws_bytes, stream, _opts(opt))
+
+
+def wkv_step(N, C, w, u, k_t, v_t, state_in, y_t, state_out, stream):
+    return lib.wkv_step(N, C, w, u, k_t, v_t, state_in, y_t, state_out, stream)
+
+
+def wkv_get_status(ws, stream):
+    return lib.wkv_get_status(ws, stream)
+
+
+def wkv_strerror(status):
+    return lib.wkv_strerror(status).decode()
+
+
+def wkv_version():
+    return lib.wkv_version()
+
+
+def check(rc: int) -> None:
+    if rc != WKV_OK:
+        raise WKVError(rc)

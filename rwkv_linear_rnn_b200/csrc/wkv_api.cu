@@ -1,0 +1,290 @@
+// wkv_api.cu -- C ABI of libwkv (declared in include/wkv.h): argument
+// checks, workspace layout and kernel selection.  Every step of the
+// operator runs in the kernels of wkv_forward.cu, wkv_backward.cu and
+// wkv_step.cu; this file only validates and launches.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/wkv.h"
+#include "wkv_internal.cuh"
+
+namespace wkv {
+cudaError_t launch_forward(const FwdArgs &a, int dtype, bool chunked, cudaStream_t st);
+cudaError_t launch_backward(const BwdArgs &a, int dtype, float *gw, float *gu, cudaStream_t st);
+cudaError_t launch_step(const StepArgs &a, bool vec, int num_sms, cudaStream_t st);
+int64_t fwd_chunk_tokens();
+}  // namespace wkv
+
+using namespace wkv;
+
+namespace {
+
+constexpr int64_t kDefaultSpin = 1000000;  // polls of ~1 us backoff: about one second
+constexpr int64_t kSeqMinChains = 148 * 1024;  // chains that fill B200 with one thread each
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline size_t esize(int dtype) { return dtype == WKV_BF16 ? 2 : 4; }
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+  return x < y + nb && y < x + na;
+}
+
+// Sizes: B, C >= 1, 0 <= T < 2^31, B*T*C < 2^62 (checked without overflow).
+bool sizes_ok(int64_t B, int64_t T, int64_t C) {
+  if (B < 1 || C < 1 || T < 0 || T >= (int64_t(1) << 31)) return false;
+  const int64_t lim = int64_t(1) << 62;
+  if (B > lim / C) return false;
+  const int64_t BC = B * C;
+  if (T > 0 && BC > lim / T) return false;
+  return true;
+}
+
+struct Layout {
+  size_t flags, desc, ckpt, part, total;
+  int64_t nct, nchains, nchunks_f, nchunks_b;
+};
+
+// Workspace: [256 B header][flags][descriptors][ckpt (backward)][partials
+// (backward)].  The flag/descriptor region is sized for the larger of the
+// forward and backward tilings so one workspace serves both.
+Layout layout(int op, int64_t B, int64_t T, int64_t C) {
+  Layout L{};
+  L.nct = cdiv(C, 32);
+  L.nchains = B * L.nct;
+  L.nchunks_f = cdiv(T, fwd_chunk_tokens());
+  L.nchunks_b = cdiv(T, kCkpt);
+  const int64_t tiles = L.nchains * (L.nchunks_f > L.nchunks_b ? L.nchunks_f : L.nchunks_b);
+  size_t off = sizeof(WsHeader);
+  L.flags = off;
+  off = align_up(off + sizeof(unsigned) * (size_t)tiles, 256);
+  L.desc = off;
+  off = align_up(off + sizeof(float) * kDescFloats * (size_t)tiles, 256);
+  L.ckpt = L.part = 0;
+  if (op == WKV_OP_BACKWARD) {
+    L.ckpt = off;
+    off = align_up(off + sizeof(float) * 3 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
+    L.part = off;
+    off = align_up(off + sizeof(float) * 2 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
+  }
+  L.total = off;
+  return L;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+bool pick_chunked(const wkv_options *opt, int64_t B, int64_t T, int64_t C) {
+  const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
+  if (kernel == WKV_KERNEL_SEQUENTIAL) return false;
+  if (kernel == WKV_KERNEL_CHUNKED) return true;
+  // Enough independent chains to fill the GPU, or too short to split.
+  return !(B * C >= kSeqMinChains || T <= 2 * fwd_chunk_tokens());
+}
+
+int64_t spin_of(const wkv_options *opt) {
+  return (opt && opt->spin_limit > 0) ? opt->spin_limit : kDefaultSpin;
+}
+
+int check_forward_args(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                       const void *k, const void *v, const float *state_in, const void *y,
+                       const float *state_out, const float *ckpt) {
+  if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_INVALID_ARG;
+  if (!sizes_ok(B, T, C)) return WKV_ERR_INVALID_ARG;
+  if (!w || !u) return WKV_ERR_INVALID_ARG;
+  if (T > 0 && (!k || !v)) return WKV_ERR_INVALID_ARG;
+  const size_t es = esize(dtype);
+  if (!aligned(w, 4) || !aligned(u, 4) || !aligned(k, es) || !aligned(v, es) ||
+      !aligned(y, es) || !aligned(state_in, 4) || !aligned(state_out, 4) || !aligned(ckpt, 4))
+    return WKV_ERR_UNSUPPORTED;
+  const size_t nb = (size_t)(B * T * C) * es;
+  if (overlaps(y, nb, k, nb) || overlaps(y, nb, v, nb)) return WKV_ERR_UNSUPPORTED;
+  const size_t sb = 3 * sizeof(float) * (size_t)(B * C);
+  if (state_in && state_out && state_in != state_out && overlaps(state_in, sb, state_out, sb))
+    return WKV_ERR_UNSUPPORTED;
+  return WKV_OK;
+}
+
+int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                 const void *k, const void *v, const float *state_in, void *y, float *state_out,
+                 float *ckpt, void *ws, size_t ws_bytes, cudaStream_t st, const wkv_options *opt) {
+  if (T == 0) {
+    // No tokens: the state passes through unchanged (the sequential kernel
+    // with T = 0 only converts state_in, or the empty state, to state_out).
+    if (!state_out) return WKV_OK;
+    FwdArgs a{};
+    a.B = B; a.T = 0; a.C = C; a.w = w; a.u = u; a.state_in = state_in; a.state_out = state_out;
+    return launch_forward(a, dtype, false, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  }
+  const Layout L = layout(WKV_OP_FORWARD, B, T, C);
+  const bool chunked = pick_chunked(opt, B, T, C);
+  if (chunked) {
+    if (!ws || !aligned(ws, 256)) return WKV_ERR_WORKSPACE;
+    if (ws_bytes < L.total) return WKV_ERR_WORKSPACE;
+  }
+  FwdArgs a{};
+  a.B = B; a.T = T; a.C = C; a.w = w; a.u = u; a.k = k; a.v = v;
+  a.state_in = state_in; a.y = y; a.state_out = state_out; a.ckpt = ckpt;
+  char *base = static_cast<char *>(ws);
+  a.hdr = reinterpret_cast<WsHeader *>(base);
+  a.flags = base ? reinterpret_cast<unsigned *>(base + L.flags) : nullptr;
+  a.desc = base ? reinterpret_cast<float *>(base + L.desc) : nullptr;
+  a.nct = L.nct; a.nchains = L.nchains; a.nchunks = L.nchunks_f;
+  a.spin_limit = spin_of(opt);
+  a.hold_first = opt ? opt->test_hold_first_chunk : 0;
+  return launch_forward(a, dtype, chunked, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t wkv_workspace_size(int op, int64_t B, int64_t T, int64_t C, int dtype) {
+  if (dtype != WKV_F32 && dtype != WKV_BF16) return 0;
+  if (!sizes_ok(B, T, C)) return 0;
+  if (op == WKV_OP_STEP) return 0;
+  if (op != WKV_OP_FORWARD && op != WKV_OP_BACKWARD) return 0;
+  return layout(op, B, T, C).total;
+}
+
+int wkv_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+  if (!ws) return WKV_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+size_t wkv_ckpt_size(int64_t B, int64_t T, int64_t C) {
+  if (!sizes_ok(B, T, C)) return 0;
+  return sizeof(float) * 3 * (size_t)(B * C) * (size_t)cdiv(T, kCkpt);
+}
+
+int wkv_forward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                   const void *k, const void *v, const float *state_in, void *y,
+                   float *state_out, float *ckpt, void *ws, size_t ws_bytes, void *stream,
+                   const wkv_options *opt) {
+  int rc = check_forward_args(B, T, C, dtype, w, u, k, v, state_in, y, state_out, ckpt);
+  if (rc != WKV_OK) return rc;
+  if (T > 0 && !y) return WKV_ERR_INVALID_ARG;
+  return forward_impl(B, T, C, dtype, w, u, k, v, state_in, y, state_out, ckpt, ws, ws_bytes,
+                      (cudaStream_t)stream, opt);
+}
+
+int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                const void *k, const void *v, const float *state_in, void *y, float *state_out,
+                float *ckpt, void *ws, size_t ws_bytes, void *stream) {
+  return wkv_forward_ex(B, T, C, dtype, w, u, k, v, state_in, y, state_out, ckpt, ws, ws_bytes,
+                        stream, nullptr);
+}
+
+int wkv_backward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                    const void *k, const void *v, const void *grad_y, const float *state_in,
+                    const float *ckpt, float *grad_w, float *grad_u, void *grad_k, void *grad_v,
+                    void *ws, size_t ws_bytes, void *stream, const wkv_options *opt) {
+  int rc = check_forward_args(B, T, C, dtype, w, u, k, v, state_in, nullptr, nullptr, ckpt);
+  if (rc != WKV_OK) return rc;
+  if (!grad_w || !grad_u) return WKV_ERR_INVALID_ARG;
+  if (T > 0 && (!grad_y || !grad_k || !grad_v)) return WKV_ERR_INVALID_ARG;
+  const size_t es = esize(dtype);
+  if (!aligned(grad_y, es) || !aligned(grad_k, es) || !aligned(grad_v, es) ||
+      !aligned(grad_w, 4) || !aligned(grad_u, 4))
+    return WKV_ERR_UNSUPPORTED;
+  const size_t nb = (size_t)(B * T * C) * es;
+  const void *ins[3] = {k, v, grad_y};
+  for (const void *in : ins)
+    if (overlaps(grad_k, nb, in, nb) || overlaps(grad_v, nb, in, nb)) return WKV_ERR_UNSUPPORTED;
+  if (overlaps(grad_k, nb, grad_v, nb) || overlaps(grad_w, 4 * C, grad_u, 4 * C))
+    return WKV_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (T == 0) {
+    if (cudaMemsetAsync(grad_w, 0, sizeof(float) * C, st) != cudaSuccess ||
+        cudaMemsetAsync(grad_u, 0, sizeof(float) * C, st) != cudaSuccess)
+      return WKV_ERR_CUDA;
+    return WKV_OK;
+  }
+  const Layout L = layout(WKV_OP_BACKWARD, B, T, C);
+  if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return WKV_ERR_WORKSPACE;
+  char *base = static_cast<char *>(ws);
+  const float *ck = ckpt;
+  if (!ck) {
+    // Recompute the per-chunk states with a forward pass that writes only
+    // the checkpoints (one extra read of k and v).
+    float *ws_ck = reinterpret_cast<float *>(base + L.ckpt);
+    rc = forward_impl(B, T, C, dtype, w, u, k, v, state_in, nullptr, nullptr, ws_ck, ws, ws_bytes,
+                      st, opt);
+    if (rc != WKV_OK) return rc;
+    ck = ws_ck;
+  }
+  BwdArgs a{};
+  a.B = B; a.T = T; a.C = C; a.w = w; a.u = u; a.k = k; a.v = v; a.gy = grad_y;
+  a.ckpt = ck; a.gk = grad_k; a.gv = grad_v;
+  a.part = reinterpret_cast<float *>(base + L.part);
+  a.hdr = reinterpret_cast<WsHeader *>(base);
+  a.flags = reinterpret_cast<unsigned *>(base + L.flags);
+  a.desc = reinterpret_cast<float *>(base + L.desc);
+  a.nct = L.nct; a.nchains = L.nchains; a.nchunks = L.nchunks_b;
+  a.spin_limit = spin_of(opt);
+  a.hold_first = opt ? opt->test_hold_first_chunk : 0;
+  return launch_backward(a, dtype, grad_w, grad_u, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+int wkv_backward(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                 const void *k, const void *v, const void *grad_y, const float *state_in,
+                 const float *ckpt, float *grad_w, float *grad_u, void *grad_k, void *grad_v,
+                 void *ws, size_t ws_bytes, void *stream) {
+  return wkv_backward_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u,
+                         grad_k, grad_v, ws, ws_bytes, stream, nullptr);
+}
+
+int wkv_step(int64_t N, int64_t C, const float *w, const float *u, const float *k_t,
+             const float *v_t, const float *state_in, float *y_t, float *state_out, void *stream) {
+  if (!sizes_ok(N, 1, C)) return WKV_ERR_INVALID_ARG;
+  if (!w || !u || !k_t || !v_t || !state_in || !y_t || !state_out) return WKV_ERR_INVALID_ARG;
+  const void *ptrs[7] = {w, u, k_t, v_t, state_in, y_t, state_out};
+  for (const void *p : ptrs)
+    if (!aligned(p, 4)) return WKV_ERR_UNSUPPORTED;
+  const size_t nb = sizeof(float) * (size_t)(N * C), sb = 3 * nb;
+  if (state_in != state_out && overlaps(state_in, sb, state_out, sb)) return WKV_ERR_UNSUPPORTED;
+  if (overlaps(y_t, nb, state_in, sb) || overlaps(y_t, nb, state_out, sb) ||
+      overlaps(y_t, nb, k_t, nb) || overlaps(y_t, nb, v_t, nb) ||
+      overlaps(state_out, sb, k_t, nb) || overlaps(state_out, sb, v_t, nb))
+    return WKV_ERR_UNSUPPORTED;
+  StepArgs a{N, C, w, u, k_t, v_t, state_in, y_t, state_out};
+  bool vec = (C % 4) == 0;
+  for (const void *p : ptrs) vec = vec && aligned(p, 16);
+  return launch_step(a, vec, num_sms(), (cudaStream_t)stream) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+int wkv_get_status(void *ws, void *stream) {
+  if (!ws) return WKV_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return WKV_ERR_CUDA;
+  int status = 0;
+  WsHeader *h = static_cast<WsHeader *>(ws);
+  if (cudaMemcpy(&status, &h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return WKV_ERR_CUDA;
+  if (status != 0 && cudaMemset(&h->status, 0, sizeof(int)) != cudaSuccess) return WKV_ERR_CUDA;
+  return status;
+}
+
+const char *wkv_strerror(int status) {
+  switch (status) {
+    case WKV_OK: return "success";
+    case WKV_ERR_INVALID_ARG: return "invalid argument (NULL pointer, size out of range, bad dtype)";
+    case WKV_ERR_UNSUPPORTED: return "unsupported layout (misaligned pointer or overlapping buffers)";
+    case WKV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case WKV_ERR_CUDA: return "CUDA runtime error or failed kernel launch";
+    case WKV_ERR_TIMEOUT: return "a bounded device-side wait gave up (results invalid)";
+    default: return "unknown status";
+  }
+}
+
+int wkv_version(void) { return WKV_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,350 @@
+// wkv_internal.cuh -- device helpers and launch descriptors shared by the
+// libwkv kernels (internal; not part of the C ABI).
+//
+// Numerical scheme.  The WKV sums are carried in the max-rescaled form
+// (a, b, P): A = a * 2^P, B = b * 2^P, where A_t, B_t are the hidden sums of
+// the RNN form (RWKV paper review, "[논문 리뷰] Reinvention RNNs for the
+// Transformer Era: RWKV", section "RNN-유사추론", eq. WKV_t).  Inside the
+// kernels every exponent is in base 2 (k, u, w are multiplied by log2(e) on
+// load) so that each exponential is one ex2.approx instruction; states that
+// cross the C ABI use natural-log exponents.  P is the largest exponent of
+// any term of the sum, so a, b stay in [0, #tokens] and nothing overflows.
+//
+// Exponent bookkeeping: while no new token takes over the maximum, the
+// exponent after n decays is formed as fma(n, w, P_anchor) (one rounding)
+// instead of by n repeated additions (n roundings), so long decays do not
+// drift.  The same anchoring is used for the adjoint scale in the backward.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace wkv {
+
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
+constexpr float kLn2 = 0.6931471805599453f;    // ln(2)
+// Exponent of the empty state.  Finite so that differences never form
+// inf - inf; 2^(anything - 1e38) flushes to exactly 0.
+constexpr float kEmptyP = -1.0e38f;
+// Scale of the empty adjoint (Ahat = ahat * 2^-r with r = +1e38).
+constexpr float kEmptyR = 1.0e38f;
+constexpr int kCkpt = 64;  // tokens between forward checkpoints
+
+// ---------------------------------------------------------------- math ---
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Forward state of one channel: A = a 2^P, B = b 2^P.
+struct St {
+  float a, b, P;
+};
+__device__ __forceinline__ St st_empty() { return St{0.f, 0.f, kEmptyP}; }
+
+// Sequence X followed by a sequence Y of lenY tokens: X's sums decay lenY
+// times (exponent + lenY * w), then the two are added at the larger scale.
+// This is the associative combine that lets the time axis be split into
+// chunks ("Transformer-유사학습": the serial WKV part is done as a scan).
+__device__ __forceinline__ St combine(const St &X, const St &Y, float lenY, float w2) {
+  const float Px = fmaf(lenY, w2, X.P);
+  const float d = Px - Y.P;
+  const float x = ex2(-fabsf(d));
+  const bool xw = d >= 0.f;
+  const float fx = xw ? 1.f : x, fy = xw ? x : 1.f;
+  St r;
+  r.a = fmaf(X.a, fx, Y.a * fy);
+  r.b = fmaf(X.b, fx, Y.b * fy);
+  r.P = fmaxf(Px, Y.P);
+  return r;
+}
+
+// Adjoint of one channel for the backward: Ahat = ah 2^-r, Hhat = hh 2^-r,
+// where Ahat_t = dL/dA_t and Hhat_t = -dL/dB_t.
+struct Adj {
+  float ah, hh, r;
+};
+__device__ __forceinline__ Adj adj_empty() { return Adj{0.f, 0.f, kEmptyR}; }
+
+// Reverse-time combine: X (earlier, lenX tokens) then Y (later).  The adjoint
+// at the start of X gains Y's adjoint decayed across X (factor 2^{lenX w}).
+__device__ __forceinline__ Adj rcombine(const Adj &X, const Adj &Y, float lenX, float w2) {
+  const float rY = fmaf(-lenX, w2, Y.r);
+  const float d = X.r - rY;
+  const float x = ex2(-fabsf(d));
+  const bool xs = d <= 0.f;  // X has the larger magnitude scale 2^-r
+  const float fx = xs ? 1.f : x, fy = xs ? x : 1.f;
+  Adj o;
+  o.ah = fmaf(X.ah, fx, Y.ah * fy);
+  o.hh = fmaf(X.hh, fx, Y.hh * fy);
+  o.r = fminf(X.r, rY);
+  return o;
+}
+
+// ---------------------------------------------------------- element I/O ---
+template <typename E>
+struct IO;
+template <>
+struct IO<float> {
+  static __device__ __forceinline__ float ld(const float *p) { return __ldcs(p); }
+  static __device__ __forceinline__ void st(float *p, float x) { __stcs(p, x); }
+};
+template <>
+struct IO<uint16_t> {  // bfloat16 storage
+  static __device__ __forceinline__ float ld(const uint16_t *p) {
+    unsigned short h;
+    asm volatile("ld.global.cs.u16 %0, [%1];" : "=h"(h) : "l"(p));
+    return __uint_as_float(((unsigned)h) << 16);
+  }
+  static __device__ __forceinline__ void st(uint16_t *p, float x) {
+    unsigned short h;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(x));
+    asm volatile("st.global.cs.u16 [%0], %1;" ::"l"(p), "h"(h));
+  }
+};
+
+// ------------------------------------------------------ workspace header ---
+// The first 256 bytes of every workspace.  Zero-filled once by the caller.
+struct WsHeader {
+  unsigned epoch;      // launches completed on this workspace
+  unsigned ticket;     // next tile ticket of the running launch
+  unsigned done;       // blocks finished in the running launch
+  unsigned abort_tag;  // epoch+1 of a launch in which a wait gave up
+  int status;          // first device-side error (sticky until read)
+  unsigned pad[59];
+};
+static_assert(sizeof(WsHeader) == 256, "header size");
+
+// Tile status flags: (epoch tag << 2) | 1 once the tile's record is
+// published.  A flag from an earlier launch carries an older tag and reads
+// as "not ready".
+constexpr unsigned kAgg = 1u;
+__device__ __forceinline__ unsigned epoch_tag(unsigned epoch) { return epoch & 0x3FFFFFFFu; }
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Per-tile descriptor: one record (the Fenwick node of the chunk) of three
+// float planes of 32 lanes each.
+constexpr int kDescFloats = 3 * 32;
+
+template <typename S>
+__device__ __forceinline__ void desc_store(float *desc, int64_t tile, int which, const S &s,
+                                           int lane) {
+  float *d = desc + tile * kDescFloats + which * 96;
+  const float *f = reinterpret_cast<const float *>(&s);
+  __stcg(d + lane, f[0]);
+  __stcg(d + 32 + lane, f[1]);
+  __stcg(d + 64 + lane, f[2]);
+}
+template <typename S>
+__device__ __forceinline__ S desc_load(const float *desc, int64_t tile, int which, int lane) {
+  const float *d = desc + tile * kDescFloats + which * 96;
+  S s;
+  float *f = reinterpret_cast<float *>(&s);
+  f[0] = __ldcg(d + lane);
+  f[1] = __ldcg(d + 32 + lane);
+  f[2] = __ldcg(d + 64 + lane);
+  return s;
+}
+
+// Publish a record and then its flag with release semantics (all lanes of
+// the warp call this together).
+template <typename S>
+__device__ __forceinline__ void publish(float *desc, unsigned *flags, int64_t tile, int which,
+                                       const S &s, unsigned epoch, int lane) {
+  desc_store(desc, tile, which, s, lane);
+  __syncwarp();
+  if (lane == 0) {
+    __threadfence();
+    st_release(flags + tile, (epoch_tag(epoch) << 2) | kAgg);
+  }
+  __syncwarp();
+}
+
+// Record a device-side error for this launch (first one wins) and mark the
+// launch aborted so that other waiting blocks give up at once.
+__device__ __forceinline__ void raise_timeout(WsHeader *h, unsigned epoch) {
+  atomicCAS(&h->status, 0, -5 /* WKV_ERR_TIMEOUT */);
+  atomicExch(&h->abort_tag, epoch + 1u);
+}
+
+// Block start: take a ticket (tiles are processed in ticket order, so every
+// tile a block waits on belongs to a block that has already started) and
+// read the launch epoch.
+__device__ __forceinline__ void take_ticket(WsHeader *h, unsigned *s_tile, unsigned *s_epoch) {
+  if (threadIdx.x == 0) {
+    *s_tile = atomicAdd(&h->ticket, 1u);
+    *s_epoch = ld_relaxed(&h->epoch);
+  }
+}
+
+// Block end (after its last flag access): the last block of the launch
+// resets the ticket and the counter and advances the epoch.
+__device__ __forceinline__ void finish_block(WsHeader *h, unsigned nblocks) {
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(&h->done, 1u);
+    if (prev == nblocks - 1u) {
+      h->ticket = 0u;
+      h->done = 0u;
+      __threadfence();
+      atomicAdd(&h->epoch, 1u);
+    }
+  }
+}
+
+// ------------------------------------------ deterministic chunk scan ---
+// The time axis of every (b, channel tile) chain is cut into chunks; chunk
+// `pos` (in scan order) publishes one record, the Fenwick node F(pos): the
+// summary of the lowbit(pos+1) chunks ending at pos, joined in a fixed
+// binary bracketing.  A chunk's exclusive prefix is the join of the nodes of
+// the binary decomposition of pos.  Every combine therefore happens in an
+// order fixed by pos alone: results are bit-identical from run to run,
+// whatever order the blocks run in.  A block waits only on nodes of smaller
+// positions, and the dependency depth is log2(#chunks).
+//
+// Position-ordered join: L covers the positions before R; R holds lenR
+// tokens.  Forward: earlier positions are earlier in time.  Backward: scan
+// order runs from the end of the sequence, so R is earlier in time.
+__device__ __forceinline__ St pjoin(const St &L, const St &R, float lenR, float w2) {
+  return combine(L, R, lenR, w2);
+}
+__device__ __forceinline__ Adj pjoin(const Adj &L, const Adj &R, float lenR, float w2) {
+  return rcombine(R, L, lenR, w2);
+}
+
+__device__ __forceinline__ bool launch_aborted(WsHeader *h, unsigned epoch) {
+  return ld_relaxed(&h->abort_tag) == epoch + 1u;
+}
+
+// Wait until every active lane's node (position q) is published.  Bounded:
+// after `spin_limit` polls (or once another block of the launch gave up) the
+// launch is marked aborted, the status word gets WKV_ERR_TIMEOUT and false is
+// returned; the caller then goes on with invalid data so nothing hangs.
+__device__ __forceinline__ bool wait_nodes(const unsigned *flags, int64_t q, bool active,
+                                           int64_t chain, int64_t nchains, unsigned epoch,
+                                           WsHeader *h, int64_t spin_limit, int lane) {
+  const unsigned want = (epoch_tag(epoch) << 2) | kAgg;
+  bool ready = !active;
+  int64_t waits = 0;
+  unsigned backoff = 32;
+  while (true) {
+    if (!ready) ready = ld_acquire(flags + (q * nchains + chain)) == want;
+    if (__all_sync(0xffffffffu, ready)) {
+      __syncwarp();
+      return true;
+    }
+    if (++waits > spin_limit || launch_aborted(h, epoch)) {
+      if (lane == 0) raise_timeout(h, epoch);
+      __syncwarp();
+      return false;
+    }
+    __nanosleep(backoff);
+    backoff = backoff < 1024u ? backoff * 2u : 1024u;
+  }
+}
+
+// Called by one warp per block.  `agg` is the block's own summary (agg_len
+// tokens), `full_len` the tokens of a full chunk, `base0` the value before
+// position 0 (initial state forward, empty adjoint backward).  Publishes
+// F(pos) when a later position needs it (`need_node`) unless `publish_ok` is
+// false (test hook), and returns the exclusive prefix of pos.
+template <typename S>
+__device__ S chunk_scan(unsigned *flags, float *desc, int64_t pos, int64_t chain, int64_t nchains,
+                        const S &agg, float agg_len, float full_len, const S &base0,
+                        const S &empty, unsigned epoch, WsHeader *h, int64_t spin_limit,
+                        bool need_node, bool publish_ok, float w2, int lane) {
+  const int64_t tile = pos * nchains + chain;
+  // (1) F(pos) = F(pos-2^(n-1)) + ... + F(pos-2) + F(pos-1) + agg, bracketed
+  //     from the right, n = log2(lowbit(pos+1)).
+  const int64_t lb = (pos + 1) & -(pos + 1);
+  const int nup = need_node ? 63 - __clzll((unsigned long long)lb) : 0;
+  wait_nodes(flags, lane < nup ? pos - ((int64_t)1 << lane) : 0, lane < nup, chain, nchains,
+             epoch, h, spin_limit, lane);
+  S F = agg;
+  float flen = agg_len;
+  for (int i = 0; i < nup; ++i) {
+    const int64_t s = (int64_t)1 << i;
+    const S left = desc_load<S>(desc, (pos - s) * nchains + chain, 0, lane);
+    F = pjoin(left, F, flen, w2);
+    flen += (float)s * full_len;
+  }
+  if (need_node && publish_ok) publish(desc, flags, tile, 0, F, epoch, lane);
+  // (2) exclusive prefix: nodes x-1 for x = pos, pos minus its lowest set
+  //     bit, ... (one per set bit of pos), joined from the right.
+  const int nd = __popcll((unsigned long long)pos);
+  int64_t xl = pos;
+  for (int k = 0; k < lane && k < nd; ++k) xl &= xl - 1;
+  wait_nodes(flags, lane < nd ? xl - 1 : 0, lane < nd, chain, nchains, epoch, h, spin_limit, lane);
+  S acc = empty;
+  float acc_len = 0.f;
+  int64_t x = pos;
+  for (int k = 0; k < nd; ++k) {
+    const int64_t sz = x & -x;
+    const S node = desc_load<S>(desc, (x - 1) * nchains + chain, 0, lane);
+    acc = pjoin(node, acc, acc_len, w2);
+    acc_len += (float)sz * full_len;
+    x &= x - 1;
+  }
+  return pjoin(base0, acc, acc_len, w2);
+}
+
+// ---------------------------------------------------- launch descriptors ---
+struct FwdArgs {
+  int64_t B, T, C;
+  const float *w, *u;
+  const void *k, *v;
+  const float *state_in;  // natural-log exponent, may be null
+  void *y;                // may be null (checkpoint-only pass)
+  float *state_out;       // natural-log exponent, may be null
+  float *ckpt;            // base-2 exponent, [nck][3][B][C], may be null
+  WsHeader *hdr;
+  unsigned *flags;
+  float *desc;
+  int64_t nct;      // channel tiles of 32 per batch row
+  int64_t nchains;  // B * nct
+  int64_t nchunks;  // chunks of the time axis
+  int64_t spin_limit;
+  int hold_first;
+};
+
+struct BwdArgs {
+  int64_t B, T, C;
+  const float *w, *u;
+  const void *k, *v, *gy;
+  const float *ckpt;  // base-2 exponent checkpoints [nck][3][B][C]
+  void *gk, *gv;
+  float *part;  // [nchunks][2][B][C] per-chunk partial dL/dw, dL/du
+  WsHeader *hdr;
+  unsigned *flags;
+  float *desc;
+  int64_t nct, nchains, nchunks;
+  int64_t spin_limit;
+  int hold_first;
+};
+
+struct StepArgs {
+  int64_t N, C;
+  const float *w, *u, *k, *v, *state_in;
+  float *y, *state_out;
+};
+
+}  // namespace wkv

@@ -1,0 +1,117 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* the library loads and exports every function ``include/wkv.h`` declares;
+* argument validation rejects bad calls with the documented code before any
+  CUDA work (these calls never reach a kernel launch);
+* workspace and checkpoint sizes follow the documented layout.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def W():
+    from rwkv_linear_rnn_b200.build import build_library
+    build_library()
+    import rwkv_linear_rnn_b200
+    return rwkv_linear_rnn_b200
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "wkv.h"), encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(wkv_[a-z_]+)\s*\(", src, flags=re.M)
+    return names
+
+
+def test_header_declares_expected(W):
+    names = header_functions()
+    assert sorted(names) == sorted(W.abi.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(W):
+    lib = ctypes.CDLL(W.library_path())
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_strerror(W):
+    assert W.wkv_version() == 100
+    for code in range(0, -6, -1):
+        assert W.wkv_strerror(code) != "unknown status"
+    assert W.wkv_strerror(7) == "unknown status"
+
+
+def test_sizes(W):
+    B, T, C = 8, 1024, 768
+    assert W.wkv_ckpt_size(B, T, C) == 4 * 3 * B * C * 16
+    assert W.wkv_workspace_size(W.WKV_OP_STEP, B, T, C, 0) == 0
+    f = W.wkv_workspace_size(W.WKV_OP_FORWARD, B, T, C, 0)
+    b = W.wkv_workspace_size(W.WKV_OP_BACKWARD, B, T, C, 0)
+    assert 256 < f < b
+    assert b >= 256 + W.wkv_ckpt_size(B, T, C) + 4 * 2 * B * C * 16
+    assert W.wkv_workspace_size(0, 0, T, C, 0) == 0     # B < 1
+    assert W.wkv_workspace_size(0, B, -1, C, 0) == 0    # T < 0
+    assert W.wkv_workspace_size(0, B, T, C, 3) == 0     # bad dtype
+    assert W.wkv_workspace_size(9, B, T, C, 0) == 0     # bad op
+    assert W.wkv_ckpt_size(1 << 40, 1 << 20, 1 << 20) == 0  # overflow
+
+
+FAKE = 1 << 20  # an aligned non-null address; validation fails before any use
+
+
+@pytest.mark.parametrize("args,code", [
+    # (B, T, C, dtype, w, u, k, v, state_in, y, state_out, ckpt, ws, ws_bytes)
+    ((1, 8, 4, 2, FAKE, FAKE, FAKE, FAKE, 0, FAKE * 2, 0, 0, 0, 0), -1),   # bad dtype
+    ((0, 8, 4, 0, FAKE, FAKE, FAKE, FAKE, 0, FAKE * 2, 0, 0, 0, 0), -1),   # B = 0
+    ((1, -1, 4, 0, FAKE, FAKE, FAKE, FAKE, 0, FAKE * 2, 0, 0, 0, 0), -1),  # T < 0
+    ((1, 8, 4, 0, 0, FAKE, FAKE, FAKE, 0, FAKE * 2, 0, 0, 0, 0), -1),      # w NULL
+    ((1, 8, 4, 0, FAKE, FAKE, 0, FAKE, 0, FAKE * 2, 0, 0, 0, 0), -1),      # k NULL
+    ((1, 8, 4, 0, FAKE, FAKE, FAKE, FAKE, 0, 0, 0, 0, 0, 0), -1),          # y NULL
+    ((1, 8, 4, 0, FAKE + 2, FAKE, FAKE, FAKE, 0, FAKE * 2, 0, 0, 0, 0), -2),  # w misaligned
+    ((1, 8, 4, 1, FAKE, FAKE, FAKE + 1, FAKE, 0, FAKE * 2, 0, 0, 0, 0), -2),  # bf16 k odd
+    ((1, 8, 4, 0, FAKE, FAKE, FAKE, FAKE, 0, FAKE + 16, 0, 0, 0, 0), -2),  # y overlaps k
+    ((1, 1 << 31, 4, 0, FAKE, FAKE, FAKE, FAKE, 0, FAKE * 2, 0, 0, 0, 0), -1),  # T too large
+])
+def test_forward_validation(W, args, code):
+    assert W.abi.wkv_forward(*args, 0) == code
+
+
+def test_forward_chunked_needs_workspace(W):
+    opt = W.abi.Options(kernel=W.WKV_KERNEL_CHUNKED)
+    base = (1, 1024, 64, 0, FAKE, FAKE, FAKE, FAKE, 0, FAKE * 4, 0, 0)
+    assert W.abi.wkv_forward_ex(*base, 0, 0, 0, opt) == -3             # NULL ws
+    assert W.abi.wkv_forward_ex(*base, FAKE * 8, 256, 0, opt) == -3    # too small
+    assert W.abi.wkv_forward_ex(*base, FAKE * 8 + 16, 1 << 30, 0, opt) == -3  # misaligned
+
+
+def test_backward_validation(W):
+    a = W.abi
+    # (B, T, C, dt, w, u, k, v, gy, state_in, ckpt, gw, gu, gk, gv, ws, ws_bytes, stream)
+    ok = [1, 64, 32, 0, FAKE, FAKE, FAKE, FAKE * 2, FAKE * 3, 0, 0, FAKE * 4, FAKE * 5,
+          FAKE * 6, FAKE * 7, 0, 0, 0]
+    bad = list(ok); bad[11] = 0
+    assert a.wkv_backward(*bad) == -1                      # grad_w NULL
+    bad = list(ok); bad[13] = FAKE                         # grad_k overlaps k
+    assert a.wkv_backward(*bad) == -2
+    bad = list(ok); bad[14] = FAKE * 6                     # grad_v overlaps grad_k
+    assert a.wkv_backward(*bad) == -2
+    assert a.wkv_backward(*ok) == -3                       # no workspace
+
+
+def test_step_validation(W):
+    a = W.abi
+    assert a.wkv_step(0, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0) == -1
+    assert a.wkv_step(1, 4, FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, 0) == -1
+    assert a.wkv_step(1, 4, FAKE, FAKE, FAKE, FAKE, FAKE + 1, FAKE, FAKE, 0) == -2
+    # state_out partly overlapping state_in
+    assert a.wkv_step(2, 4, FAKE, FAKE, FAKE * 2, FAKE * 3, FAKE * 4, FAKE * 5, FAKE * 4 + 16, 0) == -2
+
+
+def test_get_status_null(W):
+    assert W.abi.wkv_get_status(0, 0) == -3
