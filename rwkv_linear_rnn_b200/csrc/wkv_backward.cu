@@ -99,17 +99,21 @@ __global__ void __launch_bounds__(W * 32) bwd_chunked_kernel(BwdArgs p) {
 
   float K[L], V[L], G[L];
   const int64_t off = (b * T + t0) * C + c;
-  {
-    const E *kp = static_cast<const E *>(p.k) + off;
-    const E *vp = static_cast<const E *>(p.v) + off;
-    const E *gp = static_cast<const E *>(p.gy) + off;
+  if (nvalid > 0) {  // warp-uniform
+    const int64_t loff = (b * T + t0) * C + (cok ? c : C - 1);
+    load_rows<E, L>(static_cast<const E *>(p.k) + loff, C, nvalid, K);
+    load_rows<E, L>(static_cast<const E *>(p.v) + loff, C, nvalid, V);
+    load_rows<E, L>(static_cast<const E *>(p.gy) + loff, C, nvalid, G);
 #pragma unroll
     for (int j = 0; j < L; ++j) {
       const bool ok = cok && j < nvalid;
-      K[j] = ok ? IO<E>::ld(kp + (int64_t)j * C) * kLog2e : 0.f;
-      V[j] = ok ? IO<E>::ld(vp + (int64_t)j * C) : 0.f;
-      G[j] = ok ? IO<E>::ld(gp + (int64_t)j * C) : 0.f;
+      K[j] = ok ? K[j] * kLog2e : 0.f;
+      V[j] = ok ? V[j] : 0.f;
+      G[j] = ok ? G[j] : 0.f;
     }
+  } else {
+#pragma unroll
+    for (int j = 0; j < L; ++j) K[j] = V[j] = G[j] = 0.f;
   }
 
   // (2) warp start states: checkpoint, then the earlier warps' summaries.

@@ -99,25 +99,23 @@ __global__ void __launch_bounds__(256) fwd_seq_kernel(FwdArgs p) {
   Run s = run_from(load_state_in(p.state_in, idx, BC));
 
   float Kc[U], Vc[U], Kn[U], Vn[U];
-#pragma unroll
-  for (int j = 0; j < U; ++j) {
-    const bool ok = j < T;
-    Kc[j] = ok ? IO<E>::ld(kp + j * C) * kLog2e : 0.f;
-    Vc[j] = ok ? IO<E>::ld(vp + j * C) : 0.f;
+  if (T > 0) {
+    const int n0 = (int)min((int64_t)U, T);
+    load_rows<E, U>(kp, C, n0, Kc);
+    load_rows<E, U>(vp, C, n0, Vc);
   }
   for (int64_t t0 = 0; t0 < T; t0 += U) {
-#pragma unroll
-    for (int j = 0; j < U; ++j) {
-      const int64_t t = t0 + U + j;
-      const bool ok = t < T;
-      Kn[j] = ok ? IO<E>::ld(kp + t * C) * kLog2e : 0.f;
-      Vn[j] = ok ? IO<E>::ld(vp + t * C) : 0.f;
+    // prefetch the next U rows (clamped to the last row; ignored past T)
+    if (t0 + U < T) {
+      const int n1 = (int)min((int64_t)U, T - t0 - U);
+      load_rows<E, U>(kp + (t0 + U) * C, C, n1, Kn);
+      load_rows<E, U>(vp + (t0 + U) * C, C, n1, Vn);
     }
     if (p.ckpt && (t0 % kCkpt) == 0) store_ckpt(p.ckpt, t0 / kCkpt, idx, BC, run_state(s, w2));
 #pragma unroll
     for (int j = 0; j < U; ++j) {
       if (t0 + j < T) {
-        const float y = fwd_token(s, Kc[j], Vc[j], u2, w2);
+        const float y = fwd_token(s, Kc[j] * kLog2e, Vc[j], u2, w2);
         if (yp) IO<E>::st(yp + (t0 + j) * C, y);
       }
     }
@@ -197,16 +195,19 @@ __global__ void __launch_bounds__(W * 32) fwd_chunked_kernel(FwdArgs p) {
   const float u2 = cok ? p.u[c] * kLog2e : 0.f;
 
   float K[L], V[L];
-  {
-    const int64_t off = (b * T + t0) * C + c;
-    const E *kp = static_cast<const E *>(p.k) + off;
-    const E *vp = static_cast<const E *>(p.v) + off;
+  if (nvalid > 0) {  // warp-uniform
+    const int64_t off = (b * T + t0) * C + (cok ? c : C - 1);
+    load_rows<E, L>(static_cast<const E *>(p.k) + off, C, nvalid, K);
+    load_rows<E, L>(static_cast<const E *>(p.v) + off, C, nvalid, V);
 #pragma unroll
     for (int j = 0; j < L; ++j) {
       const bool ok = cok && j < nvalid;
-      K[j] = ok ? IO<E>::ld(kp + (int64_t)j * C) * kLog2e : 0.f;
-      V[j] = ok ? IO<E>::ld(vp + (int64_t)j * C) : 0.f;
+      K[j] = ok ? K[j] * kLog2e : 0.f;
+      V[j] = ok ? V[j] : 0.f;
     }
+  } else {
+#pragma unroll
+    for (int j = 0; j < L; ++j) K[j] = V[j] = 0.f;
   }
 
   // Pass 1: segment summary.

@@ -99,7 +99,7 @@ template <>
 struct IO<uint16_t> {  // bfloat16 storage
   static __device__ __forceinline__ float ld(const uint16_t *p) {
     unsigned short h;
-    asm volatile("ld.global.cs.u16 %0, [%1];" : "=h"(h) : "l"(p));
+    asm("ld.global.cs.u16 %0, [%1];" : "=h"(h) : "l"(p));
     return __uint_as_float(((unsigned)h) << 16);
   }
   static __device__ __forceinline__ void st(uint16_t *p, float x) {
@@ -108,6 +108,19 @@ struct IO<uint16_t> {  // bfloat16 storage
     asm volatile("st.global.cs.u16 [%0], %1;" ::"l"(p), "h"(h));
   }
 };
+
+// Load L rows (stride elements apart) of one column.  All L loads are issued
+// back to back from always-valid addresses -- rows at or past `nvalid` repeat
+// the last valid row and the caller ignores them -- so that the warp has
+// every load in flight before it first waits on one.  (Guarding each load
+// with a condition lets the compiler pair each load with its first use and
+// serialises the round trips.)  Requires nvalid >= 1.
+template <typename E, int L>
+__device__ __forceinline__ void load_rows(const E *base, int64_t stride, int nvalid,
+                                          float (&out)[L]) {
+#pragma unroll
+  for (int j = 0; j < L; ++j) out[j] = IO<E>::ld(base + (int64_t)min(j, nvalid - 1) * stride);
+}
 
 // ------------------------------------------------------ workspace header ---
 // The first 256 bytes of every workspace.  Zero-filled once by the caller.
