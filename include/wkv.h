@@ -82,7 +82,8 @@ typedef enum {
 enum { WKV_OP_FORWARD = 0, WKV_OP_BACKWARD = 1, WKV_OP_STEP = 2 };
 
 /* Kernel selector (wkv_options.kernel). */
-enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2 };
+enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
+       WKV_KERNEL_CHUNKED_REGS = 3, WKV_KERNEL_CHAIN = 4 };
 
 /*
  * Optional knobs for the *_ex calls.  A NULL options pointer, or all fields
@@ -90,7 +91,14 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2 };
  * floating-point rounding order.
  *   kernel      WKV_KERNEL_AUTO picks by problem shape; SEQUENTIAL runs one
  *               thread per (b, c) chain over all of T; CHUNKED splits T into
- *               chunks joined by a single-pass decoupled look-back scan.
+ *               64-token chunks joined by a single-pass scan over published
+ *               chunk summaries (TMA-fed shared-memory pipeline when rows are
+ *               16-byte aligned); CHUNKED_REGS forces the register-tile
+ *               variant of the chunked kernel (no TMA); CHAIN runs one block
+ *               per (batch row, 32-channel) chain over all of T, tiles fed
+ *               by TMA, the carry kept on chip (needs 16-byte aligned rows;
+ *               the default when they are).  The backward honours
+ *               CHAIN/AUTO (chain kernel) versus any other value (chunked).
  *   spin_limit  polls a block makes on one predecessor's flag before it gives
  *               up with WKV_ERR_TIMEOUT (0 = default, about one second).
  *   test_hold_first_chunk

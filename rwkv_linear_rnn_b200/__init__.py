@@ -17,13 +17,17 @@ import ctypes
 import os
 
 from . import abi
-from .abi import (WKV_BF16, WKV_F32, WKV_KERNEL_AUTO, WKV_KERNEL_CHUNKED, WKV_KERNEL_SEQUENTIAL,
+from .abi import (WKV_BF16, WKV_F32, WKV_KERNEL_AUTO, WKV_KERNEL_CHAIN, WKV_KERNEL_CHUNKED,
+                  WKV_KERNEL_CHUNKED_REGS,
+                  WKV_KERNEL_SEQUENTIAL,
                   WKV_OP_BACKWARD, WKV_OP_FORWARD, WKV_OP_STEP, WKVError, wkv_ckpt_size,
                   wkv_strerror, wkv_version, wkv_workspace_size)
 
 __all__ = [
     "abi", "WKVError", "WKV_F32", "WKV_BF16", "WKV_OP_FORWARD", "WKV_OP_BACKWARD", "WKV_OP_STEP",
-    "WKV_KERNEL_AUTO", "WKV_KERNEL_SEQUENTIAL", "WKV_KERNEL_CHUNKED", "Workspace", "forward",
+    "WKV_KERNEL_AUTO", "WKV_KERNEL_SEQUENTIAL", "WKV_KERNEL_CHUNKED", "WKV_KERNEL_CHUNKED_REGS",
+    "WKV_KERNEL_CHAIN",
+    "Workspace", "forward",
     "backward", "step", "WKV", "wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror",
     "wkv_version", "library_path",
 ]

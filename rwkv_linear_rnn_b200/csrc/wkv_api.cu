@@ -10,7 +10,12 @@
 #include "wkv_internal.cuh"
 
 namespace wkv {
-cudaError_t launch_forward(const FwdArgs &a, int dtype, bool chunked, cudaStream_t st);
+cudaError_t launch_forward(const FwdArgs &a, int dtype, int kind, int num_sms, cudaStream_t st);
+bool fwd_tma_eligible(const FwdArgs &a, int dtype);
+cudaError_t launch_forward_chain(const FwdArgs &a, int dtype, cudaStream_t st);
+cudaError_t launch_backward_chain(const BwdArgs &a, int dtype, cudaStream_t st);
+cudaError_t launch_reduce_wu(const float *part, int64_t nchunks, int64_t B, int64_t C, float *gw,
+                             float *gu, cudaStream_t st);
 cudaError_t launch_backward(const BwdArgs &a, int dtype, float *gw, float *gu, cudaStream_t st);
 cudaError_t launch_step(const StepArgs &a, bool vec, int num_sms, cudaStream_t st);
 int64_t fwd_chunk_tokens();
@@ -85,7 +90,9 @@ int num_sms() {
 bool pick_chunked(const wkv_options *opt, int64_t B, int64_t T, int64_t C) {
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   if (kernel == WKV_KERNEL_SEQUENTIAL) return false;
-  if (kernel == WKV_KERNEL_CHUNKED) return true;
+  if (kernel == WKV_KERNEL_CHUNKED || kernel == WKV_KERNEL_CHUNKED_REGS ||
+      kernel == WKV_KERNEL_CHAIN)
+    return true;
   // Enough independent chains to fill the GPU, or too short to split.
   return !(B * C >= kSeqMinChains || T <= 2 * fwd_chunk_tokens());
 }
@@ -122,7 +129,7 @@ int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
     if (!state_out) return WKV_OK;
     FwdArgs a{};
     a.B = B; a.T = 0; a.C = C; a.w = w; a.u = u; a.state_in = state_in; a.state_out = state_out;
-    return launch_forward(a, dtype, false, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    return launch_forward(a, dtype, 0, 1, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
   }
   const Layout L = layout(WKV_OP_FORWARD, B, T, C);
   const bool chunked = pick_chunked(opt, B, T, C);
@@ -140,7 +147,13 @@ int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
   a.nct = L.nct; a.nchains = L.nchains; a.nchunks = L.nchunks_f;
   a.spin_limit = spin_of(opt);
   a.hold_first = opt ? opt->test_hold_first_chunk : 0;
-  return launch_forward(a, dtype, chunked, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
+  if (chunked && fwd_tma_eligible(a, dtype) &&
+      (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_CHAIN))
+    return launch_forward_chain(a, dtype, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  int kind = 0;
+  if (chunked) kind = (fwd_tma_eligible(a, dtype) && kernel != WKV_KERNEL_CHUNKED_REGS) ? 2 : 1;
+  return launch_forward(a, dtype, kind, num_sms(), st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
 }  // namespace
@@ -231,6 +244,14 @@ int wkv_backward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, 
   a.nct = L.nct; a.nchains = L.nchains; a.nchunks = L.nchunks_b;
   a.spin_limit = spin_of(opt);
   a.hold_first = opt ? opt->test_hold_first_chunk : 0;
+  const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
+  FwdArgs probe{};
+  probe.B = B; probe.T = T; probe.C = C; probe.k = k; probe.v = v;
+  const bool tma_ok = fwd_tma_eligible(probe, dtype) && ((uintptr_t)grad_y % 16) == 0;
+  if (tma_ok && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_CHAIN)) {
+    if (launch_backward_chain(a, dtype, st) != cudaSuccess) return WKV_ERR_CUDA;
+    return launch_reduce_wu(a.part, 1, B, C, grad_w, grad_u, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  }
   return launch_backward(a, dtype, grad_w, grad_u, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 

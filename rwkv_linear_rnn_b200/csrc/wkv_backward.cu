@@ -38,38 +38,16 @@
 // is at most 1 (the terms e^{k_t} Ahat_{t+1} and e^w A_t Ahat_{t+1} are
 // weighted sums of g_s / D_s with weights <= 1), so nothing overflows.
 #include "wkv_internal.cuh"
+#include "wkv_math.cuh"
 
 namespace wkv {
-
-template <int L>
-__device__ __forceinline__ St summarize_b(const float (&K)[L], const float (&V)[L], float w2,
-                                          int nvalid) {
-  float e[L];
-  float m = kEmptyP;
-  const float last = (float)(nvalid - 1);
-#pragma unroll
-  for (int j = 0; j < L; ++j) {
-    e[j] = fmaf(last - (float)j, w2, K[j]);
-    if (j < nvalid) m = fmaxf(m, e[j]);
-  }
-  float a = 0.f, b = 0.f;
-#pragma unroll
-  for (int j = 0; j < L; ++j) {
-    if (j < nvalid) {
-      const float x = ex2(e[j] - m);
-      a = fmaf(x, V[j], a);
-      b += x;
-    }
-  }
-  return St{a, b, m};
-}
 
 template <typename E, int W, int L>
 __global__ void __launch_bounds__(W * 32) bwd_chunked_kernel(BwdArgs p) {
   constexpr int TC = W * L;
   static_assert(TC == kCkpt, "backward chunk must equal the checkpoint interval");
   __shared__ unsigned s_tile, s_epoch;
-  __shared__ float s_f[W][3][32];    // forward summaries, then warp start states
+  __shared__ float s_f[W][128];      // forward summaries, then warp start states (St planes)
   __shared__ float s_adj[W][3][32];  // adjoint aggregates, then later-warp suffixes
   __shared__ float s_carry[3][32];   // adjoint at the end of the block's chunk
   __shared__ float s_g[2][W][32];    // per-warp partial dL/dw, dL/du
@@ -118,10 +96,8 @@ __global__ void __launch_bounds__(W * 32) bwd_chunked_kernel(BwdArgs p) {
 
   // (2) warp start states: checkpoint, then the earlier warps' summaries.
   if (wi < W - 1) {
-    const St s = summarize_b<L>(K, V, w2, nvalid);
-    s_f[wi][0][lane] = s.a;
-    s_f[wi][1][lane] = s.b;
-    s_f[wi][2][lane] = s.P;
+    const St s = summarize<L>(K, V, w2, nvalid);
+    put_st(s_f[wi], lane, s);
   }
   __syncthreads();
   if (wi == 0) {
@@ -133,10 +109,8 @@ __global__ void __launch_bounds__(W * 32) bwd_chunked_kernel(BwdArgs p) {
 #pragma unroll
     for (int i = 0; i < W; ++i) {
       St si{};
-      if (i < W - 1) si = St{s_f[i][0][lane], s_f[i][1][lane], s_f[i][2][lane]};
-      s_f[i][0][lane] = acc.a;
-      s_f[i][1][lane] = acc.b;
-      s_f[i][2][lane] = acc.P;
+      if (i < W - 1) si = get_st(s_f[i], lane);
+      put_st(s_f[i], lane, acc);
       if (i < W - 1) {
         const int li = (int)max((int64_t)0, min((int64_t)L, T - (tc0 + (int64_t)i * L)));
         acc = combine(acc, si, (float)li, w2);
@@ -148,7 +122,8 @@ __global__ void __launch_bounds__(W * 32) bwd_chunked_kernel(BwdArgs p) {
   // (3) forward recompute of the segment.
   float q_[L], gam[L], eta[L], e2_[L], a_[L], b_[L], so_[L], sn_[L], P1_[L];
   {
-    float sa = s_f[wi][0][lane], sb = s_f[wi][1][lane], Panc = s_f[wi][2][lane], n = 0.f;
+    const St st0 = get_st(s_f[wi], lane);
+    float sa = st0.a, sb = st0.b, Panc = st0.P, n = st0.n;
 #pragma unroll
     for (int j = 0; j < L; ++j) {
       if (j < nvalid) {
@@ -324,6 +299,12 @@ static cudaError_t launch_bwd_t(const BwdArgs &a, float *gw, float *gu, cudaStre
   if (e != cudaSuccess) return e;
   reduce_wu_kernel<<<(unsigned)((a.C + 31) / 32), 256, 0, st>>>(a.part, a.nchunks, a.B, a.C, gw,
                                                                  gu);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_wu(const float *part, int64_t nchunks, int64_t B, int64_t C, float *gw,
+                             float *gu, cudaStream_t st) {
+  reduce_wu_kernel<<<(unsigned)((C + 31) / 32), 256, 0, st>>>(part, nchunks, B, C, gw, gu);
   return cudaGetLastError();
 }
 

@@ -16,67 +16,13 @@
 //                       depend on block timing); then every warp replays its
 //                       segment from the carried-in state.  k and v are read
 //                       from HBM once and stay in registers between passes.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "wkv_internal.cuh"
+#include "wkv_math.cuh"
 
 namespace wkv {
-
-// Running state of one channel with the anchored exponent P = fma(n, w, Panc).
-struct Run {
-  float a, b, Panc, n;
-};
-
-__device__ __forceinline__ Run run_from(const St &s) { return Run{s.a, s.b, s.P, 0.f}; }
-__device__ __forceinline__ St run_state(const Run &r, float w2) {
-  return St{r.a, r.b, fmaf(r.n, w2, r.Panc)};
-}
-
-// One token: output y_t = (A_t + e^{u+k} v) / (B_t + e^{u+k}) from the state
-// before the token, then A_{t+1} = e^w A_t + e^k v, B_{t+1} = e^w B_t + e^k.
-// Base-2 exponents (K = k log2 e, u2 = u log2 e, w2 = w log2 e).  In each pair
-// of scale factors one is exactly 1, so a token costs two ex2 and one rcp.
-__device__ __forceinline__ float fwd_token(Run &s, float K, float V, float u2, float w2) {
-  const float P = fmaf(s.n, w2, s.Panc);
-  const float UK = u2 + K;
-  const float d = P - UK;
-  const float x = ex2(-fabsf(d));
-  const bool pw = d >= 0.f;
-  const float e1 = pw ? 1.f : x, e2 = pw ? x : 1.f;
-  const float y = fmaf(s.a, e1, V * e2) * rcp(fmaf(s.b, e1, e2));
-  const float n1 = s.n + 1.f;
-  const float Pc = fmaf(n1, w2, s.Panc);
-  const float d2 = K - Pc;
-  const float x2 = ex2(-fabsf(d2));
-  const bool kw = d2 > 0.f;
-  const float so = kw ? x2 : 1.f, sn = kw ? 1.f : x2;
-  s.a = fmaf(s.a, so, V * sn);
-  s.b = fmaf(s.b, so, sn);
-  s.Panc = kw ? K : s.Panc;
-  s.n = kw ? 0.f : n1;
-  return y;
-}
-
-// Initial state of chain (b, c) from the caller's natural-log state.
-__device__ __forceinline__ St load_state_in(const float *st, int64_t i, int64_t BC) {
-  if (!st) return st_empty();
-  St s;
-  s.a = st[i];
-  s.b = st[BC + i];
-  s.P = fmaxf(st[2 * BC + i] * kLog2e, kEmptyP);
-  return s;
-}
-__device__ __forceinline__ void store_state(float *st, int64_t i, int64_t BC, const St &s) {
-  st[i] = s.a;
-  st[BC + i] = s.b;
-  st[2 * BC + i] = s.P * kLn2;
-}
-// Checkpoint (base-2 exponent) of the state before token ci * kCkpt.
-__device__ __forceinline__ void store_ckpt(float *ck, int64_t ci, int64_t i, int64_t BC,
-                                           const St &s) {
-  float *d = ck + ci * 3 * BC;
-  d[i] = s.a;
-  d[BC + i] = s.b;
-  d[2 * BC + i] = s.P;
-}
 
 // ------------------------------------------------------------------------
 // Sequential scan: one thread per (b, c).  Consecutive threads take
@@ -111,7 +57,7 @@ __global__ void __launch_bounds__(256) fwd_seq_kernel(FwdArgs p) {
       load_rows<E, U>(kp + (t0 + U) * C, C, n1, Kn);
       load_rows<E, U>(vp + (t0 + U) * C, C, n1, Vn);
     }
-    if (p.ckpt && (t0 % kCkpt) == 0) store_ckpt(p.ckpt, t0 / kCkpt, idx, BC, run_state(s, w2));
+    if (p.ckpt && (t0 % kCkpt) == 0) store_ckpt(p.ckpt, t0 / kCkpt, idx, BC, run_state(s), w2);
 #pragma unroll
     for (int j = 0; j < U; ++j) {
       if (t0 + j < T) {
@@ -129,7 +75,7 @@ __global__ void __launch_bounds__(256) fwd_seq_kernel(FwdArgs p) {
       Vc[j] = Vn[j];
     }
   }
-  if (p.state_out) store_state(p.state_out, idx, BC, run_state(s, w2));
+  if (p.state_out) store_state(p.state_out, idx, BC, run_state(s), w2);
 }
 
 // ------------------------------------------------------------------------
@@ -137,40 +83,14 @@ __global__ void __launch_bounds__(256) fwd_seq_kernel(FwdArgs p) {
 // block's chunk for the 32 channels of its tile (lane = channel).
 // ------------------------------------------------------------------------
 
-// Summary of a segment from the empty state: the state after its last valid
-// token, A = sum_j e^{(n-1-j) w + k_j} v_j.  Exponents are formed directly
-// (one fma each) against the segment maximum, so it costs one ex2 per token.
-template <int L>
-__device__ __forceinline__ St summarize(const float (&K)[L], const float (&V)[L], float w2,
-                                        int nvalid) {
-  float e[L];
-  float m = kEmptyP;
-  const float last = (float)(nvalid - 1);
-#pragma unroll
-  for (int j = 0; j < L; ++j) {
-    e[j] = fmaf(last - (float)j, w2, K[j]);
-    if (j < nvalid) m = fmaxf(m, e[j]);
-  }
-  float a = 0.f, b = 0.f;
-#pragma unroll
-  for (int j = 0; j < L; ++j) {
-    if (j < nvalid) {
-      const float x = ex2(e[j] - m);
-      a = fmaf(x, V[j], a);
-      b += x;
-    }
-  }
-  return St{a, b, m};
-}
-
 template <typename E, int W, int L>
 __global__ void __launch_bounds__(W * 32) fwd_chunked_kernel(FwdArgs p) {
   constexpr int TC = W * L;
   static_assert(TC % kCkpt == 0 && kCkpt % L == 0, "chunk/ckpt geometry");
   __shared__ unsigned s_tile, s_epoch;
-  __shared__ float s_agg[W][3][32];  // warp segment summaries
-  __shared__ float s_pre[W][3][32];  // block-local exclusive prefix of each warp
-  __shared__ float s_carry[3][32];   // state at the start of the block's chunk
+  __shared__ float s_agg[W][128];  // warp segment summaries (St planes)
+  __shared__ float s_pre[W][128];  // block-local exclusive prefix of each warp
+  __shared__ float s_carry[128];   // state at the start of the block's chunk
 
   const int wi = threadIdx.x >> 5, lane = threadIdx.x & 31;
   take_ticket(p.hdr, &s_tile, &s_epoch);
@@ -213,9 +133,7 @@ __global__ void __launch_bounds__(W * 32) fwd_chunked_kernel(FwdArgs p) {
   // Pass 1: segment summary.
   {
     const St s = summarize<L>(K, V, w2, nvalid);
-    s_agg[wi][0][lane] = s.a;
-    s_agg[wi][1][lane] = s.b;
-    s_agg[wi][2][lane] = s.P;
+    put_st(s_agg[wi], lane, s);
   }
   __syncthreads();
 
@@ -224,10 +142,8 @@ __global__ void __launch_bounds__(W * 32) fwd_chunked_kernel(FwdArgs p) {
     St acc = st_empty();
 #pragma unroll
     for (int i = 0; i < W; ++i) {
-      s_pre[i][0][lane] = acc.a;
-      s_pre[i][1][lane] = acc.b;
-      s_pre[i][2][lane] = acc.P;
-      const St si{s_agg[i][0][lane], s_agg[i][1][lane], s_agg[i][2][lane]};
+      put_st(s_pre[i], lane, acc);
+      const St si = get_st(s_agg[i], lane);
       const int li = (int)max((int64_t)0, min((int64_t)L, T - (tc0 + (int64_t)i * L)));
       acc = combine(acc, si, (float)li, w2);
     }
@@ -235,19 +151,17 @@ __global__ void __launch_bounds__(W * 32) fwd_chunked_kernel(FwdArgs p) {
     const St excl = chunk_scan(p.flags, p.desc, chunk, chain, p.nchains, acc, (float)chunk_len,
                                (float)TC, initial, st_empty(), epoch, p.hdr, p.spin_limit,
                                chunk + 1 < p.nchunks, !(p.hold_first && chunk == 0), w2, lane);
-    s_carry[0][lane] = excl.a;
-    s_carry[1][lane] = excl.b;
-    s_carry[2][lane] = excl.P;
+    put_st(s_carry, lane, excl);
   }
   __syncthreads();
   finish_block(p.hdr, gridDim.x);
 
   // Pass 2: replay the segment from the carried-in state.
   if (nvalid > 0) {
-    const St cin{s_carry[0][lane], s_carry[1][lane], s_carry[2][lane]};
-    const St pre{s_pre[wi][0][lane], s_pre[wi][1][lane], s_pre[wi][2][lane]};
+    const St cin = get_st(s_carry, lane);
+    const St pre = get_st(s_pre[wi], lane);
     const St start = combine(cin, pre, (float)min(wi * L, chunk_len), w2);
-    if (p.ckpt && cok && (t0 % kCkpt) == 0) store_ckpt(p.ckpt, t0 / kCkpt, b * C + c, BC, start);
+    if (p.ckpt && cok && (t0 % kCkpt) == 0) store_ckpt(p.ckpt, t0 / kCkpt, b * C + c, BC, start, w2);
     Run s = run_from(start);
     E *yp = p.y ? static_cast<E *>(p.y) + (b * T + t0) * C + c : nullptr;
 #pragma unroll
@@ -257,31 +171,315 @@ __global__ void __launch_bounds__(W * 32) fwd_chunked_kernel(FwdArgs p) {
         if (yp && cok) IO<E>::st(yp + (int64_t)j * C, y);
       }
     }
-    if (p.state_out && cok && t0 + nvalid == T) store_state(p.state_out, b * C + c, BC, run_state(s, w2));
+    if (p.state_out && cok && t0 + nvalid == T) store_state(p.state_out, b * C + c, BC, run_state(s), w2);
+  }
+}
+
+// ------------------------------------------------------------------------
+// TMA-fed persistent chunked scan (the default forward on sm_100a).
+//
+// Block = W compute warps + 1 scan warp + 1 producer warp; grid = one
+// resident wave (cooperative launch), block g owns tiles g, g+G, g+2G, ...
+// of the (position-major) tile order.  A tile is 32 channels x TC = W*L
+// tokens of one batch row.
+//   producer  lane 0 streams the k and v tiles into an S-stage shared ring
+//             with 2-D TMA loads that complete on mbarriers.
+//   compute   warp w owns rows [w*L, (w+1)*L) of every tile.  Iteration i:
+//             pass 1 (segment summary) of tile i, then pass 2 (replay, y) of
+//             tile i-1 from the carried-in state the scan warp prepared.
+//   scan      joins tile i's W summaries, runs the cross-block chunk scan
+//             (Fenwick nodes, deterministic) and writes each warp's
+//             starting state.  Running one tile behind the compute warps
+//             keeps its global-memory round trips off their critical path.
+// k and v are read from HBM once; pass 2 re-reads them from shared memory.
+// ------------------------------------------------------------------------
+template <typename E, int W, int L, int S>
+struct TmaFwdLayout {
+  static constexpr int TC = W * L;
+  static constexpr int ROWB = 32 * (int)sizeof(E);
+  static constexpr int TILEB = TC * ROWB;                 // one array, one tile
+  static constexpr int STAGE_OFF = 0;                     // [S][2][TC][32] E
+  static constexpr int SUMS_OFF = S * 2 * TILEB;          // [2][W][4][32] f32
+  static constexpr int CARRY_OFF = SUMS_OFF + 2 * W * 128 * 4;
+  static constexpr int BAR_OFF = CARRY_OFF + 2 * W * 128 * 4;  // full[S] empty[S] sfull[2] cfull[2]
+  static constexpr int FLAG_OFF = BAR_OFF + (2 * S + 4) * 8;  // abort flag
+  static constexpr int BYTES = FLAG_OFF + 16;
+};
+
+template <typename E, int W, int L, int S>
+__global__ void __launch_bounds__((W + 2) * 32) fwd_tma_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                               const __grid_constant__ CUtensorMap vmap,
+                                                               FwdArgs p) {
+  using Lay = TmaFwdLayout<E, W, L, S>;
+  constexpr int TC = Lay::TC;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  int &s_abort = *reinterpret_cast<int *>(smem + Lay::FLAG_OFF);
+  const int wi = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ntiles = p.nchains * p.nchunks;
+  const int64_t G = gridDim.x;
+  const int64_t n = (ntiles - (int64_t)blockIdx.x + G - 1) / G;  // this block's tiles
+  const uint32_t bar0 = smem_addr(smem + Lay::BAR_OFF);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (S + s); };
+  auto sfull = [&](int b) { return bar0 + 8u * (2 * S + b); };
+  auto cfull = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
+  const int64_t T = p.T, C = p.C, BC = p.B * p.C;
+  auto stage_ptr = [&](int s, int arr) {
+    return reinterpret_cast<const E *>(smem + Lay::STAGE_OFF + (size_t)(s * 2 + arr) * Lay::TILEB);
+  };
+  float *sums = reinterpret_cast<float *>(smem + Lay::SUMS_OFF);
+  float *carry = reinterpret_cast<float *>(smem + Lay::CARRY_OFF);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), W);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sfull(b), W);
+      mbar_init(cfull(b), 1);
+    }
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  volatile int *abort = &s_abort;
+  const int64_t lim = p.spin_limit * 1000;  // wait budget in ns (default ~1 s)
+
+  if (wi == W + 1) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      int64_t issued = 0;
+      for (int64_t i = 0; i < n; ++i) {
+        const int s = (int)(i % S);
+        if (i >= S && !mbar_wait(empty(s), (uint32_t)((i / S) - 1) & 1u, lim, abort)) break;
+        if (*abort) break;
+        const int64_t tile = (int64_t)blockIdx.x + i * G;
+        const int64_t chunk = tile / p.nchains, chain = tile - chunk * p.nchains;
+        const int64_t b = chain / p.nct;
+        const int x = (int)((chain - b * p.nct) * 32);
+        const int y = (int)(b * T + chunk * TC);
+        mbar_expect_tx(full(s), 2u * Lay::TILEB);
+        tma_load_2d(smem_addr(stage_ptr(s, 0)), &kmap, x, y, full(s));
+        tma_load_2d(smem_addr(stage_ptr(s, 1)), &vmap, x, y, full(s));
+        issued = i + 1;
+      }
+      if (*abort) {
+        // Let every load this block issued land before the block can exit.
+        for (int64_t i = (issued > S ? issued - S : 0); i < issued; ++i)
+          mbar_wait(full((int)(i % S)), (uint32_t)(i / S) & 1u, lim, nullptr);
+      }
+    }
+  } else if (wi == W) {
+    // -------------------------------------------------------------- scan
+    unsigned epoch = 0;
+    if (lane == 0) epoch = ld_relaxed(&p.hdr->epoch);
+    epoch = __shfl_sync(0xffffffffu, epoch, 0);
+    for (int64_t i = 0; i < n; ++i) {
+      const int buf = (int)(i & 1);
+      if (!mbar_wait(sfull(buf), (uint32_t)(i >> 1) & 1u, lim, abort)) {
+        if (lane == 0) {
+          *abort = 1;
+          raise_timeout(p.hdr, epoch);
+        }
+        break;
+      }
+      const int64_t tile = (int64_t)blockIdx.x + i * G;
+      const int64_t chunk = tile / p.nchains, chain = tile - chunk * p.nchains;
+      const int64_t b = chain / p.nct;
+      const int64_t c = (chain - b * p.nct) * 32 + lane;
+      const bool cok = c < C;
+      const float w2 = cok ? __ldg(p.w + c) * kLog2e : 0.f;
+      const int chunk_len = (int)min((int64_t)TC, T - chunk * TC);
+      // local prefixes of the W segments (block-local, from the empty state)
+      St pre[W];
+      St acc = st_empty();
+      const float *sb = sums + buf * W * 128;
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        pre[w] = acc;
+        const St si = get_st(sb + w * 128, lane);
+        const int lw = (int)max((int64_t)0, min((int64_t)L, T - (chunk * TC + (int64_t)w * L)));
+        acc = combine(acc, si, (float)lw, w2);
+      }
+      const St initial = cok ? load_state_in(p.state_in, b * C + c, BC) : st_empty();
+      const St excl = chunk_scan(p.flags, p.desc, chunk, chain, p.nchains, acc, (float)chunk_len,
+                                 (float)TC, initial, st_empty(), epoch, p.hdr, p.spin_limit,
+                                 chunk + 1 < p.nchunks, !(p.hold_first && chunk == 0), w2, lane);
+      float *cb = carry + buf * W * 128;
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const St st = combine(excl, pre[w], (float)min(w * L, chunk_len), w2);
+        put_st(cb + w * 128, lane, st);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(cfull(buf));
+    }
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      const unsigned prev = atomicAdd(&p.hdr->done, 1u);
+      if (prev == gridDim.x - 1u) {
+        p.hdr->ticket = 0u;
+        p.hdr->done = 0u;
+        __threadfence();
+        atomicAdd(&p.hdr->epoch, 1u);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- compute
+    const int w = wi;
+    for (int64_t i = 0; i <= n; ++i) {
+      if (i < n) {
+        const int s = (int)(i % S);
+        if (!mbar_wait(full(s), (uint32_t)(i / S) & 1u, lim, abort)) {
+          *abort = 1;
+          break;
+        }
+        const int64_t tile = (int64_t)blockIdx.x + i * G;
+        const int64_t chunk = tile / p.nchains, chain = tile - chunk * p.nchains;
+        const int64_t b = chain / p.nct;
+        const int64_t c = (chain - b * p.nct) * 32 + lane;
+        const bool cok = c < C;
+        const float w2 = cok ? __ldg(p.w + c) * kLog2e : 0.f;
+        const int nvalid = (int)max((int64_t)0, min((int64_t)L, T - (chunk * TC + (int64_t)w * L)));
+        const E *kr = stage_ptr(s, 0) + (size_t)w * L * 32 + lane;
+        const E *vr = stage_ptr(s, 1) + (size_t)w * L * 32 + lane;
+        float K[L], V[L];
+#pragma unroll
+        for (int j = 0; j < L; ++j) {
+          K[j] = to_f32(kr[j * 32]) * kLog2e;
+          V[j] = to_f32(vr[j * 32]);
+        }
+        const St sm = summarize<L>(K, V, w2, nvalid);
+        put_st(sums + (i & 1) * W * 128 + w * 128, lane, sm);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sfull((int)(i & 1)));
+      }
+      if (i >= 1) {
+        const int64_t j = i - 1;
+        const int s = (int)(j % S);
+        if (!mbar_wait(cfull((int)(j & 1)), (uint32_t)(j >> 1) & 1u, lim, abort)) {
+          *abort = 1;
+          break;
+        }
+        const int64_t tile = (int64_t)blockIdx.x + j * G;
+        const int64_t chunk = tile / p.nchains, chain = tile - chunk * p.nchains;
+        const int64_t b = chain / p.nct;
+        const int64_t c = (chain - b * p.nct) * 32 + lane;
+        const bool cok = c < C;
+        const float w2 = cok ? __ldg(p.w + c) * kLog2e : 0.f;
+        const float u2 = cok ? __ldg(p.u + c) * kLog2e : 0.f;
+        const int64_t t0 = chunk * TC + (int64_t)w * L;
+        const int nvalid = (int)max((int64_t)0, min((int64_t)L, T - t0));
+        const St start = get_st(carry + (j & 1) * W * 128 + w * 128, lane);
+        if (nvalid > 0) {
+          if (p.ckpt && cok && (t0 % kCkpt) == 0) store_ckpt(p.ckpt, t0 / kCkpt, b * C + c, BC, start, w2);
+          const E *kr = stage_ptr(s, 0) + (size_t)w * L * 32 + lane;
+          const E *vr = stage_ptr(s, 1) + (size_t)w * L * 32 + lane;
+          Run st = run_from(start);
+          E *yp = p.y ? static_cast<E *>(p.y) + (b * T + t0) * C + c : nullptr;
+#pragma unroll
+          for (int q = 0; q < L; ++q) {
+            if (q < nvalid) {
+              const float yv = fwd_token(st, to_f32(kr[q * 32]) * kLog2e, to_f32(vr[q * 32]), u2, w2);
+              if (yp && cok) IO<E>::st(yp + (int64_t)q * C, yv);
+            }
+          }
+          if (p.state_out && cok && t0 + nvalid == T)
+            store_state(p.state_out, b * C + c, BC, run_state(st), w2);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty(s));
+      }
+    }
   }
 }
 
 // ---------------------------------------------------------------- launch ---
 constexpr int kSeqU = 8;
-constexpr int kFwdW = 8, kFwdL = 16;
+constexpr int kFwdW = 4, kFwdL = 16;            // register-tile fallback kernel
+constexpr int kTmaW = 4, kTmaL = 16, kTmaS = 4;  // TMA kernel
+static_assert(kFwdW * kFwdL == kTmaW * kTmaL, "both chunked kernels use one chunk length");
 
 int64_t fwd_chunk_tokens() { return kFwdW * kFwdL; }
 
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// [B*T, C] view of a [B, T, C] tensor, boxes of 32 columns x `rows` rows.
+bool encode_rows(CUtensorMap *m, const void *ptr, int dtype, int64_t rows, int64_t C,
+                 int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const size_t es = dtype == 0 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(C * es)};
+  cuuint32_t box[2] = {32u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// TMA needs 16-byte aligned rows and base addresses, and row indices < 2^31.
+bool fwd_tma_eligible(const FwdArgs &a, int dtype) {
+  const int64_t es = dtype == 0 ? 4 : 2;
+  return (a.C * es) % 16 == 0 && ((uintptr_t)a.k % 16) == 0 && ((uintptr_t)a.v % 16) == 0 &&
+         a.B * a.T < (int64_t(1) << 31) && tensor_map_encoder() != nullptr;
+}
+
 template <typename E>
-static cudaError_t launch_fwd_t(const FwdArgs &a, bool chunked, cudaStream_t st) {
-  if (!chunked) {
+static cudaError_t launch_fwd_tma_t(const FwdArgs &a, int dtype, int num_sms, cudaStream_t st) {
+  using Lay = TmaFwdLayout<E, kTmaW, kTmaL, kTmaS>;
+  CUtensorMap km, vm;
+  if (!encode_rows(&km, a.k, dtype, a.B * a.T, a.C, Lay::TC) ||
+      !encode_rows(&vm, a.v, dtype, a.B * a.T, a.C, Lay::TC))
+    return cudaErrorInvalidValue;
+  auto kern = fwd_tma_kernel<E, kTmaW, kTmaL, kTmaS>;
+  const int threads = (kTmaW + 2) * 32;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::BYTES);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, Lay::BYTES);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int64_t tiles = a.nchains * a.nchunks;
+  const int64_t grid = tiles < (int64_t)per_sm * num_sms ? tiles : (int64_t)per_sm * num_sms;
+  FwdArgs args = a;
+  void *kargs[] = {&km, &vm, &args};
+  return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3(threads), kargs,
+                                     (size_t)Lay::BYTES, st);
+}
+
+template <typename E>
+static cudaError_t launch_fwd_t(const FwdArgs &a, int kind, int dtype, int num_sms, cudaStream_t st) {
+  if (kind == 0) {
     const int64_t BC = a.B * a.C;
     const unsigned grid = (unsigned)((BC + 255) / 256);
     fwd_seq_kernel<E, kSeqU><<<grid, 256, 0, st>>>(a);
-  } else {
-    const int64_t tiles = a.nchains * a.nchunks;
-    fwd_chunked_kernel<E, kFwdW, kFwdL><<<(unsigned)tiles, kFwdW * 32, 0, st>>>(a);
+    return cudaGetLastError();
   }
+  if (kind == 2) return launch_fwd_tma_t<E>(a, dtype, num_sms, st);
+  const int64_t tiles = a.nchains * a.nchunks;
+  fwd_chunked_kernel<E, kFwdW, kFwdL><<<(unsigned)tiles, kFwdW * 32, 0, st>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_forward(const FwdArgs &a, int dtype, bool chunked, cudaStream_t st) {
-  return dtype == 0 ? launch_fwd_t<float>(a, chunked, st) : launch_fwd_t<uint16_t>(a, chunked, st);
+// kind: 0 sequential, 1 register-tile chunked, 2 TMA chunked.
+cudaError_t launch_forward(const FwdArgs &a, int dtype, int kind, int num_sms, cudaStream_t st) {
+  return dtype == 0 ? launch_fwd_t<float>(a, kind, dtype, num_sms, st)
+                    : launch_fwd_t<uint16_t>(a, kind, dtype, num_sms, st);
 }
 
 }  // namespace wkv

@@ -42,26 +42,34 @@ __device__ __forceinline__ float rcp(float x) {
   return y;
 }
 
-// Forward state of one channel: A = a 2^P, B = b 2^P.
+// Forward state of one channel: A = a 2^E, B = b 2^E with the exponent in
+// anchored form E = P + n w (P: the exponent of the term that set the
+// maximum, n: decay steps since then, an exact integer in a float).  Carrying
+// (P, n) instead of the rounded sum keeps E within one rounding of exact
+// through any number of joins, however long the sequence.
 struct St {
-  float a, b, P;
+  float a, b, P, n;
 };
-__device__ __forceinline__ St st_empty() { return St{0.f, 0.f, kEmptyP}; }
+__device__ __forceinline__ St st_empty() { return St{0.f, 0.f, kEmptyP, 0.f}; }
+__device__ __forceinline__ float st_exp(const St &s, float w2) { return fmaf(s.n, w2, s.P); }
 
 // Sequence X followed by a sequence Y of lenY tokens: X's sums decay lenY
 // times (exponent + lenY * w), then the two are added at the larger scale.
 // This is the associative combine that lets the time axis be split into
 // chunks ("Transformer-유사학습": the serial WKV part is done as a scan).
 __device__ __forceinline__ St combine(const St &X, const St &Y, float lenY, float w2) {
-  const float Px = fmaf(lenY, w2, X.P);
-  const float d = Px - Y.P;
+  const float nx = X.n + lenY;
+  const float Ex = fmaf(nx, w2, X.P);
+  const float Ey = fmaf(Y.n, w2, Y.P);
+  const float d = Ex - Ey;
   const float x = ex2(-fabsf(d));
   const bool xw = d >= 0.f;
   const float fx = xw ? 1.f : x, fy = xw ? x : 1.f;
   St r;
   r.a = fmaf(X.a, fx, Y.a * fy);
   r.b = fmaf(X.b, fx, Y.b * fy);
-  r.P = fmaxf(Px, Y.P);
+  r.P = xw ? X.P : Y.P;
+  r.n = xw ? nx : Y.n;
   return r;
 }
 
@@ -154,28 +162,40 @@ __device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Per-tile descriptor: one record (the Fenwick node of the chunk) of three
-// float planes of 32 lanes each.
-constexpr int kDescFloats = 3 * 32;
+// Per-tile descriptor: one record (the Fenwick node of the chunk) of up to
+// four float planes of 32 lanes each.
+constexpr int kDescFloats = 4 * 32;
 
 template <typename S>
 __device__ __forceinline__ void desc_store(float *desc, int64_t tile, int which, const S &s,
                                            int lane) {
-  float *d = desc + tile * kDescFloats + which * 96;
+  constexpr int NF = sizeof(S) / sizeof(float);
+  static_assert(NF * 32 <= kDescFloats, "record too large");
+  float *d = desc + tile * kDescFloats + which * NF * 32;
   const float *f = reinterpret_cast<const float *>(&s);
-  __stcg(d + lane, f[0]);
-  __stcg(d + 32 + lane, f[1]);
-  __stcg(d + 64 + lane, f[2]);
+#pragma unroll
+  for (int i = 0; i < NF; ++i) __stcg(d + i * 32 + lane, f[i]);
 }
 template <typename S>
 __device__ __forceinline__ S desc_load(const float *desc, int64_t tile, int which, int lane) {
-  const float *d = desc + tile * kDescFloats + which * 96;
+  constexpr int NF = sizeof(S) / sizeof(float);
+  const float *d = desc + tile * kDescFloats + which * NF * 32;
   S s;
   float *f = reinterpret_cast<float *>(&s);
-  f[0] = __ldcg(d + lane);
-  f[1] = __ldcg(d + 32 + lane);
-  f[2] = __ldcg(d + 64 + lane);
+#pragma unroll
+  for (int i = 0; i < NF; ++i) f[i] = __ldcg(d + i * 32 + lane);
   return s;
+}
+
+// A state in four planes of 32 lanes (shared or global memory).
+__device__ __forceinline__ void put_st(float *d, int lane, const St &s) {
+  d[lane] = s.a;
+  d[32 + lane] = s.b;
+  d[64 + lane] = s.P;
+  d[96 + lane] = s.n;
+}
+__device__ __forceinline__ St get_st(const float *d, int lane) {
+  return St{d[lane], d[32 + lane], d[64 + lane], d[96 + lane]};
 }
 
 // Publish a record and then its flag with release semantics (all lanes of
@@ -318,6 +338,60 @@ __device__ S chunk_scan(unsigned *flags, float *desc, int64_t pos, int64_t chain
     x &= x - 1;
   }
   return pjoin(base0, acc, acc_len, w2);
+}
+
+// ------------------------------------------------- mbarrier / TMA (sm_100a) ---
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait for the phase of `bar` with the given parity to complete.
+// Gives up (returns false) after `budget_ns` nanoseconds or once *abort is
+// set (abort may be null).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int64_t budget_ns,
+                                          volatile int *abort) {
+  const uint64_t t0 = global_ns();
+  for (unsigned i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 15u) {
+      if (abort && *abort) return false;
+      if ((int64_t)(global_ns() - t0) > budget_ns) return false;
+    }
+  }
+}
+// 2-D tiled TMA load of box {32 columns, rows} at column x, row y into shared
+// memory, completing on `bar` (transaction bytes).  No multicast.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
 }
 
 // ---------------------------------------------------- launch descriptors ---

@@ -18,7 +18,9 @@ from gpu_util import (BF16_TOL, F32_FWD_TOL, F32_GRAD_TOL, channel_subset, dev, 
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = {"seq": W.WKV_KERNEL_SEQUENTIAL, "chunked": W.WKV_KERNEL_CHUNKED}
+KERNELS = {"seq": W.WKV_KERNEL_SEQUENTIAL, "chunked": W.WKV_KERNEL_CHUNKED,
+           "chunked_regs": W.WKV_KERNEL_CHUNKED_REGS, "chain": W.WKV_KERNEL_CHAIN}
+BWD_KERNELS = {"chain": W.WKV_KERNEL_CHAIN, "chunked": W.WKV_KERNEL_CHUNKED}
 
 
 def small_case(B, T, C, seed, dtype="f32", td=(-3.0, 1.0), kstd=1.0, state=False):
@@ -213,25 +215,36 @@ def assert_grads(got, ref, tol):
         assert e <= tol, (n, e)
 
 
+@pytest.mark.parametrize("kernel", sorted(BWD_KERNELS))
 @pytest.mark.parametrize("use_ckpt", [True, False])
 @pytest.mark.parametrize("shape", [(1, 1, 64), (2, 7, 33), (3, 200, 70), (2, 129, 64),
-                                   (1, 1000, 96)])
-def test_backward_small_shapes(shape, use_ckpt):
+                                   (1, 1000, 96), (2, 300, 40)])
+def test_backward_small_shapes(shape, use_ckpt, kernel):
     B, T, C = shape
     w, u, k, v, g, _ = small_case(B, T, C, seed=T + 3 * C)
     W_, U_, K_, V_ = dev(w), dev(u), dev(k), dev(v)
     ck = None
     if use_ckpt:
         _, _, ck = W.forward(W_, U_, K_, V_, want_ckpt=True)
-    got = W.backward(W_, U_, K_, V_, dev(g), ckpt=ck)
+    got = W.backward(W_, U_, K_, V_, dev(g), ckpt=ck, kernel=BWD_KERNELS[kernel])
     assert_grads(got, grads_ref(w, u, k, v, g), F32_GRAD_TOL)
 
 
-def test_backward_with_state_in():
+@pytest.mark.parametrize("kernel", sorted(BWD_KERNELS))
+def test_backward_with_state_in(kernel):
     B, T, C = 2, 300, 64
     w, u, k, v, g, st = small_case(B, T, C, seed=13, state=True)
-    got = W.backward(dev(w), dev(u), dev(k), dev(v), dev(g), dev(st))
+    got = W.backward(dev(w), dev(u), dev(k), dev(v), dev(g), dev(st), kernel=BWD_KERNELS[kernel])
     assert_grads(got, grads_ref(w, u, k, v, g, st), F32_GRAD_TOL)
+
+
+@pytest.mark.parametrize("kernel", sorted(BWD_KERNELS))
+def test_backward_bf16_small(kernel):
+    B, T, C = 2, 333, 64
+    w, u, k, v, g, _ = small_case(B, T, C, seed=19, dtype="bf16")
+    bf = lambda x: dev(x, torch.bfloat16)
+    got = W.backward(dev(w), dev(u), bf(k), bf(v), bf(g), kernel=BWD_KERNELS[kernel])
+    assert_grads(got, grads_ref(w, u, k, v, g), BF16_TOL)
 
 
 def test_backward_tiny_workload_vs_direct():
