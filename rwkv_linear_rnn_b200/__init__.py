@@ -13,28 +13,52 @@ There is no CPU or PyTorch fallback.
 """
 from __future__ import annotations
 
-import ctypes
-import os
+import importlib
 
-from . import abi
-from .abi import (WKV_BF16, WKV_F32, WKV_KERNEL_AUTO, WKV_KERNEL_CHAIN, WKV_KERNEL_CHUNKED,
-                  WKV_KERNEL_CHUNKED_REGS,
-                  WKV_KERNEL_SEQUENTIAL,
-                  WKV_OP_BACKWARD, WKV_OP_FORWARD, WKV_OP_STEP, WKVError, wkv_ckpt_size,
-                  wkv_strerror, wkv_version, wkv_workspace_size)
+from .constants import (WKV_BF16, WKV_F32, WKV_KERNEL_AUTO, WKV_KERNEL_CHAIN, WKV_KERNEL_CHUNKED,
+                        WKV_KERNEL_CHUNKED_REGS, WKV_KERNEL_SEQUENTIAL, WKV_OP_BACKWARD,
+                        WKV_OP_FORWARD, WKV_OP_STEP, WKV_STATIC_SCRATCH_BYTES)
 
 __all__ = [
     "abi", "WKVError", "WKV_F32", "WKV_BF16", "WKV_OP_FORWARD", "WKV_OP_BACKWARD", "WKV_OP_STEP",
     "WKV_KERNEL_AUTO", "WKV_KERNEL_SEQUENTIAL", "WKV_KERNEL_CHUNKED", "WKV_KERNEL_CHUNKED_REGS",
-    "WKV_KERNEL_CHAIN",
-    "Workspace", "forward",
-    "backward", "step", "WKV", "wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror",
-    "wkv_version", "library_path",
+    "WKV_KERNEL_CHAIN", "WKV_STATIC_SCRATCH_BYTES", "Workspace", "forward", "backward", "step",
+    "WKV", "wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror", "wkv_version",
+    "library_path",
 ]
 
 
+def __getattr__(name):
+    # The ctypes layer (and with it libwkv.so) loads on first use; it raises
+    # ImportError with a build hint if the library has not been built.
+    if name in ("abi", "WKVError"):
+        abi_mod = importlib.import_module(".abi", __name__)
+        return abi_mod if name == "abi" else abi_mod.WKVError
+    raise AttributeError(name)
+
+
+def _abi():
+    return importlib.import_module(".abi", __name__)
+
+
+def wkv_workspace_size(op, B, T, C, dtype):
+    return _abi().wkv_workspace_size(op, B, T, C, dtype)
+
+
+def wkv_ckpt_size(B, T, C):
+    return _abi().wkv_ckpt_size(B, T, C)
+
+
+def wkv_strerror(status):
+    return _abi().wkv_strerror(status)
+
+
+def wkv_version():
+    return _abi().wkv_version()
+
+
 def library_path() -> str:
-    return abi.LIB_PATH
+    return _abi().LIB_PATH
 
 
 def _torch():
@@ -98,7 +122,7 @@ class Workspace:
         """Device-side status of earlier calls (waits for the stream); clears it."""
         if self.buf is None:
             return 0
-        return abi.wkv_get_status(self.buf.data_ptr(), _stream(stream))
+        return _abi().wkv_get_status(self.buf.data_ptr(), _stream(stream))
 
 
 _default_ws = {}
@@ -130,6 +154,7 @@ def forward(w, u, k, v, state_in=None, *, want_state=False, want_ckpt=False, y=N
         ckpt = torch.empty(max(n, 1), dtype=torch.float32, device=k.device)
     ws = _ws_for(k.device, workspace)
     buf, nbytes = ws.get(WKV_OP_FORWARD, B, T, C, dt)
+    abi = _abi()
     opts = abi.Options(kernel=kernel)
     abi.check(abi.wkv_forward_ex(B, T, C, dt, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(state_in),
                                  _ptr(y), _ptr(state_out), _ptr(ckpt), _ptr(buf), nbytes,
@@ -150,6 +175,7 @@ def backward(w, u, k, v, grad_y, state_in=None, ckpt=None, *, workspace=None, st
     gv = torch.empty_like(v)
     ws = _ws_for(k.device, workspace)
     buf, nbytes = ws.get(WKV_OP_BACKWARD, B, T, C, dt)
+    abi = _abi()
     opts = abi.Options(kernel=kernel)
     abi.check(abi.wkv_backward_ex(B, T, C, dt, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(grad_y),
                                   _ptr(state_in), _ptr(ckpt), _ptr(gw), _ptr(gu), _ptr(gk),
@@ -167,6 +193,7 @@ def step(w, u, k_t, v_t, state, *, y=None, state_out=None, stream=None):
         y = torch.empty_like(k_t)
     if state_out is None:
         state_out = state
+    abi = _abi()
     abi.check(abi.wkv_step(N, C, _ptr(w), _ptr(u), _ptr(k_t), _ptr(v_t), _ptr(state), _ptr(y),
                            _ptr(state_out), _stream(stream)))
     return y, state_out

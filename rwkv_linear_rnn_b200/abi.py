@@ -11,12 +11,8 @@ import os
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwkv.so")
 
-WKV_F32, WKV_BF16 = 0, 1
-WKV_OK, WKV_ERR_INVALID_ARG, WKV_ERR_UNSUPPORTED, WKV_ERR_WORKSPACE, WKV_ERR_CUDA, \
-    WKV_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
-WKV_OP_FORWARD, WKV_OP_BACKWARD, WKV_OP_STEP = 0, 1, 2
-WKV_KERNEL_AUTO, WKV_KERNEL_SEQUENTIAL, WKV_KERNEL_CHUNKED, WKV_KERNEL_CHUNKED_REGS, \
-    WKV_KERNEL_CHAIN = 0, 1, 2, 3, 4
+from .constants import *  # noqa: F401,F403  (codes shared with include/wkv.h)
+from .constants import WKV_OK
 
 # Every symbol the header declares, in declaration order.
 EXPORTS = (
