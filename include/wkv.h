@@ -205,6 +205,36 @@ int wkv_step(int64_t N, int64_t C, const float *w, const float *u,
              float *state_out, void *stream);
 
 /*
+ * wkv_backward_static -- wkv_backward for callers that cannot allocate.
+ *
+ * The paper has no counterpart; this is a deployment convenience.  Callers
+ * running where cudaMalloc is not allowed (inside an allocator or memory-pool
+ * callback, in plugin hosts that only hand out fixed buffers, on threads of
+ * runtimes that forbid device allocation) cannot provide the workspace
+ * wkv_backward needs.  This entry point takes the same arguments minus the
+ * workspace and uses a file-scope static device array of
+ * WKV_STATIC_SCRATCH_BYTES instead; it calls no cudaMalloc/cudaFree and no
+ * allocating library routine.  Inputs and outputs are still the caller's.
+ *   - Limit: problems with wkv_workspace_size(WKV_OP_BACKWARD, B, T, C, dtype)
+ *     above WKV_STATIC_SCRATCH_BYTES are rejected with WKV_ERR_WORKSPACE.
+ *   - Set-up: the first call on each device (with that device current) looks
+ *     up the array's device address with cudaGetSymbolAddress and zero-fills
+ *     it synchronously; make that first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents.  Calls whose executions overlap on the GPU (other
+ *     streams, other host threads) race on it and give wrong results; order
+ *     them on one stream.
+ *   - Each GPU that loads the library holds the array until the process
+ *     exits.  Device-side wait failures are not reported by this entry point.
+ * Returns the codes of wkv_backward, plus WKV_ERR_CUDA if the set-up fails.
+ */
+#define WKV_STATIC_SCRATCH_BYTES (16u << 20) /* 16 MiB */
+int wkv_backward_static(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                        const float *u, const void *k, const void *v, const void *grad_y,
+                        const float *state_in, const float *ckpt, float *grad_w,
+                        float *grad_u, void *grad_k, void *grad_v, void *stream);
+
+/*
  * Waits for `stream`, then returns and clears the device-side status word of
  * the workspace: WKV_OK, or WKV_ERR_TIMEOUT if a bounded wait of an earlier
  * call on it gave up (its results are then invalid).  WKV_ERR_CUDA if the

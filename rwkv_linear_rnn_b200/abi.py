@@ -17,8 +17,8 @@ from .constants import WKV_OK
 # Every symbol the header declares, in declaration order.
 EXPORTS = (
     "wkv_workspace_size", "wkv_workspace_init", "wkv_ckpt_size", "wkv_forward", "wkv_forward_ex",
-    "wkv_backward", "wkv_backward_ex", "wkv_step", "wkv_get_status", "wkv_strerror",
-    "wkv_version",
+    "wkv_backward", "wkv_backward_ex", "wkv_step", "wkv_backward_static", "wkv_get_status",
+    "wkv_strerror", "wkv_version",
 )
 
 
@@ -49,6 +49,8 @@ _SIGS = {
     "wkv_backward_ex": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                _p, _p, _sz, _p, _opt]),
     "wkv_step": (_int, [_i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "wkv_backward_static": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p,
+                                   _p, _p, _p]),
     "wkv_get_status": (_int, [_p, _p]),
     "wkv_strerror": (ctypes.c_char_p, [_int]),
     "wkv_version": (_int, []),
@@ -106,6 +108,13 @@ def wkv_backward_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, 
 
 def wkv_step(N, C, w, u, k_t, v_t, state_in, y_t, state_out, stream):
     return lib.wkv_step(N, C, w, u, k_t, v_t, state_in, y_t, state_out, stream)
+
+
+def wkv_backward_static(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u,
+                        grad_k, grad_v, stream):
+    return lib.wkv_backward_static(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w,
+                                   grad_u, grad_k, grad_v, stream)
+
 
 
 def wkv_get_status(ws, stream):
