@@ -83,7 +83,8 @@ enum { WKV_OP_FORWARD = 0, WKV_OP_BACKWARD = 1, WKV_OP_STEP = 2 };
 
 /* Kernel selector (wkv_options.kernel). */
 enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
-       WKV_KERNEL_CHUNKED_REGS = 3, WKV_KERNEL_CHAIN = 4 };
+       WKV_KERNEL_CHUNKED_REGS = 3, WKV_KERNEL_CHAIN = 4, WKV_KERNEL_SPLIT = 5,
+       WKV_KERNEL_SEGMENT = 6 };
 
 /*
  * Optional knobs for the *_ex calls.  A NULL options pointer, or all fields
@@ -97,8 +98,14 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
  *               variant of the chunked kernel (no TMA); CHAIN runs one block
  *               per (batch row, 32-channel) chain over all of T, tiles fed
  *               by TMA, the carry kept on chip (needs 16-byte aligned rows;
- *               the default when they are).  The backward honours
- *               CHAIN/AUTO (chain kernel) versus any other value (chunked).
+ *               the default when they are).  SPLIT runs three launches: chunk
+ *               summaries, a per-chain prefix over them, and a replay of
+ *               every chunk from its start state.  SEGMENT (the forward
+ *               default when rows are 16-byte aligned) gives each warp a
+ *               128/256-token segment of one chain: summary, a fixed-order
+ *               join with at most 32 earlier records, and the replay from L2.
+ *               The backward honours CHAIN/AUTO (chain kernel) versus any
+ *               other value (chunked).
  *   spin_limit  polls a block makes on one predecessor's flag before it gives
  *               up with WKV_ERR_TIMEOUT (0 = default, about one second).
  *   test_hold_first_chunk

@@ -16,6 +16,9 @@ cudaError_t launch_forward_chain(const FwdArgs &a, int dtype, cudaStream_t st);
 cudaError_t launch_backward_chain(const BwdArgs &a, int dtype, cudaStream_t st);
 cudaError_t launch_reduce_wu(const float *part, int64_t nchunks, int64_t B, int64_t C, float *gw,
                              float *gu, cudaStream_t st);
+cudaError_t launch_forward_scan3(const FwdArgs &f, int dtype, float *sums, float *carry,
+                                 int num_sms, cudaStream_t st);
+cudaError_t launch_forward_seg(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st);
 cudaError_t launch_backward(const BwdArgs &a, int dtype, float *gw, float *gu, cudaStream_t st);
 cudaError_t launch_step(const StepArgs &a, bool vec, int num_sms, cudaStream_t st);
 int64_t fwd_chunk_tokens();
@@ -51,7 +54,7 @@ bool sizes_ok(int64_t B, int64_t T, int64_t C) {
 }
 
 struct Layout {
-  size_t flags, desc, ckpt, part, total;
+  size_t flags, desc, sums, carry, ckpt, part, total;
   int64_t nct, nchains, nchunks_f, nchunks_b;
 };
 
@@ -70,6 +73,12 @@ Layout layout(int op, int64_t B, int64_t T, int64_t C) {
   off = align_up(off + sizeof(unsigned) * (size_t)tiles, 256);
   L.desc = off;
   off = align_up(off + sizeof(float) * kDescFloats * (size_t)tiles, 256);
+  // split forward: chunk summaries (4 planes x 32 lanes per chain and chunk)
+  // and chunk start states (used when the caller passes no checkpoint buffer)
+  L.sums = off;
+  off = align_up(off + sizeof(float) * 4 * 32 * (size_t)L.nchains * (size_t)L.nchunks_b, 256);
+  L.carry = off;
+  off = align_up(off + sizeof(float) * 3 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
   L.ckpt = L.part = 0;
   if (op == WKV_OP_BACKWARD) {
     L.ckpt = off;
@@ -91,7 +100,7 @@ bool pick_chunked(const wkv_options *opt, int64_t B, int64_t T, int64_t C) {
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   if (kernel == WKV_KERNEL_SEQUENTIAL) return false;
   if (kernel == WKV_KERNEL_CHUNKED || kernel == WKV_KERNEL_CHUNKED_REGS ||
-      kernel == WKV_KERNEL_CHAIN)
+      kernel == WKV_KERNEL_CHAIN || kernel == WKV_KERNEL_SPLIT || kernel == WKV_KERNEL_SEGMENT)
     return true;
   // Enough independent chains to fill the GPU, or too short to split.
   return !(B * C >= kSeqMinChains || T <= 2 * fwd_chunk_tokens());
@@ -149,7 +158,16 @@ int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
   a.hold_first = opt ? opt->test_hold_first_chunk : 0;
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   if (chunked && fwd_tma_eligible(a, dtype) &&
-      (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_CHAIN))
+      (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT))
+    return launch_forward_seg(a, dtype, num_sms(), st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  if (chunked && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SPLIT)) {
+    float *sums = reinterpret_cast<float *>(base + L.sums);
+    float *carry = ckpt ? ckpt : reinterpret_cast<float *>(base + L.carry);
+    return launch_forward_scan3(a, dtype, sums, carry, num_sms(), st) == cudaSuccess
+               ? WKV_OK
+               : WKV_ERR_CUDA;
+  }
+  if (chunked && fwd_tma_eligible(a, dtype) && kernel == WKV_KERNEL_CHAIN)
     return launch_forward_chain(a, dtype, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
   int kind = 0;
   if (chunked) kind = (fwd_tma_eligible(a, dtype) && kernel != WKV_KERNEL_CHUNKED_REGS) ? 2 : 1;

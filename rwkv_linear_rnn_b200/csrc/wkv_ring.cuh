@@ -1,0 +1,83 @@
+// wkv_ring.cuh -- per-warp TMA ring of 16-row batches (internal).
+#pragma once
+
+#include <cuda.h>
+
+#include "wkv_internal.cuh"
+#include "wkv_split.cuh"
+
+namespace wkv {
+
+// Shared memory of a block of NW warps: all stages first (each warp's S
+// stages contiguous, every stage a multiple of 128 bytes, so every TMA
+// destination is 128-byte aligned as tensor copies require), then all the
+// mbarriers (8 bytes each).
+template <typename E, int S, int NARR = 2>
+struct WarpRing {
+  static constexpr int ARR_BYTES = kS3Batch * 32 * (int)sizeof(E);
+  static constexpr int STAGE_BYTES = NARR * ARR_BYTES;
+  static_assert(ARR_BYTES % 128 == 0, "TMA destinations must stay 128-byte aligned");
+  static constexpr int RING_BYTES = S * STAGE_BYTES;
+  static constexpr int block_bytes(int nw) { return nw * (RING_BYTES + S * 8); }
+};
+
+template <typename E, int S, int NARR = 2>
+struct Ring {
+  using L = WarpRing<E, S, NARR>;
+  unsigned char *base;
+  uint32_t bar0;
+  __device__ __forceinline__ Ring(unsigned char *smem, int wl, int nw) {
+    base = smem + (size_t)wl * L::RING_BYTES;
+    bar0 = smem_addr(smem + (size_t)nw * L::RING_BYTES) + 8u * S * wl;
+  }
+  __device__ __forceinline__ const E *stage(int s, int arr) const {
+    return reinterpret_cast<const E *>(base + (size_t)s * L::STAGE_BYTES + (size_t)arr * L::ARR_BYTES);
+  }
+  __device__ __forceinline__ uint32_t bar(int s) const { return bar0 + 8u * s; }
+  __device__ __forceinline__ void init(int lane) const {
+    if (lane == 0) {
+      for (int s = 0; s < S; ++s) mbar_init(bar(s), 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+  }
+  // Loads of batch `item` (rows y .. y+15, columns x .. x+31 of each of the
+  // NARR tensors) into stage item % S.  Returns false, issuing nothing, if a
+  // destination is not 128-byte aligned (the caller's bounded wait then
+  // fails and reports the error).
+  __device__ __forceinline__ bool issue(const CUtensorMap *const (&maps)[NARR], int64_t item, int x,
+                                       int y) const {
+    const int s = (int)(item % S);
+    uint32_t d[NARR];
+    uint32_t bad = 0;
+#pragma unroll
+    for (int a = 0; a < NARR; ++a) {
+      d[a] = smem_addr(stage(s, a));
+      bad |= d[a] & 127u;
+    }
+    if (bad) return false;
+    mbar_expect_tx(bar(s), (uint32_t)L::STAGE_BYTES);
+#pragma unroll
+    for (int a = 0; a < NARR; ++a) tma_load_2d(d[a], maps[a], x, y, bar(s));
+    return true;
+  }
+  // Same with an L2 eviction-priority policy on the loads.
+  __device__ __forceinline__ bool issue_hint(const CUtensorMap *const (&maps)[NARR], int64_t item,
+                                            int x, int y, uint64_t policy) const {
+    const int s = (int)(item % S);
+    uint32_t d[NARR];
+    uint32_t bad = 0;
+#pragma unroll
+    for (int a = 0; a < NARR; ++a) {
+      d[a] = smem_addr(stage(s, a));
+      bad |= d[a] & 127u;
+    }
+    if (bad) return false;
+    mbar_expect_tx(bar(s), (uint32_t)L::STAGE_BYTES);
+#pragma unroll
+    for (int a = 0; a < NARR; ++a) tma_load_2d_hint(d[a], maps[a], x, y, bar(s), policy);
+    return true;
+  }
+};
+
+}  // namespace wkv

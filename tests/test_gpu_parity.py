@@ -19,7 +19,8 @@ from gpu_util import (BF16_TOL, F32_FWD_TOL, F32_GRAD_TOL, channel_subset, dev, 
 pytestmark = pytest.mark.gpu
 
 KERNELS = {"seq": W.WKV_KERNEL_SEQUENTIAL, "chunked": W.WKV_KERNEL_CHUNKED,
-           "chunked_regs": W.WKV_KERNEL_CHUNKED_REGS, "chain": W.WKV_KERNEL_CHAIN}
+           "chunked_regs": W.WKV_KERNEL_CHUNKED_REGS, "chain": W.WKV_KERNEL_CHAIN,
+           "split": W.WKV_KERNEL_SPLIT, "segment": W.WKV_KERNEL_SEGMENT}
 BWD_KERNELS = {"chain": W.WKV_KERNEL_CHAIN, "chunked": W.WKV_KERNEL_CHUNKED}
 
 
