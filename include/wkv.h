@@ -98,16 +98,25 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
  *               variant of the chunked kernel (no TMA); CHAIN runs one block
  *               per (batch row, 32-channel) chain over all of T, tiles fed
  *               by TMA, the carry kept on chip (needs 16-byte aligned rows;
- *               the default when they are).  SPLIT runs three launches: chunk
+ *               the backward default when they are).  SPLIT runs three launches: chunk
  *               summaries, a per-chain prefix over them, and a replay of
  *               every chunk from its start state.  SEGMENT (the forward
  *               default when rows are 16-byte aligned) gives each warp a
  *               128/256-token segment of one chain: summary, a fixed-order
  *               join with at most 32 earlier records, and the replay from L2.
- *               The backward honours CHAIN/AUTO (chain kernel) versus any
- *               other value (chunked).
- *   spin_limit  polls a block makes on one predecessor's flag before it gives
- *               up with WKV_ERR_TIMEOUT (0 = default, about one second).
+ *               In the backward, CHAIN/AUTO select the chain kernel and
+ *               SEGMENT a one-launch segment kernel (64-token segments in
+ *               reverse order: recompute and adjoint aggregate, a
+ *               fixed-order join with at most 16 later records, then the
+ *               reverse sweep from L2; dL/dw and dL/du reduced in the same
+ *               launch after a grid barrier); both need 16-byte aligned
+ *               rows, otherwise and for any other value the chunked kernel
+ *               runs.
+ *   spin_limit  bound on any one device-side wait (a predecessor's record,
+ *               a shared-memory load, the grid barrier) in microseconds (the
+ *               chunked kernels count polls of at most about 1 us each);
+ *               past it the wait gives up with WKV_ERR_TIMEOUT (0 = default,
+ *               about one second).
  *   test_hold_first_chunk
  *               test hook: blocks of the first chunk in scan order never
  *               publish their results, so the blocks that depend on them must

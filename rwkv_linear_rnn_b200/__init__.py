@@ -163,17 +163,18 @@ def forward(w, u, k, v, state_in=None, *, want_state=False, want_ckpt=False, y=N
     return y, state_out, ckpt
 
 
-def backward(w, u, k, v, grad_y, state_in=None, ckpt=None, *, workspace=None, stream=None,
-             kernel=WKV_KERNEL_AUTO):
-    """Gradients (grad_w [C], grad_u [C], grad_k, grad_v) of L given grad_y."""
+def backward(w, u, k, v, grad_y, state_in=None, ckpt=None, *, grad_k=None, grad_v=None,
+             workspace=None, stream=None, kernel=WKV_KERNEL_AUTO):
+    """Gradients (grad_w [C], grad_u [C], grad_k, grad_v) of L given grad_y.
+    ``grad_k`` / ``grad_v`` may be given as output buffers (shape and dtype of k)."""
     torch = _torch()
-    _check_cuda(w, u, k, v, grad_y, state_in, ckpt)
+    _check_cuda(w, u, k, v, grad_y, state_in, ckpt, grad_k, grad_v)
     B, T, C = k.shape
     dt = _dtype_code(k)
     gw = torch.empty(C, dtype=torch.float32, device=k.device)
     gu = torch.empty(C, dtype=torch.float32, device=k.device)
-    gk = torch.empty_like(k)
-    gv = torch.empty_like(v)
+    gk = torch.empty_like(k) if grad_k is None else grad_k
+    gv = torch.empty_like(v) if grad_v is None else grad_v
     ws = _ws_for(k.device, workspace)
     buf, nbytes = ws.get(WKV_OP_BACKWARD, B, T, C, dt)
     abi = _abi()

@@ -19,6 +19,8 @@ cudaError_t launch_reduce_wu(const float *part, int64_t nchunks, int64_t B, int6
 cudaError_t launch_forward_scan3(const FwdArgs &f, int dtype, float *sums, float *carry,
                                  int num_sms, cudaStream_t st);
 cudaError_t launch_forward_seg(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st);
+cudaError_t launch_backward_seg(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
+                                int64_t scratch_doubles, int num_sms, cudaStream_t st);
 cudaError_t launch_backward(const BwdArgs &a, int dtype, float *gw, float *gu, cudaStream_t st);
 cudaError_t launch_step(const StepArgs &a, bool vec, int num_sms, cudaStream_t st);
 int64_t fwd_chunk_tokens();
@@ -54,7 +56,7 @@ bool sizes_ok(int64_t B, int64_t T, int64_t C) {
 }
 
 struct Layout {
-  size_t flags, desc, sums, carry, ckpt, part, total;
+  size_t flags, desc, sums, carry, ckpt, part, cnt, total;
   int64_t nct, nchains, nchunks_f, nchunks_b;
 };
 
@@ -79,12 +81,14 @@ Layout layout(int op, int64_t B, int64_t T, int64_t C) {
   off = align_up(off + sizeof(float) * 4 * 32 * (size_t)L.nchains * (size_t)L.nchunks_b, 256);
   L.carry = off;
   off = align_up(off + sizeof(float) * 3 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
-  L.ckpt = L.part = 0;
+  L.ckpt = L.part = L.cnt = 0;
   if (op == WKV_OP_BACKWARD) {
     L.ckpt = off;
     off = align_up(off + sizeof(float) * 3 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
     L.part = off;
     off = align_up(off + sizeof(float) * 2 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
+    L.cnt = off;  // per channel tile counters of the segment backward's reduction (cleared by it)
+    off = align_up(off + sizeof(unsigned) * (size_t)L.nct, 256);
   }
   L.total = off;
   return L;
@@ -266,6 +270,13 @@ int wkv_backward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, 
   FwdArgs probe{};
   probe.B = B; probe.T = T; probe.C = C; probe.k = k; probe.v = v;
   const bool tma_ok = fwd_tma_eligible(probe, dtype) && ((uintptr_t)grad_y % 16) == 0;
+  if (tma_ok && kernel == WKV_KERNEL_SEGMENT) {
+    const int64_t scratch = (int64_t)((L.sums - L.desc) / sizeof(double));
+    return launch_backward_seg(a, dtype, grad_w, grad_u, reinterpret_cast<unsigned *>(base + L.cnt), scratch,
+                               num_sms(), st) == cudaSuccess
+               ? WKV_OK
+               : WKV_ERR_CUDA;
+  }
   if (tma_ok && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_CHAIN)) {
     if (launch_backward_chain(a, dtype, st) != cudaSuccess) return WKV_ERR_CUDA;
     return launch_reduce_wu(a.part, 1, B, C, grad_w, grad_u, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;

@@ -138,7 +138,8 @@ struct WsHeader {
   unsigned done;       // blocks finished in the running launch
   unsigned abort_tag;  // epoch+1 of a launch in which a wait gave up
   int status;          // first device-side error (sticky until read)
-  unsigned pad[59];
+  unsigned bar;        // blocks arrived at the grid barrier of the running launch
+  unsigned pad[58];
 };
 static_assert(sizeof(WsHeader) == 256, "header size");
 
@@ -164,7 +165,7 @@ __device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
 
 // Per-tile descriptor: one record (the Fenwick node of the chunk) of up to
 // four float planes of 32 lanes each.
-constexpr int kDescFloats = 4 * 32;
+constexpr int kDescFloats = 5 * 32;
 
 template <typename S>
 __device__ __forceinline__ void desc_store(float *desc, int64_t tile, int which, const S &s,
@@ -238,6 +239,7 @@ __device__ __forceinline__ void finish_block(WsHeader *h, unsigned nblocks) {
     if (prev == nblocks - 1u) {
       h->ticket = 0u;
       h->done = 0u;
+      h->bar = 0u;
       __threadfence();
       atomicAdd(&h->epoch, 1u);
     }
@@ -382,6 +384,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int64_t
       if ((int64_t)(global_ns() - t0) > budget_ns) return false;
     }
   }
+}
+// Barrier over all blocks of a cooperative launch (every block resident).
+// Bounded: after `budget_ns` the block records WKV_ERR_TIMEOUT and goes on.
+// The counter is reset by the launch's last finish_block (every block has
+// left the barrier by then).
+__device__ __forceinline__ void grid_barrier(WsHeader *h, unsigned nblocks, int64_t budget_ns) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(&h->bar, 1u);
+    const uint64_t t0 = global_ns();
+    unsigned backoff = 64;
+    while (ld_acquire(&h->bar) < nblocks) {
+      if ((int64_t)(global_ns() - t0) > budget_ns) {
+        atomicCAS(&h->status, 0, -5 /* WKV_ERR_TIMEOUT */);
+        break;
+      }
+      __nanosleep(backoff);  // back off: spinning steals issue slots from working warps
+      backoff = backoff < 1024u ? backoff * 2u : 1024u;
+    }
+  }
+  __syncthreads();
 }
 // L2 eviction-priority policies for TMA loads (createpolicy).
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {

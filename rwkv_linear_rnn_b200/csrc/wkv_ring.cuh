@@ -11,19 +11,20 @@ namespace wkv {
 // Shared memory of a block of NW warps: all stages first (each warp's S
 // stages contiguous, every stage a multiple of 128 bytes, so every TMA
 // destination is 128-byte aligned as tensor copies require), then all the
-// mbarriers (8 bytes each).
-template <typename E, int S, int NARR = 2>
+// mbarriers (8 bytes each).  A stage holds ROWS rows of 32 channels of each
+// of the NARR tensors.
+template <typename E, int S, int NARR = 2, int ROWS = kS3Batch>
 struct WarpRing {
-  static constexpr int ARR_BYTES = kS3Batch * 32 * (int)sizeof(E);
+  static constexpr int ARR_BYTES = ROWS * 32 * (int)sizeof(E);
   static constexpr int STAGE_BYTES = NARR * ARR_BYTES;
   static_assert(ARR_BYTES % 128 == 0, "TMA destinations must stay 128-byte aligned");
   static constexpr int RING_BYTES = S * STAGE_BYTES;
   static constexpr int block_bytes(int nw) { return nw * (RING_BYTES + S * 8); }
 };
 
-template <typename E, int S, int NARR = 2>
+template <typename E, int S, int NARR = 2, int ROWS = kS3Batch>
 struct Ring {
-  using L = WarpRing<E, S, NARR>;
+  using L = WarpRing<E, S, NARR, ROWS>;
   unsigned char *base;
   uint32_t bar0;
   __device__ __forceinline__ Ring(unsigned char *smem, int wl, int nw) {
@@ -41,7 +42,7 @@ struct Ring {
     }
     __syncwarp();
   }
-  // Loads of batch `item` (rows y .. y+15, columns x .. x+31 of each of the
+  // Loads of batch `item` (rows y .. y+ROWS-1, columns x .. x+31 of each of the
   // NARR tensors) into stage item % S.  Returns false, issuing nothing, if a
   // destination is not 128-byte aligned (the caller's bounded wait then
   // fails and reports the error).

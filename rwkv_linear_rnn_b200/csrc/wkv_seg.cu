@@ -157,7 +157,8 @@ __global__ void __launch_bounds__(128) fwd_seg_kernel(const __grid_constant__ CU
     // inclusive prefix below instead; the chain's last segment nothing)
     const bool block_end = (sg.pos % kBlockSeg) == kBlockSeg - 1;
     const int64_t unit = sg.pos * p.nchains + sg.chain;
-    if (!block_end && sg.pos + 1 < a.nseg) publish(p.desc, p.flags, unit, 0, agg, epoch, lane);
+    const bool held = p.hold_first && sg.pos == 0;  // test hook: never publish
+    if (!block_end && sg.pos + 1 < a.nseg && !held) publish(p.desc, p.flags, unit, 0, agg, epoch, lane);
     {
       const bool act = lane < nrec;
       const unsigned *fl = p.flags + (rec0 + lane) * p.nchains + sg.chain;
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(128) fwd_seg_kernel(const __grid_constant__ CU
         }
       }
     }
-    if (block_end && sg.pos + 1 < a.nseg)
+    if (block_end && sg.pos + 1 < a.nseg && !held)
       publish(p.desc, p.flags, unit, 0, combine(carry, agg, (float)n, w2), epoch, lane);
 
     // ---- pass 2: replay from the carried-in state

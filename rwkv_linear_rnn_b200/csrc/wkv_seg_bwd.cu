@@ -1,0 +1,493 @@
+// wkv_seg_bwd.cu -- segment backward of libwkv (the default backward on
+// sm_100a when rows are 16-byte aligned): dL/dk, dL/dv, dL/dw, dL/du in one
+// launch.
+//
+// The operator is eq. wkv_t of the RWKV paper review ("[논문 리뷰] Reinvention
+// RNNs for the Transformer Era: RWKV", section "WKV 연산자"); the gradient is
+// back-propagation through the recurrence of section "RNN-유사추론" (the
+// review's BPTT remark), taken in the reverse-time scan form of the linear
+// attention paper ("Transformers are RNNs", section 3.3.1, gradient
+// computation with constant memory: cumulative sums run backwards in time).
+//
+// With D_t the denominator, G_t = g_t / D_t and H_t = g_t y_t / D_t, the
+// adjoints of the past sums obey a reverse recurrence with the constant
+// factor e^w:
+//   Ahat_t = G_t + e^w Ahat_{t+1},   Hhat_t = H_t + e^w Hhat_{t+1},
+// so a segment of tokens has an aggregate (its adjoint at the segment start
+// from a zero adjoint at its end) that joins associatively with the adjoint
+// carried in from later segments (rcombine5).  One warp owns one segment: a
+// chain (batch row b, 32 channels = lanes) and TS consecutive tokens.  Warps
+// are persistent and take segments in reverse position order (all chains'
+// last segment first):
+//   pass 1  stream k, v, g through the warp's TMA ring in forward order,
+//           recompute the forward from the checkpoint at the segment start
+//           and accumulate the segment's adjoint aggregate (in forward order:
+//           token s enters with weight e^{(s - t0) w}), keeping the forward
+//           state at every batch start (8 tokens) in shared memory;
+//   join    publish the aggregate, then fold, in a fixed order, the records
+//           of at most kBwdBlockSeg later segments of the chain (the suffix
+//           that closes the previous block of segments, then the aggregates
+//           of the later segments of this block) into the adjoint at the
+//           segment end;
+//   pass 2  stream the 8-token batches again, last first (still in L2:
+//           pass 1 loads carry an evict-last hint), recompute each batch's
+//           forward from its saved start state and sweep it in reverse,
+//           writing dL/dk, dL/dv; per-unit partial sums of dL/dw, dL/du go
+//           to the workspace.
+// After a bounded grid barrier the warps reduce the partials per channel in
+// a fixed two-level order (group sums, then the last group of a channel tile
+// adds the group sums), so the result is bit-reproducible.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "wkv_internal.cuh"
+#include "wkv_math.cuh"
+#include "wkv_ring.cuh"
+#include "wkv_split.cuh"
+
+namespace wkv {
+
+bool encode_rows(CUtensorMap *m, const void *ptr, int dtype, int64_t rows, int64_t C, int box_rows);
+
+// Adjoint aggregate with the lag-weighted terms used for dL/dw (the same
+// record as the chain backward's): Ahat = ah 2^-r, Hhat = hh 2^-r,
+// Ahat' = ahp 2^-r, Hhat' = hhp 2^-r.
+struct Adj5s {
+  float ah, hh, ahp, hhp, r;
+};
+__device__ __forceinline__ Adj5s adj5s_empty() { return Adj5s{0.f, 0.f, 0.f, 0.f, kEmptyR}; }
+
+// X (earlier, lenX tokens) then Y (later): Y's adjoint decays across X by
+// 2^{lenX w2}; its w-derivative gains lenX times Y's adjoint.
+__device__ __forceinline__ Adj5s rjoin(const Adj5s &X, const Adj5s &Y, float lenX, float w2) {
+  const float rY = fmaf(-lenX, w2, Y.r);
+  const float d = X.r - rY;
+  const float x = ex2(-fabsf(d));
+  const bool xs = d <= 0.f;
+  const float fx = xs ? 1.f : x, fy = xs ? x : 1.f;
+  Adj5s o;
+  o.ah = fmaf(X.ah, fx, Y.ah * fy);
+  o.hh = fmaf(X.hh, fx, Y.hh * fy);
+  o.ahp = fmaf(X.ahp, fx, fmaf(lenX, Y.ah, Y.ahp) * fy);
+  o.hhp = fmaf(X.hhp, fx, fmaf(lenX, Y.hh, Y.hhp) * fy);
+  o.r = fminf(X.r, rY);
+  return o;
+}
+
+struct SegBwdArgs {
+  BwdArgs p;
+  float *gw, *gu;
+  unsigned *tile_cnt;  // [nct] group counters of the final reduction
+  int64_t nseg;        // segments per chain
+  int64_t ngroups;     // row groups per channel tile in the final reduction
+};
+
+constexpr int kBwdBlockSeg = 16;  // segments per suffix block
+
+// int64 quotient through 32-bit division when both operands fit (the
+// common case; 64-bit division is a long instruction sequence).
+__device__ __forceinline__ int64_t qdiv(int64_t a, int64_t b) {
+  return (a <= 0x7fffffff && b <= 0x7fffffff) ? (int64_t)((unsigned)a / (unsigned)b) : a / b;
+}
+
+// Shared memory of a block of NW warps: the warp rings (with their
+// mbarriers), then per warp the forward state at each batch start of the
+// current segment: [NB][3][32] floats (a, b, exponent).
+template <typename E, int TS, int S, int RB>
+struct SegBwdSmem {
+  using RingL = WarpRing<E, S, 3, RB>;
+  static constexpr int NB = TS / RB;
+  static constexpr int STATE_FLOATS = NB * 3 * 32;
+  static constexpr int ring_bytes(int nw) { return (RingL::block_bytes(nw) + 15) / 16 * 16; }
+  static constexpr int bytes(int nw) { return ring_bytes(nw) + nw * STATE_FLOATS * 4; }
+};
+
+template <typename E, int TS, int S, int RB>
+__global__ void __launch_bounds__(128, 4) bwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                      const __grid_constant__ CUtensorMap vmap,
+                                                      const __grid_constant__ CUtensorMap gmap,
+                                                      SegBwdArgs a) {
+  using Sm = SegBwdSmem<E, TS, S, RB>;
+  constexpr int NB = Sm::NB;   // ring items (batches of RB tokens) per pass
+  constexpr int IPU = 2 * NB;  // ring items per segment
+  static_assert(TS % kCkpt == 0, "segments start on checkpoints");
+  const BwdArgs &p = a.p;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = (int)(blockDim.x >> 5);
+  Ring<E, S, 3, RB> ring(smem, wl, nw);
+  ring.init(lane);
+  float *sts = reinterpret_cast<float *>(smem + Sm::ring_bytes(nw)) + wl * Sm::STATE_FLOATS;
+  const CUtensorMap *const maps[3] = {&kmap, &vmap, &gmap};
+  // The reduction counters are cleared here; the grid barrier orders these
+  // stores before every increment (a workspace reused for another shape may
+  // hold anything at their offset).
+  if (blockIdx.x == 0)
+    for (int64_t i = threadIdx.x; i < p.nct; i += blockDim.x) a.tile_cnt[i] = 0u;
+  const int64_t G = (int64_t)gridDim.x * nw;
+  const int64_t g = (int64_t)blockIdx.x * nw + wl;
+  const int64_t nseg = a.nseg;
+  const int64_t total = nseg * p.nchains;
+  const int64_t nu = total > g ? qdiv(total - g + G - 1, G) : 0;
+  const int64_t nitems = nu * IPU;
+  const int64_t T = p.T, C = p.C, BC = p.B * p.C;
+  const int64_t budget = p.spin_limit * 1000;
+  unsigned epoch = 0;
+  if (lane == 0) epoch = ld_relaxed(&p.hdr->epoch);
+  epoch = __shfl_sync(0xffffffffu, epoch, 0);
+  const unsigned want = (epoch_tag(epoch) << 2) | kAgg;
+
+  // Lane 0 issues ring items ahead of the consumer.  Item r of a unit: pass 1
+  // batch r (r < NB), pass 2 batch IPU-1-r (r >= NB, last batch first).
+  int64_t pf_i = -1, pf_row0 = 0;
+  int pf_x = 0;
+  uint64_t pol_keep = 0, pol_drop = 0;
+  if (lane == 0) {
+    pol_keep = l2_policy_evict_last();
+    pol_drop = l2_policy_evict_first();
+  }
+  auto issue = [&](int64_t k) {
+    const int64_t i = k / IPU;
+    const int r = (int)(k % IPU);
+    if (i != pf_i) {
+      pf_i = i;
+      const int64_t unit = g + i * G;
+      const int64_t rpos = qdiv(unit, p.nchains), chain = unit - rpos * p.nchains;
+      const int64_t b = qdiv(chain, p.nct);
+      pf_x = (int)((chain - b * p.nct) * 32);
+      pf_row0 = b * T + (nseg - 1 - rpos) * TS;
+    }
+    const int bt = r < NB ? r : IPU - 1 - r;
+    const bool ok = ring.issue_hint(maps, k, pf_x, (int)(pf_row0 + bt * RB), r < NB ? pol_keep : pol_drop);
+    if (!ok) atomicCAS(&p.hdr->status, 0, -4 /* misaligned stage: nothing issued */);
+  };
+  if (lane == 0)
+    for (int64_t k = 0; k < min((int64_t)S - 1, nitems); ++k) issue(k);
+  bool failed = false;
+  auto take = [&](int64_t k, float(&K)[RB], float(&V)[RB], float(&Gy)[RB]) {
+    const int s = (int)(k % S);
+    if (!failed && !mbar_wait(ring.bar(s), (uint32_t)(k / S) & 1u, budget, nullptr)) {
+      failed = true;
+      if (lane == 0) atomicCAS(&p.hdr->status, 0, -5 /* WKV_ERR_TIMEOUT */);
+    }
+    const E *kr = ring.stage(s, 0) + lane;
+    const E *vr = ring.stage(s, 1) + lane;
+    const E *gr = ring.stage(s, 2) + lane;
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      K[j] = to_f32(kr[j * 32]) * kLog2e;
+      V[j] = to_f32(vr[j * 32]);
+      Gy[j] = to_f32(gr[j * 32]);
+    }
+    __syncwarp();  // the stage is read; it may be refilled
+    if (lane == 0 && k + S - 1 < nitems) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(k + S - 1);
+    }
+  };
+
+  for (int64_t i = 0; i < nu; ++i) {
+    const int64_t unit = g + i * G;
+    const int64_t rpos = qdiv(unit, p.nchains), chain = unit - rpos * p.nchains;
+    const int64_t b = qdiv(chain, p.nct);
+    const int64_t c = (chain - b * p.nct) * 32 + lane;
+    const bool cok = c < C;
+    const int64_t pos = nseg - 1 - rpos;
+    const int64_t t0 = pos * TS;
+    const int n = (int)min((int64_t)TS, T - t0);
+    const float w2 = cok ? __ldg(p.w + c) * kLog2e : 0.f;
+    const float u2 = cok ? __ldg(p.u + c) * kLog2e : 0.f;
+    const int64_t base_item = i * IPU;
+    const int64_t bc = b * C + c;
+
+    // ---- pass 1: forward recompute and the segment's adjoint aggregate
+    // The forward state is (fa, fb) 2^E with E = fP + fn w2 (anchored).
+    float fa = 0.f, fb = 0.f, fP = kEmptyP, fn = 0.f;
+    if (cok) {
+      const float *ck = p.ckpt + (t0 / kCkpt) * 3 * BC + bc;
+      fa = ck[0];
+      fb = ck[BC];
+      fP = ck[2 * BC];
+    }
+    float ah = 0.f, hh = 0.f, ahp = 0.f, hhp = 0.f, Em = -kEmptyR;
+#pragma unroll 1
+    for (int bt = 0; bt < NB; ++bt) {
+      sts[bt * 96 + lane] = fa;
+      sts[bt * 96 + 32 + lane] = fb;
+      sts[bt * 96 + 64 + lane] = fmaf(fn, w2, fP);
+      float K[RB], V[RB], Gy[RB];
+      take(base_item + bt, K, V, Gy);
+      const int nb = max(0, min(RB, n - bt * RB));
+      const float lag0 = (float)(bt * RB);
+#pragma unroll
+      for (int j = 0; j < RB; ++j) {
+        if (j < nb) {
+          const float P = fmaf(fn, w2, fP);
+          const float UK = u2 + K[j];
+          const float d = P - UK;
+          const float x = ex2(-fabsf(d));
+          const bool pw = d >= 0.f;
+          const float e1 = pw ? 1.f : x, e2 = pw ? x : 1.f;
+          const float rden = rcp(fmaf(fb, e1, e2));
+          const float y = fmaf(fa, e1, V[j] * e2) * rden;
+          const float gam = Gy[j] * rden;
+          const float eta = gam * y;
+          // token s = t0 + lag enters the aggregate with 2^{lag w2 - q_s}
+          const float lag = lag0 + (float)j;
+          const float es = fmaf(lag, w2, -fmaxf(P, UK));
+          const float da = es - Em;
+          const float xa = ex2(-fabsf(da));
+          const bool up = da > 0.f;
+          const float fo = up ? xa : 1.f, fg = up ? 1.f : xa;
+          const float gg = gam * fg, ee = eta * fg;
+          ah = fmaf(ah, fo, gg);
+          hh = fmaf(hh, fo, ee);
+          ahp = fmaf(ahp, fo, lag * gg);
+          hhp = fmaf(hhp, fo, lag * ee);
+          Em = up ? es : Em;
+          // forward state update
+          const float n1 = fn + 1.f;
+          const float Pc = fmaf(n1, w2, fP);
+          const float d2 = K[j] - Pc;
+          const float x2 = ex2(-fabsf(d2));
+          const bool kw = d2 > 0.f;
+          const float so = kw ? x2 : 1.f, snw = kw ? 1.f : x2;
+          fa = fmaf(fa, so, V[j] * snw);
+          fb = fmaf(fb, so, snw);
+          fP = kw ? K[j] : fP;
+          fn = kw ? 0.f : n1;
+        }
+      }
+    }
+    const Adj5s agg{ah, hh, ahp, hhp, -Em};
+
+    // ---- join: adjoint at the segment end from the later segments' records
+    const int64_t q = rpos - rpos % kBwdBlockSeg;  // first (latest) segment of this block
+    const int nrec = (int)(rpos - q) + (q > 0 ? 1 : 0);
+    const int64_t rec0 = q > 0 ? q - 1 : q;
+    const bool block_end = (rpos % kBwdBlockSeg) == kBwdBlockSeg - 1;
+    const bool held = p.hold_first && rpos == 0;  // test hook: never publish
+    if (!block_end && rpos + 1 < nseg && !held) publish(p.desc, p.flags, unit, 0, agg, epoch, lane);
+    {
+      const bool act = lane < nrec;
+      const unsigned *fl = p.flags + (rec0 + lane) * p.nchains + chain;
+      bool ready = !act;
+      const uint64_t t_start = global_ns();
+      unsigned backoff = 32;
+      while (true) {
+        if (!ready) ready = ld_acquire(fl) == want;
+        if (__all_sync(0xffffffffu, ready)) break;
+        if ((int64_t)(global_ns() - t_start) > budget) {
+          if (lane == 0) atomicCAS(&p.hdr->status, 0, -5 /* WKV_ERR_TIMEOUT */);
+          break;
+        }
+        __nanosleep(backoff);
+        backoff = backoff < 512u ? backoff * 2u : 512u;
+      }
+      __syncwarp();
+    }
+    const int nlast = (int)(T - (nseg - 1) * TS);  // tokens of the chain's last segment
+    Adj5s acc = adj5s_empty();
+#pragma unroll 1
+    for (int j0 = 0; j0 < nrec; j0 += 8) {
+      Adj5s rec[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j0 + j < nrec) rec[j] = desc_load<Adj5s>(p.desc, (rec0 + j0 + j) * p.nchains + chain, 0, lane);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j0 + j < nrec) {
+          const int64_t rp = rec0 + j0 + j;
+          if (q > 0 && rp == q - 1)
+            acc = rec[j];  // adjoint at the start of the previous block's last segment
+          else
+            acc = rjoin(rec[j], acc, rp == 0 ? (float)nlast : (float)TS, w2);
+        }
+      }
+    }
+    if (block_end && rpos + 1 < nseg && !held)
+      publish(p.desc, p.flags, unit, 0, rjoin(agg, acc, (float)n, w2), epoch, lane);
+
+    // ---- pass 2: batches last to first, recompute then reverse sweep
+    float gw_acc = 0.f, gu_acc = 0.f;
+    float rah = acc.ah, rhh = acc.hh, rahp = acc.ahp, rhhp = acc.hhp, Ranc = acc.r, m = 0.f;
+#pragma unroll 1
+    for (int bi = 0; bi < NB; ++bi) {
+      const int bt = NB - 1 - bi;
+      float K[RB], V[RB], Gy[RB];
+      take(base_item + NB + bi, K, V, Gy);
+      const int nb = max(0, min(RB, n - bt * RB));
+      float qv[RB], gam[RB], eta[RB], e2v[RB];
+      {
+        float xa = sts[bt * 96 + lane], xb = sts[bt * 96 + 32 + lane], xP = sts[bt * 96 + 64 + lane];
+        float xn = 0.f;
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+          qv[j] = 0.f;
+          gam[j] = eta[j] = e2v[j] = 0.f;
+          if (j < nb) {
+            const float P = fmaf(xn, w2, xP);
+            const float UK = u2 + K[j];
+            const float d = P - UK;
+            const float x = ex2(-fabsf(d));
+            const bool pw = d >= 0.f;
+            const float e1 = pw ? 1.f : x, e2 = pw ? x : 1.f;
+            const float rden = rcp(fmaf(xb, e1, e2));
+            const float y = fmaf(xa, e1, V[j] * e2) * rden;
+            qv[j] = fmaxf(P, UK);
+            gam[j] = Gy[j] * rden;
+            eta[j] = gam[j] * y;
+            e2v[j] = e2;
+            const float n1 = xn + 1.f;
+            const float Pc = fmaf(n1, w2, xP);
+            const float d2 = K[j] - Pc;
+            const float x2 = ex2(-fabsf(d2));
+            const bool kw = d2 > 0.f;
+            const float so = kw ? x2 : 1.f, snw = kw ? 1.f : x2;
+            xa = fmaf(xa, so, V[j] * snw);
+            xb = fmaf(xb, so, snw);
+            xP = kw ? K[j] : xP;
+            xn = kw ? 0.f : n1;
+          }
+        }
+      }
+      E *gkp = static_cast<E *>(p.gk) + (b * T + t0 + bt * RB) * C + c;
+      E *gvp = static_cast<E *>(p.gv) + (b * T + t0 + bt * RB) * C + c;
+#pragma unroll
+      for (int j = RB - 1; j >= 0; --j) {
+        if (j < nb) {
+          const float rn = fmaf(-m, w2, Ranc);  // scale of the adjoint after token t
+          const float tn = ex2(K[j] - rn);      // e^{k_t} 2^{-r_{t+1}} (<= 1)
+          const float gv = fmaf(gam[j], e2v[j], tn * rah);
+          const float gk = fmaf(V[j], gv, -fmaf(eta[j], e2v[j], tn * rhh));
+          gw_acc = fmaf(tn, fmaf(V[j], rahp, -rhhp), gw_acc);
+          gu_acc = fmaf(e2v[j], fmaf(gam[j], V[j], -eta[j]), gu_acc);
+          if (cok) {
+            IO<E>::st(gkp + (int64_t)j * C, gk);
+            IO<E>::st(gvp + (int64_t)j * C, gv);
+          }
+          const float m1 = m + 1.f;
+          const float Rc = fmaf(-m1, w2, Ranc);
+          const float d = qv[j] - Rc;
+          const float x = ex2(-fabsf(d));
+          const bool reset = d < 0.f;
+          const float fg = reset ? 1.f : x, fo = reset ? x : 1.f;
+          rahp = fo * (rah + rahp);
+          rhhp = fo * (rhh + rhhp);
+          rah = fmaf(rah, fo, gam[j] * fg);
+          rhh = fmaf(rhh, fo, eta[j] * fg);
+          Ranc = reset ? qv[j] : Ranc;
+          m = reset ? 0.f : m1;
+        }
+      }
+    }
+    if (cok) {
+      if (t0 == 0) {
+        // share of the initial state A_0, B_0 (zero for the empty state)
+        const float *ck = p.ckpt + bc;
+        const float r0 = fmaf(-m, w2, Ranc);
+        gw_acc = fmaf(ex2(ck[2 * BC] - r0), fmaf(ck[0], rahp, -ck[BC] * rhhp), gw_acc);
+      }
+      p.part[(pos * 2 + 0) * BC + bc] = gw_acc;
+      p.part[(pos * 2 + 1) * BC + bc] = gu_acc;
+    }
+  }
+  if (failed && lane == 0)  // every issued load lands before the block exits
+    for (int64_t k = max((int64_t)0, nitems - S); k < nitems; ++k)
+      mbar_wait(ring.bar((int)(k % S)), (uint32_t)(k / S) & 1u, budget, nullptr);
+
+  // ---- dL/dw, dL/du: fixed-order two-level reduction of the partials
+  grid_barrier(p.hdr, gridDim.x, budget);
+  {
+    const int64_t R = nseg * p.B;  // partial rows (segment position, b) per channel
+    const int64_t ng = a.ngroups;
+    double *scratch = reinterpret_cast<double *>(p.desc);  // records are dead after the barrier
+    for (int64_t task = g; task < p.nct * ng; task += G) {
+      const int64_t ct = task / ng, grp = task - ct * ng;
+      const int64_t c = ct * 32 + lane;
+      const int64_t r0 = grp * R / ng, r1 = (grp + 1) * R / ng;
+      double sw = 0.0, su = 0.0;
+      if (c < C) {
+        for (int64_t r = r0; r < r1; ++r) {
+          const int64_t ps = r / p.B, bb = r - ps * p.B;
+          sw += (double)__ldcg(p.part + (ps * 2 + 0) * BC + bb * C + c);
+          su += (double)__ldcg(p.part + (ps * 2 + 1) * BC + bb * C + c);
+        }
+      }
+      double *dst = scratch + (ct * ng + grp) * 64;
+      __stcg(dst + lane, sw);
+      __stcg(dst + 32 + lane, su);
+      __syncwarp();
+      unsigned last = 0;
+      if (lane == 0) {
+        __threadfence();
+        last = atomicAdd(a.tile_cnt + ct, 1u) == (unsigned)(ng - 1);
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        __threadfence();
+        double tw = 0.0, tu = 0.0;
+        for (int64_t k = 0; k < ng; ++k) {
+          tw += __ldcg(scratch + (ct * ng + k) * 64 + lane);
+          tu += __ldcg(scratch + (ct * ng + k) * 64 + 32 + lane);
+        }
+        if (c < C) {
+          a.gw[c] = (float)tw;
+          a.gu[c] = (float)tu;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  finish_block(p.hdr, gridDim.x);
+}
+
+template <typename E, int TS, int S, int RB>
+static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
+                                    int64_t scratch_doubles, int num_sms, cudaStream_t st) {
+  CUtensorMap km, vm, gm;
+  if (!encode_rows(&km, p.k, dtype, p.B * p.T, p.C, RB) || !encode_rows(&vm, p.v, dtype, p.B * p.T, p.C, RB) ||
+      !encode_rows(&gm, p.gy, dtype, p.B * p.T, p.C, RB))
+    return cudaErrorInvalidValue;
+  constexpr int kWarps = 4;
+  constexpr int smem = SegBwdSmem<E, TS, S, RB>::bytes(kWarps);
+  auto kern = bwd_seg_kernel<E, TS, S, RB>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int occ = 0;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kWarps * 32, smem)) != cudaSuccess)
+    return e;
+  if (occ < 1) return cudaErrorInvalidConfiguration;
+  SegBwdArgs a{};
+  a.p = p;
+  a.gw = gw;
+  a.gu = gu;
+  a.tile_cnt = tile_cnt;
+  a.nseg = (p.T + TS - 1) / TS;
+  const int64_t units = a.nseg * p.nchains;
+  // one resident wave (cooperative launch: every warp a segment may wait on,
+  // and every block of the grid barrier, is running)
+  const int64_t grid = std::min<int64_t>((units + kWarps - 1) / kWarps, (int64_t)occ * num_sms);
+  const int64_t G = grid * kWarps;
+  // row groups per channel tile: enough to spread the partial rows over the
+  // warps, at least 8 rows each, and the group sums must fit the scratch
+  const int64_t R = a.nseg * p.B;
+  int64_t ng = std::max<int64_t>(1, std::min<int64_t>(G / p.nct, R / 8));
+  while (ng > 1 && p.nct * ng * 64 > scratch_doubles) --ng;
+  a.ngroups = ng;
+  void *args[] = {&km, &vm, &gm, &a};
+  return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3(kWarps * 32), args,
+                                     (size_t)smem, st);
+}
+
+constexpr int kSegBwdTS = 64;
+
+cudaError_t launch_backward_seg(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
+                                int64_t scratch_doubles, int num_sms, cudaStream_t st) {
+  return dtype == 0
+             ? launch_bwd_seg_t<float, kSegBwdTS, 3, 8>(p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, st)
+             : launch_bwd_seg_t<uint16_t, kSegBwdTS, 4, 8>(p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, st);
+}
+
+}  // namespace wkv

@@ -56,11 +56,14 @@ extern "C" int wkv_backward_static(int64_t B, int64_t T, int64_t C, int dtype, c
   if (need > kStaticScratch) return WKV_ERR_WORKSPACE;
   void *ws = scratch_for_current_device();
   if (!ws) return WKV_ERR_CUDA;
-  // The two per-launch counters of the scratch header (block ticket and
-  // finished-block count, bytes 4..11) must read zero when a launch starts.
-  // Launches leave them at zero; clearing them here makes that explicit.
-  // The launch epoch (bytes 0..3) must persist across calls and is kept.
-  if (cudaMemsetAsync(static_cast<unsigned char *>(ws) + 4, 0, 8, (cudaStream_t)stream) != cudaSuccess)
+  // The per-launch counters of the scratch header (block ticket and
+  // finished-block count, bytes 4..11; grid-barrier arrivals, bytes 20..23)
+  // must read zero when a launch starts.  Launches leave them at zero;
+  // clearing them here makes that explicit.  The launch epoch (bytes 0..3)
+  // must persist across calls and is kept, and so is the status word.
+  unsigned char *h = static_cast<unsigned char *>(ws);
+  if (cudaMemsetAsync(h + 4, 0, 8, (cudaStream_t)stream) != cudaSuccess ||
+      cudaMemsetAsync(h + 20, 0, 4, (cudaStream_t)stream) != cudaSuccess)
     return WKV_ERR_CUDA;
   return wkv_backward(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u, grad_k,
                       grad_v, ws, kStaticScratch, stream);

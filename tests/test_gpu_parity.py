@@ -21,7 +21,8 @@ pytestmark = pytest.mark.gpu
 KERNELS = {"seq": W.WKV_KERNEL_SEQUENTIAL, "chunked": W.WKV_KERNEL_CHUNKED,
            "chunked_regs": W.WKV_KERNEL_CHUNKED_REGS, "chain": W.WKV_KERNEL_CHAIN,
            "split": W.WKV_KERNEL_SPLIT, "segment": W.WKV_KERNEL_SEGMENT}
-BWD_KERNELS = {"chain": W.WKV_KERNEL_CHAIN, "chunked": W.WKV_KERNEL_CHUNKED}
+BWD_KERNELS = {"chain": W.WKV_KERNEL_CHAIN, "chunked": W.WKV_KERNEL_CHUNKED,
+               "segment": W.WKV_KERNEL_SEGMENT}
 
 
 def small_case(B, T, C, seed, dtype="f32", td=(-3.0, 1.0), kstd=1.0, state=False):
@@ -300,27 +301,81 @@ def test_autograd_function_matches_oracle():
 
 # -------------------------------------------------- failure and edge paths ---
 
-def test_timeout_is_reported_and_context_survives():
-    """Blocks of the first chunk are told never to publish: the blocks that
-    wait on them give up after a short bounded wait, the status word reads
-    WKV_ERR_TIMEOUT, and the next normal call works."""
+@pytest.mark.parametrize("kernel", ["chunked", "segment"])
+def test_timeout_is_reported_and_context_survives(kernel):
+    """The first chunk (segment) is told never to publish its record: the
+    warps that wait on it give up after a short bounded wait, the status word
+    reads WKV_ERR_TIMEOUT, and the next normal call works."""
     B, T, C = 1, 1024, 64
+    kid = KERNELS[kernel]
     w, u, k, v, _, _ = small_case(B, T, C, seed=16)
     W_, U_, K_, V_ = dev(w), dev(u), dev(k), dev(v)
     ws = W.Workspace()
     buf, nb = ws.get(W.WKV_OP_FORWARD, B, T, C, W.WKV_F32)
     y = torch.empty_like(K_)
-    opt = abi.Options(kernel=W.WKV_KERNEL_CHUNKED, test_hold_first_chunk=1, spin_limit=2000)
+    opt = abi.Options(kernel=kid, test_hold_first_chunk=1, spin_limit=2000)
     stream = torch.cuda.current_stream().cuda_stream
     rc = abi.wkv_forward_ex(B, T, C, 0, W_.data_ptr(), U_.data_ptr(), K_.data_ptr(), V_.data_ptr(),
                             0, y.data_ptr(), 0, 0, buf.data_ptr(), nb, stream, opt)
     assert rc == 0
     assert ws.status() == abi.WKV_ERR_TIMEOUT
     assert ws.status() == 0  # cleared by the read
-    y2, _, _ = W.forward(W_, U_, K_, V_, workspace=ws, kernel=W.WKV_KERNEL_CHUNKED)
+    y2, _, _ = W.forward(W_, U_, K_, V_, workspace=ws, kernel=kid)
     assert ws.status() == 0
     y_ref, _ = oracle.fwd_recur(w, u, k, v)
     assert fwd_err(host(y2), y_ref) <= F32_FWD_TOL
+
+
+def test_backward_timeout_is_reported_and_context_survives():
+    """The segment backward with the last segment's record held back: the
+    waits and the grid barrier stay bounded, the status reads WKV_ERR_TIMEOUT,
+    and the next call on the same workspace is correct."""
+    B, T, C = 1, 1024, 64
+    w, u, k, v, g, _ = small_case(B, T, C, seed=18)
+    W_, U_, K_, V_, G_ = dev(w), dev(u), dev(k), dev(v), dev(g)
+    ws = W.Workspace()
+    _, _, ck = W.forward(W_, U_, K_, V_, want_ckpt=True, workspace=ws)
+    buf, nb = ws.get(W.WKV_OP_BACKWARD, B, T, C, W.WKV_F32)
+    gw = torch.empty(C, device="cuda"); gu = torch.empty(C, device="cuda")
+    gk = torch.empty_like(K_); gv = torch.empty_like(V_)
+    opt = abi.Options(kernel=W.WKV_KERNEL_SEGMENT, test_hold_first_chunk=1, spin_limit=2000)
+    stream = torch.cuda.current_stream().cuda_stream
+    P = lambda t: t.data_ptr()
+    rc = abi.wkv_backward_ex(B, T, C, 0, P(W_), P(U_), P(K_), P(V_), P(G_), 0, P(ck), P(gw), P(gu),
+                             P(gk), P(gv), P(buf), nb, stream, opt)
+    assert rc == 0
+    assert ws.status() == abi.WKV_ERR_TIMEOUT
+    got = W.backward(W_, U_, K_, V_, G_, ckpt=ck, workspace=ws, kernel=W.WKV_KERNEL_SEGMENT)
+    assert ws.status() == 0
+    assert_grads(got, grads_ref(w, u, k, v, g), F32_GRAD_TOL)
+
+
+def test_segment_backward_reuses_a_workspace_across_shapes():
+    """One workspace, shapes in decreasing then increasing size: whatever an
+    earlier call left in the workspace does not leak into a later result."""
+    ws = W.Workspace()
+    for (B, T, C) in [(3, 1000, 96), (2, 129, 64), (1, 300, 32), (3, 1000, 96)]:
+        w, u, k, v, g, _ = small_case(B, T, C, seed=B + T + C)
+        W_, U_, K_, V_ = dev(w), dev(u), dev(k), dev(v)
+        _, _, ck = W.forward(W_, U_, K_, V_, want_ckpt=True, workspace=ws)
+        got = W.backward(W_, U_, K_, V_, dev(g), ckpt=ck, workspace=ws, kernel=W.WKV_KERNEL_SEGMENT)
+        assert ws.status() == 0
+        assert_grads(got, grads_ref(w, u, k, v, g), F32_GRAD_TOL)
+
+
+def test_segment_outputs_stay_inside_their_buffers():
+    B, T, C = 2, 300, 96
+    w, u, k, v, g, _ = small_case(B, T, C, seed=27)
+    n = B * T * C
+    guard = 4096
+    bufs = [torch.full((n + 2 * guard,), 12345.0, device="cuda") for _ in range(3)]
+    y, gk, gv = (b_[guard:guard + n].view(B, T, C) for b_ in bufs)
+    W_, U_, K_, V_ = dev(w), dev(u), dev(k), dev(v)
+    _, _, ck = W.forward(W_, U_, K_, V_, y=y, want_ckpt=True, kernel=W.WKV_KERNEL_SEGMENT)
+    W.backward(W_, U_, K_, V_, dev(g), ckpt=ck, grad_k=gk, grad_v=gv, kernel=W.WKV_KERNEL_SEGMENT)
+    torch.cuda.synchronize()
+    for b_ in bufs:
+        assert torch.all(b_[:guard] == 12345.0) and torch.all(b_[guard + n:] == 12345.0)
 
 
 def test_outputs_do_not_write_outside_their_buffers():
