@@ -41,10 +41,20 @@ ALG_BYTES = {("fwd", "f32"): 12, ("fwd", "bf16"): 6, ("bwd", "f32"): 20, ("bwd",
              ("step", "f32"): 36}
 
 
-# kernels each call launches on TMA-eligible rows (the bench workloads):
-# wkv_forward -> fwd_seg_kernel; wkv_backward -> bwd_chain_kernel + reduce_wu_kernel
-BWD_KERNELS = "wkv_backward call: bwd_chain_kernel + reduce_wu_kernel, timed together"
-LAUNCHES_PER_STEP = 3
+# Kernels each call launches on 16-byte aligned rows (all bench workloads),
+# per kernel selector: (kernel names, launches per call).
+FWD_PLAN = {"auto": ("fwd_seg_kernel", 1), "segment": ("fwd_seg_kernel", 1),
+            "chain": ("fwd_chain_kernel", 1)}
+BWD_PLAN = {"auto": ("bwd_chain_kernel + reduce_wu_kernel", 2),
+            "chain": ("bwd_chain_kernel + reduce_wu_kernel", 2),
+            "segment": ("bwd_seg_kernel", 1)}
+KERNEL_IDS = {"auto": 0, "chain": 4, "segment": 6}
+
+# DRAM bytes (read + write) per launch of the backward's main kernel from one
+# ncu capture of this bench's workload (cold L2; gk/gv lines still dirty in
+# L2 at kernel end are not counted).  Keyed by (workload, kernel); a kernel
+# changed since its capture has no entry (traffic reported as null).
+TRAFFIC = {("rwkv169m", "bwd_chain_kernel"): 76_723_968 + 10_438_144}
 
 
 def peaks():
@@ -114,6 +124,23 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The maximum of a per-rank time over all ranks (every rank calls this
+    in the same order); identity without a process group."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(units_per_rank: int, n_ranks: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the units every rank processed in one step over
+    the slowest rank's step time (weak scaling, replicas)."""
+    return n_ranks * units_per_rank / (ms_per_step * 1e-3)
 
 
 def cpu_baseline(wl_name: str, min_seconds: float = 10.0):
@@ -211,13 +238,16 @@ def run_libwkv(args):
     sp = stream.cuda_stream
     P = lambda t: t.data_ptr()
 
+    fopt = abi.Options(kernel=KERNEL_IDS[args.fwd_kernel])
+    bopt = abi.Options(kernel=KERNEL_IDS[args.bwd_kernel])
+
     def fwd():
-        abi.check(abi.wkv_forward(B, T, C, dt, P(w), P(u), P(k), P(v), 0, P(y), 0, P(ckpt),
-                                  P(wsb), nws, sp))
+        abi.check(abi.wkv_forward_ex(B, T, C, dt, P(w), P(u), P(k), P(v), 0, P(y), 0, P(ckpt),
+                                     P(wsb), nws, sp, fopt))
 
     def bwd():
-        abi.check(abi.wkv_backward(B, T, C, dt, P(w), P(u), P(k), P(v), P(gy), 0, P(ckpt),
-                                   P(gw), P(gu), P(gk), P(gv), P(wsb), nws, sp))
+        abi.check(abi.wkv_backward_ex(B, T, C, dt, P(w), P(u), P(k), P(v), P(gy), 0, P(ckpt),
+                                      P(gw), P(gu), P(gk), P(gv), P(wsb), nws, sp, bopt))
 
     for _ in range(args.warmup):
         flush_l2()
@@ -248,11 +278,7 @@ def run_libwkv(args):
         dist.barrier()
     t_fwd = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     t_bwd = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    total_ms = sum(t_fwd) + sum(t_bwd)
-    if dist:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(t_fwd) + sum(t_bwd), dist, dev)
     status = abi.wkv_get_status(P(wsb), sp)
 
     # e2e: host buffers (pinned), copies in the timed region, through the same ABI
@@ -279,12 +305,8 @@ def run_libwkv(args):
             torch.cuda.synchronize()
             if i > 0:
                 ee.append(e0.elapsed_time(e1))
-        e2e_ms = statistics.median(ee)
-        if dist:
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": ws_n * B * T * C / (e2e_ms * 1e-3), "unit": "channel-tokens/s",
+        e2e_ms = max_over_ranks(statistics.median(ee), dist, dev)
+        e2e = {"value": aggregate_rate(B * T * C, ws_n, e2e_ms), "unit": "channel-tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     if rank == 0:
@@ -297,23 +319,31 @@ def run_libwkv(args):
         bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9
         fwd_gbs = fb / (fwd_ms * 1e-3) / 1e9
         step_ms = total_ms / K
+        bwd_names, bwd_launches = BWD_PLAN[args.bwd_kernel]
+        fwd_names, fwd_launches = FWD_PLAN[args.fwd_kernel]
+        main_bwd = bwd_names.split(" + ")[0]
+        traffic = TRAFFIC.get((args.workload, main_bwd))
         line = {
             "metric": "WKV fwd+bwd channel-tokens/s (HBM GB/s and % of roofline alongside)",
-            "value": ws_n * units / (step_ms * 1e-3), "unit": "channel-tokens/s",
+            "value": aggregate_rate(units, ws_n, step_ms), "unit": "channel-tokens/s",
             "n_gpus": ws_n, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": inp["dtype"], "data": "synthetic (seeded; the RWKV-4 layer shapes and value ranges)",
             "config": {"workload": args.workload, "B": B, "T": T, "C": C,
                        "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
                        "l2": "flushed before every timed step (2x L2 write + 2x L2 read, outside events)"},
-            "roofline": {"bound": "hbm", "kernel": BWD_KERNELS,
+            "roofline": {"bound": "hbm",
+                         "kernel": f"wkv_backward call ({bwd_names}), timed as one call",
                          "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": bwd_gbs / hbm, "traffic": None, "peak_kind": peak_kind},
-            "fwd": {"ms": fwd_ms, "gbs": fwd_gbs, "frac": fwd_gbs / hbm,
+                         "frac": bwd_gbs / hbm, "traffic": traffic,
+                         "traffic_kernel": main_bwd if traffic else None,
+                         "algorithmic_bytes": bb, "peak_kind": peak_kind},
+            "fwd": {"kernels": fwd_names, "ms": fwd_ms, "gbs": fwd_gbs, "frac": fwd_gbs / hbm,
                     "channel_tokens_per_s": units / (fwd_ms * 1e-3)},
-            "bwd": {"ms": bwd_ms, "gbs": bwd_gbs, "frac": bwd_gbs / hbm},
+            "bwd": {"kernels": bwd_names, "ms": bwd_ms, "gbs": bwd_gbs, "frac": bwd_gbs / hbm},
             "fwd_bwd_gbs": (fb + bb) / (step_ms * 1e-3) / 1e9,
-            "clocks": clocks, "gpu_launches": LAUNCHES_PER_STEP * K, "device_status": status,
+            "clocks": clocks, "gpu_launches": (fwd_launches + bwd_launches) * K,
+            "device_status": status,
         }
         if e2e:
             line["e2e"] = e2e
@@ -335,6 +365,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--fwd-kernel", default="auto", choices=sorted(FWD_PLAN))
+    ap.add_argument("--bwd-kernel", default="auto", choices=sorted(BWD_PLAN))
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
     if args.impl == "reference":

@@ -6,8 +6,9 @@
 // RNNs for the Transformer Era: RWKV", section "WKV 연산자"); the gradient is
 // back-propagation through the recurrence of section "RNN-유사추론" (the
 // review's BPTT remark), taken in the reverse-time scan form of the linear
-// attention paper ("Transformers are RNNs", section 3.3.1, gradient
-// computation with constant memory: cumulative sums run backwards in time).
+// attention post ("Transformers are RNNs: 선형 어텐션으로 만드는 빠른 자기회귀
+// 트랜스포머", section "상수 메모리 기울기 계산": the cumulative sums for the
+// key/value gradients run backwards in time).
 //
 // With D_t the denominator, G_t = g_t / D_t and H_t = g_t y_t / D_t, the
 // adjoints of the past sums obey a reverse recurrence with the constant
