@@ -45,7 +45,7 @@ ALG_BYTES = {("fwd", "f32"): 12, ("fwd", "bf16"): 6, ("bwd", "f32"): 20, ("bwd",
 # per kernel selector: (kernel names, launches per call).
 FWD_PLAN = {"auto": ("fwd_seg_kernel", 1), "segment": ("fwd_seg_kernel", 1),
             "chain": ("fwd_chain_kernel", 1)}
-BWD_PLAN = {"auto": ("bwd_chain_kernel + reduce_wu_kernel", 2),
+BWD_PLAN = {"auto": ("bwd_seg_kernel", 1),
             "chain": ("bwd_chain_kernel + reduce_wu_kernel", 2),
             "segment": ("bwd_seg_kernel", 1)}
 KERNEL_IDS = {"auto": 0, "chain": 4, "segment": 6}

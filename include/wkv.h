@@ -98,20 +98,19 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
  *               variant of the chunked kernel (no TMA); CHAIN runs one block
  *               per (batch row, 32-channel) chain over all of T, tiles fed
  *               by TMA, the carry kept on chip (needs 16-byte aligned rows;
- *               the backward default when they are).  SPLIT runs three launches: chunk
+ *               needs 16-byte aligned rows).  SPLIT runs three launches: chunk
  *               summaries, a per-chain prefix over them, and a replay of
  *               every chunk from its start state.  SEGMENT (the forward
  *               default when rows are 16-byte aligned) gives each warp a
  *               128/256-token segment of one chain: summary, a fixed-order
- *               join with at most 32 earlier records, and the replay from L2.
- *               In the backward, CHAIN/AUTO select the chain kernel and
- *               SEGMENT a one-launch segment kernel (64-token segments in
- *               reverse order: recompute and adjoint aggregate, a
- *               fixed-order join with at most 16 later records, then the
- *               reverse sweep from L2; dL/dw and dL/du reduced in the same
- *               launch after a grid barrier); both need 16-byte aligned
- *               rows, otherwise and for any other value the chunked kernel
- *               runs.
+ *               join with at most 16 earlier records, and the replay from L2.
+ *               In the backward, AUTO/SEGMENT select a one-launch segment
+ *               kernel (64-token segments in reverse order: recompute and
+ *               adjoint aggregate, a fixed-order join with at most 8 later
+ *               records, then the reverse sweep from L2; dL/dw and dL/du
+ *               reduced in the same launch after a grid barrier) and CHAIN
+ *               the chain kernel; both need 16-byte aligned rows, otherwise
+ *               and for any other value the chunked kernel runs.
  *   spin_limit  bound on any one device-side wait (a predecessor's record,
  *               a shared-memory load, the grid barrier) in microseconds (the
  *               chunked kernels count polls of at most about 1 us each);

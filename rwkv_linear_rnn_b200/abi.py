@@ -9,7 +9,10 @@ from __future__ import annotations
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwkv.so")
+# LIBWKV_PATH selects another build of the library (e.g. one compiled with
+# different tile parameters); by default the in-tree build is used.
+LIB_PATH = os.environ.get("LIBWKV_PATH") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                          "libwkv.so")
 
 from .constants import *  # noqa: F401,F403  (codes shared with include/wkv.h)
 from .constants import WKV_OK

@@ -270,14 +270,14 @@ int wkv_backward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, 
   FwdArgs probe{};
   probe.B = B; probe.T = T; probe.C = C; probe.k = k; probe.v = v;
   const bool tma_ok = fwd_tma_eligible(probe, dtype) && ((uintptr_t)grad_y % 16) == 0;
-  if (tma_ok && kernel == WKV_KERNEL_SEGMENT) {
+  if (tma_ok && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT)) {
     const int64_t scratch = (int64_t)((L.sums - L.desc) / sizeof(double));
     return launch_backward_seg(a, dtype, grad_w, grad_u, reinterpret_cast<unsigned *>(base + L.cnt), scratch,
                                num_sms(), st) == cudaSuccess
                ? WKV_OK
                : WKV_ERR_CUDA;
   }
-  if (tma_ok && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_CHAIN)) {
+  if (tma_ok && kernel == WKV_KERNEL_CHAIN) {
     if (launch_backward_chain(a, dtype, st) != cudaSuccess) return WKV_ERR_CUDA;
     return launch_reduce_wu(a.part, 1, B, C, grad_w, grad_u, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
   }

@@ -43,6 +43,56 @@ __device__ __forceinline__ float fwd_token(Run &s, float K, float V, float u2, f
   return y;
 }
 
+// Batch fast path.  Within a batch of RB tokens the state can be held
+// against one reference exponent M instead of the running maximum, which
+// removes the per-token compare/select chain.  Two per-channel modes:
+//   undecayed (RB |w2| < 40): A_t = alpha 2^{M + t w2}; alpha is a plain sum,
+//     token j enters with the exactly formed weight 2^{K_j - (j+1) w2 - M},
+//     so no rounding accumulates through repeated decay; after the batch the
+//     state is (alpha, beta) at the anchored exponent (M, RB);
+//   decaying (RB |w2| >= 40): A_t = alpha 2^M, alpha <- alpha 2^{w2} + ...;
+//     every old term shrinks by at least 2^-2.5 per token, so the rounding of
+//     the repeated factor stays negligible; the state ends at (M, 0).
+// With kj_j = K_j - j w2e (w2e = w2 undecayed, 0 decaying) and
+// M = max(E0, max_j kj_j), token j costs e0 = 2^{kj_j - M}, eu = e0 2^{u2}
+// (the bonus term e^{u+k}), ek = e0 2^{-w2e} (the term that enters the
+// state), y = (alpha + eu v) / (beta + eu).  Everything stays in the float
+// range when M - min_j kj_j < 100 (every ek >= 2^-100 relative),
+// M - min_j (kj_j + u2) < 64 (denominator >= 2^-64) and u2 < 64; the caller
+// votes and otherwise runs the batch on the per-token rescaled path.
+struct FastC {
+  float w2e;   // decay folded into the exponents (undecayed mode) or 0
+  float ewm;   // per-token multiplicative decay (decaying mode) or 1
+  float cw;    // 2^{-w2e}
+  float cu;    // 2^{u2}
+  float nend;  // anchored decay count of the state after a batch
+};
+template <int RB>
+__device__ __forceinline__ FastC fast_consts(float w2, float u2) {
+  const bool decaying = fabsf(w2) * (float)RB >= 40.f;
+  FastC f;
+  f.w2e = decaying ? 0.f : w2;
+  f.ewm = decaying ? ex2(w2) : 1.f;
+  f.cw = ex2(-f.w2e);
+  f.cu = ex2(u2);
+  f.nend = decaying ? 0.f : (float)RB;
+  return f;
+}
+// kj and the reference M of a batch; true if this lane may take the fast path.
+template <int RB>
+__device__ __forceinline__ bool fast_prep(const float (&K)[RB], float E0, float u2, float w2e,
+                                          float (&kj)[RB], float &M) {
+  float mx = E0, mn = 3.0e38f;
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    kj[j] = fmaf(-(float)j, w2e, K[j]);
+    mx = fmaxf(mx, kj[j]);
+    mn = fminf(mn, kj[j]);
+  }
+  M = mx;
+  return (mx - mn < 100.f) && (mx - mn - u2 < 64.f) && (u2 < 64.f);
+}
+
 // Initial state of chain (b, c) from the caller's natural-log state.
 __device__ __forceinline__ St load_state_in(const float *st, int64_t i, int64_t BC) {
   if (!st) return st_empty();

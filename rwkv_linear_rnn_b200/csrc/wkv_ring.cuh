@@ -62,6 +62,22 @@ struct Ring {
     for (int a = 0; a < NARR; ++a) tma_load_2d(d[a], maps[a], x, y, bar(s));
     return true;
   }
+  // True when every stage of this warp's ring is 128-byte aligned (checked
+  // once; issue_stage then skips the per-copy check).
+  __device__ __forceinline__ bool aligned() const {
+    uint32_t bad = 0;
+    for (int s = 0; s < S; ++s)
+      for (int a = 0; a < NARR; ++a) bad |= smem_addr(stage(s, a)) & 127u;
+    return bad == 0;
+  }
+  // Loads into stage s (the caller tracks stages), with an L2 policy; the
+  // ring must have passed aligned().
+  __device__ __forceinline__ void issue_stage(const CUtensorMap *const (&maps)[NARR], int s, int x, int y,
+                                              uint64_t policy) const {
+    mbar_expect_tx(bar(s), (uint32_t)L::STAGE_BYTES);
+#pragma unroll
+    for (int a = 0; a < NARR; ++a) tma_load_2d_hint(smem_addr(stage(s, a)), maps[a], x, y, bar(s), policy);
+  }
   // Same with an L2 eviction-priority policy on the loads.
   __device__ __forceinline__ bool issue_hint(const CUtensorMap *const (&maps)[NARR], int64_t item,
                                             int x, int y, uint64_t policy) const {

@@ -43,42 +43,33 @@ struct SegArgs {
   int64_t nseg;  // segments per chain
 };
 
-constexpr int kBlockSeg = 32;  // segments per prefix block (one lane each)
+#ifndef WKV_SEGF_BLOCK
+#define WKV_SEGF_BLOCK 16
+#endif
+constexpr int kBlockSeg = WKV_SEGF_BLOCK;  // segments per prefix block (at most one per lane)
+static_assert(kBlockSeg >= 1 && kBlockSeg <= 32, "one lane per record");
 
-// Geometry of a segment (computed once per segment).
-struct Seg {
-  int64_t pos, chain, b;
-  int x;         // first channel of the chain (TMA column)
-  int64_t row0;  // b*T + first token (TMA row)
-};
-__device__ __forceinline__ Seg seg_of(const FwdArgs &p, int64_t unit, int TS) {
-  Seg s;
-  s.pos = unit / p.nchains;
-  s.chain = unit - s.pos * p.nchains;
-  s.b = s.chain / p.nct;
-  s.x = (int)((s.chain - s.b * p.nct) * 32);
-  s.row0 = s.b * p.T + s.pos * TS;
-  return s;
-}
-
-template <typename E, int TS, int S>
-__global__ void __launch_bounds__(128) fwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
+template <typename E, int TS, int S, int RB>
+__global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
                                                       const __grid_constant__ CUtensorMap vmap,
                                                       SegArgs a) {
-  constexpr int NBT = TS / kS3Batch;  // batches per pass
-  constexpr int IPU = 2 * NBT;        // ring items per segment
-  static_assert(TS % kCkpt == 0, "segments start on checkpoints");
+  constexpr int NBT = TS / RB;  // ring items per pass
+  constexpr int IPU = 2 * NBT;  // ring items per segment
+  static_assert(TS % RB == 0 && kCkpt % RB == 0, "checkpoints fall on batch starts");
   const FwdArgs &p = a.f;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  Ring<E, S> ring(smem, wl, (int)(blockDim.x >> 5));
+  const int nw = (int)(blockDim.x >> 5);
+  Ring<E, S, 2, RB> ring(smem, wl, nw);
   ring.init(lane);
   const CUtensorMap *const maps[2] = {&kmap, &vmap};
-  const int64_t G = (int64_t)gridDim.x * (blockDim.x >> 5);
-  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + wl;
-  const int64_t total = a.nseg * p.nchains;
-  const int64_t nu = total > g ? (total - g + G - 1) / G : 0;
-  const int64_t nitems = nu * IPU;
+  // unit indices fit 31 bits (the launcher checks nseg * nchains)
+  const int G = (int)gridDim.x * nw;
+  const int g = (int)blockIdx.x * nw + wl;
+  const int nseg = (int)a.nseg, nchains = (int)p.nchains, nct = (int)p.nct;
+  const int total = nseg * nchains;
+  const int nu = total > g ? (total - g + G - 1) / G : 0;
+  const int nitems = nu * IPU;
   const int64_t T = p.T, C = p.C, BC = p.B * p.C;
   const int64_t budget = p.spin_limit * 1000;
   unsigned epoch = 0;
@@ -86,82 +77,94 @@ __global__ void __launch_bounds__(128) fwd_seg_kernel(const __grid_constant__ CU
   epoch = __shfl_sync(0xffffffffu, epoch, 0);
   const unsigned want = (epoch_tag(epoch) << 2) | kAgg;
 
-  // Lane 0 issues ring items ahead of the consumer; the geometry of the
-  // segment being prefetched is cached so it is computed once per segment.
-  int64_t pf_i = -1;
-  Seg pf{};
-  uint64_t pol_keep = 0, pol_drop = 0;
-  if (lane == 0) {
-    pol_keep = l2_policy_evict_last();
-    pol_drop = l2_policy_evict_first();
+  // Lane 0 issues ring items ahead of the consumer, in consumption order
+  // (pass 1 batches, then the same batches again for pass 2), tracking the
+  // item's stage and unit with running counters.
+  int iss_k = 0, iss_done = 0, iss_unit = g, iss_r = 0, iss_s = 0, iss_x = 0, iss_row0 = 0;
+  if (lane == 0 && !ring.aligned()) {  // cannot happen with this layout; never issue a misaligned copy
+    atomicCAS(&p.hdr->status, 0, -4);
+    iss_k = nitems;
   }
-  auto issue = [&](int64_t k) {
-    const int64_t i = k / IPU;
-    const int r = (int)(k % IPU);
-    if (i != pf_i) {
-      pf_i = i;
-      pf = seg_of(p, g + i * G, TS);
+  auto issue_next = [&]() {
+    if (iss_r == 0) {
+      const int pos = iss_unit / nchains, chain = iss_unit - pos * nchains;
+      const int b = chain / nct;
+      iss_x = (chain - b * nct) * 32;
+      iss_row0 = (int)((int64_t)b * T + (int64_t)pos * TS);
     }
-    const int y = (int)(pf.row0 + (r % NBT) * kS3Batch);
-    const bool ok = ring.issue_hint(maps, k, pf.x, y, r < NBT ? pol_keep : pol_drop);
-    if (!ok) atomicCAS(&p.hdr->status, 0, -4 /* misaligned stage: nothing issued */);
+    const int bt = iss_r < NBT ? iss_r : iss_r - NBT;
+    ring.issue_stage(maps, iss_s, iss_x, iss_row0 + bt * RB,
+                     iss_r < NBT ? l2_policy_evict_last() : l2_policy_evict_first());
+    iss_done = ++iss_k;
+    iss_s = iss_s + 1 == S ? 0 : iss_s + 1;
+    if (++iss_r == IPU) {
+      iss_r = 0;
+      iss_unit += G;
+    }
   };
   if (lane == 0)
-    for (int64_t k = 0; k < min((int64_t)S - 1, nitems); ++k) issue(k);
+    while (iss_k < min(S - 1, nitems)) issue_next();
   bool failed = false;
-  // Consume item k: K (base-2 scaled) and V of its 16 rows.
-  auto take = [&](int64_t k, float(&K)[kS3Batch], float(&V)[kS3Batch]) {
-    const int s = (int)(k % S);
-    if (!failed && !mbar_wait(ring.bar(s), (uint32_t)(k / S) & 1u, budget, nullptr)) {
+  int cs = 0;
+  uint32_t cph = 0;
+  // Consume the next item: K (base-2 scaled) and V of its RB rows.
+  auto take = [&](float(&K)[RB], float(&V)[RB]) {
+    if (!failed && !mbar_wait(ring.bar(cs), cph, budget, nullptr)) {
       failed = true;
       if (lane == 0) atomicCAS(&p.hdr->status, 0, -5 /* WKV_ERR_TIMEOUT */);
     }
-    const E *kr = ring.stage(s, 0) + lane;
-    const E *vr = ring.stage(s, 1) + lane;
+    const E *kr = ring.stage(cs, 0) + lane;
+    const E *vr = ring.stage(cs, 1) + lane;
 #pragma unroll
-    for (int j = 0; j < kS3Batch; ++j) {
+    for (int j = 0; j < RB; ++j) {
       K[j] = to_f32(kr[j * 32]) * kLog2e;
       V[j] = to_f32(vr[j * 32]);
     }
     __syncwarp();  // the stage is read; it may be refilled
-    if (lane == 0 && k + S - 1 < nitems) {
+    if (++cs == S) {
+      cs = 0;
+      cph ^= 1u;
+    }
+    if (lane == 0 && iss_k < nitems && !failed) {  // after a failed wait nothing new is issued
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(k + S - 1);
+      issue_next();
     }
   };
 
-  for (int64_t i = 0; i < nu; ++i) {
-    const Seg sg = seg_of(p, g + i * G, TS);
-    const int64_t c = sg.x + lane;
+  for (int i = 0; i < nu; ++i) {
+    const int unit = g + i * G;
+    const int pos = unit / nchains, chain = unit - pos * nchains;
+    const int b = chain / nct;
+    const int64_t c = (int64_t)(chain - b * nct) * 32 + lane;
     const bool cok = c < C;
-    const int64_t t0 = sg.pos * TS;
+    const int64_t t0 = (int64_t)pos * TS;
     const int n = (int)min((int64_t)TS, T - t0);
     const float w2 = cok ? __ldg(p.w + c) * kLog2e : 0.f;
     const float u2 = cok ? __ldg(p.u + c) * kLog2e : 0.f;
-    const int64_t base_item = i * IPU;
+    const int64_t bc = (int64_t)b * C + c;
 
     // ---- pass 1: segment summary
     St agg = st_empty();
+#pragma unroll 1
     for (int bt = 0; bt < NBT; ++bt) {
-      float K[kS3Batch], V[kS3Batch];
-      take(base_item + bt, K, V);
-      const int nb = max(0, min(kS3Batch, n - bt * kS3Batch));
-      agg = combine(agg, summarize<kS3Batch>(K, V, w2, nb), (float)nb, w2);
+      float K[RB], V[RB];
+      take(K, V);
+      const int nb = max(0, min(RB, n - bt * RB));
+      agg = combine(agg, summarize<RB>(K, V, w2, nb), (float)nb, w2);
     }
 
     // ---- join: fold the earlier records of this chain (fixed order)
-    const int64_t q = sg.pos - sg.pos % kBlockSeg;  // first segment of this block
-    const int nrec = (int)(sg.pos - q) + (q > 0 ? 1 : 0);
-    const int64_t rec0 = q > 0 ? q - 1 : q;  // position of record 0
+    const int q = pos - pos % kBlockSeg;  // first segment of this block
+    const int nrec = (pos - q) + (q > 0 ? 1 : 0);
+    const int rec0 = q > 0 ? q - 1 : q;  // position of record 0
     // publish own summary now (the block's last segment publishes its
     // inclusive prefix below instead; the chain's last segment nothing)
-    const bool block_end = (sg.pos % kBlockSeg) == kBlockSeg - 1;
-    const int64_t unit = sg.pos * p.nchains + sg.chain;
-    const bool held = p.hold_first && sg.pos == 0;  // test hook: never publish
-    if (!block_end && sg.pos + 1 < a.nseg && !held) publish(p.desc, p.flags, unit, 0, agg, epoch, lane);
+    const bool block_end = (pos % kBlockSeg) == kBlockSeg - 1;
+    const bool held = p.hold_first && pos == 0;  // test hook: never publish
+    if (!block_end && pos + 1 < nseg && !held) publish(p.desc, p.flags, unit, 0, agg, epoch, lane);
     {
       const bool act = lane < nrec;
-      const unsigned *fl = p.flags + (rec0 + lane) * p.nchains + sg.chain;
+      const unsigned *fl = p.flags + (int64_t)(rec0 + lane) * nchains + chain;
       bool ready = !act;
       const uint64_t t_start = global_ns();
       unsigned backoff = 32;
@@ -177,16 +180,17 @@ __global__ void __launch_bounds__(128) fwd_seg_kernel(const __grid_constant__ CU
       }
       __syncwarp();
     }
-    St carry = (q == 0 && cok) ? load_state_in(p.state_in, sg.b * C + c, BC) : st_empty();
+    St carry = (q == 0 && cok) ? load_state_in(p.state_in, bc, BC) : st_empty();
+#pragma unroll 1
     for (int j0 = 0; j0 < nrec; j0 += 8) {
       St rec[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (j0 + j < nrec) rec[j] = desc_load<St>(p.desc, (rec0 + j0 + j) * p.nchains + sg.chain, 0, lane);
+        if (j0 + j < nrec) rec[j] = desc_load<St>(p.desc, (int64_t)(rec0 + j0 + j) * nchains + chain, 0, lane);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j0 + j < nrec) {
-          const int64_t rp = rec0 + j0 + j;
+          const int rp = rec0 + j0 + j;
           if (q > 0 && rp == q - 1)
             carry = rec[j];  // inclusive prefix of everything before this block
           else
@@ -194,28 +198,46 @@ __global__ void __launch_bounds__(128) fwd_seg_kernel(const __grid_constant__ CU
         }
       }
     }
-    if (block_end && sg.pos + 1 < a.nseg && !held)
+    if (block_end && pos + 1 < nseg && !held)
       publish(p.desc, p.flags, unit, 0, combine(carry, agg, (float)n, w2), epoch, lane);
 
     // ---- pass 2: replay from the carried-in state
     Run st = run_from(carry);
+    const FastC fc = fast_consts<RB>(w2, u2);
+#pragma unroll 1
     for (int bt = 0; bt < NBT; ++bt) {
-      float K[kS3Batch], V[kS3Batch];
-      take(base_item + NBT + bt, K, V);
-      const int nb = max(0, min(kS3Batch, n - bt * kS3Batch));
-      const int64_t tb = t0 + bt * kS3Batch;
+      float K[RB], V[RB];
+      take(K, V);
+      const int nb = max(0, min(RB, n - bt * RB));
+      const int64_t tb = t0 + bt * RB;
       if (p.ckpt && cok && nb > 0 && (tb % kCkpt) == 0)
-        store_ckpt(p.ckpt, tb / kCkpt, sg.b * C + c, BC, run_state(st), w2);
-      E *yp = (p.y && cok) ? static_cast<E *>(p.y) + (sg.b * T + tb) * C + c : nullptr;
-      if (nb == kS3Batch) {
+        store_ckpt(p.ckpt, tb / kCkpt, bc, BC, run_state(st), w2);
+      E *yp = (p.y && cok) ? static_cast<E *>(p.y) + ((int64_t)b * T + tb) * C + c : nullptr;
+      const float E0 = fmaf(st.n, w2, st.Panc);
+      float kj[RB], M;
+      const bool ok = fast_prep<RB>(K, E0, u2, fc.w2e, kj, M);
+      if (__all_sync(0xffffffffu, nb == RB && ok)) {
+        const float s0 = ex2(E0 - M);
+        float al = st.a * s0, be = st.b * s0;
 #pragma unroll
-        for (int j = 0; j < kS3Batch; ++j) {
+        for (int j = 0; j < RB; ++j) {
+          const float e0 = ex2(kj[j] - M);
+          const float eu = e0 * fc.cu, ek = e0 * fc.cw;
+          const float yv = fmaf(eu, V[j], al) * rcp(be + eu);
+          al = fmaf(al, fc.ewm, ek * V[j]);
+          be = fmaf(be, fc.ewm, ek);
+          if (yp) IO<E>::st(yp + (int64_t)j * C, yv);
+        }
+        st = Run{al, be, M, fc.nend};
+      } else if (nb == RB) {
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
           const float yv = fwd_token(st, K[j], V[j], u2, w2);
           if (yp) IO<E>::st(yp + (int64_t)j * C, yv);
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < kS3Batch; ++j) {
+        for (int j = 0; j < RB; ++j) {
           if (j < nb) {
             const float yv = fwd_token(st, K[j], V[j], u2, w2);
             if (yp) IO<E>::st(yp + (int64_t)j * C, yv);
@@ -223,28 +245,24 @@ __global__ void __launch_bounds__(128) fwd_seg_kernel(const __grid_constant__ CU
         }
       }
     }
-    if (p.state_out && cok && sg.pos == a.nseg - 1)
-      store_state(p.state_out, sg.b * C + c, BC, run_state(st), w2);
+    if (p.state_out && cok && pos == nseg - 1) store_state(p.state_out, bc, BC, run_state(st), w2);
   }
   if (failed && lane == 0)  // every issued load lands before the block exits
-    for (int64_t k = max((int64_t)0, nitems - S); k < nitems; ++k)
-      mbar_wait(ring.bar((int)(k % S)), (uint32_t)(k / S) & 1u, budget, nullptr);
+    for (int k = max(0, iss_done - S); k < iss_done; ++k)
+      mbar_wait(ring.bar(k % S), (uint32_t)(k / S) & 1u, budget, nullptr);
   // the last block to finish advances the launch epoch (no flag is read after this)
   __syncthreads();
   finish_block(p.hdr, gridDim.x);
 }
 
-constexpr int kSegRing = 4;
-
-template <typename E, int TS>
+template <typename E, int TS, int S, int RB>
 static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st) {
   CUtensorMap km, vm;
-  if (!encode_rows(&km, f.k, dtype, f.B * f.T, f.C, kS3Batch) ||
-      !encode_rows(&vm, f.v, dtype, f.B * f.T, f.C, kS3Batch))
+  if (!encode_rows(&km, f.k, dtype, f.B * f.T, f.C, RB) || !encode_rows(&vm, f.v, dtype, f.B * f.T, f.C, RB))
     return cudaErrorInvalidValue;
   constexpr int kWarps = 4;
-  constexpr int smem = WarpRing<E, kSegRing>::block_bytes(kWarps);
-  auto kern = fwd_seg_kernel<E, TS, kSegRing>;
+  constexpr int smem = WarpRing<E, S, 2, RB>::block_bytes(kWarps);
+  auto kern = fwd_seg_kernel<E, TS, S, RB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int occ = 0;
@@ -253,19 +271,39 @@ static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, cudaSt
   if (occ < 1) return cudaErrorInvalidConfiguration;
   SegArgs a{f, (f.T + TS - 1) / TS};
   const int64_t units = a.nseg * f.nchains;
-  // one resident wave (cooperative launch: every warp a segment may wait on
-  // is running), warps take segments round-robin in position-major order
-  const int64_t grid = std::min<int64_t>((units + kWarps - 1) / kWarps, (int64_t)occ * num_sms);
+  if (units >= (int64_t)1 << 31) return cudaErrorInvalidValue;  // unit indices are 31-bit
+  // One resident wave (cooperative launch: every warp a segment may wait on
+  // is running); warps take segments round-robin in position-major order and
+  // the grid is trimmed so that every warp gets the same number of them.
+  const int64_t max_warps = (int64_t)occ * num_sms * kWarps;
+  const int64_t rounds = (units + max_warps - 1) / max_warps;
+  const int64_t grid = ((units + rounds - 1) / rounds + kWarps - 1) / kWarps;
   void *args[] = {&km, &vm, &a};
-  return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3(kWarps * 32),
-                                     args, (size_t)smem, st);
+  return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3(kWarps * 32), args,
+                                     (size_t)smem, st);
 }
 
-int64_t seg_tokens(int dtype) { return dtype == 0 ? 128 : 256; }
+// Tile parameters (tokens per segment, ring stages, rows per ring item) per
+// element type; compile-time tunables.
+#ifndef WKV_SEGF_TS_F32
+#define WKV_SEGF_TS_F32 128
+#endif
+#ifndef WKV_SEGF_S_F32
+#define WKV_SEGF_S_F32 3
+#endif
+#ifndef WKV_SEGF_TS_BF16
+#define WKV_SEGF_TS_BF16 256
+#endif
+#ifndef WKV_SEGF_S_BF16
+#define WKV_SEGF_S_BF16 4
+#endif
+#ifndef WKV_SEGF_RB
+#define WKV_SEGF_RB 16
+#endif
 
 cudaError_t launch_forward_seg(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st) {
-  return dtype == 0 ? launch_seg_t<float, 128>(f, dtype, num_sms, st)
-                    : launch_seg_t<uint16_t, 256>(f, dtype, num_sms, st);
+  return dtype == 0 ? launch_seg_t<float, WKV_SEGF_TS_F32, WKV_SEGF_S_F32, WKV_SEGF_RB>(f, dtype, num_sms, st)
+                    : launch_seg_t<uint16_t, WKV_SEGF_TS_BF16, WKV_SEGF_S_BF16, WKV_SEGF_RB>(f, dtype, num_sms, st);
 }
 
 }  // namespace wkv

@@ -76,6 +76,69 @@ __device__ __forceinline__ Adj5s rjoin(const Adj5s &X, const Adj5s &Y, float len
   return o;
 }
 
+// Forward recompute of one batch of RB tokens from the anchored state
+// (xa, xb) 2^{xP + xn w2}: per token the scale qv of the denominator
+// (D_t = den_t 2^{qv_t}), gam = g / den, eta = gam y and e2 = e^{u+k} / 2^{qv};
+// the state advances past the batch.  Batch fast path when every lane allows
+// it (see fast_prep), else the per-token rescaled recurrence.
+template <int RB>
+__device__ __forceinline__ void recompute_batch(const float (&K)[RB], const float (&V)[RB],
+                                                const float (&Gy)[RB], float w2, float u2,
+                                                const FastC &fc, float &xa, float &xb, float &xP,
+                                                float &xn, float (&qv)[RB], float (&gam)[RB],
+                                                float (&eta)[RB], float (&e2v)[RB]) {
+  const float E0 = fmaf(xn, w2, xP);
+  float kj[RB], M;
+  const bool ok = fast_prep<RB>(K, E0, u2, fc.w2e, kj, M);
+  if (__all_sync(0xffffffffu, ok)) {
+    const float s0 = ex2(E0 - M);
+    float al = xa * s0, be = xb * s0;
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      const float e0 = ex2(kj[j] - M);
+      const float eu = e0 * fc.cu, ek = e0 * fc.cw;
+      const float rden = rcp(be + eu);
+      const float y = fmaf(eu, V[j], al) * rden;
+      qv[j] = fmaf((float)j, fc.w2e, M);
+      gam[j] = Gy[j] * rden;
+      eta[j] = gam[j] * y;
+      e2v[j] = eu;
+      al = fmaf(al, fc.ewm, ek * V[j]);
+      be = fmaf(be, fc.ewm, ek);
+    }
+    xa = al;
+    xb = be;
+    xP = M;
+    xn = fc.nend;
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    const float P = fmaf(xn, w2, xP);
+    const float UK = u2 + K[j];
+    const float d = P - UK;
+    const float x = ex2(-fabsf(d));
+    const bool pw = d >= 0.f;
+    const float e1 = pw ? 1.f : x, e2 = pw ? x : 1.f;
+    const float rden = rcp(fmaf(xb, e1, e2));
+    const float y = fmaf(xa, e1, V[j] * e2) * rden;
+    qv[j] = fmaxf(P, UK);
+    gam[j] = Gy[j] * rden;
+    eta[j] = gam[j] * y;
+    e2v[j] = e2;
+    const float n1 = xn + 1.f;
+    const float Pc = fmaf(n1, w2, xP);
+    const float d2 = K[j] - Pc;
+    const float x2 = ex2(-fabsf(d2));
+    const bool kw = d2 > 0.f;
+    const float so = kw ? x2 : 1.f, snw = kw ? 1.f : x2;
+    xa = fmaf(xa, so, V[j] * snw);
+    xb = fmaf(xb, so, snw);
+    xP = kw ? K[j] : xP;
+    xn = kw ? 0.f : n1;
+  }
+}
+
 struct SegBwdArgs {
   BwdArgs p;
   float *gw, *gu;
@@ -84,7 +147,14 @@ struct SegBwdArgs {
   int64_t ngroups;     // row groups per channel tile in the final reduction
 };
 
-constexpr int kBwdBlockSeg = 16;  // segments per suffix block
+#ifndef WKV_SEGB_BLOCK
+#define WKV_SEGB_BLOCK 8
+#endif
+constexpr int kBwdBlockSeg = WKV_SEGB_BLOCK;  // segments per suffix block (at most one per lane)
+static_assert(kBwdBlockSeg >= 1 && kBwdBlockSeg <= 32, "one lane per record");
+#ifndef WKV_SEGB_MINB
+#define WKV_SEGB_MINB 4
+#endif
 
 // int64 quotient through 32-bit division when both operands fit (the
 // common case; 64-bit division is a long instruction sequence).
@@ -105,7 +175,7 @@ struct SegBwdSmem {
 };
 
 template <typename E, int TS, int S, int RB>
-__global__ void __launch_bounds__(128, 4) bwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
                                                       const __grid_constant__ CUtensorMap vmap,
                                                       const __grid_constant__ CUtensorMap gmap,
                                                       SegBwdArgs a) {
@@ -126,12 +196,13 @@ __global__ void __launch_bounds__(128, 4) bwd_seg_kernel(const __grid_constant__
   // hold anything at their offset).
   if (blockIdx.x == 0)
     for (int64_t i = threadIdx.x; i < p.nct; i += blockDim.x) a.tile_cnt[i] = 0u;
-  const int64_t G = (int64_t)gridDim.x * nw;
-  const int64_t g = (int64_t)blockIdx.x * nw + wl;
-  const int64_t nseg = a.nseg;
-  const int64_t total = nseg * p.nchains;
-  const int64_t nu = total > g ? qdiv(total - g + G - 1, G) : 0;
-  const int64_t nitems = nu * IPU;
+  // unit indices fit 31 bits (the launcher checks nseg * nchains)
+  const int G = (int)gridDim.x * nw;
+  const int g = (int)blockIdx.x * nw + wl;
+  const int nseg = (int)a.nseg, nchains = (int)p.nchains, nct = (int)p.nct;
+  const int total = nseg * nchains;
+  const int nu = total > g ? (total - g + G - 1) / G : 0;
+  const int nitems = nu * IPU;
   const int64_t T = p.T, C = p.C, BC = p.B * p.C;
   const int64_t budget = p.spin_limit * 1000;
   unsigned epoch = 0;
@@ -139,42 +210,48 @@ __global__ void __launch_bounds__(128, 4) bwd_seg_kernel(const __grid_constant__
   epoch = __shfl_sync(0xffffffffu, epoch, 0);
   const unsigned want = (epoch_tag(epoch) << 2) | kAgg;
 
-  // Lane 0 issues ring items ahead of the consumer.  Item r of a unit: pass 1
-  // batch r (r < NB), pass 2 batch IPU-1-r (r >= NB, last batch first).
-  int64_t pf_i = -1, pf_row0 = 0;
-  int pf_x = 0;
-  uint64_t pol_keep = 0, pol_drop = 0;
+  // Lane 0 issues ring items ahead of the consumer, in consumption order.
+  // Item r of a unit: pass 1 batch r (r < NB), pass 2 batch IPU-1-r (last
+  // batch first).  Running counters (item, stage, unit) avoid divisions.
+  int iss_k = 0, iss_unit = g, iss_r = 0, iss_s = 0, iss_x = 0, iss_row0 = 0;
+  int iss_done = 0;  // copies actually issued (lane 0)
   if (lane == 0) {
-    pol_keep = l2_policy_evict_last();
-    pol_drop = l2_policy_evict_first();
-  }
-  auto issue = [&](int64_t k) {
-    const int64_t i = k / IPU;
-    const int r = (int)(k % IPU);
-    if (i != pf_i) {
-      pf_i = i;
-      const int64_t unit = g + i * G;
-      const int64_t rpos = qdiv(unit, p.nchains), chain = unit - rpos * p.nchains;
-      const int64_t b = qdiv(chain, p.nct);
-      pf_x = (int)((chain - b * p.nct) * 32);
-      pf_row0 = b * T + (nseg - 1 - rpos) * TS;
+    if (!ring.aligned()) {  // cannot happen with this layout; never issue a misaligned copy
+      atomicCAS(&p.hdr->status, 0, -4);
+      iss_k = nitems;
     }
-    const int bt = r < NB ? r : IPU - 1 - r;
-    const bool ok = ring.issue_hint(maps, k, pf_x, (int)(pf_row0 + bt * RB), r < NB ? pol_keep : pol_drop);
-    if (!ok) atomicCAS(&p.hdr->status, 0, -4 /* misaligned stage: nothing issued */);
+  }
+  auto issue_next = [&]() {
+    if (iss_r == 0) {
+      const int rpos = iss_unit / nchains, chain = iss_unit - rpos * nchains;
+      const int b = chain / nct;
+      iss_x = (chain - b * nct) * 32;
+      iss_row0 = (int)((int64_t)b * T + (int64_t)(nseg - 1 - rpos) * TS);
+    }
+    const int bt = iss_r < NB ? iss_r : IPU - 1 - iss_r;
+    ring.issue_stage(maps, iss_s, iss_x, iss_row0 + bt * RB,
+                     iss_r < NB ? l2_policy_evict_last() : l2_policy_evict_first());
+    ++iss_k;
+    iss_done = iss_k;
+    iss_s = iss_s + 1 == S ? 0 : iss_s + 1;
+    if (++iss_r == IPU) {
+      iss_r = 0;
+      iss_unit += G;
+    }
   };
   if (lane == 0)
-    for (int64_t k = 0; k < min((int64_t)S - 1, nitems); ++k) issue(k);
+    while (iss_k < min(S - 1, nitems)) issue_next();
   bool failed = false;
-  auto take = [&](int64_t k, float(&K)[RB], float(&V)[RB], float(&Gy)[RB]) {
-    const int s = (int)(k % S);
-    if (!failed && !mbar_wait(ring.bar(s), (uint32_t)(k / S) & 1u, budget, nullptr)) {
+  int cs = 0;           // stage of the next item to consume
+  uint32_t cph = 0;     // its mbarrier phase parity
+  auto take = [&](float(&K)[RB], float(&V)[RB], float(&Gy)[RB]) {
+    if (!failed && !mbar_wait(ring.bar(cs), cph, budget, nullptr)) {
       failed = true;
       if (lane == 0) atomicCAS(&p.hdr->status, 0, -5 /* WKV_ERR_TIMEOUT */);
     }
-    const E *kr = ring.stage(s, 0) + lane;
-    const E *vr = ring.stage(s, 1) + lane;
-    const E *gr = ring.stage(s, 2) + lane;
+    const E *kr = ring.stage(cs, 0) + lane;
+    const E *vr = ring.stage(cs, 1) + lane;
+    const E *gr = ring.stage(cs, 2) + lane;
 #pragma unroll
     for (int j = 0; j < RB; ++j) {
       K[j] = to_f32(kr[j * 32]) * kLog2e;
@@ -182,25 +259,37 @@ __global__ void __launch_bounds__(128, 4) bwd_seg_kernel(const __grid_constant__
       Gy[j] = to_f32(gr[j * 32]);
     }
     __syncwarp();  // the stage is read; it may be refilled
-    if (lane == 0 && k + S - 1 < nitems) {
+    if (++cs == S) {
+      cs = 0;
+      cph ^= 1u;
+    }
+    if (lane == 0 && iss_k < nitems && !failed) {  // after a failed wait nothing new is issued
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(k + S - 1);
+      issue_next();
+    }
+  };
+  // Tokens past T (only in a chain's last segment) are computed on whatever
+  // the loads brought but enter with a zero gradient, so they add nothing.
+  auto mask_tail = [&](float(&Gy)[RB], int nb) {
+    if (nb < RB) {
+#pragma unroll
+      for (int j = 0; j < RB; ++j) Gy[j] = j < nb ? Gy[j] : 0.f;
     }
   };
 
-  for (int64_t i = 0; i < nu; ++i) {
-    const int64_t unit = g + i * G;
-    const int64_t rpos = qdiv(unit, p.nchains), chain = unit - rpos * p.nchains;
-    const int64_t b = qdiv(chain, p.nct);
-    const int64_t c = (chain - b * p.nct) * 32 + lane;
+  for (int i = 0; i < nu; ++i) {
+    const int unit = g + i * G;
+    const int rpos = unit / nchains, chain = unit - rpos * nchains;
+    const int b = chain / nct;
+    const int64_t c = (int64_t)(chain - b * nct) * 32 + lane;
     const bool cok = c < C;
-    const int64_t pos = nseg - 1 - rpos;
-    const int64_t t0 = pos * TS;
+    const int pos = nseg - 1 - rpos;
+    const int64_t t0 = (int64_t)pos * TS;
     const int n = (int)min((int64_t)TS, T - t0);
     const float w2 = cok ? __ldg(p.w + c) * kLog2e : 0.f;
     const float u2 = cok ? __ldg(p.u + c) * kLog2e : 0.f;
-    const int64_t base_item = i * IPU;
-    const int64_t bc = b * C + c;
+    const int64_t bc = (int64_t)b * C + c;
+    const FastC fc = fast_consts<RB>(w2, u2);
 
     // ---- pass 1: forward recompute and the segment's adjoint aggregate
     // The forward state is (fa, fb) 2^E with E = fP + fn w2 (anchored).
@@ -218,61 +307,40 @@ __global__ void __launch_bounds__(128, 4) bwd_seg_kernel(const __grid_constant__
       sts[bt * 96 + 32 + lane] = fb;
       sts[bt * 96 + 64 + lane] = fmaf(fn, w2, fP);
       float K[RB], V[RB], Gy[RB];
-      take(base_item + bt, K, V, Gy);
-      const int nb = max(0, min(RB, n - bt * RB));
+      take(K, V, Gy);
+      mask_tail(Gy, n - bt * RB);
+      float qv[RB], gam[RB], eta[RB], e2v[RB];
+      recompute_batch<RB>(K, V, Gy, w2, u2, fc, fa, fb, fP, fn, qv, gam, eta, e2v);
       const float lag0 = (float)(bt * RB);
 #pragma unroll
       for (int j = 0; j < RB; ++j) {
-        if (j < nb) {
-          const float P = fmaf(fn, w2, fP);
-          const float UK = u2 + K[j];
-          const float d = P - UK;
-          const float x = ex2(-fabsf(d));
-          const bool pw = d >= 0.f;
-          const float e1 = pw ? 1.f : x, e2 = pw ? x : 1.f;
-          const float rden = rcp(fmaf(fb, e1, e2));
-          const float y = fmaf(fa, e1, V[j] * e2) * rden;
-          const float gam = Gy[j] * rden;
-          const float eta = gam * y;
-          // token s = t0 + lag enters the aggregate with 2^{lag w2 - q_s}
-          const float lag = lag0 + (float)j;
-          const float es = fmaf(lag, w2, -fmaxf(P, UK));
-          const float da = es - Em;
-          const float xa = ex2(-fabsf(da));
-          const bool up = da > 0.f;
-          const float fo = up ? xa : 1.f, fg = up ? 1.f : xa;
-          const float gg = gam * fg, ee = eta * fg;
-          ah = fmaf(ah, fo, gg);
-          hh = fmaf(hh, fo, ee);
-          ahp = fmaf(ahp, fo, lag * gg);
-          hhp = fmaf(hhp, fo, lag * ee);
-          Em = up ? es : Em;
-          // forward state update
-          const float n1 = fn + 1.f;
-          const float Pc = fmaf(n1, w2, fP);
-          const float d2 = K[j] - Pc;
-          const float x2 = ex2(-fabsf(d2));
-          const bool kw = d2 > 0.f;
-          const float so = kw ? x2 : 1.f, snw = kw ? 1.f : x2;
-          fa = fmaf(fa, so, V[j] * snw);
-          fb = fmaf(fb, so, snw);
-          fP = kw ? K[j] : fP;
-          fn = kw ? 0.f : n1;
-        }
+        // token s = t0 + lag enters the aggregate with 2^{lag w2 - q_s}
+        const float lag = lag0 + (float)j;
+        const float es = fmaf(lag, w2, -qv[j]);
+        const float da = es - Em;
+        const float xa = ex2(-fabsf(da));
+        const bool up = da > 0.f;
+        const float fo = up ? xa : 1.f, fg = up ? 1.f : xa;
+        const float gg = gam[j] * fg, ee = eta[j] * fg;
+        ah = fmaf(ah, fo, gg);
+        hh = fmaf(hh, fo, ee);
+        ahp = fmaf(ahp, fo, lag * gg);
+        hhp = fmaf(hhp, fo, lag * ee);
+        Em = up ? es : Em;
       }
     }
     const Adj5s agg{ah, hh, ahp, hhp, -Em};
 
     // ---- join: adjoint at the segment end from the later segments' records
-    const int64_t q = rpos - rpos % kBwdBlockSeg;  // first (latest) segment of this block
-    const int nrec = (int)(rpos - q) + (q > 0 ? 1 : 0);
-    const int64_t rec0 = q > 0 ? q - 1 : q;
+    const int q = rpos - rpos % kBwdBlockSeg;  // first (latest) segment of this block
+    const int nrec = (rpos - q) + (q > 0 ? 1 : 0);
+    const int rec0 = q > 0 ? q - 1 : q;
     const bool block_end = (rpos % kBwdBlockSeg) == kBwdBlockSeg - 1;
     const bool held = p.hold_first && rpos == 0;  // test hook: never publish
     if (!block_end && rpos + 1 < nseg && !held) publish(p.desc, p.flags, unit, 0, agg, epoch, lane);
     {
       const bool act = lane < nrec;
-      const unsigned *fl = p.flags + (rec0 + lane) * p.nchains + chain;
+      const unsigned *fl = p.flags + (int64_t)(rec0 + lane) * nchains + chain;
       bool ready = !act;
       const uint64_t t_start = global_ns();
       unsigned backoff = 32;
@@ -295,11 +363,11 @@ __global__ void __launch_bounds__(128, 4) bwd_seg_kernel(const __grid_constant__
       Adj5s rec[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (j0 + j < nrec) rec[j] = desc_load<Adj5s>(p.desc, (rec0 + j0 + j) * p.nchains + chain, 0, lane);
+        if (j0 + j < nrec) rec[j] = desc_load<Adj5s>(p.desc, (int64_t)(rec0 + j0 + j) * nchains + chain, 0, lane);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j0 + j < nrec) {
-          const int64_t rp = rec0 + j0 + j;
+          const int rp = rec0 + j0 + j;
           if (q > 0 && rp == q - 1)
             acc = rec[j];  // adjoint at the start of the previous block's last segment
           else
@@ -317,70 +385,41 @@ __global__ void __launch_bounds__(128, 4) bwd_seg_kernel(const __grid_constant__
     for (int bi = 0; bi < NB; ++bi) {
       const int bt = NB - 1 - bi;
       float K[RB], V[RB], Gy[RB];
-      take(base_item + NB + bi, K, V, Gy);
-      const int nb = max(0, min(RB, n - bt * RB));
+      take(K, V, Gy);
+      const int nb = n - bt * RB;  // valid tokens of the batch (may be <= 0 or > RB)
+      mask_tail(Gy, nb);
       float qv[RB], gam[RB], eta[RB], e2v[RB];
       {
         float xa = sts[bt * 96 + lane], xb = sts[bt * 96 + 32 + lane], xP = sts[bt * 96 + 64 + lane];
         float xn = 0.f;
-#pragma unroll
-        for (int j = 0; j < RB; ++j) {
-          qv[j] = 0.f;
-          gam[j] = eta[j] = e2v[j] = 0.f;
-          if (j < nb) {
-            const float P = fmaf(xn, w2, xP);
-            const float UK = u2 + K[j];
-            const float d = P - UK;
-            const float x = ex2(-fabsf(d));
-            const bool pw = d >= 0.f;
-            const float e1 = pw ? 1.f : x, e2 = pw ? x : 1.f;
-            const float rden = rcp(fmaf(xb, e1, e2));
-            const float y = fmaf(xa, e1, V[j] * e2) * rden;
-            qv[j] = fmaxf(P, UK);
-            gam[j] = Gy[j] * rden;
-            eta[j] = gam[j] * y;
-            e2v[j] = e2;
-            const float n1 = xn + 1.f;
-            const float Pc = fmaf(n1, w2, xP);
-            const float d2 = K[j] - Pc;
-            const float x2 = ex2(-fabsf(d2));
-            const bool kw = d2 > 0.f;
-            const float so = kw ? x2 : 1.f, snw = kw ? 1.f : x2;
-            xa = fmaf(xa, so, V[j] * snw);
-            xb = fmaf(xb, so, snw);
-            xP = kw ? K[j] : xP;
-            xn = kw ? 0.f : n1;
-          }
-        }
+        recompute_batch<RB>(K, V, Gy, w2, u2, fc, xa, xb, xP, xn, qv, gam, eta, e2v);
       }
-      E *gkp = static_cast<E *>(p.gk) + (b * T + t0 + bt * RB) * C + c;
-      E *gvp = static_cast<E *>(p.gv) + (b * T + t0 + bt * RB) * C + c;
+      E *gkp = static_cast<E *>(p.gk) + ((int64_t)b * T + t0 + bt * RB) * C + c;
+      E *gvp = static_cast<E *>(p.gv) + ((int64_t)b * T + t0 + bt * RB) * C + c;
 #pragma unroll
       for (int j = RB - 1; j >= 0; --j) {
-        if (j < nb) {
-          const float rn = fmaf(-m, w2, Ranc);  // scale of the adjoint after token t
-          const float tn = ex2(K[j] - rn);      // e^{k_t} 2^{-r_{t+1}} (<= 1)
-          const float gv = fmaf(gam[j], e2v[j], tn * rah);
-          const float gk = fmaf(V[j], gv, -fmaf(eta[j], e2v[j], tn * rhh));
-          gw_acc = fmaf(tn, fmaf(V[j], rahp, -rhhp), gw_acc);
-          gu_acc = fmaf(e2v[j], fmaf(gam[j], V[j], -eta[j]), gu_acc);
-          if (cok) {
-            IO<E>::st(gkp + (int64_t)j * C, gk);
-            IO<E>::st(gvp + (int64_t)j * C, gv);
-          }
-          const float m1 = m + 1.f;
-          const float Rc = fmaf(-m1, w2, Ranc);
-          const float d = qv[j] - Rc;
-          const float x = ex2(-fabsf(d));
-          const bool reset = d < 0.f;
-          const float fg = reset ? 1.f : x, fo = reset ? x : 1.f;
-          rahp = fo * (rah + rahp);
-          rhhp = fo * (rhh + rhhp);
-          rah = fmaf(rah, fo, gam[j] * fg);
-          rhh = fmaf(rhh, fo, eta[j] * fg);
-          Ranc = reset ? qv[j] : Ranc;
-          m = reset ? 0.f : m1;
+        const float rn = fmaf(-m, w2, Ranc);  // scale of the adjoint after token t
+        const float tn = ex2(K[j] - rn);      // e^{k_t} 2^{-r_{t+1}} (<= 1)
+        const float gv = fmaf(gam[j], e2v[j], tn * rah);
+        const float gk = fmaf(V[j], gv, -fmaf(eta[j], e2v[j], tn * rhh));
+        gw_acc = fmaf(tn, fmaf(V[j], rahp, -rhhp), gw_acc);
+        gu_acc = fmaf(e2v[j], fmaf(gam[j], V[j], -eta[j]), gu_acc);
+        if (cok && j < nb) {
+          IO<E>::st(gkp + (int64_t)j * C, gk);
+          IO<E>::st(gvp + (int64_t)j * C, gv);
         }
+        const float m1 = m + 1.f;
+        const float Rc = fmaf(-m1, w2, Ranc);
+        const float d = qv[j] - Rc;
+        const float x = ex2(-fabsf(d));
+        const bool reset = d < 0.f;
+        const float fg = reset ? 1.f : x, fo = reset ? x : 1.f;
+        rahp = fo * (rah + rahp);
+        rhhp = fo * (rhh + rhhp);
+        rah = fmaf(rah, fo, gam[j] * fg);
+        rhh = fmaf(rhh, fo, eta[j] * fg);
+        Ranc = reset ? qv[j] : Ranc;
+        m = reset ? 0.f : m1;
       }
     }
     if (cok) {
@@ -390,13 +429,13 @@ __global__ void __launch_bounds__(128, 4) bwd_seg_kernel(const __grid_constant__
         const float r0 = fmaf(-m, w2, Ranc);
         gw_acc = fmaf(ex2(ck[2 * BC] - r0), fmaf(ck[0], rahp, -ck[BC] * rhhp), gw_acc);
       }
-      p.part[(pos * 2 + 0) * BC + bc] = gw_acc;
-      p.part[(pos * 2 + 1) * BC + bc] = gu_acc;
+      p.part[(int64_t)(pos * 2 + 0) * BC + bc] = gw_acc;
+      p.part[(int64_t)(pos * 2 + 1) * BC + bc] = gu_acc;
     }
   }
   if (failed && lane == 0)  // every issued load lands before the block exits
-    for (int64_t k = max((int64_t)0, nitems - S); k < nitems; ++k)
-      mbar_wait(ring.bar((int)(k % S)), (uint32_t)(k / S) & 1u, budget, nullptr);
+    for (int k = max(0, iss_done - S); k < iss_done; ++k)
+      mbar_wait(ring.bar(k % S), (uint32_t)(k / S) & 1u, budget, nullptr);
 
   // ---- dL/dw, dL/du: fixed-order two-level reduction of the partials
   grid_barrier(p.hdr, gridDim.x, budget);
@@ -467,9 +506,15 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
   a.tile_cnt = tile_cnt;
   a.nseg = (p.T + TS - 1) / TS;
   const int64_t units = a.nseg * p.nchains;
-  // one resident wave (cooperative launch: every warp a segment may wait on,
-  // and every block of the grid barrier, is running)
-  const int64_t grid = std::min<int64_t>((units + kWarps - 1) / kWarps, (int64_t)occ * num_sms);
+  if (units >= (int64_t)1 << 31) return cudaErrorInvalidValue;  // unit indices are 31-bit
+  // One resident wave (cooperative launch: every warp a segment may wait on,
+  // and every block of the grid barrier, is running).  Warps take segments
+  // round-robin; the grid is trimmed so that every warp gets the same number
+  // of segments (no final round with most warps idle).
+  const int64_t max_warps = (int64_t)occ * num_sms * kWarps;
+  const int64_t rounds = (units + max_warps - 1) / max_warps;
+  const int64_t want = (units + rounds - 1) / rounds;
+  const int64_t grid = (want + kWarps - 1) / kWarps;
   const int64_t G = grid * kWarps;
   // row groups per channel tile: enough to spread the partial rows over the
   // warps, at least 8 rows each, and the group sums must fit the scratch
@@ -482,13 +527,27 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
                                      (size_t)smem, st);
 }
 
-constexpr int kSegBwdTS = 64;
+// Tile parameters (tokens per segment, ring stages, rows per ring item);
+// compile-time tunables.
+#ifndef WKV_SEGB_TS
+#define WKV_SEGB_TS 64
+#endif
+#ifndef WKV_SEGB_S_F32
+#define WKV_SEGB_S_F32 3
+#endif
+#ifndef WKV_SEGB_S_BF16
+#define WKV_SEGB_S_BF16 4
+#endif
+#ifndef WKV_SEGB_RB
+#define WKV_SEGB_RB 8
+#endif
 
 cudaError_t launch_backward_seg(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
                                 int64_t scratch_doubles, int num_sms, cudaStream_t st) {
-  return dtype == 0
-             ? launch_bwd_seg_t<float, kSegBwdTS, 3, 8>(p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, st)
-             : launch_bwd_seg_t<uint16_t, kSegBwdTS, 4, 8>(p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, st);
+  return dtype == 0 ? launch_bwd_seg_t<float, WKV_SEGB_TS, WKV_SEGB_S_F32, WKV_SEGB_RB>(
+                          p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, st)
+                    : launch_bwd_seg_t<uint16_t, WKV_SEGB_TS, WKV_SEGB_S_BF16, WKV_SEGB_RB>(
+                          p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, st);
 }
 
 }  // namespace wkv

@@ -249,6 +249,43 @@ def test_backward_bf16_small(kernel):
     assert_grads(got, grads_ref(w, u, k, v, g), BF16_TOL)
 
 
+# Cases that steer the segment kernels' batch fast path and its fallback:
+# keys spread over hundreds of binades (fallback), a dominant early spike
+# followed by small keys, and a near-zero decay over a long sequence (the
+# undecayed mode, where a repeated decay factor would accumulate rounding).
+RANGE_CASES = {
+    "wide_keys": dict(B=2, T=700, C=64, td=(-6.0, 3.0), kstd=40.0),
+    "near_zero_decay": dict(B=1, T=6000, C=64, td=(-9.0, -6.0), kstd=1.0),
+    "strong_decay": dict(B=2, T=500, C=64, td=(1.5, 3.0), kstd=2.0),
+}
+
+
+def _range_case(name, seed):
+    c = RANGE_CASES[name]
+    w, u, k, v, g, _ = small_case(c["B"], c["T"], c["C"], seed=seed, td=c["td"], kstd=c["kstd"])
+    if name == "wide_keys":
+        k[:, 5, :] = 60.0   # an early spike that dominates the state for a while
+        k[:, 300:340, :] = -80.0
+    return w, u, k, v, g
+
+
+@pytest.mark.parametrize("name", sorted(RANGE_CASES))
+def test_segment_forward_ranges(name):
+    w, u, k, v, g = _range_case(name, seed=41)
+    y, _, _ = W.forward(dev(w), dev(u), dev(k), dev(v), kernel=W.WKV_KERNEL_SEGMENT)
+    y_ref, _ = oracle.fwd_recur(w, u, k, v)
+    assert fwd_err(host(y), y_ref) <= F32_FWD_TOL
+
+
+@pytest.mark.parametrize("name", sorted(RANGE_CASES))
+def test_segment_backward_ranges(name):
+    w, u, k, v, g = _range_case(name, seed=43)
+    W_, U_, K_, V_ = dev(w), dev(u), dev(k), dev(v)
+    _, _, ck = W.forward(W_, U_, K_, V_, want_ckpt=True, kernel=W.WKV_KERNEL_SEGMENT)
+    got = W.backward(W_, U_, K_, V_, dev(g), ckpt=ck, kernel=W.WKV_KERNEL_SEGMENT)
+    assert_grads(got, grads_ref(w, u, k, v, g), F32_GRAD_TOL)
+
+
 def test_backward_tiny_workload_vs_direct():
     inp = workloads.generate("tiny")
     w, u, k, v, gy = inputs_to_device(inp)
