@@ -199,17 +199,16 @@ __device__ __forceinline__ St get_st(const float *d, int lane) {
   return St{d[lane], d[32 + lane], d[64 + lane], d[96 + lane]};
 }
 
-// Publish a record and then its flag with release semantics (all lanes of
-// the warp call this together).
+// Publish a record and then its flag (all lanes of the warp call this
+// together).  The warp barrier orders every lane's record stores before lane
+// 0's flag store, and the flag store is a gpu-scope release, which is
+// cumulative: a reader that acquires the flag sees the whole record.
 template <typename S>
 __device__ __forceinline__ void publish(float *desc, unsigned *flags, int64_t tile, int which,
                                        const S &s, unsigned epoch, int lane) {
   desc_store(desc, tile, which, s, lane);
   __syncwarp();
-  if (lane == 0) {
-    __threadfence();
-    st_release(flags + tile, (epoch_tag(epoch) << 2) | kAgg);
-  }
+  if (lane == 0) st_release(flags + tile, (epoch_tag(epoch) << 2) | kAgg);
   __syncwarp();
 }
 

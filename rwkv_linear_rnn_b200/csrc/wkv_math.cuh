@@ -43,6 +43,28 @@ __device__ __forceinline__ float fwd_token(Run &s, float K, float V, float u2, f
   return y;
 }
 
+// summarize for a full batch: the maximum exponent by a plain max and the
+// state anchored at it with no decay steps (the anchor is one rounding off
+// exact, like any exponent formed from an anchored one).
+template <int L>
+__device__ __forceinline__ St summarize_full(const float (&K)[L], const float (&V)[L], float w2) {
+  float e[L];
+  float m = -3.0e38f;
+#pragma unroll
+  for (int j = 0; j < L; ++j) {
+    e[j] = fmaf((float)(L - 1 - j), w2, K[j]);
+    m = fmaxf(m, e[j]);
+  }
+  float a = 0.f, b = 0.f;
+#pragma unroll
+  for (int j = 0; j < L; ++j) {
+    const float x = ex2(e[j] - m);
+    a = fmaf(x, V[j], a);
+    b += x;
+  }
+  return St{a, b, m, 0.f};
+}
+
 // Batch fast path.  Within a batch of RB tokens the state can be held
 // against one reference exponent M instead of the running maximum, which
 // removes the per-token compare/select chain.  Two per-channel modes:

@@ -41,6 +41,8 @@ bool encode_rows(CUtensorMap *m, const void *ptr, int dtype, int64_t rows, int64
 struct SegArgs {
   FwdArgs f;
   int64_t nseg;  // segments per chain
+  int ts;        // tokens per segment (a multiple of the batch rows)
+  int nbt;       // batches per segment (ts / rows per batch)
 };
 
 #ifndef WKV_SEGF_BLOCK
@@ -49,13 +51,14 @@ struct SegArgs {
 constexpr int kBlockSeg = WKV_SEGF_BLOCK;  // segments per prefix block (at most one per lane)
 static_assert(kBlockSeg >= 1 && kBlockSeg <= 32, "one lane per record");
 
-template <typename E, int TS, int S, int RB>
+template <typename E, int S, int RB>
 __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
                                                       const __grid_constant__ CUtensorMap vmap,
                                                       SegArgs a) {
-  constexpr int NBT = TS / RB;  // ring items per pass
-  constexpr int IPU = 2 * NBT;  // ring items per segment
-  static_assert(TS % RB == 0 && kCkpt % RB == 0, "checkpoints fall on batch starts");
+  static_assert(kCkpt % RB == 0, "checkpoints fall on batch starts");
+  const int TS = a.ts;       // tokens per segment
+  const int NBT = a.nbt;     // ring items per pass
+  const int IPU = 2 * NBT;   // ring items per segment
   const FwdArgs &p = a.f;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -150,7 +153,8 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
       float K[RB], V[RB];
       take(K, V);
       const int nb = max(0, min(RB, n - bt * RB));
-      agg = combine(agg, summarize<RB>(K, V, w2, nb), (float)nb, w2);
+      const St sb = nb == RB ? summarize_full<RB>(K, V, w2) : summarize<RB>(K, V, w2, nb);
+      agg = combine(agg, sb, (float)nb, w2);
     }
 
     // ---- join: fold the earlier records of this chain (fixed order)
@@ -255,21 +259,30 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
   finish_block(p.hdr, gridDim.x);
 }
 
-template <typename E, int TS, int S, int RB>
-static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st) {
+template <typename E, int S, int RB>
+static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, int ts_max, cudaStream_t st) {
   CUtensorMap km, vm;
   if (!encode_rows(&km, f.k, dtype, f.B * f.T, f.C, RB) || !encode_rows(&vm, f.v, dtype, f.B * f.T, f.C, RB))
     return cudaErrorInvalidValue;
   constexpr int kWarps = 4;
   constexpr int smem = WarpRing<E, S, 2, RB>::block_bytes(kWarps);
-  auto kern = fwd_seg_kernel<E, TS, S, RB>;
+  auto kern = fwd_seg_kernel<E, S, RB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int occ = 0;
   if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kWarps * 32, smem)) != cudaSuccess)
     return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
-  SegArgs a{f, (f.T + TS - 1) / TS};
+  // Segment length: as short as it takes to give every resident warp a
+  // segment (more warps hide more latency), but not longer than ts_max (the
+  // rows between a segment's two passes must stay in L2) nor shorter than
+  // four batches (the join costs a segment a fixed amount).
+  const int64_t max_warps0 = (int64_t)occ * num_sms * kWarps;
+  const int64_t segs_wanted = std::max<int64_t>(1, max_warps0 / f.nchains);
+  int64_t ts = (f.T + segs_wanted - 1) / segs_wanted;
+  ts = (ts + RB - 1) / RB * RB;
+  ts = std::max<int64_t>(4 * RB, std::min<int64_t>(ts, ts_max));
+  SegArgs a{f, (f.T + ts - 1) / ts, (int)ts, (int)(ts / RB)};
   const int64_t units = a.nseg * f.nchains;
   if (units >= (int64_t)1 << 31) return cudaErrorInvalidValue;  // unit indices are 31-bit
   // One resident wave (cooperative launch: every warp a segment may wait on
@@ -283,8 +296,8 @@ static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, cudaSt
                                      (size_t)smem, st);
 }
 
-// Tile parameters (tokens per segment, ring stages, rows per ring item) per
-// element type; compile-time tunables.
+// Tile parameters per element type (compile-time tunables): the longest
+// segment (tokens), ring stages, rows per ring item.
 #ifndef WKV_SEGF_TS_F32
 #define WKV_SEGF_TS_F32 128
 #endif
@@ -302,8 +315,8 @@ static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, cudaSt
 #endif
 
 cudaError_t launch_forward_seg(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st) {
-  return dtype == 0 ? launch_seg_t<float, WKV_SEGF_TS_F32, WKV_SEGF_S_F32, WKV_SEGF_RB>(f, dtype, num_sms, st)
-                    : launch_seg_t<uint16_t, WKV_SEGF_TS_BF16, WKV_SEGF_S_BF16, WKV_SEGF_RB>(f, dtype, num_sms, st);
+  return dtype == 0 ? launch_seg_t<float, WKV_SEGF_S_F32, WKV_SEGF_RB>(f, dtype, num_sms, WKV_SEGF_TS_F32, st)
+                    : launch_seg_t<uint16_t, WKV_SEGF_S_BF16, WKV_SEGF_RB>(f, dtype, num_sms, WKV_SEGF_TS_BF16, st);
 }
 
 }  // namespace wkv

@@ -81,14 +81,17 @@ __device__ __forceinline__ Adj5s rjoin(const Adj5s &X, const Adj5s &Y, float len
 // (D_t = den_t 2^{qv_t}), gam = g / den, eta = gam y and e2 = e^{u+k} / 2^{qv};
 // the state advances past the batch.  Batch fast path when every lane allows
 // it (see fast_prep), else the per-token rescaled recurrence.
+// Returns true (warp-uniform) when the batch ran on the fast path; then M is
+// its reference exponent: qv_j = M + j w2e, and e2 2^{-u2 - w2e} is the
+// factor 2^{K_j - M - (j+1) w2e} with which token j entered the state.
 template <int RB>
-__device__ __forceinline__ void recompute_batch(const float (&K)[RB], const float (&V)[RB],
+__device__ __forceinline__ bool recompute_batch(const float (&K)[RB], const float (&V)[RB],
                                                 const float (&Gy)[RB], float w2, float u2,
                                                 const FastC &fc, float &xa, float &xb, float &xP,
                                                 float &xn, float (&qv)[RB], float (&gam)[RB],
-                                                float (&eta)[RB], float (&e2v)[RB]) {
+                                                float (&eta)[RB], float (&e2v)[RB], float &M) {
   const float E0 = fmaf(xn, w2, xP);
-  float kj[RB], M;
+  float kj[RB];
   const bool ok = fast_prep<RB>(K, E0, u2, fc.w2e, kj, M);
   if (__all_sync(0xffffffffu, ok)) {
     const float s0 = ex2(E0 - M);
@@ -110,7 +113,7 @@ __device__ __forceinline__ void recompute_batch(const float (&K)[RB], const floa
     xb = be;
     xP = M;
     xn = fc.nend;
-    return;
+    return true;
   }
 #pragma unroll
   for (int j = 0; j < RB; ++j) {
@@ -137,6 +140,7 @@ __device__ __forceinline__ void recompute_batch(const float (&K)[RB], const floa
     xP = kw ? K[j] : xP;
     xn = kw ? 0.f : n1;
   }
+  return false;
 }
 
 struct SegBwdArgs {
@@ -309,9 +313,34 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       float K[RB], V[RB], Gy[RB];
       take(K, V, Gy);
       mask_tail(Gy, n - bt * RB);
-      float qv[RB], gam[RB], eta[RB], e2v[RB];
-      recompute_batch<RB>(K, V, Gy, w2, u2, fc, fa, fb, fP, fn, qv, gam, eta, e2v);
+      float qv[RB], gam[RB], eta[RB], e2v[RB], Mb;
+      const bool fast = recompute_batch<RB>(K, V, Gy, w2, u2, fc, fa, fb, fP, fn, qv, gam, eta, e2v, Mb);
       const float lag0 = (float)(bt * RB);
+      if (fast) {
+        // token j's aggregate exponent is lag0 w2 - M + j (w2 - w2e): a batch
+        // constant times (2^{w2 - w2e})^j, so the batch enters as four sums
+        float f = 1.f, sg = 0.f, se = 0.f, sgl = 0.f, sel = 0.f;
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+          const float gf = gam[j] * f, ef = eta[j] * f;
+          sg += gf;
+          se += ef;
+          sgl = fmaf((float)j, gf, sgl);
+          sel = fmaf((float)j, ef, sel);
+          f *= fc.ewm;
+        }
+        const float es = fmaf(lag0, w2, -Mb);
+        const float da = es - Em;
+        const float xa = ex2(-fabsf(da));
+        const bool up = da > 0.f;
+        const float fo = up ? xa : 1.f, fg = up ? 1.f : xa;
+        ah = fmaf(ah, fo, sg * fg);
+        hh = fmaf(hh, fo, se * fg);
+        ahp = fmaf(ahp, fo, fmaf(lag0, sg, sgl) * fg);
+        hhp = fmaf(hhp, fo, fmaf(lag0, se, sel) * fg);
+        Em = up ? es : Em;
+        continue;
+      }
 #pragma unroll
       for (int j = 0; j < RB; ++j) {
         // token s = t0 + lag enters the aggregate with 2^{lag w2 - q_s}
@@ -388,14 +417,49 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       take(K, V, Gy);
       const int nb = n - bt * RB;  // valid tokens of the batch (may be <= 0 or > RB)
       mask_tail(Gy, nb);
-      float qv[RB], gam[RB], eta[RB], e2v[RB];
+      float qv[RB], gam[RB], eta[RB], e2v[RB], Mb;
+      bool fast;
       {
         float xa = sts[bt * 96 + lane], xb = sts[bt * 96 + 32 + lane], xP = sts[bt * 96 + 64 + lane];
         float xn = 0.f;
-        recompute_batch<RB>(K, V, Gy, w2, u2, fc, xa, xb, xP, xn, qv, gam, eta, e2v);
+        fast = recompute_batch<RB>(K, V, Gy, w2, u2, fc, xa, xb, xP, xn, qv, gam, eta, e2v, Mb);
       }
       E *gkp = static_cast<E *>(p.gk) + ((int64_t)b * T + t0 + bt * RB) * C + c;
       E *gvp = static_cast<E *>(p.gv) + ((int64_t)b * T + t0 + bt * RB) * C + c;
+      // Fast sweep: the adjoint in the batch's coordinates, a_t = A_t 2^{M + t w2e},
+      // obeys a_t = gam_t + ewm a_{t+1} (and a'_t = ewm (a'_{t+1} + a_{t+1}) for
+      // the lag-weighted one); e^{k_t} A_{t+1} = ek_t a_{t+1}.  The carried
+      // adjoint enters scaled by 2^{M + RB w2e - r}, bounded for the float range.
+      const float rn_end = fmaf(-m, w2, Ranc);
+      const float xin = fmaf((float)RB, fc.w2e, Mb) - rn_end;
+      if (__all_sync(0xffffffffu, fast && xin < 100.f)) {
+        const float F = ex2(xin);
+        float ra = rah * F, rh = rhh * F, rap = rahp * F, rhp = rhhp * F;
+        const float ck = fc.cw * ex2(-u2);  // ek = e2 * ck
+#pragma unroll
+        for (int j = RB - 1; j >= 0; --j) {
+          const float ek = e2v[j] * ck;
+          const float gv = fmaf(gam[j], e2v[j], ek * ra);
+          const float gk = fmaf(V[j], gv, -fmaf(eta[j], e2v[j], ek * rh));
+          gw_acc = fmaf(ek, fmaf(V[j], rap, -rhp), gw_acc);
+          gu_acc = fmaf(e2v[j], fmaf(gam[j], V[j], -eta[j]), gu_acc);
+          if (cok && j < nb) {
+            IO<E>::st(gkp + (int64_t)j * C, gk);
+            IO<E>::st(gvp + (int64_t)j * C, gv);
+          }
+          rap = fc.ewm * (rap + ra);
+          rhp = fc.ewm * (rhp + rh);
+          ra = fmaf(ra, fc.ewm, gam[j]);
+          rh = fmaf(rh, fc.ewm, eta[j]);
+        }
+        rah = ra;
+        rhh = rh;
+        rahp = rap;
+        rhhp = rhp;
+        Ranc = Mb;
+        m = 0.f;
+        continue;
+      }
 #pragma unroll
       for (int j = RB - 1; j >= 0; --j) {
         const float rn = fmaf(-m, w2, Ranc);  // scale of the adjoint after token t
