@@ -401,7 +401,7 @@ __device__ __forceinline__ void grid_barrier(WsHeader *h, unsigned nblocks, int6
         break;
       }
       __nanosleep(backoff);  // back off: spinning steals issue slots from working warps
-      backoff = backoff < 1024u ? backoff * 2u : 1024u;
+      backoff = backoff < 256u ? backoff * 2u : 256u;
     }
   }
   __syncthreads();

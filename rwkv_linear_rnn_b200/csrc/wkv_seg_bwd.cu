@@ -152,7 +152,7 @@ struct SegBwdArgs {
 };
 
 #ifndef WKV_SEGB_BLOCK
-#define WKV_SEGB_BLOCK 8
+#define WKV_SEGB_BLOCK 4
 #endif
 constexpr int kBwdBlockSeg = WKV_SEGB_BLOCK;  // segments per suffix block (at most one per lane)
 static_assert(kBwdBlockSeg >= 1 && kBwdBlockSeg <= 32, "one lane per record");
@@ -513,10 +513,23 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       const int64_t r0 = grp * R / ng, r1 = (grp + 1) * R / ng;
       double sw = 0.0, su = 0.0;
       if (c < C) {
-        for (int64_t r = r0; r < r1; ++r) {
-          const int64_t ps = r / p.B, bb = r - ps * p.B;
-          sw += (double)__ldcg(p.part + (ps * 2 + 0) * BC + bb * C + c);
-          su += (double)__ldcg(p.part + (ps * 2 + 1) * BC + bb * C + c);
+        // rows in fixed order; eight loads in flight per step
+        for (int64_t r = r0; r < r1; r += 8) {
+          float xw[8], xu[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int64_t rr = min(r + j, r1 - 1);
+            const int64_t ps = rr / p.B, bb = rr - ps * p.B;
+            xw[j] = __ldcg(p.part + (ps * 2 + 0) * BC + bb * C + c);
+            xu[j] = __ldcg(p.part + (ps * 2 + 1) * BC + bb * C + c);
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (r + j < r1) {
+              sw += (double)xw[j];
+              su += (double)xu[j];
+            }
+          }
         }
       }
       double *dst = scratch + (ct * ng + grp) * 64;
@@ -532,9 +545,21 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       if (last) {
         __threadfence();
         double tw = 0.0, tu = 0.0;
-        for (int64_t k = 0; k < ng; ++k) {
-          tw += __ldcg(scratch + (ct * ng + k) * 64 + lane);
-          tu += __ldcg(scratch + (ct * ng + k) * 64 + 32 + lane);
+        for (int64_t k = 0; k < ng; k += 8) {  // group sums in fixed order, eight loads in flight
+          double xw[8], xu[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int64_t kk = min(k + j, ng - 1);
+            xw[j] = __ldcg(scratch + (ct * ng + kk) * 64 + lane);
+            xu[j] = __ldcg(scratch + (ct * ng + kk) * 64 + 32 + lane);
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (k + j < ng) {
+              tw += xw[j];
+              tu += xu[j];
+            }
+          }
         }
         if (c < C) {
           a.gw[c] = (float)tw;
@@ -594,7 +619,7 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
 // Tile parameters (tokens per segment, ring stages, rows per ring item);
 // compile-time tunables.
 #ifndef WKV_SEGB_TS
-#define WKV_SEGB_TS 64
+#define WKV_SEGB_TS 128
 #endif
 #ifndef WKV_SEGB_S_F32
 #define WKV_SEGB_S_F32 3
