@@ -51,7 +51,11 @@ struct SegArgs {
 constexpr int kBlockSeg = WKV_SEGF_BLOCK;  // segments per prefix block (at most one per lane)
 static_assert(kBlockSeg >= 1 && kBlockSeg <= 32, "one lane per record");
 
-template <typename E, int S, int RB>
+// BAR: every warp owns at most one segment and the rows fit in L2; all
+// warps run pass 1, meet at one grid barrier, and fold their predecessors'
+// summaries without polling.  Otherwise segments are joined through
+// per-record flags (decoupled, at most kBlockSeg records per fold).
+template <typename E, int S, int RB, bool BAR>
 __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
                                                       const __grid_constant__ CUtensorMap vmap,
                                                       SegArgs a) {
@@ -134,8 +138,10 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
     }
   };
 
-  for (int i = 0; i < nu; ++i) {
-    const int unit = g + i * G;
+  const int iters = BAR ? 1 : nu;  // with BAR every warp passes the barrier once
+  for (int i = 0; i < iters; ++i) {
+    const bool has = i < nu;
+    const int unit = has ? g + i * G : 0;
     const int pos = unit / nchains, chain = unit - pos * nchains;
     const int b = chain / nct;
     const int64_t c = (int64_t)(chain - b * nct) * 32 + lane;
@@ -149,7 +155,7 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
     // ---- pass 1: segment summary
     St agg = st_empty();
 #pragma unroll 1
-    for (int bt = 0; bt < NBT; ++bt) {
+    for (int bt = 0; bt < (has ? NBT : 0); ++bt) {
       float K[RB], V[RB];
       take(K, V);
       const int nb = max(0, min(RB, n - bt * RB));
@@ -157,6 +163,25 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
       agg = combine(agg, sb, (float)nb, w2);
     }
 
+    St carry;
+    if constexpr (BAR) {
+      // ---- join after the grid barrier: every summary is out; fold the
+      // chain's earlier segments in order
+      if (has && pos + 1 < nseg) desc_store(p.desc, unit, 0, agg, lane);
+      grid_barrier(p.hdr, gridDim.x, budget);
+      if (!has) continue;
+      carry = cok ? load_state_in(p.state_in, bc, BC) : st_empty();
+#pragma unroll 1
+      for (int j0 = 0; j0 < pos; j0 += 8) {
+        St rec[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j0 + j < pos) rec[j] = desc_load<St>(p.desc, (int64_t)(j0 + j) * nchains + chain, 0, lane);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j0 + j < pos) carry = combine(carry, rec[j], (float)TS, w2);
+      }
+    } else {
     // ---- join: fold the earlier records of this chain (fixed order)
     const int q = pos - pos % kBlockSeg;  // first segment of this block
     const int nrec = (pos - q) + (q > 0 ? 1 : 0);
@@ -184,7 +209,7 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
       }
       __syncwarp();
     }
-    St carry = (q == 0 && cok) ? load_state_in(p.state_in, bc, BC) : st_empty();
+    carry = (q == 0 && cok) ? load_state_in(p.state_in, bc, BC) : st_empty();
 #pragma unroll 1
     for (int j0 = 0; j0 < nrec; j0 += 8) {
       St rec[8];
@@ -204,6 +229,7 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
     }
     if (block_end && pos + 1 < nseg && !held)
       publish(p.desc, p.flags, unit, 0, combine(carry, agg, (float)n, w2), epoch, lane);
+    }
 
     // ---- pass 2: replay from the carried-in state
     Run st = run_from(carry);
@@ -259,6 +285,15 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
   finish_block(p.hdr, gridDim.x);
 }
 
+template <typename E, int S, int RB, bool BAR>
+static cudaError_t launch_seg_k(const CUtensorMap &km, const CUtensorMap &vm, SegArgs a, int64_t grid,
+                                int smem, cudaStream_t st) {
+  auto kern = fwd_seg_kernel<E, S, RB, BAR>;
+  CUtensorMap k2 = km, v2 = vm;
+  void *args[] = {&k2, &v2, &a};
+  return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3(128), args, (size_t)smem, st);
+}
+
 template <typename E, int S, int RB>
 static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, int ts_max, cudaStream_t st) {
   CUtensorMap km, vm;
@@ -266,12 +301,15 @@ static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, int ts
     return cudaErrorInvalidValue;
   constexpr int kWarps = 4;
   constexpr int smem = WarpRing<E, S, 2, RB>::block_bytes(kWarps);
-  auto kern = fwd_seg_kernel<E, S, RB>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  int occ = 0;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kWarps * 32, smem)) != cudaSuccess)
-    return e;
+  // the grid is sized for the smaller occupancy of the two join variants
+  int occ = 1 << 30;
+  for (const void *kern : {(const void *)fwd_seg_kernel<E, S, RB, false>, (const void *)fwd_seg_kernel<E, S, RB, true>}) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int o = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, kWarps * 32, smem)) != cudaSuccess) return e;
+    occ = std::min(occ, o);
+  }
   if (occ < 1) return cudaErrorInvalidConfiguration;
   // Segment length: as short as it takes to give every resident warp a
   // segment (more warps hide more latency), but not longer than ts_max (the
@@ -291,9 +329,12 @@ static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, int ts
   const int64_t max_warps = (int64_t)occ * num_sms * kWarps;
   const int64_t rounds = (units + max_warps - 1) / max_warps;
   const int64_t grid = ((units + rounds - 1) / rounds + kWarps - 1) / kWarps;
-  void *args[] = {&km, &vm, &a};
-  return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3(kWarps * 32), args,
-                                     (size_t)smem, st);
+  // Barrier join when every warp has one segment (all first passes run
+  // together anyway) and chains have few segments (each fold reads all of
+  // its predecessors); the test hook needs the flag join.
+  const bool bar = rounds == 1 && a.nseg <= 32 && !f.hold_first;
+  return bar ? launch_seg_k<E, S, RB, true>(km, vm, a, grid, smem, st)
+             : launch_seg_k<E, S, RB, false>(km, vm, a, grid, smem, st);
 }
 
 // Tile parameters per element type (compile-time tunables): the longest
