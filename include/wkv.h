@@ -84,7 +84,7 @@ enum { WKV_OP_FORWARD = 0, WKV_OP_BACKWARD = 1, WKV_OP_STEP = 2 };
 /* Kernel selector (wkv_options.kernel). */
 enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
        WKV_KERNEL_CHUNKED_REGS = 3, WKV_KERNEL_CHAIN = 4, WKV_KERNEL_SPLIT = 5,
-       WKV_KERNEL_SEGMENT = 6 };
+       WKV_KERNEL_SEGMENT = 6, WKV_KERNEL_CLUSTER = 7 };
 
 /*
  * Optional knobs for the *_ex calls.  A NULL options pointer, or all fields
@@ -104,6 +104,10 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
  *               default when rows are 16-byte aligned) gives each warp a
  *               128/256-token segment of one chain: summary, a fixed-order
  *               join with at most 16 earlier records, and the replay from L2.
+ *               CLUSTER (forward only) gives each chain a thread-block
+ *               cluster whose warps take its segments round by round and
+ *               join them through distributed shared memory after a cluster
+ *               barrier (no cross-cluster waits; 16-byte aligned rows).
  *               In the backward, AUTO/SEGMENT select a one-launch segment
  *               kernel (64-token segments in reverse order: recompute and
  *               adjoint aggregate, a fixed-order join with at most 8 later

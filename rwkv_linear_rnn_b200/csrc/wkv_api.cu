@@ -19,6 +19,7 @@ cudaError_t launch_reduce_wu(const float *part, int64_t nchunks, int64_t B, int6
 cudaError_t launch_forward_scan3(const FwdArgs &f, int dtype, float *sums, float *carry,
                                  int num_sms, cudaStream_t st);
 cudaError_t launch_forward_seg(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st);
+cudaError_t launch_forward_clu(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st);
 cudaError_t launch_backward_seg(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
                                 int64_t scratch_doubles, int num_sms, cudaStream_t st);
 cudaError_t launch_backward(const BwdArgs &a, int dtype, float *gw, float *gu, cudaStream_t st);
@@ -104,7 +105,8 @@ bool pick_chunked(const wkv_options *opt, int64_t B, int64_t T, int64_t C) {
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   if (kernel == WKV_KERNEL_SEQUENTIAL) return false;
   if (kernel == WKV_KERNEL_CHUNKED || kernel == WKV_KERNEL_CHUNKED_REGS ||
-      kernel == WKV_KERNEL_CHAIN || kernel == WKV_KERNEL_SPLIT || kernel == WKV_KERNEL_SEGMENT)
+      kernel == WKV_KERNEL_CHAIN || kernel == WKV_KERNEL_SPLIT || kernel == WKV_KERNEL_SEGMENT ||
+      kernel == WKV_KERNEL_CLUSTER)
     return true;
   // Enough independent chains to fill the GPU, or too short to split.
   return !(B * C >= kSeqMinChains || T <= 2 * fwd_chunk_tokens());
@@ -161,6 +163,8 @@ int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
   a.spin_limit = spin_of(opt);
   a.hold_first = opt ? opt->test_hold_first_chunk : 0;
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
+  if (chunked && fwd_tma_eligible(a, dtype) && kernel == WKV_KERNEL_CLUSTER)
+    return launch_forward_clu(a, dtype, num_sms(), st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
   if (chunked && fwd_tma_eligible(a, dtype) &&
       (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT))
     return launch_forward_seg(a, dtype, num_sms(), st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;

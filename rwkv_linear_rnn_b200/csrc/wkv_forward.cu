@@ -436,7 +436,7 @@ bool encode_rows(CUtensorMap *m, const void *ptr, int dtype, int64_t rows, int64
 bool fwd_tma_eligible(const FwdArgs &a, int dtype) {
   const int64_t es = dtype == 0 ? 4 : 2;
   return (a.C * es) % 16 == 0 && ((uintptr_t)a.k % 16) == 0 && ((uintptr_t)a.v % 16) == 0 &&
-         a.B * a.T < (int64_t(1) << 31) && tensor_map_encoder() != nullptr;
+         a.B * a.T + 4096 < (int64_t(1) << 31) && tensor_map_encoder() != nullptr;  // rows past T stay int
 }
 
 template <typename E>

@@ -20,7 +20,8 @@ pytestmark = pytest.mark.gpu
 
 KERNELS = {"seq": W.WKV_KERNEL_SEQUENTIAL, "chunked": W.WKV_KERNEL_CHUNKED,
            "chunked_regs": W.WKV_KERNEL_CHUNKED_REGS, "chain": W.WKV_KERNEL_CHAIN,
-           "split": W.WKV_KERNEL_SPLIT, "segment": W.WKV_KERNEL_SEGMENT}
+           "split": W.WKV_KERNEL_SPLIT, "segment": W.WKV_KERNEL_SEGMENT,
+           "cluster": W.WKV_KERNEL_CLUSTER}
 BWD_KERNELS = {"chain": W.WKV_KERNEL_CHAIN, "chunked": W.WKV_KERNEL_CHUNKED,
                "segment": W.WKV_KERNEL_SEGMENT}
 
@@ -269,10 +270,11 @@ def _range_case(name, seed):
     return w, u, k, v, g
 
 
+@pytest.mark.parametrize("kernel", ["segment", "cluster"])
 @pytest.mark.parametrize("name", sorted(RANGE_CASES))
-def test_segment_forward_ranges(name):
+def test_segment_forward_ranges(name, kernel):
     w, u, k, v, g = _range_case(name, seed=41)
-    y, _, _ = W.forward(dev(w), dev(u), dev(k), dev(v), kernel=W.WKV_KERNEL_SEGMENT)
+    y, _, _ = W.forward(dev(w), dev(u), dev(k), dev(v), kernel=KERNELS[kernel])
     y_ref, _ = oracle.fwd_recur(w, u, k, v)
     assert fwd_err(host(y), y_ref) <= F32_FWD_TOL
 
