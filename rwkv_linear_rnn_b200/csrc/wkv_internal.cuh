@@ -188,6 +188,18 @@ __device__ __forceinline__ S desc_load(const float *desc, int64_t tile, int whic
   return s;
 }
 
+// Lane-major records of the segment kernels: a St record is one float4 per
+// lane (a single 16-byte load per lane, 512 bytes per warp); an adjoint
+// record of five floats adds a fifth plane after it.
+__device__ __forceinline__ void rec_store_st(float *desc, int64_t tile, const St &s, int lane) {
+  float4 *d = reinterpret_cast<float4 *>(desc + tile * kDescFloats) + lane;
+  __stcg(d, make_float4(s.a, s.b, s.P, s.n));
+}
+__device__ __forceinline__ St rec_load_st(const float *desc, int64_t tile, int lane) {
+  const float4 v = __ldcg(reinterpret_cast<const float4 *>(desc + tile * kDescFloats) + lane);
+  return St{v.x, v.y, v.z, v.w};
+}
+
 // A state in four planes of 32 lanes (shared or global memory).
 __device__ __forceinline__ void put_st(float *d, int lane, const St &s) {
   d[lane] = s.a;
@@ -197,6 +209,15 @@ __device__ __forceinline__ void put_st(float *d, int lane, const St &s) {
 }
 __device__ __forceinline__ St get_st(const float *d, int lane) {
   return St{d[lane], d[32 + lane], d[64 + lane], d[96 + lane]};
+}
+
+// Publish a lane-major St record and then its flag (as publish below).
+__device__ __forceinline__ void publish_st(float *desc, unsigned *flags, int64_t tile, const St &s,
+                                          unsigned epoch, int lane) {
+  rec_store_st(desc, tile, s, lane);
+  __syncwarp();
+  if (lane == 0) st_release(flags + tile, (epoch_tag(epoch) << 2) | kAgg);
+  __syncwarp();
 }
 
 // Publish a record and then its flag (all lanes of the warp call this

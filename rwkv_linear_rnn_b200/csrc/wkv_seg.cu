@@ -167,18 +167,18 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
     if constexpr (BAR) {
       // ---- join after the grid barrier: every summary is out; fold the
       // chain's earlier segments in order
-      if (has && pos + 1 < nseg) desc_store(p.desc, unit, 0, agg, lane);
+      if (has && pos + 1 < nseg) rec_store_st(p.desc, unit, agg, lane);
       grid_barrier(p.hdr, gridDim.x, budget);
       if (!has) continue;
       carry = cok ? load_state_in(p.state_in, bc, BC) : st_empty();
 #pragma unroll 1
-      for (int j0 = 0; j0 < pos; j0 += 8) {
-        St rec[8];
+      for (int j0 = 0; j0 < pos; j0 += 12) {  // twelve records in flight per step
+        St rec[12];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j0 + j < pos) rec[j] = desc_load<St>(p.desc, (int64_t)(j0 + j) * nchains + chain, 0, lane);
+        for (int j = 0; j < 12; ++j)
+          if (j0 + j < pos) rec[j] = rec_load_st(p.desc, (int64_t)(j0 + j) * nchains + chain, lane);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 12; ++j)
           if (j0 + j < pos) carry = combine(carry, rec[j], (float)TS, w2);
       }
     } else {
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
     // inclusive prefix below instead; the chain's last segment nothing)
     const bool block_end = (pos % kBlockSeg) == kBlockSeg - 1;
     const bool held = p.hold_first && pos == 0;  // test hook: never publish
-    if (!block_end && pos + 1 < nseg && !held) publish(p.desc, p.flags, unit, 0, agg, epoch, lane);
+    if (!block_end && pos + 1 < nseg && !held) publish_st(p.desc, p.flags, unit, agg, epoch, lane);
     {
       const bool act = lane < nrec;
       const unsigned *fl = p.flags + (int64_t)(rec0 + lane) * nchains + chain;
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
       St rec[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (j0 + j < nrec) rec[j] = desc_load<St>(p.desc, (int64_t)(rec0 + j0 + j) * nchains + chain, 0, lane);
+        if (j0 + j < nrec) rec[j] = rec_load_st(p.desc, (int64_t)(rec0 + j0 + j) * nchains + chain, lane);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j0 + j < nrec) {
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
       }
     }
     if (block_end && pos + 1 < nseg && !held)
-      publish(p.desc, p.flags, unit, 0, combine(carry, agg, (float)n, w2), epoch, lane);
+      publish_st(p.desc, p.flags, unit, combine(carry, agg, (float)n, w2), epoch, lane);
     }
 
     // ---- pass 2: replay from the carried-in state

@@ -59,6 +59,26 @@ struct Adj5s {
 };
 __device__ __forceinline__ Adj5s adj5s_empty() { return Adj5s{0.f, 0.f, 0.f, 0.f, kEmptyR}; }
 
+// Lane-major adjoint records: (ah, hh, ahp, hhp) as one float4 per lane,
+// then r in a plane after them (two loads per lane instead of five).
+__device__ __forceinline__ void rec_store_adj(float *desc, int64_t tile, const Adj5s &s, int lane) {
+  float *d = desc + tile * kDescFloats;
+  __stcg(reinterpret_cast<float4 *>(d) + lane, make_float4(s.ah, s.hh, s.ahp, s.hhp));
+  __stcg(d + 128 + lane, s.r);
+}
+__device__ __forceinline__ Adj5s rec_load_adj(const float *desc, int64_t tile, int lane) {
+  const float *d = desc + tile * kDescFloats;
+  const float4 v = __ldcg(reinterpret_cast<const float4 *>(d) + lane);
+  return Adj5s{v.x, v.y, v.z, v.w, __ldcg(d + 128 + lane)};
+}
+__device__ __forceinline__ void publish_adj(float *desc, unsigned *flags, int64_t tile, const Adj5s &s,
+                                           unsigned epoch, int lane) {
+  rec_store_adj(desc, tile, s, lane);
+  __syncwarp();
+  if (lane == 0) st_release(flags + tile, (epoch_tag(epoch) << 2) | kAgg);
+  __syncwarp();
+}
+
 // X (earlier, lenX tokens) then Y (later): Y's adjoint decays across X by
 // 2^{lenX w2}; its w-derivative gains lenX times Y's adjoint.
 __device__ __forceinline__ Adj5s rjoin(const Adj5s &X, const Adj5s &Y, float lenX, float w2) {
@@ -369,7 +389,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
     Adj5s acc = adj5s_empty();
     if constexpr (BAR) {
       // ---- join after the grid barrier: fold the later segments in order
-      if (has && rpos + 1 < nseg) desc_store(p.desc, unit, 0, agg, lane);
+      if (has && rpos + 1 < nseg) rec_store_adj(p.desc, unit, agg, lane);
       grid_barrier(p.hdr, gridDim.x, budget);
       if (!has) continue;
 #pragma unroll 1
@@ -377,7 +397,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
         Adj5s rec[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          if (j0 + j < rpos) rec[j] = desc_load<Adj5s>(p.desc, (int64_t)(j0 + j) * nchains + chain, 0, lane);
+          if (j0 + j < rpos) rec[j] = rec_load_adj(p.desc, (int64_t)(j0 + j) * nchains + chain, lane);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           if (j0 + j < rpos) acc = rjoin(rec[j], acc, j0 + j == 0 ? (float)nlast : (float)TS, w2);
@@ -389,7 +409,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
     const int rec0 = q > 0 ? q - 1 : q;
     const bool block_end = (rpos % kBwdBlockSeg) == kBwdBlockSeg - 1;
     const bool held = p.hold_first && rpos == 0;  // test hook: never publish
-    if (!block_end && rpos + 1 < nseg && !held) publish(p.desc, p.flags, unit, 0, agg, epoch, lane);
+    if (!block_end && rpos + 1 < nseg && !held) publish_adj(p.desc, p.flags, unit, agg, epoch, lane);
     {
       const bool act = lane < nrec;
       const unsigned *fl = p.flags + (int64_t)(rec0 + lane) * nchains + chain;
@@ -413,7 +433,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       Adj5s rec[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (j0 + j < nrec) rec[j] = desc_load<Adj5s>(p.desc, (int64_t)(rec0 + j0 + j) * nchains + chain, 0, lane);
+        if (j0 + j < nrec) rec[j] = rec_load_adj(p.desc, (int64_t)(rec0 + j0 + j) * nchains + chain, lane);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j0 + j < nrec) {
@@ -426,7 +446,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       }
     }
     if (block_end && rpos + 1 < nseg && !held)
-      publish(p.desc, p.flags, unit, 0, rjoin(agg, acc, (float)n, w2), epoch, lane);
+      publish_adj(p.desc, p.flags, unit, rjoin(agg, acc, (float)n, w2), epoch, lane);
     }
 
     // ---- pass 2: batches last to first, recompute then reverse sweep
