@@ -44,17 +44,16 @@ ALG_BYTES = {("fwd", "f32"): 12, ("fwd", "bf16"): 6, ("bwd", "f32"): 20, ("bwd",
 # Kernels each call launches on 16-byte aligned rows (all bench workloads),
 # per kernel selector: (kernel names, launches per call).
 FWD_PLAN = {"auto": ("fwd_seg_kernel", 1), "segment": ("fwd_seg_kernel", 1),
-            "chain": ("fwd_chain_kernel", 1)}
+            "cluster": ("fwd_clu_kernel", 1)}
 BWD_PLAN = {"auto": ("bwd_seg_kernel", 1),
-            "chain": ("bwd_chain_kernel + reduce_wu_kernel", 2),
             "segment": ("bwd_seg_kernel", 1)}
-KERNEL_IDS = {"auto": 0, "chain": 4, "segment": 6}
+KERNEL_IDS = {"auto": 0, "segment": 6, "cluster": 7}
 
 # DRAM bytes (read + write) per launch of the backward's main kernel from one
 # ncu capture of this bench's workload (cold L2; gk/gv lines still dirty in
 # L2 at kernel end are not counted).  Keyed by (workload, kernel); a kernel
 # changed since its capture has no entry (traffic reported as null).
-TRAFFIC = {("rwkv169m", "bwd_chain_kernel"): 76_723_968 + 10_438_144}
+TRAFFIC = {}
 
 
 def peaks():

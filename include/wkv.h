@@ -83,7 +83,7 @@ enum { WKV_OP_FORWARD = 0, WKV_OP_BACKWARD = 1, WKV_OP_STEP = 2 };
 
 /* Kernel selector (wkv_options.kernel). */
 enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
-       WKV_KERNEL_CHUNKED_REGS = 3, WKV_KERNEL_CHAIN = 4, WKV_KERNEL_SPLIT = 5,
+       WKV_KERNEL_CHUNKED_REGS = 3, /* 4 and 5 are retired */
        WKV_KERNEL_SEGMENT = 6, WKV_KERNEL_CLUSTER = 7 };
 
 /*
@@ -93,28 +93,23 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
  *   kernel      WKV_KERNEL_AUTO picks by problem shape; SEQUENTIAL runs one
  *               thread per (b, c) chain over all of T; CHUNKED splits T into
  *               64-token chunks joined by a single-pass scan over published
- *               chunk summaries (TMA-fed shared-memory pipeline when rows are
- *               16-byte aligned); CHUNKED_REGS forces the register-tile
- *               variant of the chunked kernel (no TMA); CHAIN runs one block
- *               per (batch row, 32-channel) chain over all of T, tiles fed
- *               by TMA, the carry kept on chip (needs 16-byte aligned rows;
- *               needs 16-byte aligned rows).  SPLIT runs three launches: chunk
- *               summaries, a per-chain prefix over them, and a replay of
- *               every chunk from its start state.  SEGMENT (the forward
- *               default when rows are 16-byte aligned) gives each warp a
- *               128/256-token segment of one chain: summary, a fixed-order
- *               join with at most 16 earlier records, and the replay from L2.
- *               CLUSTER (forward only) gives each chain a thread-block
- *               cluster whose warps take its segments round by round and
- *               join them through distributed shared memory after a cluster
- *               barrier (no cross-cluster waits; 16-byte aligned rows).
- *               In the backward, AUTO/SEGMENT select a one-launch segment
- *               kernel (64-token segments in reverse order: recompute and
- *               adjoint aggregate, a fixed-order join with at most 8 later
- *               records, then the reverse sweep from L2; dL/dw and dL/du
- *               reduced in the same launch after a grid barrier) and CHAIN
- *               the chain kernel; both need 16-byte aligned rows, otherwise
- *               and for any other value the chunked kernel runs.
+ *               chunk summaries (TMA-fed when rows are 16-byte aligned);
+ *               CHUNKED_REGS forces its register-tile variant (no TMA).
+ *               SEGMENT (the default when rows are 16-byte aligned) gives
+ *               each warp one segment of one chain at a time, its length
+ *               chosen per launch: a first pass (summary; in the backward the
+ *               forward recompute and the adjoint aggregate), a fixed-order
+ *               join with the chain's other segments (through per-record
+ *               flags, or after one grid barrier when every warp holds a
+ *               single segment), and a second pass from L2 (replay; in the
+ *               backward the reverse sweep), the backward reducing dL/dw and
+ *               dL/du in the same launch.  CLUSTER (forward only) gives each
+ *               chain a thread-block cluster whose warps take its segments
+ *               round by round and join them through distributed shared
+ *               memory.  The backward runs the segment kernel for AUTO and
+ *               SEGMENT on 16-byte aligned rows and the chunked kernel
+ *               otherwise.  Values 4 and 5 are retired and rejected with
+ *               WKV_ERR_INVALID_ARG.
  *   spin_limit  bound on any one device-side wait (a predecessor's record,
  *               a shared-memory load, the grid barrier) in microseconds (the
  *               chunked kernels count polls of at most about 1 us each);
@@ -147,8 +142,8 @@ size_t wkv_workspace_size(int op, int64_t B, int64_t T, int64_t C, int dtype);
 int wkv_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /*
- * Bytes of the forward checkpoint buffer: the state at every 64th token,
- * float32 [ceil(T/64)][3][B][C].  Its contents are private to the library
+ * Bytes of the forward checkpoint buffer: the state at every 32nd token,
+ * float32 [ceil(T/32)][3][B][C].  Its contents are private to the library
  * (the exponent is stored in base 2); it only carries the forward's
  * per-chunk states to wkv_backward so the backward does not rescan.
  */

@@ -12,12 +12,8 @@
 namespace wkv {
 cudaError_t launch_forward(const FwdArgs &a, int dtype, int kind, int num_sms, cudaStream_t st);
 bool fwd_tma_eligible(const FwdArgs &a, int dtype);
-cudaError_t launch_forward_chain(const FwdArgs &a, int dtype, cudaStream_t st);
-cudaError_t launch_backward_chain(const BwdArgs &a, int dtype, cudaStream_t st);
 cudaError_t launch_reduce_wu(const float *part, int64_t nchunks, int64_t B, int64_t C, float *gw,
                              float *gu, cudaStream_t st);
-cudaError_t launch_forward_scan3(const FwdArgs &f, int dtype, float *sums, float *carry,
-                                 int num_sms, cudaStream_t st);
 cudaError_t launch_forward_seg(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st);
 cudaError_t launch_forward_clu(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st);
 cudaError_t launch_backward_seg(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
@@ -57,7 +53,7 @@ bool sizes_ok(int64_t B, int64_t T, int64_t C) {
 }
 
 struct Layout {
-  size_t flags, desc, sums, carry, ckpt, part, cnt, total;
+  size_t flags, desc, desc_bytes, ckpt, part, cnt, total;
   int64_t nct, nchains, nchunks_f, nchunks_b;
 };
 
@@ -75,13 +71,8 @@ Layout layout(int op, int64_t B, int64_t T, int64_t C) {
   L.flags = off;
   off = align_up(off + sizeof(unsigned) * (size_t)tiles, 256);
   L.desc = off;
-  off = align_up(off + sizeof(float) * kDescFloats * (size_t)tiles, 256);
-  // split forward: chunk summaries (4 planes x 32 lanes per chain and chunk)
-  // and chunk start states (used when the caller passes no checkpoint buffer)
-  L.sums = off;
-  off = align_up(off + sizeof(float) * 4 * 32 * (size_t)L.nchains * (size_t)L.nchunks_b, 256);
-  L.carry = off;
-  off = align_up(off + sizeof(float) * 3 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
+  L.desc_bytes = sizeof(float) * kDescFloats * (size_t)tiles;
+  off = align_up(off + L.desc_bytes, 256);
   L.ckpt = L.part = L.cnt = 0;
   if (op == WKV_OP_BACKWARD) {
     L.ckpt = off;
@@ -104,12 +95,18 @@ int num_sms() {
 bool pick_chunked(const wkv_options *opt, int64_t B, int64_t T, int64_t C) {
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   if (kernel == WKV_KERNEL_SEQUENTIAL) return false;
-  if (kernel == WKV_KERNEL_CHUNKED || kernel == WKV_KERNEL_CHUNKED_REGS ||
-      kernel == WKV_KERNEL_CHAIN || kernel == WKV_KERNEL_SPLIT || kernel == WKV_KERNEL_SEGMENT ||
+  if (kernel == WKV_KERNEL_CHUNKED || kernel == WKV_KERNEL_CHUNKED_REGS || kernel == WKV_KERNEL_SEGMENT ||
       kernel == WKV_KERNEL_CLUSTER)
     return true;
   // Enough independent chains to fill the GPU, or too short to split.
   return !(B * C >= kSeqMinChains || T <= 2 * fwd_chunk_tokens());
+}
+
+bool options_ok(const wkv_options *opt) {
+  if (!opt) return true;
+  const int k = opt->kernel;
+  return k == WKV_KERNEL_AUTO || k == WKV_KERNEL_SEQUENTIAL || k == WKV_KERNEL_CHUNKED ||
+         k == WKV_KERNEL_CHUNKED_REGS || k == WKV_KERNEL_SEGMENT || k == WKV_KERNEL_CLUSTER;
 }
 
 int64_t spin_of(const wkv_options *opt) {
@@ -168,15 +165,6 @@ int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
   if (chunked && fwd_tma_eligible(a, dtype) &&
       (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT))
     return launch_forward_seg(a, dtype, num_sms(), st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
-  if (chunked && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SPLIT)) {
-    float *sums = reinterpret_cast<float *>(base + L.sums);
-    float *carry = ckpt ? ckpt : reinterpret_cast<float *>(base + L.carry);
-    return launch_forward_scan3(a, dtype, sums, carry, num_sms(), st) == cudaSuccess
-               ? WKV_OK
-               : WKV_ERR_CUDA;
-  }
-  if (chunked && fwd_tma_eligible(a, dtype) && kernel == WKV_KERNEL_CHAIN)
-    return launch_forward_chain(a, dtype, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
   int kind = 0;
   if (chunked) kind = (fwd_tma_eligible(a, dtype) && kernel != WKV_KERNEL_CHUNKED_REGS) ? 2 : 1;
   return launch_forward(a, dtype, kind, num_sms(), st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
@@ -211,6 +199,7 @@ int wkv_forward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, c
   int rc = check_forward_args(B, T, C, dtype, w, u, k, v, state_in, y, state_out, ckpt);
   if (rc != WKV_OK) return rc;
   if (T > 0 && !y) return WKV_ERR_INVALID_ARG;
+  if (!options_ok(opt)) return WKV_ERR_INVALID_ARG;
   return forward_impl(B, T, C, dtype, w, u, k, v, state_in, y, state_out, ckpt, ws, ws_bytes,
                       (cudaStream_t)stream, opt);
 }
@@ -228,6 +217,7 @@ int wkv_backward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, 
                     void *ws, size_t ws_bytes, void *stream, const wkv_options *opt) {
   int rc = check_forward_args(B, T, C, dtype, w, u, k, v, state_in, nullptr, nullptr, ckpt);
   if (rc != WKV_OK) return rc;
+  if (!options_ok(opt)) return WKV_ERR_INVALID_ARG;
   if (!grad_w || !grad_u) return WKV_ERR_INVALID_ARG;
   if (T > 0 && (!grad_y || !grad_k || !grad_v)) return WKV_ERR_INVALID_ARG;
   const size_t es = esize(dtype);
@@ -275,15 +265,11 @@ int wkv_backward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, 
   probe.B = B; probe.T = T; probe.C = C; probe.k = k; probe.v = v;
   const bool tma_ok = fwd_tma_eligible(probe, dtype) && ((uintptr_t)grad_y % 16) == 0;
   if (tma_ok && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT)) {
-    const int64_t scratch = (int64_t)((L.sums - L.desc) / sizeof(double));
+    const int64_t scratch = (int64_t)(L.desc_bytes / sizeof(double));
     return launch_backward_seg(a, dtype, grad_w, grad_u, reinterpret_cast<unsigned *>(base + L.cnt), scratch,
                                num_sms(), st) == cudaSuccess
                ? WKV_OK
                : WKV_ERR_CUDA;
-  }
-  if (tma_ok && kernel == WKV_KERNEL_CHAIN) {
-    if (launch_backward_chain(a, dtype, st) != cudaSuccess) return WKV_ERR_CUDA;
-    return launch_reduce_wu(a.part, 1, B, C, grad_w, grad_u, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
   }
   return launch_backward(a, dtype, grad_w, grad_u, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }

@@ -45,7 +45,7 @@ namespace wkv {
 template <typename E, int W, int L>
 __global__ void __launch_bounds__(W * 32) bwd_chunked_kernel(BwdArgs p) {
   constexpr int TC = W * L;
-  static_assert(TC == kCkpt, "backward chunk must equal the checkpoint interval");
+  static_assert(TC % kCkpt == 0, "backward chunks start on checkpoints");
   __shared__ unsigned s_tile, s_epoch;
   __shared__ float s_f[W][128];      // forward summaries, then warp start states (St planes)
   __shared__ float s_adj[W][3][32];  // adjoint aggregates, then later-warp suffixes
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(W * 32) bwd_chunked_kernel(BwdArgs p) {
   if (wi == 0) {
     St acc = st_empty();
     if (cok) {
-      const float *ck = p.ckpt + chunk * 3 * BC + b * C + c;
+      const float *ck = p.ckpt + chunk * (TC / kCkpt) * 3 * BC + b * C + c;
       acc = St{ck[0], ck[BC], ck[2 * BC]};
     }
 #pragma unroll
@@ -308,7 +308,9 @@ cudaError_t launch_reduce_wu(const float *part, int64_t nchunks, int64_t B, int6
   return cudaGetLastError();
 }
 
-cudaError_t launch_backward(const BwdArgs &a, int dtype, float *gw, float *gu, cudaStream_t st) {
+cudaError_t launch_backward(const BwdArgs &a0, int dtype, float *gw, float *gu, cudaStream_t st) {
+  BwdArgs a = a0;
+  a.nchunks = (a.T + kBwdW * kBwdL - 1) / (kBwdW * kBwdL);  // this kernel's chunks, not checkpoints
   return dtype == 0 ? launch_bwd_t<float>(a, gw, gu, st) : launch_bwd_t<uint16_t>(a, gw, gu, st);
 }
 

@@ -32,7 +32,6 @@
 #include "wkv_internal.cuh"
 #include "wkv_math.cuh"
 #include "wkv_ring.cuh"
-#include "wkv_split.cuh"
 
 namespace cg = cooperative_groups;
 

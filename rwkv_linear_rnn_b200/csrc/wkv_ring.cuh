@@ -1,10 +1,9 @@
-// wkv_ring.cuh -- per-warp TMA ring of 16-row batches (internal).
+// wkv_ring.cuh -- per-warp TMA ring of row batches (internal).
 #pragma once
 
 #include <cuda.h>
 
 #include "wkv_internal.cuh"
-#include "wkv_split.cuh"
 
 namespace wkv {
 
@@ -13,7 +12,7 @@ namespace wkv {
 // destination is 128-byte aligned as tensor copies require), then all the
 // mbarriers (8 bytes each).  A stage holds ROWS rows of 32 channels of each
 // of the NARR tensors.
-template <typename E, int S, int NARR = 2, int ROWS = kS3Batch>
+template <typename E, int S, int NARR, int ROWS>
 struct WarpRing {
   static constexpr int ARR_BYTES = ROWS * 32 * (int)sizeof(E);
   static constexpr int STAGE_BYTES = NARR * ARR_BYTES;
@@ -22,7 +21,7 @@ struct WarpRing {
   static constexpr int block_bytes(int nw) { return nw * (RING_BYTES + S * 8); }
 };
 
-template <typename E, int S, int NARR = 2, int ROWS = kS3Batch>
+template <typename E, int S, int NARR, int ROWS>
 struct Ring {
   using L = WarpRing<E, S, NARR, ROWS>;
   unsigned char *base;

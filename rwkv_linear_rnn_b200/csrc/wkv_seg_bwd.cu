@@ -45,7 +45,6 @@
 #include "wkv_internal.cuh"
 #include "wkv_math.cuh"
 #include "wkv_ring.cuh"
-#include "wkv_split.cuh"
 
 namespace wkv {
 
@@ -169,6 +168,8 @@ struct SegBwdArgs {
   unsigned *tile_cnt;  // [nct] group counters of the final reduction
   int64_t nseg;        // segments per chain
   int64_t ngroups;     // row groups per channel tile in the final reduction
+  int ts;              // tokens per segment (a multiple of the checkpoint interval)
+  int nb;              // batches per segment (ts / rows per batch)
 };
 
 #ifndef WKV_SEGB_BLOCK
@@ -189,34 +190,32 @@ __device__ __forceinline__ int64_t qdiv(int64_t a, int64_t b) {
 // Shared memory of a block of NW warps: the warp rings (with their
 // mbarriers), then per warp the forward state at each batch start of the
 // current segment: [NB][3][32] floats (a, b, exponent).
-template <typename E, int TS, int S, int RB>
+template <typename E, int S, int RB>
 struct SegBwdSmem {
   using RingL = WarpRing<E, S, 3, RB>;
-  static constexpr int NB = TS / RB;
-  static constexpr int STATE_FLOATS = NB * 3 * 32;
   static constexpr int ring_bytes(int nw) { return (RingL::block_bytes(nw) + 15) / 16 * 16; }
-  static constexpr int bytes(int nw) { return ring_bytes(nw) + nw * STATE_FLOATS * 4; }
+  static constexpr int bytes(int nw, int nb) { return ring_bytes(nw) + nw * nb * 96 * 4; }
 };
 
 // BAR: every warp owns at most one segment; all warps run pass 1, meet at a
 // grid barrier and fold the later segments' aggregates without polling.
 // Otherwise segments are joined through per-record flags.
-template <typename E, int TS, int S, int RB, bool BAR>
+template <typename E, int S, int RB, bool BAR>
 __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
                                                       const __grid_constant__ CUtensorMap vmap,
                                                       const __grid_constant__ CUtensorMap gmap,
                                                       SegBwdArgs a) {
-  using Sm = SegBwdSmem<E, TS, S, RB>;
-  constexpr int NB = Sm::NB;   // ring items (batches of RB tokens) per pass
-  constexpr int IPU = 2 * NB;  // ring items per segment
-  static_assert(TS % kCkpt == 0, "segments start on checkpoints");
+  using Sm = SegBwdSmem<E, S, RB>;
+  const int TS = a.ts;         // tokens per segment (segments start on checkpoints)
+  const int NB = a.nb;         // ring items (batches of RB tokens) per pass
+  const int IPU = 2 * NB;      // ring items per segment
   const BwdArgs &p = a.p;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = (int)(blockDim.x >> 5);
   Ring<E, S, 3, RB> ring(smem, wl, nw);
   ring.init(lane);
-  float *sts = reinterpret_cast<float *>(smem + Sm::ring_bytes(nw)) + wl * Sm::STATE_FLOATS;
+  float *sts = reinterpret_cast<float *>(smem + Sm::ring_bytes(nw)) + wl * NB * 96;
   const CUtensorMap *const maps[3] = {&kmap, &vmap, &gmap};
   // The reduction counters are cleared here; the grid barrier orders these
   // stores before every increment (a workspace reused for another shape may
@@ -614,39 +613,65 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
   finish_block(p.hdr, gridDim.x);
 }
 
-template <typename E, int TS, int S, int RB>
+template <typename E, int S, int RB>
 static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
-                                    int64_t scratch_doubles, int num_sms, cudaStream_t st) {
+                                    int64_t scratch_doubles, int num_sms, int ts_max, cudaStream_t st) {
   CUtensorMap km, vm, gm;
   if (!encode_rows(&km, p.k, dtype, p.B * p.T, p.C, RB) || !encode_rows(&vm, p.v, dtype, p.B * p.T, p.C, RB) ||
       !encode_rows(&gm, p.gy, dtype, p.B * p.T, p.C, RB))
     return cudaErrorInvalidValue;
   constexpr int kWarps = 4;
-  constexpr int smem = SegBwdSmem<E, TS, S, RB>::bytes(kWarps);
-  // the grid is sized for the smaller occupancy of the two join variants
-  int occ = 1 << 30;
-  for (const void *kern : {(const void *)bwd_seg_kernel<E, TS, S, RB, false>,
-                           (const void *)bwd_seg_kernel<E, TS, S, RB, true>}) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static_assert(kCkpt % RB == 0, "checkpoints fall on batch starts");
+  // Resident warps for a segment length (the per-warp batch states in shared
+  // memory grow with it); the smaller occupancy of the two join variants.
+  auto max_warps_for = [&](int ts, int &smem, int64_t &mw) -> cudaError_t {
+    smem = SegBwdSmem<E, S, RB>::bytes(kWarps, ts / RB);
+    int occ = 1 << 30;
+    for (const void *kern : {(const void *)bwd_seg_kernel<E, S, RB, false>,
+                             (const void *)bwd_seg_kernel<E, S, RB, true>}) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      int o = 0;
+      if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, kWarps * 32, smem)) != cudaSuccess) return e;
+      occ = std::min(occ, o);
+    }
+    mw = (int64_t)occ * num_sms * kWarps;
+    return occ < 1 ? cudaErrorInvalidConfiguration : cudaSuccess;
+  };
+  // Segment length: the shortest multiple of the checkpoint interval (>= 64)
+  // that lets every segment have its own resident warp (barrier join, most
+  // warps); otherwise the longest (fewest joins per token).
+  int ts = ts_max, smem = 0;
+  int64_t max_warps = 0;
+  bool fits = false;
+  for (int cand = 2 * kCkpt; cand <= ts_max; cand += kCkpt) {
+    int sm = 0;
+    int64_t mw = 0;
+    cudaError_t e = max_warps_for(cand, sm, mw);
     if (e != cudaSuccess) return e;
-    int o = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, kWarps * 32, smem)) != cudaSuccess) return e;
-    occ = std::min(occ, o);
+    if ((p.T + cand - 1) / cand * p.nchains <= mw) {
+      ts = cand, smem = sm, max_warps = mw, fits = true;
+      break;
+    }
   }
-  if (occ < 1) return cudaErrorInvalidConfiguration;
+  if (!fits) {
+    cudaError_t e = max_warps_for(ts, smem, max_warps);
+    if (e != cudaSuccess) return e;
+  }
   SegBwdArgs a{};
   a.p = p;
   a.gw = gw;
   a.gu = gu;
   a.tile_cnt = tile_cnt;
-  a.nseg = (p.T + TS - 1) / TS;
+  a.ts = ts;
+  a.nb = ts / RB;
+  a.nseg = (p.T + ts - 1) / ts;
   const int64_t units = a.nseg * p.nchains;
   if (units >= (int64_t)1 << 31) return cudaErrorInvalidValue;  // unit indices are 31-bit
   // One resident wave (cooperative launch: every warp a segment may wait on,
   // and every block of the grid barrier, is running).  Warps take segments
   // round-robin; the grid is trimmed so that every warp gets the same number
   // of segments (no final round with most warps idle).
-  const int64_t max_warps = (int64_t)occ * num_sms * kWarps;
   const int64_t rounds = (units + max_warps - 1) / max_warps;
   const int64_t want = (units + rounds - 1) / rounds;
   const int64_t grid = (want + kWarps - 1) / kWarps;
@@ -661,14 +686,14 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
   // together anyway) and chains have few segments (each fold reads all the
   // later ones); the test hook needs the flag join.
   const bool bar = rounds == 1 && a.nseg <= 32 && !p.hold_first;
-  const void *kern = bar ? (const void *)bwd_seg_kernel<E, TS, S, RB, true>
-                         : (const void *)bwd_seg_kernel<E, TS, S, RB, false>;
+  const void *kern = bar ? (const void *)bwd_seg_kernel<E, S, RB, true>
+                         : (const void *)bwd_seg_kernel<E, S, RB, false>;
   void *args[] = {&km, &vm, &gm, &a};
   return cudaLaunchCooperativeKernel(kern, dim3((unsigned)grid), dim3(kWarps * 32), args, (size_t)smem, st);
 }
 
-// Tile parameters (tokens per segment, ring stages, rows per ring item);
-// compile-time tunables.
+// Tile parameters (compile-time tunables): the longest segment (tokens),
+// ring stages, rows per ring item.
 #ifndef WKV_SEGB_TS
 #define WKV_SEGB_TS 128
 #endif
@@ -684,10 +709,10 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
 
 cudaError_t launch_backward_seg(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
                                 int64_t scratch_doubles, int num_sms, cudaStream_t st) {
-  return dtype == 0 ? launch_bwd_seg_t<float, WKV_SEGB_TS, WKV_SEGB_S_F32, WKV_SEGB_RB>(
-                          p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, st)
-                    : launch_bwd_seg_t<uint16_t, WKV_SEGB_TS, WKV_SEGB_S_BF16, WKV_SEGB_RB>(
-                          p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, st);
+  return dtype == 0 ? launch_bwd_seg_t<float, WKV_SEGB_S_F32, WKV_SEGB_RB>(p, dtype, gw, gu, tile_cnt,
+                                                                            scratch_doubles, num_sms, WKV_SEGB_TS, st)
+                    : launch_bwd_seg_t<uint16_t, WKV_SEGB_S_BF16, WKV_SEGB_RB>(p, dtype, gw, gu, tile_cnt,
+                                                                               scratch_doubles, num_sms, WKV_SEGB_TS, st);
 }
 
 }  // namespace wkv

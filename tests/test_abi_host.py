@@ -49,7 +49,7 @@ def test_version_and_strerror(W):
 
 def test_sizes(W):
     B, T, C = 8, 1024, 768
-    assert W.wkv_ckpt_size(B, T, C) == 4 * 3 * B * C * 16
+    assert W.wkv_ckpt_size(B, T, C) == 4 * 3 * B * C * (T // 32)  # a checkpoint every 32 tokens
     assert W.wkv_workspace_size(W.WKV_OP_STEP, B, T, C, 0) == 0
     f = W.wkv_workspace_size(W.WKV_OP_FORWARD, B, T, C, 0)
     b = W.wkv_workspace_size(W.WKV_OP_BACKWARD, B, T, C, 0)
@@ -88,6 +88,18 @@ def test_forward_chunked_needs_workspace(W):
     assert W.abi.wkv_forward_ex(*base, 0, 0, 0, opt) == -3             # NULL ws
     assert W.abi.wkv_forward_ex(*base, FAKE * 8, 256, 0, opt) == -3    # too small
     assert W.abi.wkv_forward_ex(*base, FAKE * 8 + 16, 1 << 30, 0, opt) == -3  # misaligned
+
+
+@pytest.mark.parametrize("kernel", [4, 5, 8, -1])
+def test_retired_and_unknown_kernel_selectors_are_rejected(W, kernel):
+    """Selector values 4 and 5 are retired; unknown values are rejected too,
+    before anything is launched."""
+    opt = W.abi.Options(kernel=kernel)
+    fwd = (1, 64, 32, 0, FAKE, FAKE, FAKE, FAKE * 2, 0, FAKE * 4, 0, 0, FAKE * 8, 1 << 30, 0)
+    assert W.abi.wkv_forward_ex(*fwd, opt) == -1
+    bwd = (1, 64, 32, 0, FAKE, FAKE, FAKE, FAKE * 2, FAKE * 3, 0, 0, FAKE * 4, FAKE * 5,
+           FAKE * 6, FAKE * 7, FAKE * 8, 1 << 30, 0)
+    assert W.abi.wkv_backward_ex(*bwd, opt) == -1
 
 
 def test_backward_validation(W):

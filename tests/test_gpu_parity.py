@@ -19,11 +19,9 @@ from gpu_util import (BF16_TOL, F32_FWD_TOL, F32_GRAD_TOL, channel_subset, dev, 
 pytestmark = pytest.mark.gpu
 
 KERNELS = {"seq": W.WKV_KERNEL_SEQUENTIAL, "chunked": W.WKV_KERNEL_CHUNKED,
-           "chunked_regs": W.WKV_KERNEL_CHUNKED_REGS, "chain": W.WKV_KERNEL_CHAIN,
-           "split": W.WKV_KERNEL_SPLIT, "segment": W.WKV_KERNEL_SEGMENT,
+           "chunked_regs": W.WKV_KERNEL_CHUNKED_REGS, "segment": W.WKV_KERNEL_SEGMENT,
            "cluster": W.WKV_KERNEL_CLUSTER}
-BWD_KERNELS = {"chain": W.WKV_KERNEL_CHAIN, "chunked": W.WKV_KERNEL_CHUNKED,
-               "segment": W.WKV_KERNEL_SEGMENT}
+BWD_KERNELS = {"chunked": W.WKV_KERNEL_CHUNKED, "segment": W.WKV_KERNEL_SEGMENT}
 
 
 def small_case(B, T, C, seed, dtype="f32", td=(-3.0, 1.0), kstd=1.0, state=False):
