@@ -121,8 +121,7 @@ __device__ __forceinline__ bool recompute_batch(const float (&K)[RB], const floa
       const float eu = e0 * fc.cu, ek = e0 * fc.cw;
       const float rden = rcp(be + eu);
       const float y = fmaf(eu, V[j], al) * rden;
-      qv[j] = fmaf((float)j, fc.w2e, M);
-      gam[j] = Gy[j] * rden;
+      gam[j] = Gy[j] * rden;  // qv is formed by the caller if it needs it: M + j w2e
       eta[j] = gam[j] * y;
       e2v[j] = eu;
       al = fmaf(al, fc.ewm, ek * V[j]);
@@ -477,6 +476,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
         const float F = ex2(xin);
         float ra = rah * F, rh = rhh * F, rap = rahp * F, rhp = rhhp * F;
         const float ck = fc.cw * ex2(-u2);  // ek = e2 * ck
+        const int jmax = cok ? min(nb, RB) : 0;  // tokens to store (all of a full batch)
 #pragma unroll
         for (int j = RB - 1; j >= 0; --j) {
           const float ek = e2v[j] * ck;
@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
           const float gk = fmaf(V[j], gv, -fmaf(eta[j], e2v[j], ek * rh));
           gw_acc = fmaf(ek, fmaf(V[j], rap, -rhp), gw_acc);
           gu_acc = fmaf(e2v[j], fmaf(gam[j], V[j], -eta[j]), gu_acc);
-          if (cok && j < nb) {
+          if (j < jmax) {
             IO<E>::st(gkp + (int64_t)j * C, gk);
             IO<E>::st(gvp + (int64_t)j * C, gv);
           }
@@ -500,6 +500,10 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
         Ranc = Mb;
         m = 0.f;
         continue;
+      }
+      if (fast) {  // the fast recompute leaves the scales implicit: D_t = den 2^{M + j w2e}
+#pragma unroll
+        for (int j = 0; j < RB; ++j) qv[j] = fmaf((float)j, fc.w2e, Mb);
       }
 #pragma unroll
       for (int j = RB - 1; j >= 0; --j) {
