@@ -80,7 +80,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -89,9 +89,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
-    def stop(self):
+    def stop(self, window=None):
+        """Summary of the samples that arrived inside `window` (monotonic
+        start, end of the timed region); all samples if none did."""
         if not self.proc:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -101,7 +103,11 @@ class ClockSampler:
             self.proc.kill()
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        inside = [ln for t, ln in self.lines if window and window[0] <= t <= window[1]]
+        scope = "timed region"
+        if not inside:
+            inside, scope = [ln for _, ln in self.lines], "whole sampler run (no sample inside the timed region)"
+        for ln in inside:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -115,7 +121,7 @@ class ClockSampler:
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "scope": scope}
 
 
 def dist_env():
@@ -263,7 +269,8 @@ def run_libwkv(args):
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.3)  # nvidia-smi is sampling before the timed region starts
+    t_begin = time.monotonic()
     for i in range(K):
         flush_l2()
         ev[i][0].record(stream)
@@ -272,7 +279,7 @@ def run_libwkv(args):
         bwd()
         ev[i][2].record(stream)
     torch.cuda.synchronize()
-    clocks = sampler.stop()
+    clocks = sampler.stop(window=(t_begin, time.monotonic()))
     if dist:
         dist.barrier()
     t_fwd = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
@@ -357,7 +364,7 @@ def run_libwkv(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=1000)  # about a second: clock samples land inside
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="libwkv", choices=["libwkv", "reference"])
     ap.add_argument("--workload", default="rwkv169m")
