@@ -41,26 +41,6 @@ struct Ring {
     }
     __syncwarp();
   }
-  // Loads of batch `item` (rows y .. y+ROWS-1, columns x .. x+31 of each of the
-  // NARR tensors) into stage item % S.  Returns false, issuing nothing, if a
-  // destination is not 128-byte aligned (the caller's bounded wait then
-  // fails and reports the error).
-  __device__ __forceinline__ bool issue(const CUtensorMap *const (&maps)[NARR], int64_t item, int x,
-                                       int y) const {
-    const int s = (int)(item % S);
-    uint32_t d[NARR];
-    uint32_t bad = 0;
-#pragma unroll
-    for (int a = 0; a < NARR; ++a) {
-      d[a] = smem_addr(stage(s, a));
-      bad |= d[a] & 127u;
-    }
-    if (bad) return false;
-    mbar_expect_tx(bar(s), (uint32_t)L::STAGE_BYTES);
-#pragma unroll
-    for (int a = 0; a < NARR; ++a) tma_load_2d(d[a], maps[a], x, y, bar(s));
-    return true;
-  }
   // True when every stage of this warp's ring is 128-byte aligned (checked
   // once; issue_stage then skips the per-copy check).
   __device__ __forceinline__ bool aligned() const {
@@ -76,23 +56,6 @@ struct Ring {
     mbar_expect_tx(bar(s), (uint32_t)L::STAGE_BYTES);
 #pragma unroll
     for (int a = 0; a < NARR; ++a) tma_load_2d_hint(smem_addr(stage(s, a)), maps[a], x, y, bar(s), policy);
-  }
-  // Same with an L2 eviction-priority policy on the loads.
-  __device__ __forceinline__ bool issue_hint(const CUtensorMap *const (&maps)[NARR], int64_t item,
-                                            int x, int y, uint64_t policy) const {
-    const int s = (int)(item % S);
-    uint32_t d[NARR];
-    uint32_t bad = 0;
-#pragma unroll
-    for (int a = 0; a < NARR; ++a) {
-      d[a] = smem_addr(stage(s, a));
-      bad |= d[a] & 127u;
-    }
-    if (bad) return false;
-    mbar_expect_tx(bar(s), (uint32_t)L::STAGE_BYTES);
-#pragma unroll
-    for (int a = 0; a < NARR; ++a) tma_load_2d_hint(d[a], maps[a], x, y, bar(s), policy);
-    return true;
   }
 };
 

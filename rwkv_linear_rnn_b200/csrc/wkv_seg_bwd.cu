@@ -180,12 +180,6 @@ static_assert(kBwdBlockSeg >= 1 && kBwdBlockSeg <= 32, "one lane per record");
 #define WKV_SEGB_MINB 4
 #endif
 
-// int64 quotient through 32-bit division when both operands fit (the
-// common case; 64-bit division is a long instruction sequence).
-__device__ __forceinline__ int64_t qdiv(int64_t a, int64_t b) {
-  return (a <= 0x7fffffff && b <= 0x7fffffff) ? (int64_t)((unsigned)a / (unsigned)b) : a / b;
-}
-
 // Shared memory of a block of NW warps: the warp rings (with their
 // mbarriers), then per warp the forward state at each batch start of the
 // current segment: [NB][3][32] floats (a, b, exponent).
