@@ -18,6 +18,12 @@ Functions and the passages they follow (see the C file for the formulas):
 * ``bwd_recur``    -- back-propagation through the recurrence (reverse-time
                       walk, the structure of the linear-attention post's
                       gradient section).
+* ``fwd_gated``    -- the review's output gating ("출력 게이팅(Output Gating)"
+                      section, eq. o_t = W_o (sigma(r_t) * WKV_t)) without the
+                      W_o projection: o_t = sigma(r_t) * wkv_t, elementwise.
+* ``bwd_gated``    -- its gradients by the chain rule: the WKV backward fed
+                      with grad_o * sigma(r), and grad_r = grad_o * wkv *
+                      sigma(r) (1 - sigma(r)).
 
 Conventions: arrays are float64, [B, T, C] row-major with C fastest; ``w``
 (the decay itself, normally -exp(time_decay)) and ``u`` are [C]; states are
@@ -199,3 +205,31 @@ def canonical_state(state):
         ratio = np.where(b > 0, a / np.where(b > 0, b, 1.0), 0.0)
         logb = np.where(b > 0, p + np.log(np.where(b > 0, b, 1.0)), -np.inf)
     return ratio, logb
+
+
+def sigmoid(x):
+    """Logistic function 1 / (1 + e^-x) in float64, without overflow for
+    large |x| (e^-x is formed only for x >= 0, e^x only for x < 0)."""
+    x = _f64(x)
+    out = np.empty_like(x)
+    pos = x >= 0
+    out[pos] = 1.0 / (1.0 + np.exp(-x[pos]))
+    ex = np.exp(x[~pos])
+    out[~pos] = ex / (1.0 + ex)
+    return out
+
+
+def fwd_gated(w, u, k, v, r, state_in=None):
+    """o_t = sigma(r_t) * wkv_t; returns (o, final state)."""
+    y, st = fwd_recur(w, u, k, v, state_in)
+    return sigmoid(r) * y, st
+
+
+def bwd_gated(w, u, k, v, r, go, state_in=None):
+    """Gradients of L = sum(go * o) for o = sigma(r) * wkv; returns
+    (gw, gu, gk, gv, gr)."""
+    y, _ = fwd_recur(w, u, k, v, state_in)
+    sr = sigmoid(r)
+    gw, gu, gk, gv = bwd_recur(w, u, k, v, _f64(go) * sr, state_in)
+    gr = _f64(go) * y * sr * (1.0 - sr)
+    return gw, gu, gk, gv, gr
