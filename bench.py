@@ -1,7 +1,7 @@
 """Benchmark: WKV fwd+bwd channel-tokens/s and achieved HBM GB/s on B200.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libwkv|reference]
-                [--workload rwkv169m|rwkv1b5_bf16|longctx|decode14b]
+                [--workload rwkv169m|rwkv1b5_bf16|longctx|decode14b] [--gate]
 
 A step is one pass of the whole hot path over one batch of the workload:
 ``wkv_forward`` (writing the checkpoints) followed by ``wkv_backward`` on the
@@ -9,7 +9,9 @@ same inputs, through the C ABI, inputs resident in HBM.  The default
 workload is the RWKV-4 169M-shaped layer (B8 T1024 C768 fp32, seeded
 synthetic inputs).  L2 is flushed (a 2x-L2 buffer is written) before every
 timed step, outside the timed events; each step is bracketed by CUDA events
-on the launching stream and the per-step times are summed.
+on the launching stream and the per-step times are summed.  ``--gate`` times
+the gated calls instead (``wkv_forward_gated`` / ``wkv_backward_gated``,
+o = sigmoid(r) * wkv, with a seeded N(0, 1) gate input r).
 
 Multi-GPU (torchrun): every rank runs an independent replica of the workload
 on its own GPU (the operator has no cross-sequence exchange; weak scaling);
@@ -37,8 +39,10 @@ sys.path.insert(0, ROOT)
 from rwkv_linear_rnn_b200 import workloads  # noqa: E402
 
 # algorithmic bytes per channel-token (per channel-step for the decode step)
+# (gated: the forward also reads r; the backward reads r and writes grad_r)
 ALG_BYTES = {("fwd", "f32"): 12, ("fwd", "bf16"): 6, ("bwd", "f32"): 20, ("bwd", "bf16"): 10,
-             ("step", "f32"): 36}
+             ("fwd_gated", "f32"): 16, ("fwd_gated", "bf16"): 8, ("bwd_gated", "f32"): 28,
+             ("bwd_gated", "bf16"): 14, ("step", "f32"): 36}
 
 
 # Kernels each call launches on 16-byte aligned rows (all bench workloads),
@@ -51,9 +55,9 @@ KERNEL_IDS = {"auto": 0, "segment": 6, "cluster": 7}
 
 # DRAM bytes (read + write) per launch of the backward's main kernel from one
 # ncu capture of this bench's workload (cold L2; gk/gv lines still dirty in
-# L2 at kernel end are not counted).  Keyed by (workload, kernel); a kernel
-# changed since its capture has no entry (traffic reported as null).
-TRAFFIC = {("rwkv169m", "bwd_seg_kernel"): 78_362_624 + 4_597_248}
+# L2 at kernel end are not counted).  Keyed by (workload, kernel, gated); a
+# kernel changed since its capture has no entry (traffic reported as null).
+TRAFFIC = {("rwkv169m", "bwd_seg_kernel", False): 78_362_624 + 4_597_248}
 
 
 def peaks():
@@ -148,43 +152,56 @@ def aggregate_rate(units_per_rank: int, n_ranks: int, ms_per_step: float) -> flo
     return n_ranks * units_per_rank / (ms_per_step * 1e-3)
 
 
-def cpu_baseline(wl_name: str, min_seconds: float = 10.0):
-    """Time the oracle (float64 recurrence fwd + reverse bwd) on the host."""
+def cpu_baseline(wl_name: str, min_seconds: float = 10.0, gate: bool = False):
+    """Time the oracle (float64 recurrence fwd + reverse bwd, gated or not)
+    on the host."""
     import oracle
     wl = workloads.WORKLOADS[wl_name]
+    what = "gated fwd+bwd" if gate else "fwd+bwd"
     if wl_name == "rwkv169m":
-        inp = workloads.generate(wl)
-        sample = "full rwkv169m workload (B8 T1024 C768) fwd+bwd, repeated"
+        inp = workloads.generate(wl, gate=gate)
+        sample = f"full rwkv169m workload (B8 T1024 C768) {what}, repeated"
     else:  # a channel slice of the big workloads keeps the sample bounded
         C = 256
-        inp = workloads.generate(wl, C=C, T=min(wl.T, 4096), grad=True)
-        sample = f"{wl_name} with C={C}, T={inp['T']} fwd+bwd, repeated"
-    args = [np.asarray(inp[n], np.float64) for n in ("w", "u", "k", "v", "gy")]
+        inp = workloads.generate(wl, C=C, T=min(wl.T, 4096), grad=True, gate=gate)
+        sample = f"{wl_name} with C={C}, T={inp['T']} {what}, repeated"
+    names = ("w", "u", "k", "v", "r", "gy") if gate else ("w", "u", "k", "v", "gy")
+    args = [np.asarray(inp[n], np.float64) for n in names]
     units = inp["B"] * inp["T"] * inp["C"]
     times = []
     t_end = time.perf_counter() + min_seconds
     while time.perf_counter() < t_end or len(times) < 3:
         t0 = time.perf_counter()
-        oracle.fwd_recur(*args[:4], want_y=True)
-        oracle.bwd_recur(*args)
+        if gate:
+            oracle.fwd_gated(*args[:5])
+            oracle.bwd_gated(*args)
+        else:
+            oracle.fwd_recur(*args[:4], want_y=True)
+            oracle.bwd_recur(*args)
         times.append(time.perf_counter() - t0)
     med = statistics.median(times)
     return {"value": units / med, "unit": "channel-tokens/s", "cores": oracle.num_threads(),
             "kind": "oracle", "sample": f"{sample} x{len(times)}, median"}
 
 
+def metric_name(gate: bool) -> str:
+    what = "gated WKV" if gate else "WKV"
+    return f"{what} fwd+bwd channel-tokens/s (HBM GB/s and % of roofline alongside)"
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return
-    cb = cpu_baseline(args.workload, min_seconds=max(1.0, 2.0 * args.steps))
+    cb = cpu_baseline(args.workload, min_seconds=max(1.0, 2.0 * args.steps), gate=args.gate)
     wl = workloads.WORKLOADS[args.workload]
-    line = {"metric": "WKV fwd+bwd channel-tokens/s (HBM GB/s and % of roofline alongside)",
+    line = {"metric": metric_name(args.gate),
             "value": cb["value"], "unit": "channel-tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": wl.channel_tokens / cb["value"] * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)", "impl": "reference",
-            "config": {"workload": args.workload, "B": wl.B, "T": wl.T, "C": wl.C},
+            "config": {"workload": args.workload, "B": wl.B, "T": wl.T, "C": wl.C,
+                       **({"gate": True} if args.gate else {})},
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "channel-tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -210,17 +227,19 @@ def run_libwkv(args):
     wl = workloads.WORKLOADS[args.workload]
     if "bwd" not in wl.ops:
         raise SystemExit(f"workload {args.workload} has no backward; pick a fwd+bwd workload")
-    inp = workloads.generate(wl, seed=wl.seed + 1000 * rank)
+    inp = workloads.generate(wl, seed=wl.seed + 1000 * rank, gate=args.gate)
     B, T, C = inp["B"], inp["T"], inp["C"]
     dt = W.WKV_BF16 if inp["dtype"] == "bf16" else W.WKV_F32
     tdt = torch.bfloat16 if dt == W.WKV_BF16 else torch.float32
 
     def to_dev(name):
-        if dt == W.WKV_BF16 and name in ("k", "v", "gy"):
+        if dt == W.WKV_BF16 and name in ("k", "v", "gy", "r"):
             return torch.from_numpy(inp[name + "_bits"].view(np.int16)).to(dev).view(torch.bfloat16)
         return torch.from_numpy(inp[name]).to(dev)
 
     w, u, k, v, gy = (to_dev(n) for n in ("w", "u", "k", "v", "gy"))
+    r = to_dev("r") if args.gate else None
+    gr = torch.empty_like(k) if args.gate else None
     y = torch.empty_like(k)
     gk = torch.empty_like(k)
     gv = torch.empty_like(v)
@@ -247,12 +266,21 @@ def run_libwkv(args):
     bopt = abi.Options(kernel=KERNEL_IDS[args.bwd_kernel])
 
     def fwd():
-        abi.check(abi.wkv_forward_ex(B, T, C, dt, P(w), P(u), P(k), P(v), 0, P(y), 0, P(ckpt),
-                                     P(wsb), nws, sp, fopt))
+        if args.gate:
+            abi.check(abi.wkv_forward_gated_ex(B, T, C, dt, P(w), P(u), P(k), P(v), P(r), 0, P(y), 0,
+                                               P(ckpt), P(wsb), nws, sp, fopt))
+        else:
+            abi.check(abi.wkv_forward_ex(B, T, C, dt, P(w), P(u), P(k), P(v), 0, P(y), 0, P(ckpt),
+                                         P(wsb), nws, sp, fopt))
 
     def bwd():
-        abi.check(abi.wkv_backward_ex(B, T, C, dt, P(w), P(u), P(k), P(v), P(gy), 0, P(ckpt),
-                                      P(gw), P(gu), P(gk), P(gv), P(wsb), nws, sp, bopt))
+        if args.gate:
+            abi.check(abi.wkv_backward_gated_ex(B, T, C, dt, P(w), P(u), P(k), P(v), P(r), P(gy), 0,
+                                                P(ckpt), P(gw), P(gu), P(gk), P(gv), P(gr), P(wsb),
+                                                nws, sp, bopt))
+        else:
+            abi.check(abi.wkv_backward_ex(B, T, C, dt, P(w), P(u), P(k), P(v), P(gy), 0, P(ckpt),
+                                          P(gw), P(gu), P(gk), P(gv), P(wsb), nws, sp, bopt))
 
     for _ in range(args.warmup):
         flush_l2()
@@ -294,8 +322,12 @@ def run_libwkv(args):
         hy = torch.empty_like(hk).pin_memory(); hgk = torch.empty_like(hk).pin_memory()
         hgv = torch.empty_like(hk).pin_memory()
         hgw = torch.empty(C).pin_memory(); hgu = torch.empty(C).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hg))
-        d2h = sum(t.numel() * t.element_size() for t in (hy, hgk, hgv, hgw, hgu))
+        hr = r.cpu().pin_memory() if args.gate else None
+        hgr = torch.empty_like(hk).pin_memory() if args.gate else None
+        ins = (hk, hv, hg) + ((hr,) if args.gate else ())
+        outs = (hy, hgk, hgv, hgw, hgu) + ((hgr,) if args.gate else ())
+        h2d = sum(t.numel() * t.element_size() for t in ins)
+        d2h = sum(t.numel() * t.element_size() for t in outs)
         ee = []
         n_e2e = max(3, min(K, 10))
         for i in range(n_e2e + 1):
@@ -303,10 +335,14 @@ def run_libwkv(args):
             e0.record(stream)
             k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
             gy.copy_(hg, non_blocking=True)
+            if args.gate:
+                r.copy_(hr, non_blocking=True)
             fwd(); bwd()
             hy.copy_(y, non_blocking=True); hgk.copy_(gk, non_blocking=True)
             hgv.copy_(gv, non_blocking=True); hgw.copy_(gw, non_blocking=True)
             hgu.copy_(gu, non_blocking=True)
+            if args.gate:
+                hgr.copy_(gr, non_blocking=True)
             e1.record(stream)
             torch.cuda.synchronize()
             if i > 0:
@@ -320,26 +356,28 @@ def run_libwkv(args):
         hbm, peak_kind = peaks()
         fwd_ms = statistics.mean(t_fwd)
         bwd_ms = statistics.mean(t_bwd)
-        fb = ALG_BYTES[("fwd", inp["dtype"])] * units
-        bb = ALG_BYTES[("bwd", inp["dtype"])] * units
+        sfx = "_gated" if args.gate else ""
+        fb = ALG_BYTES[("fwd" + sfx, inp["dtype"])] * units
+        bb = ALG_BYTES[("bwd" + sfx, inp["dtype"])] * units
         bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9
         fwd_gbs = fb / (fwd_ms * 1e-3) / 1e9
         step_ms = total_ms / K
         bwd_names, bwd_launches = BWD_PLAN[args.bwd_kernel]
         fwd_names, fwd_launches = FWD_PLAN[args.fwd_kernel]
         main_bwd = bwd_names.split(" + ")[0]
-        traffic = TRAFFIC.get((args.workload, main_bwd))
+        traffic = TRAFFIC.get((args.workload, main_bwd, bool(args.gate)))
         line = {
-            "metric": "WKV fwd+bwd channel-tokens/s (HBM GB/s and % of roofline alongside)",
+            "metric": metric_name(args.gate),
             "value": aggregate_rate(units, ws_n, step_ms), "unit": "channel-tokens/s",
             "n_gpus": ws_n, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": inp["dtype"], "data": "synthetic (seeded; the RWKV-4 layer shapes and value ranges)",
             "config": {"workload": args.workload, "B": B, "T": T, "C": C,
+                       **({"gate": True} if args.gate else {}),
                        "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
                        "l2": "flushed before every timed step (2x L2 write + 2x L2 read, outside events)"},
             "roofline": {"bound": "hbm",
-                         "kernel": f"wkv_backward call ({bwd_names}), timed as one call",
+                         "kernel": f"wkv_backward{sfx} call ({bwd_names}), timed as one call",
                          "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": bwd_gbs / hbm, "traffic": traffic,
                          "traffic_kernel": main_bwd if traffic else None,
@@ -354,7 +392,8 @@ def run_libwkv(args):
         if e2e:
             line["e2e"] = e2e
         if not args.no_cpu_baseline and ws_n == 1:
-            line["cpu_baseline"] = cpu_baseline(args.workload, min_seconds=args.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline(args.workload, min_seconds=args.cpu_seconds,
+                                                gate=args.gate)
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -373,6 +412,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--fwd-kernel", default="auto", choices=sorted(FWD_PLAN))
     ap.add_argument("--bwd-kernel", default="auto", choices=sorted(BWD_PLAN))
+    ap.add_argument("--gate", action="store_true",
+                    help="time the gated calls (o = sigmoid(r) * wkv and its gradients)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
     if args.impl == "reference":

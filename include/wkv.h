@@ -21,6 +21,8 @@
  *   wkv_backward  gradients of a scalar loss for the same mode;
  *   wkv_step      RNN mode ("RNN-유사추론" / "자기 회귀 디코딩" steps 4 and 7):
  *                 one token per sequence against a stored state.
+ * wkv_forward_gated / wkv_backward_gated add the receptance gate
+ * o = sigma(r) * y of the time-mixing block's output.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -33,7 +35,8 @@
  *   (a bounded wait that gave up) are read later with wkv_get_status().
  *   A call that returns an error has launched nothing, except WKV_ERR_CUDA,
  *   which reports a failed launch.
- * - Layout: k, v, y, grad_y, grad_k, grad_v are [B, T, C] row-major with C
+ * - Layout: k, v, y, grad_y, grad_k, grad_v (and r, o, grad_o, grad_r of
+ *   the gated calls) are [B, T, C] row-major with C
  *   fastest (the (B, T, d) layout of the sequence model); w, u, grad_w,
  *   grad_u are [C] float32.
  * - Element type of k, v, y, grad_y, grad_k, grad_v: WKV_F32 or WKV_BF16
@@ -205,6 +208,57 @@ int wkv_backward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
                     void *ws, size_t ws_bytes, void *stream, const wkv_options *opt);
 
 /*
+ * wkv_forward_gated -- the time-mixing output with its receptance gate:
+ *   o_t = sigma(r_t) * y_t,   sigma(x) = 1 / (1 + e^{-x}),
+ * y the WKV output above (RWKV paper review, section "출력 게이팅(Output
+ * Gating)": o_t = W_o (sigma(r_t) * WKV_t); the W_o projection is a plain
+ * GEMM and stays with the caller).  The gate is applied as y is stored, so o
+ * costs one extra read of r and no pass over y.
+ *   r          [B, T, C] gate input (element type dtype).
+ *   o          [B, T, C] output; must not overlap k, v or r.
+ * Every other argument is as in wkv_forward: state_out and ckpt describe the
+ * WKV recurrence (the gate does not enter it), so the checkpoints serve
+ * wkv_backward_gated and wkv_backward alike.
+ * Errors: as wkv_forward (NULL r is INVALID_ARG when T > 0).
+ */
+int wkv_forward_gated(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                      const float *u, const void *k, const void *v, const void *r,
+                      const float *state_in, void *o, float *state_out, float *ckpt,
+                      void *ws, size_t ws_bytes, void *stream);
+
+int wkv_forward_gated_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                         const float *u, const void *k, const void *v, const void *r,
+                         const float *state_in, void *o, float *state_out, float *ckpt,
+                         void *ws, size_t ws_bytes, void *stream, const wkv_options *opt);
+
+/*
+ * wkv_backward_gated -- gradients of a scalar loss L given grad_o = dL/do
+ * for o = sigma(r) * y:
+ *   dL/dy = grad_o sigma(r)  (fed to the WKV backward),
+ *   dL/dr = grad_o y sigma(r) (1 - sigma(r)).
+ *   r, grad_o  [B, T, C] (element type dtype).
+ *   grad_r     [B, T, C] output; must not overlap any input or grad_k/grad_v.
+ * Everything else is as in wkv_backward (ckpt from wkv_forward_gated or
+ * wkv_forward of the same k, v, state_in; grad_w, grad_u overwritten and
+ * reduced in a fixed order).  The segment backward forms both gradients in
+ * its own passes; with the other kernels (rows not 16-byte aligned, or a
+ * kernel chosen in opt) grad_r is first used as scratch for dL/dy.
+ * Errors: as wkv_backward (NULL r/grad_r is INVALID_ARG when T > 0).
+ */
+int wkv_backward_gated(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                       const float *u, const void *k, const void *v, const void *r,
+                       const void *grad_o, const float *state_in, const float *ckpt,
+                       float *grad_w, float *grad_u, void *grad_k, void *grad_v,
+                       void *grad_r, void *ws, size_t ws_bytes, void *stream);
+
+int wkv_backward_gated_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                          const float *u, const void *k, const void *v, const void *r,
+                          const void *grad_o, const float *state_in, const float *ckpt,
+                          float *grad_w, float *grad_u, void *grad_k, void *grad_v,
+                          void *grad_r, void *ws, size_t ws_bytes, void *stream,
+                          const wkv_options *opt);
+
+/*
  * wkv_step -- one RNN-mode token for N independent sequences (float32).
  *   k_t, v_t   [N, C] inputs of this token.
  *   state_in   [3][N][C] state before the token (required).
@@ -258,6 +312,15 @@ int wkv_get_status(void *ws, void *stream);
 
 /* Static string for a return code ("unknown status" otherwise). */
 const char *wkv_strerror(int status);
+
+/*
+ * The cudaError_t value (as an int) behind the calling thread's most recent
+ * WKV_ERR_CUDA return, 0 if there was none; wkv_cuda_error_name gives its
+ * name ("cudaErrorInvalidValue", ...).  Diagnostics only: the value is not
+ * cleared by later successful calls.
+ */
+int wkv_last_cuda_error(void);
+const char *wkv_cuda_error_name(int err);
 
 /* WKV_VERSION of the built library. */
 int wkv_version(void);

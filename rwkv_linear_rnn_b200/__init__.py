@@ -3,7 +3,8 @@
 Thin Python binding over the C ABI in ``include/wkv.h``.  The functions in
 ``abi`` carry the C names and take raw device pointers (ints) -- argument
 marshalling only.  The tensor helpers below (``forward``, ``backward``,
-``step``, ``WKV``) take torch CUDA tensors, allocate outputs with torch, and
+``step``, ``WKV`` and the gated ``forward_gated``, ``backward_gated``,
+``GatedWKV``) take torch CUDA tensors, allocate outputs with torch, and
 call the same entry points; PyTorch provides memory and streams only, every
 step of the operator runs in the library's CUDA kernels.
 
@@ -24,7 +25,7 @@ __all__ = [
     "abi", "WKVError", "WKV_F32", "WKV_BF16", "WKV_OP_FORWARD", "WKV_OP_BACKWARD", "WKV_OP_STEP",
     "WKV_KERNEL_AUTO", "WKV_KERNEL_SEQUENTIAL", "WKV_KERNEL_CHUNKED", "WKV_KERNEL_CHUNKED_REGS",
     "WKV_KERNEL_SEGMENT", "WKV_KERNEL_CLUSTER", "WKV_STATIC_SCRATCH_BYTES", "Workspace", "forward", "backward", "step",
-    "WKV", "wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror", "wkv_version",
+    "forward_gated", "backward_gated", "WKV", "wkv", "GatedWKV", "gated_wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror", "wkv_version",
     "library_path",
 ]
 
@@ -185,6 +186,56 @@ def backward(w, u, k, v, grad_y, state_in=None, ckpt=None, *, grad_k=None, grad_
     return gw, gu, gk, gv
 
 
+def forward_gated(w, u, k, v, r, state_in=None, *, want_state=False, want_ckpt=False, o=None,
+                  workspace=None, stream=None, kernel=WKV_KERNEL_AUTO):
+    """o = sigmoid(r) * WKV(w, u, k, v) for k, v, r [B, T, C].  Returns
+    (o, state_out, ckpt) as ``forward`` does (the state and checkpoints are the
+    WKV recurrence's)."""
+    torch = _torch()
+    _check_cuda(w, u, k, v, r, state_in, o)
+    B, T, C = k.shape
+    dt = _dtype_code(k)
+    if o is None:
+        o = torch.empty_like(k)
+    state_out = torch.empty((3, B, C), dtype=torch.float32, device=k.device) if want_state else None
+    ckpt = None
+    if want_ckpt:
+        n = wkv_ckpt_size(B, T, C) // 4
+        ckpt = torch.empty(max(n, 1), dtype=torch.float32, device=k.device)
+    ws = _ws_for(k.device, workspace)
+    buf, nbytes = ws.get(WKV_OP_FORWARD, B, T, C, dt)
+    abi = _abi()
+    opts = abi.Options(kernel=kernel)
+    abi.check(abi.wkv_forward_gated_ex(B, T, C, dt, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
+                                       _ptr(state_in), _ptr(o), _ptr(state_out), _ptr(ckpt),
+                                       _ptr(buf), nbytes, _stream(stream), opts))
+    return o, state_out, ckpt
+
+
+def backward_gated(w, u, k, v, r, grad_o, state_in=None, ckpt=None, *, grad_k=None, grad_v=None,
+                   grad_r=None, workspace=None, stream=None, kernel=WKV_KERNEL_AUTO):
+    """Gradients (grad_w, grad_u, grad_k, grad_v, grad_r) of L given
+    grad_o = dL/do for o = sigmoid(r) * WKV(w, u, k, v)."""
+    torch = _torch()
+    _check_cuda(w, u, k, v, r, grad_o, state_in, ckpt, grad_k, grad_v, grad_r)
+    B, T, C = k.shape
+    dt = _dtype_code(k)
+    gw = torch.empty(C, dtype=torch.float32, device=k.device)
+    gu = torch.empty(C, dtype=torch.float32, device=k.device)
+    gk = torch.empty_like(k) if grad_k is None else grad_k
+    gv = torch.empty_like(v) if grad_v is None else grad_v
+    gr = torch.empty_like(r) if grad_r is None else grad_r
+    ws = _ws_for(k.device, workspace)
+    buf, nbytes = ws.get(WKV_OP_BACKWARD, B, T, C, dt)
+    abi = _abi()
+    opts = abi.Options(kernel=kernel)
+    abi.check(abi.wkv_backward_gated_ex(B, T, C, dt, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
+                                        _ptr(grad_o), _ptr(state_in), _ptr(ckpt), _ptr(gw),
+                                        _ptr(gu), _ptr(gk), _ptr(gv), _ptr(gr), _ptr(buf), nbytes,
+                                        _stream(stream), opts))
+    return gw, gu, gk, gv, gr
+
+
 def step(w, u, k_t, v_t, state, *, y=None, state_out=None, stream=None):
     """One RNN-mode token for N sequences.  ``state_out`` defaults to updating
     ``state`` in place.  Returns (y_t, state_out)."""
@@ -232,3 +283,35 @@ class WKV:
 def wkv(w, u, k, v):
     """Differentiable WKV: y [B, T, C] from w, u [C] and k, v [B, T, C]."""
     return WKV.apply(w, u, k, v)
+
+
+class GatedWKV:
+    """torch.autograd.Function wrapper: o = GatedWKV.apply(w, u, k, v, r)."""
+
+    _fn = None
+
+    @classmethod
+    def apply(cls, w, u, k, v, r):
+        if cls._fn is None:
+            torch = _torch()
+
+            class _F(torch.autograd.Function):
+                @staticmethod
+                def forward(ctx, w, u, k, v, r):
+                    w, u, k, v, r = (t.contiguous() for t in (w, u, k, v, r))
+                    o, _, ck = forward_gated(w, u, k, v, r, want_ckpt=True)
+                    ctx.save_for_backward(w, u, k, v, r, ck)
+                    return o
+
+                @staticmethod
+                def backward(ctx, go):
+                    w, u, k, v, r, ck = ctx.saved_tensors
+                    return backward_gated(w, u, k, v, r, go.contiguous(), ckpt=ck)
+
+            cls._fn = _F
+        return cls._fn.apply(w, u, k, v, r)
+
+
+def gated_wkv(w, u, k, v, r):
+    """Differentiable gated WKV: sigmoid(r) * WKV(w, u, k, v)."""
+    return GatedWKV.apply(w, u, k, v, r)

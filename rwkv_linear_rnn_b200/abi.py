@@ -15,13 +15,14 @@ LIB_PATH = os.environ.get("LIBWKV_PATH") or os.path.join(os.path.dirname(os.path
                                                           "libwkv.so")
 
 from .constants import *  # noqa: F401,F403  (codes shared with include/wkv.h)
-from .constants import WKV_OK
+from .constants import WKV_ERR_CUDA, WKV_OK
 
 # Every symbol the header declares, in declaration order.
 EXPORTS = (
     "wkv_workspace_size", "wkv_workspace_init", "wkv_ckpt_size", "wkv_forward", "wkv_forward_ex",
-    "wkv_backward", "wkv_backward_ex", "wkv_step", "wkv_backward_static", "wkv_get_status",
-    "wkv_strerror", "wkv_version",
+    "wkv_backward", "wkv_backward_ex", "wkv_forward_gated", "wkv_forward_gated_ex",
+    "wkv_backward_gated", "wkv_backward_gated_ex", "wkv_step", "wkv_backward_static", "wkv_get_status",
+    "wkv_strerror", "wkv_last_cuda_error", "wkv_cuda_error_name", "wkv_version",
 )
 
 
@@ -51,11 +52,17 @@ _SIGS = {
                             _p, _sz, _p]),
     "wkv_backward_ex": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                _p, _p, _sz, _p, _opt]),
+    "wkv_forward_gated": (_int, [_i64, _i64, _i64, _int] + [_p] * 10 + [_sz, _p]),
+    "wkv_forward_gated_ex": (_int, [_i64, _i64, _i64, _int] + [_p] * 10 + [_sz, _p, _opt]),
+    "wkv_backward_gated": (_int, [_i64, _i64, _i64, _int] + [_p] * 14 + [_sz, _p]),
+    "wkv_backward_gated_ex": (_int, [_i64, _i64, _i64, _int] + [_p] * 14 + [_sz, _p, _opt]),
     "wkv_step": (_int, [_i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p]),
     "wkv_backward_static": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                    _p, _p, _p]),
     "wkv_get_status": (_int, [_p, _p]),
     "wkv_strerror": (ctypes.c_char_p, [_int]),
+    "wkv_last_cuda_error": (_int, []),
+    "wkv_cuda_error_name": (ctypes.c_char_p, [_int]),
     "wkv_version": (_int, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -67,7 +74,11 @@ for _name, (_res, _args) in _SIGS.items():
 class WKVError(RuntimeError):
     def __init__(self, status: int):
         self.status = status
-        super().__init__(f"libwkv error {status}: {wkv_strerror(status)}")
+        msg = f"libwkv error {status}: {wkv_strerror(status)}"
+        if status == WKV_ERR_CUDA:
+            err = wkv_last_cuda_error()
+            msg += f" ({wkv_cuda_error_name(err)} = {err})"
+        super().__init__(msg)
 
 
 def _opts(o):
@@ -109,6 +120,31 @@ def wkv_backward_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, 
                                grad_k, grad_v, ws, ws_bytes, stream, _opts(opt))
 
 
+def wkv_forward_gated(B, T, C, dtype, w, u, k, v, r, state_in, o, state_out, ckpt, ws, ws_bytes,
+                      stream):
+    return lib.wkv_forward_gated(B, T, C, dtype, w, u, k, v, r, state_in, o, state_out, ckpt, ws,
+                                 ws_bytes, stream)
+
+
+def wkv_forward_gated_ex(B, T, C, dtype, w, u, k, v, r, state_in, o, state_out, ckpt, ws,
+                         ws_bytes, stream, opt=None):
+    return lib.wkv_forward_gated_ex(B, T, C, dtype, w, u, k, v, r, state_in, o, state_out, ckpt,
+                                    ws, ws_bytes, stream, _opts(opt))
+
+
+def wkv_backward_gated(B, T, C, dtype, w, u, k, v, r, grad_o, state_in, ckpt, grad_w, grad_u,
+                       grad_k, grad_v, grad_r, ws, ws_bytes, stream):
+    return lib.wkv_backward_gated(B, T, C, dtype, w, u, k, v, r, grad_o, state_in, ckpt, grad_w,
+                                  grad_u, grad_k, grad_v, grad_r, ws, ws_bytes, stream)
+
+
+def wkv_backward_gated_ex(B, T, C, dtype, w, u, k, v, r, grad_o, state_in, ckpt, grad_w, grad_u,
+                          grad_k, grad_v, grad_r, ws, ws_bytes, stream, opt=None):
+    return lib.wkv_backward_gated_ex(B, T, C, dtype, w, u, k, v, r, grad_o, state_in, ckpt,
+                                     grad_w, grad_u, grad_k, grad_v, grad_r, ws, ws_bytes, stream,
+                                     _opts(opt))
+
+
 def wkv_step(N, C, w, u, k_t, v_t, state_in, y_t, state_out, stream):
     return lib.wkv_step(N, C, w, u, k_t, v_t, state_in, y_t, state_out, stream)
 
@@ -126,6 +162,14 @@ def wkv_get_status(ws, stream):
 
 def wkv_strerror(status):
     return lib.wkv_strerror(status).decode()
+
+
+def wkv_last_cuda_error():
+    return lib.wkv_last_cuda_error()
+
+
+def wkv_cuda_error_name(err):
+    return lib.wkv_cuda_error_name(err).decode()
 
 
 def wkv_version():

@@ -20,12 +20,25 @@ cudaError_t launch_backward_seg(const BwdArgs &p, int dtype, float *gw, float *g
                                 int64_t scratch_doubles, int num_sms, cudaStream_t st);
 cudaError_t launch_backward(const BwdArgs &a, int dtype, float *gw, float *gu, cudaStream_t st);
 cudaError_t launch_step(const StepArgs &a, bool vec, int num_sms, cudaStream_t st);
+cudaError_t launch_gate(int op, int dtype, void *x, const void *go, const void *r, int64_t n, int num_sms,
+                        cudaStream_t st);
 int64_t fwd_chunk_tokens();
 }  // namespace wkv
 
 using namespace wkv;
 
 namespace {
+
+constexpr int kGateApply = 0, kGatePre = 1, kGatePost = 2;  // launch_gate ops
+
+// The cudaError_t behind the calling thread's most recent WKV_ERR_CUDA.
+thread_local int t_last_cuda_error = 0;
+
+int cuda_rc(cudaError_t e) {
+  if (e == cudaSuccess) return WKV_OK;
+  t_last_cuda_error = (int)e;
+  return WKV_ERR_CUDA;
+}
 
 constexpr int64_t kDefaultSpin = 1000000;  // polls of ~1 us backoff: about one second
 constexpr int64_t kSeqMinChains = 148 * 1024;  // chains that fill B200 with one thread each
@@ -132,16 +145,20 @@ int check_forward_args(int64_t B, int64_t T, int64_t C, int dtype, const float *
   return WKV_OK;
 }
 
+// r: gate input (y receives sigma(r) * wkv), or NULL.  The segment forward
+// applies the gate in its store loop; the other kernels write wkv and an
+// elementwise pass gates it.
 int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
                  const void *k, const void *v, const float *state_in, void *y, float *state_out,
-                 float *ckpt, void *ws, size_t ws_bytes, cudaStream_t st, const wkv_options *opt) {
+                 float *ckpt, void *ws, size_t ws_bytes, cudaStream_t st, const wkv_options *opt,
+                 const void *r = nullptr) {
   if (T == 0) {
     // No tokens: the state passes through unchanged (the sequential kernel
     // with T = 0 only converts state_in, or the empty state, to state_out).
     if (!state_out) return WKV_OK;
     FwdArgs a{};
     a.B = B; a.T = 0; a.C = C; a.w = w; a.u = u; a.state_in = state_in; a.state_out = state_out;
-    return launch_forward(a, dtype, 0, 1, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    return cuda_rc(launch_forward(a, dtype, 0, 1, st));
   }
   const Layout L = layout(WKV_OP_FORWARD, B, T, C);
   const bool chunked = pick_chunked(opt, B, T, C);
@@ -160,14 +177,103 @@ int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
   a.spin_limit = spin_of(opt);
   a.hold_first = opt ? opt->test_hold_first_chunk : 0;
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
-  if (chunked && fwd_tma_eligible(a, dtype) && kernel == WKV_KERNEL_CLUSTER)
-    return launch_forward_clu(a, dtype, num_sms(), st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
-  if (chunked && fwd_tma_eligible(a, dtype) &&
-      (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT))
-    return launch_forward_seg(a, dtype, num_sms(), st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
-  int kind = 0;
-  if (chunked) kind = (fwd_tma_eligible(a, dtype) && kernel != WKV_KERNEL_CHUNKED_REGS) ? 2 : 1;
-  return launch_forward(a, dtype, kind, num_sms(), st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  const bool tma = chunked && fwd_tma_eligible(a, dtype);
+  const bool seg = tma && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT);
+  if (seg && (!r || aligned(r, 16))) {
+    a.r = r;  // fused gate
+    return cuda_rc(launch_forward_seg(a, dtype, num_sms(), st));
+  }
+  cudaError_t e;
+  if (tma && kernel == WKV_KERNEL_CLUSTER) {
+    e = launch_forward_clu(a, dtype, num_sms(), st);
+  } else if (seg) {
+    e = launch_forward_seg(a, dtype, num_sms(), st);
+  } else {
+    int kind = 0;
+    if (chunked) kind = (tma && kernel != WKV_KERNEL_CHUNKED_REGS) ? 2 : 1;
+    e = launch_forward(a, dtype, kind, num_sms(), st);
+  }
+  if (e == cudaSuccess && r) e = launch_gate(kGateApply, dtype, y, nullptr, r, B * T * C, num_sms(), st);
+  return cuda_rc(e);
+}
+
+// The segment backward runs for AUTO/SEGMENT when the rows of k, v and the
+// output gradient are 16-byte aligned.
+bool bwd_uses_seg(int64_t B, int64_t T, int64_t C, int dtype, const void *k, const void *v, const void *gy,
+                  const wkv_options *opt) {
+  const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
+  if (kernel != WKV_KERNEL_AUTO && kernel != WKV_KERNEL_SEGMENT) return false;
+  FwdArgs probe{};
+  probe.B = B; probe.T = T; probe.C = C; probe.k = k; probe.v = v;
+  return fwd_tma_eligible(probe, dtype) && aligned(gy, 16);
+}
+
+// Checks shared by the gated and ungated backward (grad_y: the gradient the
+// caller passes, of y or of the gated output).
+int check_backward_args(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                        const void *k, const void *v, const void *grad_y, const float *state_in,
+                        const float *ckpt, float *grad_w, float *grad_u, void *grad_k, void *grad_v,
+                        const wkv_options *opt) {
+  int rc = check_forward_args(B, T, C, dtype, w, u, k, v, state_in, nullptr, nullptr, ckpt);
+  if (rc != WKV_OK) return rc;
+  if (!options_ok(opt)) return WKV_ERR_INVALID_ARG;
+  if (!grad_w || !grad_u) return WKV_ERR_INVALID_ARG;
+  if (T > 0 && (!grad_y || !grad_k || !grad_v)) return WKV_ERR_INVALID_ARG;
+  const size_t es = esize(dtype);
+  if (!aligned(grad_y, es) || !aligned(grad_k, es) || !aligned(grad_v, es) ||
+      !aligned(grad_w, 4) || !aligned(grad_u, 4))
+    return WKV_ERR_UNSUPPORTED;
+  const size_t nb = (size_t)(B * T * C) * es;
+  const void *ins[3] = {k, v, grad_y};
+  for (const void *in : ins)
+    if (overlaps(grad_k, nb, in, nb) || overlaps(grad_v, nb, in, nb)) return WKV_ERR_UNSUPPORTED;
+  if (overlaps(grad_k, nb, grad_v, nb) || overlaps(grad_w, 4 * C, grad_u, 4 * C))
+    return WKV_ERR_UNSUPPORTED;
+  return WKV_OK;
+}
+
+// Backward after the checks.  r, gr: gate input and its gradient for the
+// fused gated segment backward (grad_y is then dL/do), else NULL.
+int backward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                  const void *k, const void *v, const void *grad_y, const float *state_in,
+                  const float *ckpt, float *grad_w, float *grad_u, void *grad_k, void *grad_v,
+                  void *ws, size_t ws_bytes, cudaStream_t st, const wkv_options *opt,
+                  const void *r = nullptr, void *gr = nullptr) {
+  if (T == 0) {
+    const int rc = cuda_rc(cudaMemsetAsync(grad_w, 0, sizeof(float) * C, st));
+    return rc != WKV_OK ? rc : cuda_rc(cudaMemsetAsync(grad_u, 0, sizeof(float) * C, st));
+  }
+  const Layout L = layout(WKV_OP_BACKWARD, B, T, C);
+  if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return WKV_ERR_WORKSPACE;
+  char *base = static_cast<char *>(ws);
+  const float *ck = ckpt;
+  if (!ck) {
+    // Recompute the per-chunk states with a forward pass that writes only
+    // the checkpoints (one extra read of k and v).
+    float *ws_ck = reinterpret_cast<float *>(base + L.ckpt);
+    int rc = forward_impl(B, T, C, dtype, w, u, k, v, state_in, nullptr, nullptr, ws_ck, ws, ws_bytes, st, opt);
+    if (rc != WKV_OK) return rc;
+    ck = ws_ck;
+  }
+  BwdArgs a{};
+  a.B = B; a.T = T; a.C = C; a.w = w; a.u = u; a.k = k; a.v = v; a.gy = grad_y;
+  a.ckpt = ck; a.gk = grad_k; a.gv = grad_v;
+  a.part = reinterpret_cast<float *>(base + L.part);
+  a.hdr = reinterpret_cast<WsHeader *>(base);
+  a.flags = reinterpret_cast<unsigned *>(base + L.flags);
+  a.desc = reinterpret_cast<float *>(base + L.desc);
+  a.nct = L.nct; a.nchains = L.nchains; a.nchunks = L.nchunks_b;
+  a.spin_limit = spin_of(opt);
+  a.hold_first = opt ? opt->test_hold_first_chunk : 0;
+  a.r = r;
+  a.gr = gr;
+  if (bwd_uses_seg(B, T, C, dtype, k, v, grad_y, opt)) {
+    const int64_t scratch = (int64_t)(L.desc_bytes / sizeof(double));
+    return cuda_rc(launch_backward_seg(a, dtype, grad_w, grad_u, reinterpret_cast<unsigned *>(base + L.cnt), scratch,
+                               num_sms(), st));
+  }
+  if (r) return WKV_ERR_UNSUPPORTED;  // callers fuse the gate only into the segment backward
+  return cuda_rc(launch_backward(a, dtype, grad_w, grad_u, st));
 }
 
 }  // namespace
@@ -184,7 +290,7 @@ size_t wkv_workspace_size(int op, int64_t B, int64_t T, int64_t C, int dtype) {
 
 int wkv_workspace_init(void *ws, size_t ws_bytes, void *stream) {
   if (!ws) return WKV_ERR_WORKSPACE;
-  return cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  return cuda_rc(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
 }
 
 size_t wkv_ckpt_size(int64_t B, int64_t T, int64_t C) {
@@ -215,63 +321,11 @@ int wkv_backward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, 
                     const void *k, const void *v, const void *grad_y, const float *state_in,
                     const float *ckpt, float *grad_w, float *grad_u, void *grad_k, void *grad_v,
                     void *ws, size_t ws_bytes, void *stream, const wkv_options *opt) {
-  int rc = check_forward_args(B, T, C, dtype, w, u, k, v, state_in, nullptr, nullptr, ckpt);
+  const int rc = check_backward_args(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u,
+                                     grad_k, grad_v, opt);
   if (rc != WKV_OK) return rc;
-  if (!options_ok(opt)) return WKV_ERR_INVALID_ARG;
-  if (!grad_w || !grad_u) return WKV_ERR_INVALID_ARG;
-  if (T > 0 && (!grad_y || !grad_k || !grad_v)) return WKV_ERR_INVALID_ARG;
-  const size_t es = esize(dtype);
-  if (!aligned(grad_y, es) || !aligned(grad_k, es) || !aligned(grad_v, es) ||
-      !aligned(grad_w, 4) || !aligned(grad_u, 4))
-    return WKV_ERR_UNSUPPORTED;
-  const size_t nb = (size_t)(B * T * C) * es;
-  const void *ins[3] = {k, v, grad_y};
-  for (const void *in : ins)
-    if (overlaps(grad_k, nb, in, nb) || overlaps(grad_v, nb, in, nb)) return WKV_ERR_UNSUPPORTED;
-  if (overlaps(grad_k, nb, grad_v, nb) || overlaps(grad_w, 4 * C, grad_u, 4 * C))
-    return WKV_ERR_UNSUPPORTED;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (T == 0) {
-    if (cudaMemsetAsync(grad_w, 0, sizeof(float) * C, st) != cudaSuccess ||
-        cudaMemsetAsync(grad_u, 0, sizeof(float) * C, st) != cudaSuccess)
-      return WKV_ERR_CUDA;
-    return WKV_OK;
-  }
-  const Layout L = layout(WKV_OP_BACKWARD, B, T, C);
-  if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return WKV_ERR_WORKSPACE;
-  char *base = static_cast<char *>(ws);
-  const float *ck = ckpt;
-  if (!ck) {
-    // Recompute the per-chunk states with a forward pass that writes only
-    // the checkpoints (one extra read of k and v).
-    float *ws_ck = reinterpret_cast<float *>(base + L.ckpt);
-    rc = forward_impl(B, T, C, dtype, w, u, k, v, state_in, nullptr, nullptr, ws_ck, ws, ws_bytes,
-                      st, opt);
-    if (rc != WKV_OK) return rc;
-    ck = ws_ck;
-  }
-  BwdArgs a{};
-  a.B = B; a.T = T; a.C = C; a.w = w; a.u = u; a.k = k; a.v = v; a.gy = grad_y;
-  a.ckpt = ck; a.gk = grad_k; a.gv = grad_v;
-  a.part = reinterpret_cast<float *>(base + L.part);
-  a.hdr = reinterpret_cast<WsHeader *>(base);
-  a.flags = reinterpret_cast<unsigned *>(base + L.flags);
-  a.desc = reinterpret_cast<float *>(base + L.desc);
-  a.nct = L.nct; a.nchains = L.nchains; a.nchunks = L.nchunks_b;
-  a.spin_limit = spin_of(opt);
-  a.hold_first = opt ? opt->test_hold_first_chunk : 0;
-  const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
-  FwdArgs probe{};
-  probe.B = B; probe.T = T; probe.C = C; probe.k = k; probe.v = v;
-  const bool tma_ok = fwd_tma_eligible(probe, dtype) && ((uintptr_t)grad_y % 16) == 0;
-  if (tma_ok && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT)) {
-    const int64_t scratch = (int64_t)(L.desc_bytes / sizeof(double));
-    return launch_backward_seg(a, dtype, grad_w, grad_u, reinterpret_cast<unsigned *>(base + L.cnt), scratch,
-                               num_sms(), st) == cudaSuccess
-               ? WKV_OK
-               : WKV_ERR_CUDA;
-  }
-  return launch_backward(a, dtype, grad_w, grad_u, st) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  return backward_impl(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u, grad_k, grad_v,
+                       ws, ws_bytes, (cudaStream_t)stream, opt);
 }
 
 int wkv_backward(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
@@ -280,6 +334,71 @@ int wkv_backward(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
                  void *ws, size_t ws_bytes, void *stream) {
   return wkv_backward_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u,
                          grad_k, grad_v, ws, ws_bytes, stream, nullptr);
+}
+
+int wkv_forward_gated_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                         const void *k, const void *v, const void *r, const float *state_in, void *o,
+                         float *state_out, float *ckpt, void *ws, size_t ws_bytes, void *stream,
+                         const wkv_options *opt) {
+  int rc = check_forward_args(B, T, C, dtype, w, u, k, v, state_in, o, state_out, ckpt);
+  if (rc != WKV_OK) return rc;
+  if (T > 0 && (!o || !r)) return WKV_ERR_INVALID_ARG;
+  if (!options_ok(opt)) return WKV_ERR_INVALID_ARG;
+  const size_t es = esize(dtype), nb = (size_t)(B * T * C) * es;
+  if (!aligned(r, es)) return WKV_ERR_UNSUPPORTED;
+  if (overlaps(o, nb, r, nb)) return WKV_ERR_UNSUPPORTED;
+  return forward_impl(B, T, C, dtype, w, u, k, v, state_in, o, state_out, ckpt, ws, ws_bytes,
+                      (cudaStream_t)stream, opt, T > 0 ? r : nullptr);
+}
+
+int wkv_forward_gated(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                      const void *k, const void *v, const void *r, const float *state_in, void *o,
+                      float *state_out, float *ckpt, void *ws, size_t ws_bytes, void *stream) {
+  return wkv_forward_gated_ex(B, T, C, dtype, w, u, k, v, r, state_in, o, state_out, ckpt, ws, ws_bytes,
+                              stream, nullptr);
+}
+
+int wkv_backward_gated_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                          const void *k, const void *v, const void *r, const void *grad_o,
+                          const float *state_in, const float *ckpt, float *grad_w, float *grad_u,
+                          void *grad_k, void *grad_v, void *grad_r, void *ws, size_t ws_bytes, void *stream,
+                          const wkv_options *opt) {
+  int rc = check_backward_args(B, T, C, dtype, w, u, k, v, grad_o, state_in, ckpt, grad_w, grad_u, grad_k,
+                               grad_v, opt);
+  if (rc != WKV_OK) return rc;
+  if (T > 0 && (!r || !grad_r)) return WKV_ERR_INVALID_ARG;
+  const size_t es = esize(dtype), nb = (size_t)(B * T * C) * es;
+  if (!aligned(r, es) || !aligned(grad_r, es)) return WKV_ERR_UNSUPPORTED;
+  const void *others[6] = {k, v, r, grad_o, grad_k, grad_v};
+  for (const void *x : others)
+    if (overlaps(grad_r, nb, x, nb)) return WKV_ERR_UNSUPPORTED;
+  if (overlaps(grad_k, nb, r, nb) || overlaps(grad_v, nb, r, nb)) return WKV_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (T > 0 && (!ws || !aligned(ws, 256) || ws_bytes < layout(WKV_OP_BACKWARD, B, T, C).total))
+    return WKV_ERR_WORKSPACE;
+  if (T == 0 || (bwd_uses_seg(B, T, C, dtype, k, v, grad_o, opt) && aligned(r, 16)))
+    return backward_impl(B, T, C, dtype, w, u, k, v, grad_o, state_in, ckpt, grad_w, grad_u, grad_k, grad_v,
+                         ws, ws_bytes, st, opt, T > 0 ? r : nullptr, grad_r);
+  // Unfused: grad_r first carries dL/dwkv = grad_o sigma(r) into the WKV
+  // backward, then wkv itself (a forward into grad_r), and finally
+  // dL/dr = grad_o wkv sigma'(r).
+  const int64_t n = B * T * C;
+  rc = cuda_rc(launch_gate(kGatePre, dtype, grad_r, grad_o, r, n, num_sms(), st));
+  if (rc != WKV_OK) return rc;
+  rc = backward_impl(B, T, C, dtype, w, u, k, v, grad_r, state_in, ckpt, grad_w, grad_u, grad_k, grad_v, ws,
+                     ws_bytes, st, opt);
+  if (rc != WKV_OK) return rc;
+  rc = forward_impl(B, T, C, dtype, w, u, k, v, state_in, grad_r, nullptr, nullptr, ws, ws_bytes, st, opt);
+  if (rc != WKV_OK) return rc;
+  return cuda_rc(launch_gate(kGatePost, dtype, grad_r, grad_o, r, n, num_sms(), st));
+}
+
+int wkv_backward_gated(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                       const void *k, const void *v, const void *r, const void *grad_o, const float *state_in,
+                       const float *ckpt, float *grad_w, float *grad_u, void *grad_k, void *grad_v,
+                       void *grad_r, void *ws, size_t ws_bytes, void *stream) {
+  return wkv_backward_gated_ex(B, T, C, dtype, w, u, k, v, r, grad_o, state_in, ckpt, grad_w, grad_u, grad_k,
+                               grad_v, grad_r, ws, ws_bytes, stream, nullptr);
 }
 
 int wkv_step(int64_t N, int64_t C, const float *w, const float *u, const float *k_t,
@@ -298,18 +417,18 @@ int wkv_step(int64_t N, int64_t C, const float *w, const float *u, const float *
   StepArgs a{N, C, w, u, k_t, v_t, state_in, y_t, state_out};
   bool vec = (C % 4) == 0;
   for (const void *p : ptrs) vec = vec && aligned(p, 16);
-  return launch_step(a, vec, num_sms(), (cudaStream_t)stream) == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  return cuda_rc(launch_step(a, vec, num_sms(), (cudaStream_t)stream));
 }
 
 int wkv_get_status(void *ws, void *stream) {
   if (!ws) return WKV_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return WKV_ERR_CUDA;
+  int rc = cuda_rc(cudaStreamSynchronize(st));
+  if (rc != WKV_OK) return rc;
   int status = 0;
   WsHeader *h = static_cast<WsHeader *>(ws);
-  if (cudaMemcpy(&status, &h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return WKV_ERR_CUDA;
-  if (status != 0 && cudaMemset(&h->status, 0, sizeof(int)) != cudaSuccess) return WKV_ERR_CUDA;
+  if ((rc = cuda_rc(cudaMemcpy(&status, &h->status, sizeof(int), cudaMemcpyDeviceToHost))) != WKV_OK) return rc;
+  if (status != 0 && (rc = cuda_rc(cudaMemset(&h->status, 0, sizeof(int)))) != WKV_OK) return rc;
   return status;
 }
 
@@ -326,5 +445,9 @@ const char *wkv_strerror(int status) {
 }
 
 int wkv_version(void) { return WKV_VERSION; }
+
+int wkv_last_cuda_error(void) { return t_last_cuda_error; }
+
+const char *wkv_cuda_error_name(int err) { return cudaGetErrorName((cudaError_t)err); }
 
 }  // extern "C"

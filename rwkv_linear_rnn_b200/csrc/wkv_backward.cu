@@ -294,18 +294,17 @@ constexpr int kBwdW = 8, kBwdL = 8;
 template <typename E>
 static cudaError_t launch_bwd_t(const BwdArgs &a, float *gw, float *gu, cudaStream_t st) {
   const int64_t tiles = a.nchains * a.nchunks;
-  bwd_chunked_kernel<E, kBwdW, kBwdL><<<(unsigned)tiles, kBwdW * 32, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(bwd_chunked_kernel<E, kBwdW, kBwdL>, dim3((unsigned)tiles), dim3(kBwdW * 32), 0,
+                                st, a);
   if (e != cudaSuccess) return e;
-  reduce_wu_kernel<<<(unsigned)((a.C + 31) / 32), 256, 0, st>>>(a.part, a.nchunks, a.B, a.C, gw,
-                                                                 gu);
-  return cudaGetLastError();
+  return launch_kernel(reduce_wu_kernel, dim3((unsigned)((a.C + 31) / 32)), dim3(256), 0, st,
+                       (const float *)a.part, a.nchunks, a.B, a.C, gw, gu);
 }
 
 cudaError_t launch_reduce_wu(const float *part, int64_t nchunks, int64_t B, int64_t C, float *gw,
                              float *gu, cudaStream_t st) {
-  reduce_wu_kernel<<<(unsigned)((C + 31) / 32), 256, 0, st>>>(part, nchunks, B, C, gw, gu);
-  return cudaGetLastError();
+  return launch_kernel(reduce_wu_kernel, dim3((unsigned)((C + 31) / 32)), dim3(256), 0, st, part, nchunks, B, C,
+                       gw, gu);
 }
 
 cudaError_t launch_backward(const BwdArgs &a0, int dtype, float *gw, float *gu, cudaStream_t st) {

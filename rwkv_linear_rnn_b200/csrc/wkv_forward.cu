@@ -404,23 +404,40 @@ static_assert(kFwdW * kFwdL == kTmaW * kTmaL, "both chunked kernels use one chun
 
 int64_t fwd_chunk_tokens() { return kFwdW * kFwdL; }
 
+// A driver entry point, looked up through the runtime (null if missing).
+static void *driver_entry(const char *name) {
+  void *f = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &f, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return f;
+}
+
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void *f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
+  // looked up once (thread-safe static initialisation)
+  static const auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(driver_entry("cuTensorMapEncodeTiled"));
   return fn;
+}
+
+// The tensor-map encoder is a driver-API call and needs a context current in
+// the calling thread.  A thread whose only CUDA use so far is this library
+// (an autograd worker, say) may have none: the runtime binds the device's
+// primary context on its first runtime call that needs one, and a thread
+// that never made such a call has none.  Bind it then; a context the caller
+// made current is left alone.
+static bool ensure_context() {
+  static const auto get = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(driver_entry("cuCtxGetCurrent"));
+  CUcontext ctx = nullptr;
+  if (get && get(&ctx) == CUDA_SUCCESS && ctx) return true;
+  int dev = 0;
+  return cudaGetDevice(&dev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess;
 }
 
 // [B*T, C] view of a [B, T, C] tensor, boxes of 32 columns x `rows` rows.
 bool encode_rows(CUtensorMap *m, const void *ptr, int dtype, int64_t rows, int64_t C,
                  int box_rows) {
   auto enc = tensor_map_encoder();
-  if (!enc) return false;
+  if (!enc || !ensure_context()) return false;
   const size_t es = dtype == 0 ? 4 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(C * es)};
@@ -467,13 +484,11 @@ static cudaError_t launch_fwd_t(const FwdArgs &a, int kind, int dtype, int num_s
   if (kind == 0) {
     const int64_t BC = a.B * a.C;
     const unsigned grid = (unsigned)((BC + 255) / 256);
-    fwd_seq_kernel<E, kSeqU><<<grid, 256, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_kernel(fwd_seq_kernel<E, kSeqU>, dim3(grid), dim3(256), 0, st, a);
   }
   if (kind == 2) return launch_fwd_tma_t<E>(a, dtype, num_sms, st);
   const int64_t tiles = a.nchains * a.nchunks;
-  fwd_chunked_kernel<E, kFwdW, kFwdL><<<(unsigned)tiles, kFwdW * 32, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(fwd_chunked_kernel<E, kFwdW, kFwdL>, dim3((unsigned)tiles), dim3(kFwdW * 32), 0, st, a);
 }
 
 // kind: 0 sequential, 1 register-tile chunked, 2 TMA chunked.

@@ -30,6 +30,21 @@ constexpr float kEmptyP = -1.0e38f;
 constexpr float kEmptyR = 1.0e38f;
 constexpr int kCkpt = 32;  // tokens between forward checkpoints
 
+// -------------------------------------------------------------- launch ---
+// Launch with the launch's own status.  (A <<<...>>> launch followed by
+// cudaGetLastError would also return a stale error that an unrelated runtime
+// call left in the calling thread.)
+template <typename... P, typename... A>
+inline cudaError_t launch_kernel(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                 A &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<A &&>(args)...);
+}
+
 // ---------------------------------------------------------------- math ---
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -427,6 +442,18 @@ __device__ __forceinline__ void grid_barrier(WsHeader *h, unsigned nblocks, int6
   }
   __syncthreads();
 }
+// Logistic gate sigma(r) = 1 / (1 + 2^{-r log2 e}) from the hardware
+// exp2 and reciprocal (saturates to 0 / 1 for large |r|).
+__device__ __forceinline__ float gate_sigmoid(float r) { return rcp(1.f + ex2(-r * kLog2e)); }
+// The gate and its slope sigma'(r) = sigma (1 - sigma) = e / (1 + e)^2 with
+// e = exp(-r), formed without the cancellation of 1 - sigma near sigma = 1;
+// e is capped so that e = inf (r -> -inf) gives slope 0, not inf * 0.
+__device__ __forceinline__ void gate_sigmoid_slope(float r, float &s, float &ds) {
+  const float e = ex2(-r * kLog2e);
+  const float q = rcp(1.f + e);
+  s = q;
+  ds = fminf(e, 1.0e30f) * q * q;
+}
 // L2 eviction-priority policies for TMA loads (createpolicy).
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
@@ -476,6 +503,7 @@ struct FwdArgs {
   int64_t nchunks;  // chunks of the time axis
   int64_t spin_limit;
   int hold_first;
+  const void *r;  // output gate input [B, T, C] (y becomes sigma(r) * wkv), or null
 };
 
 struct BwdArgs {
@@ -491,6 +519,8 @@ struct BwdArgs {
   int64_t nct, nchains, nchunks;
   int64_t spin_limit;
   int hold_first;
+  const void *r;  // output gate input (grad_y is then the gated output's gradient), or null
+  void *gr;       // gradient of the gate input (with r)
 };
 
 struct StepArgs {

@@ -49,6 +49,14 @@ struct Ring {
       for (int a = 0; a < NARR; ++a) bad |= smem_addr(stage(s, a)) & 127u;
     return bad == 0;
   }
+  // As issue_stage, loading only the first n of the NARR tensors.
+  __device__ __forceinline__ void issue_stage_n(const CUtensorMap *const (&maps)[NARR], int s, int x, int y,
+                                                uint64_t policy, int n) const {
+    mbar_expect_tx(bar(s), (uint32_t)(n * L::ARR_BYTES));
+#pragma unroll
+    for (int a = 0; a < NARR; ++a)
+      if (a < n) tma_load_2d_hint(smem_addr(stage(s, a)), maps[a], x, y, bar(s), policy);
+  }
   // Loads into stage s (the caller tracks stages), with an L2 policy; the
   // ring must have passed aligned().
   __device__ __forceinline__ void issue_stage(const CUtensorMap *const (&maps)[NARR], int s, int x, int y,

@@ -54,9 +54,12 @@ static_assert(kBlockSeg >= 1 && kBlockSeg <= 32, "one lane per record");
 // warps run pass 1, meet at one grid barrier, and fold their predecessors'
 // summaries without polling.  Otherwise segments are joined through
 // per-record flags (decoupled, at most kBlockSeg records per fold).
-template <typename E, int S, int RB, bool BAR>
+// GATE: the output is sigma(r) * wkv (the gate input r arrives with the
+// second pass's rows as a third ring array).
+template <typename E, int S, int RB, bool BAR, bool GATE>
 __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
                                                       const __grid_constant__ CUtensorMap vmap,
+                                                      const __grid_constant__ CUtensorMap rmap,
                                                       SegArgs a) {
   static_assert(kCkpt % RB == 0, "checkpoints fall on batch starts");
   const int TS = a.ts;       // tokens per segment
@@ -66,9 +69,13 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
   extern __shared__ __align__(1024) unsigned char smem[];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = (int)(blockDim.x >> 5);
-  Ring<E, S, 2, RB> ring(smem, wl, nw);
+  constexpr int NARR = GATE ? 3 : 2;
+  Ring<E, S, NARR, RB> ring(smem, wl, nw);
   ring.init(lane);
-  const CUtensorMap *const maps[2] = {&kmap, &vmap};
+  const CUtensorMap *maps[NARR];
+  maps[0] = &kmap;
+  maps[1] = &vmap;
+  if constexpr (GATE) maps[NARR - 1] = &rmap;
   // unit indices fit 31 bits (the launcher checks nseg * nchains)
   const int G = (int)gridDim.x * nw;
   const int g = (int)blockIdx.x * nw + wl;
@@ -99,8 +106,9 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
       iss_row0 = (int)((int64_t)b * T + (int64_t)pos * TS);
     }
     const int bt = iss_r < NBT ? iss_r : iss_r - NBT;
-    ring.issue_stage(maps, iss_s, iss_x, iss_row0 + bt * RB,
-                     iss_r < NBT ? l2_policy_evict_last() : l2_policy_evict_first());
+    // pass 1 needs k, v only; pass 2 also the gate input
+    ring.issue_stage_n(maps, iss_s, iss_x, iss_row0 + bt * RB,
+                       iss_r < NBT ? l2_policy_evict_last() : l2_policy_evict_first(), iss_r < NBT ? 2 : NARR);
     iss_done = ++iss_k;
     iss_s = iss_s + 1 == S ? 0 : iss_s + 1;
     if (++iss_r == IPU) {
@@ -113,8 +121,9 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
   bool failed = false;
   int cs = 0;
   uint32_t cph = 0;
-  // Consume the next item: K (base-2 scaled) and V of its RB rows.
-  auto take = [&](float(&K)[RB], float(&V)[RB]) {
+  // Consume the next item: K (base-2 scaled) and V of its RB rows, and
+  // (gated second pass) the gate sigma(r) of each row in R.
+  auto take = [&](float(&K)[RB], float(&V)[RB], float(&R)[RB], bool want_r) {
     if (!failed && !mbar_wait(ring.bar(cs), cph, budget, nullptr)) {
       failed = true;
       if (lane == 0) atomicCAS(&p.hdr->status, 0, -5 /* WKV_ERR_TIMEOUT */);
@@ -125,6 +134,13 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
     for (int j = 0; j < RB; ++j) {
       K[j] = to_f32(kr[j * 32]) * kLog2e;
       V[j] = to_f32(vr[j * 32]);
+    }
+    if constexpr (GATE) {
+      if (want_r) {
+        const E *rr = ring.stage(cs, NARR - 1) + lane;
+#pragma unroll
+        for (int j = 0; j < RB; ++j) R[j] = gate_sigmoid(to_f32(rr[j * 32]));
+      }
     }
     __syncwarp();  // the stage is read; it may be refilled
     if (++cs == S) {
@@ -155,8 +171,8 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
     St agg = st_empty();
 #pragma unroll 1
     for (int bt = 0; bt < (has ? NBT : 0); ++bt) {
-      float K[RB], V[RB];
-      take(K, V);
+      float K[RB], V[RB], R[RB];
+      take(K, V, R, false);
       const int nb = max(0, min(RB, n - bt * RB));
       const St sb = nb == RB ? summarize_full<RB>(K, V, w2) : summarize<RB>(K, V, w2, nb);
       agg = combine(agg, sb, (float)nb, w2);
@@ -235,8 +251,12 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
     const FastC fc = fast_consts<RB>(w2, u2);
 #pragma unroll 1
     for (int bt = 0; bt < NBT; ++bt) {
-      float K[RB], V[RB];
-      take(K, V);
+      float K[RB], V[RB], R[RB];
+      take(K, V, R, true);
+      if constexpr (!GATE) {
+#pragma unroll
+        for (int j = 0; j < RB; ++j) R[j] = 1.f;
+      }
       const int nb = max(0, min(RB, n - bt * RB));
       const int64_t tb = t0 + bt * RB;
       if (p.ckpt && cok && nb > 0 && (tb % kCkpt) == 0)
@@ -255,21 +275,21 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
           const float yv = fmaf(eu, V[j], al) * rcp(be + eu);
           al = fmaf(al, fc.ewm, ek * V[j]);
           be = fmaf(be, fc.ewm, ek);
-          if (yp) IO<E>::st(yp + (int64_t)j * C, yv);
+          if (yp) IO<E>::st(yp + (int64_t)j * C, GATE ? yv * R[j] : yv);
         }
         st = Run{al, be, M, fc.nend};
       } else if (nb == RB) {
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
           const float yv = fwd_token(st, K[j], V[j], u2, w2);
-          if (yp) IO<E>::st(yp + (int64_t)j * C, yv);
+          if (yp) IO<E>::st(yp + (int64_t)j * C, GATE ? yv * R[j] : yv);
         }
       } else {
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
           if (j < nb) {
             const float yv = fwd_token(st, K[j], V[j], u2, w2);
-            if (yp) IO<E>::st(yp + (int64_t)j * C, yv);
+            if (yp) IO<E>::st(yp + (int64_t)j * C, GATE ? yv * R[j] : yv);
           }
         }
       }
@@ -284,25 +304,28 @@ __global__ void __launch_bounds__(128, 4) fwd_seg_kernel(const __grid_constant__
   finish_block(p.hdr, gridDim.x);
 }
 
-template <typename E, int S, int RB, bool BAR>
-static cudaError_t launch_seg_k(const CUtensorMap &km, const CUtensorMap &vm, SegArgs a, int64_t grid,
-                                int smem, cudaStream_t st) {
-  auto kern = fwd_seg_kernel<E, S, RB, BAR>;
-  CUtensorMap k2 = km, v2 = vm;
-  void *args[] = {&k2, &v2, &a};
+template <typename E, int S, int RB, bool BAR, bool GATE>
+static cudaError_t launch_seg_k(const CUtensorMap &km, const CUtensorMap &vm, const CUtensorMap &rm, SegArgs a,
+                                int64_t grid, int smem, cudaStream_t st) {
+  auto kern = fwd_seg_kernel<E, S, RB, BAR, GATE>;
+  CUtensorMap k2 = km, v2 = vm, r2 = rm;
+  void *args[] = {&k2, &v2, &r2, &a};
   return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3(128), args, (size_t)smem, st);
 }
 
-template <typename E, int S, int RB>
+template <typename E, int S, int RB, bool GATE>
 static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, int ts_max, cudaStream_t st) {
-  CUtensorMap km, vm;
+  CUtensorMap km, vm, rm;
   if (!encode_rows(&km, f.k, dtype, f.B * f.T, f.C, RB) || !encode_rows(&vm, f.v, dtype, f.B * f.T, f.C, RB))
     return cudaErrorInvalidValue;
+  rm = vm;  // unused without the gate
+  if (GATE && !encode_rows(&rm, f.r, dtype, f.B * f.T, f.C, RB)) return cudaErrorInvalidValue;
   constexpr int kWarps = 4;
-  constexpr int smem = WarpRing<E, S, 2, RB>::block_bytes(kWarps);
+  constexpr int smem = WarpRing<E, S, GATE ? 3 : 2, RB>::block_bytes(kWarps);
   // the grid is sized for the smaller occupancy of the two join variants
   int occ = 1 << 30;
-  for (const void *kern : {(const void *)fwd_seg_kernel<E, S, RB, false>, (const void *)fwd_seg_kernel<E, S, RB, true>}) {
+  for (const void *kern : {(const void *)fwd_seg_kernel<E, S, RB, false, GATE>,
+                           (const void *)fwd_seg_kernel<E, S, RB, true, GATE>}) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int o = 0;
@@ -332,8 +355,8 @@ static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, int ts
   // together anyway) and chains have few segments (each fold reads all of
   // its predecessors); the test hook needs the flag join.
   const bool bar = rounds == 1 && a.nseg <= 32 && !f.hold_first;
-  return bar ? launch_seg_k<E, S, RB, true>(km, vm, a, grid, smem, st)
-             : launch_seg_k<E, S, RB, false>(km, vm, a, grid, smem, st);
+  return bar ? launch_seg_k<E, S, RB, true, GATE>(km, vm, rm, a, grid, smem, st)
+             : launch_seg_k<E, S, RB, false, GATE>(km, vm, rm, a, grid, smem, st);
 }
 
 // Tile parameters per element type (compile-time tunables): the longest
@@ -354,9 +377,23 @@ static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, int ts
 #define WKV_SEGF_RB 16
 #endif
 
+// Ring stages of the gated variant (its stages hold a third array).
+#ifndef WKV_SEGF_S_F32_GATE
+#define WKV_SEGF_S_F32_GATE WKV_SEGF_S_F32
+#endif
+#ifndef WKV_SEGF_S_BF16_GATE
+#define WKV_SEGF_S_BF16_GATE WKV_SEGF_S_BF16
+#endif
+
 cudaError_t launch_forward_seg(const FwdArgs &f, int dtype, int num_sms, cudaStream_t st) {
-  return dtype == 0 ? launch_seg_t<float, WKV_SEGF_S_F32, WKV_SEGF_RB>(f, dtype, num_sms, WKV_SEGF_TS_F32, st)
-                    : launch_seg_t<uint16_t, WKV_SEGF_S_BF16, WKV_SEGF_RB>(f, dtype, num_sms, WKV_SEGF_TS_BF16, st);
+  if (f.r)
+    return dtype == 0 ? launch_seg_t<float, WKV_SEGF_S_F32_GATE, WKV_SEGF_RB, true>(f, dtype, num_sms,
+                                                                                      WKV_SEGF_TS_F32, st)
+                      : launch_seg_t<uint16_t, WKV_SEGF_S_BF16_GATE, WKV_SEGF_RB, true>(f, dtype, num_sms,
+                                                                                          WKV_SEGF_TS_BF16, st);
+  return dtype == 0
+             ? launch_seg_t<float, WKV_SEGF_S_F32, WKV_SEGF_RB, false>(f, dtype, num_sms, WKV_SEGF_TS_F32, st)
+             : launch_seg_t<uint16_t, WKV_SEGF_S_BF16, WKV_SEGF_RB, false>(f, dtype, num_sms, WKV_SEGF_TS_BF16, st);
 }
 
 }  // namespace wkv

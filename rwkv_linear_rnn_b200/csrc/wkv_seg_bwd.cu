@@ -103,12 +103,15 @@ __device__ __forceinline__ Adj5s rjoin(const Adj5s &X, const Adj5s &Y, float len
 // Returns true (warp-uniform) when the batch ran on the fast path; then M is
 // its reference exponent: qv_j = M + j w2e, and e2 2^{-u2 - w2e} is the
 // factor 2^{K_j - M - (j+1) w2e} with which token j entered the state.
-template <int RB>
+// WY: Yw[j] is multiplied by the recomputed output y_j (the gated
+// backward's dL/dr = grad_o sigma'(r) y).
+template <int RB, bool WY>
 __device__ __forceinline__ bool recompute_batch(const float (&K)[RB], const float (&V)[RB],
                                                 const float (&Gy)[RB], float w2, float u2,
                                                 const FastC &fc, float &xa, float &xb, float &xP,
                                                 float &xn, float (&qv)[RB], float (&gam)[RB],
-                                                float (&eta)[RB], float (&e2v)[RB], float &M) {
+                                                float (&eta)[RB], float (&e2v)[RB], float &M,
+                                                float (&Yw)[RB]) {
   const float E0 = fmaf(xn, w2, xP);
   float kj[RB];
   const bool ok = fast_prep<RB>(K, E0, u2, fc.w2e, kj, M);
@@ -123,6 +126,7 @@ __device__ __forceinline__ bool recompute_batch(const float (&K)[RB], const floa
       const float y = fmaf(eu, V[j], al) * rden;
       gam[j] = Gy[j] * rden;  // qv is formed by the caller if it needs it: M + j w2e
       eta[j] = gam[j] * y;
+      if constexpr (WY) Yw[j] *= y;
       e2v[j] = eu;
       al = fmaf(al, fc.ewm, ek * V[j]);
       be = fmaf(be, fc.ewm, ek);
@@ -146,6 +150,7 @@ __device__ __forceinline__ bool recompute_batch(const float (&K)[RB], const floa
     qv[j] = fmaxf(P, UK);
     gam[j] = Gy[j] * rden;
     eta[j] = gam[j] * y;
+    if constexpr (WY) Yw[j] *= y;
     e2v[j] = e2;
     const float n1 = xn + 1.f;
     const float Pc = fmaf(n1, w2, xP);
@@ -182,10 +187,11 @@ static_assert(kBwdBlockSeg >= 1 && kBwdBlockSeg <= 32, "one lane per record");
 
 // Shared memory of a block of NW warps: the warp rings (with their
 // mbarriers), then per warp the forward state at each batch start of the
-// current segment: [NB][3][32] floats (a, b, exponent).
-template <typename E, int S, int RB>
+// current segment: [NB][3][32] floats (a, b, exponent).  NARR: tensors per
+// ring item (k, v, grad, and the gate input when gated).
+template <typename E, int S, int RB, int NARR>
 struct SegBwdSmem {
-  using RingL = WarpRing<E, S, 3, RB>;
+  using RingL = WarpRing<E, S, NARR, RB>;
   static constexpr int ring_bytes(int nw) { return (RingL::block_bytes(nw) + 15) / 16 * 16; }
   static constexpr int bytes(int nw, int nb) { return ring_bytes(nw) + nw * nb * 96 * 4; }
 };
@@ -193,12 +199,17 @@ struct SegBwdSmem {
 // BAR: every warp owns at most one segment; all warps run pass 1, meet at a
 // grid barrier and fold the later segments' aggregates without polling.
 // Otherwise segments are joined through per-record flags.
-template <typename E, int S, int RB, bool BAR>
+// GATE: the loss depends on o = sigma(r) * y; the ring items carry r as a
+// fourth tensor, the WKV gradient is grad_o sigma(r) and pass 2 also writes
+// dL/dr = grad_o y sigma'(r).
+template <typename E, int S, int RB, bool BAR, bool GATE>
 __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
                                                       const __grid_constant__ CUtensorMap vmap,
                                                       const __grid_constant__ CUtensorMap gmap,
+                                                      const __grid_constant__ CUtensorMap rmap,
                                                       SegBwdArgs a) {
-  using Sm = SegBwdSmem<E, S, RB>;
+  constexpr int NARR = GATE ? 4 : 3;
+  using Sm = SegBwdSmem<E, S, RB, NARR>;
   const int TS = a.ts;         // tokens per segment (segments start on checkpoints)
   const int NB = a.nb;         // ring items (batches of RB tokens) per pass
   const int IPU = 2 * NB;      // ring items per segment
@@ -206,10 +217,14 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
   extern __shared__ __align__(1024) unsigned char smem[];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = (int)(blockDim.x >> 5);
-  Ring<E, S, 3, RB> ring(smem, wl, nw);
+  Ring<E, S, NARR, RB> ring(smem, wl, nw);
   ring.init(lane);
   float *sts = reinterpret_cast<float *>(smem + Sm::ring_bytes(nw)) + wl * NB * 96;
-  const CUtensorMap *const maps[3] = {&kmap, &vmap, &gmap};
+  const CUtensorMap *maps[NARR];
+  maps[0] = &kmap;
+  maps[1] = &vmap;
+  maps[2] = &gmap;
+  if constexpr (GATE) maps[NARR - 1] = &rmap;
   // The reduction counters are cleared here; the grid barrier orders these
   // stores before every increment (a workspace reused for another shape may
   // hold anything at their offset).
@@ -263,7 +278,9 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
   bool failed = false;
   int cs = 0;           // stage of the next item to consume
   uint32_t cph = 0;     // its mbarrier phase parity
-  auto take = [&](float(&K)[RB], float(&V)[RB], float(&Gy)[RB]) {
+  // Gy: the WKV output's gradient; with the gate, Gd (pass 2 only, want_d)
+  // receives grad_o sigma'(r).
+  auto take = [&](float(&K)[RB], float(&V)[RB], float(&Gy)[RB], float(&Gd)[RB], bool want_d) {
     if (!failed && !mbar_wait(ring.bar(cs), cph, budget, nullptr)) {
       failed = true;
       if (lane == 0) atomicCAS(&p.hdr->status, 0, -5 /* WKV_ERR_TIMEOUT */);
@@ -276,6 +293,21 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       K[j] = to_f32(kr[j * 32]) * kLog2e;
       V[j] = to_f32(vr[j * 32]);
       Gy[j] = to_f32(gr[j * 32]);
+    }
+    if constexpr (GATE) {
+      const E *rr = ring.stage(cs, NARR - 1) + lane;
+      if (want_d) {
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+          float sg, ds;
+          gate_sigmoid_slope(to_f32(rr[j * 32]), sg, ds);
+          Gd[j] = Gy[j] * ds;
+          Gy[j] *= sg;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < RB; ++j) Gy[j] *= gate_sigmoid(to_f32(rr[j * 32]));
+      }
     }
     __syncwarp();  // the stage is read; it may be refilled
     if (++cs == S) {
@@ -327,11 +359,12 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       sts[bt * 96 + lane] = fa;
       sts[bt * 96 + 32 + lane] = fb;
       sts[bt * 96 + 64 + lane] = fmaf(fn, w2, fP);
-      float K[RB], V[RB], Gy[RB];
-      take(K, V, Gy);
+      float K[RB], V[RB], Gy[RB], Gd[RB];
+      take(K, V, Gy, Gd, false);
       mask_tail(Gy, n - bt * RB);
       float qv[RB], gam[RB], eta[RB], e2v[RB], Mb;
-      const bool fast = recompute_batch<RB>(K, V, Gy, w2, u2, fc, fa, fb, fP, fn, qv, gam, eta, e2v, Mb);
+      const bool fast =
+          recompute_batch<RB, false>(K, V, Gy, w2, u2, fc, fa, fb, fP, fn, qv, gam, eta, e2v, Mb, Gd);
       const float lag0 = (float)(bt * RB);
       if (fast) {
         // token j's aggregate exponent is lag0 w2 - M + j (w2 - w2e): a batch
@@ -447,8 +480,8 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
 #pragma unroll 1
     for (int bi = 0; bi < NB; ++bi) {
       const int bt = NB - 1 - bi;
-      float K[RB], V[RB], Gy[RB];
-      take(K, V, Gy);
+      float K[RB], V[RB], Gy[RB], Gd[RB];
+      take(K, V, Gy, Gd, true);
       const int nb = n - bt * RB;  // valid tokens of the batch (may be <= 0 or > RB)
       mask_tail(Gy, nb);
       float qv[RB], gam[RB], eta[RB], e2v[RB], Mb;
@@ -456,7 +489,15 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       {
         float xa = sts[bt * 96 + lane], xb = sts[bt * 96 + 32 + lane], xP = sts[bt * 96 + 64 + lane];
         float xn = 0.f;
-        fast = recompute_batch<RB>(K, V, Gy, w2, u2, fc, xa, xb, xP, xn, qv, gam, eta, e2v, Mb);
+        fast = recompute_batch<RB, GATE>(K, V, Gy, w2, u2, fc, xa, xb, xP, xn, qv, gam, eta, e2v, Mb, Gd);
+      }
+      if constexpr (GATE) {  // dL/dr = grad_o sigma'(r) y
+        if (cok) {
+          E *grp = static_cast<E *>(p.gr) + ((int64_t)b * T + t0 + bt * RB) * C + c;
+#pragma unroll
+          for (int j = 0; j < RB; ++j)
+            if (j < nb) IO<E>::st(grp + (int64_t)j * C, Gd[j]);
+        }
       }
       E *gkp = static_cast<E *>(p.gk) + ((int64_t)b * T + t0 + bt * RB) * C + c;
       E *gvp = static_cast<E *>(p.gv) + ((int64_t)b * T + t0 + bt * RB) * C + c;
@@ -611,22 +652,25 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
   finish_block(p.hdr, gridDim.x);
 }
 
-template <typename E, int S, int RB>
+template <typename E, int S, int RB, bool GATE>
 static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
                                     int64_t scratch_doubles, int num_sms, int ts_max, cudaStream_t st) {
-  CUtensorMap km, vm, gm;
+  CUtensorMap km, vm, gm, rm;
   if (!encode_rows(&km, p.k, dtype, p.B * p.T, p.C, RB) || !encode_rows(&vm, p.v, dtype, p.B * p.T, p.C, RB) ||
       !encode_rows(&gm, p.gy, dtype, p.B * p.T, p.C, RB))
     return cudaErrorInvalidValue;
+  rm = gm;  // unused without the gate
+  if (GATE && !encode_rows(&rm, p.r, dtype, p.B * p.T, p.C, RB)) return cudaErrorInvalidValue;
+  constexpr int NARR = GATE ? 4 : 3;
   constexpr int kWarps = 4;
   static_assert(kCkpt % RB == 0, "checkpoints fall on batch starts");
   // Resident warps for a segment length (the per-warp batch states in shared
   // memory grow with it); the smaller occupancy of the two join variants.
   auto max_warps_for = [&](int ts, int &smem, int64_t &mw) -> cudaError_t {
-    smem = SegBwdSmem<E, S, RB>::bytes(kWarps, ts / RB);
+    smem = SegBwdSmem<E, S, RB, NARR>::bytes(kWarps, ts / RB);
     int occ = 1 << 30;
-    for (const void *kern : {(const void *)bwd_seg_kernel<E, S, RB, false>,
-                             (const void *)bwd_seg_kernel<E, S, RB, true>}) {
+    for (const void *kern : {(const void *)bwd_seg_kernel<E, S, RB, false, GATE>,
+                             (const void *)bwd_seg_kernel<E, S, RB, true, GATE>}) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
       int o = 0;
@@ -684,9 +728,9 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
   // together anyway) and chains have few segments (each fold reads all the
   // later ones); the test hook needs the flag join.
   const bool bar = rounds == 1 && a.nseg <= 32 && !p.hold_first;
-  const void *kern = bar ? (const void *)bwd_seg_kernel<E, S, RB, true>
-                         : (const void *)bwd_seg_kernel<E, S, RB, false>;
-  void *args[] = {&km, &vm, &gm, &a};
+  const void *kern = bar ? (const void *)bwd_seg_kernel<E, S, RB, true, GATE>
+                         : (const void *)bwd_seg_kernel<E, S, RB, false, GATE>;
+  void *args[] = {&km, &vm, &gm, &rm, &a};
   return cudaLaunchCooperativeKernel(kern, dim3((unsigned)grid), dim3(kWarps * 32), args, (size_t)smem, st);
 }
 
@@ -705,12 +749,25 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
 #define WKV_SEGB_RB 8
 #endif
 
+// Ring stages of the gated variant (its items carry a fourth array).
+#ifndef WKV_SEGB_S_F32_GATE
+#define WKV_SEGB_S_F32_GATE WKV_SEGB_S_F32
+#endif
+#ifndef WKV_SEGB_S_BF16_GATE
+#define WKV_SEGB_S_BF16_GATE WKV_SEGB_S_BF16
+#endif
+
 cudaError_t launch_backward_seg(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
                                 int64_t scratch_doubles, int num_sms, cudaStream_t st) {
-  return dtype == 0 ? launch_bwd_seg_t<float, WKV_SEGB_S_F32, WKV_SEGB_RB>(p, dtype, gw, gu, tile_cnt,
-                                                                            scratch_doubles, num_sms, WKV_SEGB_TS, st)
-                    : launch_bwd_seg_t<uint16_t, WKV_SEGB_S_BF16, WKV_SEGB_RB>(p, dtype, gw, gu, tile_cnt,
-                                                                               scratch_doubles, num_sms, WKV_SEGB_TS, st);
+  if (p.r)
+    return dtype == 0 ? launch_bwd_seg_t<float, WKV_SEGB_S_F32_GATE, WKV_SEGB_RB, true>(
+                            p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, WKV_SEGB_TS, st)
+                      : launch_bwd_seg_t<uint16_t, WKV_SEGB_S_BF16_GATE, WKV_SEGB_RB, true>(
+                            p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, WKV_SEGB_TS, st);
+  return dtype == 0 ? launch_bwd_seg_t<float, WKV_SEGB_S_F32, WKV_SEGB_RB, false>(
+                          p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, WKV_SEGB_TS, st)
+                    : launch_bwd_seg_t<uint16_t, WKV_SEGB_S_BF16, WKV_SEGB_RB, false>(
+                          p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, WKV_SEGB_TS, st);
 }
 
 }  // namespace wkv

@@ -102,11 +102,8 @@ cudaError_t launch_step(const StepArgs &a, bool vec, int num_sms, cudaStream_t s
   const int64_t cap = (int64_t)num_sms * 8;  // 8 blocks of 256 per SM, grid-stride beyond
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  if (vec)
-    step_kernel<true><<<(unsigned)blocks, 256, 0, st>>>(a);
-  else
-    step_kernel<false><<<(unsigned)blocks, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return vec ? launch_kernel(step_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, st, a)
+             : launch_kernel(step_kernel<false>, dim3((unsigned)blocks), dim3(256), 0, st, a);
 }
 
 }  // namespace wkv

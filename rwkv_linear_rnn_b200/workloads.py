@@ -101,14 +101,17 @@ def _uniform(rng, lo, hi, shape):
 
 
 def generate(wl: Workload | str, B: int | None = None, T: int | None = None,
-             C: int | None = None, grad: bool = True, seed: int | None = None):
+             C: int | None = None, grad: bool = True, seed: int | None = None,
+             gate: bool = False):
     """Draw one workload's inputs (host numpy arrays).
 
     Returns a dict with ``w, u`` (float32 [C]), ``k, v`` and, if ``grad``,
     ``gy`` ([B,T,C] float32 values, already rounded to bf16 for bf16
     workloads), and for bf16 workloads also ``k_bits, v_bits, gy_bits``
     (uint16 bf16 patterns).  B, T, C and seed may be overridden to draw a
-    smaller instance with the same distributions.
+    smaller instance with the same distributions.  ``gate`` adds the output
+    gate's input ``r`` (N(0, 1), drawn after everything else so the other
+    arrays do not change; ``r_bits`` for bf16).
     """
     if isinstance(wl, str):
         wl = WORKLOADS[wl]
@@ -139,6 +142,12 @@ def generate(wl: Workload | str, B: int | None = None, T: int | None = None,
     out["v"] = v
     if gy is not None:
         out["gy"] = gy
+    if gate:
+        r = _normal(rng, (B, T, C), 1.0)
+        if wl.dtype == "bf16":
+            out["r_bits"] = bf16_round(r)
+            r = bf16_to_f32(out["r_bits"])
+        out["r"] = r
     out["B"], out["T"], out["C"], out["dtype"] = B, T, C, wl.dtype
     return out
 

@@ -127,3 +127,39 @@ def test_step_validation(W):
 
 def test_get_status_null(W):
     assert W.abi.wkv_get_status(0, 0) == -3
+
+
+def test_forward_gated_validation(W):
+    a = W.abi
+    # (B, T, C, dt, w, u, k, v, r, state_in, o, state_out, ckpt, ws, ws_bytes, stream)
+    ok = [1, 8, 4, 0, FAKE, FAKE, FAKE, FAKE * 2, FAKE * 3, 0, FAKE * 4, 0, 0, 0, 0, 0]
+    bad = list(ok); bad[8] = 0
+    assert a.wkv_forward_gated(*bad) == -1                 # r NULL
+    bad = list(ok); bad[10] = 0
+    assert a.wkv_forward_gated(*bad) == -1                 # o NULL
+    bad = list(ok); bad[10] = FAKE * 3 + 16
+    assert a.wkv_forward_gated(*bad) == -2                 # o overlaps r
+    bad = list(ok); bad[10] = FAKE * 2
+    assert a.wkv_forward_gated(*bad) == -2                 # o overlaps v
+    bad = list(ok); bad[3] = 1; bad[8] = FAKE * 3 + 1
+    assert a.wkv_forward_gated(*bad) == -2                 # bf16 r odd
+    opt = a.Options(kernel=5)
+    assert a.wkv_forward_gated_ex(*ok, opt) == -1          # retired selector
+
+
+def test_backward_gated_validation(W):
+    a = W.abi
+    # (B, T, C, dt, w, u, k, v, r, go, state_in, ckpt, gw, gu, gk, gv, gr, ws, ws_bytes, stream)
+    ok = [1, 64, 32, 0, FAKE, FAKE, FAKE, FAKE * 2, FAKE * 3, FAKE * 4, 0, 0, FAKE * 5, FAKE * 6,
+          FAKE * 7, FAKE * 8, FAKE * 9, 0, 0, 0]
+    for i in (8, 9, 16):                                   # r, grad_o, grad_r NULL
+        bad = list(ok); bad[i] = 0
+        assert a.wkv_backward_gated(*bad) == -1, i
+    for clash in (FAKE, FAKE * 3, FAKE * 4, FAKE * 7, FAKE * 8):  # grad_r on an input or output
+        bad = list(ok); bad[16] = clash
+        assert a.wkv_backward_gated(*bad) == -2, clash
+    bad = list(ok); bad[14] = FAKE * 3                     # grad_k overlaps r
+    assert a.wkv_backward_gated(*bad) == -2
+    bad = list(ok); bad[16] = FAKE * 9 + 2
+    assert a.wkv_backward_gated(*bad) == -2                # grad_r misaligned
+    assert a.wkv_backward_gated(*ok) == -3                 # no workspace
