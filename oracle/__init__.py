@@ -18,6 +18,11 @@ Functions and the passages they follow (see the C file for the formulas):
 * ``bwd_recur``    -- back-propagation through the recurrence (reverse-time
                       walk, the structure of the linear-attention post's
                       gradient section).
+* ``bwd_state``    -- ``bwd_recur`` with the state terms of a sequence split
+                      across calls (truncated back-propagation through the
+                      RNN form of "RNN-유사추론"): a loss term on the final
+                      state enters as the adjoints of A_T, B_T, and the
+                      gradient of the initial state (a, b, p) comes out.
 * ``fwd_gated``    -- the review's output gating ("출력 게이팅(Output Gating)"
                       section, eq. o_t = W_o (sigma(r_t) * WKV_t)) without the
                       W_o projection: o_t = sigma(r_t) * wkv_t, elementwise.
@@ -83,6 +88,7 @@ def _load():
                                           _P, _P, _P, _P],
                 "wkv_oracle_bwd_recur": [_I, _I, _I, _P, _P, _P, _P, _P, _P,
                                          _P, _P, _P, _P],
+                "wkv_oracle_bwd_recur_state": [_I, _I, _I] + [_P] * 14,
             }
             for name, args in sigs.items():
                 fn = getattr(lib, name)
@@ -233,3 +239,47 @@ def bwd_gated(w, u, k, v, r, go, state_in=None):
     gw, gu, gk, gv = bwd_recur(w, u, k, v, _f64(go) * sr, state_in)
     gr = _f64(go) * y * sr * (1.0 - sr)
     return gw, gu, gk, gv, gr
+
+
+def bwd_state(w, u, k, v, gy, state_in=None, state_out=None, grad_state_out=None):
+    """``bwd_recur`` with the recurrent state's gradients; returns
+    (gw, gu, gk, gv, grad_state_in [3, B, C]).
+
+    ``grad_state_out`` [3, B, C] is dL/d(a, b, p) of the state after the last
+    token in the representation ``state_out`` (any (a, b, p) of that state:
+    only its p is read).  The loss is taken to depend on the state only
+    through the sums it represents, A = a e^p and B = b e^p, so
+    dL/dA_T = ga e^{-p}, dL/dB_T = gb e^{-p}, and the p component (then
+    a ga + b gb, no extra information) is not read.  An empty state
+    (p = -inf) passes no gradient.  ``grad_state_in`` is dL/d(a, b, p) of
+    ``state_in`` exactly as given: (dL/dA_0 e^p, dL/dB_0 e^p,
+    A_0 dL/dA_0 + B_0 dL/dB_0); zeros for ``state_in=None`` (the empty
+    state, p = -inf).
+    """
+    w, u, k, v, gy = _f64(w), _f64(u), _f64(k), _f64(v), _f64(gy)
+    s = None if state_in is None else _f64(state_in)
+    B, T, C = _shape3(k)
+    gA_T = gB_T = None
+    if grad_state_out is not None:
+        if state_out is None:
+            raise ValueError("grad_state_out needs the state_out it refers to")
+        go, so = _f64(grad_state_out), _f64(state_out)
+        p = so[2]
+        with np.errstate(over="ignore", invalid="ignore"):
+            scale = np.where(np.isneginf(p), 0.0, np.exp(-np.where(np.isneginf(p), 0.0, p)))
+        gA_T = np.ascontiguousarray(go[0] * scale)
+        gB_T = np.ascontiguousarray(go[1] * scale)
+    gw, gu = np.empty(C), np.empty(C)
+    gk, gv = np.empty((B, T, C)), np.empty((B, T, C))
+    gA_0, gB_0 = np.empty((B, C)), np.empty((B, C))
+    _load().wkv_oracle_bwd_recur_state(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(s),
+                                       _ptr(gy), _ptr(gA_T), _ptr(gB_T), _ptr(gw), _ptr(gu),
+                                       _ptr(gk), _ptr(gv), _ptr(gA_0), _ptr(gB_0))
+    gs_in = np.zeros((3, B, C))
+    if s is not None:
+        a, b, p = s[0], s[1], s[2]
+        e = np.exp(p)  # 0 for an empty state
+        gs_in[0] = gA_0 * e
+        gs_in[1] = gB_0 * e
+        gs_in[2] = a * gs_in[0] + b * gs_in[1]  # A_0 dL/dA_0 + B_0 dL/dB_0
+    return gw, gu, gk, gv, gs_in

@@ -364,3 +364,73 @@ void wkv_oracle_bwd_recur(int64_t B, int64_t T, int64_t C, const double *w,
   free(pw);
   free(pu);
 }
+
+/*
+ * Back-propagation through the recurrence with the state terms, for
+ * sequences split across calls (truncated BPTT, the RNN mode of [RWKV
+ * review] "RNN-유사추론" carried between calls):
+ *   gA_T, gB_T  [B][C] dL/dA_T, dL/dB_T for the hidden sums after the last
+ *               token (NULL: no loss term on the final state);
+ *   gA_0, gB_0  [B][C] receive dL/dA_0, dL/dB_0 for the sums before token 0
+ *               (NULL: not wanted).
+ * The same reverse walk as wkv_oracle_bwd_recur, started from the given
+ * adjoints instead of zero; every other output is as there.
+ */
+void wkv_oracle_bwd_recur_state(int64_t B, int64_t T, int64_t C, const double *w,
+                                const double *u, const double *k, const double *v,
+                                const double *state_in, const double *gy, const double *gA_T,
+                                const double *gB_T, double *gw, double *gu, double *gk,
+                                double *gv, double *gA_0, double *gB_0) {
+  double *pw = (double *)calloc((size_t)(B * C), sizeof(double));
+  double *pu = (double *)calloc((size_t)(B * C), sizeof(double));
+#pragma omp parallel
+  {
+    double *As = (double *)malloc(sizeof(double) * (size_t)(T + 1));
+    double *Bv = (double *)malloc(sizeof(double) * (size_t)(T + 1));
+#pragma omp for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b)
+      for (int64_t c = 0; c < C; ++c) {
+        const double wc = w[c], uc = u[c], ew = exp(wc);
+        initial_sums(state_in, B, C, b, c, &As[0], &Bv[0]);
+        for (int64_t t = 0; t < T; ++t) {
+          const double e_k = exp(k[IDX(b, t, c)]);
+          As[t + 1] = ew * As[t] + e_k * v[IDX(b, t, c)];
+          Bv[t + 1] = ew * Bv[t] + e_k;
+        }
+        /* adjoints of A_T, B_T: the loss term on the final state */
+        double Ah = gA_T ? gA_T[b * C + c] : 0.0;
+        double Bh = gB_T ? gB_T[b * C + c] : 0.0;
+        double sw = 0.0, su = 0.0;
+        for (int64_t t = T - 1; t >= 0; --t) {
+          const double kt = k[IDX(b, t, c)], vt = v[IDX(b, t, c)];
+          const double g = gy[IDX(b, t, c)];
+          const double e_cur = exp(uc + kt), e_k = exp(kt);
+          const double D = Bv[t] + e_cur;
+          const double yt = (As[t] + e_cur * vt) / D;
+          gv[IDX(b, t, c)] = g * e_cur / D + e_k * Ah;
+          gk[IDX(b, t, c)] = g * e_cur * (vt - yt) / D + e_k * (vt * Ah + Bh);
+          su += g * e_cur * (vt - yt) / D;
+          sw += ew * (As[t] * Ah + Bv[t] * Bh);
+          Ah = g / D + ew * Ah;
+          Bh = -g * yt / D + ew * Bh;
+        }
+        pw[b * C + c] = sw;
+        pu[b * C + c] = su;
+        if (gA_0) gA_0[b * C + c] = Ah;
+        if (gB_0) gB_0[b * C + c] = Bh;
+      }
+    free(As);
+    free(Bv);
+  }
+  for (int64_t c = 0; c < C; ++c) {
+    double sw = 0.0, su = 0.0;
+    for (int64_t b = 0; b < B; ++b) {
+      sw += pw[b * C + c];
+      su += pu[b * C + c];
+    }
+    gw[c] = sw;
+    gu[c] = su;
+  }
+  free(pw);
+  free(pu);
+}
