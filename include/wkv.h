@@ -21,8 +21,9 @@
  *   wkv_backward  gradients of a scalar loss for the same mode;
  *   wkv_step      RNN mode ("RNN-유사추론" / "자기 회귀 디코딩" steps 4 and 7):
  *                 one token per sequence against a stored state.
- * wkv_forward_gated / wkv_backward_gated add the receptance gate
- * o = sigma(r) * y of the time-mixing block's output.
+ * wkv_backward_state adds the gradients through the recurrent state for
+ * sequences split across calls; wkv_forward_gated / wkv_backward_gated add
+ * the receptance gate o = sigma(r) * y of the time-mixing block's output.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -206,6 +207,47 @@ int wkv_backward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
                     const void *grad_y, const float *state_in, const float *ckpt,
                     float *grad_w, float *grad_u, void *grad_k, void *grad_v,
                     void *ws, size_t ws_bytes, void *stream, const wkv_options *opt);
+
+/*
+ * wkv_backward_state -- wkv_backward with the state terms of a sequence
+ * split across calls (truncated back-propagation through time: the RNN form
+ * of the RWKV review, section "RNN-유사추론", carried from one call to the
+ * next through state_in / state_out).
+ *   state_out       [3][B][C] the state after the last token in the
+ *                   representation grad_state_out refers to: the forward's
+ *                   state_out, or any (a, b, p) of that state.  Only its p
+ *                   plane is read.  Required when grad_state_out is given.
+ *   grad_state_out  [3][B][C] float32 dL/d(a, b, p) of that state, or NULL
+ *                   (no loss term on the final state).  The loss is taken to
+ *                   depend on a state only through the sums it represents,
+ *                   A = a e^p and B = b e^p (true of every call of this
+ *                   library), so dL/dA = ga e^{-p}, dL/dB = gb e^{-p}; the p
+ *                   component carries nothing more (it equals a ga + b gb)
+ *                   and is not read.  An empty state (p = -inf) passes no
+ *                   gradient.
+ *   grad_state_in   [3][B][C] float32 output dL/d(a, b, p) of state_in as
+ *                   given: (dL/dA_0 e^p, dL/dB_0 e^p, a dL/da + b dL/db), or
+ *                   NULL.  Zeros when state_in is NULL (the empty state).
+ *                   Must not overlap any other argument.
+ * Everything else is as in wkv_backward; grad_w also receives the final-state
+ * term's share.  Chaining: a call's grad_state_in, passed with its state_in
+ * as the previous call's grad_state_out and state_out, gives that call the
+ * gradients a single call over both ranges would give.
+ * Errors: as wkv_backward; grad_state_out without state_out is INVALID_ARG.
+ */
+int wkv_backward_state(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                       const float *u, const void *k, const void *v, const void *grad_y,
+                       const float *state_in, const float *ckpt, const float *state_out,
+                       const float *grad_state_out, float *grad_w, float *grad_u,
+                       void *grad_k, void *grad_v, float *grad_state_in, void *ws,
+                       size_t ws_bytes, void *stream);
+
+int wkv_backward_state_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
+                          const float *u, const void *k, const void *v, const void *grad_y,
+                          const float *state_in, const float *ckpt, const float *state_out,
+                          const float *grad_state_out, float *grad_w, float *grad_u,
+                          void *grad_k, void *grad_v, float *grad_state_in, void *ws,
+                          size_t ws_bytes, void *stream, const wkv_options *opt);
 
 /*
  * wkv_forward_gated -- the time-mixing output with its receptance gate:

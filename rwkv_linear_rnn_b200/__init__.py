@@ -3,7 +3,7 @@
 Thin Python binding over the C ABI in ``include/wkv.h``.  The functions in
 ``abi`` carry the C names and take raw device pointers (ints) -- argument
 marshalling only.  The tensor helpers below (``forward``, ``backward``,
-``step``, ``WKV`` and the gated ``forward_gated``, ``backward_gated``,
+``step``, ``WKV``, ``backward_state`` and the gated ``forward_gated``, ``backward_gated``,
 ``GatedWKV``) take torch CUDA tensors, allocate outputs with torch, and
 call the same entry points; PyTorch provides memory and streams only, every
 step of the operator runs in the library's CUDA kernels.
@@ -24,8 +24,8 @@ from .constants import (WKV_BF16, WKV_F32, WKV_KERNEL_AUTO, WKV_KERNEL_CHUNKED,
 __all__ = [
     "abi", "WKVError", "WKV_F32", "WKV_BF16", "WKV_OP_FORWARD", "WKV_OP_BACKWARD", "WKV_OP_STEP",
     "WKV_KERNEL_AUTO", "WKV_KERNEL_SEQUENTIAL", "WKV_KERNEL_CHUNKED", "WKV_KERNEL_CHUNKED_REGS",
-    "WKV_KERNEL_SEGMENT", "WKV_KERNEL_CLUSTER", "WKV_STATIC_SCRATCH_BYTES", "Workspace", "forward", "backward", "step",
-    "forward_gated", "backward_gated", "WKV", "wkv", "GatedWKV", "gated_wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror", "wkv_version",
+    "WKV_KERNEL_SEGMENT", "WKV_KERNEL_CLUSTER", "WKV_STATIC_SCRATCH_BYTES", "Workspace", "forward", "backward", "backward_state", "step",
+    "forward_gated", "backward_gated", "WKV", "wkv", "WKVState", "wkv_state", "GatedWKV", "gated_wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror", "wkv_version",
     "library_path",
 ]
 
@@ -186,6 +186,35 @@ def backward(w, u, k, v, grad_y, state_in=None, ckpt=None, *, grad_k=None, grad_
     return gw, gu, gk, gv
 
 
+def backward_state(w, u, k, v, grad_y, state_in=None, ckpt=None, *, state_out=None,
+                   grad_state_out=None, want_grad_state_in=True, grad_k=None, grad_v=None,
+                   workspace=None, stream=None, kernel=WKV_KERNEL_AUTO):
+    """``backward`` with the state terms of a sequence split across calls.
+    ``grad_state_out`` is dL/d(a, b, p) of the state after the last token,
+    given in the representation ``state_out`` (only its p is read).  Returns
+    (grad_w, grad_u, grad_k, grad_v, grad_state_in); grad_state_in is
+    dL/d(a, b, p) of ``state_in`` as given (None unless wanted)."""
+    torch = _torch()
+    _check_cuda(w, u, k, v, grad_y, state_in, ckpt, state_out, grad_state_out, grad_k, grad_v)
+    B, T, C = k.shape
+    dt = _dtype_code(k)
+    gw = torch.empty(C, dtype=torch.float32, device=k.device)
+    gu = torch.empty(C, dtype=torch.float32, device=k.device)
+    gk = torch.empty_like(k) if grad_k is None else grad_k
+    gv = torch.empty_like(v) if grad_v is None else grad_v
+    gs = torch.empty((3, B, C), dtype=torch.float32, device=k.device) if want_grad_state_in else None
+    ws = _ws_for(k.device, workspace)
+    buf, nbytes = ws.get(WKV_OP_BACKWARD, B, T, C, dt)
+    abi = _abi()
+    opts = abi.Options(kernel=kernel)
+    abi.check(abi.wkv_backward_state_ex(B, T, C, dt, _ptr(w), _ptr(u), _ptr(k), _ptr(v),
+                                        _ptr(grad_y), _ptr(state_in), _ptr(ckpt), _ptr(state_out),
+                                        _ptr(grad_state_out), _ptr(gw), _ptr(gu), _ptr(gk),
+                                        _ptr(gv), _ptr(gs), _ptr(buf), nbytes, _stream(stream),
+                                        opts))
+    return gw, gu, gk, gv, gs
+
+
 def forward_gated(w, u, k, v, r, state_in=None, *, want_state=False, want_ckpt=False, o=None,
                   workspace=None, stream=None, kernel=WKV_KERNEL_AUTO):
     """o = sigmoid(r) * WKV(w, u, k, v) for k, v, r [B, T, C].  Returns
@@ -283,6 +312,45 @@ class WKV:
 def wkv(w, u, k, v):
     """Differentiable WKV: y [B, T, C] from w, u [C] and k, v [B, T, C]."""
     return WKV.apply(w, u, k, v)
+
+
+class WKVState:
+    """torch.autograd.Function wrapper with the recurrent state:
+    (y, state_out) = WKVState.apply(w, u, k, v, state_in).  Gradients reach
+    state_in through both y and state_out, so a sequence split across calls
+    back-propagates through the state (truncated BPTT)."""
+
+    _fn = None
+
+    @classmethod
+    def apply(cls, w, u, k, v, state_in):
+        if cls._fn is None:
+            torch = _torch()
+
+            class _F(torch.autograd.Function):
+                @staticmethod
+                def forward(ctx, w, u, k, v, state_in):
+                    w, u, k, v, state_in = (t.contiguous() for t in (w, u, k, v, state_in))
+                    y, s_out, ck = forward(w, u, k, v, state_in, want_state=True, want_ckpt=True)
+                    ctx.save_for_backward(w, u, k, v, state_in, s_out, ck)
+                    return y, s_out
+
+                @staticmethod
+                def backward(ctx, gy, gs):
+                    w, u, k, v, state_in, s_out, ck = ctx.saved_tensors
+                    gy = torch.zeros_like(k) if gy is None else gy.contiguous()
+                    gs = None if gs is None else gs.contiguous()
+                    return backward_state(w, u, k, v, gy, state_in, ck, state_out=s_out,
+                                          grad_state_out=gs)
+
+            cls._fn = _F
+        return cls._fn.apply(w, u, k, v, state_in)
+
+
+def wkv_state(w, u, k, v, state_in):
+    """Differentiable WKV with the state: (y, state_out) from w, u [C],
+    k, v [B, T, C] and state_in [3, B, C]."""
+    return WKVState.apply(w, u, k, v, state_in)
 
 
 class GatedWKV:

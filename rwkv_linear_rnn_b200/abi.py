@@ -20,7 +20,8 @@ from .constants import WKV_ERR_CUDA, WKV_OK
 # Every symbol the header declares, in declaration order.
 EXPORTS = (
     "wkv_workspace_size", "wkv_workspace_init", "wkv_ckpt_size", "wkv_forward", "wkv_forward_ex",
-    "wkv_backward", "wkv_backward_ex", "wkv_forward_gated", "wkv_forward_gated_ex",
+    "wkv_backward", "wkv_backward_ex", "wkv_backward_state", "wkv_backward_state_ex",
+    "wkv_forward_gated", "wkv_forward_gated_ex",
     "wkv_backward_gated", "wkv_backward_gated_ex", "wkv_step", "wkv_backward_static", "wkv_get_status",
     "wkv_strerror", "wkv_last_cuda_error", "wkv_cuda_error_name", "wkv_version",
 )
@@ -52,6 +53,8 @@ _SIGS = {
                             _p, _sz, _p]),
     "wkv_backward_ex": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                _p, _p, _sz, _p, _opt]),
+    "wkv_backward_state": (_int, [_i64, _i64, _i64, _int] + [_p] * 15 + [_sz, _p]),
+    "wkv_backward_state_ex": (_int, [_i64, _i64, _i64, _int] + [_p] * 15 + [_sz, _p, _opt]),
     "wkv_forward_gated": (_int, [_i64, _i64, _i64, _int] + [_p] * 10 + [_sz, _p]),
     "wkv_forward_gated_ex": (_int, [_i64, _i64, _i64, _int] + [_p] * 10 + [_sz, _p, _opt]),
     "wkv_backward_gated": (_int, [_i64, _i64, _i64, _int] + [_p] * 14 + [_sz, _p]),
@@ -118,6 +121,22 @@ def wkv_backward_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, 
                     grad_v, ws, ws_bytes, stream, opt=None):
     return lib.wkv_backward_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u,
                                grad_k, grad_v, ws, ws_bytes, stream, _opts(opt))
+
+
+def wkv_backward_state(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, state_out,
+                       grad_state_out, grad_w, grad_u, grad_k, grad_v, grad_state_in, ws, ws_bytes,
+                       stream):
+    return lib.wkv_backward_state(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, state_out,
+                                  grad_state_out, grad_w, grad_u, grad_k, grad_v, grad_state_in, ws,
+                                  ws_bytes, stream)
+
+
+def wkv_backward_state_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, state_out,
+                          grad_state_out, grad_w, grad_u, grad_k, grad_v, grad_state_in, ws,
+                          ws_bytes, stream, opt=None):
+    return lib.wkv_backward_state_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt,
+                                     state_out, grad_state_out, grad_w, grad_u, grad_k, grad_v,
+                                     grad_state_in, ws, ws_bytes, stream, _opts(opt))
 
 
 def wkv_forward_gated(B, T, C, dtype, w, u, k, v, r, state_in, o, state_out, ckpt, ws, ws_bytes,

@@ -22,6 +22,8 @@ cudaError_t launch_backward(const BwdArgs &a, int dtype, float *gw, float *gu, c
 cudaError_t launch_step(const StepArgs &a, bool vec, int num_sms, cudaStream_t st);
 cudaError_t launch_gate(int op, int dtype, void *x, const void *go, const void *r, int64_t n, int num_sms,
                         cudaStream_t st);
+cudaError_t launch_state_grad_t0(const float *gs_out, const float *p_out, const float *s_in, float *gs_in,
+                                 int64_t BC, int num_sms, cudaStream_t st);
 int64_t fwd_chunk_tokens();
 }  // namespace wkv
 
@@ -232,16 +234,27 @@ int check_backward_args(int64_t B, int64_t T, int64_t C, int dtype, const float 
   return WKV_OK;
 }
 
+// State terms of a backward (all null when unused): the final state's
+// gradient with the p plane of the representation it refers to, and the
+// output for the initial state's gradient.
+struct StateTerms {
+  const float *gs_out = nullptr, *p_out = nullptr;
+  float *gs_in = nullptr;
+};
+
 // Backward after the checks.  r, gr: gate input and its gradient for the
 // fused gated segment backward (grad_y is then dL/do), else NULL.
 int backward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
                   const void *k, const void *v, const void *grad_y, const float *state_in,
                   const float *ckpt, float *grad_w, float *grad_u, void *grad_k, void *grad_v,
                   void *ws, size_t ws_bytes, cudaStream_t st, const wkv_options *opt,
-                  const void *r = nullptr, void *gr = nullptr) {
+                  const void *r = nullptr, void *gr = nullptr, const StateTerms &sg = StateTerms()) {
   if (T == 0) {
-    const int rc = cuda_rc(cudaMemsetAsync(grad_w, 0, sizeof(float) * C, st));
-    return rc != WKV_OK ? rc : cuda_rc(cudaMemsetAsync(grad_u, 0, sizeof(float) * C, st));
+    int rc = cuda_rc(cudaMemsetAsync(grad_w, 0, sizeof(float) * C, st));
+    if (rc == WKV_OK) rc = cuda_rc(cudaMemsetAsync(grad_u, 0, sizeof(float) * C, st));
+    if (rc == WKV_OK && sg.gs_in)
+      rc = cuda_rc(launch_state_grad_t0(sg.gs_out, sg.p_out, state_in, sg.gs_in, B * C, num_sms(), st));
+    return rc;
   }
   const Layout L = layout(WKV_OP_BACKWARD, B, T, C);
   if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return WKV_ERR_WORKSPACE;
@@ -267,6 +280,10 @@ int backward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, co
   a.hold_first = opt ? opt->test_hold_first_chunk : 0;
   a.r = r;
   a.gr = gr;
+  a.gs_out = sg.gs_out;
+  a.p_out = sg.p_out;
+  a.gs_in = sg.gs_in;
+  a.state_in = state_in;
   if (bwd_uses_seg(B, T, C, dtype, k, v, grad_y, opt)) {
     const int64_t scratch = (int64_t)(L.desc_bytes / sizeof(double));
     return cuda_rc(launch_backward_seg(a, dtype, grad_w, grad_u, reinterpret_cast<unsigned *>(base + L.cnt), scratch,
@@ -334,6 +351,48 @@ int wkv_backward(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
                  void *ws, size_t ws_bytes, void *stream) {
   return wkv_backward_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u,
                          grad_k, grad_v, ws, ws_bytes, stream, nullptr);
+}
+
+int wkv_backward_state_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                          const void *k, const void *v, const void *grad_y, const float *state_in,
+                          const float *ckpt, const float *state_out, const float *grad_state_out,
+                          float *grad_w, float *grad_u, void *grad_k, void *grad_v, float *grad_state_in,
+                          void *ws, size_t ws_bytes, void *stream, const wkv_options *opt) {
+  const int rc = check_backward_args(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u,
+                                     grad_k, grad_v, opt);
+  if (rc != WKV_OK) return rc;
+  if (grad_state_out && !state_out) return WKV_ERR_INVALID_ARG;
+  if (!aligned(state_out, 4) || !aligned(grad_state_out, 4) || !aligned(grad_state_in, 4))
+    return WKV_ERR_UNSUPPORTED;
+  const size_t es = esize(dtype), nb = (size_t)(B * T * C) * es, sb = 3 * sizeof(float) * (size_t)(B * C);
+  if (grad_state_in) {
+    const void *big[4] = {k, v, grad_y, ckpt};
+    for (const void *x : big)
+      if (overlaps(grad_state_in, sb, x, x == ckpt ? wkv_ckpt_size(B, T, C) : nb)) return WKV_ERR_UNSUPPORTED;
+    const void *st3[3] = {state_in, state_out, grad_state_out};
+    for (const void *x : st3)
+      if (overlaps(grad_state_in, sb, x, sb)) return WKV_ERR_UNSUPPORTED;
+    if (overlaps(grad_state_in, sb, grad_k, nb) || overlaps(grad_state_in, sb, grad_v, nb) ||
+        overlaps(grad_state_in, sb, grad_w, 4 * C) || overlaps(grad_state_in, sb, grad_u, 4 * C))
+      return WKV_ERR_UNSUPPORTED;
+  }
+  if (grad_state_out && (overlaps(grad_k, nb, grad_state_out, sb) || overlaps(grad_v, nb, grad_state_out, sb)))
+    return WKV_ERR_UNSUPPORTED;
+  StateTerms sg;
+  sg.gs_out = grad_state_out;
+  sg.p_out = grad_state_out ? state_out + 2 * B * C : nullptr;
+  sg.gs_in = grad_state_in;
+  return backward_impl(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u, grad_k, grad_v, ws,
+                       ws_bytes, (cudaStream_t)stream, opt, nullptr, nullptr, sg);
+}
+
+int wkv_backward_state(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,
+                       const void *k, const void *v, const void *grad_y, const float *state_in,
+                       const float *ckpt, const float *state_out, const float *grad_state_out, float *grad_w,
+                       float *grad_u, void *grad_k, void *grad_v, float *grad_state_in, void *ws,
+                       size_t ws_bytes, void *stream) {
+  return wkv_backward_state_ex(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, state_out, grad_state_out,
+                               grad_w, grad_u, grad_k, grad_v, grad_state_in, ws, ws_bytes, stream, nullptr);
 }
 
 int wkv_forward_gated_ex(int64_t B, int64_t T, int64_t C, int dtype, const float *w, const float *u,

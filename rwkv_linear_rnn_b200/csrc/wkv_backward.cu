@@ -194,9 +194,18 @@ __global__ void __launch_bounds__(W * 32) bwd_chunked_kernel(BwdArgs p) {
       const int li = (int)max((int64_t)0, min((int64_t)L, T - (tc0 + (int64_t)i * L)));
       acc = rcombine(ai, acc, (float)li, w2);
     }
-    const Adj excl = chunk_scan(p.flags, p.desc, rpos, chain, p.nchains, acc, (float)chunk_len,
-                                (float)TC, adj_empty(), adj_empty(), epoch, p.hdr, p.spin_limit,
-                                rpos + 1 < p.nchunks, !(p.hold_first && rpos == 0), w2, lane);
+    Adj excl = chunk_scan(p.flags, p.desc, rpos, chain, p.nchains, acc, (float)chunk_len, (float)TC,
+                          adj_empty(), adj_empty(), epoch, p.hdr, p.spin_limit, rpos + 1 < p.nchunks,
+                          !(p.hold_first && rpos == 0), w2, lane);
+    // the adjoint after the last token (a loss term on the final state, if
+    // any) decays across the tokens after this chunk (the scan counts every
+    // later chunk as full, so it is joined here with the exact count)
+    if (p.gs_out && cok) {
+      const int64_t bc = b * C + c;
+      Adj fin;
+      end_adjoint(p.gs_out[bc], p.gs_out[BC + bc], p.p_out[bc], fin.ah, fin.hh, fin.r);
+      excl = rcombine(excl, fin, (float)(T - tc0 - chunk_len), w2);
+    }
     s_carry[0][lane] = excl.ah;
     s_carry[1][lane] = excl.hh;
     s_carry[2][lane] = excl.r;
@@ -240,6 +249,8 @@ __global__ void __launch_bounds__(W * 32) bwd_chunked_kernel(BwdArgs p) {
         m = reset ? 0.f : m1;
       }
     }
+    // warp 0 of the first chunk ends at token 0: the initial state's gradient
+    if (p.gs_in && cok && t0 == 0) store_state_grad(p.gs_in, p.state_in, b * C + c, BC, ah, hh, fmaf(-m, w2, Ranc));
   }
   s_g[0][wi][lane] = gw;
   s_g[1][wi][lane] = gu;
@@ -286,6 +297,35 @@ __global__ void __launch_bounds__(256) reduce_wu_kernel(const float *part, int64
     gw[c] = (float)tw;
     gu[c] = (float)tu;
   }
+}
+
+// T = 0: the state passes through unchanged, so the initial state's
+// gradient is the final state's, moved from the representation with
+// exponent p_out to the caller's state_in: dL/d(a, b) scale by e^{p_in -
+// p_out}, dL/dp = a dL/da + b dL/db.  gs_out null, an empty final state or
+// a null state_in give zeros.
+__global__ void __launch_bounds__(256) state_grad_t0_kernel(const float *gs_out, const float *p_out,
+                                                            const float *s_in, float *gs_in, int64_t BC) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < BC; i += (int64_t)gridDim.x * blockDim.x) {
+    float ga = 0.f, gb = 0.f, gp = 0.f;
+    if (gs_out && s_in && p_out[i] != -INFINITY) {
+      const float f = expf(s_in[2 * BC + i] - p_out[i]);
+      ga = gs_out[i] * f;
+      gb = gs_out[BC + i] * f;
+      gp = fmaf(s_in[i], ga, s_in[BC + i] * gb);
+    }
+    gs_in[i] = ga;
+    gs_in[BC + i] = gb;
+    gs_in[2 * BC + i] = gp;
+  }
+}
+
+cudaError_t launch_state_grad_t0(const float *gs_out, const float *p_out, const float *s_in, float *gs_in,
+                                 int64_t BC, int num_sms, cudaStream_t st) {
+  const int64_t want = (BC + 255) / 256;
+  const int64_t grid = want < (int64_t)num_sms * 8 ? want : (int64_t)num_sms * 8;
+  return launch_kernel(state_grad_t0_kernel, dim3((unsigned)(grid > 0 ? grid : 1)), dim3(256), 0, st, gs_out,
+                       p_out, s_in, gs_in, BC);
 }
 
 // ---------------------------------------------------------------- launch ---

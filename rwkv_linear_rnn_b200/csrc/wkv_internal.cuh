@@ -521,7 +521,51 @@ struct BwdArgs {
   int hold_first;
   const void *r;  // output gate input (grad_y is then the gated output's gradient), or null
   void *gr;       // gradient of the gate input (with r)
+  // State terms of a sequence split across calls (all null when unused):
+  const float *gs_out;    // [3][B][C] dL/d(a, b, p) of the state after the last token
+  const float *p_out;     // [B][C] the p plane of the representation gs_out refers to
+  float *gs_in;           // [3][B][C] receives dL/d(a, b, p) of state_in
+  const float *state_in;  // the caller's initial state as given (null: empty)
 };
+
+// Adjoint of the final sums from dL/d(a, b) of a state representation with
+// exponent p (natural log): dL/dA_T = ga e^{-p}, dL/dB_T = gb e^{-p}, held as
+// Ahat = ah 2^{-r}, Hhat = hh 2^{-r} (Hhat = -dL/dB) scaled by an exact power
+// of two so that |ah| + |hh| lies in [1, 2) (the adjoint joins pick their
+// anchor from r and assume normalised values).  Zero gradients and an empty
+// state (p = -inf) give the empty adjoint; NaN and inf pass unscaled.
+__device__ __forceinline__ void end_adjoint(float ga, float gb, float p, float &ah, float &hh, float &r) {
+  const float m = fabsf(ga) + fabsf(gb);
+  if (m == 0.f || p == -INFINITY) {
+    ah = 0.f;
+    hh = 0.f;
+    r = kEmptyR;
+    return;
+  }
+  const int e = m < INFINITY ? ilogbf(m) : 0;
+  ah = ldexpf(ga, -e);
+  hh = -ldexpf(gb, -e);
+  r = fmaf(p, kLog2e, -(float)e);
+}
+
+// dL/d(a, b, p) of the caller's initial state (a, b, p) from the adjoint of
+// the initial sums, Ahat_0 = ah 2^{-r0}, Hhat_0 = hh 2^{-r0}:
+// dL/da = Ahat_0 e^p, dL/db = -Hhat_0 e^p, dL/dp = a dL/da + b dL/db.
+// s_in null (the empty state) gives zeros.
+__device__ __forceinline__ void store_state_grad(float *gs, const float *s_in, int64_t bc, int64_t BC,
+                                                 float ah, float hh, float r0) {
+  float ga = 0.f, gb = 0.f, gp = 0.f;
+  if (s_in) {
+    const float a = s_in[bc], b = s_in[BC + bc], p = s_in[2 * BC + bc];
+    const float f = ex2(fmaf(p, kLog2e, -r0));
+    ga = ah * f;
+    gb = -hh * f;
+    gp = fmaf(a, ga, b * gb);
+  }
+  gs[bc] = ga;
+  gs[BC + bc] = gb;
+  gs[2 * BC + bc] = gp;
+}
 
 struct StepArgs {
   int64_t N, C;

@@ -202,7 +202,13 @@ struct SegBwdSmem {
 // GATE: the loss depends on o = sigma(r) * y; the ring items carry r as a
 // fourth tensor, the WKV gradient is grad_o sigma(r) and pass 2 also writes
 // dL/dr = grad_o y sigma'(r).
-template <typename E, int S, int RB, bool BAR, bool GATE>
+// STATE: the state terms of a sequence split across calls: the folds start
+// from the adjoint after the last token (the final state's gradient), the
+// last segment's sweep stops exactly at token T-1 (its padding would decay
+// that adjoint), and the first segment writes the initial state's gradient.
+// A variant of its own so that the common path keeps its instruction
+// schedule.
+template <typename E, int S, int RB, bool BAR, bool GATE, bool STATE>
 __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __grid_constant__ CUtensorMap kmap,
                                                       const __grid_constant__ CUtensorMap vmap,
                                                       const __grid_constant__ CUtensorMap gmap,
@@ -411,7 +417,12 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
     const Adj5s agg{ah, hh, ahp, hhp, -Em};
 
     const int nlast = (int)(T - (nseg - 1) * TS);  // tokens of the chain's last segment
+    // the adjoint after the chain's last token (a loss term on the final
+    // state, if any): the start of every fold
     Adj5s acc = adj5s_empty();
+    if constexpr (STATE) {
+      if (p.gs_out && cok) end_adjoint(p.gs_out[bc], p.gs_out[BC + bc], p.p_out[bc], acc.ah, acc.hh, acc.r);
+    }
     if constexpr (BAR) {
       // ---- join after the grid barrier: fold the later segments in order
       if (has && rpos + 1 < nseg) rec_store_adj(p.desc, unit, agg, lane);
@@ -505,9 +516,16 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       // obeys a_t = gam_t + ewm a_{t+1} (and a'_t = ewm (a'_{t+1} + a_{t+1}) for
       // the lag-weighted one); e^{k_t} A_{t+1} = ek_t a_{t+1}.  The carried
       // adjoint enters scaled by 2^{M + RB w2e - r}, bounded for the float range.
+      if constexpr (STATE) {
+        if (nb <= 0) continue;  // only tokens past T (a chain's last segment): nothing to sweep
+      }
       const float rn_end = fmaf(-m, w2, Ranc);
       const float xin = fmaf((float)RB, fc.w2e, Mb) - rn_end;
-      if (__all_sync(0xffffffffu, fast && xin < 100.f)) {
+      // (with STATE a partial batch takes the per-token sweep, which stops at
+      // the last token: the carried adjoint starts after token T-1, not after
+      // the batch's padding; without it the adjoint there is zero and the
+      // padding, whose gradient is masked, adds nothing)
+      if (__all_sync(0xffffffffu, fast && xin < 100.f && (!STATE || nb >= RB))) {
         const float F = ex2(xin);
         float ra = rah * F, rh = rhh * F, rap = rahp * F, rhp = rhhp * F;
         const float ck = fc.cw * ex2(-u2);  // ek = e2 * ck
@@ -542,6 +560,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       }
 #pragma unroll
       for (int j = RB - 1; j >= 0; --j) {
+        if (STATE && j >= nb) continue;  // past T
         const float rn = fmaf(-m, w2, Ranc);  // scale of the adjoint after token t
         const float tn = ex2(K[j] - rn);      // e^{k_t} 2^{-r_{t+1}} (<= 1)
         const float gv = fmaf(gam[j], e2v[j], tn * rah);
@@ -572,6 +591,9 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
         const float *ck = p.ckpt + bc;
         const float r0 = fmaf(-m, w2, Ranc);
         gw_acc = fmaf(ex2(ck[2 * BC] - r0), fmaf(ck[0], rahp, -ck[BC] * rhhp), gw_acc);
+      }
+      if constexpr (STATE) {
+        if (t0 == 0 && p.gs_in) store_state_grad(p.gs_in, p.state_in, bc, BC, rah, rhh, fmaf(-m, w2, Ranc));
       }
       p.part[(int64_t)(pos * 2 + 0) * BC + bc] = gw_acc;
       p.part[(int64_t)(pos * 2 + 1) * BC + bc] = gu_acc;
@@ -652,7 +674,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
   finish_block(p.hdr, gridDim.x);
 }
 
-template <typename E, int S, int RB, bool GATE>
+template <typename E, int S, int RB, bool GATE, bool STATE>
 static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
                                     int64_t scratch_doubles, int num_sms, int ts_max, cudaStream_t st) {
   CUtensorMap km, vm, gm, rm;
@@ -669,8 +691,8 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
   auto max_warps_for = [&](int ts, int &smem, int64_t &mw) -> cudaError_t {
     smem = SegBwdSmem<E, S, RB, NARR>::bytes(kWarps, ts / RB);
     int occ = 1 << 30;
-    for (const void *kern : {(const void *)bwd_seg_kernel<E, S, RB, false, GATE>,
-                             (const void *)bwd_seg_kernel<E, S, RB, true, GATE>}) {
+    for (const void *kern : {(const void *)bwd_seg_kernel<E, S, RB, false, GATE, STATE>,
+                             (const void *)bwd_seg_kernel<E, S, RB, true, GATE, STATE>}) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
       int o = 0;
@@ -728,8 +750,8 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
   // together anyway) and chains have few segments (each fold reads all the
   // later ones); the test hook needs the flag join.
   const bool bar = rounds == 1 && a.nseg <= 32 && !p.hold_first;
-  const void *kern = bar ? (const void *)bwd_seg_kernel<E, S, RB, true, GATE>
-                         : (const void *)bwd_seg_kernel<E, S, RB, false, GATE>;
+  const void *kern = bar ? (const void *)bwd_seg_kernel<E, S, RB, true, GATE, STATE>
+                         : (const void *)bwd_seg_kernel<E, S, RB, false, GATE, STATE>;
   void *args[] = {&km, &vm, &gm, &rm, &a};
   return cudaLaunchCooperativeKernel(kern, dim3((unsigned)grid), dim3(kWarps * 32), args, (size_t)smem, st);
 }
@@ -760,15 +782,26 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
 
 cudaError_t launch_backward_seg(const BwdArgs &p, int dtype, float *gw, float *gu, unsigned *tile_cnt,
                                 int64_t scratch_doubles, int num_sms, cudaStream_t st) {
+  const int64_t sc = scratch_doubles;
+  const int ts = WKV_SEGB_TS;
+  if (p.r && (p.gs_out || p.gs_in)) return cudaErrorInvalidValue;  // no entry point asks for both
   if (p.r)
-    return dtype == 0 ? launch_bwd_seg_t<float, WKV_SEGB_S_F32_GATE, WKV_SEGB_RB, true>(
-                            p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, WKV_SEGB_TS, st)
-                      : launch_bwd_seg_t<uint16_t, WKV_SEGB_S_BF16_GATE, WKV_SEGB_RB, true>(
-                            p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, WKV_SEGB_TS, st);
-  return dtype == 0 ? launch_bwd_seg_t<float, WKV_SEGB_S_F32, WKV_SEGB_RB, false>(
-                          p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, WKV_SEGB_TS, st)
-                    : launch_bwd_seg_t<uint16_t, WKV_SEGB_S_BF16, WKV_SEGB_RB, false>(
-                          p, dtype, gw, gu, tile_cnt, scratch_doubles, num_sms, WKV_SEGB_TS, st);
+    return dtype == 0
+               ? launch_bwd_seg_t<float, WKV_SEGB_S_F32_GATE, WKV_SEGB_RB, true, false>(p, dtype, gw, gu, tile_cnt,
+                                                                                         sc, num_sms, ts, st)
+               : launch_bwd_seg_t<uint16_t, WKV_SEGB_S_BF16_GATE, WKV_SEGB_RB, true, false>(
+                     p, dtype, gw, gu, tile_cnt, sc, num_sms, ts, st);
+  if (p.gs_out || p.gs_in)
+    return dtype == 0
+               ? launch_bwd_seg_t<float, WKV_SEGB_S_F32, WKV_SEGB_RB, false, true>(p, dtype, gw, gu, tile_cnt, sc,
+                                                                                    num_sms, ts, st)
+               : launch_bwd_seg_t<uint16_t, WKV_SEGB_S_BF16, WKV_SEGB_RB, false, true>(p, dtype, gw, gu, tile_cnt,
+                                                                                       sc, num_sms, ts, st);
+  return dtype == 0
+             ? launch_bwd_seg_t<float, WKV_SEGB_S_F32, WKV_SEGB_RB, false, false>(p, dtype, gw, gu, tile_cnt, sc,
+                                                                                   num_sms, ts, st)
+             : launch_bwd_seg_t<uint16_t, WKV_SEGB_S_BF16, WKV_SEGB_RB, false, false>(p, dtype, gw, gu, tile_cnt,
+                                                                                      sc, num_sms, ts, st);
 }
 
 }  // namespace wkv

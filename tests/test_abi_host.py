@@ -163,3 +163,23 @@ def test_backward_gated_validation(W):
     bad = list(ok); bad[16] = FAKE * 9 + 2
     assert a.wkv_backward_gated(*bad) == -2                # grad_r misaligned
     assert a.wkv_backward_gated(*ok) == -3                 # no workspace
+
+
+def test_backward_state_validation(W):
+    a = W.abi
+    # (B, T, C, dt, w, u, k, v, gy, state_in, ckpt, state_out, gso, gw, gu, gk, gv, gsi,
+    #  ws, ws_bytes, stream)
+    ok = [1, 64, 32, 0, FAKE, FAKE, FAKE, FAKE * 2, FAKE * 3, FAKE * 10, 0, FAKE * 11, FAKE * 12,
+          FAKE * 4, FAKE * 5, FAKE * 6, FAKE * 7, FAKE * 13, 0, 0, 0]
+    bad = list(ok); bad[11] = 0
+    assert a.wkv_backward_state(*bad) == -1                # grad_state_out without state_out
+    bad = list(ok); bad[17] = FAKE * 13 + 2
+    assert a.wkv_backward_state(*bad) == -2                # grad_state_in misaligned
+    for clash in (FAKE, FAKE * 10, FAKE * 11, FAKE * 12, FAKE * 6):  # on k, state_in, state_out, gso, grad_k
+        bad = list(ok); bad[17] = clash
+        assert a.wkv_backward_state(*bad) == -2, clash
+    bad = list(ok); bad[12] = FAKE * 6                     # grad_state_out inside grad_k
+    assert a.wkv_backward_state(*bad) == -2
+    assert a.wkv_backward_state(*ok) == -3                 # no workspace
+    opt = a.Options(kernel=4)
+    assert a.wkv_backward_state_ex(*ok, opt) == -1         # retired selector
