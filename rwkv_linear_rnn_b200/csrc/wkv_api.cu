@@ -435,7 +435,8 @@ int wkv_backward_gated_ex(int64_t B, int64_t T, int64_t C, int dtype, const floa
   cudaStream_t st = (cudaStream_t)stream;
   if (T > 0 && (!ws || !aligned(ws, 256) || ws_bytes < layout(WKV_OP_BACKWARD, B, T, C).total))
     return WKV_ERR_WORKSPACE;
-  if (T == 0 || (bwd_uses_seg(B, T, C, dtype, k, v, grad_o, opt) && aligned(r, 16)))
+  // (the fused kernel also reads grad_k's rows back through TMA)
+  if (T == 0 || (bwd_uses_seg(B, T, C, dtype, k, v, grad_o, opt) && aligned(r, 16) && aligned(grad_k, 16)))
     return backward_impl(B, T, C, dtype, w, u, k, v, grad_o, state_in, ckpt, grad_w, grad_u, grad_k, grad_v,
                          ws, ws_bytes, st, opt, T > 0 ? r : nullptr, grad_r);
   // Unfused: grad_r first carries dL/dwkv = grad_o sigma(r) into the WKV

@@ -117,6 +117,8 @@ template <>
 struct IO<float> {
   static __device__ __forceinline__ float ld(const float *p) { return __ldcs(p); }
   static __device__ __forceinline__ void st(float *p, float x) { __stcs(p, x); }
+  // a store whose line should stay in L2 (read back soon)
+  static __device__ __forceinline__ void st_keep(float *p, float x) { *p = x; }
 };
 template <>
 struct IO<uint16_t> {  // bfloat16 storage
@@ -129,6 +131,11 @@ struct IO<uint16_t> {  // bfloat16 storage
     unsigned short h;
     asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(x));
     asm volatile("st.global.cs.u16 [%0], %1;" ::"l"(p), "h"(h));
+  }
+  static __device__ __forceinline__ void st_keep(uint16_t *p, float x) {
+    unsigned short h;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(x));
+    asm volatile("st.global.u16 [%0], %1;" ::"l"(p), "h"(h) : "memory");
   }
 };
 

@@ -199,9 +199,16 @@ struct SegBwdSmem {
 // BAR: every warp owns at most one segment; all warps run pass 1, meet at a
 // grid barrier and fold the later segments' aggregates without polling.
 // Otherwise segments are joined through per-record flags.
-// GATE: the loss depends on o = sigma(r) * y; the ring items carry r as a
-// fourth tensor, the WKV gradient is grad_o sigma(r) and pass 2 also writes
-// dL/dr = grad_o y sigma'(r).
+// GATE: the loss depends on o = sigma(r) * y.  Pass 1's ring items carry
+// grad_o and r as the third and fourth tensors; pass 1 forms the WKV
+// gradient grad_o sigma(r), writes dL/dr = grad_o y sigma'(r) from its
+// recompute, and leaves grad_o sigma(r) in grad_k's rows (which pass 2
+// overwrites with dL/dk after reading them).  Pass 2's items carry k, v and
+// those rows, as in the ungated kernel: grad_o and r are not re-read, and
+// only k, v and the scratch rows need to stay in L2 between the passes.
+// The scratch rows are written with generic stores and read by TMA: each
+// writer fences them for the async proxy, and a unit's pass-2 items are
+// issued only after its pass 1 is done.
 // STATE: the state terms of a sequence split across calls: the folds start
 // from the adjoint after the last token (the final state's gradient), the
 // last segment's sweep stops exactly at token T-1 (its padding would decay
@@ -213,6 +220,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
                                                       const __grid_constant__ CUtensorMap vmap,
                                                       const __grid_constant__ CUtensorMap gmap,
                                                       const __grid_constant__ CUtensorMap rmap,
+                                                      const __grid_constant__ CUtensorMap smap,
                                                       SegBwdArgs a) {
   constexpr int NARR = GATE ? 4 : 3;
   using Sm = SegBwdSmem<E, S, RB, NARR>;
@@ -255,6 +263,9 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
   // batch first).  Running counters (item, stage, unit) avoid divisions.
   int iss_k = 0, iss_unit = g, iss_r = 0, iss_s = 0, iss_x = 0, iss_row0 = 0;
   int iss_done = 0;  // copies actually issued (lane 0)
+  // GATE: items at or past iss_lim wait (a unit's pass-2 items read rows its
+  // pass 1 writes); `consumed` counts the items taken
+  int iss_lim = GATE ? NB : 1 << 30, consumed = 0;
   if (lane == 0) {
     if (!ring.aligned()) {  // cannot happen with this layout; never issue a misaligned copy
       atomicCAS(&p.hdr->status, 0, -4);
@@ -269,8 +280,30 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       iss_row0 = (int)((int64_t)b * T + (int64_t)(nseg - 1 - rpos) * TS);
     }
     const int bt = iss_r < NB ? iss_r : IPU - 1 - iss_r;
-    ring.issue_stage(maps, iss_s, iss_x, iss_row0 + bt * RB,
-                     iss_r < NB ? l2_policy_evict_last() : l2_policy_evict_first());
+    if constexpr (GATE) {
+      // pass 1: k, v (kept in L2 for pass 2), grad_o, r (read once);
+      // pass 2: k, v and the WKV-gradient rows left in grad_k
+      const int y = iss_row0 + bt * RB;
+      const uint32_t bar = ring.bar(iss_s);
+      const uint64_t first = l2_policy_evict_first();
+      constexpr uint32_t AB = (uint32_t)WarpRing<E, S, NARR, RB>::ARR_BYTES;
+      if (iss_r < NB) {
+        const uint64_t keep = l2_policy_evict_last();
+        mbar_expect_tx(bar, 4u * AB);
+        tma_load_2d_hint(smem_addr(ring.stage(iss_s, 0)), &kmap, iss_x, y, bar, keep);
+        tma_load_2d_hint(smem_addr(ring.stage(iss_s, 1)), &vmap, iss_x, y, bar, keep);
+        tma_load_2d_hint(smem_addr(ring.stage(iss_s, 2)), &gmap, iss_x, y, bar, first);
+        tma_load_2d_hint(smem_addr(ring.stage(iss_s, 3)), &rmap, iss_x, y, bar, first);
+      } else {
+        mbar_expect_tx(bar, 3u * AB);
+        tma_load_2d_hint(smem_addr(ring.stage(iss_s, 0)), &kmap, iss_x, y, bar, first);
+        tma_load_2d_hint(smem_addr(ring.stage(iss_s, 1)), &vmap, iss_x, y, bar, first);
+        tma_load_2d_hint(smem_addr(ring.stage(iss_s, 2)), &smap, iss_x, y, bar, first);
+      }
+    } else {
+      ring.issue_stage(maps, iss_s, iss_x, iss_row0 + bt * RB,
+                       iss_r < NB ? l2_policy_evict_last() : l2_policy_evict_first());
+    }
     ++iss_k;
     iss_done = iss_k;
     iss_s = iss_s + 1 == S ? 0 : iss_s + 1;
@@ -280,13 +313,13 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
     }
   };
   if (lane == 0)
-    while (iss_k < min(S - 1, nitems)) issue_next();
+    while (iss_k < min(min(S - 1, nitems), iss_lim)) issue_next();
   bool failed = false;
   int cs = 0;           // stage of the next item to consume
   uint32_t cph = 0;     // its mbarrier phase parity
-  // Gy: the WKV output's gradient; with the gate, Gd (pass 2 only, want_d)
-  // receives grad_o sigma'(r).
-  auto take = [&](float(&K)[RB], float(&V)[RB], float(&Gy)[RB], float(&Gd)[RB], bool want_d) {
+  // Gy: the WKV output's gradient; with the gate, in pass 1 (first) Gy is
+  // formed as grad_o sigma(r) and Gd receives grad_o sigma'(r).
+  auto take = [&](float(&K)[RB], float(&V)[RB], float(&Gy)[RB], float(&Gd)[RB], bool first) {
     if (!failed && !mbar_wait(ring.bar(cs), cph, budget, nullptr)) {
       failed = true;
       if (lane == 0) atomicCAS(&p.hdr->status, 0, -5 /* WKV_ERR_TIMEOUT */);
@@ -301,8 +334,8 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       Gy[j] = to_f32(gr[j * 32]);
     }
     if constexpr (GATE) {
-      const E *rr = ring.stage(cs, NARR - 1) + lane;
-      if (want_d) {
+      if (first) {
+        const E *rr = ring.stage(cs, NARR - 1) + lane;
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
           float sg, ds;
@@ -310,9 +343,6 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
           Gd[j] = Gy[j] * ds;
           Gy[j] *= sg;
         }
-      } else {
-#pragma unroll
-        for (int j = 0; j < RB; ++j) Gy[j] *= gate_sigmoid(to_f32(rr[j * 32]));
       }
     }
     __syncwarp();  // the stage is read; it may be refilled
@@ -320,7 +350,9 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       cs = 0;
       cph ^= 1u;
     }
-    if (lane == 0 && iss_k < nitems && !failed) {  // after a failed wait nothing new is issued
+    ++consumed;
+    // after a failed wait nothing new is issued
+    if (lane == 0 && iss_k < nitems && !failed && iss_k < iss_lim) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       issue_next();
     }
@@ -366,11 +398,28 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       sts[bt * 96 + 32 + lane] = fb;
       sts[bt * 96 + 64 + lane] = fmaf(fn, w2, fP);
       float K[RB], V[RB], Gy[RB], Gd[RB];
-      take(K, V, Gy, Gd, false);
+      take(K, V, Gy, Gd, true);
       mask_tail(Gy, n - bt * RB);
       float qv[RB], gam[RB], eta[RB], e2v[RB], Mb;
       const bool fast =
-          recompute_batch<RB, false>(K, V, Gy, w2, u2, fc, fa, fb, fP, fn, qv, gam, eta, e2v, Mb, Gd);
+          recompute_batch<RB, GATE>(K, V, Gy, w2, u2, fc, fa, fb, fP, fn, qv, gam, eta, e2v, Mb, Gd);
+      if constexpr (GATE) {
+        // dL/dr = grad_o sigma'(r) y, and the WKV gradient for pass 2 in
+        // grad_k's rows (a plain store: it should stay in L2 until read)
+        if (cok) {
+          const int64_t row = ((int64_t)b * T + t0 + bt * RB) * C + c;
+          E *grp = static_cast<E *>(p.gr) + row;
+          E *gsp = static_cast<E *>(p.gk) + row;
+          const int jn = n - bt * RB;
+#pragma unroll
+          for (int j = 0; j < RB; ++j) {
+            if (j < jn) {
+              IO<E>::st(grp + (int64_t)j * C, Gd[j]);
+              IO<E>::st_keep(gsp + (int64_t)j * C, Gy[j]);
+            }
+          }
+        }
+      }
       const float lag0 = (float)(bt * RB);
       if (fast) {
         // token j's aggregate exponent is lag0 w2 - M + j (w2 - w2e): a batch
@@ -415,6 +464,19 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       }
     }
     const Adj5s agg{ah, hh, ahp, hhp, -Em};
+    if constexpr (GATE) {
+      // pass 1 of this unit is done: its scratch rows are written.  Make them
+      // visible to the async proxy, then issue the held items (this unit's
+      // pass 2 and the next unit's pass 1).
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        iss_lim = (i + 1) * IPU + NB;
+        if (!failed)
+          while (iss_k < nitems && iss_k < iss_lim && iss_k < consumed + S - 1) issue_next();
+      }
+      __syncwarp();
+    }
 
     const int nlast = (int)(T - (nseg - 1) * TS);  // tokens of the chain's last segment
     // the adjoint after the chain's last token (a loss term on the final
@@ -492,7 +554,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
     for (int bi = 0; bi < NB; ++bi) {
       const int bt = NB - 1 - bi;
       float K[RB], V[RB], Gy[RB], Gd[RB];
-      take(K, V, Gy, Gd, true);
+      take(K, V, Gy, Gd, false);
       const int nb = n - bt * RB;  // valid tokens of the batch (may be <= 0 or > RB)
       mask_tail(Gy, nb);
       float qv[RB], gam[RB], eta[RB], e2v[RB], Mb;
@@ -500,15 +562,7 @@ __global__ void __launch_bounds__(128, WKV_SEGB_MINB) bwd_seg_kernel(const __gri
       {
         float xa = sts[bt * 96 + lane], xb = sts[bt * 96 + 32 + lane], xP = sts[bt * 96 + 64 + lane];
         float xn = 0.f;
-        fast = recompute_batch<RB, GATE>(K, V, Gy, w2, u2, fc, xa, xb, xP, xn, qv, gam, eta, e2v, Mb, Gd);
-      }
-      if constexpr (GATE) {  // dL/dr = grad_o sigma'(r) y
-        if (cok) {
-          E *grp = static_cast<E *>(p.gr) + ((int64_t)b * T + t0 + bt * RB) * C + c;
-#pragma unroll
-          for (int j = 0; j < RB; ++j)
-            if (j < nb) IO<E>::st(grp + (int64_t)j * C, Gd[j]);
-        }
+        fast = recompute_batch<RB, false>(K, V, Gy, w2, u2, fc, xa, xb, xP, xn, qv, gam, eta, e2v, Mb, Gd);
       }
       E *gkp = static_cast<E *>(p.gk) + ((int64_t)b * T + t0 + bt * RB) * C + c;
       E *gvp = static_cast<E *>(p.gv) + ((int64_t)b * T + t0 + bt * RB) * C + c;
@@ -682,7 +736,10 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
       !encode_rows(&gm, p.gy, dtype, p.B * p.T, p.C, RB))
     return cudaErrorInvalidValue;
   rm = gm;  // unused without the gate
-  if (GATE && !encode_rows(&rm, p.r, dtype, p.B * p.T, p.C, RB)) return cudaErrorInvalidValue;
+  CUtensorMap sm = gm;
+  if (GATE && (!encode_rows(&rm, p.r, dtype, p.B * p.T, p.C, RB) ||
+               !encode_rows(&sm, p.gk, dtype, p.B * p.T, p.C, RB)))
+    return cudaErrorInvalidValue;
   constexpr int NARR = GATE ? 4 : 3;
   constexpr int kWarps = 4;
   static_assert(kCkpt % RB == 0, "checkpoints fall on batch starts");
@@ -752,7 +809,7 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
   const bool bar = rounds == 1 && a.nseg <= 32 && !p.hold_first;
   const void *kern = bar ? (const void *)bwd_seg_kernel<E, S, RB, true, GATE, STATE>
                          : (const void *)bwd_seg_kernel<E, S, RB, false, GATE, STATE>;
-  void *args[] = {&km, &vm, &gm, &rm, &a};
+  void *args[] = {&km, &vm, &gm, &rm, &sm, &a};
   return cudaLaunchCooperativeKernel(kern, dim3((unsigned)grid), dim3(kWarps * 32), args, (size_t)smem, st);
 }
 
@@ -771,10 +828,12 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
 #define WKV_SEGB_RB 8
 #endif
 
-// Ring stages of the gated variant (its items carry a fourth array; for bf16
-// three stages measured faster than four: 525 vs 615 us on B8 T4096 C2048).
+// Ring stages of the gated variant (its first-pass items carry four arrays).
+// fp32: two stages, measured faster than three (65.8 vs 68.7 us on B8 T1024
+// C768: the smaller ring lets 4 blocks share an SM).  bf16: three stages,
+// faster than four (525 vs 615 us on B8 T4096 C2048) and than two.
 #ifndef WKV_SEGB_S_F32_GATE
-#define WKV_SEGB_S_F32_GATE WKV_SEGB_S_F32
+#define WKV_SEGB_S_F32_GATE 2
 #endif
 #ifndef WKV_SEGB_S_BF16_GATE
 #define WKV_SEGB_S_BF16_GATE 3

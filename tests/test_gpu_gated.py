@@ -140,6 +140,16 @@ def test_backward_gated_unaligned_gate_input():
     assert_grads5(got, oracle.bwd_gated(w, u, k, v, r, g), F32_GRAD_TOL)
 
 
+def test_backward_gated_unaligned_grad_k():
+    """The fused backward reads grad_k's rows back through TMA, so grad_k off
+    a 16-byte boundary takes the unfused path."""
+    B, T, C = 2, 300, 64
+    w, u, k, v, r, g, _ = gated_case(B, T, C, seed=18)
+    gk = torch.empty(B * T * C + 1, device="cuda")[1:].view(B, T, C)
+    got = W.backward_gated(dev(w), dev(u), dev(k), dev(v), dev(r), dev(g), grad_k=gk)
+    assert_grads5(got, oracle.bwd_gated(w, u, k, v, r, g), F32_GRAD_TOL)
+
+
 def test_backward_gated_wide_keys():
     """Keys over hundreds of binades (the segment kernels' slow path) with a
     saturated gate on part of the sequence."""
