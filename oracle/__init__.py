@@ -37,7 +37,8 @@ canonical (A/B, 1, ln B), or (0, 0, -inf) for an empty state.  gw, gu are
 summed over the batch.
 
 The submodule ``oracle.linattn`` (numpy) holds the causal linear-attention
-operator of the linear attention post, the second workload's checker.
+operator of the linear attention post, the second workload's checker, and
+``oracle.tokenshift`` the token shift of the review's "토큰 변환" section.
 
 Every function here is pinned by tests in ``tests/test_oracle_pins.py``
 against closed forms, library routines, invariants and finite differences.
