@@ -1,7 +1,7 @@
 """Benchmark: WKV fwd+bwd channel-tokens/s and achieved HBM GB/s on B200.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libwkv|reference]
-                [--workload rwkv169m|rwkv1b5_bf16|longctx|decode14b] [--gate]
+                [--workload rwkv169m|rwkv1b5_bf16|longctx|decode14b] [--gate | --token-shift]
 
 A step is one pass of the whole hot path over one batch of the workload:
 ``wkv_forward`` (writing the checkpoints) followed by ``wkv_backward`` on the
@@ -11,7 +11,8 @@ synthetic inputs).  L2 is flushed (a 2x-L2 buffer is written) before every
 timed step, outside the timed events; each step is bracketed by CUDA events
 on the launching stream and the per-step times are summed.  ``--gate`` times
 the gated calls instead (``wkv_forward_gated`` / ``wkv_backward_gated``,
-o = sigmoid(r) * wkv, with a seeded N(0, 1) gate input r).
+o = sigmoid(r) * wkv, with a seeded N(0, 1) gate input r); ``--token-shift``
+times the token shift (three interpolations) on the workload's layer shape.
 
 Multi-GPU (torchrun): every rank runs an independent replica of the workload
 on its own GPU (the operator has no cross-sequence exchange; weak scaling);
@@ -401,6 +402,148 @@ def run_libwkv(args):
         dist.destroy_process_group()
 
 
+def run_token_shift(args):
+    """--token-shift: the three time-mixing interpolations (n = 3) of the
+    workload's layer shape, forward then backward, through the C ABI."""
+    import torch
+    import rwkv_linear_rnn_b200 as W
+    from rwkv_linear_rnn_b200 import abi
+
+    ws_n, rank, local = dist_env()
+    dist = None
+    if ws_n > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = workloads.WORKLOADS[args.workload]
+    B, T, C, n = wl.B, wl.T, wl.C, 3
+    dt = W.WKV_BF16 if wl.dtype == "bf16" else W.WKV_F32
+    tdt = torch.bfloat16 if dt == W.WKV_BF16 else torch.float32
+    es = 2 if dt == W.WKV_BF16 else 4
+    gen = torch.Generator(device="cpu").manual_seed(wl.seed + 1000 * rank)
+    x = torch.randn((B, T, C), generator=gen).to(dev, tdt)
+    xp = torch.randn((B, C), generator=gen).to(dev, tdt)
+    mu = torch.rand((n, C), generator=gen).to(dev)
+    g = torch.randn((n, B, T, C), generator=gen).to(dev, tdt)
+    out = torch.empty((n, B, T, C), device=dev, dtype=tdt)
+    gx = torch.empty_like(x)
+    gmu = torch.empty((n, C), device=dev)
+    gxp = torch.empty_like(xp)
+    nws = abi.wkv_token_shift_workspace_size(B, T, C, n)
+    wsb = torch.empty(nws, dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_w = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    P = lambda t: t.data_ptr()
+
+    def fwd():
+        abi.check(abi.wkv_token_shift(B, T, C, dt, n, P(mu), P(x), P(xp), P(out), sp))
+
+    def bwd():
+        abi.check(abi.wkv_token_shift_backward(B, T, C, dt, n, P(mu), P(x), P(xp), P(g), P(gx), P(gmu),
+                                               P(gxp), P(wsb), nws, sp))
+
+    for _ in range(args.warmup):
+        flush_w.zero_(); flush_r.sum(); fwd(); bwd()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t_begin = time.monotonic()
+    for i in range(K):
+        flush_w.zero_(); flush_r.sum()
+        ev[i][0].record(stream); fwd(); ev[i][1].record(stream); bwd(); ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop(window=(t_begin, time.monotonic()))
+    if dist:
+        dist.barrier()
+    t_fwd = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    t_bwd = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    total_ms = max_over_ranks(sum(t_fwd) + sum(t_bwd), dist, dev)
+
+    e2e = None
+    if not args.no_e2e:
+        hx = x.cpu().pin_memory(); hg = g.cpu().pin_memory()
+        hout = torch.empty_like(out, device="cpu").pin_memory(); hgx = torch.empty_like(hx).pin_memory()
+        hgmu = torch.empty((n, C)).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hx, hg))
+        d2h = sum(t.numel() * t.element_size() for t in (hout, hgx, hgmu))
+        ee = []
+        for i in range(max(3, min(K, 10)) + 1):
+            e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            x.copy_(hx, non_blocking=True); g.copy_(hg, non_blocking=True)
+            fwd(); bwd()
+            hout.copy_(out, non_blocking=True); hgx.copy_(gx, non_blocking=True)
+            hgmu.copy_(gmu, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i > 0:
+                ee.append(e0.elapsed_time(e1))
+        e2e_ms = max_over_ranks(statistics.median(ee), dist, dev)
+        e2e = {"value": aggregate_rate(B * T * C, ws_n, e2e_ms), "unit": "channel-tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if rank == 0:
+        units = B * T * C
+        hbm, peak_kind = peaks()
+        fwd_ms, bwd_ms = statistics.mean(t_fwd), statistics.mean(t_bwd)
+        fb = (1 + n) * es * units           # x read, n outputs written
+        bb = (2 + n) * es * units           # x, n gradients read, grad_x written
+        fwd_gbs = fb / (fwd_ms * 1e-3) / 1e9
+        bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9
+        step_ms = total_ms / K
+        line = {
+            "metric": "token-shift fwd+bwd channel-tokens/s (3 interpolations; HBM GB/s alongside)",
+            "value": aggregate_rate(units, ws_n, step_ms), "unit": "channel-tokens/s",
+            "n_gpus": ws_n, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+            "data": "synthetic (seeded normal x, uniform mu)",
+            "config": {"workload": args.workload, "op": "token_shift", "B": B, "T": T, "C": C, "n": n,
+                       "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
+                       "l2": "flushed before every timed step (2x L2 write + 2x L2 read, outside events)"},
+            "roofline": {"bound": "hbm", "kernel": "wkv_token_shift_backward call, timed as one call",
+                         "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s", "frac": bwd_gbs / hbm,
+                         "traffic": None, "algorithmic_bytes": bb, "peak_kind": peak_kind},
+            "fwd": {"ms": fwd_ms, "gbs": fwd_gbs, "frac": fwd_gbs / hbm},
+            "bwd": {"ms": bwd_ms, "gbs": bwd_gbs, "frac": bwd_gbs / hbm},
+            "clocks": clocks, "gpu_launches": 3 * K,
+        }
+        if e2e:
+            line["e2e"] = e2e
+        if not args.no_cpu_baseline and ws_n == 1:
+            from oracle import tokenshift as ots
+            hx64, hmu, hxp = x.double().cpu().numpy(), mu.double().cpu().numpy(), xp.double().cpu().numpy()
+            hg64 = g.double().cpu().numpy()
+            times = []
+            t_end = time.perf_counter() + args.cpu_seconds
+            while time.perf_counter() < t_end or len(times) < 3:
+                t0 = time.perf_counter()
+                ots.shift(hx64, hmu, hxp)
+                ots.shift_bwd(hx64, hmu, hg64, hxp)
+                times.append(time.perf_counter() - t0)
+            med = statistics.median(times)
+            line["cpu_baseline"] = {"value": units / med, "unit": "channel-tokens/s", "cores": 1,
+                                    "kind": "oracle",
+                                    "sample": f"full {args.workload} token shift fwd+bwd x{len(times)}, median"}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,10 +558,14 @@ def main():
     ap.add_argument("--bwd-kernel", default="auto", choices=sorted(BWD_PLAN))
     ap.add_argument("--gate", action="store_true",
                     help="time the gated calls (o = sigmoid(r) * wkv and its gradients)")
+    ap.add_argument("--token-shift", action="store_true",
+                    help="time the token shift (3 interpolations) on the workload's layer shape")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.token_shift:
+        run_token_shift(args)
     else:
         run_libwkv(args)
 

@@ -21,6 +21,8 @@
  *   wkv_backward  gradients of a scalar loss for the same mode;
  *   wkv_step      RNN mode ("RNN-유사추론" / "자기 회귀 디코딩" steps 4 and 7):
  *                 one token per sequence against a stored state.
+ * wkv_token_shift forms the operator's inputs' time interpolation (the
+ * "토큰 변환" token shift), and its backward.
  * wkv_backward_state adds the gradients through the recurrent state for
  * sequences split across calls; wkv_forward_gated / wkv_backward_gated add
  * the receptance gate o = sigma(r) * y of the time-mixing block's output.
@@ -299,6 +301,48 @@ int wkv_backward_gated_ex(int64_t B, int64_t T, int64_t C, int dtype, const floa
                           float *grad_w, float *grad_u, void *grad_k, void *grad_v,
                           void *grad_r, void *ws, size_t ws_bytes, void *stream,
                           const wkv_options *opt);
+
+/*
+ * wkv_token_shift -- the token shift that forms the time-mixing inputs
+ * (RWKV review, section "토큰 변환": each of R, K, V is a linear
+ * interpolation of the current and the previous token), n interpolations
+ * from one read of x:
+ *   out_m[t] = mu_m * x[t] + (1 - mu_m) * x[t-1],   m < n, per channel,
+ * x[-1] = x_prev (the previous call's last token) or 0 when x_prev is NULL.
+ *   n          1..4 interpolated inputs.
+ *   mu         [n][C] float32 mixing coefficients.
+ *   x          [B, T, C] (element type dtype).
+ *   x_prev     [B, C] (dtype) or NULL.
+ *   out        [n][B, T, C] (dtype): n consecutive tensors; must not overlap
+ *              x, x_prev or mu.
+ * Needs no workspace.  Errors: INVALID_ARG (n outside 1..4, NULL mu, NULL
+ * x/out with T > 0, bad sizes or dtype), UNSUPPORTED (misaligned,
+ * overlapping), CUDA.
+ */
+int wkv_token_shift(int64_t B, int64_t T, int64_t C, int dtype, int n,
+                    const float *mu, const void *x, const void *x_prev, void *out,
+                    void *stream);
+
+/* Bytes of the workspace wkv_token_shift_backward needs (0 for bad sizes). */
+size_t wkv_token_shift_workspace_size(int64_t B, int64_t T, int64_t C, int n);
+
+/*
+ * wkv_token_shift_backward -- gradients of a scalar loss L given
+ * grad_out = dL/dout [n][B, T, C]:
+ *   grad_x[t]   = sum_m mu_m grad_out_m[t] + (1 - mu_m) grad_out_m[t+1]
+ *                 (grad_out_m[T] = 0), [B, T, C] (dtype);
+ *   grad_mu     [n][C] float32, sum over b, t of grad_out_m[t] (x[t] - x[t-1]),
+ *               added in a fixed order (bit-reproducible; overwritten);
+ *   grad_x_prev [B, C] (dtype) sum_m (1 - mu_m) grad_out_m[0], or NULL.
+ * x, x_prev, mu as in the forward.  Outputs must not overlap the inputs or
+ * one another.  ws: wkv_token_shift_workspace_size() bytes, 256-byte
+ * aligned (contents need not be initialised).
+ * Errors: as wkv_token_shift; NULL grad_mu is INVALID_ARG; WORKSPACE.
+ */
+int wkv_token_shift_backward(int64_t B, int64_t T, int64_t C, int dtype, int n,
+                             const float *mu, const void *x, const void *x_prev,
+                             const void *grad_out, void *grad_x, float *grad_mu,
+                             void *grad_x_prev, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * wkv_step -- one RNN-mode token for N independent sequences (float32).

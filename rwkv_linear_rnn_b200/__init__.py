@@ -3,7 +3,7 @@
 Thin Python binding over the C ABI in ``include/wkv.h``.  The functions in
 ``abi`` carry the C names and take raw device pointers (ints) -- argument
 marshalling only.  The tensor helpers below (``forward``, ``backward``,
-``step``, ``WKV``, ``backward_state`` and the gated ``forward_gated``, ``backward_gated``,
+``step``, ``WKV``, ``backward_state``, ``token_shift`` and the gated ``forward_gated``, ``backward_gated``,
 ``GatedWKV``) take torch CUDA tensors, allocate outputs with torch, and
 call the same entry points; PyTorch provides memory and streams only, every
 step of the operator runs in the library's CUDA kernels.
@@ -24,7 +24,8 @@ from .constants import (WKV_BF16, WKV_F32, WKV_KERNEL_AUTO, WKV_KERNEL_CHUNKED,
 __all__ = [
     "abi", "WKVError", "WKV_F32", "WKV_BF16", "WKV_OP_FORWARD", "WKV_OP_BACKWARD", "WKV_OP_STEP",
     "WKV_KERNEL_AUTO", "WKV_KERNEL_SEQUENTIAL", "WKV_KERNEL_CHUNKED", "WKV_KERNEL_CHUNKED_REGS",
-    "WKV_KERNEL_SEGMENT", "WKV_KERNEL_CLUSTER", "WKV_STATIC_SCRATCH_BYTES", "Workspace", "forward", "backward", "backward_state", "step",
+    "WKV_KERNEL_SEGMENT", "WKV_KERNEL_CLUSTER", "WKV_STATIC_SCRATCH_BYTES", "Workspace", "forward", "backward", "backward_state", "step", "token_shift",
+    "token_shift_backward", "TokenShift",
     "forward_gated", "backward_gated", "WKV", "wkv", "WKVState", "wkv_state", "GatedWKV", "gated_wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror", "wkv_version",
     "library_path",
 ]
@@ -215,6 +216,40 @@ def backward_state(w, u, k, v, grad_y, state_in=None, ckpt=None, *, state_out=No
     return gw, gu, gk, gv, gs
 
 
+def token_shift(x, mu, x_prev=None, *, out=None, stream=None):
+    """out[m] = mu[m] * x[t] + (1 - mu[m]) * x[t-1] for x [B, T, C] and
+    mu [n, C] (float32); x[-1] = x_prev [B, C] or 0.  Returns out [n, B, T, C]."""
+    torch = _torch()
+    _check_cuda(x, mu, x_prev, out)
+    B, T, C = x.shape
+    n = mu.shape[0]
+    if out is None:
+        out = torch.empty((n, B, T, C), dtype=x.dtype, device=x.device)
+    abi = _abi()
+    abi.check(abi.wkv_token_shift(B, T, C, _dtype_code(x), n, _ptr(mu), _ptr(x), _ptr(x_prev),
+                                  _ptr(out), _stream(stream)))
+    return out
+
+
+def token_shift_backward(x, mu, grad_out, x_prev=None, *, want_grad_x_prev=False, stream=None):
+    """Gradients (grad_x, grad_mu, grad_x_prev or None) of L given
+    grad_out = dL/dout [n, B, T, C]."""
+    torch = _torch()
+    _check_cuda(x, mu, grad_out, x_prev)
+    B, T, C = x.shape
+    n = mu.shape[0]
+    gx = torch.empty_like(x)
+    gmu = torch.empty((n, C), dtype=torch.float32, device=x.device)
+    gxp = torch.empty((B, C), dtype=x.dtype, device=x.device) if want_grad_x_prev else None
+    abi = _abi()
+    nws = abi.wkv_token_shift_workspace_size(B, T, C, n)
+    ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=x.device)
+    abi.check(abi.wkv_token_shift_backward(B, T, C, _dtype_code(x), n, _ptr(mu), _ptr(x),
+                                           _ptr(x_prev), _ptr(grad_out), _ptr(gx), _ptr(gmu),
+                                           _ptr(gxp), _ptr(ws), nws, _stream(stream)))
+    return gx, gmu, gxp
+
+
 def forward_gated(w, u, k, v, r, state_in=None, *, want_state=False, want_ckpt=False, o=None,
                   workspace=None, stream=None, kernel=WKV_KERNEL_AUTO):
     """o = sigmoid(r) * WKV(w, u, k, v) for k, v, r [B, T, C].  Returns
@@ -351,6 +386,36 @@ def wkv_state(w, u, k, v, state_in):
     """Differentiable WKV with the state: (y, state_out) from w, u [C],
     k, v [B, T, C] and state_in [3, B, C]."""
     return WKVState.apply(w, u, k, v, state_in)
+
+
+class TokenShift:
+    """torch.autograd.Function wrapper: out = TokenShift.apply(x, mu, x_prev)
+    (x_prev may be None)."""
+
+    _fn = None
+
+    @classmethod
+    def apply(cls, x, mu, x_prev=None):
+        if cls._fn is None:
+            torch = _torch()
+
+            class _F(torch.autograd.Function):
+                @staticmethod
+                def forward(ctx, x, mu, x_prev):
+                    x, mu = x.contiguous(), mu.contiguous()
+                    x_prev = None if x_prev is None else x_prev.contiguous()
+                    ctx.save_for_backward(x, mu, x_prev)
+                    return token_shift(x, mu, x_prev)
+
+                @staticmethod
+                def backward(ctx, g):
+                    x, mu, x_prev = ctx.saved_tensors
+                    gx, gmu, gxp = token_shift_backward(x, mu, g.contiguous(), x_prev,
+                                                        want_grad_x_prev=x_prev is not None)
+                    return gx, gmu, gxp
+
+            cls._fn = _F
+        return cls._fn.apply(x, mu, x_prev)
 
 
 class GatedWKV:

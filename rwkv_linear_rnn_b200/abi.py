@@ -21,8 +21,9 @@ from .constants import WKV_ERR_CUDA, WKV_OK
 EXPORTS = (
     "wkv_workspace_size", "wkv_workspace_init", "wkv_ckpt_size", "wkv_forward", "wkv_forward_ex",
     "wkv_backward", "wkv_backward_ex", "wkv_backward_state", "wkv_backward_state_ex",
-    "wkv_forward_gated", "wkv_forward_gated_ex",
-    "wkv_backward_gated", "wkv_backward_gated_ex", "wkv_step", "wkv_backward_static", "wkv_get_status",
+    "wkv_forward_gated", "wkv_forward_gated_ex", "wkv_backward_gated", "wkv_backward_gated_ex",
+    "wkv_token_shift", "wkv_token_shift_workspace_size", "wkv_token_shift_backward",
+    "wkv_step", "wkv_backward_static", "wkv_get_status",
     "wkv_strerror", "wkv_last_cuda_error", "wkv_cuda_error_name", "wkv_version",
 )
 
@@ -59,6 +60,9 @@ _SIGS = {
     "wkv_forward_gated_ex": (_int, [_i64, _i64, _i64, _int] + [_p] * 10 + [_sz, _p, _opt]),
     "wkv_backward_gated": (_int, [_i64, _i64, _i64, _int] + [_p] * 14 + [_sz, _p]),
     "wkv_backward_gated_ex": (_int, [_i64, _i64, _i64, _int] + [_p] * 14 + [_sz, _p, _opt]),
+    "wkv_token_shift": (_int, [_i64, _i64, _i64, _int, _int, _p, _p, _p, _p, _p]),
+    "wkv_token_shift_workspace_size": (_sz, [_i64, _i64, _i64, _int]),
+    "wkv_token_shift_backward": (_int, [_i64, _i64, _i64, _int, _int] + [_p] * 8 + [_sz, _p]),
     "wkv_step": (_int, [_i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p]),
     "wkv_backward_static": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                    _p, _p, _p]),
@@ -162,6 +166,20 @@ def wkv_backward_gated_ex(B, T, C, dtype, w, u, k, v, r, grad_o, state_in, ckpt,
     return lib.wkv_backward_gated_ex(B, T, C, dtype, w, u, k, v, r, grad_o, state_in, ckpt,
                                      grad_w, grad_u, grad_k, grad_v, grad_r, ws, ws_bytes, stream,
                                      _opts(opt))
+
+
+def wkv_token_shift(B, T, C, dtype, n, mu, x, x_prev, out, stream):
+    return lib.wkv_token_shift(B, T, C, dtype, n, mu, x, x_prev, out, stream)
+
+
+def wkv_token_shift_workspace_size(B, T, C, n):
+    return lib.wkv_token_shift_workspace_size(B, T, C, n)
+
+
+def wkv_token_shift_backward(B, T, C, dtype, n, mu, x, x_prev, grad_out, grad_x, grad_mu,
+                             grad_x_prev, ws, ws_bytes, stream):
+    return lib.wkv_token_shift_backward(B, T, C, dtype, n, mu, x, x_prev, grad_out, grad_x,
+                                        grad_mu, grad_x_prev, ws, ws_bytes, stream)
 
 
 def wkv_step(N, C, w, u, k_t, v_t, state_in, y_t, state_out, stream):

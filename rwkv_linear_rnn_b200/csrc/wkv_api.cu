@@ -22,6 +22,10 @@ cudaError_t launch_backward(const BwdArgs &a, int dtype, float *gw, float *gu, c
 cudaError_t launch_step(const StepArgs &a, bool vec, int num_sms, cudaStream_t st);
 cudaError_t launch_gate(int op, int dtype, void *x, const void *go, const void *r, int64_t n, int num_sms,
                         cudaStream_t st);
+cudaError_t launch_token_shift(int64_t B, int64_t T, int64_t C, int dtype, int n, const float *mu, const void *x,
+                               const void *x_prev, void *out, const void *g, void *gx, void *gx_prev, float *part,
+                               float *gmu, bool bwd, bool vec, int num_sms, cudaStream_t st);
+int64_t token_shift_rows(int64_t B, int64_t T);
 cudaError_t launch_state_grad_t0(const float *gs_out, const float *p_out, const float *s_in, float *gs_in,
                                  int64_t BC, int num_sms, cudaStream_t st);
 int64_t fwd_chunk_tokens();
@@ -459,6 +463,64 @@ int wkv_backward_gated(int64_t B, int64_t T, int64_t C, int dtype, const float *
                        void *grad_r, void *ws, size_t ws_bytes, void *stream) {
   return wkv_backward_gated_ex(B, T, C, dtype, w, u, k, v, r, grad_o, state_in, ckpt, grad_w, grad_u, grad_k,
                                grad_v, grad_r, ws, ws_bytes, stream, nullptr);
+}
+
+size_t wkv_token_shift_workspace_size(int64_t B, int64_t T, int64_t C, int n) {
+  if (n < 1 || n > 4 || !sizes_ok(B, T, C)) return 0;
+  const size_t bytes = sizeof(float) * (size_t)token_shift_rows(B, T) * (size_t)n * (size_t)C;
+  return align_up(bytes > 0 ? bytes : 1, 256);
+}
+
+int wkv_token_shift(int64_t B, int64_t T, int64_t C, int dtype, int n, const float *mu, const void *x,
+                    const void *x_prev, void *out, void *stream) {
+  if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_INVALID_ARG;
+  if (n < 1 || n > 4 || !sizes_ok(B, T, C) || !mu) return WKV_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !out)) return WKV_ERR_INVALID_ARG;
+  const size_t es = esize(dtype), nb = (size_t)(B * T * C) * es, pb = (size_t)(B * C) * es;
+  if (!aligned(mu, 4) || !aligned(x, es) || !aligned(x_prev, es) || !aligned(out, es)) return WKV_ERR_UNSUPPORTED;
+  if (overlaps(out, n * nb, x, nb) || overlaps(out, n * nb, x_prev, pb) || overlaps(out, n * nb, mu, 4 * n * C))
+    return WKV_ERR_UNSUPPORTED;
+  if (T == 0) return WKV_OK;
+  const size_t va = 4 * es;
+  const bool vec = C % 4 == 0 && aligned(x, va) && aligned(x_prev, va) && aligned(out, va);
+  return cuda_rc(launch_token_shift(B, T, C, dtype, n, mu, x, x_prev, out, nullptr, nullptr, nullptr, nullptr,
+                                    nullptr, false, vec, num_sms(), (cudaStream_t)stream));
+}
+
+int wkv_token_shift_backward(int64_t B, int64_t T, int64_t C, int dtype, int n, const float *mu, const void *x,
+                             const void *x_prev, const void *grad_out, void *grad_x, float *grad_mu,
+                             void *grad_x_prev, void *ws, size_t ws_bytes, void *stream) {
+  if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_INVALID_ARG;
+  if (n < 1 || n > 4 || !sizes_ok(B, T, C) || !mu || !grad_mu) return WKV_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !grad_out || !grad_x)) return WKV_ERR_INVALID_ARG;
+  const size_t es = esize(dtype), nb = (size_t)(B * T * C) * es, pb = (size_t)(B * C) * es;
+  const size_t mb = 4 * (size_t)n * (size_t)C;
+  if (!aligned(mu, 4) || !aligned(grad_mu, 4) || !aligned(x, es) || !aligned(x_prev, es) ||
+      !aligned(grad_out, es) || !aligned(grad_x, es) || !aligned(grad_x_prev, es))
+    return WKV_ERR_UNSUPPORTED;
+  // outputs must not overlap the inputs or each other
+  struct Span { const void *p; size_t n; };
+  const Span ins[4] = {{x, nb}, {x_prev, pb}, {grad_out, n * nb}, {mu, mb}};
+  const Span outs[3] = {{grad_x, nb}, {grad_mu, mb}, {grad_x_prev, pb}};
+  for (const Span &o : outs) {
+    for (const Span &i : ins)
+      if (overlaps(o.p, o.n, i.p, i.n)) return WKV_ERR_UNSUPPORTED;
+    for (const Span &o2 : outs)
+      if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return WKV_ERR_UNSUPPORTED;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  if (T == 0) {
+    int rc = cuda_rc(cudaMemsetAsync(grad_mu, 0, mb, st));
+    if (rc == WKV_OK && grad_x_prev) rc = cuda_rc(cudaMemsetAsync(grad_x_prev, 0, pb, st));
+    return rc;
+  }
+  const size_t need = wkv_token_shift_workspace_size(B, T, C, n);
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return WKV_ERR_WORKSPACE;
+  const size_t va = 4 * es;
+  const bool vec = C % 4 == 0 && aligned(x, va) && aligned(x_prev, va) && aligned(grad_out, va) &&
+                   aligned(grad_x, va) && aligned(grad_x_prev, va);
+  return cuda_rc(launch_token_shift(B, T, C, dtype, n, mu, x, x_prev, nullptr, grad_out, grad_x, grad_x_prev,
+                                    static_cast<float *>(ws), grad_mu, true, vec, num_sms(), st));
 }
 
 int wkv_step(int64_t N, int64_t C, const float *w, const float *u, const float *k_t,

@@ -183,3 +183,31 @@ def test_backward_state_validation(W):
     assert a.wkv_backward_state(*ok) == -3                 # no workspace
     opt = a.Options(kernel=4)
     assert a.wkv_backward_state_ex(*ok, opt) == -1         # retired selector
+
+
+def test_token_shift_validation(W):
+    a = W.abi
+    # (B, T, C, dt, n, mu, x, x_prev, out, stream)
+    ok = [2, 8, 16, 0, 3, FAKE, FAKE * 2, 0, FAKE * 4, 0]
+    for i, val in ((4, 0), (4, 5), (5, 0), (3, 2)):          # n = 0, n = 5, NULL mu, bad dtype
+        bad = list(ok); bad[i] = val
+        assert a.wkv_token_shift(*bad) == -1, (i, val)
+    bad = list(ok); bad[8] = FAKE * 2 + 64
+    assert a.wkv_token_shift(*bad) == -2                     # out overlaps x
+    bad = list(ok); bad[6] = FAKE * 2 + 2
+    assert a.wkv_token_shift(*bad) == -2                     # x misaligned
+    assert a.wkv_token_shift(2, 0, 16, 0, 3, FAKE, 0, 0, 0, 0) == 0  # T = 0: nothing to do
+    # 2 strips of 32 tokens: one partial row per batch row (B = 2), n = 3, C = 16,
+    # rounded up to 256 bytes
+    assert a.wkv_token_shift_workspace_size(2, 33, 16, 3) == 512
+    assert a.wkv_token_shift_workspace_size(2, 33, 16, 5) == 0
+    # (B, T, C, dt, n, mu, x, x_prev, g, gx, gmu, gx_prev, ws, ws_bytes, stream)
+    okb = [2, 8, 16, 0, 3, FAKE, FAKE * 2, 0, FAKE * 3, FAKE * 5, FAKE * 6, 0, FAKE * 8, 1 << 20, 0]
+    bad = list(okb); bad[10] = 0
+    assert a.wkv_token_shift_backward(*bad) == -1            # NULL grad_mu
+    bad = list(okb); bad[9] = FAKE * 3
+    assert a.wkv_token_shift_backward(*bad) == -2            # grad_x on grad_out
+    bad = list(okb); bad[12] = 0
+    assert a.wkv_token_shift_backward(*bad) == -3            # no workspace
+    bad = list(okb); bad[13] = 64
+    assert a.wkv_token_shift_backward(*bad) == -3            # workspace too small
