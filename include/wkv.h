@@ -284,9 +284,12 @@ int wkv_forward_gated_ex(int64_t B, int64_t T, int64_t C, int dtype, const float
  *   grad_r     [B, T, C] output; must not overlap any input or grad_k/grad_v.
  * Everything else is as in wkv_backward (ckpt from wkv_forward_gated or
  * wkv_forward of the same k, v, state_in; grad_w, grad_u overwritten and
- * reduced in a fixed order).  The segment backward forms both gradients in
- * its own passes; with the other kernels (rows not 16-byte aligned, or a
- * kernel chosen in opt) grad_r is first used as scratch for dL/dy.
+ * reduced in a fixed order).  The segment backward (k, v, r, grad_o and
+ * grad_k 16-byte aligned, C * element size a multiple of 16) forms both
+ * gradients in its own passes and holds dL/dy in grad_k's rows until it
+ * overwrites them with dL/dk; with the other kernels grad_r is first used
+ * as scratch for dL/dy.  Either way the outputs' contents are only defined
+ * once the call has completed without error.
  * Errors: as wkv_backward (NULL r/grad_r is INVALID_ARG when T > 0).
  */
 int wkv_backward_gated(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
