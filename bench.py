@@ -191,9 +191,47 @@ def metric_name(gate: bool) -> str:
     return f"{what} fwd+bwd channel-tokens/s (HBM GB/s and % of roofline alongside)"
 
 
+def token_shift_cpu_baseline(wl_name: str, min_seconds: float):
+    """Time the token-shift oracle (float64 numpy, forward + backward of the
+    three interpolations) on the workload's layer shape."""
+    from oracle import tokenshift as ots
+    wl = workloads.WORKLOADS[wl_name]
+    B, T, C, n = wl.B, min(wl.T, 4096), wl.C, 3
+    rng = np.random.Generator(np.random.PCG64(wl.seed))
+    x = rng.standard_normal((B, T, C))
+    xp = rng.standard_normal((B, C))
+    mu = rng.random((n, C))
+    g = rng.standard_normal((n, B, T, C))
+    times = []
+    t_end = time.perf_counter() + min_seconds
+    while time.perf_counter() < t_end or len(times) < 3:
+        t0 = time.perf_counter()
+        ots.shift(x, mu, xp)
+        ots.shift_bwd(x, mu, g, xp)
+        times.append(time.perf_counter() - t0)
+    med = statistics.median(times)
+    return {"value": B * T * C / med, "unit": "channel-tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{wl_name} token shift (B{B} T{T} C{C}, n=3) fwd+bwd x{len(times)}, median"}
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
+        return
+    if args.token_shift:
+        cb = token_shift_cpu_baseline(args.workload, min_seconds=max(1.0, 2.0 * args.steps))
+        wl = workloads.WORKLOADS[args.workload]
+        line = {"metric": "token-shift fwd+bwd channel-tokens/s (3 interpolations; HBM GB/s alongside)",
+                "value": cb["value"], "unit": "channel-tokens/s", "n_gpus": 1, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": wl.channel_tokens / cb["value"] * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded)", "impl": "reference",
+                "config": {"workload": args.workload, "op": "token_shift", "B": wl.B, "T": wl.T, "C": wl.C,
+                           "n": 3},
+                "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "channel-tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
         return
     cb = cpu_baseline(args.workload, min_seconds=max(1.0, 2.0 * args.steps), gate=args.gate)
     wl = workloads.WORKLOADS[args.workload]
@@ -554,20 +592,7 @@ def run_token_shift(args):
         if e2e:
             line["e2e"] = e2e
         if not args.no_cpu_baseline and ws_n == 1:
-            from oracle import tokenshift as ots
-            hx64, hmu, hxp = x.double().cpu().numpy(), mu.double().cpu().numpy(), xp.double().cpu().numpy()
-            hg64 = g.double().cpu().numpy()
-            times = []
-            t_end = time.perf_counter() + args.cpu_seconds
-            while time.perf_counter() < t_end or len(times) < 3:
-                t0 = time.perf_counter()
-                ots.shift(hx64, hmu, hxp)
-                ots.shift_bwd(hx64, hmu, hg64, hxp)
-                times.append(time.perf_counter() - t0)
-            med = statistics.median(times)
-            line["cpu_baseline"] = {"value": units / med, "unit": "channel-tokens/s", "cores": 1,
-                                    "kind": "oracle",
-                                    "sample": f"full {args.workload} token shift fwd+bwd x{len(times)}, median"}
+            line["cpu_baseline"] = token_shift_cpu_baseline(args.workload, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
