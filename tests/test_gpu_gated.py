@@ -301,3 +301,17 @@ def test_calls_from_a_fresh_thread():
     assert rcs == [0, 0, 0]
     assert fwd_err(host(o), oracle.fwd_gated(w, u, k, v, r)[0]) <= F32_FWD_TOL
     assert_grads5((gw, gu, gk, gv, gr), oracle.bwd_gated(w, u, k, v, r, g), F32_GRAD_TOL)
+
+
+def test_gated_long_sequence_flag_join():
+    """5000 tokens in one chain: more than 32 segments, so both segment
+    kernels join through per-record flags instead of the grid barrier.
+    (Warps holding several segments, with the gated backward's held
+    second-pass loads, run in the bf16 1.5B-shaped test below.)"""
+    B, T, C = 1, 5000, 64
+    w, u, k, v, r, g, _ = gated_case(B, T, C, seed=33)
+    W_, U_, K_, V_, R_ = dev(w), dev(u), dev(k), dev(v), dev(r)
+    o, _, ck = W.forward_gated(W_, U_, K_, V_, R_, want_ckpt=True)
+    assert fwd_err(host(o), oracle.fwd_gated(w, u, k, v, r)[0]) <= F32_FWD_TOL
+    got = W.backward_gated(W_, U_, K_, V_, R_, dev(g), ckpt=ck)
+    assert_grads5(got, oracle.bwd_gated(w, u, k, v, r, g), F32_GRAD_TOL)

@@ -187,3 +187,14 @@ def test_backward_state_rwkv169m_full():
     got = W.backward_state(w, u, k, v, gy, dev(s_in), ck, state_out=dev(s_out), grad_state_out=dev(gso))
     ref = oracle.bwd_state(inp["w"], inp["u"], inp["k"], inp["v"], inp["gy"], s_in, s_out, gso)
     assert_grads_state(got, ref, F32_GRAD_TOL)
+
+
+def test_backward_state_long_sequence_flag_join():
+    """5000 tokens in one chain: more than 32 segments, so the segment
+    backward joins through per-record flags (blocks of segments with suffix
+    records), the final-state gradient entering the first block's folds."""
+    B, T, C = 1, 5000, 64
+    w, u, k, v, g, s_in, s_out, gso = state_case(B, T, C, seed=32, td=(-5.0, -1.0))
+    got = W.backward_state(dev(w), dev(u), dev(k), dev(v), dev(g), dev(s_in), state_out=dev(s_out),
+                           grad_state_out=dev(gso), kernel=W.WKV_KERNEL_SEGMENT)
+    assert_grads_state(got, oracle.bwd_state(w, u, k, v, g, s_in, s_out, gso), F32_GRAD_TOL)
