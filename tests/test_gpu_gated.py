@@ -307,7 +307,7 @@ def test_gated_long_sequence_flag_join():
     """5000 tokens in one chain: more than 32 segments, so both segment
     kernels join through per-record flags instead of the grid barrier.
     (Warps holding several segments, with the gated backward's held
-    second-pass loads, run in the bf16 1.5B-shaped test below.)"""
+    second-pass loads, run in test_gated_rwkv1b5_bf16_subset.)"""
     B, T, C = 1, 5000, 64
     w, u, k, v, r, g, _ = gated_case(B, T, C, seed=33)
     W_, U_, K_, V_, R_ = dev(w), dev(u), dev(k), dev(v), dev(r)
