@@ -69,7 +69,7 @@
 extern "C" {
 #endif
 
-#define WKV_VERSION 100 /* 1.0.0 */
+#define WKV_VERSION 110 /* 1.1.0: gated, state-gradient and token-shift calls */
 
 /* Element type of the [B, T, C] tensors. */
 typedef enum { WKV_F32 = 0, WKV_BF16 = 1 } wkv_dtype;

@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(W):
 
 
 def test_version_and_strerror(W):
-    assert W.wkv_version() == 100
+    assert W.wkv_version() == 110
     for code in range(0, -6, -1):
         assert W.wkv_strerror(code) != "unknown status"
     assert W.wkv_strerror(7) == "unknown status"
