@@ -23,7 +23,7 @@ EXPORTS = (
     "wkv_backward", "wkv_backward_ex", "wkv_backward_state", "wkv_backward_state_ex",
     "wkv_forward_gated", "wkv_forward_gated_ex", "wkv_backward_gated", "wkv_backward_gated_ex",
     "wkv_token_shift", "wkv_token_shift_workspace_size", "wkv_token_shift_backward",
-    "wkv_step", "wkv_backward_static", "wkv_get_status",
+    "wkv_step", "wkv_backward_static", "wkv_backward_static_status", "wkv_get_status",
     "wkv_strerror", "wkv_last_cuda_error", "wkv_cuda_error_name", "wkv_version",
 )
 
@@ -66,6 +66,7 @@ _SIGS = {
     "wkv_step": (_int, [_i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p]),
     "wkv_backward_static": (_int, [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                    _p, _p, _p]),
+    "wkv_backward_static_status": (_int, [_p]),
     "wkv_get_status": (_int, [_p, _p]),
     "wkv_strerror": (ctypes.c_char_p, [_int]),
     "wkv_last_cuda_error": (_int, []),
@@ -191,6 +192,9 @@ def wkv_backward_static(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad
     return lib.wkv_backward_static(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w,
                                    grad_u, grad_k, grad_v, stream)
 
+
+def wkv_backward_static_status(stream):
+    return lib.wkv_backward_static_status(stream)
 
 
 def wkv_get_status(ws, stream):

@@ -11,6 +11,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "../../include/wkv.h"
 
@@ -18,34 +19,52 @@ namespace {
 
 // File-scope scratch.  Every GPU that loads the library holds it until the
 // process exits.  In host code `g_wkv_scratch` is only a host-side stand-in
-// for the symbol: its device address must be fetched per device.
+// for the symbol: its device address must be looked up in the context that
+// runs the kernels.
 constexpr size_t kStaticScratch = WKV_STATIC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_wkv_scratch[kStaticScratch];
 
-constexpr int kMaxDevices = 64;
-std::atomic<void *> g_scratch_ptr[kMaxDevices];
+// Device addresses of the array that have been zero-filled.  Every context
+// that loads the library gets its own instance of the array, at its own
+// address in the process's unified address space; an address not in this
+// set belongs to a context not set up yet (the first call on a device, or the
+// first after the device was reset and the library's module loaded again).
+constexpr int kSlots = 64;
+std::atomic<void *> g_ready[kSlots];
+std::atomic<int> g_next{0};
+std::mutex g_setup;
 
-// Device address of the scratch on the current device.  The first call on a
-// device looks the address up and zero-fills the array (the workspace
-// protocol needs a zeroed header once); later calls only read the cached
-// pointer.  Returns nullptr on failure.
-void *scratch_for_current_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  void *p = g_scratch_ptr[dev].load(std::memory_order_acquire);
-  if (p) return p;
+bool ready(void *q) {
+  for (int i = 0; i < kSlots; ++i)
+    if (g_ready[i].load(std::memory_order_acquire) == q) return true;
+  return false;
+}
+
+// Device address of the scratch in the current context.  The address is
+// looked up on every call (cudaGetSymbolAddress allocates nothing), so it is
+// never stale; the first call that meets a new address zero-fills the array
+// synchronously (the workspace protocol needs a zeroed header once).
+// Returns nullptr on failure.
+void *scratch_for_current_context() {
   void *q = nullptr;
   if (cudaGetSymbolAddress(&q, g_wkv_scratch) != cudaSuccess || !q) return nullptr;
+  if (ready(q)) return q;
+  std::lock_guard<std::mutex> lock(g_setup);
+  if (ready(q)) return q;
   if (cudaMemset(q, 0, kStaticScratch) != cudaSuccess) return nullptr;
   if (cudaDeviceSynchronize() != cudaSuccess) return nullptr;
-  void *expected = nullptr;
-  if (!g_scratch_ptr[dev].compare_exchange_strong(expected, q, std::memory_order_acq_rel))
-    return expected;  // another thread finished the set-up first
+  g_ready[g_next.fetch_add(1) % kSlots].store(q, std::memory_order_release);
   return q;
 }
 
 }  // namespace
 
+// The launch protocol keeps the array consistent from call to call: the
+// per-launch counters of its header (ticket, finished blocks, grid-barrier
+// arrivals) are back at zero when every launch ends, and the launch epoch in
+// the header makes the flags of earlier calls read as stale.  So nothing is
+// cleared between calls, and a call that fails its argument checks has
+// launched nothing.
 extern "C" int wkv_backward_static(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
                                    const float *u, const void *k, const void *v,
                                    const void *grad_y, const float *state_in, const float *ckpt,
@@ -54,17 +73,14 @@ extern "C" int wkv_backward_static(int64_t B, int64_t T, int64_t C, int dtype, c
   const size_t need = wkv_workspace_size(WKV_OP_BACKWARD, B, T, C, dtype);
   if (need == 0) return WKV_ERR_INVALID_ARG;
   if (need > kStaticScratch) return WKV_ERR_WORKSPACE;
-  void *ws = scratch_for_current_device();
+  void *ws = scratch_for_current_context();
   if (!ws) return WKV_ERR_CUDA;
-  // The per-launch counters of the scratch header (block ticket and
-  // finished-block count, bytes 4..11; grid-barrier arrivals, bytes 20..23)
-  // must read zero when a launch starts.  Launches leave them at zero;
-  // clearing them here makes that explicit.  The launch epoch (bytes 0..3)
-  // must persist across calls and is kept, and so is the status word.
-  unsigned char *h = static_cast<unsigned char *>(ws);
-  if (cudaMemsetAsync(h + 4, 0, 8, (cudaStream_t)stream) != cudaSuccess ||
-      cudaMemsetAsync(h + 20, 0, 4, (cudaStream_t)stream) != cudaSuccess)
-    return WKV_ERR_CUDA;
   return wkv_backward(B, T, C, dtype, w, u, k, v, grad_y, state_in, ckpt, grad_w, grad_u, grad_k,
                       grad_v, ws, kStaticScratch, stream);
+}
+
+extern "C" int wkv_backward_static_status(void *stream) {
+  void *ws = scratch_for_current_context();
+  if (!ws) return WKV_ERR_CUDA;
+  return wkv_get_status(ws, stream);
 }
