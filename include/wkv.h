@@ -30,8 +30,11 @@
  * Conventions shared by every call
  * --------------------------------
  * - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *   allocates and frees nothing and keeps no global state; scratch lives in a
- *   caller-provided workspace.
+ *   allocates and frees nothing; scratch lives in a caller-provided
+ *   workspace.  One exception: wkv_backward_static keeps its scratch in a
+ *   file-scope device array of the library (see there), and the library
+ *   caches per device the occupancy of its kernels and that array's set-up;
+ *   nothing else is kept between calls.
  * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *   NULL = legacy default stream).  The return value covers host-side
  *   argument checks and the launch itself; conditions detected on the device
@@ -69,7 +72,7 @@
 extern "C" {
 #endif
 
-#define WKV_VERSION 110 /* 1.1.0: gated, state-gradient and token-shift calls */
+#define WKV_VERSION 120 /* 1.2.0: tile kernels, wkv_backward_static_status */
 
 /* Element type of the [B, T, C] tensors. */
 typedef enum { WKV_F32 = 0, WKV_BF16 = 1 } wkv_dtype;
@@ -90,7 +93,7 @@ enum { WKV_OP_FORWARD = 0, WKV_OP_BACKWARD = 1, WKV_OP_STEP = 2 };
 /* Kernel selector (wkv_options.kernel). */
 enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
        WKV_KERNEL_CHUNKED_REGS = 3, /* 4 and 5 are retired */
-       WKV_KERNEL_SEGMENT = 6, WKV_KERNEL_CLUSTER = 7 };
+       WKV_KERNEL_SEGMENT = 6, WKV_KERNEL_CLUSTER = 7, WKV_KERNEL_TILE = 8 };
 
 /*
  * Optional knobs for the *_ex calls.  A NULL options pointer, or all fields
@@ -112,10 +115,17 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
  *               dL/du in the same launch.  CLUSTER (forward only) gives each
  *               chain a thread-block cluster whose warps take its segments
  *               round by round and join them through distributed shared
- *               memory.  The backward runs the segment kernel for AUTO and
- *               SEGMENT on 16-byte aligned rows and the chunked kernel
- *               otherwise.  Values 4 and 5 are retired and rejected with
- *               WKV_ERR_INVALID_ARG.
+ *               memory.  TILE (forward and backward) gives each warp units
+ *               of 32 (fp32) or 64 (bf16) tokens of one chain whose tiles
+ *               stay in shared memory between the unit's two passes, joins
+ *               units by a decoupled look-back over records that carry their
+ *               own validity tags (no fences), and, in the forward, runs the
+ *               next unit's first pass before the current unit's join.  AUTO
+ *               runs TILE on 16-byte aligned rows when a chain (batch row, 32
+ *               channels) has at most about four resident warps' units in
+ *               flight, SEGMENT otherwise, and the chunked kernels on
+ *               unaligned rows.  Values 4 and 5 are retired and rejected
+ *               with WKV_ERR_INVALID_ARG.
  *   spin_limit  bound on any one device-side wait (a predecessor's record,
  *               a shared-memory load, the grid barrier) in microseconds (the
  *               chunked kernels count polls of at most about 1 us each);
@@ -374,22 +384,37 @@ int wkv_step(int64_t N, int64_t C, const float *w, const float *u,
  * allocating library routine.  Inputs and outputs are still the caller's.
  *   - Limit: problems with wkv_workspace_size(WKV_OP_BACKWARD, B, T, C, dtype)
  *     above WKV_STATIC_SCRATCH_BYTES are rejected with WKV_ERR_WORKSPACE.
- *   - Set-up: the first call on each device (with that device current) looks
- *     up the array's device address with cudaGetSymbolAddress and zero-fills
- *     it synchronously; make that first call before any stream capture.
- *   - Every call on a device shares the one array, which keeps the previous
+ *   - Set-up: every call looks up the array's device address in the current
+ *     context with cudaGetSymbolAddress (which allocates nothing), so a
+ *     device reset or another context on the same device never leaves a
+ *     stale address.  The first call that meets an address (the first call
+ *     on each device, with that device current) zero-fills the array
+ *     synchronously (cudaMemset, cudaDeviceSynchronize); make that first
+ *     call before any stream capture.
+ *   - Every call in a context shares the one array, which keeps the previous
  *     call's contents.  Calls whose executions overlap on the GPU (other
  *     streams, other host threads) race on it and give wrong results; order
  *     them on one stream.
  *   - Each GPU that loads the library holds the array until the process
- *     exits.  Device-side wait failures are not reported by this entry point.
+ *     exits.  A device-side wait that gave up is read, like wkv_get_status,
+ *     with wkv_backward_static_status.
  * Returns the codes of wkv_backward, plus WKV_ERR_CUDA if the set-up fails.
+ * Argument errors are found before anything is launched.
  */
 #define WKV_STATIC_SCRATCH_BYTES (16u << 20) /* 16 MiB */
 int wkv_backward_static(int64_t B, int64_t T, int64_t C, int dtype, const float *w,
                         const float *u, const void *k, const void *v, const void *grad_y,
                         const float *state_in, const float *ckpt, float *grad_w,
                         float *grad_u, void *grad_k, void *grad_v, void *stream);
+
+/*
+ * wkv_get_status for wkv_backward_static's array in the current context:
+ * waits for `stream`, then returns and clears the device-side status word
+ * (WKV_OK, or WKV_ERR_TIMEOUT if a bounded wait of an earlier call gave up
+ * and its gradients are invalid).  WKV_ERR_CUDA if the look-up, the
+ * synchronisation or the copy failed.
+ */
+int wkv_backward_static_status(void *stream);
 
 /*
  * Waits for `stream`, then returns and clears the device-side status word of

@@ -6,8 +6,11 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "../../include/wkv.h"
 #include "wkv_internal.cuh"
+#include "wkv_tile.cuh"
 
 namespace wkv {
 cudaError_t launch_forward(const FwdArgs &a, int dtype, int kind, int num_sms, cudaStream_t st);
@@ -29,6 +32,9 @@ int64_t token_shift_rows(int64_t B, int64_t T);
 cudaError_t launch_state_grad_t0(const float *gs_out, const float *p_out, const float *s_in, float *gs_in,
                                  int64_t BC, int num_sms, cudaStream_t st);
 int64_t fwd_chunk_tokens();
+cudaError_t launch_forward_tile(const FwdArgs &f, float4 *rec, int dtype, int num_sms, cudaStream_t st);
+cudaError_t launch_backward_tile(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *rec, float4 *chain_sum,
+                                 int num_sms, cudaStream_t st);
 }  // namespace wkv
 
 using namespace wkv;
@@ -72,7 +78,7 @@ bool sizes_ok(int64_t B, int64_t T, int64_t C) {
 }
 
 struct Layout {
-  size_t flags, desc, desc_bytes, ckpt, part, cnt, total;
+  size_t flags, desc, desc_bytes, ckpt, part, cnt, rec, total;
   int64_t nct, nchains, nchunks_f, nchunks_b;
 };
 
@@ -92,12 +98,19 @@ Layout layout(int op, int64_t B, int64_t T, int64_t C) {
   L.desc = off;
   L.desc_bytes = sizeof(float) * kDescFloats * (size_t)tiles;
   off = align_up(off + L.desc_bytes, 256);
+  // tile kernels: two records per unit of at most 32 tokens, 16 bytes per
+  // lane each (forward) or 32 (backward); their flags share the flag region.
+  // The region sits at the same offset in the forward and the backward
+  // layout: a backward without checkpoints runs the forward on its own
+  // workspace, and the forward's records must not reach the regions below.
+  L.rec = off;
+  off = align_up(off + (op == WKV_OP_BACKWARD ? 2048 : 1536) * (size_t)(L.nchains * L.nchunks_b), 256);
   L.ckpt = L.part = L.cnt = 0;
   if (op == WKV_OP_BACKWARD) {
     L.ckpt = off;
     off = align_up(off + sizeof(float) * 3 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
-    L.part = off;
-    off = align_up(off + sizeof(float) * 2 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
+    L.part = off;  // dL/dw, dL/du partials: 2 floats per (chunk, b, c); the tile kernel's tagged words: 4
+    off = align_up(off + sizeof(float) * 4 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
     L.cnt = off;  // per channel tile counters of the segment backward's reduction (cleared by it)
     off = align_up(off + sizeof(unsigned) * (size_t)L.nct, 256);
   }
@@ -105,17 +118,31 @@ Layout layout(int op, int64_t B, int64_t T, int64_t C) {
   return L;
 }
 
+
+// SM count of the current device, looked up once per device.
 int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
+
+// AUTO picks the tile kernels when a chain has few units in flight at once
+// (at most about four of the resident warps per chain): their joins then find
+// the records they need published a step earlier.  With more (long chains
+// over few batch rows and channels) the segment kernels' longer segments
+// amortise their joins better.  warps_per_sm: resident warps of the kernel.
+bool tile_pays(int64_t nchains, int warps_per_sm) { return nchains * 4 >= (int64_t)warps_per_sm * num_sms(); }
 
 bool pick_chunked(const wkv_options *opt, int64_t B, int64_t T, int64_t C) {
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   if (kernel == WKV_KERNEL_SEQUENTIAL) return false;
   if (kernel == WKV_KERNEL_CHUNKED || kernel == WKV_KERNEL_CHUNKED_REGS || kernel == WKV_KERNEL_SEGMENT ||
-      kernel == WKV_KERNEL_CLUSTER)
+      kernel == WKV_KERNEL_CLUSTER || kernel == WKV_KERNEL_TILE)
     return true;
   // Enough independent chains to fill the GPU, or too short to split.
   return !(B * C >= kSeqMinChains || T <= 2 * fwd_chunk_tokens());
@@ -125,7 +152,8 @@ bool options_ok(const wkv_options *opt) {
   if (!opt) return true;
   const int k = opt->kernel;
   return k == WKV_KERNEL_AUTO || k == WKV_KERNEL_SEQUENTIAL || k == WKV_KERNEL_CHUNKED ||
-         k == WKV_KERNEL_CHUNKED_REGS || k == WKV_KERNEL_SEGMENT || k == WKV_KERNEL_CLUSTER;
+         k == WKV_KERNEL_CHUNKED_REGS || k == WKV_KERNEL_SEGMENT || k == WKV_KERNEL_CLUSTER ||
+         k == WKV_KERNEL_TILE;
 }
 
 int64_t spin_of(const wkv_options *opt) {
@@ -184,7 +212,13 @@ int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
   a.hold_first = opt ? opt->test_hold_first_chunk : 0;
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   const bool tma = chunked && fwd_tma_eligible(a, dtype);
-  const bool seg = tma && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT);
+  // tile forward: whole units of tokens, y (and r) loaded and stored by TMA
+  if (tma && (kernel == WKV_KERNEL_TILE || (kernel == WKV_KERNEL_AUTO && tile_pays(L.nchains, r ? 6 : 9))) &&
+      T >= tile_fwd_tokens(dtype) && aligned(y, 16) && aligned(r, 16)) {
+    a.r = r;
+    return cuda_rc(launch_forward_tile(a, reinterpret_cast<float4 *>(base + L.rec), dtype, num_sms(), st));
+  }
+  const bool seg = tma && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT || kernel == WKV_KERNEL_TILE);
   if (seg && (!r || aligned(r, 16))) {
     a.r = r;  // fused gate
     return cuda_rc(launch_forward_seg(a, dtype, num_sms(), st));
@@ -208,7 +242,7 @@ int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
 bool bwd_uses_seg(int64_t B, int64_t T, int64_t C, int dtype, const void *k, const void *v, const void *gy,
                   const wkv_options *opt) {
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
-  if (kernel != WKV_KERNEL_AUTO && kernel != WKV_KERNEL_SEGMENT) return false;
+  if (kernel != WKV_KERNEL_AUTO && kernel != WKV_KERNEL_SEGMENT && kernel != WKV_KERNEL_TILE) return false;
   FwdArgs probe{};
   probe.B = B; probe.T = T; probe.C = C; probe.k = k; probe.v = v;
   return fwd_tma_eligible(probe, dtype) && aligned(gy, 16);
@@ -288,6 +322,16 @@ int backward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, co
   a.p_out = sg.p_out;
   a.gs_in = sg.gs_in;
   a.state_in = state_in;
+  const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
+  if ((!r || (aligned(r, 16) && aligned(gr, 16))) &&
+      (kernel == WKV_KERNEL_TILE || (kernel == WKV_KERNEL_AUTO && tile_pays(L.nchains, r ? 6 : 8))) &&
+      T >= tile_fwd_tokens(dtype) && bwd_uses_seg(B, T, C, dtype, k, v, grad_y, nullptr) && aligned(grad_k, 16) &&
+      aligned(grad_v, 16)) {
+    // the per-chain sums of dL/dw, dL/du use the descriptor region (16 bytes
+    // per (b, c) <= 640 bytes per chain and chunk), idle in the tile kernels
+    return cuda_rc(launch_backward_tile(a, dtype, grad_w, grad_u, reinterpret_cast<float4 *>(base + L.rec),
+                                        reinterpret_cast<float4 *>(base + L.desc), num_sms(), st));
+  }
   if (bwd_uses_seg(B, T, C, dtype, k, v, grad_y, opt)) {
     const int64_t scratch = (int64_t)(L.desc_bytes / sizeof(double));
     return cuda_rc(launch_backward_seg(a, dtype, grad_w, grad_u, reinterpret_cast<unsigned *>(base + L.cnt), scratch,

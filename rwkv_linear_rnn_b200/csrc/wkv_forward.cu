@@ -449,6 +449,23 @@ bool encode_rows(CUtensorMap *m, const void *ptr, int dtype, int64_t rows, int64
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [B, T, C] tensor as a 3-D map (C fastest), boxes of 32 channels x `box_t`
+// tokens x 1 batch row.  Loads past T or C read zeros and stores there are
+// clipped, so a box never reaches into the next batch row.
+bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T, int64_t C, int box_t) {
+  auto enc = tensor_map_encoder();
+  if (!enc || !ensure_context()) return false;
+  const size_t es = dtype == 0 ? 4 : 2;
+  cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)(C * es), (cuuint64_t)(T * C * es)};
+  cuuint32_t box[3] = {32u, (cuuint32_t)box_t, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // TMA needs 16-byte aligned rows and base addresses, and row indices < 2^31.
 bool fwd_tma_eligible(const FwdArgs &a, int dtype) {
   const int64_t es = dtype == 0 ? 4 : 2;

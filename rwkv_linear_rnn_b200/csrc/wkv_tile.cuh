@@ -1,0 +1,117 @@
+// wkv_tile.cuh -- definitions shared by the tile kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "wkv_internal.cuh"
+
+namespace wkv {
+
+constexpr int kTileWarps = 4;   // warps per block (backward)
+constexpr int kTileFwdWarps = 3;  // warps per block (forward: three blocks of 3 x 24 KB fit an SM)
+constexpr int kTileLF32 = 32;   // tokens per unit, fp32 tensors
+constexpr int kTileLBF16 = 64;  // tokens per unit, bf16 tensors (same tile bytes)
+constexpr int kTileRB = 16;     // tokens per batch of the fast path
+constexpr int kMaxDevices = 64; // per-device launch caches
+
+struct TileFwdArgs {
+  FwdArgs f;
+  float4 *rec;   // [units][2][32] records: summary, inclusive prefix
+  int64_t nseg;  // units per chain
+};
+
+// Round a float to the tensor element type (bf16: to nearest, ties to even).
+template <typename E>
+__device__ __forceinline__ E from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ uint16_t from_f32<uint16_t>(float x) {
+  unsigned short h;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(x));
+  return h;
+}
+
+// ------------------------------------------------------------- TMA (3-D) ---
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *map, int x, int y, int z, uint32_t bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const void *map, int x, int y, int z, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every bulk store of this thread has read its shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every bulk store of this thread is complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Generic-proxy accesses to shared memory ordered before later async-proxy ones.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------------------- records ---
+// The tile kernels join their units through records in the workspace that
+// carry their own validity: every 16-byte word of a record holds, in its
+// last 32 bits, a tag made of the launch epoch and the record kind, and is
+// written and read with single 16-byte accesses (aligned 16-byte vector
+// accesses are performed as one access, the property decoupled look-back
+// scans rely on).  A reader that sees the expected tag in a word sees that
+// word's payload; a word from an earlier launch, or not yet written, shows
+// another tag and is read again.  So publishing needs no fence: payload and
+// tag travel together.  A per-unit status word (the tag of the latest record
+// published) is a hint that tells a reader how far back to look; the words
+// themselves decide.
+constexpr unsigned kFlagAgg = 1u, kFlagInc = 2u;
+__device__ __forceinline__ unsigned tile_flag(unsigned epoch, unsigned what) {
+  return (epoch_tag(epoch) << 2) | what;
+}
+__device__ __forceinline__ void st_relaxed_v4(float4 *p, float4 v) {
+  asm volatile("st.relaxed.gpu.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ float4 ld_relaxed_v4(const float4 *p) {
+  float4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u32(unsigned *p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ float tagf(unsigned t) { return __uint_as_float(t); }
+__device__ __forceinline__ bool tag_is(float x, unsigned t) { return __float_as_uint(x) == t; }
+
+// Forward records, 1.5 KB per unit: the unit's summary (a, b, E, tag) at
+// rec[unit * 96 + lane] with its exponent evaluated (E = P + n w2, one
+// rounding: a summary enters a prefix once, so nothing accumulates), then
+// its inclusive prefix in two words, (a, b, P, tag) at +32 and (n, tag, 0, 0)
+// at +64, with the anchored exponent kept exact along the chain.
+constexpr int kFwdRecWords = 96;
+__device__ __forceinline__ void tile_put_agg(float4 *rec, int64_t unit, const St &s, float w2, unsigned tag,
+                                             int lane) {
+  st_relaxed_v4(rec + unit * kFwdRecWords + lane, make_float4(s.a, s.b, st_exp(s, w2), tagf(tag)));
+}
+__device__ __forceinline__ void tile_put_inc(float4 *rec, int64_t unit, const St &s, unsigned tag, int lane) {
+  float4 *d = rec + unit * kFwdRecWords + lane;
+  st_relaxed_v4(d + 32, make_float4(s.a, s.b, s.P, tagf(tag)));
+  st_relaxed_v4(d + 64, make_float4(s.n, tagf(tag), 0.f, 0.f));
+}
+
+// Tokens per unit of the tile kernels for an element type (0 fp32, 1 bf16).
+int tile_fwd_tokens(int dtype);
+
+}  // namespace wkv

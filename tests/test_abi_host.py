@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(W):
 
 
 def test_version_and_strerror(W):
-    assert W.wkv_version() == 110
+    assert W.wkv_version() == 120
     for code in range(0, -6, -1):
         assert W.wkv_strerror(code) != "unknown status"
     assert W.wkv_strerror(7) == "unknown status"
@@ -90,7 +90,7 @@ def test_forward_chunked_needs_workspace(W):
     assert W.abi.wkv_forward_ex(*base, FAKE * 8 + 16, 1 << 30, 0, opt) == -3  # misaligned
 
 
-@pytest.mark.parametrize("kernel", [4, 5, 8, -1])
+@pytest.mark.parametrize("kernel", [4, 5, 9, -1])
 def test_retired_and_unknown_kernel_selectors_are_rejected(W, kernel):
     """Selector values 4 and 5 are retired; unknown values are rejected too,
     before anything is launched."""

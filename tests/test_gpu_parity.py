@@ -20,8 +20,8 @@ pytestmark = pytest.mark.gpu
 
 KERNELS = {"seq": W.WKV_KERNEL_SEQUENTIAL, "chunked": W.WKV_KERNEL_CHUNKED,
            "chunked_regs": W.WKV_KERNEL_CHUNKED_REGS, "segment": W.WKV_KERNEL_SEGMENT,
-           "cluster": W.WKV_KERNEL_CLUSTER}
-BWD_KERNELS = {"chunked": W.WKV_KERNEL_CHUNKED, "segment": W.WKV_KERNEL_SEGMENT}
+           "cluster": W.WKV_KERNEL_CLUSTER, "tile": W.WKV_KERNEL_TILE}
+BWD_KERNELS = {"chunked": W.WKV_KERNEL_CHUNKED, "segment": W.WKV_KERNEL_SEGMENT, "tile": W.WKV_KERNEL_TILE}
 
 
 def small_case(B, T, C, seed, dtype="f32", td=(-3.0, 1.0), kstd=1.0, state=False):
@@ -268,7 +268,7 @@ def _range_case(name, seed):
     return w, u, k, v, g
 
 
-@pytest.mark.parametrize("kernel", ["segment", "cluster"])
+@pytest.mark.parametrize("kernel", ["segment", "cluster", "tile"])
 @pytest.mark.parametrize("name", sorted(RANGE_CASES))
 def test_segment_forward_ranges(name, kernel):
     w, u, k, v, g = _range_case(name, seed=41)
@@ -277,12 +277,13 @@ def test_segment_forward_ranges(name, kernel):
     assert fwd_err(host(y), y_ref) <= F32_FWD_TOL
 
 
+@pytest.mark.parametrize("kernel", ["segment", "tile"])
 @pytest.mark.parametrize("name", sorted(RANGE_CASES))
-def test_segment_backward_ranges(name):
+def test_segment_backward_ranges(name, kernel):
     w, u, k, v, g = _range_case(name, seed=43)
     W_, U_, K_, V_ = dev(w), dev(u), dev(k), dev(v)
-    _, _, ck = W.forward(W_, U_, K_, V_, want_ckpt=True, kernel=W.WKV_KERNEL_SEGMENT)
-    got = W.backward(W_, U_, K_, V_, dev(g), ckpt=ck, kernel=W.WKV_KERNEL_SEGMENT)
+    _, _, ck = W.forward(W_, U_, K_, V_, want_ckpt=True, kernel=KERNELS[kernel])
+    got = W.backward(W_, U_, K_, V_, dev(g), ckpt=ck, kernel=BWD_KERNELS[kernel])
     assert_grads(got, grads_ref(w, u, k, v, g), F32_GRAD_TOL)
 
 
@@ -338,7 +339,7 @@ def test_autograd_function_matches_oracle():
 
 # -------------------------------------------------- failure and edge paths ---
 
-@pytest.mark.parametrize("kernel", ["chunked", "segment"])
+@pytest.mark.parametrize("kernel", ["chunked", "segment", "tile"])
 def test_timeout_is_reported_and_context_survives(kernel):
     """The first chunk (segment) is told never to publish its record: the
     warps that wait on it give up after a short bounded wait, the status word
@@ -363,8 +364,9 @@ def test_timeout_is_reported_and_context_survives(kernel):
     assert fwd_err(host(y2), y_ref) <= F32_FWD_TOL
 
 
-def test_backward_timeout_is_reported_and_context_survives():
-    """The segment backward with the last segment's record held back: the
+@pytest.mark.parametrize("kernel", ["segment", "tile"])
+def test_backward_timeout_is_reported_and_context_survives(kernel):
+    """The backward with the last segment's (unit's) record held back: the
     waits and the grid barrier stay bounded, the status reads WKV_ERR_TIMEOUT,
     and the next call on the same workspace is correct."""
     B, T, C = 1, 1024, 64
@@ -375,19 +377,20 @@ def test_backward_timeout_is_reported_and_context_survives():
     buf, nb = ws.get(W.WKV_OP_BACKWARD, B, T, C, W.WKV_F32)
     gw = torch.empty(C, device="cuda"); gu = torch.empty(C, device="cuda")
     gk = torch.empty_like(K_); gv = torch.empty_like(V_)
-    opt = abi.Options(kernel=W.WKV_KERNEL_SEGMENT, test_hold_first_chunk=1, spin_limit=2000)
+    opt = abi.Options(kernel=BWD_KERNELS[kernel], test_hold_first_chunk=1, spin_limit=2000)
     stream = torch.cuda.current_stream().cuda_stream
     P = lambda t: t.data_ptr()
     rc = abi.wkv_backward_ex(B, T, C, 0, P(W_), P(U_), P(K_), P(V_), P(G_), 0, P(ck), P(gw), P(gu),
                              P(gk), P(gv), P(buf), nb, stream, opt)
     assert rc == 0
     assert ws.status() == abi.WKV_ERR_TIMEOUT
-    got = W.backward(W_, U_, K_, V_, G_, ckpt=ck, workspace=ws, kernel=W.WKV_KERNEL_SEGMENT)
+    got = W.backward(W_, U_, K_, V_, G_, ckpt=ck, workspace=ws, kernel=BWD_KERNELS[kernel])
     assert ws.status() == 0
     assert_grads(got, grads_ref(w, u, k, v, g), F32_GRAD_TOL)
 
 
-def test_segment_backward_reuses_a_workspace_across_shapes():
+@pytest.mark.parametrize("kernel", ["segment", "tile"])
+def test_segment_backward_reuses_a_workspace_across_shapes(kernel):
     """One workspace, shapes in decreasing then increasing size: whatever an
     earlier call left in the workspace does not leak into a later result."""
     ws = W.Workspace()
@@ -395,12 +398,13 @@ def test_segment_backward_reuses_a_workspace_across_shapes():
         w, u, k, v, g, _ = small_case(B, T, C, seed=B + T + C)
         W_, U_, K_, V_ = dev(w), dev(u), dev(k), dev(v)
         _, _, ck = W.forward(W_, U_, K_, V_, want_ckpt=True, workspace=ws)
-        got = W.backward(W_, U_, K_, V_, dev(g), ckpt=ck, workspace=ws, kernel=W.WKV_KERNEL_SEGMENT)
+        got = W.backward(W_, U_, K_, V_, dev(g), ckpt=ck, workspace=ws, kernel=BWD_KERNELS[kernel])
         assert ws.status() == 0
         assert_grads(got, grads_ref(w, u, k, v, g), F32_GRAD_TOL)
 
 
-def test_segment_outputs_stay_inside_their_buffers():
+@pytest.mark.parametrize("fwd_kernel", ["segment", "tile"])
+def test_segment_outputs_stay_inside_their_buffers(fwd_kernel):
     B, T, C = 2, 300, 96
     w, u, k, v, g, _ = small_case(B, T, C, seed=27)
     n = B * T * C
@@ -408,8 +412,8 @@ def test_segment_outputs_stay_inside_their_buffers():
     bufs = [torch.full((n + 2 * guard,), 12345.0, device="cuda") for _ in range(3)]
     y, gk, gv = (b_[guard:guard + n].view(B, T, C) for b_ in bufs)
     W_, U_, K_, V_ = dev(w), dev(u), dev(k), dev(v)
-    _, _, ck = W.forward(W_, U_, K_, V_, y=y, want_ckpt=True, kernel=W.WKV_KERNEL_SEGMENT)
-    W.backward(W_, U_, K_, V_, dev(g), ckpt=ck, grad_k=gk, grad_v=gv, kernel=W.WKV_KERNEL_SEGMENT)
+    _, _, ck = W.forward(W_, U_, K_, V_, y=y, want_ckpt=True, kernel=KERNELS[fwd_kernel])
+    W.backward(W_, U_, K_, V_, dev(g), ckpt=ck, grad_k=gk, grad_v=gv, kernel=BWD_KERNELS[fwd_kernel])
     torch.cuda.synchronize()
     for b_ in bufs:
         assert torch.all(b_[:guard] == 12345.0) and torch.all(b_[guard + n:] == 12345.0)
@@ -441,3 +445,18 @@ def test_argument_errors_launch_nothing():
     assert abi.wkv_forward_ex(1, 8, C, 0, p(w), p(w), p(k), p(k), 0, p(y), 0, 0, 0, 0, s,
                               abi.Options(kernel=2)) == -3
     torch.cuda.synchronize()
+
+
+def test_tile_results_are_bit_reproducible_at_full_size():
+    """The tile kernels' look-backs take whatever prefix is published first,
+    but every prefix is the same left fold of unit records: two runs of the
+    RWKV-4 169M-shaped layer give identical bits."""
+    inp = workloads.generate("rwkv169m")
+    w, u, k, v, gy = inputs_to_device(inp)
+    runs = []
+    for _ in range(2):
+        y, s, ck = W.forward(w, u, k, v, want_state=True, want_ckpt=True, kernel=W.WKV_KERNEL_TILE)
+        grads = W.backward(w, u, k, v, gy, ckpt=ck, kernel=W.WKV_KERNEL_TILE)
+        runs.append((y, s, ck) + tuple(grads))
+    for a, b in zip(*runs):
+        assert torch.equal(a, b)
