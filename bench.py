@@ -1,18 +1,25 @@
-"""Benchmark: WKV fwd+bwd channel-tokens/s and achieved HBM GB/s on B200.
+"""Benchmark: WKV channel-tokens/s and achieved HBM GB/s on B200.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libwkv|reference]
-                [--workload rwkv169m|rwkv1b5_bf16|longctx|decode14b] [--gate | --token-shift]
+                [--workload rwkv1b5_bf16|rwkv169m|longctx|decode14b|tiny]
+                [--gate | --token-shift]
 
-A step is one pass of the whole hot path over one batch of the workload:
-``wkv_forward`` (writing the checkpoints) followed by ``wkv_backward`` on the
-same inputs, through the C ABI, inputs resident in HBM.  The default
-workload is the RWKV-4 169M-shaped layer (B8 T1024 C768 fp32, seeded
-synthetic inputs).  L2 is flushed (a 2x-L2 buffer is written) before every
-timed step, outside the timed events; each step is bracketed by CUDA events
-on the launching stream and the per-step times are summed.  ``--gate`` times
-the gated calls instead (``wkv_forward_gated`` / ``wkv_backward_gated``,
-o = sigmoid(r) * wkv, with a seeded N(0, 1) gate input r); ``--token-shift``
-times the token shift (three interpolations) on the workload's layer shape.
+A step is one pass of the hot path over one batch of the workload, through
+the C ABI, with the inputs resident in HBM:
+
+* fwd+bwd workloads (the default, the RWKV-4 1.5B-shaped layer B8 T4096
+  C2048 with bf16 I/O; also rwkv169m, tiny): ``wkv_forward`` (writing the
+  checkpoints) then ``wkv_backward``; value = channel-tokens/s of the pair;
+* ``longctx`` (B1 T65536 C2560 fp32, forward only): ``wkv_forward``;
+* ``decode14b`` (512 sequences x C5120 fp32): after an untimed T128 prefill,
+  32 ``wkv_step`` calls, each with its own pre-staged k_t, v_t, y_t buffers
+  and the state updated in place; value = channel-steps/s over the 32 steps.
+
+L2 is flushed (a 2x-L2 buffer is written, then another read) before every
+timed step, outside the timed events; every kernel call is bracketed by CUDA
+events on the launching stream.  ``--gate`` times the gated calls;
+``--token-shift`` the token shift (three interpolations) on the workload's
+layer shape.
 
 Multi-GPU (torchrun): every rank runs an independent replica of the workload
 on its own GPU (the operator has no cross-sequence exchange; weak scaling);
@@ -24,6 +31,7 @@ operator has) on a bounded sample of the same workload, on rank 0 only.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -39,27 +47,63 @@ sys.path.insert(0, ROOT)
 
 from rwkv_linear_rnn_b200 import workloads  # noqa: E402
 
+CSRC = os.path.join(ROOT, "rwkv_linear_rnn_b200", "csrc")
+
 # algorithmic bytes per channel-token (per channel-step for the decode step)
 # (gated: the forward also reads r; the backward reads r and writes grad_r)
 ALG_BYTES = {("fwd", "f32"): 12, ("fwd", "bf16"): 6, ("bwd", "f32"): 20, ("bwd", "bf16"): 10,
              ("fwd_gated", "f32"): 16, ("fwd_gated", "bf16"): 8, ("bwd_gated", "f32"): 28,
              ("bwd_gated", "bf16"): 14, ("step", "f32"): 36}
 
+# Kernels each call launches on 16-byte aligned rows (every bench workload):
+# (kernel name, launches per call) per kernel selector.  The gated and
+# state-gradient backwards run the segment kernel.
+FWD_PLAN = {"tile": ("fwd_tile_kernel", 1), "segment": ("fwd_seg_kernel", 1), "cluster": ("fwd_clu_kernel", 1)}
+BWD_PLAN = {"tile": ("bwd_tile_kernel", 1), "segment": ("bwd_seg_kernel", 1)}
 
-# Kernels each call launches on 16-byte aligned rows (all bench workloads),
-# per kernel selector: (kernel names, launches per call).
-FWD_PLAN = {"auto": ("fwd_seg_kernel", 1), "segment": ("fwd_seg_kernel", 1),
-            "cluster": ("fwd_clu_kernel", 1)}
-BWD_PLAN = {"auto": ("bwd_seg_kernel", 1),
-            "segment": ("bwd_seg_kernel", 1)}
-KERNEL_IDS = {"auto": 0, "segment": 6, "cluster": 7}
 
-# DRAM bytes (read + write) per launch of the backward's main kernel from one
-# ncu capture of this bench's workload (cold L2; gk/gv lines still dirty in
-# L2 at kernel end are not counted).  Keyed by (workload, kernel, gated); a
-# kernel changed since its capture has no entry (traffic reported as null).
-TRAFFIC = {("rwkv169m", "bwd_seg_kernel", False): 78_219_776 + 416_768,
-           ("rwkv169m", "bwd_seg_kernel", True): 112_421_120 + 24_960_768}
+def auto_kernel(op: str, B: int, C: int, gate: bool, num_sms: int = 148) -> str:
+    """The kernel the library's AUTO selector runs on 16-byte aligned rows of
+    at least one tile unit: the tile kernels when a chain (batch row, 32
+    channels) has at most about four resident warps' units in flight, the
+    segment kernels otherwise (mirrors tile_pays in the C ABI)."""
+    nchains = B * ((C + 31) // 32)
+    warps = (6 if gate else 9) if op == "fwd" else (6 if gate else 8)
+    return "tile" if nchains * 4 >= warps * num_sms else "segment"
+KERNEL_IDS = {"auto": 0, "segment": 6, "cluster": 7, "tile": 8}
+
+# The source files each kernel is built from: a DRAM-traffic figure measured
+# by ncu is reported only while these files are unchanged since the capture.
+KERNEL_SOURCES = {
+    "fwd_tile_kernel": ["wkv_tile.cu", "wkv_tile.cuh", "wkv_internal.cuh", "wkv_math.cuh"],
+    "bwd_tile_kernel": ["wkv_tile_bwd.cu", "wkv_tile.cuh", "wkv_bwd_math.cuh", "wkv_internal.cuh",
+                        "wkv_math.cuh"],
+    "bwd_seg_kernel": ["wkv_seg_bwd.cu", "wkv_ring.cuh", "wkv_bwd_math.cuh", "wkv_internal.cuh",
+                       "wkv_math.cuh"],
+    "fwd_seg_kernel": ["wkv_seg.cu", "wkv_ring.cuh", "wkv_internal.cuh", "wkv_math.cuh"],
+    "step_kernel": ["wkv_step.cu", "wkv_internal.cuh"],
+}
+
+# DRAM bytes (read + write) per launch of a workload's dominant kernel, from
+# one ncu capture (the summaries under profiles/ give the commands), keyed by
+# (workload, kernel, gated, source hash).  A kernel whose sources changed
+# since its capture has no entry: its traffic is reported as null.
+TRAFFIC = {}
+
+
+def kernel_hash(kernel: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, []):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def workload_mode(name: str) -> str:
+    ops = workloads.WORKLOADS[name].ops
+    if "step" in ops:
+        return "step"
+    return "fwdbwd" if "bwd" in ops else "fwd"
 
 
 def peaks():
@@ -154,41 +198,101 @@ def aggregate_rate(units_per_rank: int, n_ranks: int, ms_per_step: float) -> flo
     return n_ranks * units_per_rank / (ms_per_step * 1e-3)
 
 
-def cpu_baseline(wl_name: str, min_seconds: float = 10.0, gate: bool = False):
-    """Time the oracle (float64 recurrence fwd + reverse bwd, gated or not)
-    on the host."""
-    import oracle
-    wl = workloads.WORKLOADS[wl_name]
-    what = "gated fwd+bwd" if gate else "fwd+bwd"
-    if wl_name == "rwkv169m":
-        inp = workloads.generate(wl, gate=gate)
-        sample = f"full rwkv169m workload (B8 T1024 C768) {what}, repeated"
-    else:  # a channel slice of the big workloads keeps the sample bounded
-        C = 256
-        inp = workloads.generate(wl, C=C, T=min(wl.T, 4096), grad=True, gate=gate)
-        sample = f"{wl_name} with C={C}, T={inp['T']} {what}, repeated"
-    names = ("w", "u", "k", "v", "r", "gy") if gate else ("w", "u", "k", "v", "gy")
-    args = [np.asarray(inp[n], np.float64) for n in names]
-    units = inp["B"] * inp["T"] * inp["C"]
+# ------------------------------------------------------------- descriptions ---
+
+def metric_name(mode: str, gate: bool) -> str:
+    what = "gated WKV" if gate else "WKV"
+    if mode == "fwd":
+        return f"{what} fwd channel-tokens/s, long-context scan (HBM GB/s and % of roofline alongside)"
+    if mode == "step":
+        return "WKV decode-step channel-steps/s, RNN mode (HBM GB/s and % of roofline alongside)"
+    return f"{what} fwd+bwd channel-tokens/s (HBM GB/s and % of roofline alongside)"
+
+
+def units_per_step(wl) -> int:
+    """Channel-tokens (channel-steps for the decode workload) of one step."""
+    if workload_mode(wl.name) == "step":
+        return wl.B * wl.C * wl.steps
+    return wl.B * wl.T * wl.C
+
+
+def make_config(args, wl, ws_n: int) -> dict:
+    """The workload description both arms print."""
+    mode = workload_mode(wl.name)
+    cfg = {"workload": wl.name, "mode": mode, "io_dtype": wl.dtype}
+    if mode == "step":
+        cfg.update({"N": wl.B, "C": wl.C, "prefill_T": wl.T, "steps": wl.steps,
+                    "l2": "flushed once before the 32 timed steps (outside events); the state is updated in place"})
+    else:
+        cfg.update({"B": wl.B, "T": wl.T, "C": wl.C,
+                    "l2": "flushed before every timed step (2x L2 write + 2x L2 read, outside events)"})
+    if args.gate:
+        cfg["gate"] = True
+    cfg["parallelism"] = f"replicas x{ws_n}" if ws_n > 1 else "single GPU"
+    return cfg
+
+
+# ------------------------------------------------------------- CPU baseline ---
+
+def _time_loop(fn, min_seconds: float, min_reps: int = 3):
     times = []
     t_end = time.perf_counter() + min_seconds
-    while time.perf_counter() < t_end or len(times) < 3:
+    while time.perf_counter() < t_end or len(times) < min_reps:
         t0 = time.perf_counter()
-        if gate:
-            oracle.fwd_gated(*args[:5])
-            oracle.bwd_gated(*args)
-        else:
-            oracle.fwd_recur(*args[:4], want_y=True)
-            oracle.bwd_recur(*args)
+        fn()
         times.append(time.perf_counter() - t0)
-    med = statistics.median(times)
-    return {"value": units / med, "unit": "channel-tokens/s", "cores": oracle.num_threads(),
-            "kind": "oracle", "sample": f"{sample} x{len(times)}, median"}
+    return statistics.median(times), len(times)
 
 
-def metric_name(gate: bool) -> str:
-    what = "gated WKV" if gate else "WKV"
-    return f"{what} fwd+bwd channel-tokens/s (HBM GB/s and % of roofline alongside)"
+def cpu_baseline(wl_name: str, min_seconds: float = 10.0, gate: bool = False):
+    """Time the oracle (float64) on the host on a bounded sample of the
+    workload: the recurrence forward (+ the reverse-time backward for the
+    fwd+bwd workloads), or the decode step.  Reported on all host threads
+    (OpenMP over the independent chains) and on one thread."""
+    import oracle
+    wl = workloads.WORKLOADS[wl_name]
+    mode = workload_mode(wl_name)
+    if mode == "step":
+        N, C = 512, 512
+        d = workloads.generate_decode_steps(wl, N=N, C=C, steps=2)
+        w, u = np.asarray(d["w"], np.float64), np.asarray(d["u"], np.float64)
+        _, st = oracle.fwd_recur(d["w"], d["u"], d["k"], d["v"], want_y=False)
+        kt, vt = np.asarray(d["k_steps"][0], np.float64), np.asarray(d["v_steps"][0], np.float64)
+        fn = lambda: oracle.step(w, u, kt, vt, st)
+        units = N * C
+        sample = f"decode14b slice N={N} C={C}, one step after the T128 prefill"
+        unit = "channel-steps/s"
+    else:
+        what = "gated fwd+bwd" if gate else ("fwd+bwd" if mode == "fwdbwd" else "fwd")
+        if wl_name in ("rwkv169m", "tiny"):
+            inp = workloads.generate(wl, gate=gate)
+            sample = f"full {wl_name} workload (B{wl.B} T{wl.T} C{wl.C}) {what}"
+        else:  # a channel slice of the big workloads keeps the sample bounded
+            C = 128 if mode == "fwd" else 256
+            inp = workloads.generate(wl, C=C, T=min(wl.T, 65536 if mode == "fwd" else 4096),
+                                     grad=mode == "fwdbwd", gate=gate)
+            sample = f"{wl_name} with C={C}, T={inp['T']} {what}"
+        names = ("w", "u", "k", "v", "r", "gy") if gate else ("w", "u", "k", "v", "gy")
+        args = [np.asarray(inp[n], np.float64) for n in names if n in inp]
+        units = inp["B"] * inp["T"] * inp["C"]
+        unit = "channel-tokens/s"
+        if mode == "fwd":
+            fn = lambda: oracle.fwd_recur(*args[:4], want_y=True)
+        elif gate:
+            fn = lambda: (oracle.fwd_gated(*args[:5]), oracle.bwd_gated(*args))
+        else:
+            fn = lambda: (oracle.fwd_recur(*args[:4], want_y=True), oracle.bwd_recur(*args))
+    cores = oracle.num_threads()
+    med, reps = _time_loop(fn, min_seconds)
+    oracle.set_threads(1)
+    try:
+        med1, reps1 = _time_loop(fn, max(1.0, min_seconds / 4), min_reps=1)
+    finally:
+        oracle.set_threads(cores)
+    return {"value": units / med, "unit": unit, "cores": cores, "kind": "oracle",
+            "sample": f"{sample}, x{reps}, median",
+            "single_thread": {"value": units / med1, "unit": unit, "cores": 1,
+                              "sample": f"{sample}, x{reps1}, median"}}
 
 
 def token_shift_cpu_baseline(wl_name: str, min_seconds: float):
@@ -202,57 +306,47 @@ def token_shift_cpu_baseline(wl_name: str, min_seconds: float):
     xp = rng.standard_normal((B, C))
     mu = rng.random((n, C))
     g = rng.standard_normal((n, B, T, C))
-    times = []
-    t_end = time.perf_counter() + min_seconds
-    while time.perf_counter() < t_end or len(times) < 3:
-        t0 = time.perf_counter()
-        ots.shift(x, mu, xp)
-        ots.shift_bwd(x, mu, g, xp)
-        times.append(time.perf_counter() - t0)
-    med = statistics.median(times)
+    med, reps = _time_loop(lambda: (ots.shift(x, mu, xp), ots.shift_bwd(x, mu, g, xp)), min_seconds)
     return {"value": B * T * C / med, "unit": "channel-tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{wl_name} token shift (B{B} T{T} C{C}, n=3) fwd+bwd x{len(times)}, median"}
+            "sample": f"{wl_name} token shift (B{B} T{T} C{C}, n=3) fwd+bwd x{reps}, median"}
+
+
+def token_shift_config(args, wl, ws_n):
+    return {"workload": args.workload, "op": "token_shift", "B": wl.B, "T": wl.T, "C": wl.C, "n": 3,
+            "io_dtype": wl.dtype, "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
+            "l2": "flushed before every timed step (2x L2 write + 2x L2 read, outside events)"}
 
 
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return
-    if args.token_shift:
-        cb = token_shift_cpu_baseline(args.workload, min_seconds=max(1.0, 2.0 * args.steps))
-        wl = workloads.WORKLOADS[args.workload]
-        line = {"metric": "token-shift fwd+bwd channel-tokens/s (3 interpolations; HBM GB/s alongside)",
-                "value": cb["value"], "unit": "channel-tokens/s", "n_gpus": 1, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": wl.channel_tokens / cb["value"] * 1e3,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic (seeded)", "impl": "reference",
-                "config": {"workload": args.workload, "op": "token_shift", "B": wl.B, "T": wl.T, "C": wl.C,
-                           "n": 3},
-                "cpu_baseline": cb,
-                "e2e": {"value": cb["value"], "unit": "channel-tokens/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
-        return
-    cb = cpu_baseline(args.workload, min_seconds=max(1.0, 2.0 * args.steps), gate=args.gate)
     wl = workloads.WORKLOADS[args.workload]
-    line = {"metric": metric_name(args.gate),
-            "value": cb["value"], "unit": "channel-tokens/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": wl.channel_tokens / cb["value"] * 1e3,
+    secs = max(1.0, 2.0 * args.steps)
+    if args.token_shift:
+        cb = token_shift_cpu_baseline(args.workload, min_seconds=secs)
+        metric = "token-shift fwd+bwd channel-tokens/s (3 interpolations; HBM GB/s alongside)"
+        cfg = token_shift_config(args, wl, 1)
+        units = wl.B * wl.T * wl.C
+    else:
+        cb = cpu_baseline(args.workload, min_seconds=secs, gate=args.gate)
+        metric = metric_name(workload_mode(args.workload), args.gate)
+        cfg = make_config(args, wl, 1)
+        units = units_per_step(wl)
+    line = {"metric": metric, "value": cb["value"], "unit": cb["unit"], "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": units / cb["value"] * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded)", "impl": "reference",
-            "config": {"workload": args.workload, "B": wl.B, "T": wl.T, "C": wl.C,
-                       **({"gate": True} if args.gate else {})},
+            "data": "synthetic (seeded)", "impl": "reference", "config": cfg,
             "cpu_baseline": cb,
-            "e2e": {"value": cb["value"], "unit": "channel-tokens/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": cb["value"], "unit": cb["unit"], "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def run_libwkv(args):
-    import torch
-    import rwkv_linear_rnn_b200 as W
-    from rwkv_linear_rnn_b200 import abi
+# ----------------------------------------------------------------- GPU arm ---
 
+def setup_device():
+    import torch
     ws_n, rank, local = dist_env()
     dist = None
     if ws_n > 1:
@@ -264,30 +358,11 @@ def run_libwkv(args):
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
-    wl = workloads.WORKLOADS[args.workload]
-    if "bwd" not in wl.ops:
-        raise SystemExit(f"workload {args.workload} has no backward; pick a fwd+bwd workload")
-    inp = workloads.generate(wl, seed=wl.seed + 1000 * rank, gate=args.gate)
-    B, T, C = inp["B"], inp["T"], inp["C"]
-    dt = W.WKV_BF16 if inp["dtype"] == "bf16" else W.WKV_F32
-    tdt = torch.bfloat16 if dt == W.WKV_BF16 else torch.float32
+    return ws_n, rank, dist, dev
 
-    def to_dev(name):
-        if dt == W.WKV_BF16 and name in ("k", "v", "gy", "r"):
-            return torch.from_numpy(inp[name + "_bits"].view(np.int16)).to(dev).view(torch.bfloat16)
-        return torch.from_numpy(inp[name]).to(dev)
 
-    w, u, k, v, gy = (to_dev(n) for n in ("w", "u", "k", "v", "gy"))
-    r = to_dev("r") if args.gate else None
-    gr = torch.empty_like(k) if args.gate else None
-    y = torch.empty_like(k)
-    gk = torch.empty_like(k)
-    gv = torch.empty_like(v)
-    gw = torch.empty(C, device=dev)
-    gu = torch.empty(C, device=dev)
-    ckpt = torch.empty(W.wkv_ckpt_size(B, T, C) // 4, device=dev)
-    nws = W.wkv_workspace_size(W.WKV_OP_BACKWARD, B, T, C, dt)
-    wsb = torch.zeros(nws, dtype=torch.uint8, device=dev)
+def make_flush(dev):
+    import torch
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush_w = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
     flush_r = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
@@ -298,34 +373,115 @@ def run_libwkv(args):
         # inputs in L2 nor pay for write-backs of the flush
         flush_w.zero_()
         flush_r.sum()
+    return flush_l2
+
+
+def pipeline_e2e(nsteps, timed, in_names, out_names, host_in, host_out, sets, step_on, streams):
+    """Steps pipelined over three streams (PCIe is full duplex): step i+1's
+    inputs are copied in while step i computes and step i's results are
+    copied out; device tensors are double buffered and events order each
+    buffer's reuse.  Returns ms per step (first H2D start to last D2H end)."""
+    import torch
+    s_in, s_cmp, s_out = streams
+    ev = lambda: torch.cuda.Event(enable_timing=timed)
+    in_done, cmp_done, out_done = [], [], []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(s_in)
+    for i in range(nsteps):
+        bs = sets[i % 2]
+        hin = host_in[i % len(host_in)]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(cmp_done[i - 2])
+            for n in in_names:
+                bs[n].copy_(hin[n], non_blocking=True)
+            in_done.append(ev()); in_done[-1].record(s_in)
+        s_cmp.wait_event(in_done[i])
+        if i >= 2:
+            s_cmp.wait_event(out_done[i - 2])
+        step_on(bs, s_cmp.cuda_stream, i)
+        cmp_done.append(ev()); cmp_done[-1].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(cmp_done[i])
+            for n in out_names:
+                host_out[n].copy_(bs[n], non_blocking=True)
+            out_done.append(ev()); out_done[-1].record(s_out)
+    e1.record(s_out)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / nsteps
+
+
+def traffic_for(workload, kernel, gated):
+    return TRAFFIC.get((workload, kernel, bool(gated), kernel_hash(kernel)))
+
+
+def run_libwkv(args):
+    mode = workload_mode(args.workload)
+    if mode == "step":
+        return run_step(args)
+    import torch
+    import rwkv_linear_rnn_b200 as W
+    from rwkv_linear_rnn_b200 import abi
+
+    ws_n, rank, dist, dev = setup_device()
+    wl = workloads.WORKLOADS[args.workload]
+    with_bwd = mode == "fwdbwd"
+    inp = workloads.generate(wl, seed=wl.seed + 1000 * rank, gate=args.gate, grad=with_bwd)
+    B, T, C = inp["B"], inp["T"], inp["C"]
+    dt = W.WKV_BF16 if inp["dtype"] == "bf16" else W.WKV_F32
+
+    def to_dev(name):
+        if dt == W.WKV_BF16 and name in ("k", "v", "gy", "r"):
+            return torch.from_numpy(inp[name + "_bits"].view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(inp[name]).to(dev)
+
+    w, u, k, v = (to_dev(n) for n in ("w", "u", "k", "v"))
+    del inp["k"], inp["v"]
+    gy = to_dev("gy") if with_bwd else None
+    r = to_dev("r") if args.gate else None
+    gr = torch.empty_like(k) if args.gate and with_bwd else None
+    y = torch.empty_like(k)
+    gk = torch.empty_like(k) if with_bwd else None
+    gv = torch.empty_like(v) if with_bwd else None
+    gw = torch.empty(C, device=dev)
+    gu = torch.empty(C, device=dev)
+    state = torch.empty(3, B, C, device=dev)
+    ckpt = torch.empty(W.wkv_ckpt_size(B, T, C) // 4, device=dev) if with_bwd else None
+    nws = W.wkv_workspace_size(W.WKV_OP_BACKWARD if with_bwd else W.WKV_OP_FORWARD, B, T, C, dt)
+    wsb = torch.zeros(nws, dtype=torch.uint8, device=dev)
+    flush_l2 = make_flush(dev)
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
-    P = lambda t: t.data_ptr()
-
+    P = lambda t: 0 if t is None else t.data_ptr()
     fopt = abi.Options(kernel=KERNEL_IDS[args.fwd_kernel])
     bopt = abi.Options(kernel=KERNEL_IDS[args.bwd_kernel])
 
-    def fwd():
+    def fwd(bs, sp_):
         if args.gate:
-            abi.check(abi.wkv_forward_gated_ex(B, T, C, dt, P(w), P(u), P(k), P(v), P(r), 0, P(y), 0,
-                                               P(ckpt), P(wsb), nws, sp, fopt))
+            abi.check(abi.wkv_forward_gated_ex(B, T, C, dt, P(w), P(u), P(bs["k"]), P(bs["v"]), P(bs["r"]), 0,
+                                               P(bs["y"]), P(bs["state"]), P(ckpt), P(wsb), nws, sp_, fopt))
         else:
-            abi.check(abi.wkv_forward_ex(B, T, C, dt, P(w), P(u), P(k), P(v), 0, P(y), 0, P(ckpt),
-                                         P(wsb), nws, sp, fopt))
+            abi.check(abi.wkv_forward_ex(B, T, C, dt, P(w), P(u), P(bs["k"]), P(bs["v"]), 0, P(bs["y"]),
+                                         P(bs["state"]), P(ckpt), P(wsb), nws, sp_, fopt))
 
-    def bwd():
+    def bwd(bs, sp_):
         if args.gate:
-            abi.check(abi.wkv_backward_gated_ex(B, T, C, dt, P(w), P(u), P(k), P(v), P(r), P(gy), 0,
-                                                P(ckpt), P(gw), P(gu), P(gk), P(gv), P(gr), P(wsb),
-                                                nws, sp, bopt))
+            abi.check(abi.wkv_backward_gated_ex(B, T, C, dt, P(w), P(u), P(bs["k"]), P(bs["v"]), P(bs["r"]),
+                                                P(bs["gy"]), 0, P(ckpt), P(bs["gw"]), P(bs["gu"]), P(bs["gk"]),
+                                                P(bs["gv"]), P(bs["gr"]), P(wsb), nws, sp_, bopt))
         else:
-            abi.check(abi.wkv_backward_ex(B, T, C, dt, P(w), P(u), P(k), P(v), P(gy), 0, P(ckpt),
-                                          P(gw), P(gu), P(gk), P(gv), P(wsb), nws, sp, bopt))
+            abi.check(abi.wkv_backward_ex(B, T, C, dt, P(w), P(u), P(bs["k"]), P(bs["v"]), P(bs["gy"]), 0,
+                                          P(ckpt), P(bs["gw"]), P(bs["gu"]), P(bs["gk"]), P(bs["gv"]), P(wsb),
+                                          nws, sp_, bopt))
 
+    resident = {"k": k, "v": v, "gy": gy, "r": r, "y": y, "gk": gk, "gv": gv, "gw": gw, "gu": gu, "gr": gr,
+                "state": state}
     for _ in range(args.warmup):
         flush_l2()
-        fwd()
-        bwd()
+        fwd(resident, sp)
+        if with_bwd:
+            bwd(resident, sp)
     torch.cuda.synchronize()
     if abi.wkv_get_status(P(wsb), sp) != 0:
         raise SystemExit("device-side status error during warm-up")
@@ -342,9 +498,10 @@ def run_libwkv(args):
     for i in range(K):
         flush_l2()
         ev[i][0].record(stream)
-        fwd()
+        fwd(resident, sp)
         ev[i][1].record(stream)
-        bwd()
+        if with_bwd:
+            bwd(resident, sp)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop(window=(t_begin, time.monotonic()))
@@ -355,68 +512,25 @@ def run_libwkv(args):
     total_ms = max_over_ranks(sum(t_fwd) + sum(t_bwd), dist, dev)
     status = abi.wkv_get_status(P(wsb), sp)
 
-    # e2e: pinned host buffers, every step's copies inside the timed region,
-    # through the same ABI.  Steps are pipelined over three streams (PCIe is
-    # full duplex): step i+1's inputs are copied in while step i computes and
-    # step i's results are copied out; device inputs and outputs are double
-    # buffered, and the events order each buffer's reuse.
     e2e = None
     if not args.no_e2e:
-        in_names = ["k", "v", "gy"] + (["r"] if args.gate else [])
-        out_names = ["y", "gk", "gv", "gw", "gu"] + (["gr"] if args.gate else [])
-        dev_now = {"k": k, "v": v, "gy": gy, "r": r, "y": y, "gk": gk, "gv": gv, "gw": gw, "gu": gu, "gr": gr}
-        host_in = {n: dev_now[n].cpu().pin_memory() for n in in_names}
-        host_out = {n: torch.empty_like(dev_now[n], device="cpu").pin_memory() for n in out_names}
-        sets = [{n: torch.empty_like(dev_now[n]) for n in in_names + out_names} for _ in range(2)]
-        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        in_names = ["k", "v"] + (["gy"] if with_bwd else []) + (["r"] if args.gate else [])
+        out_names = (["y", "gk", "gv", "gw", "gu"] + (["gr"] if args.gate else [])) if with_bwd else ["y", "state"]
+        host_in = [{n: resident[n].cpu().pin_memory() for n in in_names}]
+        host_out = {n: torch.empty_like(resident[n], device="cpu").pin_memory() for n in out_names}
+        sets = [{n: torch.empty_like(resident[n]) for n in in_names + out_names + (["state"] if with_bwd else [])}
+                for _ in range(2)]
+        h2d = sum(t.numel() * t.element_size() for t in host_in[0].values())
         d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-        s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        streams = (torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream())
 
-        def step_on(bs, sp_):
-            if args.gate:
-                abi.check(abi.wkv_forward_gated_ex(B, T, C, dt, P(w), P(u), P(bs["k"]), P(bs["v"]), P(bs["r"]), 0,
-                                                   P(bs["y"]), 0, P(ckpt), P(wsb), nws, sp_, fopt))
-                abi.check(abi.wkv_backward_gated_ex(B, T, C, dt, P(w), P(u), P(bs["k"]), P(bs["v"]), P(bs["r"]),
-                                                    P(bs["gy"]), 0, P(ckpt), P(bs["gw"]), P(bs["gu"]),
-                                                    P(bs["gk"]), P(bs["gv"]), P(bs["gr"]), P(wsb), nws, sp_,
-                                                    bopt))
-            else:
-                abi.check(abi.wkv_forward_ex(B, T, C, dt, P(w), P(u), P(bs["k"]), P(bs["v"]), 0, P(bs["y"]), 0,
-                                             P(ckpt), P(wsb), nws, sp_, fopt))
-                abi.check(abi.wkv_backward_ex(B, T, C, dt, P(w), P(u), P(bs["k"]), P(bs["v"]), P(bs["gy"]), 0,
-                                              P(ckpt), P(bs["gw"]), P(bs["gu"]), P(bs["gk"]), P(bs["gv"]),
-                                              P(wsb), nws, sp_, bopt))
-
-        def pipeline(nsteps, timed):
-            ev = lambda: torch.cuda.Event(enable_timing=timed)
-            in_done, cmp_done, out_done = [], [], []
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            torch.cuda.synchronize()
-            e0.record(s_in)
-            for i in range(nsteps):
-                bs = sets[i % 2]
-                with torch.cuda.stream(s_in):  # inputs of step i (after step i-2 has read this set)
-                    if i >= 2:
-                        s_in.wait_event(cmp_done[i - 2])
-                    for n in in_names:
-                        bs[n].copy_(host_in[n], non_blocking=True)
-                    in_done.append(ev()); in_done[-1].record(s_in)
-                s_cmp.wait_event(in_done[i])  # compute (after step i-2's results are copied out)
-                if i >= 2:
-                    s_cmp.wait_event(out_done[i - 2])
-                step_on(bs, s_cmp.cuda_stream)
-                cmp_done.append(ev()); cmp_done[-1].record(s_cmp)
-                with torch.cuda.stream(s_out):  # results of step i
-                    s_out.wait_event(cmp_done[i])
-                    for n in out_names:
-                        host_out[n].copy_(bs[n], non_blocking=True)
-                    out_done.append(ev()); out_done[-1].record(s_out)
-            e1.record(s_out)
-            torch.cuda.synchronize()
-            return e0.elapsed_time(e1) / nsteps
-
-        pipeline(3, False)  # warm-up
-        e2e_ms = max_over_ranks(pipeline(max(10, min(K, 40)), True), dist, dev)
+        def step_on(bs, sp_, i):
+            fwd(bs, sp_)
+            if with_bwd:
+                bwd(bs, sp_)
+        pipeline_e2e(3, False, in_names, out_names, host_in, host_out, sets, step_on, streams)
+        e2e_ms = max_over_ranks(pipeline_e2e(max(10, min(K, 40)), True, in_names, out_names, host_in, host_out,
+                                             sets, step_on, streams), dist, dev)
         e2e = {"value": aggregate_rate(B * T * C, ws_n, e2e_ms), "unit": "channel-tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "pipelined": "copies of adjacent steps overlap compute and each other"}
@@ -425,45 +539,184 @@ def run_libwkv(args):
         units = B * T * C
         hbm, peak_kind = peaks()
         fwd_ms = statistics.mean(t_fwd)
-        bwd_ms = statistics.mean(t_bwd)
         sfx = "_gated" if args.gate else ""
-        fb = ALG_BYTES[("fwd" + sfx, inp["dtype"])] * units
-        bb = ALG_BYTES[("bwd" + sfx, inp["dtype"])] * units
-        bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9
+        io = inp["dtype"]
+        fb = ALG_BYTES[("fwd" + sfx, io)] * units
         fwd_gbs = fb / (fwd_ms * 1e-3) / 1e9
         step_ms = total_ms / K
-        bwd_names, bwd_launches = BWD_PLAN[args.bwd_kernel]
-        fwd_names, fwd_launches = FWD_PLAN[args.fwd_kernel]
-        main_bwd = bwd_names.split(" + ")[0]
-        traffic = TRAFFIC.get((args.workload, main_bwd, bool(args.gate)))
+        nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+        fsel = auto_kernel("fwd", B, C, args.gate, nsm) if args.fwd_kernel == "auto" else args.fwd_kernel
+        bsel = auto_kernel("bwd", B, C, args.gate, nsm) if args.bwd_kernel == "auto" else args.bwd_kernel
+        fwd_names, fwd_launches = FWD_PLAN[fsel]
+        bwd_names, bwd_launches = BWD_PLAN[bsel]
         line = {
-            "metric": metric_name(args.gate),
+            "metric": metric_name(mode, args.gate),
             "value": aggregate_rate(units, ws_n, step_ms), "unit": "channel-tokens/s",
             "n_gpus": ws_n, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": inp["dtype"], "data": "synthetic (seeded; the RWKV-4 layer shapes and value ranges)",
-            "config": {"workload": args.workload, "B": B, "T": T, "C": C,
-                       **({"gate": True} if args.gate else {}),
-                       "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
-                       "l2": "flushed before every timed step (2x L2 write + 2x L2 read, outside events)"},
-            "roofline": {"bound": "hbm",
-                         "kernel": f"wkv_backward{sfx} call ({bwd_names}), timed as one call",
-                         "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": bwd_gbs / hbm, "traffic": traffic,
-                         "traffic_kernel": main_bwd if traffic else None,
-                         "algorithmic_bytes": bb, "peak_kind": peak_kind},
+            "dtype": "f32", "data": "synthetic (seeded; the RWKV-4 layer shapes and value ranges)",
+            "config": make_config(args, wl, ws_n),
             "fwd": {"kernels": fwd_names, "ms": fwd_ms, "gbs": fwd_gbs, "frac": fwd_gbs / hbm,
-                    "channel_tokens_per_s": units / (fwd_ms * 1e-3)},
-            "bwd": {"kernels": bwd_names, "ms": bwd_ms, "gbs": bwd_gbs, "frac": bwd_gbs / hbm},
-            "fwd_bwd_gbs": (fb + bb) / (step_ms * 1e-3) / 1e9,
-            "clocks": clocks, "gpu_launches": (fwd_launches + bwd_launches) * K,
-            "device_status": status,
+                    "channel_tokens_per_s": units / (fwd_ms * 1e-3), "algorithmic_bytes": fb},
+            "clocks": clocks, "device_status": status,
+            "gpu_launches": (fwd_launches + (bwd_launches if with_bwd else 0)) * K,
+        }
+        if with_bwd:
+            bwd_ms = statistics.mean(t_bwd)
+            bb = ALG_BYTES[("bwd" + sfx, io)] * units
+            bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9
+            line["bwd"] = {"kernels": bwd_names, "ms": bwd_ms, "gbs": bwd_gbs, "frac": bwd_gbs / hbm,
+                           "algorithmic_bytes": bb}
+            line["fwd_bwd_gbs"] = (fb + bb) / (step_ms * 1e-3) / 1e9
+            dom, dom_ms, dom_b, dom_gbs = bwd_names, bwd_ms, bb, bwd_gbs
+            call = f"wkv_backward{sfx}"
+        else:
+            dom, dom_ms, dom_b, dom_gbs = fwd_names, fwd_ms, fb, fwd_gbs
+            call = f"wkv_forward{sfx}"
+        traffic = traffic_for(args.workload, dom, args.gate)
+        line["roofline"] = {"bound": "hbm", "kernel": f"{call} call ({dom}), timed as one call with CUDA events",
+                            "achieved": dom_gbs, "peak": hbm, "unit": "GB/s", "frac": dom_gbs / hbm,
+                            "traffic": traffic, "traffic_kernel": dom if traffic else None,
+                            "algorithmic_bytes": dom_b, "ms": dom_ms, "peak_kind": peak_kind}
+        if e2e:
+            line["e2e"] = e2e
+        if not args.no_cpu_baseline and ws_n == 1:
+            line["cpu_baseline"] = cpu_baseline(args.workload, min_seconds=args.cpu_seconds, gate=args.gate)
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_step(args):
+    """decode14b: an untimed T128 prefill sets the state of N sequences; a
+    step is 32 wkv_step calls, each with its own k_t, v_t, y_t buffers."""
+    import torch
+    import rwkv_linear_rnn_b200 as W
+    from rwkv_linear_rnn_b200 import abi
+
+    ws_n, rank, dist, dev = setup_device()
+    wl = workloads.WORKLOADS[args.workload]
+    d = workloads.generate_decode_steps(wl, seed=wl.seed + 1000 * rank)
+    N, T0, C, S = d["N"], d["T"], d["C"], wl.steps
+    w = torch.from_numpy(d["w"]).to(dev)
+    u = torch.from_numpy(d["u"]).to(dev)
+    kp = torch.from_numpy(d["k"]).to(dev)
+    vp = torch.from_numpy(d["v"]).to(dev)
+    ks = torch.from_numpy(d["k_steps"]).to(dev)
+    vs = torch.from_numpy(d["v_steps"]).to(dev)
+    ys = torch.empty_like(ks)
+    state0 = torch.empty(3, N, C, device=dev)
+    state = torch.empty_like(state0)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    P = lambda t: t.data_ptr()
+    yp = torch.empty_like(kp)
+    nws = W.wkv_workspace_size(W.WKV_OP_FORWARD, N, T0, C, W.WKV_F32)
+    wsb = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
+    abi.check(abi.wkv_forward(N, T0, C, W.WKV_F32, P(w), P(u), P(kp), P(vp), 0, P(yp), P(state0), 0, P(wsb),
+                              nws, sp))
+    del kp, vp, yp
+    flush_l2 = make_flush(dev)
+
+    def one(i, kt, vt, yt, sp_):
+        abi.check(abi.wkv_step(N, C, P(w), P(u), P(kt), P(vt), P(state), P(yt), P(state), sp_))
+
+    for _ in range(args.warmup):
+        state.copy_(state0)
+        flush_l2()
+        for i in range(S):
+            one(i, ks[i], vs[i], ys[i], sp)
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(S + 1)] for _ in range(K)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t_begin = time.monotonic()
+    for it in range(K):
+        state.copy_(state0)  # every timed step decodes from the prefill state
+        flush_l2()
+        ev[it][0].record(stream)
+        for i in range(S):
+            one(i, ks[i], vs[i], ys[i], sp)
+            ev[it][i + 1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop(window=(t_begin, time.monotonic()))
+    if dist:
+        dist.barrier()
+    per_call = [ev[it][i].elapsed_time(ev[it][i + 1]) for it in range(K) for i in range(S)]
+    seq = [ev[it][0].elapsed_time(ev[it][S]) for it in range(K)]
+    total_ms = max_over_ranks(sum(seq), dist, dev)
+    # the same step kernel with L2 flushed before every call (each call's
+    # state then comes from HBM): a per-call figure free of L2 reuse
+    flushed = []
+    for it in range(min(K, 5)):
+        state.copy_(state0)
+        for i in range(S):
+            flush_l2()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            one(i, ks[i], vs[i], ys[i], sp)
+            e1.record(stream)
+            flushed.append((e0, e1))
+    torch.cuda.synchronize()
+    flushed_ms = statistics.mean(a.elapsed_time(b) for a, b in flushed)
+
+    e2e = None
+    if not args.no_e2e:
+        # each call's k_t, v_t come from pinned host memory and its y_t goes
+        # back; the state stays resident (it is the decoder's own state)
+        host_in = [{"kt": ks[i].cpu().pin_memory(), "vt": vs[i].cpu().pin_memory()} for i in range(S)]
+        host_out = {"yt": torch.empty_like(ys[0], device="cpu").pin_memory()}
+        sets = [{"kt": torch.empty_like(ks[0]), "vt": torch.empty_like(vs[0]), "yt": torch.empty_like(ys[0])}
+                for _ in range(2)]
+        streams = (torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream())
+
+        def step_on(bs, sp_, i):
+            one(i, bs["kt"], bs["vt"], bs["yt"], sp_)
+        state.copy_(state0)
+        pipeline_e2e(3, False, ["kt", "vt"], ["yt"], host_in, host_out, sets, step_on, streams)
+        state.copy_(state0)
+        torch.cuda.synchronize()
+        call_ms = max_over_ranks(pipeline_e2e(S, True, ["kt", "vt"], ["yt"], host_in, host_out, sets, step_on,
+                                              streams), dist, dev)
+        e2e = {"value": aggregate_rate(N * C, ws_n, call_ms), "unit": "channel-steps/s",
+               "h2d_bytes_per_step": S * 2 * N * C * 4, "d2h_bytes_per_step": S * N * C * 4,
+               "ms_per_step": call_ms * S,
+               "pipelined": "each call's k_t, v_t copied in while the previous call computes; y_t copied out"}
+
+    if rank == 0:
+        hbm, peak_kind = peaks()
+        step_ms = total_ms / K
+        call_ms_dev = statistics.mean(per_call)
+        b_call = ALG_BYTES[("step", "f32")] * N * C
+        gbs = b_call / (call_ms_dev * 1e-3) / 1e9
+        gbs_flushed = b_call / (flushed_ms * 1e-3) / 1e9
+        traffic = traffic_for(args.workload, "step_kernel", False)
+        line = {
+            "metric": metric_name("step", False),
+            "value": aggregate_rate(N * C * S, ws_n, step_ms), "unit": "channel-steps/s",
+            "n_gpus": ws_n, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded; RWKV-4 14B-shaped decode batch)",
+            "config": make_config(args, wl, ws_n),
+            "roofline": {"bound": "hbm", "kernel": "wkv_step call (step_kernel), mean of the 32 calls of a step",
+                         "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm, "traffic": traffic,
+                         "traffic_kernel": "step_kernel" if traffic else None, "algorithmic_bytes": b_call,
+                         "ms": call_ms_dev, "peak_kind": peak_kind,
+                         "note": "the state written by one call is partly still in L2 when the next reads it"},
+            "step_l2_flushed_each_call": {"ms": flushed_ms, "gbs": gbs_flushed, "frac": gbs_flushed / hbm},
+            "clocks": clocks, "gpu_launches": S * K,
         }
         if e2e:
             line["e2e"] = e2e
         if not args.no_cpu_baseline and ws_n == 1:
-            line["cpu_baseline"] = cpu_baseline(args.workload, min_seconds=args.cpu_seconds,
-                                                gate=args.gate)
+            line["cpu_baseline"] = cpu_baseline(args.workload, min_seconds=args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -477,17 +730,7 @@ def run_token_shift(args):
     import rwkv_linear_rnn_b200 as W
     from rwkv_linear_rnn_b200 import abi
 
-    ws_n, rank, local = dist_env()
-    dist = None
-    if ws_n > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    dev = torch.device("cuda", torch.cuda.current_device())
+    ws_n, rank, dist, dev = setup_device()
     wl = workloads.WORKLOADS[args.workload]
     B, T, C, n = wl.B, wl.T, wl.C, 3
     dt = W.WKV_BF16 if wl.dtype == "bf16" else W.WKV_F32
@@ -504,9 +747,7 @@ def run_token_shift(args):
     gxp = torch.empty_like(xp)
     nws = abi.wkv_token_shift_workspace_size(B, T, C, n)
     wsb = torch.empty(nws, dtype=torch.uint8, device=dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush_w = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
-    flush_r = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
+    flush_l2 = make_flush(dev)
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
     P = lambda t: t.data_ptr()
@@ -519,7 +760,7 @@ def run_token_shift(args):
                                                P(gxp), P(wsb), nws, sp))
 
     for _ in range(args.warmup):
-        flush_w.zero_(); flush_r.sum(); fwd(); bwd()
+        flush_l2(); fwd(); bwd()
     torch.cuda.synchronize()
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
@@ -531,7 +772,7 @@ def run_token_shift(args):
     time.sleep(0.3)
     t_begin = time.monotonic()
     for i in range(K):
-        flush_w.zero_(); flush_r.sum()
+        flush_l2()
         ev[i][0].record(stream); fwd(); ev[i][1].record(stream); bwd(); ev[i][2].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop(window=(t_begin, time.monotonic()))
@@ -577,11 +818,9 @@ def run_token_shift(args):
             "metric": "token-shift fwd+bwd channel-tokens/s (3 interpolations; HBM GB/s alongside)",
             "value": aggregate_rate(units, ws_n, step_ms), "unit": "channel-tokens/s",
             "n_gpus": ws_n, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded normal x, uniform mu)",
-            "config": {"workload": args.workload, "op": "token_shift", "B": B, "T": T, "C": C, "n": n,
-                       "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
-                       "l2": "flushed before every timed step (2x L2 write + 2x L2 read, outside events)"},
+            "config": token_shift_config(args, wl, ws_n),
             "roofline": {"bound": "hbm", "kernel": "wkv_token_shift_backward call, timed as one call",
                          "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s", "frac": bwd_gbs / hbm,
                          "traffic": None, "algorithmic_bytes": bb, "peak_kind": peak_kind},
@@ -602,21 +841,23 @@ def run_token_shift(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)  # about a second: clock samples land inside
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="libwkv", choices=["libwkv", "reference"])
-    ap.add_argument("--workload", default="rwkv169m")
+    ap.add_argument("--workload", default="rwkv1b5_bf16", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--fwd-kernel", default="auto", choices=sorted(FWD_PLAN))
-    ap.add_argument("--bwd-kernel", default="auto", choices=sorted(BWD_PLAN))
+    ap.add_argument("--fwd-kernel", default="auto", choices=["auto"] + sorted(FWD_PLAN))
+    ap.add_argument("--bwd-kernel", default="auto", choices=["auto"] + sorted(BWD_PLAN))
     ap.add_argument("--gate", action="store_true",
                     help="time the gated calls (o = sigmoid(r) * wkv and its gradients)")
     ap.add_argument("--token-shift", action="store_true",
                     help="time the token shift (3 interpolations) on the workload's layer shape")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    if args.gate and workload_mode(args.workload) == "step":
+        raise SystemExit("--gate applies to the forward/backward workloads")
     if args.impl == "reference":
         run_reference(args)
     elif args.token_shift:
