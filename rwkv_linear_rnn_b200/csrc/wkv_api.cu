@@ -78,7 +78,7 @@ bool sizes_ok(int64_t B, int64_t T, int64_t C) {
 }
 
 struct Layout {
-  size_t flags, desc, desc_bytes, ckpt, part, cnt, rec, total;
+  size_t flags, desc, desc_bytes, ckpt, part, cnt, rec, sums, total;
   int64_t nct, nchains, nchunks_f, nchunks_b;
 };
 
@@ -113,6 +113,10 @@ Layout layout(int op, int64_t B, int64_t T, int64_t C) {
     off = align_up(off + sizeof(float) * 4 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
     L.cnt = off;  // per channel tile counters of the segment backward's reduction (cleared by it)
     off = align_up(off + sizeof(unsigned) * (size_t)L.nct, 256);
+    // the tile backward's per-chain sums of dL/dw, dL/du, then its
+    // first-level sums (one 16-byte word per (b, c) and group of 16 units)
+    L.sums = off;
+    off = align_up(off + 16 * (size_t)(B * C) * (size_t)(1 + cdiv(L.nchunks_b, 16)), 256);
   }
   L.total = off;
   return L;
@@ -329,8 +333,8 @@ int backward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, co
       aligned(grad_v, 16)) {
     // the per-chain sums of dL/dw, dL/du use the descriptor region (16 bytes
     // per (b, c) <= 640 bytes per chain and chunk), idle in the tile kernels
-    return cuda_rc(launch_backward_tile(a, dtype, grad_w, grad_u, reinterpret_cast<float4 *>(base + L.rec),
-                                        reinterpret_cast<float4 *>(base + L.desc), num_sms(), st));
+    float4 *rec = reinterpret_cast<float4 *>(base + L.rec), *sums = reinterpret_cast<float4 *>(base + L.sums);
+    return cuda_rc(launch_backward_tile(a, dtype, grad_w, grad_u, rec, sums, num_sms(), st));
   }
   if (bwd_uses_seg(B, T, C, dtype, k, v, grad_y, opt)) {
     const int64_t scratch = (int64_t)(L.desc_bytes / sizeof(double));

@@ -299,22 +299,24 @@ __global__ void __launch_bounds__(kTileFwdWarps * 32, 3) fwd_tile_kernel(const _
 #pragma unroll 1
   for (int t = 0; t < nu; ++t) {
     // ---- u_t's look-back, predicted: the units of its chain that run in
-    // step t (positions p0 .. pos-1) published their summaries in step t-1,
-    // and the unit before them (position p0-1, run in step t-1) its prefix.
-    // Their loads are issued now and checked after the next unit's pass 1.
+    // step t (positions from p0) published their summaries in step t-1, and
+    // the unit before them (position p0-1, run in step t-1) its prefix; a
+    // chain's first unit publishes only its prefix, so the fold starts from
+    // the prefix at position qi = max(p0 - 1, 0) and adds the summaries of
+    // positions qi+1 .. pos-1.  Their loads are issued now and checked after
+    // the next unit's pass 1.
     const int p0 = max(0, (int)(((int64_t)t * G - cur.chain + nchains - 1) / nchains));
-    const int dspec = cur.pos - p0;
+    const int qi = max(p0 - 1, 0);
+    const int dspec = cur.pos - 1 - qi;
     const bool spec = cur.pos > 0 && dspec <= kSpecDepth;
     float4 sx = make_float4(0.f, 0.f, 0.f, 0.f), sy = sx, sa[kSpecDepth];
     if (spec) {
-      if (p0 > 0) {
-        const float4 *d = a.rec + ((int64_t)(p0 - 1) * nchains + cur.chain) * kFwdRecWords + lane;
-        sx = ld_relaxed_v4(d + 32);
-        sy = ld_relaxed_v4(d + 64);
-      }
+      const float4 *d = a.rec + ((int64_t)qi * nchains + cur.chain) * kFwdRecWords + lane;
+      sx = ld_relaxed_v4(d + 32);
+      sy = ld_relaxed_v4(d + 64);
 #pragma unroll
       for (int j = 0; j < kSpecDepth; ++j)
-        if (j < dspec) sa[j] = ld_relaxed_v4(a.rec + ((int64_t)(p0 + j) * nchains + cur.chain) * kFwdRecWords + lane);
+        if (j < dspec) sa[j] = ld_relaxed_v4(a.rec + ((int64_t)(qi + 1 + j) * nchains + cur.chain) * kFwdRecWords + lane);
     }
     // ---- pass 1 of the next unit
     TileUnit nxt = cur;
@@ -338,17 +340,37 @@ __global__ void __launch_bounds__(kTileFwdWarps * 32, 3) fwd_tile_kernel(const _
     if (U.pos > 0) {
       bool got = false;
       if (spec) {
-        bool ok = p0 == 0 || (tag_is(sx.w, t_inc) && tag_is(sy.y, t_inc));
-        St acc = p0 == 0 ? s_in : St{sx.x, sx.y, sx.z, sy.x};
+        // the predicted records; a word that does not check yet is read
+        // again until it does (its unit runs in this step or the last, and
+        // publishes without waiting on this warp), within the wait bound
+        const float4 *dinc = a.rec + ((int64_t)qi * nchains + U.chain) * kFwdRecWords + lane;
+        const uint64_t t_start = global_ns();
+        for (;;) {
+          bool ok = tag_is(sx.w, t_inc) && tag_is(sy.y, t_inc);
 #pragma unroll
-        for (int j = 0; j < kSpecDepth; ++j) {
-          if (j < dspec) {
-            ok = ok && tag_is(sa[j].w, t_agg);
-            acc = combine(acc, St{sa[j].x, sa[j].y, sa[j].z, 0.f}, (float)L, U.w2);
+          for (int j = 0; j < kSpecDepth; ++j) ok = ok && (j >= dspec || tag_is(sa[j].w, t_agg));
+          if (__all_sync(0xffffffffu, ok)) {
+            got = true;
+            break;
           }
+          if ((int64_t)(global_ns() - t_start) > budget || launch_aborted(p.hdr, epoch)) break;
+          __nanosleep(64);
+          if (!(tag_is(sx.w, t_inc) && tag_is(sy.y, t_inc))) {
+            sx = ld_relaxed_v4(dinc + 32);
+            sy = ld_relaxed_v4(dinc + 64);
+          }
+#pragma unroll
+          for (int j = 0; j < kSpecDepth; ++j)
+            if (j < dspec && !tag_is(sa[j].w, t_agg))
+              sa[j] = ld_relaxed_v4(a.rec + ((int64_t)(qi + 1 + j) * nchains + U.chain) * kFwdRecWords + lane);
         }
-        got = __all_sync(0xffffffffu, ok);
-        if (got) carry = acc;
+        if (got) {
+          St acc = St{sx.x, sx.y, sx.z, sy.x};
+#pragma unroll
+          for (int j = 0; j < kSpecDepth; ++j)
+            if (j < dspec) acc = combine(acc, St{sa[j].x, sa[j].y, sa[j].z, 0.f}, (float)L, U.w2);
+          carry = acc;
+        }
       }
       if (!got)
         carry = tile_lookback(p.flags, a.rec, U.pos, U.chain, nchains, epoch, s_in, (float)L, U.w2, budget, p.hdr,

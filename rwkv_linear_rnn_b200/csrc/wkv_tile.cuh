@@ -111,6 +111,68 @@ __device__ __forceinline__ void tile_put_inc(float4 *rec, int64_t unit, const St
   st_relaxed_v4(d + 64, make_float4(s.n, tagf(tag), 0.f, 0.f));
 }
 
+// dL/dw, dL/du partials of the tile backwards: one tagged word (gw, gu, tag,
+// 0) per (unit position, b, c).  Sums of n such words spaced `stride` words
+// apart, in index order in float64, sixteen loads in flight, re-reading
+// words whose tag does not check yet (their stores may still be on the way).
+// False if the wait bound ran out.  (Eight loads in flight.)
+constexpr int kPartGroup = 16;  // positions per first-level sum
+__device__ __forceinline__ bool sum_tagged(const float4 *p, int64_t stride, int n, unsigned tag, double &sx,
+                                           double &sy, int64_t budget_ns) {
+  sx = 0.0;
+  sy = 0.0;
+  const uint64_t t0 = global_ns();
+  for (int i0 = 0; i0 < n; i0 += 8) {
+    float4 r[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (i0 + j < n) r[j] = ld_relaxed_v4(p + (int64_t)(i0 + j) * stride);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (i0 + j < n) {
+        while (!tag_is(r[j].z, tag)) {
+          if ((int64_t)(global_ns() - t0) > budget_ns) return false;
+          __nanosleep(64);
+          r[j] = ld_relaxed_v4(p + (int64_t)(i0 + j) * stride);
+        }
+        sx += (double)r[j].x;
+        sy += (double)r[j].y;
+      }
+    }
+  }
+  return true;
+}
+// The fixed-order sums of one channel's partials, called by the warp that ran
+// the unit at position `pos` after it stored its own partial: a unit at a
+// position that is a multiple of kPartGroup adds the partials of its group
+// (positions pos .. pos + kPartGroup - 1, later in time, so earlier in scan
+// order) into a first-level word; the chain's first unit adds the first-level
+// words into the chain's sum; the chain of the last batch row of a channel
+// tile then adds the chains.  Every word waited on comes from a unit earlier
+// in scan order, which never waits on this warp.  part: [nseg][B][C] words,
+// l1: [ceil(nseg / kPartGroup)][B][C], chain: [B][C].  Out of line: it runs
+// once per kPartGroup units and keeps its registers out of the unit loop.
+static __device__ __noinline__ void reduce_partials(const float4 *part, float4 *l1, float4 *chain, float *gw, float *gu,
+                                                int pos, int nseg, int64_t b, int64_t B, int64_t c, int64_t C,
+                                                unsigned tag, int64_t budget_ns, WsHeader *hdr, unsigned epoch) {
+  if (pos % kPartGroup != 0) return;
+  const int64_t BC = B * C, bc = b * C + c;
+  bool ok = true;
+  double sw, su;
+  ok = sum_tagged(part + (int64_t)pos * BC + bc, BC, min(kPartGroup, nseg - pos), tag, sw, su, budget_ns) && ok;
+  st_relaxed_v4(l1 + (int64_t)(pos / kPartGroup) * BC + bc, make_float4((float)sw, (float)su, tagf(tag), 0.f));
+  if (pos == 0) {
+    ok = sum_tagged(l1 + bc, BC, (nseg + kPartGroup - 1) / kPartGroup, tag, sw, su, budget_ns) && ok;
+    st_relaxed_v4(chain + bc, make_float4((float)sw, (float)su, tagf(tag), 0.f));
+    if (b == B - 1) {
+      ok = sum_tagged(chain + c, C, (int)B, tag, sw, su, budget_ns) && ok;
+      gw[c] = (float)sw;
+      gu[c] = (float)su;
+    }
+  }
+  if (!ok) raise_timeout(hdr, epoch);
+}
+
 // Tokens per unit of the tile kernels for an element type (0 fp32, 1 bf16).
 int tile_fwd_tokens(int dtype);
 

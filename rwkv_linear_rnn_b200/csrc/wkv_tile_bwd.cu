@@ -49,40 +49,11 @@ bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T
 struct TileBwdArgs {
   BwdArgs p;
   float *gw, *gu;
-  float4 *chain_sum;        // [B][C] tagged per-chain sums (dL/dw, dL/du, tag, 0)
+  float4 *chain_sum;        // [B][C] per-chain sums, then [ceil(nseg/16)][B][C] first-level sums
   float4 *rec;         // [units][2 slots][2 words][32 lanes] tagged adjoint records
   int64_t nseg;        // units per chain
 };
 
-// Reads n tagged words (x, y, tag, _) spaced `stride` float4 apart and adds
-// their (x, y) in index order in float64, re-reading words whose tag does not
-// check yet (their stores may still be on the way).  Bounded like the
-// look-back.
-__device__ __forceinline__ bool sum_tagged(const float4 *p, int64_t stride, int n, unsigned tag, double &sx,
-                                           double &sy, int64_t budget_ns) {
-  sx = 0.0;
-  sy = 0.0;
-  const uint64_t t0 = global_ns();
-  for (int i0 = 0; i0 < n; i0 += 8) {
-    float4 r[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (i0 + j < n) r[j] = ld_relaxed_v4(p + (int64_t)(i0 + j) * stride);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (i0 + j < n) {
-        while (!tag_is(r[j].z, tag)) {
-          if ((int64_t)(global_ns() - t0) > budget_ns) return false;
-          __nanosleep(64);
-          r[j] = ld_relaxed_v4(p + (int64_t)(i0 + j) * stride);
-        }
-        sx += (double)r[j].x;
-        sy += (double)r[j].y;
-      }
-    }
-  }
-  return true;
-}
 
 // Adjoint records, 2 KB per unit, tagged as the forward's (see wkv_tile.cuh):
 // slot 0 the unit's aggregate, slot 1 its inclusive suffix (the adjoint at
@@ -476,26 +447,14 @@ __global__ void __launch_bounds__(NW * 32, NW == 4 ? 2 : 3) bwd_tile_kernel(cons
         if (t0 == 0 && p.gs_in) store_state_grad(p.gs_in, p.state_in, bc, BC, rah, rhh, fmaf(-m, w2, Ranc));
       }
     }
-    // dL/dw, dL/du: the unit's partial as a tagged word.  The chain's first
-    // unit in time is the last in scan order: the warp that runs it adds the
-    // chain's partials in position order once their words check, and the
-    // warp that runs the last chain of a channel tile (batch row B-1) adds
-    // the tile's chains in batch-row order (both in float64; the order depends
-    // on the shapes alone).  Every word waited on comes from a unit earlier in
-    // scan order, which never waits on these warps: no deadlock.
+    // dL/dw, dL/du: the unit's partial as a tagged word, then the
+    // fixed-order sums (reduce_partials)
     const unsigned t_part = tile_flag(epoch, 3u);
     float4 *part = reinterpret_cast<float4 *>(p.part);
-    if (cok) st_relaxed_v4(part + (int64_t)pos * BC + bc, make_float4(gw_acc, gu_acc, tagf(t_part), 0.f));
-    if (pos == 0 && cok) {
-      double sw, su;
-      if (!sum_tagged(part + bc, BC, nseg, t_part, sw, su, budget)) raise_timeout(p.hdr, epoch);
-      st_relaxed_v4(a.chain_sum + bc, make_float4((float)sw, (float)su, tagf(t_part), 0.f));
-      if (b == p.B - 1) {
-        double tw, tu;
-        if (!sum_tagged(a.chain_sum + c, C, (int)p.B, t_part, tw, tu, budget)) raise_timeout(p.hdr, epoch);
-        a.gw[c] = (float)tw;
-        a.gu[c] = (float)tu;
-      }
+    if (cok) {
+      st_relaxed_v4(part + (int64_t)pos * BC + bc, make_float4(gw_acc, gu_acc, tagf(t_part), 0.f));
+      reduce_partials(part, a.chain_sum + BC, a.chain_sum, a.gw, a.gu, pos, nseg, b, p.B, c, C, t_part, budget,
+                      p.hdr, epoch);
     }
     fence_proxy_async_smem();
     __syncwarp();

@@ -460,3 +460,23 @@ def test_tile_results_are_bit_reproducible_at_full_size():
         runs.append((y, s, ck) + tuple(grads))
     for a, b in zip(*runs):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [32, 33, 64, 65, 96])
+def test_tile_unit_boundaries(T, dtype):
+    """Lengths at and just past one and two tile units (32 fp32 / 64 bf16
+    tokens): a chain of a single unit, a ragged last unit, and the group
+    boundaries of the backward's fixed-order sums."""
+    B, C = 3, 96
+    w, u, k, v, g, _ = small_case(B, T, C, seed=T * 11 + len(dtype), dtype=dtype)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    K_, V_, G_ = dev(k, tdt), dev(v, tdt), dev(g, tdt)
+    W_, U_ = dev(w), dev(u)
+    y, s, ck = W.forward(W_, U_, K_, V_, want_state=True, want_ckpt=True, kernel=W.WKV_KERNEL_TILE)
+    y_ref, s_ref = oracle.fwd_recur(w, u, k, v)
+    tol_f = BF16_TOL if dtype == "bf16" else F32_FWD_TOL
+    assert fwd_err(host(y), y_ref) <= tol_f
+    assert state_err(host(s), s_ref) <= F32_FWD_TOL * (10 if dtype == "bf16" else 1)
+    got = W.backward(W_, U_, K_, V_, G_, ckpt=ck, kernel=W.WKV_KERNEL_TILE)
+    assert_grads(got, grads_ref(w, u, k, v, g), BF16_TOL if dtype == "bf16" else F32_GRAD_TOL)
