@@ -88,7 +88,12 @@ KERNEL_SOURCES = {
 # one ncu capture (the summaries under profiles/ give the commands), keyed by
 # (workload, kernel, gated, source hash).  A kernel whose sources changed
 # since its capture has no entry: its traffic is reported as null.
-TRAFFIC = {}
+TRAFFIC = {
+    ("rwkv1b5_bf16", "bwd_tile_kernel", False, "3e37f5ec7a6ae4a4"): 419_564_544 + 294_213_120,
+    ("rwkv1b5_bf16", "fwd_tile_kernel", False, "8c380ad936d96fa8"): 279_003_904 + 155_246_848,
+    ("longctx", "fwd_seg_kernel", False, "90dd4931d4709195"): 1_569_629_184 + 639_891_200,
+    ("decode14b", "step_kernel", False, "7c9eb86718fc5d51"): 52_482_920 + 68_656,
+}
 
 
 def kernel_hash(kernel: str) -> str:
@@ -557,7 +562,8 @@ def run_libwkv(args):
             "dtype": "f32", "data": "synthetic (seeded; the RWKV-4 layer shapes and value ranges)",
             "config": make_config(args, wl, ws_n),
             "fwd": {"kernels": fwd_names, "ms": fwd_ms, "gbs": fwd_gbs, "frac": fwd_gbs / hbm,
-                    "channel_tokens_per_s": units / (fwd_ms * 1e-3), "algorithmic_bytes": fb},
+                    "channel_tokens_per_s": units / (fwd_ms * 1e-3), "algorithmic_bytes": fb,
+                    "traffic": traffic_for(args.workload, fwd_names, args.gate)},
             "clocks": clocks, "device_status": status,
             "gpu_launches": (fwd_launches + (bwd_launches if with_bwd else 0)) * K,
         }
