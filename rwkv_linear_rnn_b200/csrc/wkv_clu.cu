@@ -271,10 +271,9 @@ static cudaError_t launch_clu_t(const FwdArgs &f, int dtype, int num_sms, int ts
     return cudaErrorInvalidValue;
   using Sm = CluSmem<E, S, RB, W>;
   auto kern = fwd_clu_kernel<E, S, RB, W>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::BYTES);
-  if (e != cudaSuccess) return e;
   int occ = 0;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, W * 32, Sm::BYTES)) != cudaSuccess) return e;
+  cudaError_t e = blocks_per_sm((const void *)kern, W * 32, Sm::BYTES, &occ);
+  if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   // Slots per chain: enough warps to fill the GPU once (at least one block,
   // at most eight per cluster); then rounds so that segments stay within

@@ -18,6 +18,9 @@
 //                       from HBM once and stay in registers between passes.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <string.h>
+
+#include <mutex>
 
 #include "wkv_internal.cuh"
 #include "wkv_math.cuh"
@@ -433,9 +436,110 @@ static bool ensure_context() {
   return cudaGetDevice(&dev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess;
 }
 
+// Encoded tensor maps, remembered by their arguments.  A map is a pure
+// function of (rank, address, element type, extents, box): the same key
+// always encodes to the same 128 bytes, whichever context or thread asks, so
+// a hit is returned as is and a training loop that calls with the same
+// buffers pays for each encoding once.  A small table with round-robin
+// replacement; the lock is held only for the lookup or the insertion.
+namespace {
+struct MapKey {
+  const void *ptr;
+  int64_t d0, d1, d2;
+  int dtype, rank, box;
+  bool operator==(const MapKey &o) const {
+    return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && dtype == o.dtype && rank == o.rank &&
+           box == o.box;
+  }
+};
+constexpr int kMapSlots = 64;
+struct MapCache {
+  std::mutex mu;
+  MapKey key[kMapSlots];
+  bool used[kMapSlots] = {};
+  alignas(64) CUtensorMap map[kMapSlots];
+  int next = 0;
+};
+MapCache &map_cache() {
+  static MapCache c;
+  return c;
+}
+bool map_lookup(const MapKey &k, CUtensorMap *out) {
+  MapCache &c = map_cache();
+  std::lock_guard<std::mutex> lock(c.mu);
+  for (int i = 0; i < kMapSlots; ++i)
+    if (c.used[i] && c.key[i] == k) {
+      memcpy(out, &c.map[i], sizeof(CUtensorMap));
+      return true;
+    }
+  return false;
+}
+void map_insert(const MapKey &k, const CUtensorMap &m) {
+  MapCache &c = map_cache();
+  std::lock_guard<std::mutex> lock(c.mu);
+  const int i = c.next;
+  c.next = (c.next + 1) % kMapSlots;
+  c.key[i] = k;
+  memcpy(&c.map[i], &m, sizeof(CUtensorMap));
+  c.used[i] = true;
+}
+
+struct OccKey {
+  int dev;
+  const void *kern;
+  int threads, smem;
+};
+constexpr int kOccSlots = 256;
+struct OccCache {
+  std::mutex mu;
+  OccKey key[kOccSlots];
+  int blocks[kOccSlots];
+  int n = 0;
+  // per (device, kernel): the dynamic shared memory limit set so far
+  OccKey limit[kOccSlots];
+  int nlimit = 0;
+};
+OccCache &occ_cache() {
+  static OccCache c;
+  return c;
+}
+}  // namespace
+
+cudaError_t blocks_per_sm(const void *kern, int threads, int smem, int *blocks) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  OccCache &c = occ_cache();
+  std::lock_guard<std::mutex> lock(c.mu);
+  for (int i = 0; i < c.n; ++i)
+    if (c.key[i].dev == dev && c.key[i].kern == kern && c.key[i].threads == threads && c.key[i].smem == smem) {
+      *blocks = c.blocks[i];
+      return cudaSuccess;
+    }
+  // The limit only ever grows, so a size remembered earlier stays launchable.
+  int li = -1;
+  for (int i = 0; i < c.nlimit; ++i)
+    if (c.limit[i].dev == dev && c.limit[i].kern == kern) li = i;
+  if (li < 0 || c.limit[li].smem < smem) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
+    if (li < 0 && c.nlimit < kOccSlots) li = c.nlimit++;
+    if (li >= 0) c.limit[li] = OccKey{dev, kern, 0, smem};
+  }
+  int o = 0;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, threads, smem)) != cudaSuccess) return e;
+  if (c.n < kOccSlots) {
+    c.key[c.n] = OccKey{dev, kern, threads, smem};
+    c.blocks[c.n++] = o;
+  }
+  *blocks = o;
+  return cudaSuccess;
+}
+
 // [B*T, C] view of a [B, T, C] tensor, boxes of 32 columns x `rows` rows.
 bool encode_rows(CUtensorMap *m, const void *ptr, int dtype, int64_t rows, int64_t C,
                  int box_rows) {
+  const MapKey key{ptr, C, rows, 0, dtype, 2, box_rows};
+  if (map_lookup(key, m)) return true;
   auto enc = tensor_map_encoder();
   if (!enc || !ensure_context()) return false;
   const size_t es = dtype == 0 ? 4 : 2;
@@ -443,16 +547,21 @@ bool encode_rows(CUtensorMap *m, const void *ptr, int dtype, int64_t rows, int64
   cuuint64_t strides[1] = {(cuuint64_t)(C * es)};
   cuuint32_t box[2] = {32u, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
-  return enc(m, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-             const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (enc(m, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+          const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  map_insert(key, *m);
+  return true;
 }
 
 // [B, T, C] tensor as a 3-D map (C fastest), boxes of 32 channels x `box_t`
 // tokens x 1 batch row.  Loads past T or C read zeros and stores there are
 // clipped, so a box never reaches into the next batch row.
 bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T, int64_t C, int box_t) {
+  const MapKey key{ptr, C, T, B, dtype, 3, box_t};
+  if (map_lookup(key, m)) return true;
   auto enc = tensor_map_encoder();
   if (!enc || !ensure_context()) return false;
   const size_t es = dtype == 0 ? 4 : 2;
@@ -463,10 +572,13 @@ bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T
   // a box row is 32 channels (128 bytes fp32, 64 bytes bf16) of one token;
   // L2 fills are promoted to that size and no further, so the neighbouring
   // chain-tile's bytes are not fetched on this tile's behalf
-  return enc(m, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-             const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_NONE, dtype == 0 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_64B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (enc(m, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+          const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_NONE, dtype == 0 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_64B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  map_insert(key, *m);
+  return true;
 }
 
 // TMA needs 16-byte aligned rows and base addresses, and row indices < 2^31.
@@ -485,10 +597,8 @@ static cudaError_t launch_fwd_tma_t(const FwdArgs &a, int dtype, int num_sms, cu
     return cudaErrorInvalidValue;
   auto kern = fwd_tma_kernel<E, kTmaW, kTmaL, kTmaS>;
   const int threads = (kTmaW + 2) * 32;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::BYTES);
-  if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, Lay::BYTES);
+  cudaError_t e = blocks_per_sm((const void *)kern, threads, Lay::BYTES, &per_sm);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   const int64_t tiles = a.nchains * a.nchunks;

@@ -45,6 +45,13 @@ inline cudaError_t launch_kernel(void (*kern)(P...), dim3 grid, dim3 block, size
   return cudaLaunchKernelEx(&cfg, kern, static_cast<A &&>(args)...);
 }
 
+// Resident blocks per SM of `kern` launched with `threads` threads and `smem`
+// bytes of dynamic shared memory, on the current device.  The first query of
+// each (device, kernel, threads, smem) raises the kernel's dynamic shared
+// memory limit as far as needed and asks the occupancy calculator; the answer
+// is remembered, so later launches make no runtime call for it.
+cudaError_t blocks_per_sm(const void *kern, int threads, int smem, int *blocks);
+
 // ---------------------------------------------------------------- math ---
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -326,10 +326,9 @@ static cudaError_t launch_seg_t(const FwdArgs &f, int dtype, int num_sms, int ts
   int occ = 1 << 30;
   for (const void *kern : {(const void *)fwd_seg_kernel<E, S, RB, false, GATE>,
                            (const void *)fwd_seg_kernel<E, S, RB, true, GATE>}) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
     int o = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, kWarps * 32, smem)) != cudaSuccess) return e;
+    cudaError_t e = blocks_per_sm(kern, kWarps * 32, smem, &o);
+    if (e != cudaSuccess) return e;
     occ = std::min(occ, o);
   }
   if (occ < 1) return cudaErrorInvalidConfiguration;

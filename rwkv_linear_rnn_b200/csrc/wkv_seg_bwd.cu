@@ -571,10 +571,9 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
     int occ = 1 << 30;
     for (const void *kern : {(const void *)bwd_seg_kernel<E, S, RB, false, GATE, STATE>,
                              (const void *)bwd_seg_kernel<E, S, RB, true, GATE, STATE>}) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return e;
       int o = 0;
-      if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, kWarps * 32, smem)) != cudaSuccess) return e;
+      cudaError_t e = blocks_per_sm(kern, kWarps * 32, smem, &o);
+      if (e != cudaSuccess) return e;
       occ = std::min(occ, o);
     }
     mw = (int64_t)occ * num_sms * kWarps;

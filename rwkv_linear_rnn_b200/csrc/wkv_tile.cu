@@ -465,24 +465,6 @@ __global__ void __launch_bounds__(kTileFwdWarps * 32, 3) fwd_tile_kernel(const _
 }
 
 // ------------------------------------------------------------------ host ---
-// Per device: the dynamic shared memory attribute set once and the resident
-// blocks per SM, computed on the first launch of each kernel instantiation.
-struct LaunchCache {
-  std::atomic<int> blocks[kMaxDevices];
-};
-template <typename K>
-static int resident_blocks(LaunchCache &cache, K kern, int threads, int smem) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
-  int v = cache.blocks[dev].load(std::memory_order_acquire);
-  if (v > 0) return v;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -1;
-  int o = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, threads, smem) != cudaSuccess || o < 1) return -1;
-  cache.blocks[dev].store(o, std::memory_order_release);
-  return o;
-}
-
 template <typename E, int L, int RB, bool GATE>
 static cudaError_t launch_fwd_tile_t(const FwdArgs &f, float4 *rec, int dtype, int num_sms, cudaStream_t st) {
   CUtensorMap km, vm, rm, ym;
@@ -494,9 +476,10 @@ static cudaError_t launch_fwd_tile_t(const FwdArgs &f, float4 *rec, int dtype, i
   if (f.y && !encode_btc(&ym, f.y, dtype, f.B, f.T, f.C, L)) return cudaErrorInvalidValue;
   constexpr int NARR = GATE ? 3 : 2;
   constexpr int smem = TileLayout<E, L, NARR>::bytes(kTileFwdWarps);
-  static LaunchCache cache;
   auto kern = fwd_tile_kernel<E, L, RB, GATE>;
-  const int occ = resident_blocks(cache, kern, kTileFwdWarps * 32, smem);
+  int occ = 0;
+  cudaError_t e = blocks_per_sm((const void *)kern, kTileFwdWarps * 32, smem, &occ);
+  if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   TileFwdArgs a{};
   a.f = f;

@@ -476,10 +476,6 @@ __global__ void __launch_bounds__(NW * 32, NW == 4 ? 2 : 3) bwd_tile_kernel(cons
   finish_block(p.hdr, gridDim.x);
 }
 
-struct BwdLaunchCache {
-  std::atomic<int> blocks[kMaxDevices];
-};
-
 template <typename E, int L, int RB, int NW, bool STATE, bool GATE>
 static cudaError_t launch_bwd_tile_t(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *rec,
                                      float4 *chain_sum, int num_sms, cudaStream_t st) {
@@ -494,17 +490,10 @@ static cudaError_t launch_bwd_tile_t(const BwdArgs &p, int dtype, float *gw, flo
     return cudaErrorInvalidValue;
   constexpr int smem = TileBwdLayout<E, L, RB, GATE ? 4 : 3>::bytes(NW);
   auto kern = bwd_tile_kernel<E, L, RB, NW, STATE, GATE>;
-  static BwdLaunchCache cache;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  int occ = cache.blocks[dev].load(std::memory_order_acquire);
-  if (occ <= 0) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NW * 32, smem)) != cudaSuccess) return e;
-    if (occ < 1) return cudaErrorInvalidConfiguration;
-    cache.blocks[dev].store(occ, std::memory_order_release);
-  }
+  int occ = 0;
+  cudaError_t e = blocks_per_sm((const void *)kern, NW * 32, smem, &occ);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) return cudaErrorInvalidConfiguration;
   TileBwdArgs a{};
   a.p = p;
   a.gw = gw;

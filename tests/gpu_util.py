@@ -66,11 +66,3 @@ def inputs_to_device(inp):
         gy = dev(inp["gy"]) if "gy" in inp else None
     return w, u, k, v, gy
 
-
-def channel_subset(C, n, seed=0):
-    """A sorted random subset of channels, always including the first and last."""
-    rng = np.random.default_rng(seed)
-    if n >= C:
-        return np.arange(C)
-    idx = set(rng.choice(C, size=n - 2, replace=False).tolist()) | {0, C - 1}
-    return np.array(sorted(idx))

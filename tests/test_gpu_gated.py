@@ -252,20 +252,15 @@ def test_gated_rwkv169m_full():
     assert_grads5(got, ref, F32_GRAD_TOL)
 
 
-def test_gated_rwkv1b5_bf16_subset():
+def test_gated_rwkv1b5_bf16_full():
     inp = workloads.generate("rwkv1b5_bf16", gate=True)
     w, u, k, v, go = inputs_to_device(inp)
     r = dev_bf16_bits(inp["r_bits"])
     o, _, ck = W.forward_gated(w, u, k, v, r, want_ckpt=True)
     got = W.backward_gated(w, u, k, v, r, go, ckpt=ck)
-    rng = np.random.default_rng(5)
-    cs = np.array(sorted(set(rng.choice(inp["C"], 190, replace=False).tolist()) | {0, inp["C"] - 1}))
-    sub = lambda a: a[:, :, cs]
-    args = (inp["w"][cs], inp["u"][cs], sub(inp["k"]), sub(inp["v"]), sub(inp["r"]))
-    assert fwd_err(host(o[:, :, cs]), oracle.fwd_gated(*args)[0]) <= BF16_TOL
-    ref = oracle.bwd_gated(*args, sub(inp["gy"]))
-    got_s = (got[0][cs], got[1][cs], got[2][:, :, cs], got[3][:, :, cs], got[4][:, :, cs])
-    assert_grads5(got_s, ref, BF16_TOL)
+    args = (inp["w"], inp["u"], inp["k"], inp["v"], inp["r"])
+    assert fwd_err(host(o), oracle.fwd_gated(*args)[0]) <= BF16_TOL
+    assert_grads5(got, oracle.bwd_gated(*args, inp["gy"]), BF16_TOL)
 
 
 def test_calls_from_a_fresh_thread():
@@ -307,7 +302,7 @@ def test_gated_long_sequence_flag_join():
     """5000 tokens in one chain: more than 32 segments, so both segment
     kernels join through per-record flags instead of the grid barrier.
     (Warps holding several segments, with the gated backward's held
-    second-pass loads, run in test_gated_rwkv1b5_bf16_subset.)"""
+    second-pass loads, run in test_gated_rwkv1b5_bf16_full.)"""
     B, T, C = 1, 5000, 64
     w, u, k, v, r, g, _ = gated_case(B, T, C, seed=33)
     W_, U_, K_, V_, R_ = dev(w), dev(u), dev(k), dev(v), dev(r)

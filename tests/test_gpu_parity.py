@@ -2,9 +2,9 @@
 
 All calls go through the C ABI (the package's tensor helpers only marshal
 pointers).  Inputs are the seeded workloads of ``rwkv_linear_rnn_b200.workloads``
-at their full sizes (large ones compared on a channel subset: channels are
-independent chains, so the oracle runs the same chains on the CPU) plus
-small and ragged shapes that exercise tile edges.
+at their full sizes, every output element compared (the OpenMP oracle runs
+every chain of the largest workloads in seconds), plus small and ragged
+shapes that exercise tile edges.
 """
 import numpy as np
 import pytest
@@ -13,7 +13,7 @@ import torch
 import oracle
 import rwkv_linear_rnn_b200 as W
 from rwkv_linear_rnn_b200 import abi, workloads
-from gpu_util import (BF16_TOL, F32_FWD_TOL, F32_GRAD_TOL, channel_subset, dev, fwd_err, host,
+from gpu_util import (BF16_TOL, F32_FWD_TOL, F32_GRAD_TOL, dev, fwd_err, host,
                       inputs_to_device, rel_l2, state_err)
 
 pytestmark = pytest.mark.gpu
@@ -98,21 +98,18 @@ def test_forward_rwkv1b5_bf16():
     inp = workloads.generate("rwkv1b5_bf16", grad=False)
     w, u, k, v, _ = inputs_to_device(inp)
     y, s, _ = W.forward(w, u, k, v, want_state=True)
-    cs = channel_subset(inp["C"], 256, seed=2)
-    kk, vv = inp["k"][:, :, cs], inp["v"][:, :, cs]
-    y_ref, s_ref = oracle.fwd_recur(inp["w"][cs], inp["u"][cs], kk, vv)
-    assert fwd_err(host(y[:, :, cs]), y_ref) <= BF16_TOL
-    assert state_err(host(s[:, :, cs]), s_ref) <= F32_FWD_TOL * 10
+    y_ref, s_ref = oracle.fwd_recur(inp["w"], inp["u"], inp["k"], inp["v"])
+    assert fwd_err(host(y), y_ref) <= BF16_TOL
+    assert state_err(host(s), s_ref) <= F32_FWD_TOL * 10
 
 
 def test_forward_longctx():
     inp = workloads.generate("longctx", grad=False)
     w, u, k, v, _ = inputs_to_device(inp)
     y, s, _ = W.forward(w, u, k, v, want_state=True)
-    cs = channel_subset(inp["C"], 96, seed=3)
-    y_ref, s_ref = oracle.fwd_recur(inp["w"][cs], inp["u"][cs], inp["k"][:, :, cs], inp["v"][:, :, cs])
-    assert fwd_err(host(y[:, :, cs]), y_ref) <= F32_FWD_TOL
-    assert state_err(host(s[:, :, cs]), s_ref) <= F32_FWD_TOL
+    y_ref, s_ref = oracle.fwd_recur(inp["w"], inp["u"], inp["k"], inp["v"])
+    assert fwd_err(host(y), y_ref) <= F32_FWD_TOL
+    assert state_err(host(s), s_ref) <= F32_FWD_TOL
 
 
 def test_sequential_equals_chunked_longctx_slice():
@@ -183,17 +180,15 @@ def test_decode14b_prefill_and_32_steps():
     N, C = d["N"], d["C"]
     w, u = dev(d["w"]), dev(d["u"])
     _, s, _ = W.forward(w, u, dev(d["k"]), dev(d["v"]), want_state=True)
-    cs = channel_subset(C, 64, seed=4)
-    _, s_ref = oracle.fwd_recur(d["w"][cs], d["u"][cs], d["k"][:, :, cs], d["v"][:, :, cs])
-    assert state_err(host(s[:, :, cs]), s_ref) <= F32_FWD_TOL
+    _, s_ref = oracle.fwd_recur(d["w"], d["u"], d["k"], d["v"])
+    assert state_err(host(s), s_ref) <= F32_FWD_TOL
     worst = 0.0
     for i in range(d["k_steps"].shape[0]):
         y, s = W.step(w, u, dev(d["k_steps"][i]), dev(d["v_steps"][i]), s)
-        y_ref, s_ref = oracle.step(d["w"][cs], d["u"][cs], d["k_steps"][i][:, cs],
-                                   d["v_steps"][i][:, cs], s_ref)
-        worst = max(worst, fwd_err(host(y[:, cs]), y_ref))
+        y_ref, s_ref = oracle.step(d["w"], d["u"], d["k_steps"][i], d["v_steps"][i], s_ref)
+        worst = max(worst, fwd_err(host(y), y_ref))
     assert worst <= F32_FWD_TOL
-    assert state_err(host(s[:, :, cs]), s_ref) <= F32_FWD_TOL
+    assert state_err(host(s), s_ref) <= F32_FWD_TOL
 
 
 # --------------------------------------------------------------- backward ---
@@ -305,16 +300,20 @@ def test_backward_rwkv169m_full():
     assert_grads(got, ref, F32_GRAD_TOL)
 
 
-def test_backward_rwkv1b5_bf16_subset():
+def test_backward_rwkv1b5_bf16_full():
     inp = workloads.generate("rwkv1b5_bf16")
     w, u, k, v, gy = inputs_to_device(inp)
     _, _, ck = W.forward(w, u, k, v, want_ckpt=True)
     got = W.backward(w, u, k, v, gy, ckpt=ck)
-    cs = channel_subset(inp["C"], 192, seed=5)
-    sub = lambda a: a[:, :, cs]
-    ref = grads_ref(inp["w"][cs], inp["u"][cs], sub(inp["k"]), sub(inp["v"]), sub(inp["gy"]))
-    got_s = (got[0][cs], got[1][cs], got[2][:, :, cs], got[3][:, :, cs])
-    assert_grads(got_s, ref, BF16_TOL)
+    ref = grads_ref(inp["w"], inp["u"], inp["k"], inp["v"], inp["gy"])
+    assert_grads(got, ref, BF16_TOL)
+    # every channel of dL/dk and dL/dv, each on its own (a channel-wise fault
+    # would hide in the whole tensor's relative L2)
+    for name, a, b in (("gk", got[2], ref[2]), ("gv", got[3], ref[3])):
+        x = host(a)
+        num = np.sqrt(((x - b) ** 2).sum(axis=(0, 1)))
+        den = np.sqrt((b ** 2).sum(axis=(0, 1)))
+        assert np.max(num / den) <= BF16_TOL, (name, int(np.argmax(num / den)))
 
 
 def test_backward_deterministic():
@@ -480,3 +479,34 @@ def test_tile_unit_boundaries(T, dtype):
     assert state_err(host(s), s_ref) <= F32_FWD_TOL * (10 if dtype == "bf16" else 1)
     got = W.backward(W_, U_, K_, V_, G_, ckpt=ck, kernel=W.WKV_KERNEL_TILE)
     assert_grads(got, grads_ref(w, u, k, v, g), BF16_TOL if dtype == "bf16" else F32_GRAD_TOL)
+
+
+@pytest.mark.parametrize("kernel", ["segment", "tile"])
+def test_cached_tensor_maps_follow_shape_changes(kernel):
+    """The library remembers encoded tensor maps by (address, shape, dtype,
+    box).  One pair of buffers viewed as several shapes in turn (same base
+    address, different extents), then the first shape again: every call
+    matches the oracle, and the repeated shape gives the same bits as its
+    first call."""
+    kern = KERNELS[kernel]
+    C = 64
+    cap = 3 * 400 * C
+    kbuf = torch.empty(cap, device="cuda")
+    vbuf = torch.empty(cap, device="cuda")
+    gbuf = torch.empty(cap, device="cuda")
+    seen = {}
+    for call, (B, T) in enumerate([(3, 400), (2, 150), (1, 400), (3, 97), (3, 400)]):
+        w, u, k, v, g, _ = small_case(B, T, C, seed=200 + B * T)
+        n = B * T * C
+        K_, V_, G_ = (buf[:n].view(B, T, C) for buf in (kbuf, vbuf, gbuf))
+        K_.copy_(dev(k)), V_.copy_(dev(v)), G_.copy_(dev(g))
+        W_, U_ = dev(w), dev(u)
+        y, _, ck = W.forward(W_, U_, K_, V_, want_ckpt=True, kernel=kern)
+        gw, gu, gk, gv = W.backward(W_, U_, K_, V_, G_, ckpt=ck, kernel=BWD_KERNELS[kernel])
+        assert fwd_err(host(y), oracle.fwd_recur(w, u, k, v)[0]) <= F32_FWD_TOL, call
+        assert_grads((gw, gu, gk, gv), grads_ref(w, u, k, v, g), F32_GRAD_TOL)
+        out = (y.clone(), gw.clone(), gu.clone(), gk.clone(), gv.clone())
+        if (B, T) in seen:
+            for a, b in zip(seen[(B, T)], out):
+                assert torch.equal(a, b), call
+        seen[(B, T)] = out
