@@ -1,6 +1,8 @@
 """libwkv: the RWKV-4 WKV time-mixing operator on NVIDIA B200 (sm_100a).
 
-Thin Python binding over the C ABI in ``include/wkv.h``.  The functions in
+Thin Python binding over the C ABI in ``include/wkv.h`` and
+``include/linattn.h`` (causal linear attention: ``linattn_forward``,
+``linattn_backward``).  The functions in
 ``abi`` carry the C names and take raw device pointers (ints) -- argument
 marshalling only.  The tensor helpers below (``forward``, ``backward``,
 ``step``, ``WKV``, ``backward_state``, ``token_shift`` and the gated ``forward_gated``, ``backward_gated``,
@@ -27,7 +29,8 @@ __all__ = [
     "WKV_KERNEL_SEGMENT", "WKV_KERNEL_CLUSTER", "WKV_KERNEL_TILE", "WKV_STATIC_SCRATCH_BYTES", "Workspace", "forward", "backward", "backward_state", "step", "token_shift",
     "token_shift_backward", "TokenShift",
     "forward_gated", "backward_gated", "WKV", "wkv", "WKVState", "wkv_state", "GatedWKV", "gated_wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror", "wkv_version",
-    "library_path",
+    "library_path", "LINATTN_OP_FORWARD", "LINATTN_OP_BACKWARD", "linattn_workspace_size",
+    "linattn_forward", "linattn_backward",
 ]
 
 
@@ -112,8 +115,10 @@ class Workspace:
         self.buf = None
 
     def get(self, op, B, T, C, dtype):
+        return self.get_bytes(wkv_workspace_size(op, B, T, C, dtype))
+
+    def get_bytes(self, need):
         torch = _torch()
-        need = wkv_workspace_size(op, B, T, C, dtype)
         if need == 0:
             return None, 0
         if self.buf is None or self.buf.numel() < need:
@@ -214,6 +219,63 @@ def backward_state(w, u, k, v, grad_y, state_in=None, ckpt=None, *, state_out=No
                                         _ptr(gv), _ptr(gs), _ptr(buf), nbytes, _stream(stream),
                                         opts))
     return gw, gu, gk, gv, gs
+
+
+# ------------------------------------------------ causal linear attention ---
+
+LINATTN_OP_FORWARD, LINATTN_OP_BACKWARD = 0, 1
+
+
+def linattn_workspace_size(op, BH, N, D, M):
+    return _abi().linattn_workspace_size(op, BH, N, D, M)
+
+
+def _check_linattn(q, k, v, *more):
+    torch = _torch()
+    _check_cuda(q, k, v, *more)
+    for t in (q, k, v) + tuple(x for x in more if x is not None):
+        if t.dtype != torch.bfloat16 or t.dim() != 3:
+            raise ValueError("linear attention takes bfloat16 [BH, N, D] tensors")
+    BH, N, D = q.shape
+    if k.shape != q.shape or v.shape[:2] != (BH, N):
+        raise ValueError("q, k must be [BH, N, D] and v [BH, N, M]")
+    return BH, N, D, v.shape[2]
+
+
+def linattn_forward(q, k, v, *, want_state=False, out=None, workspace=None, stream=None):
+    """Causal linear attention (elu + 1 feature map) for q, k [BH, N, D] and
+    v [BH, N, M], bfloat16 (include/linattn.h).  Returns (out [BH, N, M],
+    state or None) with state = (S [BH, D, M], Z [BH, D]) float32 after the
+    last position."""
+    torch = _torch()
+    BH, N, D, M = _check_linattn(q, k, v, out)
+    if out is None:
+        out = torch.empty((BH, N, M), dtype=torch.bfloat16, device=q.device)
+    st = torch.empty(BH * (D * M + D), dtype=torch.float32, device=q.device) if want_state else None
+    ws = _ws_for(q.device, workspace)
+    buf, nbytes = ws.get_bytes(linattn_workspace_size(LINATTN_OP_FORWARD, BH, N, D, M))
+    abi = _abi()
+    abi.check(abi.linattn_forward(BH, N, D, M, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(st),
+                                  _ptr(buf), nbytes, _stream(stream)))
+    if st is not None:
+        st = (st[:BH * D * M].view(BH, D, M), st[BH * D * M:].view(BH, D))
+    return out, st
+
+
+def linattn_backward(q, k, v, grad_out, *, grad_q=None, grad_k=None, grad_v=None, workspace=None,
+                     stream=None):
+    """Gradients (grad_q, grad_k, grad_v) of L given grad_out = dL/dV'."""
+    torch = _torch()
+    BH, N, D, M = _check_linattn(q, k, v, grad_out, grad_q, grad_k, grad_v)
+    grad_q = torch.empty_like(q) if grad_q is None else grad_q
+    grad_k = torch.empty_like(k) if grad_k is None else grad_k
+    grad_v = torch.empty_like(v) if grad_v is None else grad_v
+    ws = _ws_for(q.device, workspace)
+    buf, nbytes = ws.get_bytes(linattn_workspace_size(LINATTN_OP_BACKWARD, BH, N, D, M))
+    abi = _abi()
+    abi.check(abi.linattn_backward(BH, N, D, M, _ptr(q), _ptr(k), _ptr(v), _ptr(grad_out), _ptr(grad_q),
+                                   _ptr(grad_k), _ptr(grad_v), _ptr(buf), nbytes, _stream(stream)))
+    return grad_q, grad_k, grad_v
 
 
 def token_shift(x, mu, x_prev=None, *, out=None, stream=None):

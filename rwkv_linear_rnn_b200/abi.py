@@ -1,4 +1,4 @@
-"""ctypes declarations of the libwkv C ABI (``include/wkv.h``).
+"""ctypes declarations of the libwkv C ABI (``include/wkv.h``, ``include/linattn.h``).
 
 Each function keeps its C name and signature; pointers are passed as Python
 ints (device addresses), streams as ``cudaStream_t`` ints.  Loading fails
@@ -25,6 +25,8 @@ EXPORTS = (
     "wkv_token_shift", "wkv_token_shift_workspace_size", "wkv_token_shift_backward",
     "wkv_step", "wkv_backward_static", "wkv_backward_static_status", "wkv_get_status",
     "wkv_strerror", "wkv_last_cuda_error", "wkv_cuda_error_name", "wkv_version",
+    # include/linattn.h
+    "linattn_workspace_size", "linattn_forward", "linattn_backward",
 )
 
 
@@ -72,6 +74,9 @@ _SIGS = {
     "wkv_last_cuda_error": (_int, []),
     "wkv_cuda_error_name": (ctypes.c_char_p, [_int]),
     "wkv_version": (_int, []),
+    "linattn_workspace_size": (_sz, [_int, _i64, _i64, _int, _int]),
+    "linattn_forward": (_int, [_i64, _i64, _int, _int, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "linattn_backward": (_int, [_i64, _i64, _int, _int] + [_p] * 7 + [_p, _sz, _p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -215,6 +220,19 @@ def wkv_cuda_error_name(err):
 
 def wkv_version():
     return lib.wkv_version()
+
+
+def linattn_workspace_size(op, BH, N, D, M):
+    return lib.linattn_workspace_size(op, BH, N, D, M)
+
+
+def linattn_forward(BH, N, D, M, q, k, v, out, state_out, ws, ws_bytes, stream):
+    return lib.linattn_forward(BH, N, D, M, q, k, v, out, state_out, ws, ws_bytes, stream)
+
+
+def linattn_backward(BH, N, D, M, q, k, v, grad_out, grad_q, grad_k, grad_v, ws, ws_bytes, stream):
+    return lib.linattn_backward(BH, N, D, M, q, k, v, grad_out, grad_q, grad_k, grad_v, ws, ws_bytes,
+                                stream)
 
 
 def check(rc: int) -> None:

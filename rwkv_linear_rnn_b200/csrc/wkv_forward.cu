@@ -581,6 +581,27 @@ bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T
   return true;
 }
 
+// [BH, N, width] bfloat16 tensor as a 3-D map (width fastest), boxes of
+// width x 128 rows x 1 head in the 64-byte swizzle, which is the layout the
+// tensor cores read their operands in (width * 2 must be 64 bytes).  Rows
+// past N read zeros and stores there are clipped.
+bool encode_heads_sw64(CUtensorMap *m, const void *ptr, int64_t BH, int64_t N, int width) {
+  const MapKey key{ptr, width, N, BH, 1, 103, 128};
+  if (map_lookup(key, m)) return true;
+  auto enc = tensor_map_encoder();
+  if (!enc || !ensure_context() || width * 2 != 64) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)(width * 2), (cuuint64_t)(N * width * 2)};
+  cuuint32_t box[3] = {(cuuint32_t)width, 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  if (enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  map_insert(key, *m);
+  return true;
+}
+
 // TMA needs 16-byte aligned rows and base addresses, and row indices < 2^31.
 bool fwd_tma_eligible(const FwdArgs &a, int dtype) {
   const int64_t es = dtype == 0 ? 4 : 2;

@@ -179,3 +179,52 @@ def generate_decode_steps(wl: Workload | str = "decode14b", N: int | None = None
         vs[s] = _normal(rng, (N, C), 1.0)
     return {"w": w, "u": u, "time_decay": td, "k": k, "v": v,
             "k_steps": ks, "v_steps": vs, "N": N, "T": wl.T, "C": C}
+
+
+# ----------------------------------------------- causal linear attention ---
+# Shapes of the linear attention post's experiments (section "실험 설정"):
+# heads of 32 dimensions (8 heads over a 256-wide embedding); MNIST image
+# generation runs 784-position sequences at batch 10, CIFAR-10 3072-position
+# sequences at batch 4 for the linear model.  The post states no value
+# distributions; q, k, v and the output gradient are drawn N(0, 1) (unit-
+# variance projections) and rounded to bfloat16, the operator's storage type.
+# ``la_cifar_b32`` is the CIFAR-10 head shape at batch 32, a throughput case
+# larger than L2.
+
+@dataclass(frozen=True)
+class LinAttnWorkload:
+    name: str
+    BH: int  # batch x heads
+    N: int
+    D: int   # = M
+    seed: int
+    note: str = ""
+
+
+LINATTN_WORKLOADS = {
+    "la_mnist": LinAttnWorkload("la_mnist", 10 * 8, 784, 32, 10, "MNIST: batch 10, 8 heads, N784, D=M=32"),
+    "la_cifar": LinAttnWorkload("la_cifar", 4 * 8, 3072, 32, 11, "CIFAR-10: batch 4, 8 heads, N3072, D=M=32"),
+    "la_cifar_b32": LinAttnWorkload("la_cifar_b32", 32 * 8, 3072, 32, 12,
+                                    "CIFAR-10 head shape at batch 32: 256 heads, N3072, D=M=32"),
+}
+
+
+def generate_linattn(wl: LinAttnWorkload | str, BH: int | None = None, N: int | None = None,
+                     grad: bool = True, seed: int | None = None):
+    """Draw q, k [BH, N, D], v [BH, N, M] and (if ``grad``) g = dL/dV'.
+
+    Draw order: q, k, v, g, each N(0, 1) float32 rounded to bfloat16.
+    Returns a dict with the bf16 bit patterns (``q_bits`` ...) and the same
+    values widened to float32 (``q`` ...), plus BH, N, D, M.
+    """
+    if isinstance(wl, str):
+        wl = LINATTN_WORKLOADS[wl]
+    BH = wl.BH if BH is None else BH
+    N = wl.N if N is None else N
+    rng = np.random.Generator(np.random.PCG64(wl.seed if seed is None else seed))
+    out = {"BH": BH, "N": N, "D": wl.D, "M": wl.D}
+    for name in ("q", "k", "v", "g") if grad else ("q", "k", "v"):
+        bits = bf16_round(_normal(rng, (BH, N, wl.D), 1.0))
+        out[name + "_bits"] = bits
+        out[name] = bf16_to_f32(bits)
+    return out

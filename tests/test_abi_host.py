@@ -1,6 +1,6 @@
 """Host-side checks of the C ABI (no GPU needed).
 
-* the library loads and exports every function ``include/wkv.h`` declares;
+* the library loads and exports every function ``include/*.h`` declares;
 * argument validation rejects bad calls with the documented code before any
   CUDA work (these calls never reach a kernel launch);
 * workspace and checkpoint sizes follow the documented layout.
@@ -23,9 +23,14 @@ def W():
 
 
 def header_functions():
-    src = open(os.path.join(ROOT, "include", "wkv.h"), encoding="utf-8").read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(wkv_[a-z_]+)\s*\(", src, flags=re.M)
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", h), encoding="utf-8").read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*((?:wkv|linattn)_[a-z_]+)\s*\(", src,
+                            flags=re.M)
     return names
 
 
@@ -211,3 +216,40 @@ def test_token_shift_validation(W):
     assert a.wkv_token_shift_backward(*bad) == -3            # no workspace
     bad = list(okb); bad[13] = 64
     assert a.wkv_token_shift_backward(*bad) == -3            # workspace too small
+
+
+def test_linattn_sizes_and_argument_checks(W):
+    """Linear attention: workspace sizes, and calls rejected before any
+    launch (unsupported head size, null or misaligned pointers, a small
+    workspace, bad sizes)."""
+    abi = W.abi
+    f = W.linattn_workspace_size(0, 32, 3072, 32, 32)
+    b = W.linattn_workspace_size(1, 32, 3072, 32, 32)
+    nch = 3072 // 128
+    assert f >= 256 + 32 * nch * (32 * 32 + 32) * 4
+    assert b >= f + 32 * nch * (32 * 32 + 32) * 4 + 32 * 3072 * (32 * 2 + 4)
+    assert W.linattn_workspace_size(0, 32, 3072, 64, 64) == 0   # head size not supported
+    assert W.linattn_workspace_size(0, 0, 3072, 32, 32) == 0    # BH < 1
+    assert W.linattn_workspace_size(0, 1, -1, 32, 32) == 0      # N < 0
+    assert W.linattn_workspace_size(2, 1, 8, 32, 32) == 0       # bad op
+    F = FAKE
+    ws = 1 << 24
+    big = 1 << 30
+    # (BH, N, D, M, q, k, v, out, state_out, ws, ws_bytes) -> code
+    cases = [
+        ((1, 8, 64, 64, F, F * 2, F * 3, F * 4, 0, ws, big), -2),   # D = 64
+        ((1, 8, 32, 32, 0, F * 2, F * 3, F * 4, 0, ws, big), -1),   # q NULL
+        ((1, 8, 32, 32, F, F * 2, F * 3, F, 0, ws, big), -1),       # out is q
+        ((0, 8, 32, 32, F, F * 2, F * 3, F * 4, 0, ws, big), -1),   # BH = 0
+        ((1, 8, 32, 32, F + 2, F * 2, F * 3, F * 4, 0, ws, big), -2),  # q misaligned
+        ((1, 8, 32, 32, F, F * 2, F * 3, F * 4, 0, ws, 16), -3),    # workspace too small
+        ((1, 8, 32, 32, F, F * 2, F * 3, F * 4, 0, ws + 16, big), -2),  # workspace misaligned
+        ((1, 8, 32, 32, F, F * 2, F * 3, F * 4, 0, 0, big), -1),    # no workspace
+    ]
+    for args, code in cases:
+        assert abi.linattn_forward(*args, 0) == code, args
+    bargs = (1, 8, 32, 32, F, F * 2, F * 3, F * 4, F * 5, F * 6, F * 7, ws, big, 0)
+    assert abi.linattn_backward(*bargs[:4], 0, *bargs[5:]) == -1           # q NULL
+    assert abi.linattn_backward(1, 8, 32, 32, F, F * 2, F * 3, F * 4, F, F * 6, F * 7, ws, big, 0) == -1  # grad_q is q
+    assert abi.linattn_backward(1, 8, 16, 16, *bargs[4:]) == -2            # head size
+    assert abi.linattn_backward(*bargs[:11], ws, 16, 0) == -3              # workspace too small
