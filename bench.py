@@ -348,6 +348,22 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_linattn_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    wl = workloads.LINATTN_WORKLOADS[args.workload]
+    cb = linattn_cpu_baseline(args.workload, max(1.0, 2.0 * args.steps))
+    line = {"metric": "causal linear attention fwd+bwd head-positions/s (HBM GB/s and % of roofline alongside)",
+            "value": cb["value"], "unit": cb["unit"], "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": wl.BH * wl.N / cb["value"] * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "impl": "reference", "config": linattn_config(wl, 1),
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": cb["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------- GPU arm ---
 
 def setup_device():
@@ -844,13 +860,158 @@ def run_token_shift(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------- causal linear attention ---
+
+LA_FWD_BYTES = 4 * 32 * 2   # q, k, v read, out written (bf16, D = M = 32), per head-position
+LA_BWD_BYTES = 7 * 32 * 2   # q, k, v, grad_out read, grad_q, grad_k, grad_v written
+
+
+def linattn_config(wl, ws_n):
+    return {"workload": wl.name, "op": "causal linear attention (elu+1)", "BH": wl.BH, "N": wl.N,
+            "D": wl.D, "M": wl.D, "io_dtype": "bf16", "note": wl.note,
+            "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
+            "l2": "flushed before every timed step (2x L2 write + 2x L2 read, outside events)"}
+
+
+def linattn_cpu_baseline(wl_name: str, min_seconds: float):
+    """The linear-attention oracle (float64 numpy, forward then backward) on a
+    few heads of the workload, full length."""
+    from oracle import linattn as la
+    wl = workloads.LINATTN_WORKLOADS[wl_name]
+    heads = 4
+    inp = workloads.generate_linattn(wl, BH=heads)
+    med, reps = _time_loop(lambda: la.bwd_recur(inp["q"], inp["k"], inp["v"], inp["g"]), min_seconds)
+    # bwd_recur runs the forward recurrence inside it, so one call is fwd + bwd
+    return {"value": heads * wl.N / med, "unit": "head-positions/s", "cores": 1, "kind": "oracle",
+            "sample": f"{wl_name}: {heads} heads x N{wl.N} fwd+bwd (numpy, one thread) x{reps}, median"}
+
+
+def run_linattn(args):
+    """Causal linear attention forward then backward through the C ABI
+    (include/linattn.h), one call each per step."""
+    import torch
+    import rwkv_linear_rnn_b200 as W
+    from rwkv_linear_rnn_b200 import abi
+
+    ws_n, rank, dist, dev = setup_device()
+    wl = workloads.LINATTN_WORKLOADS[args.workload]
+    inp = workloads.generate_linattn(wl, seed=wl.seed + 1000 * rank)
+    BH, N, D = inp["BH"], inp["N"], inp["D"]
+    t = {n: torch.from_numpy(inp[n + "_bits"].view(np.int16)).to(dev).view(torch.bfloat16)
+         for n in ("q", "k", "v", "g")}
+    out = torch.empty_like(t["v"])
+    dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
+    nf = abi.linattn_workspace_size(0, BH, N, D, D)
+    nb = abi.linattn_workspace_size(1, BH, N, D, D)
+    wsb = torch.zeros(max(nf, nb), dtype=torch.uint8, device=dev)
+    flush_l2 = make_flush(dev)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    P = lambda x: x.data_ptr()
+
+    def fwd():
+        abi.check(abi.linattn_forward(BH, N, D, D, P(t["q"]), P(t["k"]), P(t["v"]), P(out), None, P(wsb),
+                                      wsb.numel(), sp))
+
+    def bwd():
+        abi.check(abi.linattn_backward(BH, N, D, D, P(t["q"]), P(t["k"]), P(t["v"]), P(t["g"]), P(dq), P(dk),
+                                       P(dv), P(wsb), wsb.numel(), sp))
+
+    for _ in range(args.warmup):
+        flush_l2(); fwd(); bwd()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t_begin = time.monotonic()
+    for i in range(K):
+        flush_l2()
+        ev[i][0].record(stream); fwd(); ev[i][1].record(stream); bwd(); ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop(window=(t_begin, time.monotonic()))
+    if dist:
+        dist.barrier()
+    t_fwd = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    t_bwd = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    total_ms = max_over_ranks(sum(t_fwd) + sum(t_bwd), dist, dev)
+    status = abi.wkv_get_status(P(wsb), sp)
+
+    units = BH * N
+    e2e = None
+    if not args.no_e2e:
+        hin = {n: t[n].cpu().pin_memory() for n in t}
+        hout = [torch.empty_like(x, device="cpu").pin_memory() for x in (out, dq, dk, dv)]
+        h2d = sum(x.numel() * x.element_size() for x in hin.values())
+        d2h = sum(x.numel() * x.element_size() for x in hout)
+        ee = []
+        for i in range(max(3, min(K, 10)) + 1):
+            e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for n in t:
+                t[n].copy_(hin[n], non_blocking=True)
+            fwd(); bwd()
+            for h, d in zip(hout, (out, dq, dk, dv)):
+                h.copy_(d, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i > 0:
+                ee.append(e0.elapsed_time(e1))
+        e2e_ms = max_over_ranks(statistics.median(ee), dist, dev)
+        e2e = {"value": aggregate_rate(units, ws_n, e2e_ms), "unit": "head-positions/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if rank == 0:
+        hbm, peak_kind = peaks()
+        fwd_ms, bwd_ms = statistics.mean(t_fwd), statistics.mean(t_bwd)
+        fb, bb = LA_FWD_BYTES * units, LA_BWD_BYTES * units
+        fwd_gbs = fb / (fwd_ms * 1e-3) / 1e9
+        bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9
+        nch = -(-N // 128)
+        # tensor-core work issued per 128-position chunk (M = 128 tiles, padding included)
+        mf = lambda m, n, k: 2.0 * m * n * k
+        f_chunk = mf(128, 128, 32) + mf(128, 32, 128) + mf(128, 32, 32) + mf(128, 48, 128)
+        b_chunk = (mf(128, 48, 128) + mf(128, 128, 32) + mf(128, 32, 128) + mf(128, 32, 32) + mf(128, 48, 128)
+                   + 2 * mf(128, 128, 32) + 3 * (mf(128, 32, 128) + mf(128, 32, 32)))
+        step_ms = total_ms / K
+        line = {
+            "metric": "causal linear attention fwd+bwd head-positions/s (HBM GB/s and % of roofline alongside)",
+            "value": aggregate_rate(units, ws_n, step_ms), "unit": "head-positions/s",
+            "n_gpus": ws_n, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) q, k, v, grad_out rounded to bf16)",
+            "config": linattn_config(wl, ws_n),
+            "roofline": {"bound": "hbm", "kernel": "linattn_backward call (5 launches), timed as one call",
+                         "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s", "frac": bwd_gbs / hbm,
+                         "traffic": None, "algorithmic_bytes": bb, "peak_kind": peak_kind},
+            "fwd": {"ms": fwd_ms, "gbs": fwd_gbs, "frac": fwd_gbs / hbm, "launches": 3,
+                    "tensor_tflops_issued": f_chunk * BH * nch / (fwd_ms * 1e-3) / 1e12},
+            "bwd": {"ms": bwd_ms, "gbs": bwd_gbs, "frac": bwd_gbs / hbm, "launches": 5,
+                    "tensor_tflops_issued": b_chunk * BH * nch / (bwd_ms * 1e-3) / 1e12},
+            "clocks": clocks, "device_status": status, "gpu_launches": 8 * K,
+        }
+        if e2e:
+            line["e2e"] = e2e
+        if not args.no_cpu_baseline and ws_n == 1:
+            line["cpu_baseline"] = linattn_cpu_baseline(args.workload, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="libwkv", choices=["libwkv", "reference"])
-    ap.add_argument("--workload", default="rwkv1b5_bf16", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="rwkv1b5_bf16",
+                    choices=sorted(workloads.WORKLOADS) + sorted(workloads.LINATTN_WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -862,6 +1023,14 @@ def main():
                     help="time the token shift (3 interpolations) on the workload's layer shape")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    if args.workload in workloads.LINATTN_WORKLOADS:
+        if args.gate or args.token_shift:
+            raise SystemExit("--gate / --token-shift apply to the WKV workloads")
+        if args.impl == "reference":
+            run_linattn_reference(args)
+        else:
+            run_linattn(args)
+        return
     if args.gate and workload_mode(args.workload) == "step":
         raise SystemExit("--gate applies to the forward/backward workloads")
     if args.impl == "reference":

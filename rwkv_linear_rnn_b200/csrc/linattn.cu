@@ -326,11 +326,24 @@ __global__ void la_scan_kernel(float *rec, int64_t BH, int nch, int reverse, flo
   const int f = (int)(e % kRec);
   float *base = rec + h * nch * kRec + f;
   float run = 0.f;
-  for (int s = 0; s < nch; ++s) {
-    const int c = reverse ? nch - 1 - s : s;
-    const float x = base[(int64_t)c * kRec];
-    base[(int64_t)c * kRec] = run;
-    run += x;
+  // 16 chunks at a time: their loads are independent, so they are all in
+  // flight together; the running sum then goes through them in order
+  constexpr int kBatch = 16;
+  for (int s0 = 0; s0 < nch; s0 += kBatch) {
+    float x[kBatch];
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      const int s = s0 + t;
+      x[t] = s < nch ? base[(int64_t)(reverse ? nch - 1 - s : s) * kRec] : 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      const int s = s0 + t;
+      if (s < nch) {
+        base[(int64_t)(reverse ? nch - 1 - s : s) * kRec] = run;
+        run += x[t];
+      }
+    }
   }
   if (total) {
     if (f < kDM)

@@ -42,6 +42,15 @@
 #include "wkv_math.cuh"
 #include "wkv_tile.cuh"
 
+// Build-time knobs of the ungated kernels: the blocks per SM their
+// registers are sized for, and the tokens per unit for bf16 tensors.
+#ifndef WKV_TILEB_MINB
+#define WKV_TILEB_MINB 2
+#endif
+#ifndef WKV_TILEB_LBF16
+#define WKV_TILEB_LBF16 kTileLBF16
+#endif
+
 namespace wkv {
 
 bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T, int64_t C, int box_t);
@@ -151,7 +160,7 @@ struct TileBwdLayout {
 // tile, which leaves by TMA with dL/dk and dL/dv.  Nothing but the
 // algorithmic bytes crosses HBM.
 template <typename E, int L, int RB, int NW, bool STATE, bool GATE>
-__global__ void __launch_bounds__(NW * 32, NW == 4 ? 2 : 3) bwd_tile_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(NW * 32, NW == 4 ? WKV_TILEB_MINB : 3) bwd_tile_kernel(const __grid_constant__ CUtensorMap kmap,
                                                            const __grid_constant__ CUtensorMap vmap,
                                                            const __grid_constant__ CUtensorMap gmap,
                                                            const __grid_constant__ CUtensorMap rmap,
@@ -524,11 +533,11 @@ cudaError_t launch_backward_tile(const BwdArgs &p, int dtype, float *gw, float *
   if (p.gs_out || p.gs_in)
     return dtype == 0 ? launch_bwd_tile_t<float, kTileLF32, 8, kTileWarps, true, false>(
                             p, dtype, gw, gu, rec, chain_sum, num_sms, st)
-                      : launch_bwd_tile_t<uint16_t, kTileLBF16, 8, kTileWarps, true, false>(
+                      : launch_bwd_tile_t<uint16_t, WKV_TILEB_LBF16, 8, kTileWarps, true, false>(
                             p, dtype, gw, gu, rec, chain_sum, num_sms, st);
   return dtype == 0 ? launch_bwd_tile_t<float, kTileLF32, 8, kTileWarps, false, false>(
                           p, dtype, gw, gu, rec, chain_sum, num_sms, st)
-                    : launch_bwd_tile_t<uint16_t, kTileLBF16, 8, kTileWarps, false, false>(
+                    : launch_bwd_tile_t<uint16_t, WKV_TILEB_LBF16, 8, kTileWarps, false, false>(
                           p, dtype, gw, gu, rec, chain_sum, num_sms, st);
 }
 
