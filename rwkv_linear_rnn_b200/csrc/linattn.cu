@@ -38,6 +38,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "../../include/linattn.h"
 #include "../../include/wkv.h"
 #include "wkv_internal.cuh"
@@ -263,57 +265,119 @@ __device__ __forceinline__ uint8_t *align1k(uint8_t *p) {
 }
 
 // ------------------------------------------------------------- kernels ---
-// Chunk state: phi(K)^T V (32 x 32) and phi(K)^T 1 (32) of one chunk, as
-// one MMA with M = 128 (rows 32..127 of its A operand are other tiles' bytes
-// and their results are not read) and N = 48 (B = [V | ones]).
-// Shared memory: phi(K) at 0, V at 8K, ones at 16K, spare at 24K.
+// Chunk states: phi(K)^T V (32 x 32) and phi(K)^T 1 (32) of every chunk,
+// each as one MMA chain with M = 128 (rows 32..127 of its A operand are
+// other tiles' bytes and their results are not read) and N = 48
+// (B = [V | ones]).  Persistent: CTA g takes chunks g, g + G, ... and keeps
+// two chunks' loads in flight (a stage is refilled as soon as its MMAs are
+// complete).  Shared memory: stages (phi(K), V) at 0 and 16K, the ones tile
+// at 32K; the spare rows of stage 1's A operand reach to 48K.
+constexpr uint32_t kSStage = 2 * kTile, kSOnes = 2 * kSStage;
 __global__ void __launch_bounds__(kThreads) la_state_kernel(const __grid_constant__ CUtensorMap kmap,
                                                             const __grid_constant__ CUtensorMap vmap, LaArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ Ctl ctl;
+  __shared__ uint64_t bar_ld[2], bar_mma;
+  __shared__ uint32_t tmem_s;
   uint8_t *sm = align1k(smem_raw);
   const uint32_t s0 = smem_addr(sm);
-  const int h = (int)(blockIdx.x / a.nch), c = (int)(blockIdx.x % a.nch);
-  const int64_t rem = a.N - (int64_t)c * kL;
-  const int valid = rem < kL ? (int)rem : kL;
-  ctl_setup(&ctl, 64);
-  const uint32_t bl = smem_addr(&ctl.bar[0]), bm = smem_addr(&ctl.bar[1]);
+  const int64_t total = a.BH * a.nch;
+  const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    const uint64_t pol = l2_policy_evict_last();  // read again by the output kernel
-    mbar_expect_tx(bl, 2 * kTile);
-    tma_load_3d(s0, &kmap, 0, c * kL, h, bl, pol);
-    tma_load_3d(s0 + kTile, &vmap, 0, c * kL, h, bl, pol);
+    mbar_init(smem_addr(&bar_ld[0]), 1);
+    mbar_init(smem_addr(&bar_ld[1]), 1);
+    mbar_init(smem_addr(&bar_mma), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  {  // ones (bf16 1.0 = 0x3F80)
-    uint4 *o = reinterpret_cast<uint4 *>(sm + 2 * kTile);
-    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kThreads) o[g] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  if (warp == 0) {
+    tmem_alloc(smem_addr(&tmem_s), 64);
+    tmem_relinquish();
   }
-  if (ctl_wait(&ctl, 0, 0, a)) {
-    phi_tile(sm, valid, true);
+  {
+    uint4 *o = reinterpret_cast<uint4 *>(sm + kSOnes);
+    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kThreads)
+      o[g] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // bf16 1.0
+  }
+  tc_before_sync();
+  __syncthreads();
+  tc_after_sync();
+  const uint32_t tm = tmem_s;
+  const uint64_t pol = l2_policy_evict_last();  // read again by the output kernel
+  auto issue = [&](int64_t idx, int st) {
+    const int h = (int)(idx / a.nch), c = (int)(idx % a.nch);
+    const uint32_t dst = s0 + st * kSStage, bar = smem_addr(&bar_ld[st]);
+    mbar_expect_tx(bar, 2 * kTile);
+    tma_load_3d(dst, &kmap, 0, c * kL, h, bar, pol);
+    tma_load_3d(dst + kTile, &vmap, 0, c * kL, h, bar, pol);
+  };
+  int64_t issued = 0;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < 2; ++st)
+      if ((int64_t)blockIdx.x + (int64_t)st * gridDim.x < total) {
+        issue((int64_t)blockIdx.x + (int64_t)st * gridDim.x, st);
+        ++issued;
+      }
+  }
+  uint32_t mma_phase = 0;
+  int it = 0;
+  bool failed = false, mma_pending = false;  // uniform over the CTA
+  for (int64_t idx = blockIdx.x; idx < total; idx += gridDim.x, ++it) {
+    const int st = it & 1;
+    const int h = (int)(idx / a.nch), c = (int)(idx % a.nch);
+    const int64_t rem = a.N - (int64_t)c * kL;
+    const int valid = rem < kL ? (int)rem : kL;
+    const uint32_t ak = s0 + st * kSStage, av = ak + kTile;
+    failed = !__syncthreads_and(mbar_wait(smem_addr(&bar_ld[st]), (uint32_t)(it >> 1) & 1u, a.budget_ns, nullptr));
+    if (failed) break;
+    phi_tile(sm + st * kSStage, valid, true);
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {
       tc_after_sync();
       constexpr uint32_t id = idesc(128, 48, true, true);
+      const uint32_t ones_off = s0 + kSOnes - av;
 #pragma unroll
-      for (int s = 0; s < kL / 16; ++s) mma(ctl.tmem, mnmaj64(s0, s, kTile), mnmaj64(s0 + kTile, s, kTile), id, s > 0);
-      mma_commit(bm);
+      for (int k16 = 0; k16 < kL / 16; ++k16)
+        mma(tm, mnmaj64(ak, k16, kTile), mnmaj64(av, k16, ones_off), id, k16 > 0);
+      mma_commit(smem_addr(&bar_mma));
     }
-    if (ctl_wait(&ctl, 1, 0, a)) {
-      tc_after_sync();
-      if (threadIdx.x < 32) {
-        float sv[32];
-        tmem_ld32(ctl.tmem, sv);
-        const float z = tmem_ld1(ctl.tmem + 32u);
-        float *r = a.rec + ((int64_t)h * a.nch + c) * kRec;
-        float4 *row = reinterpret_cast<float4 *>(r + threadIdx.x * kD);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) row[q] = make_float4(sv[4 * q], sv[4 * q + 1], sv[4 * q + 2], sv[4 * q + 3]);
-        r[kDM + threadIdx.x] = z;
+    mma_pending = true;
+    failed = !__syncthreads_and(mbar_wait(smem_addr(&bar_mma), mma_phase, a.budget_ns, nullptr));
+    if (failed) break;
+    mma_pending = false;
+    mma_phase ^= 1u;
+    tc_after_sync();
+    if (threadIdx.x == 0) {  // this stage's tiles are consumed: load the chunk two ahead into it
+      const int64_t nxt = idx + 2 * (int64_t)gridDim.x;
+      if (nxt < total) {
+        issue(nxt, st);
+        ++issued;
       }
     }
+    if (warp == 0) {
+      float sv[32];
+      tmem_ld32(tm, sv);
+      const float z = tmem_ld1(tm + 32u);
+      float *r = a.rec + ((int64_t)h * a.nch + c) * kRec;
+      float4 *row = reinterpret_cast<float4 *>(r + threadIdx.x * kD);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) row[q] = make_float4(sv[4 * q], sv[4 * q + 1], sv[4 * q + 2], sv[4 * q + 3]);
+      r[kDM + threadIdx.x] = z;
+    }
+    tc_before_sync();
+    __syncthreads();  // the accumulator is read before the next chunk's MMAs overwrite it
   }
-  ctl_finish(&ctl, 64, a);
+  if (failed && threadIdx.x == 0) {
+    atomicCAS(&a.hdr->status, 0, -5 /* WKV_ERR_TIMEOUT */);
+    if (mma_pending) mbar_wait(smem_addr(&bar_mma), mma_phase, a.budget_ns, nullptr);
+    for (int64_t m = it; m < issued; ++m)
+      mbar_wait(smem_addr(&bar_ld[m & 1]), (uint32_t)(m >> 1) & 1u, a.budget_ns, nullptr);
+  }
+  tc_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_after_sync();
+    tmem_dealloc(tm, 64);
+  }
 }
 
 // Exclusive prefix (or, reversed, suffix) of the chunk states of every head,
@@ -373,36 +437,106 @@ __device__ __forceinline__ float scores_to_tile(uint32_t tm_row, uint8_t *tile, 
   return rs;
 }
 
-// Forward outputs of one chunk.  Shared memory: phi(Q) at 0, phi(K) at 8K
-// (then the output tile), V at 16K, S_prev (bf16) at 24K, the masked scores
-// at 32K (32K bytes).
+// Masked scores of the thread's row (warp w holds rows 32w..32w+31) into
+// a [128 x 128] bf16 tile.  Column blocks left of the warp's diagonal block
+// need no mask, those right of it are zero (their TMEM columns are not read).
+__device__ __forceinline__ void causal_scores_to_tile(uint32_t tm_row, uint8_t *tile, int i) {
+  const int w = i >> 5;
+#pragma unroll 1
+  for (int b = 0; b < 4; ++b) {
+    float v[32];
+    if (b <= w) {
+      tmem_ld32(tm_row + 32u * b, v);
+      if (b == w) {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) v[r] = (32 * b + r <= i) ? v[r] : 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < 32; ++r) v[r] = 0.f;
+    }
+    put_row128(tile, i, b, v);
+  }
+}
+
+// Forward outputs.  Persistent: CTA g takes chunks g, g + G, ... (G = the
+// grid) and double-buffers their Q, K, V tiles, so a chunk's loads run
+// while the one before it is computed.  Per chunk: scores phi(Q) phi(K)^T
+// (2 MMAs), the masked score tile, then numerators and denominator in one
+// accumulator, A [V | 1] + phi(Q) [S_prev | Z_prev] (10 MMAs, N = 48:
+// column 32 is the denominator), and out = numerators / denominator.
+// Shared memory: two stages of (phi(Q), phi(K) then the output tile, V) at
+// 0 and 24K, a ones tile at 48K, S_prev and Z_prev (bf16) at 56K and 58K,
+// the score tile at 64K (32K bytes).
+constexpr uint32_t kFStage = 3 * kTile, kFOnes = 2 * kFStage, kFS = kFOnes + kTile, kFZ = kFS + kStile,
+                   kFP = 8 * kTile;
 __global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant__ CUtensorMap qmap,
                                                           const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap vmap,
                                                           const __grid_constant__ CUtensorMap omap, LaArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ Ctl ctl;
-  __shared__ float zprev[kD];
+  __shared__ uint64_t bar_ld[2], bar_mma;
+  __shared__ uint32_t tmem_s;
   uint8_t *sm = align1k(smem_raw);
   const uint32_t s0 = smem_addr(sm);
-  uint8_t *tq = sm, *tk = sm + kTile, *ts = sm + 3 * kTile, *tp = sm + 4 * kTile;
-  const uint32_t aq = s0, ak = s0 + kTile, av = s0 + 2 * kTile, as = s0 + 3 * kTile, ap = s0 + 4 * kTile;
-  const int h = (int)(blockIdx.x / a.nch), c = (int)(blockIdx.x % a.nch);
-  const int i = threadIdx.x;
+  const int64_t total = a.BH * a.nch;
+  const int i = threadIdx.x, warp = threadIdx.x >> 5;
   const uint32_t lane_off = (uint32_t)(threadIdx.x & ~31) << 16;
-  ctl_setup(&ctl, 128);
-  const uint32_t bl = smem_addr(&ctl.bar[0]), bm = smem_addr(&ctl.bar[1]);
   if (threadIdx.x == 0) {
-    const uint64_t pol = l2_policy_evict_first();
-    mbar_expect_tx(bl, 3 * kTile);
-    tma_load_3d(aq, &qmap, 0, c * kL, h, bl, pol);
-    tma_load_3d(ak, &kmap, 0, c * kL, h, bl, pol);
-    tma_load_3d(av, &vmap, 0, c * kL, h, bl, pol);
+    mbar_init(smem_addr(&bar_ld[0]), 1);
+    mbar_init(smem_addr(&bar_ld[1]), 1);
+    mbar_init(smem_addr(&bar_mma), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  const float *prev = a.rec + ((int64_t)h * a.nch + c) * kRec;
-  put_state_tile(ts, prev);
-  if (threadIdx.x < kD) zprev[threadIdx.x] = prev[kDM + threadIdx.x];
-  if (ctl_wait(&ctl, 0, 0, a)) {
+  if (warp == 0) {
+    tmem_alloc(smem_addr(&tmem_s), 128);
+    tmem_relinquish();
+  }
+  {
+    uint4 *o = reinterpret_cast<uint4 *>(sm + kFOnes);
+    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kThreads)
+      o[g] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // bf16 1.0
+  }
+  tc_before_sync();
+  __syncthreads();
+  tc_after_sync();
+  const uint32_t tm = tmem_s;
+  const uint64_t pol = l2_policy_evict_first();
+  auto issue = [&](int64_t idx, int st) {
+    const int h = (int)(idx / a.nch), c = (int)(idx % a.nch);
+    const uint32_t dst = s0 + st * kFStage, bar = smem_addr(&bar_ld[st]);
+    mbar_expect_tx(bar, 3 * kTile);
+    tma_load_3d(dst, &qmap, 0, c * kL, h, bar, pol);
+    tma_load_3d(dst + kTile, &kmap, 0, c * kL, h, bar, pol);
+    tma_load_3d(dst + 2 * kTile, &vmap, 0, c * kL, h, bar, pol);
+  };
+  int64_t issued = 0;  // chunks of this CTA whose loads were issued (thread 0)
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < 2; ++st)
+      if ((int64_t)blockIdx.x + (int64_t)st * gridDim.x < total) {
+        issue((int64_t)blockIdx.x + (int64_t)st * gridDim.x, st);
+        ++issued;
+      }
+  }
+  uint32_t mma_phase = 0;
+  int it = 0;
+  bool failed = false, mma_pending = false;  // uniform over the CTA
+  for (int64_t idx = blockIdx.x; idx < total; idx += gridDim.x, ++it) {
+    const int st = it & 1;
+    const int h = (int)(idx / a.nch), c = (int)(idx % a.nch);
+    uint8_t *tq = sm + st * kFStage, *tk = tq + kTile;
+    const uint32_t aq = s0 + st * kFStage, ak = aq + kTile, av = aq + 2 * kTile;
+    // S_prev and Z_prev of this chunk (the previous chunk's MMAs are complete)
+    const float *prev = a.rec + ((int64_t)h * a.nch + c) * kRec;
+    put_state_tile(sm + kFS, prev);
+    if (threadIdx.x < kD) {
+      const uint32_t zz = pack2(prev[kDM + threadIdx.x], prev[kDM + threadIdx.x]);
+      const uint4 x = make_uint4(zz, zz, zz, zz);
+      uint4 *row = reinterpret_cast<uint4 *>(sm + kFZ + 64 * threadIdx.x);
+      row[0] = x, row[1] = x, row[2] = x, row[3] = x;
+    }
+    failed = !__syncthreads_and(mbar_wait(smem_addr(&bar_ld[st]), (uint32_t)(it >> 1) & 1u, a.budget_ns, nullptr));
+    if (failed) break;
     phi_tile(tq, kL, false);
     phi_tile(tk, kL, false);
     fence_proxy_async_smem();
@@ -410,50 +544,75 @@ __global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant_
     if (threadIdx.x == 0) {  // scores phi(Q) phi(K)^T
       tc_after_sync();
       constexpr uint32_t id = idesc(128, 128, false, false);
-      mma(ctl.tmem, kmaj64(aq, 0), kmaj64(ak, 0), id, false);
-      mma(ctl.tmem, kmaj64(aq, 1), kmaj64(ak, 1), id, true);
-      mma_commit(bm);
+      mma(tm, kmaj64(aq, 0), kmaj64(ak, 0), id, false);
+      mma(tm, kmaj64(aq, 1), kmaj64(ak, 1), id, true);
+      mma_commit(smem_addr(&bar_mma));
+      // the previous chunk's stage is free once its output store has read
+      // it: load the chunk after this one there
+      const int64_t nxt = idx + gridDim.x;
+      if (it >= 1 && nxt < total) {
+        bulk_wait_read_all();
+        issue(nxt, st ^ 1);
+        ++issued;
+      }
     }
-    if (ctl_wait(&ctl, 1, 0, a)) {
+    mma_pending = true;
+    failed = !__syncthreads_and(mbar_wait(smem_addr(&bar_mma), mma_phase, a.budget_ns, nullptr));
+    if (failed) break;
+    mma_pending = false;
+    mma_phase ^= 1u;
+    tc_after_sync();
+    causal_scores_to_tile(tm + lane_off, sm + kFP, i);
+    tc_before_sync();
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {  // A [V | 1] + phi(Q) [S_prev | Z_prev]
       tc_after_sync();
-      const float rs = scores_to_tile(ctl.tmem + lane_off, tp, i, 0.f);
-      float fq[32];
-      get_row64(tq, i, fq);
-      float qz = 0.f;
+      constexpr uint32_t id = idesc(128, 48, false, true);
+      const uint32_t ones_off = s0 + kFOnes - av;
 #pragma unroll
-      for (int d = 0; d < kD; ++d) qz = fmaf(fq[d], zprev[d], qz);
-      const float den = rs + qz;
-      tc_before_sync();
-      fence_proxy_async_smem();
-      __syncthreads();
-      if (threadIdx.x == 0) {  // numerators A V + phi(Q) S_prev, into columns 0..31
-        tc_after_sync();
-        constexpr uint32_t id = idesc(128, 32, false, true);
+      for (int k16 = 0; k16 < kL / 16; ++k16) mma(tm, kmaj128(s0 + kFP, k16), mnmaj64(av, k16, ones_off), id, k16 > 0);
+      mma(tm, kmaj64(aq, 0), mnmaj64(s0 + kFS, 0, kStile), id, true);
+      mma(tm, kmaj64(aq, 1), mnmaj64(s0 + kFS, 1, kStile), id, true);
+      mma_commit(smem_addr(&bar_mma));
+    }
+    mma_pending = true;
+    failed = !__syncthreads_and(mbar_wait(smem_addr(&bar_mma), mma_phase, a.budget_ns, nullptr));
+    if (failed) break;
+    mma_pending = false;
+    mma_phase ^= 1u;
+    tc_after_sync();
+    float o[32];
+    tmem_ld32(tm + lane_off, o);
+    const float inv = 1.f / tmem_ld1(tm + lane_off + 32u);
 #pragma unroll
-        for (int s = 0; s < kL / 16; ++s) mma(ctl.tmem, kmaj128(ap, s), mnmaj64(av, s, kTile), id, s > 0);
-        mma(ctl.tmem, kmaj64(aq, 0), mnmaj64(as, 0, kTile), id, true);
-        mma(ctl.tmem, kmaj64(aq, 1), mnmaj64(as, 1, kTile), id, true);
-        mma_commit(bm);
-      }
-      if (ctl_wait(&ctl, 1, 1, a)) {
-        tc_after_sync();
-        float o[32];
-        tmem_ld32(ctl.tmem + lane_off, o);
-        const float inv = 1.f / den;
-#pragma unroll
-        for (int m = 0; m < kD; ++m) o[m] *= inv;
-        put_row64(tk, i, o);  // phi(K) is no longer read
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (threadIdx.x == 0) {
-          tma_store_3d(&omap, 0, c * kL, h, ak);
-          bulk_commit();
-          bulk_wait_all();
-        }
-      }
+    for (int m = 0; m < kD; ++m) o[m] *= inv;
+    put_row64(tk, i, o);  // phi(K) is no longer read
+    tc_before_sync();
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tma_store_3d(&omap, 0, c * kL, h, ak);
+      bulk_commit();
     }
   }
-  ctl_finish(&ctl, 128, a);
+  if (failed) {
+    // a wait gave up (WKV_ERR_TIMEOUT): wait once more, bounded, for what is
+    // still in flight before the shared and tensor memory are released
+    if (threadIdx.x == 0) {
+      atomicCAS(&a.hdr->status, 0, -5 /* WKV_ERR_TIMEOUT */);
+      if (mma_pending) mbar_wait(smem_addr(&bar_mma), mma_phase, a.budget_ns, nullptr);
+      for (int64_t m = it; m < issued; ++m)
+        mbar_wait(smem_addr(&bar_ld[m & 1]), (uint32_t)(m >> 1) & 1u, a.budget_ns, nullptr);
+    }
+  }
+  if (threadIdx.x == 0) bulk_wait_all();
+  tc_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_after_sync();
+    tmem_dealloc(tm, 128);
+  }
 }
 
 // Backward, first part, of one chunk: den and out again, gnum = G / den
@@ -709,8 +868,8 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
 }
 
 // Shared-memory bytes of each kernel (tiles plus the 1 KB alignment slack).
-constexpr int kStateSmem = 4 * kTile + 1024;
-constexpr int kFwdSmem = 4 * kTile + 4 * kTile + 1024;   // Q, K, V, S | scores
+constexpr int kStateSmem = 6 * kTile + 1024;             // 2 x (K, V), ones, spare rows
+constexpr int kFwdSmem = 12 * kTile + 1024;              // 2 x (Q, K, V), ones, S, Z | scores
 constexpr int kPrepSmem = 8 * kTile + 4 * kTile + 1024;  // Q, gnum, gden, K, V, G, S (+pad) | scores
 constexpr int kBwdSmem = 13 * kTile + 1024;              // Q, K, V, gnum, S+U (+pad) | A, P
 
@@ -747,12 +906,36 @@ bool la_layout(int op, int64_t BH, int64_t N, LaLayout *L) {
 }
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Grid of a persistent kernel: one wave of resident CTAs, at most one per
+// chunk.  Residency is counted from the shared memory per SM and the tensor
+// memory each CTA allocates (512 columns per SM); the occupancy calculator
+// does not know the latter.
+int la_num_sms();
+template <typename K>
+int64_t persistent_grid(K kern, int smem, int tmem_cols, int64_t units) {
+  int dev = 0, per_sm = 0, reserved = 0;
+  cudaFuncAttributes fa{};
+  int occ = 1;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) == cudaSuccess &&
+      cudaFuncGetAttributes(&fa, (const void *)kern) == cudaSuccess)
+    occ = per_sm / (smem + (int)fa.sharedSizeBytes + reserved);
+  occ = std::max(1, std::min(occ, std::min(512 / tmem_cols, 2048 / kThreads)));
+  return std::min<int64_t>(units, (int64_t)occ * la_num_sms());
+}
 template <typename K>
 int prepare(K kern, int smem) {
   int occ = 0;
   return blocks_per_sm((const void *)kern, kThreads, smem, &occ) == cudaSuccess && occ >= 1 ? 0 : -1;
 }
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? WKV_OK : WKV_ERR_CUDA; }
+int la_num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 148;
+  return n;
+}
 constexpr int64_t kBudgetNs = 1000000000;  // one second per bounded wait
 
 int check_common(int64_t BH, int64_t N, int D, int M, void *ws, size_t ws_bytes, int op, LaLayout *L) {
@@ -797,13 +980,15 @@ extern "C" int linattn_forward(int64_t BH, int64_t N, int D, int M, const void *
         !encode_heads_sw64(&vm, v, BH, N, kD) || !encode_heads_sw64(&om, out, BH, N, kD))
       return WKV_ERR_UNSUPPORTED;
     if (prepare(la_state_kernel, kStateSmem) || prepare(la_fwd_kernel, kFwdSmem)) return WKV_ERR_CUDA;
-    cudaError_t e = launch_kernel(la_state_kernel, dim3((unsigned)units), dim3(kThreads), kStateSmem, st, km, vm, a);
+    cudaError_t e = launch_kernel(la_state_kernel, dim3((unsigned)persistent_grid(la_state_kernel, kStateSmem, 64, units)),
+                                  dim3(kThreads), kStateSmem, st, km, vm, a);
     if (e != cudaSuccess) return WKV_ERR_CUDA;
     const int64_t n = BH * kRec;
     e = launch_kernel(la_scan_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, a.rec, BH, a.nch, 0,
                       state_out);
     if (e != cudaSuccess) return WKV_ERR_CUDA;
-    return cuda_rc(launch_kernel(la_fwd_kernel, dim3((unsigned)units), dim3(kThreads), kFwdSmem, st, qm, km, vm, om, a));
+    return cuda_rc(launch_kernel(la_fwd_kernel, dim3((unsigned)persistent_grid(la_fwd_kernel, kFwdSmem, 128, units)),
+                                 dim3(kThreads), kFwdSmem, st, qm, km, vm, om, a));
   }
   if (state_out)  // N = 0: the empty state
     return cuda_rc(cudaMemsetAsync(state_out, 0, (size_t)BH * kRec * sizeof(float), st));
@@ -857,7 +1042,8 @@ extern "C" int linattn_backward(int64_t BH, int64_t N, int D, int M, const void 
   const int64_t units = BH * a.nch;
   const int64_t n = BH * kRec;
   const dim3 sgrid((unsigned)((n + 255) / 256));
-  cudaError_t e = launch_kernel(la_state_kernel, dim3((unsigned)units), dim3(kThreads), kStateSmem, st, km, vm, a);
+  cudaError_t e = launch_kernel(la_state_kernel, dim3((unsigned)persistent_grid(la_state_kernel, kStateSmem, 64, units)),
+                                dim3(kThreads), kStateSmem, st, km, vm, a);
   if (e == cudaSuccess) e = launch_kernel(la_scan_kernel, sgrid, dim3(256), 0, st, a.rec, BH, a.nch, 0, (float *)nullptr);
   if (e == cudaSuccess)
     e = launch_kernel(la_bwd_prep_kernel, dim3((unsigned)units), dim3(kThreads), kPrepSmem, st, qm, km, vm, gm, nm, a);
