@@ -89,10 +89,10 @@ KERNEL_SOURCES = {
 # (workload, kernel, gated, source hash).  A kernel whose sources changed
 # since its capture has no entry: its traffic is reported as null.
 TRAFFIC = {
-    ("rwkv1b5_bf16", "bwd_tile_kernel", False, "3e37f5ec7a6ae4a4"): 419_564_544 + 294_213_120,
-    ("rwkv1b5_bf16", "fwd_tile_kernel", False, "8c380ad936d96fa8"): 279_003_904 + 155_246_848,
-    ("longctx", "fwd_seg_kernel", False, "90dd4931d4709195"): 1_569_629_184 + 639_891_200,
-    ("decode14b", "step_kernel", False, "7c9eb86718fc5d51"): 52_482_920 + 68_656,
+    ("rwkv1b5_bf16", "bwd_tile_kernel", False, "7081082af783b8f4"): 417_490_176 + 294_261_504,
+    ("rwkv1b5_bf16", "fwd_tile_kernel", False, "9336be216ceb647f"): 278_985_472 + 155_384_320,
+    ("longctx", "fwd_seg_kernel", False, "fb83390fdf2b28e1"): 1_578_090_752 + 640_600_320,
+    ("decode14b", "step_kernel", False, "ceedfbaab295393e"): 52_483_344 + 71_440,
 }
 
 
