@@ -75,12 +75,12 @@ KERNEL_IDS = {"auto": 0, "segment": 6, "cluster": 7, "tile": 8}
 # The source files each kernel is built from: a DRAM-traffic figure measured
 # by ncu is reported only while these files are unchanged since the capture.
 KERNEL_SOURCES = {
-    "fwd_tile_kernel": ["wkv_tile.cu", "wkv_tile.cuh", "wkv_internal.cuh", "wkv_math.cuh"],
+    "fwd_tile_kernel": ["wkv_tile.cu", "wkv_tile.cuh", "wkv_internal.cuh", "wkv_math.cuh", "wkv_forward.cu"],
     "bwd_tile_kernel": ["wkv_tile_bwd.cu", "wkv_tile.cuh", "wkv_bwd_math.cuh", "wkv_internal.cuh",
-                        "wkv_math.cuh"],
+                        "wkv_math.cuh", "wkv_forward.cu"],
     "bwd_seg_kernel": ["wkv_seg_bwd.cu", "wkv_ring.cuh", "wkv_bwd_math.cuh", "wkv_internal.cuh",
-                       "wkv_math.cuh"],
-    "fwd_seg_kernel": ["wkv_seg.cu", "wkv_ring.cuh", "wkv_internal.cuh", "wkv_math.cuh"],
+                       "wkv_math.cuh", "wkv_forward.cu"],
+    "fwd_seg_kernel": ["wkv_seg.cu", "wkv_ring.cuh", "wkv_internal.cuh", "wkv_math.cuh", "wkv_forward.cu"],
     "step_kernel": ["wkv_step.cu", "wkv_internal.cuh"],
 }
 

@@ -547,10 +547,13 @@ bool encode_rows(CUtensorMap *m, const void *ptr, int dtype, int64_t rows, int64
   cuuint64_t strides[1] = {(cuuint64_t)(C * es)};
   cuuint32_t box[2] = {32u, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
+  // L2 fills promoted to the box row (32 columns) and no further: a wider
+  // fill fetches the neighbouring chain's bytes on this chain's behalf, and
+  // they may leave L2 before that chain's warp reads them
+  const auto promo = dtype == 0 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
   if (enc(m, dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
           const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+          CU_TENSOR_MAP_SWIZZLE_NONE, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
   map_insert(key, *m);
   return true;
