@@ -59,6 +59,7 @@ constexpr uint32_t kTile = kL * kD * 2;  // bytes of a [128 x 32] bf16 tile
 constexpr uint32_t kStile = kD * kD * 2; // bytes of a [32 x 32] bf16 tile
 constexpr uint32_t kPhalf = kL * 64 * 2; // bytes of one [128 x 64] half of a score tile
 constexpr int kThreads = 128;
+constexpr int kFwdThreads = 256;  // the persistent kernels: two warpgroups
 
 struct LaArgs {
   int64_t BH, N;
@@ -114,12 +115,33 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
+// 16 consecutive columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
+}
 // One column of this warp's 32 lanes.
 __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
   uint32_t r;
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
   return __uint_as_float(r);
+}
+
+// Bulk copy (no tensor map) of `bytes` from global memory into shared memory,
+// completing on `bar`; both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
 // Shared-memory matrix descriptor: start address, leading and stride byte
@@ -165,11 +187,13 @@ __device__ __forceinline__ uint32_t phi2(uint32_t w) { return pack2(phi(lo16(w))
 __device__ __forceinline__ uint32_t sw64(int r, int u) { return (uint32_t)(r * 64 + ((u ^ ((r >> 1) & 3)) << 4)); }
 __device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
-// phi in place over a [128 x 32] tile; rows >= `valid` become 0 if `zero_tail`.
+// phi in place over a [128 x 32] tile by NT threads; rows >= `valid` become
+// 0 if `zero_tail`.
+template <int NT = kThreads>
 __device__ __forceinline__ void phi_tile(uint8_t *t, int valid, bool zero_tail) {
 #pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const int g = it * kThreads + (int)threadIdx.x;  // 16-byte unit; its row is g / 4
+  for (int it = 0; it < 512 / NT; ++it) {
+    const int g = it * NT + (int)threadIdx.x;  // 16-byte unit; its row is g / 4
     uint4 *p = reinterpret_cast<uint4 *>(t + 16 * g);
     uint4 x = *p;
     if (zero_tail && (g >> 2) >= valid) {
@@ -205,8 +229,8 @@ __device__ __forceinline__ void put_row128(uint8_t *t, int r, int b, const float
                    pack2(v[8 * q + 4], v[8 * q + 5]), pack2(v[8 * q + 6], v[8 * q + 7]));
 }
 // A [32 x 32] float32 chunk state (row-major) into a bf16 64-byte-swizzle tile.
-__device__ __forceinline__ void put_state_tile(uint8_t *t, const float *src) {
-  const int d = threadIdx.x >> 2, u = threadIdx.x & 3;
+__device__ __forceinline__ void put_state_tile(uint8_t *t, const float *src, int tid = threadIdx.x) {
+  const int d = tid >> 2, u = tid & 3;  // 128 threads
   const float4 a = *reinterpret_cast<const float4 *>(src + d * kD + 8 * u);
   const float4 b = *reinterpret_cast<const float4 *>(src + d * kD + 8 * u + 4);
   *reinterpret_cast<uint4 *>(t + sw64(d, u)) = make_uint4(pack2(a.x, a.y), pack2(a.z, a.w), pack2(b.x, b.y),
@@ -273,7 +297,7 @@ __device__ __forceinline__ uint8_t *align1k(uint8_t *p) {
 // complete).  Shared memory: stages (phi(K), V) at 0 and 16K, the ones tile
 // at 32K; the spare rows of stage 1's A operand reach to 48K.
 constexpr uint32_t kSStage = 2 * kTile, kSOnes = 2 * kSStage;
-__global__ void __launch_bounds__(kThreads) la_state_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(kFwdThreads) la_state_kernel(const __grid_constant__ CUtensorMap kmap,
                                                             const __grid_constant__ CUtensorMap vmap, LaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_ld[2], bar_mma;
@@ -294,7 +318,7 @@ __global__ void __launch_bounds__(kThreads) la_state_kernel(const __grid_constan
   }
   {
     uint4 *o = reinterpret_cast<uint4 *>(sm + kSOnes);
-    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kThreads)
+    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kFwdThreads)
       o[g] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // bf16 1.0
   }
   tc_before_sync();
@@ -328,7 +352,7 @@ __global__ void __launch_bounds__(kThreads) la_state_kernel(const __grid_constan
     const uint32_t ak = s0 + st * kSStage, av = ak + kTile;
     failed = !__syncthreads_and(mbar_wait(smem_addr(&bar_ld[st]), (uint32_t)(it >> 1) & 1u, a.budget_ns, nullptr));
     if (failed) break;
-    phi_tile(sm + st * kSStage, valid, true);
+    phi_tile<kFwdThreads>(sm + st * kSStage, valid, true);
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -417,37 +441,54 @@ __global__ void la_scan_kernel(float *rec, int64_t BH, int nch, int reverse, flo
   }
 }
 
-// Masked scores of the thread's row into a [128 x 128] bf16 tile; returns
-// the row sum (float32, before rounding).  With `gden` >= its sentinel the
-// kept entries get + gden (the backward's P).
+// Masked scores of the thread's row into a [128 x 128] bf16 tile (4 warps,
+// warp w holding rows 32w..32w+31); returns the row sum (float32, before
+// rounding).  Kept entries get + `add` (the backward's P).  Column blocks
+// left of the warp's diagonal block need no mask, those right of it are
+// zero and their TMEM columns are not read.
 __device__ __forceinline__ float scores_to_tile(uint32_t tm_row, uint8_t *tile, int i, float add) {
+  const int w = i >> 5;
   float rs = 0.f;
 #pragma unroll 1
   for (int b = 0; b < 4; ++b) {
     float v[32];
-    tmem_ld32(tm_row + 32u * b, v);
+    if (b <= w) {
+      tmem_ld32(tm_row + 32u * b, v);
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      const float x = (32 * b + r <= i) ? v[r] + add : 0.f;
-      v[r] = x;
-      rs += x;
+      for (int r = 0; r < 32; ++r) {
+        const float x = (b < w || 32 * b + r <= i) ? v[r] + add : 0.f;
+        v[r] = x;
+        rs += x;
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < 32; ++r) v[r] = 0.f;
     }
     put_row128(tile, i, b, v);
   }
   return rs;
 }
 
-// Masked scores of the thread's row (warp w holds rows 32w..32w+31) into
-// a [128 x 128] bf16 tile.  Column blocks left of the warp's diagonal block
-// need no mask, those right of it are zero (their TMEM columns are not read).
-__device__ __forceinline__ void causal_scores_to_tile(uint32_t tm_row, uint8_t *tile, int i) {
+// Masked scores of the thread's row (its warp holds rows 32w..32w+31) into
+// a [128 x 128] bf16 tile, for two of the four 32-column blocks: warpgroup 0
+// takes blocks 0 and 3, warpgroup 1 blocks 1 and 2 (the causal mask gives
+// both about the same work).  Column blocks left of the warp's diagonal
+// block need no mask, those right of it are zero (their TMEM columns are
+// not read).
+template <bool ADD = false>
+__device__ __forceinline__ void causal_scores_to_tile(uint32_t tm_row, uint8_t *tile, int i, int wg,
+                                                      float add = 0.f) {
   const int w = i >> 5;
 #pragma unroll 1
-  for (int b = 0; b < 4; ++b) {
+  for (int q = 0; q < 2; ++q) {
+    const int b = wg == 0 ? 3 * q : 1 + q;
     float v[32];
     if (b <= w) {
       tmem_ld32(tm_row + 32u * b, v);
-      if (b == w) {
+      if (ADD) {
+#pragma unroll
+        for (int r = 0; r < 32; ++r) v[r] = (b < w || 32 * b + r <= i) ? v[r] + add : 0.f;
+      } else if (b == w) {
 #pragma unroll
         for (int r = 0; r < 32; ++r) v[r] = (32 * b + r <= i) ? v[r] : 0.f;
       }
@@ -467,10 +508,12 @@ __device__ __forceinline__ void causal_scores_to_tile(uint32_t tm_row, uint8_t *
 // column 32 is the denominator), and out = numerators / denominator.
 // Shared memory: two stages of (phi(Q), phi(K) then the output tile, V) at
 // 0 and 24K, a ones tile at 48K, S_prev and Z_prev (bf16) at 56K and 58K,
-// the score tile at 64K (32K bytes).
+// the score tile at 64K (32K bytes), and per stage the chunk's float32
+// (S_prev, Z_prev) record, copied in with its tiles, at 96K.
 constexpr uint32_t kFStage = 3 * kTile, kFOnes = 2 * kFStage, kFS = kFOnes + kTile, kFZ = kFS + kStile,
-                   kFP = 8 * kTile;
-__global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant__ CUtensorMap qmap,
+                   kFP = 8 * kTile, kFRec = 12 * kTile, kRecBytes = kRec * 4;
+static_assert(kRecBytes % 128 == 0, "records stay 128-byte aligned in shared memory");
+__global__ void __launch_bounds__(kFwdThreads) la_fwd_kernel(const __grid_constant__ CUtensorMap qmap,
                                                           const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap vmap,
                                                           const __grid_constant__ CUtensorMap omap, LaArgs a) {
@@ -480,8 +523,10 @@ __global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant_
   uint8_t *sm = align1k(smem_raw);
   const uint32_t s0 = smem_addr(sm);
   const int64_t total = a.BH * a.nch;
-  const int i = threadIdx.x, warp = threadIdx.x >> 5;
-  const uint32_t lane_off = (uint32_t)(threadIdx.x & ~31) << 16;
+  // 8 warps: row i = thread % 128 (warp w % 4 reads TMEM lanes 32(w % 4)..);
+  // the two warpgroups split the epilogues' columns
+  const int i = threadIdx.x & 127, wg = threadIdx.x >> 7, warp = threadIdx.x >> 5;
+  const uint32_t lane_off = (uint32_t)(i & ~31) << 16;
   if (threadIdx.x == 0) {
     mbar_init(smem_addr(&bar_ld[0]), 1);
     mbar_init(smem_addr(&bar_ld[1]), 1);
@@ -494,7 +539,7 @@ __global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant_
   }
   {
     uint4 *o = reinterpret_cast<uint4 *>(sm + kFOnes);
-    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kThreads)
+    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kFwdThreads)
       o[g] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // bf16 1.0
   }
   tc_before_sync();
@@ -505,10 +550,11 @@ __global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant_
   auto issue = [&](int64_t idx, int st) {
     const int h = (int)(idx / a.nch), c = (int)(idx % a.nch);
     const uint32_t dst = s0 + st * kFStage, bar = smem_addr(&bar_ld[st]);
-    mbar_expect_tx(bar, 3 * kTile);
+    mbar_expect_tx(bar, 3 * kTile + kRecBytes);
     tma_load_3d(dst, &qmap, 0, c * kL, h, bar, pol);
     tma_load_3d(dst + kTile, &kmap, 0, c * kL, h, bar, pol);
     tma_load_3d(dst + 2 * kTile, &vmap, 0, c * kL, h, bar, pol);
+    bulk_load(s0 + kFRec + st * kRecBytes, a.rec + ((int64_t)h * a.nch + c) * kRec, kRecBytes, bar);
   };
   int64_t issued = 0;  // chunks of this CTA whose loads were issued (thread 0)
   if (threadIdx.x == 0) {
@@ -526,19 +572,21 @@ __global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant_
     const int h = (int)(idx / a.nch), c = (int)(idx % a.nch);
     uint8_t *tq = sm + st * kFStage, *tk = tq + kTile;
     const uint32_t aq = s0 + st * kFStage, ak = aq + kTile, av = aq + 2 * kTile;
-    // S_prev and Z_prev of this chunk (the previous chunk's MMAs are complete)
-    const float *prev = a.rec + ((int64_t)h * a.nch + c) * kRec;
-    put_state_tile(sm + kFS, prev);
-    if (threadIdx.x < kD) {
-      const uint32_t zz = pack2(prev[kDM + threadIdx.x], prev[kDM + threadIdx.x]);
-      const uint4 x = make_uint4(zz, zz, zz, zz);
-      uint4 *row = reinterpret_cast<uint4 *>(sm + kFZ + 64 * threadIdx.x);
-      row[0] = x, row[1] = x, row[2] = x, row[3] = x;
-    }
     failed = !__syncthreads_and(mbar_wait(smem_addr(&bar_ld[st]), (uint32_t)(it >> 1) & 1u, a.budget_ns, nullptr));
     if (failed) break;
-    phi_tile(tq, kL, false);
-    phi_tile(tk, kL, false);
+    // S_prev and Z_prev of this chunk, from the copy that came with its tiles,
+    // as bf16 operand tiles (the previous chunk's MMAs are complete)
+    const float *prev = reinterpret_cast<const float *>(sm + kFRec + st * kRecBytes);
+    if (threadIdx.x < kThreads) put_state_tile(sm + kFS, prev);
+    if (threadIdx.x >= kThreads && threadIdx.x < kThreads + kD) {
+      const int d = threadIdx.x - kThreads;
+      const uint32_t zz = pack2(prev[kDM + d], prev[kDM + d]);
+      const uint4 x = make_uint4(zz, zz, zz, zz);
+      uint4 *row = reinterpret_cast<uint4 *>(sm + kFZ + 64 * d);
+      row[0] = x, row[1] = x, row[2] = x, row[3] = x;
+    }
+    phi_tile<kFwdThreads>(tq, kL, false);
+    phi_tile<kFwdThreads>(tk, kL, false);
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {  // scores phi(Q) phi(K)^T
@@ -562,7 +610,7 @@ __global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant_
     mma_pending = false;
     mma_phase ^= 1u;
     tc_after_sync();
-    causal_scores_to_tile(tm + lane_off, sm + kFP, i);
+    causal_scores_to_tile(tm + lane_off, sm + kFP, i, wg);
     tc_before_sync();
     fence_proxy_async_smem();
     __syncthreads();
@@ -582,12 +630,14 @@ __global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant_
     mma_pending = false;
     mma_phase ^= 1u;
     tc_after_sync();
-    float o[32];
-    tmem_ld32(tm + lane_off, o);
+    float o[16];  // this warpgroup's 16 of the 32 output columns
+    tmem_ld16(tm + lane_off + 16u * wg, o);
     const float inv = 1.f / tmem_ld1(tm + lane_off + 32u);
 #pragma unroll
-    for (int m = 0; m < kD; ++m) o[m] *= inv;
-    put_row64(tk, i, o);  // phi(K) is no longer read
+    for (int u = 0; u < 2; ++u)  // phi(K) is no longer read: the output goes there
+      *reinterpret_cast<uint4 *>(tk + sw64(i, 2 * wg + u)) =
+          make_uint4(pack2(o[8 * u] * inv, o[8 * u + 1] * inv), pack2(o[8 * u + 2] * inv, o[8 * u + 3] * inv),
+                     pack2(o[8 * u + 4] * inv, o[8 * u + 5] * inv), pack2(o[8 * u + 6] * inv, o[8 * u + 7] * inv));
     tc_before_sync();
     fence_proxy_async_smem();
     __syncthreads();
@@ -615,30 +665,34 @@ __global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant_
   }
 }
 
-// Backward, first part, of one chunk: den and out again, gnum = G / den
-// (bf16, to the workspace) and gden = -rowsum(G * out) / den (float32, to the
-// workspace), and the chunk's reverse state phi(Q)^T [gnum | gden].
-// Shared memory: phi(Q) 0, gnum 8K, gden (each row filled with its value)
-// 16K, phi(K) 24K, V 32K, G 40K, S_prev 48K, scores 64K (32K bytes).
-__global__ void __launch_bounds__(kThreads) la_bwd_prep_kernel(const __grid_constant__ CUtensorMap qmap,
-                                                               const __grid_constant__ CUtensorMap kmap,
-                                                               const __grid_constant__ CUtensorMap vmap,
-                                                               const __grid_constant__ CUtensorMap gmap,
-                                                               const __grid_constant__ CUtensorMap nmap, LaArgs a) {
+// Backward, first part, of one chunk: numerators and denominator again (as
+// the forward: A [V | 1] + phi(Q) [S_prev | Z_prev]), gnum = G / den (bf16,
+// to the workspace) and gden = -rowsum(G * out) / den (float32, to the
+// workspace), and the chunk's reverse state phi(Q)^T [gnum | gden].  Two
+// warpgroups: row i = thread % 128, the epilogues' columns split between
+// them.  Shared memory: phi(Q) 0, gnum 8K, gden (each row filled with its
+// value) 16K, phi(K) 24K, V 32K, G 40K, S_prev 48K, Z_prev 50K, scores 64K
+// (32K bytes), ones 96K.
+constexpr uint32_t kPOnes = 12 * kTile;
+__global__ void __launch_bounds__(kFwdThreads) la_bwd_prep_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                  const __grid_constant__ CUtensorMap kmap,
+                                                                  const __grid_constant__ CUtensorMap vmap,
+                                                                  const __grid_constant__ CUtensorMap gmap,
+                                                                  const __grid_constant__ CUtensorMap nmap, LaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ Ctl ctl;
-  __shared__ float zprev[kD];
+  __shared__ float gpart[kL];  // warpgroup 1's part of rowsum(G * out)
   uint8_t *sm = align1k(smem_raw);
   const uint32_t s0 = smem_addr(sm);
   uint8_t *tq = sm, *tn = sm + kTile, *tg_den = sm + 2 * kTile, *tk = sm + 3 * kTile, *tgo = sm + 5 * kTile,
-          *ts = sm + 6 * kTile, *tp = sm + 8 * kTile;
+          *ts = sm + 6 * kTile, *tz = sm + 6 * kTile + kStile, *tp = sm + 8 * kTile;
   const uint32_t aq = s0, an = s0 + kTile, ak = s0 + 3 * kTile, av = s0 + 4 * kTile, ag = s0 + 5 * kTile,
                  as = s0 + 6 * kTile, ap = s0 + 8 * kTile;
   const int h = (int)(blockIdx.x / a.nch), c = (int)(blockIdx.x % a.nch);
-  const int i = threadIdx.x;
+  const int i = threadIdx.x & 127, wg = threadIdx.x >> 7;
   const int64_t rem = a.N - (int64_t)c * kL;
   const int valid = rem < kL ? (int)rem : kL;
-  const uint32_t lane_off = (uint32_t)(threadIdx.x & ~31) << 16;
+  const uint32_t lane_off = (uint32_t)(i & ~31) << 16;
   ctl_setup(&ctl, 128);
   const uint32_t bl = smem_addr(&ctl.bar[0]), bm = smem_addr(&ctl.bar[1]);
   if (threadIdx.x == 0) {
@@ -649,12 +703,22 @@ __global__ void __launch_bounds__(kThreads) la_bwd_prep_kernel(const __grid_cons
     tma_load_3d(av, &vmap, 0, c * kL, h, bl, pol);
     tma_load_3d(ag, &gmap, 0, c * kL, h, bl, l2_policy_evict_first());
   }
+  {
+    uint4 *o = reinterpret_cast<uint4 *>(sm + kPOnes);
+    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kFwdThreads)
+      o[g] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // bf16 1.0
+  }
   const float *prev = a.rec + ((int64_t)h * a.nch + c) * kRec;
-  put_state_tile(ts, prev);
-  if (threadIdx.x < kD) zprev[threadIdx.x] = prev[kDM + threadIdx.x];
+  if (wg == 0) put_state_tile(ts, prev, i);
+  if (wg == 1 && i < kD) {  // Z_prev[d] across row d
+    const uint32_t zz = pack2(prev[kDM + i], prev[kDM + i]);
+    const uint4 x = make_uint4(zz, zz, zz, zz);
+    uint4 *row = reinterpret_cast<uint4 *>(tz + 64 * i);
+    row[0] = x, row[1] = x, row[2] = x, row[3] = x;
+  }
   if (ctl_wait(&ctl, 0, 0, a)) {
-    phi_tile(tq, kL, false);
-    phi_tile(tk, kL, false);
+    phi_tile<kFwdThreads>(tq, kL, false);
+    phi_tile<kFwdThreads>(tk, kL, false);
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -666,46 +730,52 @@ __global__ void __launch_bounds__(kThreads) la_bwd_prep_kernel(const __grid_cons
     }
     if (ctl_wait(&ctl, 1, 0, a)) {
       tc_after_sync();
-      const float rs = scores_to_tile(ctl.tmem + lane_off, tp, i, 0.f);
-      float fq[32];
-      get_row64(tq, i, fq);
-      float qz = 0.f;
-#pragma unroll
-      for (int d = 0; d < kD; ++d) qz = fmaf(fq[d], zprev[d], qz);
-      const float den = rs + qz;
+      causal_scores_to_tile(ctl.tmem + lane_off, tp, i, wg);
       tc_before_sync();
       fence_proxy_async_smem();
       __syncthreads();
-      if (threadIdx.x == 0) {
+      if (threadIdx.x == 0) {  // A [V | 1] + phi(Q) [S_prev | Z_prev]: column 32 is den
         tc_after_sync();
-        constexpr uint32_t id = idesc(128, 32, false, true);
+        constexpr uint32_t id = idesc(128, 48, false, true);
 #pragma unroll
-        for (int s = 0; s < kL / 16; ++s) mma(ctl.tmem, kmaj128(ap, s), mnmaj64(av, s, kTile), id, s > 0);
-        mma(ctl.tmem, kmaj64(aq, 0), mnmaj64(as, 0, kTile), id, true);
-        mma(ctl.tmem, kmaj64(aq, 1), mnmaj64(as, 1, kTile), id, true);
+        for (int k16 = 0; k16 < kL / 16; ++k16)
+          mma(ctl.tmem, kmaj128(ap, k16), mnmaj64(av, k16, s0 + kPOnes - av), id, k16 > 0);
+        mma(ctl.tmem, kmaj64(aq, 0), mnmaj64(as, 0, kStile), id, true);
+        mma(ctl.tmem, kmaj64(aq, 1), mnmaj64(as, 1, kStile), id, true);
         mma_commit(bm);
       }
       if (ctl_wait(&ctl, 1, 1, a)) {
         tc_after_sync();
-        float o[32], g[32];
-        tmem_ld32(ctl.tmem + lane_off, o);
-        get_row64(tgo, i, g);
-        const float inv = 1.f / den;
+        float o[16], g[16];  // this warpgroup's 16 columns
+        tmem_ld16(ctl.tmem + lane_off + 16u * wg, o);
+        const float inv = 1.f / tmem_ld1(ctl.tmem + lane_off + 32u);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const uint4 x = *reinterpret_cast<const uint4 *>(tgo + sw64(i, 2 * wg + u));
+          g[8 * u + 0] = lo16(x.x), g[8 * u + 1] = hi16(x.x), g[8 * u + 2] = lo16(x.y), g[8 * u + 3] = hi16(x.y);
+          g[8 * u + 4] = lo16(x.z), g[8 * u + 5] = hi16(x.z), g[8 * u + 6] = lo16(x.w), g[8 * u + 7] = hi16(x.w);
+        }
         float go = 0.f;
 #pragma unroll
-        for (int m = 0; m < kD; ++m) {
+        for (int m = 0; m < 16; ++m) {
           go = fmaf(g[m], o[m] * inv, go);
           g[m] *= inv;  // gnum
         }
-        const float gden = -go * inv;
-        put_row64(tn, i, g);
-        {
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          *reinterpret_cast<uint4 *>(tn + sw64(i, 2 * wg + u)) =
+              make_uint4(pack2(g[8 * u], g[8 * u + 1]), pack2(g[8 * u + 2], g[8 * u + 3]),
+                         pack2(g[8 * u + 4], g[8 * u + 5]), pack2(g[8 * u + 6], g[8 * u + 7]));
+        if (wg == 1) gpart[i] = go;
+        __syncthreads();
+        if (wg == 0) {
+          const float gden = -(go + gpart[i]) * inv;
           const uint32_t w = pack2(gden, gden);
           const uint4 x = make_uint4(w, w, w, w);
 #pragma unroll
           for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4 *>(tg_den + 64 * i + 16 * u) = x;
+          if (i < valid) a.gden[(int64_t)h * a.N + (int64_t)c * kL + i] = gden;
         }
-        if (i < valid) a.gden[(int64_t)h * a.N + (int64_t)c * kL + i] = gden;
         tc_before_sync();
         fence_proxy_async_smem();
         __syncthreads();
@@ -717,7 +787,8 @@ __global__ void __launch_bounds__(kThreads) la_bwd_prep_kernel(const __grid_cons
           tc_after_sync();
           constexpr uint32_t id3 = idesc(128, 48, true, true);
 #pragma unroll
-          for (int s = 0; s < kL / 16; ++s) mma(ctl.tmem, mnmaj64(aq, s, kTile), mnmaj64(an, s, kTile), id3, s > 0);
+          for (int k16 = 0; k16 < kL / 16; ++k16)
+            mma(ctl.tmem, mnmaj64(aq, k16, kTile), mnmaj64(an, k16, kTile), id3, k16 > 0);
           mma_commit(bm);
         }
         if (ctl_wait(&ctl, 1, 0, a)) {
@@ -742,8 +813,9 @@ __global__ void __launch_bounds__(kThreads) la_bwd_prep_kernel(const __grid_cons
 
 // Backward, gradients of one chunk.  Shared memory: phi(Q) 0, phi(K) 8K,
 // V 16K, gnum 24K, S_prev 32K, U_next 34K, masked A 40K, P 72K (32K bytes
-// each); the three output tiles reuse 40K, 48K, 56K at the end.
-__global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant__ CUtensorMap qmap,
+// each); the three output tiles reuse 40K, 48K, 56K at the end.  Two
+// warpgroups: row i = thread % 128, the epilogues' columns split between them.
+__global__ void __launch_bounds__(kFwdThreads) la_bwd_kernel(const __grid_constant__ CUtensorMap qmap,
                                                           const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap vmap,
                                                           const __grid_constant__ CUtensorMap nmap,
@@ -760,10 +832,10 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
   const uint32_t aq = s0, ak = s0 + kTile, av = s0 + 2 * kTile, an = s0 + 3 * kTile, as = s0 + 4 * kTile,
                  au = s0 + 4 * kTile + kStile, aa = s0 + 5 * kTile, app = s0 + 9 * kTile;
   const int h = (int)(blockIdx.x / a.nch), c = (int)(blockIdx.x % a.nch);
-  const int i = threadIdx.x;
+  const int i = threadIdx.x & 127, wg = threadIdx.x >> 7;
   const int64_t rem = a.N - (int64_t)c * kL;
   const int valid = rem < kL ? (int)rem : kL;
-  const uint32_t lane_off = (uint32_t)(threadIdx.x & ~31) << 16;
+  const uint32_t lane_off = (uint32_t)(i & ~31) << 16;
   ctl_setup(&ctl, 128);
   const uint32_t bl = smem_addr(&ctl.bar[0]), bm = smem_addr(&ctl.bar[1]);
   if (threadIdx.x == 0) {
@@ -776,16 +848,12 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
   }
   const float *prev = a.rec + ((int64_t)h * a.nch + c) * kRec;
   const float *next = a.rec_r + ((int64_t)h * a.nch + c) * kRec;
-  put_state_tile(ts, prev);
-  put_state_tile(tu, next);
-  if (threadIdx.x < kD) {
-    zprev[threadIdx.x] = prev[kDM + threadIdx.x];
-    unext[threadIdx.x] = next[kDM + threadIdx.x];
-  }
-  gden_s[i] = i < valid ? a.gden[(int64_t)h * a.N + (int64_t)c * kL + i] : 0.f;
+  put_state_tile(wg == 0 ? ts : tu, wg == 0 ? prev : next, i);
+  if (i < kD) (wg == 0 ? zprev : unext)[i] = (wg == 0 ? prev : next)[kDM + i];
+  if (wg == 0) gden_s[i] = i < valid ? a.gden[(int64_t)h * a.N + (int64_t)c * kL + i] : 0.f;
   if (ctl_wait(&ctl, 0, 0, a)) {
-    phi_tile(tq, kL, false);
-    phi_tile(tk, kL, false);
+    phi_tile<kFwdThreads>(tq, kL, false);
+    phi_tile<kFwdThreads>(tk, kL, false);
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {  // scores
@@ -797,7 +865,7 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
     }
     if (ctl_wait(&ctl, 1, 0, a)) {
       tc_after_sync();
-      scores_to_tile(ctl.tmem + lane_off, ta, i, 0.f);
+      causal_scores_to_tile(ctl.tmem + lane_off, ta, i, wg);
       tc_before_sync();
       __syncthreads();
       if (threadIdx.x == 0) {  // gnum V^T
@@ -809,7 +877,7 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
       }
       if (ctl_wait(&ctl, 1, 1, a)) {
         tc_after_sync();
-        scores_to_tile(ctl.tmem + lane_off, tpp, i, gden_s[i]);  // P = tril(gnum V^T + gden 1^T)
+        causal_scores_to_tile<true>(ctl.tmem + lane_off, tpp, i, wg, gden_s[i]);  // P = tril(gnum V^T + gden 1^T)
         tc_before_sync();
         fence_proxy_async_smem();
         __syncthreads();
@@ -838,19 +906,25 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
           tc_after_sync();
           float x[32], f[32];
           uint8_t *oq = ta, *ok = ta + kTile, *ov = ta + 2 * kTile;  // the score tiles are no longer read
-          const float gd = gden_s[i];
-          tmem_ld32(ctl.tmem + lane_off, x);
-          get_row64(tq, i, f);
+          // warpgroup 0: dL/dq and dL/dv's columns 0..15; warpgroup 1: dL/dk and columns 16..31
+          tmem_ld32(ctl.tmem + lane_off + 32u * wg, x);
+          get_row64(wg == 0 ? tq : tk, i, f);
+          if (wg == 0) {
+            const float gd = gden_s[i];
 #pragma unroll
-          for (int d = 0; d < kD; ++d) x[d] = fmaf(gd, zprev[d], x[d]) * fminf(f[d], 1.f);
-          put_row64(oq, i, x);
-          tmem_ld32(ctl.tmem + lane_off + 32u, x);
-          get_row64(tk, i, f);
+            for (int d = 0; d < kD; ++d) x[d] = fmaf(gd, zprev[d], x[d]) * fminf(f[d], 1.f);
+          } else {
 #pragma unroll
-          for (int d = 0; d < kD; ++d) x[d] = (x[d] + unext[d]) * fminf(f[d], 1.f);
-          put_row64(ok, i, x);
-          tmem_ld32(ctl.tmem + lane_off + 64u, x);
-          put_row64(ov, i, x);
+            for (int d = 0; d < kD; ++d) x[d] = (x[d] + unext[d]) * fminf(f[d], 1.f);
+          }
+          put_row64(wg == 0 ? oq : ok, i, x);
+          float y[16];
+          tmem_ld16(ctl.tmem + lane_off + 64u + 16u * wg, y);
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+            *reinterpret_cast<uint4 *>(ov + sw64(i, 2 * wg + u)) =
+                make_uint4(pack2(y[8 * u], y[8 * u + 1]), pack2(y[8 * u + 2], y[8 * u + 3]),
+                           pack2(y[8 * u + 4], y[8 * u + 5]), pack2(y[8 * u + 6], y[8 * u + 7]));
           fence_proxy_async_smem();
           __syncthreads();
           if (threadIdx.x == 0) {
@@ -869,8 +943,8 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
 
 // Shared-memory bytes of each kernel (tiles plus the 1 KB alignment slack).
 constexpr int kStateSmem = 6 * kTile + 1024;             // 2 x (K, V), ones, spare rows
-constexpr int kFwdSmem = 12 * kTile + 1024;              // 2 x (Q, K, V), ones, S, Z | scores
-constexpr int kPrepSmem = 8 * kTile + 4 * kTile + 1024;  // Q, gnum, gden, K, V, G, S (+pad) | scores
+constexpr int kFwdSmem = 12 * kTile + 2 * kRecBytes + 1024;  // 2 x (Q, K, V), ones, S, Z | scores | 2 records
+constexpr int kPrepSmem = 13 * kTile + 1024;             // Q, gnum, gden, K, V, G, S, Z (+pad) | scores | ones
 constexpr int kBwdSmem = 13 * kTile + 1024;              // Q, K, V, gnum, S+U (+pad) | A, P
 
 }  // namespace la
@@ -921,13 +995,13 @@ int64_t persistent_grid(K kern, int smem, int tmem_cols, int64_t units) {
       cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) == cudaSuccess &&
       cudaFuncGetAttributes(&fa, (const void *)kern) == cudaSuccess)
     occ = per_sm / (smem + (int)fa.sharedSizeBytes + reserved);
-  occ = std::max(1, std::min(occ, std::min(512 / tmem_cols, 2048 / kThreads)));
+  occ = std::max(1, std::min(occ, std::min(512 / tmem_cols, 2048 / kFwdThreads)));
   return std::min<int64_t>(units, (int64_t)occ * la_num_sms());
 }
 template <typename K>
-int prepare(K kern, int smem) {
+int prepare(K kern, int smem, int threads = kThreads) {
   int occ = 0;
-  return blocks_per_sm((const void *)kern, kThreads, smem, &occ) == cudaSuccess && occ >= 1 ? 0 : -1;
+  return blocks_per_sm((const void *)kern, threads, smem, &occ) == cudaSuccess && occ >= 1 ? 0 : -1;
 }
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? WKV_OK : WKV_ERR_CUDA; }
 int la_num_sms() {
@@ -979,16 +1053,16 @@ extern "C" int linattn_forward(int64_t BH, int64_t N, int D, int M, const void *
     if (!encode_heads_sw64(&qm, q, BH, N, kD) || !encode_heads_sw64(&km, k, BH, N, kD) ||
         !encode_heads_sw64(&vm, v, BH, N, kD) || !encode_heads_sw64(&om, out, BH, N, kD))
       return WKV_ERR_UNSUPPORTED;
-    if (prepare(la_state_kernel, kStateSmem) || prepare(la_fwd_kernel, kFwdSmem)) return WKV_ERR_CUDA;
+    if (prepare(la_state_kernel, kStateSmem, kFwdThreads) || prepare(la_fwd_kernel, kFwdSmem, kFwdThreads)) return WKV_ERR_CUDA;
     cudaError_t e = launch_kernel(la_state_kernel, dim3((unsigned)persistent_grid(la_state_kernel, kStateSmem, 64, units)),
-                                  dim3(kThreads), kStateSmem, st, km, vm, a);
+                                  dim3(kFwdThreads), kStateSmem, st, km, vm, a);
     if (e != cudaSuccess) return WKV_ERR_CUDA;
     const int64_t n = BH * kRec;
     e = launch_kernel(la_scan_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, a.rec, BH, a.nch, 0,
                       state_out);
     if (e != cudaSuccess) return WKV_ERR_CUDA;
     return cuda_rc(launch_kernel(la_fwd_kernel, dim3((unsigned)persistent_grid(la_fwd_kernel, kFwdSmem, 128, units)),
-                                 dim3(kThreads), kFwdSmem, st, qm, km, vm, om, a));
+                                 dim3(kFwdThreads), kFwdSmem, st, qm, km, vm, om, a));
   }
   if (state_out)  // N = 0: the empty state
     return cuda_rc(cudaMemsetAsync(state_out, 0, (size_t)BH * kRec * sizeof(float), st));
@@ -1036,21 +1110,22 @@ extern "C" int linattn_backward(int64_t BH, int64_t N, int D, int M, const void 
       !encode_heads_sw64(&nm, gnum, BH, N, kD) || !encode_heads_sw64(&dqm, grad_q, BH, N, kD) ||
       !encode_heads_sw64(&dkm, grad_k, BH, N, kD) || !encode_heads_sw64(&dvm, grad_v, BH, N, kD))
     return WKV_ERR_UNSUPPORTED;
-  if (prepare(la_state_kernel, kStateSmem) || prepare(la_bwd_prep_kernel, kPrepSmem) ||
-      prepare(la_bwd_kernel, kBwdSmem))
+  if (prepare(la_state_kernel, kStateSmem, kFwdThreads) || prepare(la_bwd_prep_kernel, kPrepSmem, kFwdThreads) ||
+      prepare(la_bwd_kernel, kBwdSmem, kFwdThreads))
     return WKV_ERR_CUDA;
   const int64_t units = BH * a.nch;
   const int64_t n = BH * kRec;
   const dim3 sgrid((unsigned)((n + 255) / 256));
   cudaError_t e = launch_kernel(la_state_kernel, dim3((unsigned)persistent_grid(la_state_kernel, kStateSmem, 64, units)),
-                                dim3(kThreads), kStateSmem, st, km, vm, a);
+                                dim3(kFwdThreads), kStateSmem, st, km, vm, a);
   if (e == cudaSuccess) e = launch_kernel(la_scan_kernel, sgrid, dim3(256), 0, st, a.rec, BH, a.nch, 0, (float *)nullptr);
   if (e == cudaSuccess)
-    e = launch_kernel(la_bwd_prep_kernel, dim3((unsigned)units), dim3(kThreads), kPrepSmem, st, qm, km, vm, gm, nm, a);
+    e = launch_kernel(la_bwd_prep_kernel, dim3((unsigned)units), dim3(kFwdThreads), kPrepSmem, st, qm, km, vm, gm, nm,
+                      a);
   if (e == cudaSuccess)
     e = launch_kernel(la_scan_kernel, sgrid, dim3(256), 0, st, a.rec_r, BH, a.nch, 1, (float *)nullptr);
   if (e == cudaSuccess)
-    e = launch_kernel(la_bwd_kernel, dim3((unsigned)units), dim3(kThreads), kBwdSmem, st, qm, km, vm, nm, dqm, dkm,
+    e = launch_kernel(la_bwd_kernel, dim3((unsigned)units), dim3(kFwdThreads), kBwdSmem, st, qm, km, vm, nm, dqm, dkm,
                       dvm, a);
   return cuda_rc(e);
 }
