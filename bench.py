@@ -82,6 +82,7 @@ KERNEL_SOURCES = {
                        "wkv_math.cuh", "wkv_forward.cu"],
     "fwd_seg_kernel": ["wkv_seg.cu", "wkv_ring.cuh", "wkv_internal.cuh", "wkv_math.cuh", "wkv_forward.cu"],
     "step_kernel": ["wkv_step.cu", "wkv_internal.cuh"],
+    "linattn_backward": ["linattn.cu", "wkv_forward.cu", "wkv_tile.cuh", "wkv_internal.cuh"],
 }
 
 # DRAM bytes (read + write) per launch of a workload's dominant kernel, from
@@ -89,10 +90,15 @@ KERNEL_SOURCES = {
 # (workload, kernel, gated, source hash).  A kernel whose sources changed
 # since its capture has no entry: its traffic is reported as null.
 TRAFFIC = {
-    ("rwkv1b5_bf16", "bwd_tile_kernel", False, "7081082af783b8f4"): 417_490_176 + 294_261_504,
-    ("rwkv1b5_bf16", "fwd_tile_kernel", False, "9336be216ceb647f"): 278_985_472 + 155_384_320,
-    ("longctx", "fwd_seg_kernel", False, "fb83390fdf2b28e1"): 1_578_090_752 + 640_600_320,
+    ("rwkv1b5_bf16", "bwd_tile_kernel", False, "58a8fbacfed79601"): 417_523_200 + 294_170_368,
+    ("rwkv1b5_bf16", "fwd_tile_kernel", False, "0c7dfb9fca3999a0"): 278_965_504 + 155_403_520,
+    ("rwkv169m", "bwd_seg_kernel", False, "48dab62625fb429b"): 77_597_952 + 529_152,
+    ("rwkv169m", "fwd_seg_kernel", False, "4338b6e39aebfeeb"): 50_392_064 + 1_318_400,
+    ("longctx", "fwd_seg_kernel", False, "4338b6e39aebfeeb"): 1_463_432_192 + 639_096_320,
     ("decode14b", "step_kernel", False, "ceedfbaab295393e"): 52_483_344 + 71_440,
+    # the five launches of one linattn_backward call
+    ("la_cifar_b32", "linattn_backward", False, "7744b6f65c330276"): (100_684_800 + 25_963_264 + 227_313_408 + 25_962_752
+                                                             + 256_419_072 + 3_025_408 + 51_338_752 + 96_120_576),
 }
 
 
@@ -987,7 +993,8 @@ def run_linattn(args):
             "config": linattn_config(wl, ws_n),
             "roofline": {"bound": "hbm", "kernel": "linattn_backward call (5 launches), timed as one call",
                          "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s", "frac": bwd_gbs / hbm,
-                         "traffic": None, "algorithmic_bytes": bb, "peak_kind": peak_kind},
+                         "traffic": traffic_for(args.workload, "linattn_backward", False),
+                         "algorithmic_bytes": bb, "peak_kind": peak_kind},
             "fwd": {"ms": fwd_ms, "gbs": fwd_gbs, "frac": fwd_gbs / hbm, "launches": 3,
                     "tensor_tflops_issued": f_chunk * BH * nch / (fwd_ms * 1e-3) / 1e12},
             "bwd": {"ms": bwd_ms, "gbs": bwd_gbs, "frac": bwd_gbs / hbm, "launches": 5,
