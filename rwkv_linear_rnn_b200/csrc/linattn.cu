@@ -58,8 +58,8 @@ constexpr int kRec = kDM + kD;           // floats of one chunk state (S, then Z
 constexpr uint32_t kTile = kL * kD * 2;  // bytes of a [128 x 32] bf16 tile
 constexpr uint32_t kStile = kD * kD * 2; // bytes of a [32 x 32] bf16 tile
 constexpr uint32_t kPhalf = kL * 64 * 2; // bytes of one [128 x 64] half of a score tile
-constexpr int kThreads = 128;
-constexpr int kFwdThreads = 256;  // the persistent kernels: two warpgroups
+constexpr int kWarpgroup = 128;   // threads of one warpgroup: one per tile row
+constexpr int kThreads = 256;     // threads per CTA: two warpgroups
 
 struct LaArgs {
   int64_t BH, N;
@@ -229,8 +229,8 @@ __device__ __forceinline__ void put_row128(uint8_t *t, int r, int b, const float
                    pack2(v[8 * q + 4], v[8 * q + 5]), pack2(v[8 * q + 6], v[8 * q + 7]));
 }
 // A [32 x 32] float32 chunk state (row-major) into a bf16 64-byte-swizzle tile.
-__device__ __forceinline__ void put_state_tile(uint8_t *t, const float *src, int tid = threadIdx.x) {
-  const int d = tid >> 2, u = tid & 3;  // 128 threads
+__device__ __forceinline__ void put_state_tile(uint8_t *t, const float *src, int tid) {
+  const int d = tid >> 2, u = tid & 3;  // one warpgroup: tid in 0..127
   const float4 a = *reinterpret_cast<const float4 *>(src + d * kD + 8 * u);
   const float4 b = *reinterpret_cast<const float4 *>(src + d * kD + 8 * u + 4);
   *reinterpret_cast<uint4 *>(t + sw64(d, u)) = make_uint4(pack2(a.x, a.y), pack2(a.z, a.w), pack2(b.x, b.y),
@@ -297,7 +297,7 @@ __device__ __forceinline__ uint8_t *align1k(uint8_t *p) {
 // complete).  Shared memory: stages (phi(K), V) at 0 and 16K, the ones tile
 // at 32K; the spare rows of stage 1's A operand reach to 48K.
 constexpr uint32_t kSStage = 2 * kTile, kSOnes = 2 * kSStage;
-__global__ void __launch_bounds__(kFwdThreads) la_state_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(kThreads) la_state_kernel(const __grid_constant__ CUtensorMap kmap,
                                                             const __grid_constant__ CUtensorMap vmap, LaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_ld[2], bar_mma;
@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kFwdThreads) la_state_kernel(const __grid_cons
   }
   {
     uint4 *o = reinterpret_cast<uint4 *>(sm + kSOnes);
-    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kFwdThreads)
+    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kThreads)
       o[g] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // bf16 1.0
   }
   tc_before_sync();
@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kFwdThreads) la_state_kernel(const __grid_cons
     const uint32_t ak = s0 + st * kSStage, av = ak + kTile;
     failed = !__syncthreads_and(mbar_wait(smem_addr(&bar_ld[st]), (uint32_t)(it >> 1) & 1u, a.budget_ns, nullptr));
     if (failed) break;
-    phi_tile<kFwdThreads>(sm + st * kSStage, valid, true);
+    phi_tile<kThreads>(sm + st * kSStage, valid, true);
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -441,34 +441,6 @@ __global__ void la_scan_kernel(float *rec, int64_t BH, int nch, int reverse, flo
   }
 }
 
-// Masked scores of the thread's row into a [128 x 128] bf16 tile (4 warps,
-// warp w holding rows 32w..32w+31); returns the row sum (float32, before
-// rounding).  Kept entries get + `add` (the backward's P).  Column blocks
-// left of the warp's diagonal block need no mask, those right of it are
-// zero and their TMEM columns are not read.
-__device__ __forceinline__ float scores_to_tile(uint32_t tm_row, uint8_t *tile, int i, float add) {
-  const int w = i >> 5;
-  float rs = 0.f;
-#pragma unroll 1
-  for (int b = 0; b < 4; ++b) {
-    float v[32];
-    if (b <= w) {
-      tmem_ld32(tm_row + 32u * b, v);
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        const float x = (b < w || 32 * b + r <= i) ? v[r] + add : 0.f;
-        v[r] = x;
-        rs += x;
-      }
-    } else {
-#pragma unroll
-      for (int r = 0; r < 32; ++r) v[r] = 0.f;
-    }
-    put_row128(tile, i, b, v);
-  }
-  return rs;
-}
-
 // Masked scores of the thread's row (its warp holds rows 32w..32w+31) into
 // a [128 x 128] bf16 tile, for two of the four 32-column blocks: warpgroup 0
 // takes blocks 0 and 3, warpgroup 1 blocks 1 and 2 (the causal mask gives
@@ -513,7 +485,7 @@ __device__ __forceinline__ void causal_scores_to_tile(uint32_t tm_row, uint8_t *
 constexpr uint32_t kFStage = 3 * kTile, kFOnes = 2 * kFStage, kFS = kFOnes + kTile, kFZ = kFS + kStile,
                    kFP = 8 * kTile, kFRec = 12 * kTile, kRecBytes = kRec * 4;
 static_assert(kRecBytes % 128 == 0, "records stay 128-byte aligned in shared memory");
-__global__ void __launch_bounds__(kFwdThreads) la_fwd_kernel(const __grid_constant__ CUtensorMap qmap,
+__global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant__ CUtensorMap qmap,
                                                           const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap vmap,
                                                           const __grid_constant__ CUtensorMap omap, LaArgs a) {
@@ -539,7 +511,7 @@ __global__ void __launch_bounds__(kFwdThreads) la_fwd_kernel(const __grid_consta
   }
   {
     uint4 *o = reinterpret_cast<uint4 *>(sm + kFOnes);
-    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kFwdThreads)
+    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kThreads)
       o[g] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // bf16 1.0
   }
   tc_before_sync();
@@ -577,16 +549,16 @@ __global__ void __launch_bounds__(kFwdThreads) la_fwd_kernel(const __grid_consta
     // S_prev and Z_prev of this chunk, from the copy that came with its tiles,
     // as bf16 operand tiles (the previous chunk's MMAs are complete)
     const float *prev = reinterpret_cast<const float *>(sm + kFRec + st * kRecBytes);
-    if (threadIdx.x < kThreads) put_state_tile(sm + kFS, prev);
-    if (threadIdx.x >= kThreads && threadIdx.x < kThreads + kD) {
-      const int d = threadIdx.x - kThreads;
+    if (threadIdx.x < kWarpgroup) put_state_tile(sm + kFS, prev, threadIdx.x);
+    if (threadIdx.x >= kWarpgroup && threadIdx.x < kWarpgroup + kD) {
+      const int d = threadIdx.x - kWarpgroup;
       const uint32_t zz = pack2(prev[kDM + d], prev[kDM + d]);
       const uint4 x = make_uint4(zz, zz, zz, zz);
       uint4 *row = reinterpret_cast<uint4 *>(sm + kFZ + 64 * d);
       row[0] = x, row[1] = x, row[2] = x, row[3] = x;
     }
-    phi_tile<kFwdThreads>(tq, kL, false);
-    phi_tile<kFwdThreads>(tk, kL, false);
+    phi_tile<kThreads>(tq, kL, false);
+    phi_tile<kThreads>(tk, kL, false);
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {  // scores phi(Q) phi(K)^T
@@ -674,7 +646,7 @@ __global__ void __launch_bounds__(kFwdThreads) la_fwd_kernel(const __grid_consta
 // value) 16K, phi(K) 24K, V 32K, G 40K, S_prev 48K, Z_prev 50K, scores 64K
 // (32K bytes), ones 96K.
 constexpr uint32_t kPOnes = 12 * kTile;
-__global__ void __launch_bounds__(kFwdThreads) la_bwd_prep_kernel(const __grid_constant__ CUtensorMap qmap,
+__global__ void __launch_bounds__(kThreads) la_bwd_prep_kernel(const __grid_constant__ CUtensorMap qmap,
                                                                   const __grid_constant__ CUtensorMap kmap,
                                                                   const __grid_constant__ CUtensorMap vmap,
                                                                   const __grid_constant__ CUtensorMap gmap,
@@ -705,7 +677,7 @@ __global__ void __launch_bounds__(kFwdThreads) la_bwd_prep_kernel(const __grid_c
   }
   {
     uint4 *o = reinterpret_cast<uint4 *>(sm + kPOnes);
-    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kFwdThreads)
+    for (int g = threadIdx.x; g < (int)(kTile / 16); g += kThreads)
       o[g] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // bf16 1.0
   }
   const float *prev = a.rec + ((int64_t)h * a.nch + c) * kRec;
@@ -717,8 +689,8 @@ __global__ void __launch_bounds__(kFwdThreads) la_bwd_prep_kernel(const __grid_c
     row[0] = x, row[1] = x, row[2] = x, row[3] = x;
   }
   if (ctl_wait(&ctl, 0, 0, a)) {
-    phi_tile<kFwdThreads>(tq, kL, false);
-    phi_tile<kFwdThreads>(tk, kL, false);
+    phi_tile<kThreads>(tq, kL, false);
+    phi_tile<kThreads>(tk, kL, false);
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -815,7 +787,7 @@ __global__ void __launch_bounds__(kFwdThreads) la_bwd_prep_kernel(const __grid_c
 // V 16K, gnum 24K, S_prev 32K, U_next 34K, masked A 40K, P 72K (32K bytes
 // each); the three output tiles reuse 40K, 48K, 56K at the end.  Two
 // warpgroups: row i = thread % 128, the epilogues' columns split between them.
-__global__ void __launch_bounds__(kFwdThreads) la_bwd_kernel(const __grid_constant__ CUtensorMap qmap,
+__global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant__ CUtensorMap qmap,
                                                           const __grid_constant__ CUtensorMap kmap,
                                                           const __grid_constant__ CUtensorMap vmap,
                                                           const __grid_constant__ CUtensorMap nmap,
@@ -852,8 +824,8 @@ __global__ void __launch_bounds__(kFwdThreads) la_bwd_kernel(const __grid_consta
   if (i < kD) (wg == 0 ? zprev : unext)[i] = (wg == 0 ? prev : next)[kDM + i];
   if (wg == 0) gden_s[i] = i < valid ? a.gden[(int64_t)h * a.N + (int64_t)c * kL + i] : 0.f;
   if (ctl_wait(&ctl, 0, 0, a)) {
-    phi_tile<kFwdThreads>(tq, kL, false);
-    phi_tile<kFwdThreads>(tk, kL, false);
+    phi_tile<kThreads>(tq, kL, false);
+    phi_tile<kThreads>(tk, kL, false);
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {  // scores
@@ -995,7 +967,7 @@ int64_t persistent_grid(K kern, int smem, int tmem_cols, int64_t units) {
       cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) == cudaSuccess &&
       cudaFuncGetAttributes(&fa, (const void *)kern) == cudaSuccess)
     occ = per_sm / (smem + (int)fa.sharedSizeBytes + reserved);
-  occ = std::max(1, std::min(occ, std::min(512 / tmem_cols, 2048 / kFwdThreads)));
+  occ = std::max(1, std::min(occ, std::min(512 / tmem_cols, 2048 / kThreads)));
   return std::min<int64_t>(units, (int64_t)occ * la_num_sms());
 }
 template <typename K>
@@ -1053,16 +1025,16 @@ extern "C" int linattn_forward(int64_t BH, int64_t N, int D, int M, const void *
     if (!encode_heads_sw64(&qm, q, BH, N, kD) || !encode_heads_sw64(&km, k, BH, N, kD) ||
         !encode_heads_sw64(&vm, v, BH, N, kD) || !encode_heads_sw64(&om, out, BH, N, kD))
       return WKV_ERR_UNSUPPORTED;
-    if (prepare(la_state_kernel, kStateSmem, kFwdThreads) || prepare(la_fwd_kernel, kFwdSmem, kFwdThreads)) return WKV_ERR_CUDA;
+    if (prepare(la_state_kernel, kStateSmem, kThreads) || prepare(la_fwd_kernel, kFwdSmem, kThreads)) return WKV_ERR_CUDA;
     cudaError_t e = launch_kernel(la_state_kernel, dim3((unsigned)persistent_grid(la_state_kernel, kStateSmem, 64, units)),
-                                  dim3(kFwdThreads), kStateSmem, st, km, vm, a);
+                                  dim3(kThreads), kStateSmem, st, km, vm, a);
     if (e != cudaSuccess) return WKV_ERR_CUDA;
     const int64_t n = BH * kRec;
     e = launch_kernel(la_scan_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, a.rec, BH, a.nch, 0,
                       state_out);
     if (e != cudaSuccess) return WKV_ERR_CUDA;
     return cuda_rc(launch_kernel(la_fwd_kernel, dim3((unsigned)persistent_grid(la_fwd_kernel, kFwdSmem, 128, units)),
-                                 dim3(kFwdThreads), kFwdSmem, st, qm, km, vm, om, a));
+                                 dim3(kThreads), kFwdSmem, st, qm, km, vm, om, a));
   }
   if (state_out)  // N = 0: the empty state
     return cuda_rc(cudaMemsetAsync(state_out, 0, (size_t)BH * kRec * sizeof(float), st));
@@ -1110,22 +1082,22 @@ extern "C" int linattn_backward(int64_t BH, int64_t N, int D, int M, const void 
       !encode_heads_sw64(&nm, gnum, BH, N, kD) || !encode_heads_sw64(&dqm, grad_q, BH, N, kD) ||
       !encode_heads_sw64(&dkm, grad_k, BH, N, kD) || !encode_heads_sw64(&dvm, grad_v, BH, N, kD))
     return WKV_ERR_UNSUPPORTED;
-  if (prepare(la_state_kernel, kStateSmem, kFwdThreads) || prepare(la_bwd_prep_kernel, kPrepSmem, kFwdThreads) ||
-      prepare(la_bwd_kernel, kBwdSmem, kFwdThreads))
+  if (prepare(la_state_kernel, kStateSmem, kThreads) || prepare(la_bwd_prep_kernel, kPrepSmem, kThreads) ||
+      prepare(la_bwd_kernel, kBwdSmem, kThreads))
     return WKV_ERR_CUDA;
   const int64_t units = BH * a.nch;
   const int64_t n = BH * kRec;
   const dim3 sgrid((unsigned)((n + 255) / 256));
   cudaError_t e = launch_kernel(la_state_kernel, dim3((unsigned)persistent_grid(la_state_kernel, kStateSmem, 64, units)),
-                                dim3(kFwdThreads), kStateSmem, st, km, vm, a);
+                                dim3(kThreads), kStateSmem, st, km, vm, a);
   if (e == cudaSuccess) e = launch_kernel(la_scan_kernel, sgrid, dim3(256), 0, st, a.rec, BH, a.nch, 0, (float *)nullptr);
   if (e == cudaSuccess)
-    e = launch_kernel(la_bwd_prep_kernel, dim3((unsigned)units), dim3(kFwdThreads), kPrepSmem, st, qm, km, vm, gm, nm,
+    e = launch_kernel(la_bwd_prep_kernel, dim3((unsigned)units), dim3(kThreads), kPrepSmem, st, qm, km, vm, gm, nm,
                       a);
   if (e == cudaSuccess)
     e = launch_kernel(la_scan_kernel, sgrid, dim3(256), 0, st, a.rec_r, BH, a.nch, 1, (float *)nullptr);
   if (e == cudaSuccess)
-    e = launch_kernel(la_bwd_kernel, dim3((unsigned)units), dim3(kFwdThreads), kBwdSmem, st, qm, km, vm, nm, dqm, dkm,
+    e = launch_kernel(la_bwd_kernel, dim3((unsigned)units), dim3(kThreads), kBwdSmem, st, qm, km, vm, nm, dqm, dkm,
                       dvm, a);
   return cuda_rc(e);
 }

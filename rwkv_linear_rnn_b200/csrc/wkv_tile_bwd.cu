@@ -50,6 +50,9 @@
 #ifndef WKV_TILEB_LBF16
 #define WKV_TILEB_LBF16 kTileLBF16
 #endif
+#ifndef WKV_TILEB_RB
+#define WKV_TILEB_RB 8
+#endif
 
 namespace wkv {
 
@@ -535,9 +538,9 @@ cudaError_t launch_backward_tile(const BwdArgs &p, int dtype, float *gw, float *
                             p, dtype, gw, gu, rec, chain_sum, num_sms, st)
                       : launch_bwd_tile_t<uint16_t, WKV_TILEB_LBF16, 8, kTileWarps, true, false>(
                             p, dtype, gw, gu, rec, chain_sum, num_sms, st);
-  return dtype == 0 ? launch_bwd_tile_t<float, kTileLF32, 8, kTileWarps, false, false>(
+  return dtype == 0 ? launch_bwd_tile_t<float, kTileLF32, WKV_TILEB_RB, kTileWarps, false, false>(
                           p, dtype, gw, gu, rec, chain_sum, num_sms, st)
-                    : launch_bwd_tile_t<uint16_t, WKV_TILEB_LBF16, 8, kTileWarps, false, false>(
+                    : launch_bwd_tile_t<uint16_t, WKV_TILEB_LBF16, WKV_TILEB_RB, kTileWarps, false, false>(
                           p, dtype, gw, gu, rec, chain_sum, num_sms, st);
 }
 
