@@ -83,6 +83,7 @@ KERNEL_SOURCES = {
     "fwd_seg_kernel": ["wkv_seg.cu", "wkv_ring.cuh", "wkv_internal.cuh", "wkv_math.cuh", "wkv_forward.cu"],
     "step_kernel": ["wkv_step.cu", "wkv_internal.cuh"],
     "linattn_backward": ["linattn.cu", "wkv_forward.cu", "wkv_tile.cuh", "wkv_internal.cuh"],
+    "linattn_backward_saved": ["linattn.cu", "wkv_forward.cu", "wkv_tile.cuh", "wkv_internal.cuh"],
 }
 
 # DRAM bytes (read + write) per launch of a workload's dominant kernel, from
@@ -364,7 +365,7 @@ def run_linattn_reference(args):
             "value": cb["value"], "unit": cb["unit"], "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": wl.BH * wl.N / cb["value"] * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded)", "impl": "reference", "config": linattn_config(wl, 1),
+            "data": "synthetic (seeded)", "impl": "reference", "config": linattn_config(wl, 1, not args.la_recompute),
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": cb["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -872,9 +873,10 @@ LA_FWD_BYTES = 4 * 32 * 2   # q, k, v read, out written (bf16, D = M = 32), per 
 LA_BWD_BYTES = 7 * 32 * 2   # q, k, v, grad_out read, grad_q, grad_k, grad_v written
 
 
-def linattn_config(wl, ws_n):
+def linattn_config(wl, ws_n, saved=True):
     return {"workload": wl.name, "op": "causal linear attention (elu+1)", "BH": wl.BH, "N": wl.N,
             "D": wl.D, "M": wl.D, "io_dtype": "bf16", "note": wl.note,
+            "backward": "from the forward's saved state" if saved else "recomputing the forward",
             "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
             "l2": "flushed before every timed step (2x L2 write + 2x L2 read, outside events)"}
 
@@ -919,9 +921,15 @@ def run_linattn(args):
         abi.check(abi.linattn_forward(BH, N, D, D, P(t["q"]), P(t["k"]), P(t["v"]), P(out), None, P(wsb),
                                       wsb.numel(), sp))
 
+    saved = not args.la_recompute
+
     def bwd():
-        abi.check(abi.linattn_backward(BH, N, D, D, P(t["q"]), P(t["k"]), P(t["v"]), P(t["g"]), P(dq), P(dk),
-                                       P(dv), P(wsb), wsb.numel(), sp))
+        if saved:  # from the state the forward just left in the workspace
+            abi.check(abi.linattn_backward_saved(BH, N, D, D, P(t["q"]), P(t["k"]), P(t["v"]), P(out), P(t["g"]),
+                                                 P(dq), P(dk), P(dv), P(wsb), wsb.numel(), sp))
+        else:
+            abi.check(abi.linattn_backward(BH, N, D, D, P(t["q"]), P(t["k"]), P(t["v"]), P(t["g"]), P(dq), P(dk),
+                                           P(dv), P(wsb), wsb.numel(), sp))
 
     for _ in range(args.warmup):
         flush_l2(); fwd(); bwd()
@@ -981,8 +989,9 @@ def run_linattn(args):
         # tensor-core work issued per 128-position chunk (M = 128 tiles, padding included)
         mf = lambda m, n, k: 2.0 * m * n * k
         f_chunk = mf(128, 128, 32) + mf(128, 32, 128) + mf(128, 32, 32) + mf(128, 48, 128)
-        b_chunk = (mf(128, 48, 128) + mf(128, 128, 32) + mf(128, 32, 128) + mf(128, 32, 32) + mf(128, 48, 128)
-                   + 2 * mf(128, 128, 32) + 3 * (mf(128, 32, 128) + mf(128, 32, 32)))
+        b_recompute = mf(128, 48, 128) + mf(128, 128, 32) + mf(128, 48, 128) + mf(128, 48, 32)  # state, scores, A[V|1], Q[S|Z]
+        b_chunk = (mf(128, 48, 128) + 2 * mf(128, 128, 32) + 3 * (mf(128, 32, 128) + mf(128, 32, 32))
+                   + (0 if saved else b_recompute))
         step_ms = total_ms / K
         line = {
             "metric": "causal linear attention fwd+bwd head-positions/s (HBM GB/s and % of roofline alongside)",
@@ -990,16 +999,19 @@ def run_linattn(args):
             "n_gpus": ws_n, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) q, k, v, grad_out rounded to bf16)",
-            "config": linattn_config(wl, ws_n),
-            "roofline": {"bound": "hbm", "kernel": "linattn_backward call (5 launches), timed as one call",
+            "config": linattn_config(wl, ws_n, saved),
+            "roofline": {"bound": "hbm",
+                         "kernel": ("linattn_backward_saved call (3 launches)" if saved
+                                    else "linattn_backward call (5 launches)") + ", timed as one call",
                          "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s", "frac": bwd_gbs / hbm,
-                         "traffic": traffic_for(args.workload, "linattn_backward", False),
+                         "traffic": traffic_for(args.workload,
+                                                "linattn_backward_saved" if saved else "linattn_backward", False),
                          "algorithmic_bytes": bb, "peak_kind": peak_kind},
             "fwd": {"ms": fwd_ms, "gbs": fwd_gbs, "frac": fwd_gbs / hbm, "launches": 3,
                     "tensor_tflops_issued": f_chunk * BH * nch / (fwd_ms * 1e-3) / 1e12},
-            "bwd": {"ms": bwd_ms, "gbs": bwd_gbs, "frac": bwd_gbs / hbm, "launches": 5,
+            "bwd": {"ms": bwd_ms, "gbs": bwd_gbs, "frac": bwd_gbs / hbm, "launches": 3 if saved else 5,
                     "tensor_tflops_issued": b_chunk * BH * nch / (bwd_ms * 1e-3) / 1e12},
-            "clocks": clocks, "device_status": status, "gpu_launches": 8 * K,
+            "clocks": clocks, "device_status": status, "gpu_launches": (6 if saved else 8) * K,
         }
         if e2e:
             line["e2e"] = e2e
@@ -1026,6 +1038,9 @@ def main():
     ap.add_argument("--bwd-kernel", default="auto", choices=["auto"] + sorted(BWD_PLAN))
     ap.add_argument("--gate", action="store_true",
                     help="time the gated calls (o = sigmoid(r) * wkv and its gradients)")
+    ap.add_argument("--la-recompute", action="store_true",
+                    help="linear attention: time the backward that recomputes the forward instead of the one "
+                         "from the forward's saved state")
     ap.add_argument("--token-shift", action="store_true",
                     help="time the token shift (3 interpolations) on the workload's layer shape")
     args = ap.parse_args()

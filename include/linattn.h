@@ -93,6 +93,23 @@ int linattn_backward(int64_t BH, int64_t N, int D, int M, const void *q, const v
                      const void *grad_out, void *grad_q, void *grad_k, void *grad_v, void *ws, size_t ws_bytes,
                      void *stream);
 
+/*
+ * The same gradients from the forward's saved state (the saved-statistics
+ * form of the backward): `ws` must be the workspace that the linattn_forward
+ * call computing `out` from these q, k, v used, sized
+ * linattn_workspace_size(LINATTN_OP_BACKWARD, ...) (a backward-sized
+ * workspace serves the forward too), with no other call on it since.  That
+ * call left in it each chunk's prefix state and its denominators; this call
+ * reads them instead of recomputing the forward, and needs the forward's
+ * output:
+ *   out       [BH, N, M] bf16, read: linattn_forward's output
+ * Other arguments and return codes as linattn_backward.  Results differ from
+ * linattn_backward's by rounding only (dL/d den uses the bf16 output).
+ */
+int linattn_backward_saved(int64_t BH, int64_t N, int D, int M, const void *q, const void *k, const void *v,
+                           const void *out, const void *grad_out, void *grad_q, void *grad_k, void *grad_v, void *ws,
+                           size_t ws_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

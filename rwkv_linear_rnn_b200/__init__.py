@@ -253,7 +253,9 @@ def linattn_forward(q, k, v, *, want_state=False, out=None, workspace=None, stre
         out = torch.empty((BH, N, M), dtype=torch.bfloat16, device=q.device)
     st = torch.empty(BH * (D * M + D), dtype=torch.float32, device=q.device) if want_state else None
     ws = _ws_for(q.device, workspace)
-    buf, nbytes = ws.get_bytes(linattn_workspace_size(LINATTN_OP_FORWARD, BH, N, D, M))
+    # backward-sized, so that linattn_backward(..., out=out) can reuse the
+    # state this call leaves in the workspace
+    buf, nbytes = ws.get_bytes(linattn_workspace_size(LINATTN_OP_BACKWARD, BH, N, D, M))
     abi = _abi()
     abi.check(abi.linattn_forward(BH, N, D, M, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(st),
                                   _ptr(buf), nbytes, _stream(stream)))
@@ -262,19 +264,29 @@ def linattn_forward(q, k, v, *, want_state=False, out=None, workspace=None, stre
     return out, st
 
 
-def linattn_backward(q, k, v, grad_out, *, grad_q=None, grad_k=None, grad_v=None, workspace=None,
+def linattn_backward(q, k, v, grad_out, *, out=None, grad_q=None, grad_k=None, grad_v=None, workspace=None,
                      stream=None):
-    """Gradients (grad_q, grad_k, grad_v) of L given grad_out = dL/dV'."""
+    """Gradients (grad_q, grad_k, grad_v) of L given grad_out = dL/dV'.
+
+    With ``out`` (the output of the ``linattn_forward`` call on these q, k, v
+    that used the same workspace, with no call on it since), the forward's
+    saved chunk states and denominators are reused instead of recomputed
+    (``linattn_backward_saved``)."""
     torch = _torch()
-    BH, N, D, M = _check_linattn(q, k, v, grad_out, grad_q, grad_k, grad_v)
+    BH, N, D, M = _check_linattn(q, k, v, grad_out, out, grad_q, grad_k, grad_v)
     grad_q = torch.empty_like(q) if grad_q is None else grad_q
     grad_k = torch.empty_like(k) if grad_k is None else grad_k
     grad_v = torch.empty_like(v) if grad_v is None else grad_v
     ws = _ws_for(q.device, workspace)
     buf, nbytes = ws.get_bytes(linattn_workspace_size(LINATTN_OP_BACKWARD, BH, N, D, M))
     abi = _abi()
-    abi.check(abi.linattn_backward(BH, N, D, M, _ptr(q), _ptr(k), _ptr(v), _ptr(grad_out), _ptr(grad_q),
-                                   _ptr(grad_k), _ptr(grad_v), _ptr(buf), nbytes, _stream(stream)))
+    if out is not None:
+        abi.check(abi.linattn_backward_saved(BH, N, D, M, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(grad_out),
+                                             _ptr(grad_q), _ptr(grad_k), _ptr(grad_v), _ptr(buf), nbytes,
+                                             _stream(stream)))
+    else:
+        abi.check(abi.linattn_backward(BH, N, D, M, _ptr(q), _ptr(k), _ptr(v), _ptr(grad_out), _ptr(grad_q),
+                                       _ptr(grad_k), _ptr(grad_v), _ptr(buf), nbytes, _stream(stream)))
     return grad_q, grad_k, grad_v
 
 

@@ -26,7 +26,7 @@ EXPORTS = (
     "wkv_step", "wkv_backward_static", "wkv_backward_static_status", "wkv_get_status",
     "wkv_strerror", "wkv_last_cuda_error", "wkv_cuda_error_name", "wkv_version",
     # include/linattn.h
-    "linattn_workspace_size", "linattn_forward", "linattn_backward",
+    "linattn_workspace_size", "linattn_forward", "linattn_backward", "linattn_backward_saved",
 )
 
 
@@ -77,6 +77,7 @@ _SIGS = {
     "linattn_workspace_size": (_sz, [_int, _i64, _i64, _int, _int]),
     "linattn_forward": (_int, [_i64, _i64, _int, _int, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "linattn_backward": (_int, [_i64, _i64, _int, _int] + [_p] * 7 + [_p, _sz, _p]),
+    "linattn_backward_saved": (_int, [_i64, _i64, _int, _int] + [_p] * 8 + [_p, _sz, _p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -233,6 +234,11 @@ def linattn_forward(BH, N, D, M, q, k, v, out, state_out, ws, ws_bytes, stream):
 def linattn_backward(BH, N, D, M, q, k, v, grad_out, grad_q, grad_k, grad_v, ws, ws_bytes, stream):
     return lib.linattn_backward(BH, N, D, M, q, k, v, grad_out, grad_q, grad_k, grad_v, ws, ws_bytes,
                                 stream)
+
+
+def linattn_backward_saved(BH, N, D, M, q, k, v, out, grad_out, grad_q, grad_k, grad_v, ws, ws_bytes, stream):
+    return lib.linattn_backward_saved(BH, N, D, M, q, k, v, out, grad_out, grad_q, grad_k, grad_v, ws, ws_bytes,
+                                      stream)
 
 
 def check(rc: int) -> None:

@@ -67,6 +67,7 @@ struct LaArgs {
   float *rec;       // [BH][nch][kRec]: chunk states, then their exclusive prefix
   float *rec_r;     // [BH][nch][kRec]: reverse chunk states, then exclusive suffix
   float *gden;      // [BH][N]
+  float *den;       // [BH][nch * 128]: the forward's denominators (kept for a saved-state backward)
   WsHeader *hdr;
   int64_t budget_ns;
 };
@@ -604,7 +605,9 @@ __global__ void __launch_bounds__(kThreads) la_fwd_kernel(const __grid_constant_
     tc_after_sync();
     float o[16];  // this warpgroup's 16 of the 32 output columns
     tmem_ld16(tm + lane_off + 16u * wg, o);
-    const float inv = 1.f / tmem_ld1(tm + lane_off + 32u);
+    const float den = tmem_ld1(tm + lane_off + 32u);
+    const float inv = 1.f / den;
+    if (wg == 0) a.den[((int64_t)h * a.nch + c) * kL + i] = den;
 #pragma unroll
     for (int u = 0; u < 2; ++u)  // phi(K) is no longer read: the output goes there
       *reinterpret_cast<uint4 *>(tk + sw64(i, 2 * wg + u)) =
@@ -783,6 +786,104 @@ __global__ void __launch_bounds__(kThreads) la_bwd_prep_kernel(const __grid_cons
   ctl_finish(&ctl, 128, a);
 }
 
+// Backward, first part, from the forward's saved state: the forward's
+// output and denominators give gnum = G / den (bf16, to the workspace) and
+// gden = -rowsum(G * out) / den (float32, to the workspace) directly, and
+// one MMA chain the chunk's reverse state phi(Q)^T [gnum | gden].  Shared
+// memory: phi(Q) 0, gnum 8K, gden (rows filled with their value) 16K, G 24K
+// (also the spare rows of the MMA's A operand), out 32K, den 40K.
+__global__ void __launch_bounds__(kThreads) la_bwd_prep_saved_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                     const __grid_constant__ CUtensorMap gmap,
+                                                                     const __grid_constant__ CUtensorMap omap,
+                                                                     const __grid_constant__ CUtensorMap nmap,
+                                                                     LaArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ Ctl ctl;
+  __shared__ float gpart[kL];  // warpgroup 1's part of rowsum(G * out)
+  uint8_t *sm = align1k(smem_raw);
+  const uint32_t s0 = smem_addr(sm);
+  uint8_t *tq = sm, *tn = sm + kTile, *tg_den = sm + 2 * kTile, *tgo = sm + 3 * kTile, *tout = sm + 4 * kTile;
+  const float *dens = reinterpret_cast<const float *>(sm + 5 * kTile);
+  const uint32_t aq = s0, an = s0 + kTile;
+  const int h = (int)(blockIdx.x / a.nch), c = (int)(blockIdx.x % a.nch);
+  const int i = threadIdx.x & 127, wg = threadIdx.x >> 7;
+  const int64_t rem = a.N - (int64_t)c * kL;
+  const int valid = rem < kL ? (int)rem : kL;
+  ctl_setup(&ctl, 64);
+  const uint32_t bl = smem_addr(&ctl.bar[0]), bm = smem_addr(&ctl.bar[1]);
+  if (threadIdx.x == 0) {
+    const uint64_t pol = l2_policy_evict_first();
+    mbar_expect_tx(bl, 3 * kTile + kL * 4);
+    tma_load_3d(aq, &qmap, 0, c * kL, h, bl, l2_policy_evict_last());  // read again by the gradient kernel
+    tma_load_3d(s0 + 3 * kTile, &gmap, 0, c * kL, h, bl, pol);
+    tma_load_3d(s0 + 4 * kTile, &omap, 0, c * kL, h, bl, pol);
+    bulk_load(s0 + 5 * kTile, a.den + ((int64_t)h * a.nch + c) * kL, kL * 4, bl);
+  }
+  if (ctl_wait(&ctl, 0, 0, a)) {
+    phi_tile<kThreads>(tq, kL, false);
+    float g[16], o[16];  // this warpgroup's 16 columns of G and out
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const uint4 x = *reinterpret_cast<const uint4 *>(tgo + sw64(i, 2 * wg + u));
+      const uint4 y = *reinterpret_cast<const uint4 *>(tout + sw64(i, 2 * wg + u));
+      g[8 * u + 0] = lo16(x.x), g[8 * u + 1] = hi16(x.x), g[8 * u + 2] = lo16(x.y), g[8 * u + 3] = hi16(x.y);
+      g[8 * u + 4] = lo16(x.z), g[8 * u + 5] = hi16(x.z), g[8 * u + 6] = lo16(x.w), g[8 * u + 7] = hi16(x.w);
+      o[8 * u + 0] = lo16(y.x), o[8 * u + 1] = hi16(y.x), o[8 * u + 2] = lo16(y.y), o[8 * u + 3] = hi16(y.y);
+      o[8 * u + 4] = lo16(y.z), o[8 * u + 5] = hi16(y.z), o[8 * u + 6] = lo16(y.w), o[8 * u + 7] = hi16(y.w);
+    }
+    const float inv = 1.f / dens[i];
+    float go = 0.f;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      go = fmaf(g[m], o[m], go);
+      g[m] *= inv;  // gnum
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      *reinterpret_cast<uint4 *>(tn + sw64(i, 2 * wg + u)) =
+          make_uint4(pack2(g[8 * u], g[8 * u + 1]), pack2(g[8 * u + 2], g[8 * u + 3]),
+                     pack2(g[8 * u + 4], g[8 * u + 5]), pack2(g[8 * u + 6], g[8 * u + 7]));
+    if (wg == 1) gpart[i] = go;
+    __syncthreads();
+    if (wg == 0) {
+      const float gden = -(go + gpart[i]) * inv;
+      const uint32_t w = pack2(gden, gden);
+      const uint4 x = make_uint4(w, w, w, w);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4 *>(tg_den + 64 * i + 16 * u) = x;
+      if (i < valid) a.gden[(int64_t)h * a.N + (int64_t)c * kL + i] = gden;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tma_store_3d(&nmap, 0, c * kL, h, an);
+      bulk_commit();
+      // reverse state phi(Q)^T [gnum | gden]: M = 128 over the tiles at
+      // 0, 8K, 16K, 24K (rows 32..127 unused), N = 48 over gnum, gden
+      tc_after_sync();
+      constexpr uint32_t id3 = idesc(128, 48, true, true);
+#pragma unroll
+      for (int k16 = 0; k16 < kL / 16; ++k16) mma(ctl.tmem, mnmaj64(aq, k16, kTile), mnmaj64(an, k16, kTile), id3, k16 > 0);
+      mma_commit(bm);
+    }
+    if (ctl_wait(&ctl, 1, 0, a)) {
+      tc_after_sync();
+      if (threadIdx.x < 32) {
+        float rv[32];
+        tmem_ld32(ctl.tmem, rv);
+        const float uz = tmem_ld1(ctl.tmem + 32u);
+        float *r = a.rec_r + ((int64_t)h * a.nch + c) * kRec;
+        float4 *row = reinterpret_cast<float4 *>(r + threadIdx.x * kD);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) row[q] = make_float4(rv[4 * q], rv[4 * q + 1], rv[4 * q + 2], rv[4 * q + 3]);
+        r[kDM + threadIdx.x] = uz;
+      }
+    }
+    if (threadIdx.x == 0) bulk_wait_all();
+  }
+  ctl_finish(&ctl, 64, a);
+}
+
 // Backward, gradients of one chunk.  Shared memory: phi(Q) 0, phi(K) 8K,
 // V 16K, gnum 24K, S_prev 32K, U_next 34K, masked A 40K, P 72K (32K bytes
 // each); the three output tiles reuse 40K, 48K, 56K at the end.  Two
@@ -918,6 +1019,7 @@ constexpr int kStateSmem = 6 * kTile + 1024;             // 2 x (K, V), ones, sp
 constexpr int kFwdSmem = 12 * kTile + 2 * kRecBytes + 1024;  // 2 x (Q, K, V), ones, S, Z | scores | 2 records
 constexpr int kPrepSmem = 13 * kTile + 1024;             // Q, gnum, gden, K, V, G, S, Z (+pad) | scores | ones
 constexpr int kBwdSmem = 13 * kTile + 1024;              // Q, K, V, gnum, S+U (+pad) | A, P
+constexpr int kPrepSavedSmem = 5 * kTile + kL * 4 + 1024;  // Q, gnum, gden, G, out, den
 
 }  // namespace la
 }  // namespace wkv
@@ -928,7 +1030,7 @@ using namespace wkv;
 using namespace wkv::la;
 
 struct LaLayout {
-  size_t rec, rec_r, gnum, gden, total;
+  size_t rec, den, rec_r, gnum, gden, total;
 };
 bool la_layout(int op, int64_t BH, int64_t N, LaLayout *L) {
   if (BH < 1 || N < 0 || BH > (int64_t(1) << 31) || N > (int64_t(1) << 31) || BH * N >= (int64_t(1) << 31))
@@ -936,8 +1038,13 @@ bool la_layout(int op, int64_t BH, int64_t N, LaLayout *L) {
   const int64_t nch = (N + kL - 1) / kL;
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   size_t off = 256;  // header
+  // The forward's regions come first and sit at the same offsets in both
+  // layouts, so a backward-sized workspace can carry the forward's state
+  // into linattn_backward_saved.
   L->rec = off;
   off = up(off + (size_t)BH * nch * kRec * 4);
+  L->den = off;
+  off = up(off + (size_t)BH * nch * kL * 4);
   L->rec_r = L->gnum = L->gden = 0;
   if (op == LINATTN_OP_BACKWARD) {
     L->rec_r = off;
@@ -1017,6 +1124,7 @@ extern "C" int linattn_forward(int64_t BH, int64_t N, int D, int M, const void *
   a.N = N;
   a.nch = (int)((N + kL - 1) / kL);
   a.rec = reinterpret_cast<float *>(base + L.rec);
+  a.den = reinterpret_cast<float *>(base + L.den);
   a.hdr = reinterpret_cast<WsHeader *>(base);
   a.budget_ns = kBudgetNs;
   const int64_t units = BH * a.nch;
@@ -1096,6 +1204,64 @@ extern "C" int linattn_backward(int64_t BH, int64_t N, int D, int M, const void 
                       a);
   if (e == cudaSuccess)
     e = launch_kernel(la_scan_kernel, sgrid, dim3(256), 0, st, a.rec_r, BH, a.nch, 1, (float *)nullptr);
+  if (e == cudaSuccess)
+    e = launch_kernel(la_bwd_kernel, dim3((unsigned)units), dim3(kThreads), kBwdSmem, st, qm, km, vm, nm, dqm, dkm,
+                      dvm, a);
+  return cuda_rc(e);
+}
+
+extern "C" int linattn_backward_saved(int64_t BH, int64_t N, int D, int M, const void *q, const void *k,
+                                      const void *v, const void *out, const void *grad_out, void *grad_q,
+                                      void *grad_k, void *grad_v, void *ws, size_t ws_bytes, void *stream) {
+  LaLayout L;
+  const void *ins[5] = {q, k, v, out, grad_out};
+  const void *outs[3] = {grad_q, grad_k, grad_v};
+  if (N != 0) {  // empty tensors may be null
+    for (const void *p : ins)
+      if (!p) return WKV_ERR_INVALID_ARG;
+    for (const void *o : outs) {
+      if (!o) return WKV_ERR_INVALID_ARG;
+      for (const void *in : ins)
+        if (o == in) return WKV_ERR_INVALID_ARG;
+    }
+    if (grad_q == grad_k || grad_q == grad_v || grad_k == grad_v) return WKV_ERR_INVALID_ARG;
+  }
+  const int rc = check_common(BH, N, D, M, ws, ws_bytes, LINATTN_OP_BACKWARD, &L);
+  if (rc != WKV_OK) return rc;
+  for (const void *p : ins)
+    if (!aligned16(p)) return WKV_ERR_UNSUPPORTED;
+  for (const void *p : outs)
+    if (!aligned16(p)) return WKV_ERR_UNSUPPORTED;
+  if (N == 0) return WKV_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  LaArgs a{};
+  a.BH = BH;
+  a.N = N;
+  a.nch = (int)((N + kL - 1) / kL);
+  a.rec = reinterpret_cast<float *>(base + L.rec);  // the forward's chunk prefixes
+  a.den = reinterpret_cast<float *>(base + L.den);  // and its denominators
+  a.rec_r = reinterpret_cast<float *>(base + L.rec_r);
+  a.gden = reinterpret_cast<float *>(base + L.gden);
+  a.hdr = reinterpret_cast<WsHeader *>(base);
+  a.budget_ns = kBudgetNs;
+  void *gnum = base + L.gnum;
+  CUtensorMap qm, km, vm, om, gm, nm, dqm, dkm, dvm;
+  if (!encode_heads_sw64(&qm, q, BH, N, kD) || !encode_heads_sw64(&km, k, BH, N, kD) ||
+      !encode_heads_sw64(&vm, v, BH, N, kD) || !encode_heads_sw64(&om, out, BH, N, kD) ||
+      !encode_heads_sw64(&gm, grad_out, BH, N, kD) || !encode_heads_sw64(&nm, gnum, BH, N, kD) ||
+      !encode_heads_sw64(&dqm, grad_q, BH, N, kD) || !encode_heads_sw64(&dkm, grad_k, BH, N, kD) ||
+      !encode_heads_sw64(&dvm, grad_v, BH, N, kD))
+    return WKV_ERR_UNSUPPORTED;
+  if (prepare(la_bwd_prep_saved_kernel, kPrepSavedSmem, kThreads) || prepare(la_bwd_kernel, kBwdSmem, kThreads))
+    return WKV_ERR_CUDA;
+  const int64_t units = BH * a.nch;
+  const int64_t n = BH * kRec;
+  cudaError_t e = launch_kernel(la_bwd_prep_saved_kernel, dim3((unsigned)units), dim3(kThreads), kPrepSavedSmem, st,
+                                qm, gm, om, nm, a);
+  if (e == cudaSuccess)
+    e = launch_kernel(la_scan_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, a.rec_r, BH, a.nch, 1,
+                      (float *)nullptr);
   if (e == cudaSuccess)
     e = launch_kernel(la_bwd_kernel, dim3((unsigned)units), dim3(kThreads), kBwdSmem, st, qm, km, vm, nm, dqm, dkm,
                       dvm, a);

@@ -253,3 +253,17 @@ def test_linattn_sizes_and_argument_checks(W):
     assert abi.linattn_backward(1, 8, 32, 32, F, F * 2, F * 3, F * 4, F, F * 6, F * 7, ws, big, 0) == -1  # grad_q is q
     assert abi.linattn_backward(1, 8, 16, 16, *bargs[4:]) == -2            # head size
     assert abi.linattn_backward(*bargs[:11], ws, 16, 0) == -3              # workspace too small
+
+
+def test_linattn_backward_saved_argument_checks(W):
+    abi = W.abi
+    F = FAKE
+    ws = 1 << 24
+    big = 1 << 30
+    # (BH, N, D, M, q, k, v, out, grad_out, grad_q, grad_k, grad_v, ws, ws_bytes, stream)
+    ok = (1, 8, 32, 32, F, F * 2, F * 3, F * 4, F * 5, F * 6, F * 7, F * 8, ws, big, 0)
+    assert abi.linattn_backward_saved(*ok[:7], 0, *ok[8:]) == -1                  # out NULL
+    assert abi.linattn_backward_saved(*ok[:9], F, *ok[10:]) == -1                 # grad_q is q
+    assert abi.linattn_backward_saved(1, 8, 64, 64, *ok[4:]) == -2                # head size
+    assert abi.linattn_backward_saved(*ok[:12], ws, 16, 0) == -3                  # workspace too small
+    assert abi.linattn_backward_saved(*ok[:4], F + 2, *ok[5:]) == -2              # q misaligned

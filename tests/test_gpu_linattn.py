@@ -154,3 +154,45 @@ def test_outputs_stay_inside_their_buffers():
     for b in bufs:
         assert torch.all(b[:guard] == 7.0) and torch.all(b[guard + n:] == 7.0)
     assert fwd_err(host(out), la.fwd_recur(inp["q"], inp["k"], inp["v"])[0]) <= BF16_TOL
+
+
+def check_backward_saved(inp, heads=None):
+    """The backward from the forward's saved state: forward, then the
+    gradients with its output, on one workspace."""
+    q, k, v, g = on_device(inp)
+    ws = W.Workspace()
+    out, _ = W.linattn_forward(q, k, v, workspace=ws)
+    got = W.linattn_backward(q, k, v, g, out=out, workspace=ws)
+    sel = slice(None) if heads is None else heads
+    ref = la.bwd_recur(inp["q"][sel], inp["k"][sel], inp["v"][sel], inp["g"][sel])
+    for name, a, b in zip(("gq", "gk", "gv"), got, ref):
+        x = host(a)[sel]
+        if np.linalg.norm(b) <= 1e-9 * np.sqrt(b.size):
+            assert np.max(np.abs(x)) <= BF16_TOL, (name, np.max(np.abs(x)))
+            continue
+        assert rel_l2(x, b) <= BF16_TOL, (name, rel_l2(x, b))
+    return got
+
+
+@pytest.mark.parametrize("BH,N", [(1, 1), (2, 5), (1, 128), (3, 129), (2, 300), (1, 1000)])
+def test_backward_saved_small_and_ragged(BH, N):
+    check_backward_saved(case(BH, N, seed=11 * BH + N))
+
+
+@pytest.mark.parametrize("name", ["la_mnist", "la_cifar"])
+def test_backward_saved_workloads(name):
+    check_backward_saved(workloads.generate_linattn(name))
+
+
+def test_backward_saved_agrees_with_recompute():
+    """The saved-state backward and the recomputing one differ by rounding
+    only: the reused state is the forward's own, and dL/d(den) takes the
+    bf16 output instead of the float32 one."""
+    inp = case(4, 700, seed=21)
+    q, k, v, g = on_device(inp)
+    ws = W.Workspace()
+    out, _ = W.linattn_forward(q, k, v, workspace=ws)
+    saved = W.linattn_backward(q, k, v, g, out=out, workspace=ws)
+    recomputed = W.linattn_backward(q, k, v, g, workspace=W.Workspace())
+    for a, b in zip(saved, recomputed):
+        assert rel_l2(host(a), host(b)) <= 5e-3
