@@ -909,7 +909,7 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
   const int64_t rem = a.N - (int64_t)c * kL;
   const int valid = rem < kL ? (int)rem : kL;
   const uint32_t lane_off = (uint32_t)(i & ~31) << 16;
-  ctl_setup(&ctl, 128);
+  ctl_setup(&ctl, 256);
   const uint32_t bl = smem_addr(&ctl.bar[0]), bm = smem_addr(&ctl.bar[1]);
   if (threadIdx.x == 0) {
     const uint64_t pol = l2_policy_evict_first();
@@ -929,28 +929,21 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
     phi_tile<kThreads>(tk, kL, false);
     fence_proxy_async_smem();
     __syncthreads();
-    if (threadIdx.x == 0) {  // scores
+    if (threadIdx.x == 0) {  // scores into columns 0..127, gnum V^T into 128..255
       tc_after_sync();
       constexpr uint32_t id = idesc(128, 128, false, false);
       mma(ctl.tmem, kmaj64(aq, 0), kmaj64(ak, 0), id, false);
       mma(ctl.tmem, kmaj64(aq, 1), kmaj64(ak, 1), id, true);
+      mma(ctl.tmem + 128u, kmaj64(an, 0), kmaj64(av, 0), id, false);
+      mma(ctl.tmem + 128u, kmaj64(an, 1), kmaj64(av, 1), id, true);
       mma_commit(bm);
     }
     if (ctl_wait(&ctl, 1, 0, a)) {
       tc_after_sync();
       causal_scores_to_tile(ctl.tmem + lane_off, ta, i, wg);
-      tc_before_sync();
-      __syncthreads();
-      if (threadIdx.x == 0) {  // gnum V^T
-        tc_after_sync();
-        constexpr uint32_t id = idesc(128, 128, false, false);
-        mma(ctl.tmem, kmaj64(an, 0), kmaj64(av, 0), id, false);
-        mma(ctl.tmem, kmaj64(an, 1), kmaj64(av, 1), id, true);
-        mma_commit(bm);
-      }
-      if (ctl_wait(&ctl, 1, 1, a)) {
-        tc_after_sync();
-        causal_scores_to_tile<true>(ctl.tmem + lane_off, tpp, i, wg, gden_s[i]);  // P = tril(gnum V^T + gden 1^T)
+      // P = tril(gnum V^T + gden 1^T)
+      causal_scores_to_tile<true>(ctl.tmem + 128u + lane_off, tpp, i, wg, gden_s[i]);
+      {
         tc_before_sync();
         fence_proxy_async_smem();
         __syncthreads();
@@ -975,7 +968,7 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
           mma(ctl.tmem + 64u, kmaj64(ak, 1), mnmaj64(au, 1, kTile), kmn, true);
           mma_commit(bm);
         }
-        if (ctl_wait(&ctl, 1, 0, a)) {
+        if (ctl_wait(&ctl, 1, 1, a)) {
           tc_after_sync();
           float x[32], f[32];
           uint8_t *oq = ta, *ok = ta + kTile, *ov = ta + 2 * kTile;  // the score tiles are no longer read
@@ -1011,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
       }
     }
   }
-  ctl_finish(&ctl, 128, a);
+  ctl_finish(&ctl, 256, a);
 }
 
 // Shared-memory bytes of each kernel (tiles plus the 1 KB alignment slack).
