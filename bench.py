@@ -91,15 +91,15 @@ KERNEL_SOURCES = {
 # (workload, kernel, gated, source hash).  A kernel whose sources changed
 # since its capture has no entry: its traffic is reported as null.
 TRAFFIC = {
-    ("rwkv1b5_bf16", "bwd_tile_kernel", False, "58a8fbacfed79601"): 417_523_200 + 294_170_368,
+    ("rwkv1b5_bf16", "bwd_tile_kernel", False, "f96009b55fb50d0e"): 417_612_800 + 294_274_048,
     ("rwkv1b5_bf16", "fwd_tile_kernel", False, "0c7dfb9fca3999a0"): 278_965_504 + 155_403_520,
     ("rwkv169m", "bwd_seg_kernel", False, "48dab62625fb429b"): 77_597_952 + 529_152,
     ("rwkv169m", "fwd_seg_kernel", False, "4338b6e39aebfeeb"): 50_392_064 + 1_318_400,
     ("longctx", "fwd_seg_kernel", False, "4338b6e39aebfeeb"): 1_463_432_192 + 639_096_320,
     ("decode14b", "step_kernel", False, "ceedfbaab295393e"): 52_483_344 + 71_440,
-    # the five launches of one linattn_backward call
-    ("la_cifar_b32", "linattn_backward", False, "7744b6f65c330276"): (100_684_800 + 25_963_264 + 227_313_408 + 25_962_752
-                                                             + 256_419_072 + 3_025_408 + 51_338_752 + 96_120_576),
+    # the three launches of one linattn_backward_saved call
+    ("la_cifar_b32", "linattn_backward_saved", False, "f2e6951884305da9"): (154_164_736 + 25_962_752 + 256_558_336
+                                                                           + 28_006_144 + 96_240_640),
 }
 
 
