@@ -32,6 +32,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -88,26 +89,35 @@ KERNEL_SOURCES = {
 
 # DRAM bytes (read + write) per launch of a workload's dominant kernel, from
 # one ncu capture (the summaries under profiles/ give the commands), keyed by
-# (workload, kernel, gated, source hash).  A kernel whose sources changed
+# (workload, kernel, gated, hash of the kernel's code).  A kernel whose code changed
 # since its capture has no entry: its traffic is reported as null.
 TRAFFIC = {
-    ("rwkv1b5_bf16", "bwd_tile_kernel", False, "f96009b55fb50d0e"): 417_612_800 + 294_274_048,
-    ("rwkv1b5_bf16", "fwd_tile_kernel", False, "0c7dfb9fca3999a0"): 278_965_504 + 155_403_520,
-    ("rwkv169m", "bwd_seg_kernel", False, "48dab62625fb429b"): 77_597_952 + 529_152,
-    ("rwkv169m", "fwd_seg_kernel", False, "4338b6e39aebfeeb"): 50_392_064 + 1_318_400,
-    ("longctx", "fwd_seg_kernel", False, "4338b6e39aebfeeb"): 1_463_432_192 + 639_096_320,
-    ("decode14b", "step_kernel", False, "ceedfbaab295393e"): 52_483_344 + 71_440,
+    ("rwkv1b5_bf16", "bwd_tile_kernel", False, "b8cbf6bf4c53f50a"): 417_612_800 + 294_274_048,
+    ("rwkv1b5_bf16", "fwd_tile_kernel", False, "bc53deb1657ced5a"): 278_965_504 + 155_403_520,
+    ("rwkv169m", "bwd_seg_kernel", False, "c5e242ca4e035480"): 77_597_952 + 529_152,
+    ("rwkv169m", "fwd_seg_kernel", False, "1edb76594a20115c"): 50_392_064 + 1_318_400,
+    ("longctx", "fwd_seg_kernel", False, "1edb76594a20115c"): 1_463_432_192 + 639_096_320,
+    ("decode14b", "step_kernel", False, "21aab8ba04a9606b"): 52_483_344 + 71_440,
     # the three launches of one linattn_backward_saved call
-    ("la_cifar_b32", "linattn_backward_saved", False, "f2e6951884305da9"): (154_164_736 + 25_962_752 + 256_558_336
+    ("la_cifar_b32", "linattn_backward_saved", False, "b21fed1a36c98a9a"): (154_164_736 + 25_962_752 + 256_558_336
                                                                            + 28_006_144 + 96_240_640),
 }
 
 
+def _code_only(text: str) -> str:
+    """Source without comments and blank lines: what the compiler sees
+    (string literals in these files hold no comment markers)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_hash(kernel: str) -> str:
+    """Hash of the code (comments excluded) of the files a kernel is built from."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES.get(kernel, []):
-        with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(CSRC, f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

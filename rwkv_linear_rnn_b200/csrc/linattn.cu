@@ -478,7 +478,8 @@ __device__ __forceinline__ void causal_scores_to_tile(uint32_t tm_row, uint8_t *
 // while the one before it is computed.  Per chunk: scores phi(Q) phi(K)^T
 // (2 MMAs), the masked score tile, then numerators and denominator in one
 // accumulator, A [V | 1] + phi(Q) [S_prev | Z_prev] (10 MMAs, N = 48:
-// column 32 is the denominator), and out = numerators / denominator.
+// column 32 is the denominator), and out = numerators / denominator; each
+// row's denominator also goes to the workspace for the saved-state backward.
 // Shared memory: two stages of (phi(Q), phi(K) then the output tile, V) at
 // 0 and 24K, a ones tile at 48K, S_prev and Z_prev (bf16) at 56K and 58K,
 // the score tile at 64K (32K bytes), and per stage the chunk's float32
