@@ -72,7 +72,7 @@
 extern "C" {
 #endif
 
-#define WKV_VERSION 120 /* 1.2.0: tile kernels, wkv_backward_static_status */
+#define WKV_VERSION 130 /* 1.3.0: causal linear attention (linattn.h) */
 
 /* Element type of the [B, T, C] tensors. */
 typedef enum { WKV_F32 = 0, WKV_BF16 = 1 } wkv_dtype;

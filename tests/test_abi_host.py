@@ -46,7 +46,7 @@ def test_every_declared_symbol_is_exported(W):
 
 
 def test_version_and_strerror(W):
-    assert W.wkv_version() == 120
+    assert W.wkv_version() == 130
     for code in range(0, -6, -1):
         assert W.wkv_strerror(code) != "unknown status"
     assert W.wkv_strerror(7) == "unknown status"
