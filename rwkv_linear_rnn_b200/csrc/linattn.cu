@@ -885,32 +885,35 @@ __global__ void __launch_bounds__(kThreads) la_bwd_prep_saved_kernel(const __gri
   ctl_finish(&ctl, 64, a);
 }
 
-// Backward, gradients of one chunk.  Shared memory: phi(Q) 0, phi(K) 8K,
-// V 16K, gnum 24K, S_prev 32K, U_next 34K, masked A 40K, P 72K (32K bytes
-// each); the three output tiles reuse 40K, 48K, 56K at the end.  Two
-// warpgroups: row i = thread % 128, the epilogues' columns split between them.
-__global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant__ CUtensorMap qmap,
-                                                          const __grid_constant__ CUtensorMap kmap,
-                                                          const __grid_constant__ CUtensorMap vmap,
-                                                          const __grid_constant__ CUtensorMap nmap,
-                                                          const __grid_constant__ CUtensorMap dqmap,
-                                                          const __grid_constant__ CUtensorMap dkmap,
-                                                          const __grid_constant__ CUtensorMap dvmap, LaArgs a) {
+// Backward, gradients of one chunk.  One score tile and 128 tensor-memory
+// columns, so that three CTAs fit per SM (registers capped to match): the
+// masked A feeds A^T gnum first, whose result waits in registers, and is
+// then overwritten by P = tril(gnum V^T + gden 1^T).  Two warpgroups: row
+// i = thread % 128, the epilogues' columns split between them.  Shared
+// memory: phi(Q) 0, phi(K) 8K, V 16K, gnum 24K, S_prev 32K, U_next 34K, the
+// score tile 36K (32K bytes); the output tiles reuse 36K, 44K, 52K.
+__global__ void __launch_bounds__(kThreads, 3) la_bwd_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                           const __grid_constant__ CUtensorMap kmap,
+                                                           const __grid_constant__ CUtensorMap vmap,
+                                                           const __grid_constant__ CUtensorMap nmap,
+                                                           const __grid_constant__ CUtensorMap dqmap,
+                                                           const __grid_constant__ CUtensorMap dkmap,
+                                                           const __grid_constant__ CUtensorMap dvmap, LaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ Ctl ctl;
   __shared__ float zprev[kD], unext[kD], gden_s[kL];
   uint8_t *sm = align1k(smem_raw);
   const uint32_t s0 = smem_addr(sm);
-  uint8_t *tq = sm, *tk = sm + kTile, *ts = sm + 4 * kTile, *tu = sm + 4 * kTile + kStile, *ta = sm + 5 * kTile,
-          *tpp = sm + 9 * kTile;
+  constexpr uint32_t kT = 4 * kTile + 2 * kStile;  // the score tile (1024-aligned)
+  uint8_t *tq = sm, *tk = sm + kTile, *ts = sm + 4 * kTile, *tu = sm + 4 * kTile + kStile, *tt = sm + kT;
   const uint32_t aq = s0, ak = s0 + kTile, av = s0 + 2 * kTile, an = s0 + 3 * kTile, as = s0 + 4 * kTile,
-                 au = s0 + 4 * kTile + kStile, aa = s0 + 5 * kTile, app = s0 + 9 * kTile;
+                 au = s0 + 4 * kTile + kStile, at = s0 + kT;
   const int h = (int)(blockIdx.x / a.nch), c = (int)(blockIdx.x % a.nch);
   const int i = threadIdx.x & 127, wg = threadIdx.x >> 7;
   const int64_t rem = a.N - (int64_t)c * kL;
   const int valid = rem < kL ? (int)rem : kL;
   const uint32_t lane_off = (uint32_t)(i & ~31) << 16;
-  ctl_setup(&ctl, 256);
+  ctl_setup(&ctl, 128);
   const uint32_t bl = smem_addr(&ctl.bar[0]), bm = smem_addr(&ctl.bar[1]);
   if (threadIdx.x == 0) {
     const uint64_t pol = l2_policy_evict_first();
@@ -930,95 +933,116 @@ __global__ void __launch_bounds__(kThreads) la_bwd_kernel(const __grid_constant_
     phi_tile<kThreads>(tk, kL, false);
     fence_proxy_async_smem();
     __syncthreads();
-    if (threadIdx.x == 0) {  // scores into columns 0..127, gnum V^T into 128..255
+    constexpr uint32_t sq = idesc(128, 128, false, false), kk = idesc(128, 32, false, false),
+                       kmn = idesc(128, 32, false, true), mnmn = idesc(128, 32, true, true);
+    if (threadIdx.x == 0) {  // scores
       tc_after_sync();
-      constexpr uint32_t id = idesc(128, 128, false, false);
-      mma(ctl.tmem, kmaj64(aq, 0), kmaj64(ak, 0), id, false);
-      mma(ctl.tmem, kmaj64(aq, 1), kmaj64(ak, 1), id, true);
-      mma(ctl.tmem + 128u, kmaj64(an, 0), kmaj64(av, 0), id, false);
-      mma(ctl.tmem + 128u, kmaj64(an, 1), kmaj64(av, 1), id, true);
+      mma(ctl.tmem, kmaj64(aq, 0), kmaj64(ak, 0), sq, false);
+      mma(ctl.tmem, kmaj64(aq, 1), kmaj64(ak, 1), sq, true);
       mma_commit(bm);
     }
     if (ctl_wait(&ctl, 1, 0, a)) {
       tc_after_sync();
-      causal_scores_to_tile(ctl.tmem + lane_off, ta, i, wg);
-      // P = tril(gnum V^T + gden 1^T)
-      causal_scores_to_tile<true>(ctl.tmem + 128u + lane_off, tpp, i, wg, gden_s[i]);
-      {
+      causal_scores_to_tile(ctl.tmem + lane_off, tt, i, wg);  // A
+      tc_before_sync();
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (threadIdx.x == 0) {  // A^T gnum, dL/dV's first part, into columns 0..31
+        tc_after_sync();
+#pragma unroll
+        for (int k16 = 0; k16 < kL / 16; ++k16)
+          mma(ctl.tmem, mnmaj128(at, k16), mnmaj64(an, k16, kTile), mnmn, k16 > 0);
+        mma_commit(bm);
+      }
+      if (ctl_wait(&ctl, 1, 1, a)) {
+        tc_after_sync();
+        float dv1[16];  // this warpgroup's 16 columns, kept until the end
+        tmem_ld16(ctl.tmem + lane_off + 16u * wg, dv1);
         tc_before_sync();
-        fence_proxy_async_smem();
         __syncthreads();
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0) {  // gnum V^T
           tc_after_sync();
-          constexpr uint32_t kk = idesc(128, 32, false, false), kmn = idesc(128, 32, false, true),
-                             mnmn = idesc(128, 32, true, true);
-          // dphi(Q) -> columns 0..31: P phi(K) + gnum S_prev^T
-#pragma unroll
-          for (int s = 0; s < kL / 16; ++s) mma(ctl.tmem, kmaj128(app, s), mnmaj64(ak, s, kTile), kmn, s > 0);
-          mma(ctl.tmem, kmaj64(an, 0), kmaj64(as, 0), kk, true);
-          mma(ctl.tmem, kmaj64(an, 1), kmaj64(as, 1), kk, true);
-          // dphi(K) -> columns 32..63: P^T phi(Q) + V U_next^T
-#pragma unroll
-          for (int s = 0; s < kL / 16; ++s) mma(ctl.tmem + 32u, mnmaj128(app, s), mnmaj64(aq, s, kTile), mnmn, s > 0);
-          mma(ctl.tmem + 32u, kmaj64(av, 0), kmaj64(au, 0), kk, true);
-          mma(ctl.tmem + 32u, kmaj64(av, 1), kmaj64(au, 1), kk, true);
-          // dV -> columns 64..95: A^T gnum + phi(K) U_next
-#pragma unroll
-          for (int s = 0; s < kL / 16; ++s) mma(ctl.tmem + 64u, mnmaj128(aa, s), mnmaj64(an, s, kTile), mnmn, s > 0);
-          mma(ctl.tmem + 64u, kmaj64(ak, 0), mnmaj64(au, 0, kTile), kmn, true);
-          mma(ctl.tmem + 64u, kmaj64(ak, 1), mnmaj64(au, 1, kTile), kmn, true);
+          mma(ctl.tmem, kmaj64(an, 0), kmaj64(av, 0), sq, false);
+          mma(ctl.tmem, kmaj64(an, 1), kmaj64(av, 1), sq, true);
           mma_commit(bm);
         }
-        if (ctl_wait(&ctl, 1, 1, a)) {
+        if (ctl_wait(&ctl, 1, 0, a)) {
           tc_after_sync();
-          float x[32], f[32];
-          uint8_t *oq = ta, *ok = ta + kTile, *ov = ta + 2 * kTile;  // the score tiles are no longer read
-          // warpgroup 0: dL/dq and dL/dv's columns 0..15; warpgroup 1: dL/dk and columns 16..31
-          tmem_ld32(ctl.tmem + lane_off + 32u * wg, x);
-          get_row64(wg == 0 ? tq : tk, i, f);
-          if (wg == 0) {
-            const float gd = gden_s[i];
-#pragma unroll
-            for (int d = 0; d < kD; ++d) x[d] = fmaf(gd, zprev[d], x[d]) * fminf(f[d], 1.f);
-          } else {
-#pragma unroll
-            for (int d = 0; d < kD; ++d) x[d] = (x[d] + unext[d]) * fminf(f[d], 1.f);
-          }
-          put_row64(wg == 0 ? oq : ok, i, x);
-          float y[16];
-          tmem_ld16(ctl.tmem + lane_off + 64u + 16u * wg, y);
-#pragma unroll
-          for (int u = 0; u < 2; ++u)
-            *reinterpret_cast<uint4 *>(ov + sw64(i, 2 * wg + u)) =
-                make_uint4(pack2(y[8 * u], y[8 * u + 1]), pack2(y[8 * u + 2], y[8 * u + 3]),
-                           pack2(y[8 * u + 4], y[8 * u + 5]), pack2(y[8 * u + 6], y[8 * u + 7]));
+          causal_scores_to_tile<true>(ctl.tmem + lane_off, tt, i, wg, gden_s[i]);  // P over A
+          tc_before_sync();
           fence_proxy_async_smem();
           __syncthreads();
           if (threadIdx.x == 0) {
-            tma_store_3d(&dqmap, 0, c * kL, h, aa);
-            tma_store_3d(&dkmap, 0, c * kL, h, aa + kTile);
-            tma_store_3d(&dvmap, 0, c * kL, h, aa + 2 * kTile);
-            bulk_commit();
-            bulk_wait_all();
+            tc_after_sync();
+            // dphi(Q) -> columns 0..31: P phi(K) + gnum S_prev^T
+#pragma unroll
+            for (int k16 = 0; k16 < kL / 16; ++k16) mma(ctl.tmem, kmaj128(at, k16), mnmaj64(ak, k16, kTile), kmn, k16 > 0);
+            mma(ctl.tmem, kmaj64(an, 0), kmaj64(as, 0), kk, true);
+            mma(ctl.tmem, kmaj64(an, 1), kmaj64(as, 1), kk, true);
+            // dphi(K) -> columns 32..63: P^T phi(Q) + V U_next^T
+#pragma unroll
+            for (int k16 = 0; k16 < kL / 16; ++k16)
+              mma(ctl.tmem + 32u, mnmaj128(at, k16), mnmaj64(aq, k16, kTile), mnmn, k16 > 0);
+            mma(ctl.tmem + 32u, kmaj64(av, 0), kmaj64(au, 0), kk, true);
+            mma(ctl.tmem + 32u, kmaj64(av, 1), kmaj64(au, 1), kk, true);
+            // dL/dV's second part -> columns 64..95: phi(K) U_next
+            mma(ctl.tmem + 64u, kmaj64(ak, 0), mnmaj64(au, 0, kTile), kmn, false);
+            mma(ctl.tmem + 64u, kmaj64(ak, 1), mnmaj64(au, 1, kTile), kmn, true);
+            mma_commit(bm);
+          }
+          if (ctl_wait(&ctl, 1, 1, a)) {
+            tc_after_sync();
+            float x[32], f[32];
+            uint8_t *oq = tt, *ok = tt + kTile, *ov = tt + 2 * kTile;  // the score tile is no longer read
+            tmem_ld32(ctl.tmem + lane_off + 32u * wg, x);
+            get_row64(wg == 0 ? tq : tk, i, f);
+            if (wg == 0) {
+              const float gd = gden_s[i];
+#pragma unroll
+              for (int d = 0; d < kD; ++d) x[d] = fmaf(gd, zprev[d], x[d]) * fminf(f[d], 1.f);
+            } else {
+#pragma unroll
+              for (int d = 0; d < kD; ++d) x[d] = (x[d] + unext[d]) * fminf(f[d], 1.f);
+            }
+            put_row64(wg == 0 ? oq : ok, i, x);
+            float y[16];
+            tmem_ld16(ctl.tmem + lane_off + 64u + 16u * wg, y);
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+              *reinterpret_cast<uint4 *>(ov + sw64(i, 2 * wg + u)) = make_uint4(
+                  pack2(y[8 * u] + dv1[8 * u], y[8 * u + 1] + dv1[8 * u + 1]),
+                  pack2(y[8 * u + 2] + dv1[8 * u + 2], y[8 * u + 3] + dv1[8 * u + 3]),
+                  pack2(y[8 * u + 4] + dv1[8 * u + 4], y[8 * u + 5] + dv1[8 * u + 5]),
+                  pack2(y[8 * u + 6] + dv1[8 * u + 6], y[8 * u + 7] + dv1[8 * u + 7]));
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (threadIdx.x == 0) {
+              tma_store_3d(&dqmap, 0, c * kL, h, at);
+              tma_store_3d(&dkmap, 0, c * kL, h, at + kTile);
+              tma_store_3d(&dvmap, 0, c * kL, h, at + 2 * kTile);
+              bulk_commit();
+              bulk_wait_all();
+            }
           }
         }
       }
     }
   }
-  ctl_finish(&ctl, 256, a);
+  ctl_finish(&ctl, 128, a);
 }
 
 // Shared-memory bytes of each kernel (tiles plus the 1 KB alignment slack).
 constexpr int kStateSmem = 6 * kTile + 1024;             // 2 x (K, V), ones, spare rows
 constexpr int kFwdSmem = 12 * kTile + 2 * kRecBytes + 1024;  // 2 x (Q, K, V), ones, S, Z | scores | 2 records
 constexpr int kPrepSmem = 13 * kTile + 1024;             // Q, gnum, gden, K, V, G, S, Z (+pad) | scores | ones
-constexpr int kBwdSmem = 13 * kTile + 1024;              // Q, K, V, gnum, S+U (+pad) | A, P
+constexpr int kBwdSmem = 8 * kTile + 2 * kStile + 1024;     // Q, K, V, gnum, S, U | one score tile
 constexpr int kPrepSavedSmem = 5 * kTile + kL * 4 + 1024;  // Q, gnum, gden, G, out, den
 
 }  // namespace la
 }  // namespace wkv
 
 // ---------------------------------------------------------------- host ---
+
 namespace {
 using namespace wkv;
 using namespace wkv::la;
