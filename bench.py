@@ -99,8 +99,8 @@ TRAFFIC = {
     ("longctx", "fwd_seg_kernel", False, "1edb76594a20115c"): 1_463_432_192 + 639_096_320,
     ("decode14b", "step_kernel", False, "21aab8ba04a9606b"): 52_483_344 + 71_440,
     # the three launches of one linattn_backward_saved call
-    ("la_cifar_b32", "linattn_backward_saved", False, "b21fed1a36c98a9a"): (154_164_736 + 25_962_752 + 256_558_336
-                                                                           + 28_006_144 + 96_240_640),
+    ("la_cifar_b32", "linattn_backward_saved", False, "af5c298cf6a97dd3"): (154_172_672 + 25_963_008 + 256_456_704
+                                                                           + 27_880_448 + 107_828_224),
 }
 
 
