@@ -59,19 +59,25 @@ ALG_BYTES = {("fwd", "f32"): 12, ("fwd", "bf16"): 6, ("bwd", "f32"): 20, ("bwd",
 # Kernels each call launches on 16-byte aligned rows (every bench workload):
 # (kernel name, launches per call) per kernel selector.  The gated and
 # state-gradient backwards run the segment kernel.
-FWD_PLAN = {"tile": ("fwd_tile_kernel", 1), "segment": ("fwd_seg_kernel", 1), "cluster": ("fwd_clu_kernel", 1)}
-BWD_PLAN = {"tile": ("bwd_tile_kernel", 1), "segment": ("bwd_seg_kernel", 1)}
+FWD_PLAN = {"tile": ("fwd_tile_kernel", 1), "segment": ("fwd_seg_kernel", 1), "cluster": ("fwd_clu_kernel", 1),
+            "chain": ("fwd_chain_kernel", 1)}
+BWD_PLAN = {"tile": ("bwd_tile_kernel", 1), "segment": ("bwd_seg_kernel", 1), "chain": ("bwd_chain_kernel", 1)}
 
 
 def auto_kernel(op: str, B: int, C: int, gate: bool, num_sms: int = 148) -> str:
     """The kernel the library's AUTO selector runs on 16-byte aligned rows of
-    at least one tile unit: the tile kernels when a chain (batch row, 32
-    channels) has at most about four resident warps' units in flight, the
-    segment kernels otherwise (mirrors tile_pays in the C ABI)."""
+    at least one tile unit (mirrors chain_pays and tile_pays in the C ABI):
+    the chain kernels when the chains (batch row, 32 channels) fill three
+    quarters or more of the warp schedulers in one wave (the gated backward
+    excepted); else the tile kernels when a chain has at most about four
+    resident warps' units in flight; else the segment kernels."""
     nchains = B * ((C + 31) // 32)
+    slots = 4 * num_sms
+    if nchains * 4 >= slots * 3 and nchains <= slots and not (gate and op == "bwd"):
+        return "chain"
     warps = (6 if gate else 9) if op == "fwd" else (6 if gate else 8)
     return "tile" if nchains * 4 >= warps * num_sms else "segment"
-KERNEL_IDS = {"auto": 0, "segment": 6, "cluster": 7, "tile": 8}
+KERNEL_IDS = {"auto": 0, "segment": 6, "cluster": 7, "tile": 8, "chain": 9}
 
 # The source files each kernel is built from: a DRAM-traffic figure measured
 # by ncu is reported only while these files are unchanged since the capture.
@@ -82,6 +88,9 @@ KERNEL_SOURCES = {
     "bwd_seg_kernel": ["wkv_seg_bwd.cu", "wkv_ring.cuh", "wkv_bwd_math.cuh", "wkv_internal.cuh",
                        "wkv_math.cuh", "wkv_forward.cu"],
     "fwd_seg_kernel": ["wkv_seg.cu", "wkv_ring.cuh", "wkv_internal.cuh", "wkv_math.cuh", "wkv_forward.cu"],
+    "fwd_chain_kernel": ["wkv_chain.cu", "wkv_tile.cuh", "wkv_internal.cuh", "wkv_math.cuh", "wkv_forward.cu"],
+    "bwd_chain_kernel": ["wkv_chain.cu", "wkv_tile.cuh", "wkv_bwd_math.cuh", "wkv_internal.cuh", "wkv_math.cuh",
+                         "wkv_forward.cu"],
     "step_kernel": ["wkv_step.cu", "wkv_internal.cuh"],
     "linattn_backward": ["linattn.cu", "wkv_forward.cu", "wkv_tile.cuh", "wkv_internal.cuh"],
     "linattn_backward_saved": ["linattn.cu", "wkv_forward.cu", "wkv_tile.cuh", "wkv_internal.cuh"],

@@ -93,7 +93,8 @@ enum { WKV_OP_FORWARD = 0, WKV_OP_BACKWARD = 1, WKV_OP_STEP = 2 };
 /* Kernel selector (wkv_options.kernel). */
 enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
        WKV_KERNEL_CHUNKED_REGS = 3, /* 4 and 5 are retired */
-       WKV_KERNEL_SEGMENT = 6, WKV_KERNEL_CLUSTER = 7, WKV_KERNEL_TILE = 8 };
+       WKV_KERNEL_SEGMENT = 6, WKV_KERNEL_CLUSTER = 7, WKV_KERNEL_TILE = 8,
+       WKV_KERNEL_CHAIN = 9 };
 
 /*
  * Optional knobs for the *_ex calls.  A NULL options pointer, or all fields
@@ -120,7 +121,14 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
  *               stay in shared memory between the unit's two passes, joins
  *               units by a decoupled look-back over records that carry their
  *               own validity tags (no fences), and, in the forward, runs the
- *               next unit's first pass before the current unit's join.  AUTO
+ *               next unit's first pass before the current unit's join.
+ *               CHAIN (16-byte aligned rows; the backward without the gate
+ *               and the state terms) gives each warp whole chains, run in
+ *               time order from a ring of TMA tiles with the state (or the
+ *               adjoint) carried in registers: no joins and a single pass
+ *               over every token, for problems whose chains alone fill the
+ *               GPU's warp schedulers; where it does not apply, the call
+ *               runs TILE (SEGMENT for the gate and state terms).  AUTO
  *               runs TILE on 16-byte aligned rows when a chain (batch row, 32
  *               channels) has at most about four resident warps' units in
  *               flight, SEGMENT otherwise, and the chunked kernels on

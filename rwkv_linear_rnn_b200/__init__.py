@@ -19,14 +19,14 @@ from __future__ import annotations
 import importlib
 
 from .constants import (WKV_BF16, WKV_F32, WKV_KERNEL_AUTO, WKV_KERNEL_CHUNKED,
-                        WKV_KERNEL_CLUSTER, WKV_KERNEL_SEGMENT, WKV_KERNEL_TILE,
+                        WKV_KERNEL_CLUSTER, WKV_KERNEL_SEGMENT, WKV_KERNEL_TILE, WKV_KERNEL_CHAIN,
                         WKV_KERNEL_CHUNKED_REGS, WKV_KERNEL_SEQUENTIAL, WKV_OP_BACKWARD,
                         WKV_OP_FORWARD, WKV_OP_STEP, WKV_STATIC_SCRATCH_BYTES)
 
 __all__ = [
     "abi", "WKVError", "WKV_F32", "WKV_BF16", "WKV_OP_FORWARD", "WKV_OP_BACKWARD", "WKV_OP_STEP",
     "WKV_KERNEL_AUTO", "WKV_KERNEL_SEQUENTIAL", "WKV_KERNEL_CHUNKED", "WKV_KERNEL_CHUNKED_REGS",
-    "WKV_KERNEL_SEGMENT", "WKV_KERNEL_CLUSTER", "WKV_KERNEL_TILE", "WKV_STATIC_SCRATCH_BYTES", "Workspace", "forward", "backward", "backward_state", "step", "token_shift",
+    "WKV_KERNEL_SEGMENT", "WKV_KERNEL_CLUSTER", "WKV_KERNEL_TILE", "WKV_KERNEL_CHAIN", "WKV_STATIC_SCRATCH_BYTES", "Workspace", "forward", "backward", "backward_state", "step", "token_shift",
     "token_shift_backward", "TokenShift",
     "forward_gated", "backward_gated", "WKV", "wkv", "WKVState", "wkv_state", "GatedWKV", "gated_wkv", "wkv_workspace_size", "wkv_ckpt_size", "wkv_strerror", "wkv_version",
     "library_path", "LINATTN_OP_FORWARD", "LINATTN_OP_BACKWARD", "linattn_workspace_size",

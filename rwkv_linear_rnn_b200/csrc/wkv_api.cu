@@ -35,6 +35,9 @@ int64_t fwd_chunk_tokens();
 cudaError_t launch_forward_tile(const FwdArgs &f, float4 *rec, int dtype, int num_sms, cudaStream_t st);
 cudaError_t launch_backward_tile(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *rec, float4 *chain_sum,
                                  int num_sms, cudaStream_t st);
+cudaError_t launch_forward_chain(const FwdArgs &f, int dtype, cudaStream_t st);
+cudaError_t launch_backward_chain(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *chain_sum, int num_sms,
+                                  cudaStream_t st);
 }  // namespace wkv
 
 using namespace wkv;
@@ -142,11 +145,20 @@ int num_sms() {
 // amortise their joins better.  warps_per_sm: resident warps of the kernel.
 bool tile_pays(int64_t nchains, int warps_per_sm) { return nchains * 4 >= (int64_t)warps_per_sm * num_sms(); }
 
+// AUTO picks the chain kernels when the chains alone come close to filling
+// the warp schedulers (four per SM, one chain each) in one wave: from three
+// quarters of them up.  With fewer, the idle schedulers cost more than the
+// time-parallel kernels' joins.
+bool chain_pays(int64_t nchains) {
+  const int64_t slots = 4 * (int64_t)num_sms();
+  return nchains * 4 >= slots * 3 && nchains <= slots;
+}
+
 bool pick_chunked(const wkv_options *opt, int64_t B, int64_t T, int64_t C) {
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   if (kernel == WKV_KERNEL_SEQUENTIAL) return false;
   if (kernel == WKV_KERNEL_CHUNKED || kernel == WKV_KERNEL_CHUNKED_REGS || kernel == WKV_KERNEL_SEGMENT ||
-      kernel == WKV_KERNEL_CLUSTER || kernel == WKV_KERNEL_TILE)
+      kernel == WKV_KERNEL_CLUSTER || kernel == WKV_KERNEL_TILE || kernel == WKV_KERNEL_CHAIN)
     return true;
   // Enough independent chains to fill the GPU, or too short to split.
   return !(B * C >= kSeqMinChains || T <= 2 * fwd_chunk_tokens());
@@ -157,7 +169,7 @@ bool options_ok(const wkv_options *opt) {
   const int k = opt->kernel;
   return k == WKV_KERNEL_AUTO || k == WKV_KERNEL_SEQUENTIAL || k == WKV_KERNEL_CHUNKED ||
          k == WKV_KERNEL_CHUNKED_REGS || k == WKV_KERNEL_SEGMENT || k == WKV_KERNEL_CLUSTER ||
-         k == WKV_KERNEL_TILE;
+         k == WKV_KERNEL_TILE || k == WKV_KERNEL_CHAIN;
 }
 
 int64_t spin_of(const wkv_options *opt) {
@@ -216,13 +228,21 @@ int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
   a.hold_first = opt ? opt->test_hold_first_chunk : 0;
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   const bool tma = chunked && fwd_tma_eligible(a, dtype);
+  // chain forward: whole chains per warp, y (and r) loaded and stored by TMA
+  if (tma && (kernel == WKV_KERNEL_CHAIN || (kernel == WKV_KERNEL_AUTO && chain_pays(L.nchains))) &&
+      aligned(y, 16) && aligned(r, 16)) {
+    a.r = r;
+    return cuda_rc(launch_forward_chain(a, dtype, st));
+  }
   // tile forward: whole units of tokens, y (and r) loaded and stored by TMA
-  if (tma && (kernel == WKV_KERNEL_TILE || (kernel == WKV_KERNEL_AUTO && tile_pays(L.nchains, r ? 6 : 9))) &&
+  if (tma && (kernel == WKV_KERNEL_TILE || kernel == WKV_KERNEL_CHAIN ||
+              (kernel == WKV_KERNEL_AUTO && tile_pays(L.nchains, r ? 6 : 9))) &&
       T >= tile_fwd_tokens(dtype) && aligned(y, 16) && aligned(r, 16)) {
     a.r = r;
     return cuda_rc(launch_forward_tile(a, reinterpret_cast<float4 *>(base + L.rec), dtype, num_sms(), st));
   }
-  const bool seg = tma && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT || kernel == WKV_KERNEL_TILE);
+  const bool seg = tma && (kernel == WKV_KERNEL_AUTO || kernel == WKV_KERNEL_SEGMENT || kernel == WKV_KERNEL_TILE ||
+                           kernel == WKV_KERNEL_CHAIN);
   if (seg && (!r || aligned(r, 16))) {
     a.r = r;  // fused gate
     return cuda_rc(launch_forward_seg(a, dtype, num_sms(), st));
@@ -246,7 +266,9 @@ int forward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, con
 bool bwd_uses_seg(int64_t B, int64_t T, int64_t C, int dtype, const void *k, const void *v, const void *gy,
                   const wkv_options *opt) {
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
-  if (kernel != WKV_KERNEL_AUTO && kernel != WKV_KERNEL_SEGMENT && kernel != WKV_KERNEL_TILE) return false;
+  if (kernel != WKV_KERNEL_AUTO && kernel != WKV_KERNEL_SEGMENT && kernel != WKV_KERNEL_TILE &&
+      kernel != WKV_KERNEL_CHAIN)
+    return false;
   FwdArgs probe{};
   probe.B = B; probe.T = T; probe.C = C; probe.k = k; probe.v = v;
   return fwd_tma_eligible(probe, dtype) && aligned(gy, 16);
@@ -327,8 +349,16 @@ int backward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, co
   a.gs_in = sg.gs_in;
   a.state_in = state_in;
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
+  const bool bwd_tma = bwd_uses_seg(B, T, C, dtype, k, v, grad_y, nullptr) && aligned(grad_k, 16) &&
+                       aligned(grad_v, 16);
+  if (!r && !sg.gs_out && !sg.gs_in && bwd_tma &&
+      (kernel == WKV_KERNEL_CHAIN || (kernel == WKV_KERNEL_AUTO && chain_pays(L.nchains)))) {
+    float4 *sums = reinterpret_cast<float4 *>(base + L.sums);
+    return cuda_rc(launch_backward_chain(a, dtype, grad_w, grad_u, sums, num_sms(), st));
+  }
   if ((!r || (aligned(r, 16) && aligned(gr, 16))) &&
-      (kernel == WKV_KERNEL_TILE || (kernel == WKV_KERNEL_AUTO && tile_pays(L.nchains, r ? 6 : 8))) &&
+      (kernel == WKV_KERNEL_TILE || kernel == WKV_KERNEL_CHAIN ||
+       (kernel == WKV_KERNEL_AUTO && tile_pays(L.nchains, r ? 6 : 8))) &&
       T >= tile_fwd_tokens(dtype) && bwd_uses_seg(B, T, C, dtype, k, v, grad_y, nullptr) && aligned(grad_k, 16) &&
       aligned(grad_v, 16)) {
     // the per-chain sums of dL/dw, dL/du use the descriptor region (16 bytes

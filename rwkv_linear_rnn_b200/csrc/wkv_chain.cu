@@ -1,0 +1,803 @@
+// wkv_chain.cu -- chain kernels of libwkv: one warp runs one chain (batch
+// row b, 32 channels = the 32 lanes) through all of its tokens in order.
+//
+// The operator is eq. wkv_t of the RWKV paper review ("[논문 리뷰] Reinvention
+// RNNs for the Transformer Era: RWKV", section "WKV 연산자"), run in the RNN
+// form of section "RNN-유사추론" over the max-rescaled state; the gradient
+// is back-propagation through that recurrence, taken backwards in time as
+// in the linear attention post ("Transformers are RNNs: 선형 어텐션으로
+// 만드는 빠른 자기회귀 트랜스포머", section "상수 메모리 기울기 계산").
+//
+// When a problem has about as many chains as the GPU has warp schedulers,
+// splitting the time axis buys nothing: every scheduler already has a chain
+// to run, and the joins of a time-parallel scan (summaries, look-backs, a
+// second pass over every token) more than double the instructions per token.
+// Here a chain's state, or its adjoint, is carried from one unit of L tokens
+// to the next in registers.  Per warp, S tile buffers form a TMA ring that
+// keeps S units of input in flight ahead of the arithmetic, and the outputs
+// leave through two staging buffers by TMA stores, so the copy engine, not
+// the warp, moves every byte.  Blocks hold four warps (one per scheduler of
+// an SM) and nothing else is resident beside them.
+//
+// Forward, per unit: the recurrence over the unit's tokens, in batches of
+// RB tokens on the batch fast path of wkv_math.cuh where the warp allows it;
+// y, the checkpoints every 32 tokens and the final state are written.
+// Backward, per unit, units last to first: the forward state at every batch
+// start (from the checkpoints, and by advancing a batch where a checkpoint
+// does not fall on it), then batches last to first: recompute, reverse
+// sweep of the adjoint, dL/dk and dL/dv.  dL/dw and dL/du are summed per
+// chain (per unit in float, across units in float64), and the chain of the
+// last batch row of each channel tile adds the B chains in batch-row order:
+// the result is bit-reproducible.
+#include <cuda.h>
+
+#include "wkv_bwd_math.cuh"
+#include "wkv_internal.cuh"
+#include "wkv_math.cuh"
+#include "wkv_tile.cuh"
+
+// Tokens per batch of the fast paths (build-time knobs).
+#ifndef WKV_CHAIN_FRB
+#define WKV_CHAIN_FRB 32
+#endif
+#ifndef WKV_CHAIN_BRB
+#define WKV_CHAIN_BRB 16
+#endif
+
+namespace wkv {
+
+bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T, int64_t C, int box_t);
+
+constexpr int kChainWarps = 4;  // warps per block: one per scheduler
+constexpr int kChainStages = 4;  // units of input in flight per warp
+
+// Largest and smallest of n values as balanced trees: log2(n) dependent
+// steps instead of n (with one warp per scheduler, dependent chains are
+// what the arithmetic waits on).  Max and min are exact, so the order does
+// not change the result.
+template <int N>
+__device__ __forceinline__ void tree_minmax(const float (&x)[N], float &mx, float &mn) {
+  static_assert((N & (N - 1)) == 0, "power of two");
+  float a[N / 2], b[N / 2];
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    a[i] = fmaxf(x[2 * i], x[2 * i + 1]);
+    b[i] = fminf(x[2 * i], x[2 * i + 1]);
+  }
+#pragma unroll
+  for (int s = N / 4; s >= 1; s /= 2) {
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      a[i] = fmaxf(a[i], a[i + s]);
+      b[i] = fminf(b[i], b[i + s]);
+    }
+  }
+  mx = a[0];
+  mn = b[0];
+}
+
+// fast_prep of wkv_math.cuh with the reductions as trees (same results).
+template <int RB>
+__device__ __forceinline__ bool fast_prep_tree(const float (&K)[RB], float E0, float u2, float w2e, float (&kj)[RB],
+                                               float &M) {
+#pragma unroll
+  for (int j = 0; j < RB; ++j) kj[j] = fmaf(-(float)j, w2e, K[j]);
+  float mx, mn;
+  tree_minmax<RB>(kj, mx, mn);
+  mx = fmaxf(E0, mx);
+  mn = fminf(3.0e38f, mn);
+  M = mx;
+  return (mx - mn < 100.f) && (mx - mn - u2 < 64.f) && (u2 < 64.f);
+}
+
+// Round two floats to the element type and store them (bf16: one packed
+// conversion for both, to nearest even).
+template <typename E>
+__device__ __forceinline__ void store2(E *p0, E *p1, float x0, float x1);
+template <>
+__device__ __forceinline__ void store2<float>(float *p0, float *p1, float x0, float x1) {
+  *p0 = x0;
+  *p1 = x1;
+}
+template <>
+__device__ __forceinline__ void store2<uint16_t>(uint16_t *p0, uint16_t *p1, float x0, float x1) {
+  unsigned u;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(x1), "f"(x0));  // x1 to the upper half
+  *p0 = (uint16_t)(u & 0xffffu);
+  *p1 = (uint16_t)(u >> 16);
+}
+
+// Wait until at most one bulk store group of this thread still reads its
+// shared memory (the most recent one).
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
+// Per warp: S input stages of NARR tiles [L][32], NOUT output tiles twice
+// (double-buffered staging), STS bytes of batch-start states; after every
+// warp's region, S mbarriers per warp.
+template <typename E, int L, int NARR, int NOUT, int S, int STS>
+struct ChainLayout {
+  static constexpr int ARR = L * 32 * (int)sizeof(E);
+  static constexpr int STAGE = NARR * ARR;
+  static constexpr int OUT = NOUT * ARR;
+  static constexpr int WARP = S * STAGE + 2 * OUT + STS;
+  static_assert(ARR % 128 == 0 && STS % 128 == 0, "TMA buffers stay 128-byte aligned");
+  static constexpr int bytes(int nw) { return nw * (WARP + 8 * S); }
+};
+
+// ------------------------------------------------------------- forward ---
+template <typename E, int L, int RB, int S, bool GATE>
+__global__ void __launch_bounds__(kChainWarps * 32, 1) fwd_chain_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                        const __grid_constant__ CUtensorMap vmap,
+                                                                        const __grid_constant__ CUtensorMap rmap,
+                                                                        const __grid_constant__ CUtensorMap ymap,
+                                                                        FwdArgs p) {
+  static_assert(L % kCkpt == 0 && kCkpt % RB == 0, "units hold whole checkpoint intervals");
+  constexpr int NARR = GATE ? 3 : 2;
+  using Lay = ChainLayout<E, L, NARR, 1, S, 0>;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned char *wbuf = smem + (size_t)wl * Lay::WARP;
+  unsigned char *ybuf = wbuf + S * Lay::STAGE;
+  const uint32_t bar0 = smem_addr(smem + (size_t)kChainWarps * Lay::WARP) + 8u * S * wl;
+  if (lane == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  const int64_t chain = (int64_t)blockIdx.x * kChainWarps + wl;
+  if (chain >= p.nchains) return;  // warp-uniform; no block-wide barrier follows
+  const int64_t T = p.T, C = p.C, BC = p.B * p.C;
+  const int b = (int)(chain / p.nct);
+  const int x0 = (int)(chain - (int64_t)b * p.nct) * 32;
+  const int64_t c = (int64_t)x0 + lane;
+  const bool cok = c < C;
+  const int64_t bc = (int64_t)b * C + c;
+  const float w = cok ? __ldg(p.w + c) : 0.f, u = cok ? __ldg(p.u + c) : 0.f;
+  const float w2 = w * kLog2e, u2 = u * kLog2e;
+  const int nseg = (int)((T + L - 1) / L);
+  const int64_t budget = p.spin_limit * 1000;
+  unsigned epoch = 0;
+  if (lane == 0) epoch = ld_relaxed(&p.hdr->epoch);
+  epoch = __shfl_sync(0xffffffffu, epoch, 0);
+  const uint64_t pol = l2_policy_evict_first();  // inputs are read once
+
+  auto issue = [&](int t) {
+    const int s = t % S;
+    const uint32_t dst = smem_addr(wbuf + (size_t)s * Lay::STAGE), bar = bar0 + 8u * s;
+    mbar_expect_tx(bar, (uint32_t)Lay::STAGE);
+    tma_load_3d(dst, &kmap, x0, t * L, b, bar, pol);
+    tma_load_3d(dst + Lay::ARR, &vmap, x0, t * L, b, bar, pol);
+    if constexpr (GATE) tma_load_3d(dst + 2 * Lay::ARR, &rmap, x0, t * L, b, bar, pol);
+  };
+  int issued = -1, landed = -1;
+  if (lane == 0)
+    for (int t = 0; t < S && t < nseg; ++t) {
+      issue(t);
+      issued = t;
+    }
+  Run st = run_from(cok ? load_state_in(p.state_in, bc, BC) : st_empty());
+  const TileFast fc = tile_fast<RB>(w, w2, u2);
+  bool failed = false;
+#pragma unroll 1
+  for (int t = 0; t < nseg; ++t) {
+    const int s = t % S;
+    if (!__all_sync(0xffffffffu, mbar_wait(bar0 + 8u * s, (uint32_t)(t / S) & 1u, budget, nullptr))) {
+      failed = true;
+      if (lane == 0) raise_timeout(p.hdr, epoch);
+      break;
+    }
+    landed = t;
+    if (lane == 0) bulk_wait_read_1();  // the y store of unit t-2 is done with its buffer
+    __syncwarp();
+    const E *ks = reinterpret_cast<const E *>(wbuf + (size_t)s * Lay::STAGE) + lane;
+    const E *vs = ks + L * 32;
+    const E *rs = ks + 2 * L * 32;
+    E *ys = reinterpret_cast<E *>(ybuf + (size_t)(t & 1) * Lay::ARR) + lane;
+    const int64_t t0 = (int64_t)t * L;
+    const int n = (int)min((int64_t)L, T - t0);
+#pragma unroll 1
+    for (int bt = 0; bt < L / RB; ++bt) {
+      const int nb = n - bt * RB;
+      if (nb <= 0) break;
+      const int64_t tb = t0 + bt * RB;
+      if (p.ckpt && cok && (tb % kCkpt) == 0) store_ckpt(p.ckpt, tb / kCkpt, bc, BC, run_state(st), w2);
+      const E *kb = ks + bt * RB * 32;
+      const E *vb = vs + bt * RB * 32;
+      const E *rb = rs + bt * RB * 32;
+      E *yb = ys + bt * RB * 32;
+      const float E0 = fmaf(st.n, w2, st.Panc);
+      // the batch's inputs into registers first: the y stores below may
+      // alias them as far as the compiler knows, and a load ordered behind
+      // a store would expose its latency on every token
+      float kj[RB], Vj[RB], Rj[RB];
+#pragma unroll
+      for (int j = 0; j < RB; ++j) {
+        kj[j] = fmaf(-(float)j, fc.we, to_f32(kb[j * 32]));
+        Vj[j] = to_f32(vb[j * 32]);
+        if constexpr (GATE) Rj[j] = to_f32(rb[j * 32]);
+      }
+      float mx, mn;
+      tree_minmax<RB>(kj, mx, mn);
+      const float M = fmaxf(E0, mx * kLog2e);
+      const float span = M - mn * kLog2e;  // >= 0
+      // the range conditions of the tile forward's fast path (wkv_tile.cu)
+      const bool dens_ok = span < 100.f && span - u2 - fc.sh < 60.f;
+      const bool state_ok = fc.ewm == 1.f && E0 - M > -90.f;
+      const bool ok = fc.ok && (dens_ok || state_ok);
+      if (__all_sync(0xffffffffu, ok && nb >= RB)) {
+        const float s0 = ex2(E0 - M + fc.sh);
+        float al = st.a * s0, be = st.b * s0;
+        float yprev = 0.f;
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+          const float e0 = ex2(fmaf(kj[j], kLog2e, -M));
+          const float V = Vj[j];
+          const float eu = e0 * fc.cu;
+          float yv = fmaf(eu, V, al) * rcp(be + eu);
+          if constexpr (GATE) yv *= gate_sigmoid(Rj[j]);
+          al = fmaf(al, fc.ewm, e0 * V);
+          be = fmaf(be, fc.ewm, e0);
+          if (j & 1)
+            store2<E>(yb + (j - 1) * 32, yb + j * 32, yprev, yv);
+          else
+            yprev = yv;
+        }
+        st = Run{al, be, M, fc.nend};
+      } else {
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+          if (j < nb) {
+            float yv = fwd_token(st, to_f32(kb[j * 32]) * kLog2e, Vj[j], u2, w2);
+            if constexpr (GATE) yv *= gate_sigmoid(Rj[j]);
+            yb[j * 32] = from_f32<E>(yv);
+          }
+        }
+      }
+    }
+    __syncwarp();  // every lane is done with stage s
+    if (lane == 0 && t + S < nseg) {
+      issue(t + S);
+      issued = t + S;
+    }
+    fence_proxy_async_smem();  // y before the async proxy reads it
+    __syncwarp();
+    if (lane == 0 && p.y) {
+      tma_store_3d(&ymap, x0, (int)t0, b, smem_addr(ybuf + (size_t)(t & 1) * Lay::ARR));
+      bulk_commit();
+    }
+  }
+  if (!failed && p.state_out && cok) store_state(p.state_out, bc, BC, run_state(st), w2);
+  if (lane == 0) {
+    bulk_wait_all();  // every y store complete before the warp exits
+    for (int t = landed + 1; t <= issued; ++t)  // and every issued load landed (after a failure)
+      mbar_wait(bar0 + 8u * (t % S), (uint32_t)(t / S) & 1u, budget, nullptr);
+  }
+  __syncwarp();
+}
+
+// ------------------------------------------------------------ backward ---
+struct ChainBwdArgs {
+  BwdArgs p;
+  float *gw, *gu;
+  float4 *chain_sum;  // [B][C] tagged per-chain sums of dL/dw, dL/du
+};
+
+// Advance the forward state over one full batch (the state update of
+// recompute_batch without its outputs).
+template <int RB>
+__device__ __forceinline__ void advance_batch(const float (&K)[RB], const float (&V)[RB], float w2, float u2,
+                                              const FastC &fc, float &xa, float &xb, float &xP, float &xn) {
+  const float E0 = fmaf(xn, w2, xP);
+  float kj[RB], M;
+  const bool ok = fast_prep_tree<RB>(K, E0, u2, fc.w2e, kj, M);
+  if (__all_sync(0xffffffffu, ok)) {
+    const float s0 = ex2(E0 - M);
+    float al = xa * s0, be = xb * s0;
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      const float ek = ex2(kj[j] - M) * fc.cw;
+      al = fmaf(al, fc.ewm, ek * V[j]);
+      be = fmaf(be, fc.ewm, ek);
+    }
+    xa = al;
+    xb = be;
+    xP = M;
+    xn = fc.nend;
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    const float n1 = xn + 1.f;
+    const float Pc = fmaf(n1, w2, xP);
+    const float d2 = K[j] - Pc;
+    const float x2 = ex2(-fabsf(d2));
+    const bool kw = d2 > 0.f;
+    const float so = kw ? x2 : 1.f, snw = kw ? 1.f : x2;
+    xa = fmaf(xa, so, V[j] * snw);
+    xb = fmaf(xb, so, snw);
+    xP = kw ? K[j] : xP;
+    xn = kw ? 0.f : n1;
+  }
+}
+
+// recompute_batch of wkv_bwd_math.cuh (without the gate's extra output),
+// with the batch maximum taken as a tree.
+template <int RB>
+__device__ __forceinline__ bool chain_recompute(const float (&K)[RB], const float (&V)[RB], const float (&Gy)[RB],
+                                                float w2, float u2, const FastC &fc, float xa, float xb, float xP,
+                                                float (&qv)[RB], float (&gam)[RB], float (&eta)[RB],
+                                                float (&e2v)[RB], float &M) {
+  const float E0 = xP;
+  float kj[RB];
+  const bool ok = fast_prep_tree<RB>(K, E0, u2, fc.w2e, kj, M);
+  if (__all_sync(0xffffffffu, ok)) {
+    const float s0 = ex2(E0 - M);
+    float al = xa * s0, be = xb * s0;
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      const float e0 = ex2(kj[j] - M);
+      const float eu = e0 * fc.cu, ek = e0 * fc.cw;
+      const float rden = rcp(be + eu);
+      const float y = fmaf(eu, V[j], al) * rden;
+      gam[j] = Gy[j] * rden;
+      eta[j] = gam[j] * y;
+      e2v[j] = eu;
+      al = fmaf(al, fc.ewm, ek * V[j]);
+      be = fmaf(be, fc.ewm, ek);
+    }
+    return true;
+  }
+  float xn = 0.f;
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    const float P = fmaf(xn, w2, xP);
+    const float UK = u2 + K[j];
+    const float d = P - UK;
+    const float x = ex2(-fabsf(d));
+    const bool pw = d >= 0.f;
+    const float e1 = pw ? 1.f : x, e2 = pw ? x : 1.f;
+    const float rden = rcp(fmaf(xb, e1, e2));
+    const float y = fmaf(xa, e1, V[j] * e2) * rden;
+    qv[j] = fmaxf(P, UK);
+    gam[j] = Gy[j] * rden;
+    eta[j] = gam[j] * y;
+    e2v[j] = e2;
+    const float n1 = xn + 1.f;
+    const float Pc = fmaf(n1, w2, xP);
+    const float d2 = K[j] - Pc;
+    const float x2 = ex2(-fabsf(d2));
+    const bool kw = d2 > 0.f;
+    const float so = kw ? x2 : 1.f, snw = kw ? 1.f : x2;
+    xa = fmaf(xa, so, V[j] * snw);
+    xb = fmaf(xb, so, snw);
+    xP = kw ? K[j] : xP;
+    xn = kw ? 0.f : n1;
+  }
+  return false;
+}
+
+// advance_batch for two independent batches at once (each from its own
+// state): one vote, and both batches' arithmetic in one block the compiler
+// can interleave.
+template <int RB>
+__device__ __forceinline__ void advance_two(const float (&K0)[RB], const float (&V0)[RB], const float (&K1)[RB],
+                                            const float (&V1)[RB], float w2, float u2, const FastC &fc, float &a0,
+                                            float &b0, float &P0, float &n0, float &a1, float &b1, float &P1,
+                                            float &n1) {
+  const float E00 = fmaf(n0, w2, P0), E01 = fmaf(n1, w2, P1);
+  float kj0[RB], kj1[RB], M0, M1;
+  const bool ok0 = fast_prep_tree<RB>(K0, E00, u2, fc.w2e, kj0, M0);
+  const bool ok1 = fast_prep_tree<RB>(K1, E01, u2, fc.w2e, kj1, M1);
+  if (__all_sync(0xffffffffu, ok0 && ok1)) {
+    const float s00 = ex2(E00 - M0), s01 = ex2(E01 - M1);
+    float al0 = a0 * s00, be0 = b0 * s00, al1 = a1 * s01, be1 = b1 * s01;
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      const float ek0 = ex2(kj0[j] - M0) * fc.cw, ek1 = ex2(kj1[j] - M1) * fc.cw;
+      al0 = fmaf(al0, fc.ewm, ek0 * V0[j]);
+      be0 = fmaf(be0, fc.ewm, ek0);
+      al1 = fmaf(al1, fc.ewm, ek1 * V1[j]);
+      be1 = fmaf(be1, fc.ewm, ek1);
+    }
+    a0 = al0;
+    b0 = be0;
+    P0 = M0;
+    n0 = fc.nend;
+    a1 = al1;
+    b1 = be1;
+    P1 = M1;
+    n1 = fc.nend;
+    return;
+  }
+  advance_batch<RB>(K0, V0, w2, u2, fc, a0, b0, P0, n0);
+  advance_batch<RB>(K1, V1, w2, u2, fc, a1, b1, P1, n1);
+}
+
+template <typename E, int L, int RB, int S>
+__global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                        const __grid_constant__ CUtensorMap vmap,
+                                                                        const __grid_constant__ CUtensorMap gmap,
+                                                                        const __grid_constant__ CUtensorMap gkmap,
+                                                                        const __grid_constant__ CUtensorMap gvmap,
+                                                                        ChainBwdArgs a) {
+  static_assert(L % kCkpt == 0 && kCkpt % RB == 0, "units start on checkpoints");
+  constexpr int NB = L / RB;
+  constexpr int STS = (NB * 96 * 4 + 127) / 128 * 128;
+  using Lay = ChainLayout<E, L, 3, 2, S, STS>;
+  const BwdArgs &p = a.p;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned char *wbuf = smem + (size_t)wl * Lay::WARP;
+  unsigned char *obuf = wbuf + S * Lay::STAGE;
+  float *sts = reinterpret_cast<float *>(obuf + 2 * Lay::OUT);
+  const uint32_t bar0 = smem_addr(smem + (size_t)kChainWarps * Lay::WARP) + 8u * S * wl;
+  if (lane == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  const int G = (int)gridDim.x * kChainWarps;
+  const int g = (int)blockIdx.x * kChainWarps + wl;
+  const int nchains = (int)p.nchains, nct = (int)p.nct;
+  const int64_t T = p.T, C = p.C, BC = p.B * p.C;
+  const int nseg = (int)((T + L - 1) / L);
+  const int nmine = nchains > g ? (nchains - g + G - 1) / G : 0;  // chains of this warp
+  const int total = nmine * nseg;                                 // units of this warp
+  const int64_t budget = p.spin_limit * 1000;
+  unsigned epoch = 0;
+  if (lane == 0) epoch = ld_relaxed(&p.hdr->epoch);
+  epoch = __shfl_sync(0xffffffffu, epoch, 0);
+  const unsigned t_sum = tile_flag(epoch, 3u);
+  const uint64_t pol = l2_policy_evict_first();
+
+  // unit j of this warp: chain g + (j / nseg) G, position nseg - 1 - j % nseg,
+  // followed by cursors (no divisions in the unit loop)
+  struct Cursor {
+    int chain, pos, b, x0;
+  };
+  auto first = [&]() {
+    Cursor u{g, nseg - 1, g / nct, 0};
+    u.x0 = (g - u.b * nct) * 32;
+    return u;
+  };
+  auto next = [&](Cursor &u) {
+    if (--u.pos < 0) {
+      u.pos = nseg - 1;
+      u.chain += G;
+      u.b = u.chain / nct;
+      u.x0 = (u.chain - u.b * nct) * 32;
+    }
+  };
+  Cursor ic = first();  // the next unit to load
+  auto issue = [&](int j) {
+    const int s = j % S;
+    const uint32_t dst = smem_addr(wbuf + (size_t)s * Lay::STAGE), bar = bar0 + 8u * s;
+    mbar_expect_tx(bar, (uint32_t)Lay::STAGE);
+    tma_load_3d(dst, &kmap, ic.x0, ic.pos * L, ic.b, bar, pol);
+    tma_load_3d(dst + Lay::ARR, &vmap, ic.x0, ic.pos * L, ic.b, bar, pol);
+    tma_load_3d(dst + 2 * Lay::ARR, &gmap, ic.x0, ic.pos * L, ic.b, bar, pol);
+    next(ic);
+  };
+  int issued = -1, landed = -1;
+  if (lane == 0)
+    for (int j = 0; j < S && j < total; ++j) {
+      issue(j);
+      issued = j;
+    }
+  // checkpoints of unit jj (the states before its tokens t0, t0 + 32, ...),
+  // loaded one unit ahead so that their latency stays off the critical path
+  constexpr int NCK = L / kCkpt;
+  Cursor kc = first();  // the unit whose checkpoints load next
+  auto load_ck = [&](int jj, float(&ck)[NCK][3]) {
+    if (jj >= total) return;
+    const Cursor u = kc;
+    next(kc);
+    const int64_t cc = (int64_t)u.x0 + lane;
+    if (cc >= C) return;
+#pragma unroll
+    for (int q = 0; q < NCK; ++q) {
+      const int64_t tb = (int64_t)u.pos * L + q * kCkpt;
+      if (tb < T) {
+        const float *src = p.ckpt + (tb / kCkpt) * 3 * BC + (int64_t)u.b * C + cc;
+        ck[q][0] = __ldcg(src);
+        ck[q][1] = __ldcg(src + BC);
+        ck[q][2] = __ldcg(src + 2 * BC);
+      }
+    }
+  };
+  float ckn[NCK][3];
+#pragma unroll
+  for (int q = 0; q < NCK; ++q) ckn[q][0] = ckn[q][1] = 0.f, ckn[q][2] = kEmptyP;
+  load_ck(0, ckn);
+  bool failed = false;
+  int b = 0, x0 = 0;
+  int64_t c = 0, bc = 0;
+  bool cok = false;
+  float w2 = 0.f, u2 = 0.f;
+  FastC fc{};
+  float rah = 0.f, rhh = 0.f, rahp = 0.f, rhhp = 0.f, Ranc = kEmptyR, m = 0.f;
+  double gw_d = 0.0, gu_d = 0.0;
+  Cursor uc = first();
+#pragma unroll 1
+  for (int j = 0; j < total; ++j, next(uc)) {
+    const int s = j % S;
+    const int pos = uc.pos;
+    if (pos == nseg - 1) {
+      // a new chain: its constants, and the adjoint after its last token (empty)
+      b = uc.b;
+      x0 = uc.x0;
+      c = (int64_t)x0 + lane;
+      cok = c < C;
+      bc = (int64_t)b * C + c;
+      w2 = cok ? __ldg(p.w + c) * kLog2e : 0.f;
+      u2 = cok ? __ldg(p.u + c) * kLog2e : 0.f;
+      fc = fast_consts<RB>(w2, u2);
+      rah = rhh = rahp = rhhp = 0.f;
+      Ranc = kEmptyR;
+      m = 0.f;
+      gw_d = gu_d = 0.0;
+    }
+    if (!failed && !__all_sync(0xffffffffu, mbar_wait(bar0 + 8u * s, (uint32_t)(j / S) & 1u, budget, nullptr))) {
+      failed = true;
+      if (lane == 0) raise_timeout(p.hdr, epoch);
+    }
+    if (failed) break;
+    landed = j;
+    const int64_t t0 = (int64_t)pos * L;
+    const int n = (int)min((int64_t)L, T - t0);
+    const E *kt = reinterpret_cast<const E *>(wbuf + (size_t)s * Lay::STAGE) + lane;
+    const E *vt = kt + L * 32;
+    const E *gt = kt + 2 * L * 32;
+    auto load_batch = [&](int bt, float(&K)[RB], float(&V)[RB], float(&Gy)[RB]) {
+#pragma unroll
+      for (int q = 0; q < RB; ++q) {
+        K[q] = to_f32(kt[(bt * RB + q) * 32]) * kLog2e;
+        V[q] = to_f32(vt[(bt * RB + q) * 32]);
+        Gy[q] = to_f32(gt[(bt * RB + q) * 32]);
+      }
+    };
+
+    float ckc[NCK][3];
+#pragma unroll
+    for (int q = 0; q < NCK; ++q) ckc[q][0] = ckn[q][0], ckc[q][1] = ckn[q][1], ckc[q][2] = ckn[q][2];
+    load_ck(j + 1, ckn);
+
+    // ---- pass 1: the forward state at every batch start (exponent evaluated)
+    if constexpr (RB * 2 == kCkpt && NB == 4) {
+      // batches 0 and 2 start on checkpoints; 1 and 3 by advancing 0 and 2
+      // (independent of each other, so both advance together)
+      const bool h2 = t0 + kCkpt < T;  // the second interval holds tokens
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        sts[2 * q * 96 + lane] = ckc[q][0];
+        sts[2 * q * 96 + 32 + lane] = ckc[q][1];
+        sts[2 * q * 96 + 64 + lane] = ckc[q][2];
+      }
+      float a0 = ckc[0][0], b0 = ckc[0][1], P0 = ckc[0][2], n0 = 0.f;
+      float a1 = ckc[1][0], b1 = ckc[1][1], P1 = ckc[1][2], n1 = 0.f;
+      float K0[RB], V0[RB], K1[RB], V1[RB], G_[RB];
+      load_batch(0, K0, V0, G_);
+      if (__all_sync(0xffffffffu, h2)) {
+        load_batch(2, K1, V1, G_);
+        advance_two<RB>(K0, V0, K1, V1, w2, u2, fc, a0, b0, P0, n0, a1, b1, P1, n1);
+      } else {
+        advance_batch<RB>(K0, V0, w2, u2, fc, a0, b0, P0, n0);
+      }
+      sts[96 + lane] = a0;
+      sts[96 + 32 + lane] = b0;
+      sts[96 + 64 + lane] = fmaf(n0, w2, P0);
+      sts[3 * 96 + lane] = a1;
+      sts[3 * 96 + 32 + lane] = b1;
+      sts[3 * 96 + 64 + lane] = fmaf(n1, w2, P1);
+    } else {
+      float fa = 0.f, fb = 0.f, fP = kEmptyP, fn = 0.f;
+#pragma unroll
+      for (int bt = 0; bt < NB; ++bt) {
+        const int64_t tb = t0 + bt * RB;
+        if (tb >= T) break;  // padding: never swept
+        if ((bt * RB) % kCkpt == 0) {
+          fa = ckc[bt * RB / kCkpt][0];
+          fb = ckc[bt * RB / kCkpt][1];
+          fP = ckc[bt * RB / kCkpt][2];
+          fn = 0.f;
+        }
+        sts[bt * 96 + lane] = fa;
+        sts[bt * 96 + 32 + lane] = fb;
+        sts[bt * 96 + 64 + lane] = fmaf(fn, w2, fP);
+        if (bt + 1 < NB && ((bt + 1) * RB) % kCkpt != 0) {
+          float K[RB], V[RB], Gy[RB];
+          load_batch(bt, K, V, Gy);
+          advance_batch<RB>(K, V, w2, u2, fc, fa, fb, fP, fn);
+        }
+      }
+    }
+
+    // ---- pass 2: batches last to first, recompute then reverse sweep
+    if (lane == 0) bulk_wait_read_1();  // the stores of unit j-2 are done with this staging buffer
+    __syncwarp();
+    E *okp = reinterpret_cast<E *>(obuf + (size_t)(j & 1) * Lay::OUT) + lane;
+    E *ovp = okp + L * 32;
+    float gw_acc = 0.f, gu_acc = 0.f;
+#pragma unroll 1
+    for (int bi = 0; bi < NB; ++bi) {
+      const int bt = NB - 1 - bi;
+      if (n - bt * RB <= 0) continue;  // only padding past T: nothing to sweep
+      float K[RB], V[RB], Gy[RB];
+      load_batch(bt, K, V, Gy);
+      float qv[RB], gam[RB], eta[RB], e2v[RB], Mb;
+      const bool fast = chain_recompute<RB>(K, V, Gy, w2, u2, fc, sts[bt * 96 + lane], sts[bt * 96 + 32 + lane],
+                                            sts[bt * 96 + 64 + lane], qv, gam, eta, e2v, Mb);
+      E *gkp = okp + bt * RB * 32;
+      E *gvp = ovp + bt * RB * 32;
+      // the reverse sweep of the tile backward (wkv_tile_bwd.cu): fast in the
+      // batch's coordinates when the carried adjoint's scale allows, else per
+      // token with the running anchor
+      const float rn_end = fmaf(-m, w2, Ranc);
+      const float xin = fmaf((float)RB, fc.w2e, Mb) - rn_end;
+      if (__all_sync(0xffffffffu, fast && xin < 100.f)) {
+        const float F = ex2(xin);
+        float ra = rah * F, rh = rhh * F, rap = rahp * F, rhp = rhhp * F;
+        const float ckf = fc.cw * ex2(-u2);  // ek = e2 * ckf
+#pragma unroll
+        for (int q = RB - 1; q >= 0; --q) {
+          const float ek = e2v[q] * ckf;
+          const float gv = fmaf(gam[q], e2v[q], ek * ra);
+          const float gk = fmaf(V[q], gv, -fmaf(eta[q], e2v[q], ek * rh));
+          gw_acc = fmaf(ek, fmaf(V[q], rap, -rhp), gw_acc);
+          gu_acc = fmaf(e2v[q], fmaf(gam[q], V[q], -eta[q]), gu_acc);
+          store2<E>(gkp + q * 32, gvp + q * 32, gk, gv);
+          rap = fc.ewm * (rap + ra);
+          rhp = fc.ewm * (rhp + rh);
+          ra = fmaf(ra, fc.ewm, gam[q]);
+          rh = fmaf(rh, fc.ewm, eta[q]);
+        }
+        rah = ra;
+        rhh = rh;
+        rahp = rap;
+        rhhp = rhp;
+        Ranc = Mb;
+        m = 0.f;
+        continue;
+      }
+      if (fast) {  // the fast recompute leaves the scales implicit: D_t = den 2^{M + q w2e}
+#pragma unroll
+        for (int q = 0; q < RB; ++q) qv[q] = fmaf((float)q, fc.w2e, Mb);
+      }
+#pragma unroll
+      for (int q = RB - 1; q >= 0; --q) {
+        const float rn = fmaf(-m, w2, Ranc);  // scale of the adjoint after token t
+        const float tn = ex2(K[q] - rn);      // e^{k_t} 2^{-r_{t+1}} (<= 1)
+        const float gv = fmaf(gam[q], e2v[q], tn * rah);
+        const float gk = fmaf(V[q], gv, -fmaf(eta[q], e2v[q], tn * rhh));
+        gw_acc = fmaf(tn, fmaf(V[q], rahp, -rhhp), gw_acc);
+        gu_acc = fmaf(e2v[q], fmaf(gam[q], V[q], -eta[q]), gu_acc);
+        store2<E>(gkp + q * 32, gvp + q * 32, gk, gv);
+        const float m1 = m + 1.f;
+        const float Rc = fmaf(-m1, w2, Ranc);
+        const float d = qv[q] - Rc;
+        const float x = ex2(-fabsf(d));
+        const bool reset = d < 0.f;
+        const float fg = reset ? 1.f : x, fo = reset ? x : 1.f;
+        rahp = fo * (rah + rahp);
+        rhhp = fo * (rhh + rhhp);
+        rah = fmaf(rah, fo, gam[q] * fg);
+        rhh = fmaf(rhh, fo, eta[q] * fg);
+        Ranc = reset ? qv[q] : Ranc;
+        m = reset ? 0.f : m1;
+      }
+    }
+    __syncwarp();  // every lane is done with stage s
+    if (lane == 0 && j + S < total) {
+      issue(j + S);
+      issued = j + S;
+    }
+    if (pos == 0 && cok) {
+      // share of the initial state A_0, B_0 (zero for the empty state): the
+      // checkpoint before token 0
+      const float r0 = fmaf(-m, w2, Ranc);
+      gw_acc = fmaf(ex2(ckc[0][2] - r0), fmaf(ckc[0][0], rahp, -ckc[0][1] * rhhp), gw_acc);
+    }
+    gw_d += (double)gw_acc;
+    gu_d += (double)gu_acc;
+    fence_proxy_async_smem();  // dL/dk, dL/dv before the async proxy reads them
+    __syncwarp();
+    if (lane == 0) {
+      const uint32_t src = smem_addr(obuf + (size_t)(j & 1) * Lay::OUT);
+      tma_store_3d(&gkmap, x0, (int)t0, b, src);
+      tma_store_3d(&gvmap, x0, (int)t0, b, src + Lay::ARR);
+      bulk_commit();
+    }
+    if (pos == 0 && cok) {
+      // the chain's sums, then (last batch row) the B chains in batch-row order
+      st_relaxed_v4(a.chain_sum + bc, make_float4((float)gw_d, (float)gu_d, tagf(t_sum), 0.f));
+      if (b == (int)p.B - 1) {
+        double sw, su;
+        if (!sum_tagged(a.chain_sum + c, C, (int)p.B, t_sum, sw, su, budget)) raise_timeout(p.hdr, epoch);
+        a.gw[c] = (float)sw;
+        a.gu[c] = (float)su;
+      }
+    }
+  }
+  if (lane == 0) {
+    bulk_wait_all();
+    for (int j = landed + 1; j <= issued; ++j)
+      mbar_wait(bar0 + 8u * (j % S), (uint32_t)(j / S) & 1u, budget, nullptr);
+  }
+  __syncthreads();
+  finish_block(p.hdr, gridDim.x);
+}
+
+// ------------------------------------------------------------------ host ---
+template <typename E, int L, int RB, bool GATE>
+static cudaError_t launch_fwd_chain_t(const FwdArgs &f, int dtype, cudaStream_t st) {
+  CUtensorMap km, vm, rm, ym;
+  if (!encode_btc(&km, f.k, dtype, f.B, f.T, f.C, L) || !encode_btc(&vm, f.v, dtype, f.B, f.T, f.C, L))
+    return cudaErrorInvalidValue;
+  rm = vm;
+  ym = km;  // unused placeholders when there is no gate / no y
+  if (GATE && !encode_btc(&rm, f.r, dtype, f.B, f.T, f.C, L)) return cudaErrorInvalidValue;
+  if (f.y && !encode_btc(&ym, f.y, dtype, f.B, f.T, f.C, L)) return cudaErrorInvalidValue;
+  constexpr int S = GATE ? 3 : kChainStages;
+  constexpr int smem = ChainLayout<E, L, GATE ? 3 : 2, 1, S, 0>::bytes(kChainWarps);
+  auto kern = fwd_chain_kernel<E, L, RB, S, GATE>;
+  int occ = 0;
+  cudaError_t e = blocks_per_sm((const void *)kern, kChainWarps * 32, smem, &occ);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) return cudaErrorInvalidConfiguration;
+  if ((f.T + L - 1) / L >= (int64_t)1 << 31 || f.T >= (int64_t)1 << 31) return cudaErrorInvalidValue;
+  const int64_t grid = (f.nchains + kChainWarps - 1) / kChainWarps;
+  if (grid >= (int64_t)1 << 31) return cudaErrorInvalidValue;
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kChainWarps * 32), (size_t)smem, st, km, vm, rm, ym, f);
+}
+
+cudaError_t launch_forward_chain(const FwdArgs &f, int dtype, cudaStream_t st) {
+  if (f.r)
+    return dtype == 0 ? launch_fwd_chain_t<float, kTileLF32, WKV_CHAIN_FRB, true>(f, dtype, st)
+                      : launch_fwd_chain_t<uint16_t, kTileLBF16, WKV_CHAIN_FRB, true>(f, dtype, st);
+  return dtype == 0 ? launch_fwd_chain_t<float, kTileLF32, WKV_CHAIN_FRB, false>(f, dtype, st)
+                    : launch_fwd_chain_t<uint16_t, kTileLBF16, WKV_CHAIN_FRB, false>(f, dtype, st);
+}
+
+template <typename E, int L, int RB>
+static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *chain_sum,
+                                      int num_sms, cudaStream_t st) {
+  CUtensorMap km, vm, gm, gkm, gvm;
+  if (!encode_btc(&km, p.k, dtype, p.B, p.T, p.C, L) || !encode_btc(&vm, p.v, dtype, p.B, p.T, p.C, L) ||
+      !encode_btc(&gm, p.gy, dtype, p.B, p.T, p.C, L) || !encode_btc(&gkm, p.gk, dtype, p.B, p.T, p.C, L) ||
+      !encode_btc(&gvm, p.gv, dtype, p.B, p.T, p.C, L))
+    return cudaErrorInvalidValue;
+  constexpr int S = 3;
+  constexpr int NB = L / RB;
+  constexpr int STS = (NB * 96 * 4 + 127) / 128 * 128;
+  constexpr int smem = ChainLayout<E, L, 3, 2, S, STS>::bytes(kChainWarps);
+  auto kern = bwd_chain_kernel<E, L, RB, S>;
+  int occ = 0;
+  cudaError_t e = blocks_per_sm((const void *)kern, kChainWarps * 32, smem, &occ);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) return cudaErrorInvalidConfiguration;
+  const int64_t nseg = (p.T + L - 1) / L;
+  if (nseg * p.nchains >= (int64_t)1 << 31) return cudaErrorInvalidValue;  // unit indices are 31-bit
+  // one resident wave (cooperative launch: the last batch row's chains wait
+  // on the other rows' sums), the chains dealt out evenly
+  const int64_t max_warps = (int64_t)occ * num_sms * kChainWarps;
+  const int64_t rounds = (p.nchains + max_warps - 1) / max_warps;
+  const int64_t grid = ((p.nchains + rounds - 1) / rounds + kChainWarps - 1) / kChainWarps;
+  ChainBwdArgs a{};
+  a.p = p;
+  a.gw = gw;
+  a.gu = gu;
+  a.chain_sum = chain_sum;
+  void *args[] = {&km, &vm, &gm, &gkm, &gvm, &a};
+  return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3(kChainWarps * 32), args,
+                                     (size_t)smem, st);
+}
+
+cudaError_t launch_backward_chain(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *chain_sum, int num_sms,
+                                  cudaStream_t st) {
+  if (p.r || p.gs_out || p.gs_in) return cudaErrorInvalidValue;  // plain backward only
+  return dtype == 0 ? launch_bwd_chain_t<float, kTileLF32, WKV_CHAIN_BRB>(p, dtype, gw, gu, chain_sum, num_sms, st)
+                    : launch_bwd_chain_t<uint16_t, kTileLBF16, WKV_CHAIN_BRB>(p, dtype, gw, gu, chain_sum, num_sms, st);
+}
+
+}  // namespace wkv
+

@@ -33,6 +33,32 @@ __device__ __forceinline__ uint16_t from_f32<uint16_t>(float x) {
   return h;
 }
 
+// Per-lane constants of the batch fast path in the form the tile and chain
+// kernels use (see FastC in wkv_math.cuh for the two modes).  The undecayed mode
+// carries the state as alpha' = alpha 2^{w2}, which removes one multiply per
+// token: alpha' += e0 v, and the bonus factor becomes 2^{u2 + w2}.
+struct TileFast {
+  float we;    // decay folded into the keys (natural log): w undecayed, 0 decaying
+  float ewm;   // per-token multiplicative decay (decaying) or 1
+  float cu;    // bonus factor relative to e0: 2^{u2 + w2e}
+  float sh;    // w2e: added to the state's scale exponent at batch start
+  float nend;  // anchored decay count after a batch: RB - 1 undecayed, 0 decaying
+  bool ok;     // the fast path is valid for this lane's decay (no growth)
+};
+template <int RB>
+__device__ __forceinline__ TileFast tile_fast(float w, float w2, float u2) {
+  const bool decaying = fabsf(w2) * (float)RB >= 40.f;
+  TileFast f;
+  f.we = decaying ? 0.f : w;
+  const float w2e = decaying ? 0.f : w2;
+  f.ewm = decaying ? ex2(w2) : 1.f;
+  f.cu = ex2(u2 + w2e);
+  f.sh = w2e;
+  f.nend = decaying ? 0.f : (float)(RB - 1);
+  f.ok = !(decaying && w2 > 0.f) && u2 < 60.f;  // a growing state could overflow within a batch
+  return f;
+}
+
 // ------------------------------------------------------------- TMA (3-D) ---
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *map, int x, int y, int z, uint32_t bar,
                                             uint64_t policy) {

@@ -95,7 +95,7 @@ def test_forward_chunked_needs_workspace(W):
     assert W.abi.wkv_forward_ex(*base, FAKE * 8 + 16, 1 << 30, 0, opt) == -3  # misaligned
 
 
-@pytest.mark.parametrize("kernel", [4, 5, 9, -1])
+@pytest.mark.parametrize("kernel", [4, 5, 10, -1])
 def test_retired_and_unknown_kernel_selectors_are_rejected(W, kernel):
     """Selector values 4 and 5 are retired; unknown values are rejected too,
     before anything is launched."""

@@ -23,8 +23,8 @@ pytestmark = pytest.mark.gpu
 
 KERNELS = {"seq": W.WKV_KERNEL_SEQUENTIAL, "chunked": W.WKV_KERNEL_CHUNKED,
            "chunked_regs": W.WKV_KERNEL_CHUNKED_REGS, "segment": W.WKV_KERNEL_SEGMENT,
-           "cluster": W.WKV_KERNEL_CLUSTER, "tile": W.WKV_KERNEL_TILE}
-BWD_KERNELS = {"chunked": W.WKV_KERNEL_CHUNKED, "segment": W.WKV_KERNEL_SEGMENT, "tile": W.WKV_KERNEL_TILE}
+           "cluster": W.WKV_KERNEL_CLUSTER, "tile": W.WKV_KERNEL_TILE, "chain": W.WKV_KERNEL_CHAIN}
+BWD_KERNELS = {"chunked": W.WKV_KERNEL_CHUNKED, "segment": W.WKV_KERNEL_SEGMENT, "tile": W.WKV_KERNEL_TILE, "chain": W.WKV_KERNEL_CHAIN}
 
 
 def gated_case(B, T, C, seed, dtype="f32", rstd=1.5, state=False):

@@ -20,8 +20,9 @@ pytestmark = pytest.mark.gpu
 
 KERNELS = {"seq": W.WKV_KERNEL_SEQUENTIAL, "chunked": W.WKV_KERNEL_CHUNKED,
            "chunked_regs": W.WKV_KERNEL_CHUNKED_REGS, "segment": W.WKV_KERNEL_SEGMENT,
-           "cluster": W.WKV_KERNEL_CLUSTER, "tile": W.WKV_KERNEL_TILE}
-BWD_KERNELS = {"chunked": W.WKV_KERNEL_CHUNKED, "segment": W.WKV_KERNEL_SEGMENT, "tile": W.WKV_KERNEL_TILE}
+           "cluster": W.WKV_KERNEL_CLUSTER, "tile": W.WKV_KERNEL_TILE, "chain": W.WKV_KERNEL_CHAIN}
+BWD_KERNELS = {"chunked": W.WKV_KERNEL_CHUNKED, "segment": W.WKV_KERNEL_SEGMENT, "tile": W.WKV_KERNEL_TILE,
+               "chain": W.WKV_KERNEL_CHAIN}
 
 
 def small_case(B, T, C, seed, dtype="f32", td=(-3.0, 1.0), kstd=1.0, state=False):
@@ -94,10 +95,12 @@ def test_forward_rwkv169m_full():
     assert fwd_err(host(y)[pb, pt, pc], yp) <= F32_FWD_TOL
 
 
-def test_forward_rwkv1b5_bf16():
+@pytest.mark.parametrize("kernel", ["auto", "tile"])
+def test_forward_rwkv1b5_bf16(kernel):
     inp = workloads.generate("rwkv1b5_bf16", grad=False)
     w, u, k, v, _ = inputs_to_device(inp)
-    y, s, _ = W.forward(w, u, k, v, want_state=True)
+    kid = W.WKV_KERNEL_AUTO if kernel == "auto" else KERNELS[kernel]
+    y, s, _ = W.forward(w, u, k, v, want_state=True, kernel=kid)
     y_ref, s_ref = oracle.fwd_recur(inp["w"], inp["u"], inp["k"], inp["v"])
     assert fwd_err(host(y), y_ref) <= BF16_TOL
     assert state_err(host(s), s_ref) <= F32_FWD_TOL * 10
@@ -263,7 +266,7 @@ def _range_case(name, seed):
     return w, u, k, v, g
 
 
-@pytest.mark.parametrize("kernel", ["segment", "cluster", "tile"])
+@pytest.mark.parametrize("kernel", ["segment", "cluster", "tile", "chain"])
 @pytest.mark.parametrize("name", sorted(RANGE_CASES))
 def test_segment_forward_ranges(name, kernel):
     w, u, k, v, g = _range_case(name, seed=41)
@@ -272,7 +275,7 @@ def test_segment_forward_ranges(name, kernel):
     assert fwd_err(host(y), y_ref) <= F32_FWD_TOL
 
 
-@pytest.mark.parametrize("kernel", ["segment", "tile"])
+@pytest.mark.parametrize("kernel", ["segment", "tile", "chain"])
 @pytest.mark.parametrize("name", sorted(RANGE_CASES))
 def test_segment_backward_ranges(name, kernel):
     w, u, k, v, g = _range_case(name, seed=43)
@@ -300,11 +303,13 @@ def test_backward_rwkv169m_full():
     assert_grads(got, ref, F32_GRAD_TOL)
 
 
-def test_backward_rwkv1b5_bf16_full():
+@pytest.mark.parametrize("kernel", ["auto", "tile"])
+def test_backward_rwkv1b5_bf16_full(kernel):
     inp = workloads.generate("rwkv1b5_bf16")
     w, u, k, v, gy = inputs_to_device(inp)
-    _, _, ck = W.forward(w, u, k, v, want_ckpt=True)
-    got = W.backward(w, u, k, v, gy, ckpt=ck)
+    kid = W.WKV_KERNEL_AUTO if kernel == "auto" else KERNELS[kernel]
+    _, _, ck = W.forward(w, u, k, v, want_ckpt=True, kernel=kid)
+    got = W.backward(w, u, k, v, gy, ckpt=ck, kernel=kid)
     ref = grads_ref(inp["w"], inp["u"], inp["k"], inp["v"], inp["gy"])
     assert_grads(got, ref, BF16_TOL)
     # every channel of dL/dk and dL/dv, each on its own (a channel-wise fault
@@ -314,6 +319,25 @@ def test_backward_rwkv1b5_bf16_full():
         num = np.sqrt(((x - b) ** 2).sum(axis=(0, 1)))
         den = np.sqrt((b ** 2).sum(axis=(0, 1)))
         assert np.max(num / den) <= BF16_TOL, (name, int(np.argmax(num / den)))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_chain_kernels_over_more_chains_than_one_wave(dtype):
+    """More chains (batch rows x 32-channel tiles) than four warps per SM can
+    hold at once: the forward runs its blocks in several waves, the
+    backward's warps take several chains each, and the batch rows' dL/dw,
+    dL/du sums still meet."""
+    B, T, C = 50, 100, 416  # 650 chains, a ragged channel tile
+    w, u, k, v, g, _ = small_case(B, T, C, seed=51, dtype=dtype)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    K_, V_, G_ = dev(k, tdt), dev(v, tdt), dev(g, tdt)
+    W_, U_ = dev(w), dev(u)
+    y, s, ck = W.forward(W_, U_, K_, V_, want_state=True, want_ckpt=True, kernel=W.WKV_KERNEL_CHAIN)
+    y_ref, s_ref = oracle.fwd_recur(w, u, k, v)
+    assert fwd_err(host(y), y_ref) <= (BF16_TOL if dtype == "bf16" else F32_FWD_TOL)
+    assert state_err(host(s), s_ref) <= F32_FWD_TOL * (10 if dtype == "bf16" else 1)
+    got = W.backward(W_, U_, K_, V_, G_, ckpt=ck, kernel=W.WKV_KERNEL_CHAIN)
+    assert_grads(got, grads_ref(w, u, k, v, g), BF16_TOL if dtype == "bf16" else F32_GRAD_TOL)
 
 
 def test_backward_deterministic():
@@ -388,7 +412,7 @@ def test_backward_timeout_is_reported_and_context_survives(kernel):
     assert_grads(got, grads_ref(w, u, k, v, g), F32_GRAD_TOL)
 
 
-@pytest.mark.parametrize("kernel", ["segment", "tile"])
+@pytest.mark.parametrize("kernel", ["segment", "tile", "chain"])
 def test_segment_backward_reuses_a_workspace_across_shapes(kernel):
     """One workspace, shapes in decreasing then increasing size: whatever an
     earlier call left in the workspace does not leak into a later result."""
@@ -402,7 +426,7 @@ def test_segment_backward_reuses_a_workspace_across_shapes(kernel):
         assert_grads(got, grads_ref(w, u, k, v, g), F32_GRAD_TOL)
 
 
-@pytest.mark.parametrize("fwd_kernel", ["segment", "tile"])
+@pytest.mark.parametrize("fwd_kernel", ["segment", "tile", "chain"])
 def test_segment_outputs_stay_inside_their_buffers(fwd_kernel):
     B, T, C = 2, 300, 96
     w, u, k, v, g, _ = small_case(B, T, C, seed=27)
@@ -446,42 +470,48 @@ def test_argument_errors_launch_nothing():
     torch.cuda.synchronize()
 
 
-def test_tile_results_are_bit_reproducible_at_full_size():
+@pytest.mark.parametrize("kernel", ["tile", "chain"])
+def test_tile_results_are_bit_reproducible_at_full_size(kernel):
     """The tile kernels' look-backs take whatever prefix is published first,
-    but every prefix is the same left fold of unit records: two runs of the
-    RWKV-4 169M-shaped layer give identical bits."""
+    but every prefix is the same left fold of unit records; the chain
+    kernels add the batch rows' dL/dw, dL/du in a fixed order whichever
+    finishes first: two runs of the RWKV-4 169M-shaped layer give identical
+    bits."""
     inp = workloads.generate("rwkv169m")
     w, u, k, v, gy = inputs_to_device(inp)
     runs = []
     for _ in range(2):
-        y, s, ck = W.forward(w, u, k, v, want_state=True, want_ckpt=True, kernel=W.WKV_KERNEL_TILE)
-        grads = W.backward(w, u, k, v, gy, ckpt=ck, kernel=W.WKV_KERNEL_TILE)
+        y, s, ck = W.forward(w, u, k, v, want_state=True, want_ckpt=True, kernel=KERNELS[kernel])
+        grads = W.backward(w, u, k, v, gy, ckpt=ck, kernel=KERNELS[kernel])
         runs.append((y, s, ck) + tuple(grads))
     for a, b in zip(*runs):
         assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("kernel", ["tile", "chain"])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("T", [32, 33, 64, 65, 96])
-def test_tile_unit_boundaries(T, dtype):
+@pytest.mark.parametrize("T", [1, 15, 16, 17, 32, 33, 48, 64, 65, 96, 129])
+def test_tile_unit_boundaries(T, dtype, kernel):
     """Lengths at and just past one and two tile units (32 fp32 / 64 bf16
-    tokens): a chain of a single unit, a ragged last unit, and the group
-    boundaries of the backward's fixed-order sums."""
+    tokens) and the batches inside them (16 tokens): a chain of a single
+    unit, a ragged last unit and batch, and the group boundaries of the
+    backward's fixed-order sums."""
+    kid = KERNELS[kernel]
     B, C = 3, 96
     w, u, k, v, g, _ = small_case(B, T, C, seed=T * 11 + len(dtype), dtype=dtype)
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     K_, V_, G_ = dev(k, tdt), dev(v, tdt), dev(g, tdt)
     W_, U_ = dev(w), dev(u)
-    y, s, ck = W.forward(W_, U_, K_, V_, want_state=True, want_ckpt=True, kernel=W.WKV_KERNEL_TILE)
+    y, s, ck = W.forward(W_, U_, K_, V_, want_state=True, want_ckpt=True, kernel=kid)
     y_ref, s_ref = oracle.fwd_recur(w, u, k, v)
     tol_f = BF16_TOL if dtype == "bf16" else F32_FWD_TOL
     assert fwd_err(host(y), y_ref) <= tol_f
     assert state_err(host(s), s_ref) <= F32_FWD_TOL * (10 if dtype == "bf16" else 1)
-    got = W.backward(W_, U_, K_, V_, G_, ckpt=ck, kernel=W.WKV_KERNEL_TILE)
+    got = W.backward(W_, U_, K_, V_, G_, ckpt=ck, kernel=kid)
     assert_grads(got, grads_ref(w, u, k, v, g), BF16_TOL if dtype == "bf16" else F32_GRAD_TOL)
 
 
-@pytest.mark.parametrize("kernel", ["segment", "tile"])
+@pytest.mark.parametrize("kernel", ["segment", "tile", "chain"])
 def test_cached_tensor_maps_follow_shape_changes(kernel):
     """The library remembers encoded tensor maps by (address, shape, dtype,
     box).  One pair of buffers viewed as several shapes in turn (same base

@@ -24,7 +24,7 @@ from gpu_util import BF16_TOL, F32_GRAD_TOL, dev, host, inputs_to_device, rel_l2
 
 pytestmark = pytest.mark.gpu
 
-BWD_KERNELS = {"chunked": W.WKV_KERNEL_CHUNKED, "segment": W.WKV_KERNEL_SEGMENT, "tile": W.WKV_KERNEL_TILE}
+BWD_KERNELS = {"chunked": W.WKV_KERNEL_CHUNKED, "segment": W.WKV_KERNEL_SEGMENT, "tile": W.WKV_KERNEL_TILE, "chain": W.WKV_KERNEL_CHAIN}
 
 
 def state_case(B, T, C, seed, dtype="f32", kstd=1.0, td=(-3.0, 1.0)):
