@@ -101,8 +101,8 @@ KERNEL_SOURCES = {
 # (workload, kernel, gated, hash of the kernel's code).  A kernel whose code changed
 # since its capture has no entry: its traffic is reported as null.
 TRAFFIC = {
-    ("rwkv1b5_bf16", "bwd_tile_kernel", False, "b8cbf6bf4c53f50a"): 417_612_800 + 294_274_048,
-    ("rwkv1b5_bf16", "fwd_tile_kernel", False, "bc53deb1657ced5a"): 278_965_504 + 155_403_520,
+    ("rwkv1b5_bf16", "bwd_chain_kernel", False, "82881209cade8efe"): 427_978_752 + 211_177_216,
+    ("rwkv1b5_bf16", "fwd_chain_kernel", False, "0db41f984c0c885b"): 268_591_616 + 104_592_896,
     ("rwkv169m", "bwd_seg_kernel", False, "c5e242ca4e035480"): 77_597_952 + 529_152,
     ("rwkv169m", "fwd_seg_kernel", False, "1edb76594a20115c"): 50_392_064 + 1_318_400,
     ("longctx", "fwd_seg_kernel", False, "1edb76594a20115c"): 1_463_432_192 + 639_096_320,
