@@ -72,7 +72,7 @@
 extern "C" {
 #endif
 
-#define WKV_VERSION 130 /* 1.3.0: causal linear attention (linattn.h) */
+#define WKV_VERSION 140 /* 1.4.0: chain kernels; a checkpoint every 16 tokens */
 
 /* Element type of the [B, T, C] tensors. */
 typedef enum { WKV_F32 = 0, WKV_BF16 = 1 } wkv_dtype;
@@ -166,8 +166,8 @@ size_t wkv_workspace_size(int op, int64_t B, int64_t T, int64_t C, int dtype);
 int wkv_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /*
- * Bytes of the forward checkpoint buffer: the state at every 32nd token,
- * float32 [ceil(T/32)][3][B][C].  Its contents are private to the library
+ * Bytes of the forward checkpoint buffer: the state at every 16th token,
+ * float32 [ceil(T/16)][3][B][C].  Its contents are private to the library
  * (the exponent is stored in base 2); it only carries the forward's
  * per-chunk states to wkv_backward so the backward does not rescan.
  */

@@ -82,7 +82,7 @@ bool sizes_ok(int64_t B, int64_t T, int64_t C) {
 
 struct Layout {
   size_t flags, desc, desc_bytes, ckpt, part, cnt, rec, sums, total;
-  int64_t nct, nchains, nchunks_f, nchunks_b;
+  int64_t nct, nchains, nchunks_f, nchunks_b, nck;
 };
 
 // Workspace: [256 B header][flags][descriptors][ckpt (backward)][partials
@@ -93,7 +93,8 @@ Layout layout(int op, int64_t B, int64_t T, int64_t C) {
   L.nct = cdiv(C, 32);
   L.nchains = B * L.nct;
   L.nchunks_f = cdiv(T, fwd_chunk_tokens());
-  L.nchunks_b = cdiv(T, kCkpt);
+  L.nchunks_b = cdiv(T, 32);  // the backward kernels' records: units of at least 32 tokens
+  L.nck = cdiv(T, kCkpt);     // checkpoints
   const int64_t tiles = L.nchains * (L.nchunks_f > L.nchunks_b ? L.nchunks_f : L.nchunks_b);
   size_t off = sizeof(WsHeader);
   L.flags = off;
@@ -111,7 +112,7 @@ Layout layout(int op, int64_t B, int64_t T, int64_t C) {
   L.ckpt = L.part = L.cnt = 0;
   if (op == WKV_OP_BACKWARD) {
     L.ckpt = off;
-    off = align_up(off + sizeof(float) * 3 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
+    off = align_up(off + sizeof(float) * 3 * (size_t)(B * C) * (size_t)L.nck, 256);
     L.part = off;  // dL/dw, dL/du partials: 2 floats per (chunk, b, c); the tile kernel's tagged words: 4
     off = align_up(off + sizeof(float) * 4 * (size_t)(B * C) * (size_t)L.nchunks_b, 256);
     L.cnt = off;  // per channel tile counters of the segment backward's reduction (cleared by it)
@@ -351,7 +352,7 @@ int backward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, co
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   const bool bwd_tma = bwd_uses_seg(B, T, C, dtype, k, v, grad_y, nullptr) && aligned(grad_k, 16) &&
                        aligned(grad_v, 16);
-  if (!r && !sg.gs_out && !sg.gs_in && bwd_tma &&
+  if (!r && !sg.gs_out && !sg.gs_in && bwd_tma && aligned(ck, 16) &&
       (kernel == WKV_KERNEL_CHAIN || (kernel == WKV_KERNEL_AUTO && chain_pays(L.nchains)))) {
     float4 *sums = reinterpret_cast<float4 *>(base + L.sums);
     return cuda_rc(launch_backward_chain(a, dtype, grad_w, grad_u, sums, num_sms(), st));

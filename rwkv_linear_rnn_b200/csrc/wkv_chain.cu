@@ -21,11 +21,10 @@
 //
 // Forward, per unit: the recurrence over the unit's tokens, in batches of
 // RB tokens on the batch fast path of wkv_math.cuh where the warp allows it;
-// y, the checkpoints every 32 tokens and the final state are written.
-// Backward, per unit, units last to first: the forward state at every batch
-// start (from the checkpoints, and by advancing a batch where a checkpoint
-// does not fall on it), then batches last to first: recompute, reverse
-// sweep of the adjoint, dL/dk and dL/dv.  dL/dw and dL/du are summed per
+// y, the checkpoints every 16 tokens and the final state are written.
+// Backward, per unit, units last to first: batches of one checkpoint
+// interval, last to first, each from its checkpoint (loaded by TMA with the
+// unit's tiles): recompute, reverse sweep of the adjoint, dL/dk and dL/dv.  dL/dw and dL/du are summed per
 // chain (per unit in float, across units in float64), and the chain of the
 // last batch row of each channel tile adds the B chains in batch-row order:
 // the result is bit-reproducible.
@@ -40,13 +39,11 @@
 #ifndef WKV_CHAIN_FRB
 #define WKV_CHAIN_FRB 32
 #endif
-#ifndef WKV_CHAIN_BRB
-#define WKV_CHAIN_BRB 16
-#endif
 
 namespace wkv {
 
 bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T, int64_t C, int box_t);
+bool encode_ckpt(CUtensorMap *m, const float *ck, int64_t B, int64_t C, int64_t nck, int box_ck);
 
 constexpr int kChainWarps = 4;  // warps per block: one per scheduler
 constexpr int kChainStages = 4;  // units of input in flight per warp
@@ -111,16 +108,16 @@ __device__ __forceinline__ void store2<uint16_t>(uint16_t *p0, uint16_t *p1, flo
 // shared memory (the most recent one).
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 
-// Per warp: S input stages of NARR tiles [L][32], NOUT output tiles twice
-// (double-buffered staging), STS bytes of batch-start states; after every
-// warp's region, S mbarriers per warp.
-template <typename E, int L, int NARR, int NOUT, int S, int STS>
+// Per warp: S input stages of NARR tiles [L][32] (and XST bytes more),
+// NOUT output tiles twice (double-buffered staging), STS bytes of scratch;
+// after every warp's region, S mbarriers per warp.
+template <typename E, int L, int NARR, int NOUT, int S, int STS, int XST = 0>
 struct ChainLayout {
   static constexpr int ARR = L * 32 * (int)sizeof(E);
-  static constexpr int STAGE = NARR * ARR;
+  static constexpr int STAGE = NARR * ARR + XST;  // + XST bytes more per stage (after the tiles)
   static constexpr int OUT = NOUT * ARR;
   static constexpr int WARP = S * STAGE + 2 * OUT + STS;
-  static_assert(ARR % 128 == 0 && STS % 128 == 0, "TMA buffers stay 128-byte aligned");
+  static_assert(ARR % 128 == 0 && STS % 128 == 0 && XST % 128 == 0, "TMA buffers stay 128-byte aligned");
   static constexpr int bytes(int nw) { return nw * (WARP + 8 * S); }
 };
 
@@ -131,7 +128,7 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) fwd_chain_kernel(const __
                                                                         const __grid_constant__ CUtensorMap rmap,
                                                                         const __grid_constant__ CUtensorMap ymap,
                                                                         FwdArgs p) {
-  static_assert(L % kCkpt == 0 && kCkpt % RB == 0, "units hold whole checkpoint intervals");
+  static_assert(L % RB == 0 && RB % kCkpt == 0, "batches hold whole checkpoint intervals");
   constexpr int NARR = GATE ? 3 : 2;
   using Lay = ChainLayout<E, L, NARR, 1, S, 0>;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -228,8 +225,14 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) fwd_chain_kernel(const __
         const float s0 = ex2(E0 - M + fc.sh);
         float al = st.a * s0, be = st.b * s0;
         float yprev = 0.f;
+        // the sums at the checkpoints inside the batch, stored after it
+        float cka[RB / kCkpt], ckb[RB / kCkpt];
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
+          if (j > 0 && j % kCkpt == 0) {
+            cka[j / kCkpt] = al;
+            ckb[j / kCkpt] = be;
+          }
           const float e0 = ex2(fmaf(kj[j], kLog2e, -M));
           const float V = Vj[j];
           const float eu = e0 * fc.cu;
@@ -243,10 +246,20 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) fwd_chain_kernel(const __
             yprev = yv;
         }
         st = Run{al, be, M, fc.nend};
+        // after j tokens the sums sit at the exponent M + (j - 1) w2
+        // (undecayed mode) or M (decaying mode)
+        if (p.ckpt && cok) {
+#pragma unroll
+          for (int q = 1; q < RB / kCkpt; ++q)
+            store_ckpt(p.ckpt, tb / kCkpt + q, bc, BC,
+                       St{cka[q], ckb[q], M, fc.nend == 0.f ? 0.f : (float)(q * kCkpt - 1)}, w2);
+        }
       } else {
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
           if (j < nb) {
+            if (j > 0 && j % kCkpt == 0 && p.ckpt && cok)
+              store_ckpt(p.ckpt, (tb + j) / kCkpt, bc, BC, run_state(st), w2);
             float yv = fwd_token(st, to_f32(kb[j * 32]) * kLog2e, Vj[j], u2, w2);
             if constexpr (GATE) yv *= gate_sigmoid(Rj[j]);
             yb[j * 32] = from_f32<E>(yv);
@@ -281,44 +294,6 @@ struct ChainBwdArgs {
   float *gw, *gu;
   float4 *chain_sum;  // [B][C] tagged per-chain sums of dL/dw, dL/du
 };
-
-// Advance the forward state over one full batch (the state update of
-// recompute_batch without its outputs).
-template <int RB>
-__device__ __forceinline__ void advance_batch(const float (&K)[RB], const float (&V)[RB], float w2, float u2,
-                                              const FastC &fc, float &xa, float &xb, float &xP, float &xn) {
-  const float E0 = fmaf(xn, w2, xP);
-  float kj[RB], M;
-  const bool ok = fast_prep_tree<RB>(K, E0, u2, fc.w2e, kj, M);
-  if (__all_sync(0xffffffffu, ok)) {
-    const float s0 = ex2(E0 - M);
-    float al = xa * s0, be = xb * s0;
-#pragma unroll
-    for (int j = 0; j < RB; ++j) {
-      const float ek = ex2(kj[j] - M) * fc.cw;
-      al = fmaf(al, fc.ewm, ek * V[j]);
-      be = fmaf(be, fc.ewm, ek);
-    }
-    xa = al;
-    xb = be;
-    xP = M;
-    xn = fc.nend;
-    return;
-  }
-#pragma unroll
-  for (int j = 0; j < RB; ++j) {
-    const float n1 = xn + 1.f;
-    const float Pc = fmaf(n1, w2, xP);
-    const float d2 = K[j] - Pc;
-    const float x2 = ex2(-fabsf(d2));
-    const bool kw = d2 > 0.f;
-    const float so = kw ? x2 : 1.f, snw = kw ? 1.f : x2;
-    xa = fmaf(xa, so, V[j] * snw);
-    xb = fmaf(xb, so, snw);
-    xP = kw ? K[j] : xP;
-    xn = kw ? 0.f : n1;
-  }
-}
 
 // recompute_batch of wkv_bwd_math.cuh (without the gate's extra output),
 // with the batch maximum taken as a tree.
@@ -376,60 +351,37 @@ __device__ __forceinline__ bool chain_recompute(const float (&K)[RB], const floa
   return false;
 }
 
-// advance_batch for two independent batches at once (each from its own
-// state): one vote, and both batches' arithmetic in one block the compiler
-// can interleave.
-template <int RB>
-__device__ __forceinline__ void advance_two(const float (&K0)[RB], const float (&V0)[RB], const float (&K1)[RB],
-                                            const float (&V1)[RB], float w2, float u2, const FastC &fc, float &a0,
-                                            float &b0, float &P0, float &n0, float &a1, float &b1, float &P1,
-                                            float &n1) {
-  const float E00 = fmaf(n0, w2, P0), E01 = fmaf(n1, w2, P1);
-  float kj0[RB], kj1[RB], M0, M1;
-  const bool ok0 = fast_prep_tree<RB>(K0, E00, u2, fc.w2e, kj0, M0);
-  const bool ok1 = fast_prep_tree<RB>(K1, E01, u2, fc.w2e, kj1, M1);
-  if (__all_sync(0xffffffffu, ok0 && ok1)) {
-    const float s00 = ex2(E00 - M0), s01 = ex2(E01 - M1);
-    float al0 = a0 * s00, be0 = b0 * s00, al1 = a1 * s01, be1 = b1 * s01;
-#pragma unroll
-    for (int j = 0; j < RB; ++j) {
-      const float ek0 = ex2(kj0[j] - M0) * fc.cw, ek1 = ex2(kj1[j] - M1) * fc.cw;
-      al0 = fmaf(al0, fc.ewm, ek0 * V0[j]);
-      be0 = fmaf(be0, fc.ewm, ek0);
-      al1 = fmaf(al1, fc.ewm, ek1 * V1[j]);
-      be1 = fmaf(be1, fc.ewm, ek1);
-    }
-    a0 = al0;
-    b0 = be0;
-    P0 = M0;
-    n0 = fc.nend;
-    a1 = al1;
-    b1 = be1;
-    P1 = M1;
-    n1 = fc.nend;
-    return;
-  }
-  advance_batch<RB>(K0, V0, w2, u2, fc, a0, b0, P0, n0);
-  advance_batch<RB>(K1, V1, w2, u2, fc, a1, b1, P1, n1);
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *map, int x, int y, int z, int w, uint32_t bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar), "l"(policy)
+      : "memory");
 }
 
+// Batches are one checkpoint interval (RB = kCkpt tokens), so every batch
+// starts on a checkpoint: the unit's checkpoints arrive by TMA with its k,
+// v and grad_y tiles (a fourth region of the stage, [L/RB][3][32] floats)
+// and are the batch-start states as they are; no forward pass over the
+// unit precedes its sweep.
 template <typename E, int L, int RB, int S>
 __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                         const __grid_constant__ CUtensorMap vmap,
                                                                         const __grid_constant__ CUtensorMap gmap,
+                                                                        const __grid_constant__ CUtensorMap ckmap,
                                                                         const __grid_constant__ CUtensorMap gkmap,
                                                                         const __grid_constant__ CUtensorMap gvmap,
                                                                         ChainBwdArgs a) {
-  static_assert(L % kCkpt == 0 && kCkpt % RB == 0, "units start on checkpoints");
+  static_assert(L % kCkpt == 0 && RB == kCkpt, "batches are checkpoint intervals");
   constexpr int NB = L / RB;
-  constexpr int STS = (NB * 96 * 4 + 127) / 128 * 128;
-  using Lay = ChainLayout<E, L, 3, 2, S, STS>;
+  constexpr int CKB = NB * 96 * 4;  // the unit's checkpoints
+  using Lay = ChainLayout<E, L, 3, 2, S, 0, CKB>;
   const BwdArgs &p = a.p;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char *wbuf = smem + (size_t)wl * Lay::WARP;
   unsigned char *obuf = wbuf + S * Lay::STAGE;
-  float *sts = reinterpret_cast<float *>(obuf + 2 * Lay::OUT);
   const uint32_t bar0 = smem_addr(smem + (size_t)kChainWarps * Lay::WARP) + 8u * S * wl;
   if (lane == 0) {
     for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1);
@@ -439,7 +391,7 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
   const int G = (int)gridDim.x * kChainWarps;
   const int g = (int)blockIdx.x * kChainWarps + wl;
   const int nchains = (int)p.nchains, nct = (int)p.nct;
-  const int64_t T = p.T, C = p.C, BC = p.B * p.C;
+  const int64_t T = p.T, C = p.C;
   const int nseg = (int)((T + L - 1) / L);
   const int nmine = nchains > g ? (nchains - g + G - 1) / G : 0;  // chains of this warp
   const int total = nmine * nseg;                                 // units of this warp
@@ -476,6 +428,7 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
     tma_load_3d(dst, &kmap, ic.x0, ic.pos * L, ic.b, bar, pol);
     tma_load_3d(dst + Lay::ARR, &vmap, ic.x0, ic.pos * L, ic.b, bar, pol);
     tma_load_3d(dst + 2 * Lay::ARR, &gmap, ic.x0, ic.pos * L, ic.b, bar, pol);
+    tma_load_4d(dst + 3 * Lay::ARR, &ckmap, ic.x0, ic.b, 0, ic.pos * NB, bar, pol);
     next(ic);
   };
   int issued = -1, landed = -1;
@@ -484,31 +437,6 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
       issue(j);
       issued = j;
     }
-  // checkpoints of unit jj (the states before its tokens t0, t0 + 32, ...),
-  // loaded one unit ahead so that their latency stays off the critical path
-  constexpr int NCK = L / kCkpt;
-  Cursor kc = first();  // the unit whose checkpoints load next
-  auto load_ck = [&](int jj, float(&ck)[NCK][3]) {
-    if (jj >= total) return;
-    const Cursor u = kc;
-    next(kc);
-    const int64_t cc = (int64_t)u.x0 + lane;
-    if (cc >= C) return;
-#pragma unroll
-    for (int q = 0; q < NCK; ++q) {
-      const int64_t tb = (int64_t)u.pos * L + q * kCkpt;
-      if (tb < T) {
-        const float *src = p.ckpt + (tb / kCkpt) * 3 * BC + (int64_t)u.b * C + cc;
-        ck[q][0] = __ldcg(src);
-        ck[q][1] = __ldcg(src + BC);
-        ck[q][2] = __ldcg(src + 2 * BC);
-      }
-    }
-  };
-  float ckn[NCK][3];
-#pragma unroll
-  for (int q = 0; q < NCK; ++q) ckn[q][0] = ckn[q][1] = 0.f, ckn[q][2] = kEmptyP;
-  load_ck(0, ckn);
   bool failed = false;
   int b = 0, x0 = 0;
   int64_t c = 0, bc = 0;
@@ -557,60 +485,8 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
       }
     };
 
-    float ckc[NCK][3];
-#pragma unroll
-    for (int q = 0; q < NCK; ++q) ckc[q][0] = ckn[q][0], ckc[q][1] = ckn[q][1], ckc[q][2] = ckn[q][2];
-    load_ck(j + 1, ckn);
-
-    // ---- pass 1: the forward state at every batch start (exponent evaluated)
-    if constexpr (RB * 2 == kCkpt && NB == 4) {
-      // batches 0 and 2 start on checkpoints; 1 and 3 by advancing 0 and 2
-      // (independent of each other, so both advance together)
-      const bool h2 = t0 + kCkpt < T;  // the second interval holds tokens
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        sts[2 * q * 96 + lane] = ckc[q][0];
-        sts[2 * q * 96 + 32 + lane] = ckc[q][1];
-        sts[2 * q * 96 + 64 + lane] = ckc[q][2];
-      }
-      float a0 = ckc[0][0], b0 = ckc[0][1], P0 = ckc[0][2], n0 = 0.f;
-      float a1 = ckc[1][0], b1 = ckc[1][1], P1 = ckc[1][2], n1 = 0.f;
-      float K0[RB], V0[RB], K1[RB], V1[RB], G_[RB];
-      load_batch(0, K0, V0, G_);
-      if (__all_sync(0xffffffffu, h2)) {
-        load_batch(2, K1, V1, G_);
-        advance_two<RB>(K0, V0, K1, V1, w2, u2, fc, a0, b0, P0, n0, a1, b1, P1, n1);
-      } else {
-        advance_batch<RB>(K0, V0, w2, u2, fc, a0, b0, P0, n0);
-      }
-      sts[96 + lane] = a0;
-      sts[96 + 32 + lane] = b0;
-      sts[96 + 64 + lane] = fmaf(n0, w2, P0);
-      sts[3 * 96 + lane] = a1;
-      sts[3 * 96 + 32 + lane] = b1;
-      sts[3 * 96 + 64 + lane] = fmaf(n1, w2, P1);
-    } else {
-      float fa = 0.f, fb = 0.f, fP = kEmptyP, fn = 0.f;
-#pragma unroll
-      for (int bt = 0; bt < NB; ++bt) {
-        const int64_t tb = t0 + bt * RB;
-        if (tb >= T) break;  // padding: never swept
-        if ((bt * RB) % kCkpt == 0) {
-          fa = ckc[bt * RB / kCkpt][0];
-          fb = ckc[bt * RB / kCkpt][1];
-          fP = ckc[bt * RB / kCkpt][2];
-          fn = 0.f;
-        }
-        sts[bt * 96 + lane] = fa;
-        sts[bt * 96 + 32 + lane] = fb;
-        sts[bt * 96 + 64 + lane] = fmaf(fn, w2, fP);
-        if (bt + 1 < NB && ((bt + 1) * RB) % kCkpt != 0) {
-          float K[RB], V[RB], Gy[RB];
-          load_batch(bt, K, V, Gy);
-          advance_batch<RB>(K, V, w2, u2, fc, fa, fb, fP, fn);
-        }
-      }
-    }
+    // the batch-start states: the unit's checkpoints ([NB][3][32] floats)
+    const float *sts = reinterpret_cast<const float *>(wbuf + (size_t)s * Lay::STAGE + 3 * Lay::ARR);
 
     // ---- pass 2: batches last to first, recompute then reverse sweep
     if (lane == 0) bulk_wait_read_1();  // the stores of unit j-2 are done with this staging buffer
@@ -695,7 +571,7 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
       // share of the initial state A_0, B_0 (zero for the empty state): the
       // checkpoint before token 0
       const float r0 = fmaf(-m, w2, Ranc);
-      gw_acc = fmaf(ex2(ckc[0][2] - r0), fmaf(ckc[0][0], rahp, -ckc[0][1] * rhhp), gw_acc);
+      gw_acc = fmaf(ex2(sts[64 + lane] - r0), fmaf(sts[lane], rahp, -sts[32 + lane] * rhhp), gw_acc);
     }
     gw_d += (double)gw_acc;
     gu_d += (double)gu_acc;
@@ -761,15 +637,15 @@ cudaError_t launch_forward_chain(const FwdArgs &f, int dtype, cudaStream_t st) {
 template <typename E, int L, int RB>
 static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *chain_sum,
                                       int num_sms, cudaStream_t st) {
-  CUtensorMap km, vm, gm, gkm, gvm;
+  CUtensorMap km, vm, gm, ckm, gkm, gvm;
+  constexpr int NB = L / RB;
   if (!encode_btc(&km, p.k, dtype, p.B, p.T, p.C, L) || !encode_btc(&vm, p.v, dtype, p.B, p.T, p.C, L) ||
       !encode_btc(&gm, p.gy, dtype, p.B, p.T, p.C, L) || !encode_btc(&gkm, p.gk, dtype, p.B, p.T, p.C, L) ||
-      !encode_btc(&gvm, p.gv, dtype, p.B, p.T, p.C, L))
+      !encode_btc(&gvm, p.gv, dtype, p.B, p.T, p.C, L) ||
+      !encode_ckpt(&ckm, p.ckpt, p.B, p.C, (p.T + kCkpt - 1) / kCkpt, NB))
     return cudaErrorInvalidValue;
   constexpr int S = 3;
-  constexpr int NB = L / RB;
-  constexpr int STS = (NB * 96 * 4 + 127) / 128 * 128;
-  constexpr int smem = ChainLayout<E, L, 3, 2, S, STS>::bytes(kChainWarps);
+  constexpr int smem = ChainLayout<E, L, 3, 2, S, 0, NB * 96 * 4>::bytes(kChainWarps);
   auto kern = bwd_chain_kernel<E, L, RB, S>;
   int occ = 0;
   cudaError_t e = blocks_per_sm((const void *)kern, kChainWarps * 32, smem, &occ);
@@ -787,7 +663,7 @@ static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, fl
   a.gw = gw;
   a.gu = gu;
   a.chain_sum = chain_sum;
-  void *args[] = {&km, &vm, &gm, &gkm, &gvm, &a};
+  void *args[] = {&km, &vm, &gm, &ckm, &gkm, &gvm, &a};
   return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3(kChainWarps * 32), args,
                                      (size_t)smem, st);
 }
@@ -795,8 +671,8 @@ static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, fl
 cudaError_t launch_backward_chain(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *chain_sum, int num_sms,
                                   cudaStream_t st) {
   if (p.r || p.gs_out || p.gs_in) return cudaErrorInvalidValue;  // plain backward only
-  return dtype == 0 ? launch_bwd_chain_t<float, kTileLF32, WKV_CHAIN_BRB>(p, dtype, gw, gu, chain_sum, num_sms, st)
-                    : launch_bwd_chain_t<uint16_t, kTileLBF16, WKV_CHAIN_BRB>(p, dtype, gw, gu, chain_sum, num_sms, st);
+  return dtype == 0 ? launch_bwd_chain_t<float, kTileLF32, kCkpt>(p, dtype, gw, gu, chain_sum, num_sms, st)
+                    : launch_bwd_chain_t<uint16_t, kTileLBF16, kCkpt>(p, dtype, gw, gu, chain_sum, num_sms, st);
 }
 
 }  // namespace wkv

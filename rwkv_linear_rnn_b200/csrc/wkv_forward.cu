@@ -584,6 +584,27 @@ bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T
   return true;
 }
 
+// Checkpoints [nck][3][B][C] float32 as a 4-D map (channels fastest),
+// boxes of 32 channels x 1 batch row x 3 planes x box_ck checkpoints: one
+// chain's consecutive checkpoints land as [box_ck][3][32] floats.  Indices
+// past nck or C read zeros.
+bool encode_ckpt(CUtensorMap *m, const float *ck, int64_t B, int64_t C, int64_t nck, int box_ck) {
+  const MapKey key{ck, C, B, nck, 0, 104, box_ck};
+  if (map_lookup(key, m)) return true;
+  auto enc = tensor_map_encoder();
+  if (!enc || !ensure_context()) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)B, 3u, (cuuint64_t)nck};
+  cuuint64_t strides[3] = {(cuuint64_t)(C * 4), (cuuint64_t)(B * C * 4), (cuuint64_t)(3 * B * C * 4)};
+  cuuint32_t box[4] = {32u, 1u, 3u, (cuuint32_t)box_ck};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  if (enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float *>(ck), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  map_insert(key, *m);
+  return true;
+}
+
 // [BH, N, width] bfloat16 tensor as a 3-D map (width fastest), boxes of
 // width x 128 rows x 1 head in the 64-byte swizzle, which is the layout the
 // tensor cores read their operands in (width * 2 must be 64 bytes).  Rows

@@ -28,7 +28,7 @@ constexpr float kLn2 = 0.6931471805599453f;    // ln(2)
 constexpr float kEmptyP = -1.0e38f;
 // Scale of the empty adjoint (Ahat = ahat * 2^-r with r = +1e38).
 constexpr float kEmptyR = 1.0e38f;
-constexpr int kCkpt = 32;  // tokens between forward checkpoints
+constexpr int kCkpt = 16;  // tokens between forward checkpoints
 
 // -------------------------------------------------------------- launch ---
 // Launch with the launch's own status.  (A <<<...>>> launch followed by

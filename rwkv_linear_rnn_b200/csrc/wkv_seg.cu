@@ -21,7 +21,7 @@
 //   pass 2  stream the same rows again (they are still in L2: pass 1 loads
 //           with an evict-last hint, pass 2 with evict-first) and replay the
 //           recurrence from the joined state, writing y, the checkpoints at
-//           every 32-token boundary, and the final state.
+//           every 16-token boundary, and the final state.
 // Per token: pass 1 is one ex2 and ~8 FMA-pipe ops, pass 2 two ex2 + one rcp
 // and ~22 ops.  HBM traffic is the algorithmic 12 B (fp32) / 6 B (bf16) per
 // channel-token plus a 16-byte record per segment and lane.

@@ -579,13 +579,15 @@ static cudaError_t launch_bwd_seg_t(const BwdArgs &p, int dtype, float *gw, floa
     mw = (int64_t)occ * num_sms * kWarps;
     return occ < 1 ? cudaErrorInvalidConfiguration : cudaSuccess;
   };
-  // Segment length: the shortest multiple of the checkpoint interval (>= 64)
-  // that lets every segment have its own resident warp (barrier join, most
-  // warps); otherwise the longest (fewest joins per token).
+  // Segment length: the shortest multiple of 32 tokens (>= 64, whole
+  // checkpoint intervals) that lets every segment have its own resident
+  // warp (barrier join, most warps); otherwise the longest (fewest joins
+  // per token).
+  static_assert(32 % kCkpt == 0, "segments start on checkpoints");
   int ts = ts_max, smem = 0;
   int64_t max_warps = 0;
   bool fits = false;
-  for (int cand = 2 * kCkpt; cand <= ts_max; cand += kCkpt) {
+  for (int cand = 64; cand <= ts_max; cand += 32) {
     int sm = 0;
     int64_t mw = 0;
     cudaError_t e = max_warps_for(cand, sm, mw);

@@ -24,7 +24,7 @@
 //           chain start, whoever computes it: results are bit-reproducible;
 //   pass 2  the recurrence replayed from the joined state over the resident
 //           tile; y overwrites k in shared memory and leaves by one TMA store;
-//           checkpoints every 32 tokens and the final state are written.
+//           checkpoints every 16 tokens and the final state are written.
 // HBM traffic is the algorithmic 12 B (fp32) / 6 B (bf16) per channel-token
 // plus two 16-byte records per unit and lane.
 #include <cuda.h>

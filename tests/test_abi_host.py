@@ -46,7 +46,7 @@ def test_every_declared_symbol_is_exported(W):
 
 
 def test_version_and_strerror(W):
-    assert W.wkv_version() == 130
+    assert W.wkv_version() == 140
     for code in range(0, -6, -1):
         assert W.wkv_strerror(code) != "unknown status"
     assert W.wkv_strerror(7) == "unknown status"
@@ -54,7 +54,7 @@ def test_version_and_strerror(W):
 
 def test_sizes(W):
     B, T, C = 8, 1024, 768
-    assert W.wkv_ckpt_size(B, T, C) == 4 * 3 * B * C * (T // 32)  # a checkpoint every 32 tokens
+    assert W.wkv_ckpt_size(B, T, C) == 4 * 3 * B * C * (T // 16)  # a checkpoint every 16 tokens
     assert W.wkv_workspace_size(W.WKV_OP_STEP, B, T, C, 0) == 0
     f = W.wkv_workspace_size(W.WKV_OP_FORWARD, B, T, C, 0)
     b = W.wkv_workspace_size(W.WKV_OP_BACKWARD, B, T, C, 0)
