@@ -366,7 +366,7 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *map, int x
 // and are the batch-start states as they are; no forward pass over the
 // unit precedes its sweep.
 template <typename E, int L, int RB, int S>
-__global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                         const __grid_constant__ CUtensorMap vmap,
                                                                         const __grid_constant__ CUtensorMap gmap,
                                                                         const __grid_constant__ CUtensorMap ckmap,
@@ -376,40 +376,42 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
   static_assert(L % kCkpt == 0 && RB == kCkpt, "batches are checkpoint intervals");
   constexpr int NB = L / RB;
   constexpr int CKB = NB * 96 * 4;  // the unit's checkpoints
-  using Lay = ChainLayout<E, L, 3, 2, S, 0, CKB>;
+  using Lay = ChainLayout<E, L, 3, 0, S, 0, CKB>;  // dL/dk, dL/dv overwrite k, v in the stage
   const BwdArgs &p = a.p;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned char *wbuf = smem + (size_t)wl * Lay::WARP;
-  unsigned char *obuf = wbuf + S * Lay::STAGE;
-  const uint32_t bar0 = smem_addr(smem + (size_t)kChainWarps * Lay::WARP) + 8u * S * wl;
-  if (lane == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1);
+  // per compute warp w: full[S] (its stages landed), done[S] (it is done
+  // with a stage and its outputs are in it)
+  const uint32_t barb = smem_addr(smem + (size_t)kChainWarps * Lay::WARP);
+  auto full = [&](int w, int s) { return barb + 8u * (2 * S * w + s); };
+  auto done = [&](int w, int s) { return barb + 8u * (2 * S * w + S + s); };
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * S * kChainWarps; ++i) mbar_init(barb + 8u * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  __syncwarp();
+  __syncthreads();
   const int G = (int)gridDim.x * kChainWarps;
-  const int g = (int)blockIdx.x * kChainWarps + wl;
   const int nchains = (int)p.nchains, nct = (int)p.nct;
   const int64_t T = p.T, C = p.C;
   const int nseg = (int)((T + L - 1) / L);
-  const int nmine = nchains > g ? (nchains - g + G - 1) / G : 0;  // chains of this warp
-  const int total = nmine * nseg;                                 // units of this warp
   const int64_t budget = p.spin_limit * 1000;
   unsigned epoch = 0;
   if (lane == 0) epoch = ld_relaxed(&p.hdr->epoch);
   epoch = __shfl_sync(0xffffffffu, epoch, 0);
   const unsigned t_sum = tile_flag(epoch, 3u);
-  const uint64_t pol = l2_policy_evict_first();
-
-  // unit j of this warp: chain g + (j / nseg) G, position nseg - 1 - j % nseg,
-  // followed by cursors (no divisions in the unit loop)
+  // units of compute warp w: chain gw + (j / nseg) G, position
+  // nseg - 1 - j % nseg, followed by cursors (no divisions in the unit loop)
+  auto units_of = [&](int w) {
+    const int gw = (int)blockIdx.x * kChainWarps + w;
+    return (nchains > gw ? (nchains - gw + G - 1) / G : 0) * nseg;
+  };
   struct Cursor {
     int chain, pos, b, x0;
   };
-  auto first = [&]() {
-    Cursor u{g, nseg - 1, g / nct, 0};
-    u.x0 = (g - u.b * nct) * 32;
+  auto first = [&](int w) {
+    const int gw = (int)blockIdx.x * kChainWarps + w;
+    Cursor u{gw, nseg - 1, gw / nct, 0};
+    u.x0 = (gw - u.b * nct) * 32;
     return u;
   };
   auto next = [&](Cursor &u) {
@@ -420,23 +422,84 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
       u.x0 = (u.chain - u.b * nct) * 32;
     }
   };
-  Cursor ic = first();  // the next unit to load
-  auto issue = [&](int j) {
-    const int s = j % S;
-    const uint32_t dst = smem_addr(wbuf + (size_t)s * Lay::STAGE), bar = bar0 + 8u * s;
-    mbar_expect_tx(bar, (uint32_t)Lay::STAGE);
-    tma_load_3d(dst, &kmap, ic.x0, ic.pos * L, ic.b, bar, pol);
-    tma_load_3d(dst + Lay::ARR, &vmap, ic.x0, ic.pos * L, ic.b, bar, pol);
-    tma_load_3d(dst + 2 * Lay::ARR, &gmap, ic.x0, ic.pos * L, ic.b, bar, pol);
-    tma_load_4d(dst + 3 * Lay::ARR, &ckmap, ic.x0, ic.b, 0, ic.pos * NB, bar, pol);
-    next(ic);
-  };
-  int issued = -1, landed = -1;
-  if (lane == 0)
-    for (int j = 0; j < S && j < total; ++j) {
-      issue(j);
-      issued = j;
+  auto stage = [&](int w, int s) { return smem + (size_t)w * Lay::WARP + (size_t)s * Lay::STAGE; };
+
+  if (wl == kChainWarps) {
+    // ------------------------------------------------------ the TMA warp
+    // Issues every copy of the block's compute warps, so that none of them
+    // waits on a copy instruction: each warp's first S units, then round by
+    // round (unit j of every warp): the stores of dL/dk and dL/dv from the
+    // stages the warps are done with, and, once those stores have read
+    // them, the loads of units j + S into the same stages.
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      Cursor ic[kChainWarps], sc[kChainWarps];  // the next unit to load, to store
+      int tot[kChainWarps], maxtot = 0;
+      for (int w = 0; w < kChainWarps; ++w) {
+        ic[w] = sc[w] = first(w);
+        tot[w] = units_of(w);
+        maxtot = max(maxtot, tot[w]);
+      }
+      auto load = [&](int w, int j) {
+        const int s = j % S;
+        const uint32_t dst = smem_addr(stage(w, s)), bar = full(w, s);
+        mbar_expect_tx(bar, (uint32_t)Lay::STAGE);
+        const Cursor &u = ic[w];
+        tma_load_3d(dst, &kmap, u.x0, u.pos * L, u.b, bar, pol);
+        tma_load_3d(dst + Lay::ARR, &vmap, u.x0, u.pos * L, u.b, bar, pol);
+        tma_load_3d(dst + 2 * Lay::ARR, &gmap, u.x0, u.pos * L, u.b, bar, pol);
+        tma_load_4d(dst + 3 * Lay::ARR, &ckmap, u.x0, u.b, 0, u.pos * NB, bar, pol);
+        next(ic[w]);
+      };
+      int issued[kChainWarps];
+      for (int w = 0; w < kChainWarps; ++w) {
+        issued[w] = -1;
+        for (int j = 0; j < S && j < tot[w]; ++j) {
+          load(w, j);
+          issued[w] = j;
+        }
+      }
+      bool failed = false;
+      for (int j = 0; j < maxtot && !failed; ++j) {
+        const int s = j % S;
+        for (int w = 0; w < kChainWarps; ++w) {
+          if (j >= tot[w]) continue;
+          if (!mbar_wait(done(w, s), (uint32_t)(j / S) & 1u, budget, nullptr)) {
+            raise_timeout(p.hdr, epoch);
+            failed = true;
+            break;
+          }
+          const uint32_t src = smem_addr(stage(w, s));
+          tma_store_3d(&gkmap, sc[w].x0, sc[w].pos * L, sc[w].b, src);
+          tma_store_3d(&gvmap, sc[w].x0, sc[w].pos * L, sc[w].b, src + Lay::ARR);
+          next(sc[w]);
+        }
+        bulk_commit();
+        bulk_wait_read_all();  // this round's stores are done with their stages
+        if (failed) break;
+        for (int w = 0; w < kChainWarps; ++w)
+          if (j + S < tot[w]) {
+            load(w, j + S);
+            issued[w] = j + S;
+          }
+      }
+      bulk_wait_all();  // every store complete before the block exits
+      if (failed) {
+        // every issued load lands before the block exits (each warp's
+        // stages in order; those it consumed have completed already)
+        for (int w = 0; w < kChainWarps; ++w)
+          for (int j = max(0, issued[w] - S + 1); j <= issued[w]; ++j)
+            mbar_wait(full(w, j % S), (uint32_t)(j / S) & 1u, budget, nullptr);
+      }
     }
+    __syncthreads();
+    finish_block(p.hdr, gridDim.x);
+    return;
+  }
+
+  // -------------------------------------------------------- compute warps
+  const int total = units_of(wl);
+  unsigned char *const wbuf = stage(wl, 0);
   bool failed = false;
   int b = 0, x0 = 0;
   int64_t c = 0, bc = 0;
@@ -445,7 +508,7 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
   FastC fc{};
   float rah = 0.f, rhh = 0.f, rahp = 0.f, rhhp = 0.f, Ranc = kEmptyR, m = 0.f;
   double gw_d = 0.0, gu_d = 0.0;
-  Cursor uc = first();
+  Cursor uc = first(wl);
 #pragma unroll 1
   for (int j = 0; j < total; ++j, next(uc)) {
     const int s = j % S;
@@ -465,12 +528,11 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
       m = 0.f;
       gw_d = gu_d = 0.0;
     }
-    if (!failed && !__all_sync(0xffffffffu, mbar_wait(bar0 + 8u * s, (uint32_t)(j / S) & 1u, budget, nullptr))) {
+    if (!__all_sync(0xffffffffu, mbar_wait(full(wl, s), (uint32_t)(j / S) & 1u, budget, nullptr))) {
       failed = true;
       if (lane == 0) raise_timeout(p.hdr, epoch);
+      break;
     }
-    if (failed) break;
-    landed = j;
     const int64_t t0 = (int64_t)pos * L;
     const int n = (int)min((int64_t)L, T - t0);
     const E *kt = reinterpret_cast<const E *>(wbuf + (size_t)s * Lay::STAGE) + lane;
@@ -488,11 +550,11 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
     // the batch-start states: the unit's checkpoints ([NB][3][32] floats)
     const float *sts = reinterpret_cast<const float *>(wbuf + (size_t)s * Lay::STAGE + 3 * Lay::ARR);
 
-    // ---- pass 2: batches last to first, recompute then reverse sweep
-    if (lane == 0) bulk_wait_read_1();  // the stores of unit j-2 are done with this staging buffer
-    __syncwarp();
-    E *okp = reinterpret_cast<E *>(obuf + (size_t)(j & 1) * Lay::OUT) + lane;
-    E *ovp = okp + L * 32;
+    // ---- batches last to first, recompute then reverse sweep; dL/dk and
+    // dL/dv overwrite k and v of the stage (a batch's k and v are in
+    // registers before its sweep writes them)
+    E *okp = const_cast<E *>(kt);
+    E *ovp = const_cast<E *>(vt);
     float gw_acc = 0.f, gu_acc = 0.f;
 #pragma unroll 1
     for (int bi = 0; bi < NB; ++bi) {
@@ -562,11 +624,6 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
         m = reset ? 0.f : m1;
       }
     }
-    __syncwarp();  // every lane is done with stage s
-    if (lane == 0 && j + S < total) {
-      issue(j + S);
-      issued = j + S;
-    }
     if (pos == 0 && cok) {
       // share of the initial state A_0, B_0 (zero for the empty state): the
       // checkpoint before token 0
@@ -577,12 +634,7 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
     gu_d += (double)gu_acc;
     fence_proxy_async_smem();  // dL/dk, dL/dv before the async proxy reads them
     __syncwarp();
-    if (lane == 0) {
-      const uint32_t src = smem_addr(obuf + (size_t)(j & 1) * Lay::OUT);
-      tma_store_3d(&gkmap, x0, (int)t0, b, src);
-      tma_store_3d(&gvmap, x0, (int)t0, b, src + Lay::ARR);
-      bulk_commit();
-    }
+    if (lane == 0) mbar_arrive(done(wl, s));  // the TMA warp stores them and reloads the stage
     if (pos == 0 && cok) {
       // the chain's sums, then (last batch row) the B chains in batch-row order
       st_relaxed_v4(a.chain_sum + bc, make_float4((float)gw_d, (float)gu_d, tagf(t_sum), 0.f));
@@ -593,11 +645,6 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) bwd_chain_kernel(const __
         a.gu[c] = (float)su;
       }
     }
-  }
-  if (lane == 0) {
-    bulk_wait_all();
-    for (int j = landed + 1; j <= issued; ++j)
-      mbar_wait(bar0 + 8u * (j % S), (uint32_t)(j / S) & 1u, budget, nullptr);
   }
   __syncthreads();
   finish_block(p.hdr, gridDim.x);
@@ -644,11 +691,12 @@ static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, fl
       !encode_btc(&gvm, p.gv, dtype, p.B, p.T, p.C, L) ||
       !encode_ckpt(&ckm, p.ckpt, p.B, p.C, (p.T + kCkpt - 1) / kCkpt, NB))
     return cudaErrorInvalidValue;
-  constexpr int S = 3;
-  constexpr int smem = ChainLayout<E, L, 3, 2, S, 0, NB * 96 * 4>::bytes(kChainWarps);
+  constexpr int S = 4;
+  // the compute warps' stages, then two barriers per stage and warp
+  constexpr int smem = kChainWarps * (ChainLayout<E, L, 3, 0, S, 0, NB * 96 * 4>::WARP + 16 * S);
   auto kern = bwd_chain_kernel<E, L, RB, S>;
   int occ = 0;
-  cudaError_t e = blocks_per_sm((const void *)kern, kChainWarps * 32, smem, &occ);
+  cudaError_t e = blocks_per_sm((const void *)kern, (kChainWarps + 1) * 32, smem, &occ);
   if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   const int64_t nseg = (p.T + L - 1) / L;
@@ -664,7 +712,7 @@ static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, fl
   a.gu = gu;
   a.chain_sum = chain_sum;
   void *args[] = {&km, &vm, &gm, &ckm, &gkm, &gvm, &a};
-  return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3(kChainWarps * 32), args,
+  return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3((kChainWarps + 1) * 32), args,
                                      (size_t)smem, st);
 }
 
