@@ -46,7 +46,7 @@ bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T
 bool encode_ckpt(CUtensorMap *m, const float *ck, int64_t B, int64_t C, int64_t nck, int box_ck);
 
 constexpr int kChainWarps = 4;  // warps per block: one per scheduler
-constexpr int kChainStages = 4;  // units of input in flight per warp
+constexpr int kChainStages = 6;  // units of input in flight per warp (forward)
 
 // Largest and smallest of n values as balanced trees: log2(n) dependent
 // steps instead of n (with one warp per scheduler, dependent chains are
@@ -123,27 +123,92 @@ struct ChainLayout {
 
 // ------------------------------------------------------------- forward ---
 template <typename E, int L, int RB, int S, bool GATE>
-__global__ void __launch_bounds__(kChainWarps * 32, 1) fwd_chain_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) fwd_chain_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                         const __grid_constant__ CUtensorMap vmap,
                                                                         const __grid_constant__ CUtensorMap rmap,
                                                                         const __grid_constant__ CUtensorMap ymap,
                                                                         FwdArgs p) {
   static_assert(L % RB == 0 && RB % kCkpt == 0, "batches hold whole checkpoint intervals");
   constexpr int NARR = GATE ? 3 : 2;
-  using Lay = ChainLayout<E, L, NARR, 1, S, 0>;
+  using Lay = ChainLayout<E, L, NARR, 0, S, 0>;  // y overwrites k in the stage
   extern __shared__ __align__(1024) unsigned char smem[];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned char *wbuf = smem + (size_t)wl * Lay::WARP;
-  unsigned char *ybuf = wbuf + S * Lay::STAGE;
-  const uint32_t bar0 = smem_addr(smem + (size_t)kChainWarps * Lay::WARP) + 8u * S * wl;
-  if (lane == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1);
+  // per compute warp w: full[S] (its stages landed), done[S] (it is done
+  // with a stage and y is in it)
+  const uint32_t barb = smem_addr(smem + (size_t)kChainWarps * Lay::WARP);
+  auto full = [&](int w, int s) { return barb + 8u * (2 * S * w + s); };
+  auto done = [&](int w, int s) { return barb + 8u * (2 * S * w + S + s); };
+  auto stage = [&](int w, int s) { return smem + (size_t)w * Lay::WARP + (size_t)s * Lay::STAGE; };
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * S * kChainWarps; ++i) mbar_init(barb + 8u * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  __syncwarp();
+  __syncthreads();
+  const int64_t T = p.T, C = p.C, BC = p.B * p.C;
+  const int nseg = (int)((T + L - 1) / L);
+  const int64_t budget = p.spin_limit * 1000;
+  unsigned epoch = 0;
+  if (lane == 0) epoch = ld_relaxed(&p.hdr->epoch);
+  epoch = __shfl_sync(0xffffffffu, epoch, 0);
+
+  if (wl == kChainWarps) {
+    // ------------------------------------------------------ the TMA warp
+    // Every copy of the block's compute warps: their first S units, then
+    // round by round (unit t of every warp) the y stores from the stages
+    // they are done with and, once those have read them, the loads of unit
+    // t + S into the same stages.
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();  // inputs are read once
+      int nw = 0;
+      int xw[kChainWarps], bw[kChainWarps];
+      for (int w = 0; w < kChainWarps; ++w) {
+        const int64_t ch = (int64_t)blockIdx.x * kChainWarps + w;
+        if (ch < p.nchains) {
+          bw[w] = (int)(ch / p.nct);
+          xw[w] = (int)(ch - (int64_t)bw[w] * p.nct) * 32;
+          nw = w + 1;
+        }
+      }
+      auto load = [&](int w, int t) {
+        const int s = t % S;
+        const uint32_t dst = smem_addr(stage(w, s)), bar = full(w, s);
+        mbar_expect_tx(bar, (uint32_t)Lay::STAGE);
+        tma_load_3d(dst, &kmap, xw[w], t * L, bw[w], bar, pol);
+        tma_load_3d(dst + Lay::ARR, &vmap, xw[w], t * L, bw[w], bar, pol);
+        if constexpr (GATE) tma_load_3d(dst + 2 * Lay::ARR, &rmap, xw[w], t * L, bw[w], bar, pol);
+      };
+      for (int w = 0; w < nw; ++w)
+        for (int t = 0; t < S && t < nseg; ++t) load(w, t);
+      int issued = min(S, nseg) - 1;
+      bool failed = false;
+      for (int t = 0; t < nseg && !failed; ++t) {
+        const int s = t % S;
+        for (int w = 0; w < nw; ++w) {
+          if (!mbar_wait(done(w, s), (uint32_t)(t / S) & 1u, budget, nullptr)) {
+            raise_timeout(p.hdr, epoch);
+            failed = true;
+            break;
+          }
+          if (p.y) tma_store_3d(&ymap, xw[w], t * L, bw[w], smem_addr(stage(w, s)));
+        }
+        bulk_commit();
+        bulk_wait_read_all();  // this round's stores are done with their stages
+        if (failed || t + S >= nseg) continue;
+        for (int w = 0; w < nw; ++w) load(w, t + S);
+        issued = t + S;
+      }
+      bulk_wait_all();  // every y store complete before the block exits
+      if (failed)       // and every issued load landed
+        for (int w = 0; w < nw; ++w)
+          for (int t = max(0, issued - S + 1); t <= issued; ++t)
+            mbar_wait(full(w, t % S), (uint32_t)(t / S) & 1u, budget, nullptr);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------- compute warps
   const int64_t chain = (int64_t)blockIdx.x * kChainWarps + wl;
   if (chain >= p.nchains) return;  // warp-uniform; no block-wide barrier follows
-  const int64_t T = p.T, C = p.C, BC = p.B * p.C;
   const int b = (int)(chain / p.nct);
   const int x0 = (int)(chain - (int64_t)b * p.nct) * 32;
   const int64_t c = (int64_t)x0 + lane;
@@ -151,45 +216,22 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) fwd_chain_kernel(const __
   const int64_t bc = (int64_t)b * C + c;
   const float w = cok ? __ldg(p.w + c) : 0.f, u = cok ? __ldg(p.u + c) : 0.f;
   const float w2 = w * kLog2e, u2 = u * kLog2e;
-  const int nseg = (int)((T + L - 1) / L);
-  const int64_t budget = p.spin_limit * 1000;
-  unsigned epoch = 0;
-  if (lane == 0) epoch = ld_relaxed(&p.hdr->epoch);
-  epoch = __shfl_sync(0xffffffffu, epoch, 0);
-  const uint64_t pol = l2_policy_evict_first();  // inputs are read once
-
-  auto issue = [&](int t) {
-    const int s = t % S;
-    const uint32_t dst = smem_addr(wbuf + (size_t)s * Lay::STAGE), bar = bar0 + 8u * s;
-    mbar_expect_tx(bar, (uint32_t)Lay::STAGE);
-    tma_load_3d(dst, &kmap, x0, t * L, b, bar, pol);
-    tma_load_3d(dst + Lay::ARR, &vmap, x0, t * L, b, bar, pol);
-    if constexpr (GATE) tma_load_3d(dst + 2 * Lay::ARR, &rmap, x0, t * L, b, bar, pol);
-  };
-  int issued = -1, landed = -1;
-  if (lane == 0)
-    for (int t = 0; t < S && t < nseg; ++t) {
-      issue(t);
-      issued = t;
-    }
+  unsigned char *const wbuf = stage(wl, 0);
   Run st = run_from(cok ? load_state_in(p.state_in, bc, BC) : st_empty());
   const TileFast fc = tile_fast<RB>(w, w2, u2);
   bool failed = false;
 #pragma unroll 1
   for (int t = 0; t < nseg; ++t) {
     const int s = t % S;
-    if (!__all_sync(0xffffffffu, mbar_wait(bar0 + 8u * s, (uint32_t)(t / S) & 1u, budget, nullptr))) {
+    if (!__all_sync(0xffffffffu, mbar_wait(full(wl, s), (uint32_t)(t / S) & 1u, budget, nullptr))) {
       failed = true;
       if (lane == 0) raise_timeout(p.hdr, epoch);
       break;
     }
-    landed = t;
-    if (lane == 0) bulk_wait_read_1();  // the y store of unit t-2 is done with its buffer
-    __syncwarp();
     const E *ks = reinterpret_cast<const E *>(wbuf + (size_t)s * Lay::STAGE) + lane;
     const E *vs = ks + L * 32;
     const E *rs = ks + 2 * L * 32;
-    E *ys = reinterpret_cast<E *>(ybuf + (size_t)(t & 1) * Lay::ARR) + lane;
+    E *ys = const_cast<E *>(ks);  // y overwrites k (a batch's keys are in registers before its y is written)
     const int64_t t0 = (int64_t)t * L;
     const int n = (int)min((int64_t)L, T - t0);
 #pragma unroll 1
@@ -267,25 +309,11 @@ __global__ void __launch_bounds__(kChainWarps * 32, 1) fwd_chain_kernel(const __
         }
       }
     }
-    __syncwarp();  // every lane is done with stage s
-    if (lane == 0 && t + S < nseg) {
-      issue(t + S);
-      issued = t + S;
-    }
     fence_proxy_async_smem();  // y before the async proxy reads it
     __syncwarp();
-    if (lane == 0 && p.y) {
-      tma_store_3d(&ymap, x0, (int)t0, b, smem_addr(ybuf + (size_t)(t & 1) * Lay::ARR));
-      bulk_commit();
-    }
+    if (lane == 0) mbar_arrive(done(wl, s));  // the TMA warp stores y and reloads the stage
   }
   if (!failed && p.state_out && cok) store_state(p.state_out, bc, BC, run_state(st), w2);
-  if (lane == 0) {
-    bulk_wait_all();  // every y store complete before the warp exits
-    for (int t = landed + 1; t <= issued; ++t)  // and every issued load landed (after a failure)
-      mbar_wait(bar0 + 8u * (t % S), (uint32_t)(t / S) & 1u, budget, nullptr);
-  }
-  __syncwarp();
 }
 
 // ------------------------------------------------------------ backward ---
@@ -660,17 +688,19 @@ static cudaError_t launch_fwd_chain_t(const FwdArgs &f, int dtype, cudaStream_t 
   ym = km;  // unused placeholders when there is no gate / no y
   if (GATE && !encode_btc(&rm, f.r, dtype, f.B, f.T, f.C, L)) return cudaErrorInvalidValue;
   if (f.y && !encode_btc(&ym, f.y, dtype, f.B, f.T, f.C, L)) return cudaErrorInvalidValue;
-  constexpr int S = GATE ? 3 : kChainStages;
-  constexpr int smem = ChainLayout<E, L, GATE ? 3 : 2, 1, S, 0>::bytes(kChainWarps);
+  constexpr int S = GATE ? 4 : kChainStages;
+  // the compute warps' stages, then two barriers per stage and warp
+  constexpr int smem = kChainWarps * (ChainLayout<E, L, GATE ? 3 : 2, 0, S, 0>::WARP + 16 * S);
   auto kern = fwd_chain_kernel<E, L, RB, S, GATE>;
   int occ = 0;
-  cudaError_t e = blocks_per_sm((const void *)kern, kChainWarps * 32, smem, &occ);
+  cudaError_t e = blocks_per_sm((const void *)kern, (kChainWarps + 1) * 32, smem, &occ);
   if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   if ((f.T + L - 1) / L >= (int64_t)1 << 31 || f.T >= (int64_t)1 << 31) return cudaErrorInvalidValue;
   const int64_t grid = (f.nchains + kChainWarps - 1) / kChainWarps;
   if (grid >= (int64_t)1 << 31) return cudaErrorInvalidValue;
-  return launch_kernel(kern, dim3((unsigned)grid), dim3(kChainWarps * 32), (size_t)smem, st, km, vm, rm, ym, f);
+  return launch_kernel(kern, dim3((unsigned)grid), dim3((kChainWarps + 1) * 32), (size_t)smem, st, km, vm, rm, ym,
+                       f);
 }
 
 cudaError_t launch_forward_chain(const FwdArgs &f, int dtype, cudaStream_t st) {
