@@ -101,15 +101,15 @@ KERNEL_SOURCES = {
 # (workload, kernel, gated, hash of the kernel's code).  A kernel whose code changed
 # since its capture has no entry: its traffic is reported as null.
 TRAFFIC = {
-    ("rwkv1b5_bf16", "bwd_chain_kernel", False, "82881209cade8efe"): 427_978_752 + 211_177_216,
-    ("rwkv1b5_bf16", "fwd_chain_kernel", False, "0db41f984c0c885b"): 268_591_616 + 104_592_896,
-    ("rwkv169m", "bwd_seg_kernel", False, "c5e242ca4e035480"): 77_597_952 + 529_152,
-    ("rwkv169m", "fwd_seg_kernel", False, "1edb76594a20115c"): 50_392_064 + 1_318_400,
-    ("longctx", "fwd_seg_kernel", False, "1edb76594a20115c"): 1_463_432_192 + 639_096_320,
-    ("decode14b", "step_kernel", False, "21aab8ba04a9606b"): 52_483_344 + 71_440,
+    ("rwkv1b5_bf16", "bwd_chain_kernel", False, "3d1d96462ca9c9e8"): 453_308_160 + 211_563_520,
+    ("rwkv1b5_bf16", "fwd_chain_kernel", False, "537462e38304278c"): 268_545_536 + 130_038_528,
+    ("rwkv169m", "bwd_seg_kernel", False, "f3ee2d2581da2ffd"): 77_673_472 + 485_376,
+    ("rwkv169m", "fwd_seg_kernel", False, "fbcb48b606b747e2"): 50_391_552 + 1_572_608,
+    ("longctx", "fwd_seg_kernel", False, "fbcb48b606b747e2"): 1_454_121_728 + 638_856_704,
+    ("decode14b", "step_kernel", False, "5da4a196be76b807"): (1_679_439_616 + 4_633_856) // 32,
     # the three launches of one linattn_backward_saved call
-    ("la_cifar_b32", "linattn_backward_saved", False, "af5c298cf6a97dd3"): (154_172_672 + 25_963_008 + 256_456_704
-                                                                           + 27_880_448 + 107_828_224),
+    ("la_cifar_b32", "linattn_backward_saved", False, "d137bd8b0b6bb8ce"): (154_165_248 + 27_663_616 + 25_963_008
+                                                                           + 256_460_288 + 107_953_408),
 }
 
 

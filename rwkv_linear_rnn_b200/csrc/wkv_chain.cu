@@ -37,7 +37,18 @@
 
 // Tokens per batch of the fast paths (build-time knobs).
 #ifndef WKV_CHAIN_FRB
-#define WKV_CHAIN_FRB 32
+#define WKV_CHAIN_FRB 64
+#endif
+// Tokens per bf16 unit of the forward and backward, and TMA stages per warp
+// of the backward (the forward takes as many as 48 KB of input per warp hold).
+#ifndef WKV_CHAIN_LF
+#define WKV_CHAIN_LF 128
+#endif
+#ifndef WKV_CHAIN_LB
+#define WKV_CHAIN_LB 128
+#endif
+#ifndef WKV_CHAIN_SB
+#define WKV_CHAIN_SB 2
 #endif
 
 namespace wkv {
@@ -46,7 +57,10 @@ bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T
 bool encode_ckpt(CUtensorMap *m, const float *ck, int64_t B, int64_t C, int64_t nck, int box_ck);
 
 constexpr int kChainWarps = 4;  // warps per block: one per scheduler
-constexpr int kChainStages = 6;  // units of input in flight per warp (forward)
+// tokens per forward batch: at most a unit (32 tokens for fp32), and at
+// most 32 with the gate (its third input array in registers)
+constexpr int kFrbF32 = WKV_CHAIN_FRB < kTileLF32 ? WKV_CHAIN_FRB : kTileLF32;
+constexpr int kChainFwdBytes = 48 * 1024;  // input stages per warp of the forward
 
 // Largest and smallest of n values as balanced trees: log2(n) dependent
 // steps instead of n (with one warp per scheduler, dependent chains are
@@ -688,7 +702,8 @@ static cudaError_t launch_fwd_chain_t(const FwdArgs &f, int dtype, cudaStream_t 
   ym = km;  // unused placeholders when there is no gate / no y
   if (GATE && !encode_btc(&rm, f.r, dtype, f.B, f.T, f.C, L)) return cudaErrorInvalidValue;
   if (f.y && !encode_btc(&ym, f.y, dtype, f.B, f.T, f.C, L)) return cudaErrorInvalidValue;
-  constexpr int S = GATE ? 4 : kChainStages;
+  constexpr int STG = (GATE ? 3 : 2) * L * 32 * (int)sizeof(E);
+  constexpr int S = kChainFwdBytes / STG > 2 ? kChainFwdBytes / STG : 2;
   // the compute warps' stages, then two barriers per stage and warp
   constexpr int smem = kChainWarps * (ChainLayout<E, L, GATE ? 3 : 2, 0, S, 0>::WARP + 16 * S);
   auto kern = fwd_chain_kernel<E, L, RB, S, GATE>;
@@ -705,10 +720,10 @@ static cudaError_t launch_fwd_chain_t(const FwdArgs &f, int dtype, cudaStream_t 
 
 cudaError_t launch_forward_chain(const FwdArgs &f, int dtype, cudaStream_t st) {
   if (f.r)
-    return dtype == 0 ? launch_fwd_chain_t<float, kTileLF32, WKV_CHAIN_FRB, true>(f, dtype, st)
-                      : launch_fwd_chain_t<uint16_t, kTileLBF16, WKV_CHAIN_FRB, true>(f, dtype, st);
-  return dtype == 0 ? launch_fwd_chain_t<float, kTileLF32, WKV_CHAIN_FRB, false>(f, dtype, st)
-                    : launch_fwd_chain_t<uint16_t, kTileLBF16, WKV_CHAIN_FRB, false>(f, dtype, st);
+    return dtype == 0 ? launch_fwd_chain_t<float, kTileLF32, kFrbF32, true>(f, dtype, st)
+                      : launch_fwd_chain_t<uint16_t, WKV_CHAIN_LF, kFrbF32, true>(f, dtype, st);
+  return dtype == 0 ? launch_fwd_chain_t<float, kTileLF32, kFrbF32, false>(f, dtype, st)
+                    : launch_fwd_chain_t<uint16_t, WKV_CHAIN_LF, WKV_CHAIN_FRB, false>(f, dtype, st);
 }
 
 template <typename E, int L, int RB>
@@ -721,7 +736,7 @@ static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, fl
       !encode_btc(&gvm, p.gv, dtype, p.B, p.T, p.C, L) ||
       !encode_ckpt(&ckm, p.ckpt, p.B, p.C, (p.T + kCkpt - 1) / kCkpt, NB))
     return cudaErrorInvalidValue;
-  constexpr int S = 4;
+  constexpr int S = WKV_CHAIN_SB;
   // the compute warps' stages, then two barriers per stage and warp
   constexpr int smem = kChainWarps * (ChainLayout<E, L, 3, 0, S, 0, NB * 96 * 4>::WARP + 16 * S);
   auto kern = bwd_chain_kernel<E, L, RB, S>;
@@ -750,7 +765,7 @@ cudaError_t launch_backward_chain(const BwdArgs &p, int dtype, float *gw, float 
                                   cudaStream_t st) {
   if (p.r || p.gs_out || p.gs_in) return cudaErrorInvalidValue;  // plain backward only
   return dtype == 0 ? launch_bwd_chain_t<float, kTileLF32, kCkpt>(p, dtype, gw, gu, chain_sum, num_sms, st)
-                    : launch_bwd_chain_t<uint16_t, kTileLBF16, kCkpt>(p, dtype, gw, gu, chain_sum, num_sms, st);
+                    : launch_bwd_chain_t<uint16_t, WKV_CHAIN_LB, kCkpt>(p, dtype, gw, gu, chain_sum, num_sms, st);
 }
 
 }  // namespace wkv
