@@ -122,18 +122,19 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
  *               units by a decoupled look-back over records that carry their
  *               own validity tags (no fences), and, in the forward, runs the
  *               next unit's first pass before the current unit's join.
- *               CHAIN (16-byte aligned rows; the backward without the gate
- *               and the state terms) gives each warp whole chains, run in
+ *               CHAIN (16-byte aligned rows; the backward without the
+ *               state terms) gives each warp whole chains, run in
  *               time order from a ring of TMA tiles with the state (or the
  *               adjoint) carried in registers: no joins and a single pass
  *               over every token, for problems whose chains alone fill the
  *               GPU's warp schedulers; where it does not apply, the call
- *               runs TILE (SEGMENT for the gate and state terms).  AUTO
- *               runs TILE on 16-byte aligned rows when a chain (batch row, 32
- *               channels) has at most about four resident warps' units in
- *               flight, SEGMENT otherwise, and the chunked kernels on
- *               unaligned rows.  Values 4 and 5 are retired and rejected
- *               with WKV_ERR_INVALID_ARG.
+ *               runs TILE.  AUTO runs CHAIN on 16-byte aligned rows when the
+ *               chains (batch rows x 32-channel tiles) number from three
+ *               quarters of to all the warp schedulers (4 per SM), else TILE
+ *               when a chain has at most about four resident warps' units in
+ *               flight, else SEGMENT, and the chunked kernels on unaligned
+ *               rows.  Values 4 and 5 are retired and rejected with
+ *               WKV_ERR_INVALID_ARG.
  *   spin_limit  bound on any one device-side wait (a predecessor's record,
  *               a shared-memory load, the grid barrier) in microseconds (the
  *               chunked kernels count polls of at most about 1 us each);

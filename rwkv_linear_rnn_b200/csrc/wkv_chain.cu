@@ -44,6 +44,9 @@
 #ifndef WKV_CHAIN_LF
 #define WKV_CHAIN_LF 128
 #endif
+#ifndef WKV_CHAIN_SLEEP
+#define WKV_CHAIN_SLEEP 500
+#endif
 #ifndef WKV_CHAIN_LB
 #define WKV_CHAIN_LB 128
 #endif
@@ -116,6 +119,22 @@ __device__ __forceinline__ void store2<uint16_t>(uint16_t *p0, uint16_t *p1, flo
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(x1), "f"(x0));  // x1 to the upper half
   *p0 = (uint16_t)(u & 0xffffu);
   *p1 = (uint16_t)(u >> 16);
+}
+
+// mbar_wait for the TMA warp, which shares a scheduler with a compute warp:
+// between polls it sleeps instead of spinning, leaving the issue slots to
+// the compute warp (the copies it then issues have stages of slack).
+__device__ __forceinline__ bool mbar_wait_sleepy(uint32_t bar, uint32_t parity, int64_t budget_ns) {
+#if WKV_CHAIN_SLEEP
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if ((int64_t)(global_ns() - t0) > budget_ns) return false;
+    __nanosleep(WKV_CHAIN_SLEEP);
+  }
+  return true;
+#else
+  return mbar_wait(bar, parity, budget_ns, nullptr);
+#endif
 }
 
 // Wait until at most one bulk store group of this thread still reads its
@@ -198,7 +217,7 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) fwd_chain_kernel(co
       for (int t = 0; t < nseg && !failed; ++t) {
         const int s = t % S;
         for (int w = 0; w < nw; ++w) {
-          if (!mbar_wait(done(w, s), (uint32_t)(t / S) & 1u, budget, nullptr)) {
+          if (!mbar_wait_sleepy(done(w, s), (uint32_t)(t / S) & 1u, budget)) {
             raise_timeout(p.hdr, epoch);
             failed = true;
             break;
@@ -337,13 +356,14 @@ struct ChainBwdArgs {
   float4 *chain_sum;  // [B][C] tagged per-chain sums of dL/dw, dL/du
 };
 
-// recompute_batch of wkv_bwd_math.cuh (without the gate's extra output),
-// with the batch maximum taken as a tree.
-template <int RB>
+// recompute_batch of wkv_bwd_math.cuh with the batch maximum taken as a
+// tree.  WY: Yw[j] is multiplied by the recomputed output y_j (the gated
+// backward's dL/dr = grad_o sigma'(r) y).
+template <int RB, bool WY>
 __device__ __forceinline__ bool chain_recompute(const float (&K)[RB], const float (&V)[RB], const float (&Gy)[RB],
                                                 float w2, float u2, const FastC &fc, float xa, float xb, float xP,
                                                 float (&qv)[RB], float (&gam)[RB], float (&eta)[RB],
-                                                float (&e2v)[RB], float &M) {
+                                                float (&e2v)[RB], float &M, float (&Yw)[RB]) {
   const float E0 = xP;
   float kj[RB];
   const bool ok = fast_prep_tree<RB>(K, E0, u2, fc.w2e, kj, M);
@@ -358,6 +378,7 @@ __device__ __forceinline__ bool chain_recompute(const float (&K)[RB], const floa
       const float y = fmaf(eu, V[j], al) * rden;
       gam[j] = Gy[j] * rden;
       eta[j] = gam[j] * y;
+      if constexpr (WY) Yw[j] *= y;
       e2v[j] = eu;
       al = fmaf(al, fc.ewm, ek * V[j]);
       be = fmaf(be, fc.ewm, ek);
@@ -378,6 +399,7 @@ __device__ __forceinline__ bool chain_recompute(const float (&K)[RB], const floa
     qv[j] = fmaxf(P, UK);
     gam[j] = Gy[j] * rden;
     eta[j] = gam[j] * y;
+    if constexpr (WY) Yw[j] *= y;
     e2v[j] = e2;
     const float n1 = xn + 1.f;
     const float Pc = fmaf(n1, w2, xP);
@@ -407,18 +429,25 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *map, int x
 // v and grad_y tiles (a fourth region of the stage, [L/RB][3][32] floats)
 // and are the batch-start states as they are; no forward pass over the
 // unit precedes its sweep.
-template <typename E, int L, int RB, int S>
+// GATE: the loss depends on o = sigma(r) * y and grad_y is dL/do (the tile
+// backward's gate, wkv_tile_bwd.cu): r arrives with k, v and grad_o, the
+// WKV gradient is grad_o sigma(r), and dL/dr = grad_o sigma'(r) y from the
+// recomputed y overwrites r and leaves with dL/dk and dL/dv.
+template <typename E, int L, int RB, int S, bool GATE>
 __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                         const __grid_constant__ CUtensorMap vmap,
                                                                         const __grid_constant__ CUtensorMap gmap,
+                                                                        const __grid_constant__ CUtensorMap rmap,
                                                                         const __grid_constant__ CUtensorMap ckmap,
                                                                         const __grid_constant__ CUtensorMap gkmap,
                                                                         const __grid_constant__ CUtensorMap gvmap,
+                                                                        const __grid_constant__ CUtensorMap grmap,
                                                                         ChainBwdArgs a) {
   static_assert(L % kCkpt == 0 && RB == kCkpt, "batches are checkpoint intervals");
   constexpr int NB = L / RB;
-  constexpr int CKB = NB * 96 * 4;  // the unit's checkpoints
-  using Lay = ChainLayout<E, L, 3, 0, S, 0, CKB>;  // dL/dk, dL/dv overwrite k, v in the stage
+  constexpr int NARR = GATE ? 4 : 3;  // k, v, grad_y (and r)
+  constexpr int CKB = NB * 96 * 4;    // the unit's checkpoints
+  using Lay = ChainLayout<E, L, NARR, 0, S, 0, CKB>;  // the gradients overwrite k, v (and r) in the stage
   const BwdArgs &p = a.p;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -490,7 +519,8 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
         tma_load_3d(dst, &kmap, u.x0, u.pos * L, u.b, bar, pol);
         tma_load_3d(dst + Lay::ARR, &vmap, u.x0, u.pos * L, u.b, bar, pol);
         tma_load_3d(dst + 2 * Lay::ARR, &gmap, u.x0, u.pos * L, u.b, bar, pol);
-        tma_load_4d(dst + 3 * Lay::ARR, &ckmap, u.x0, u.b, 0, u.pos * NB, bar, pol);
+        if constexpr (GATE) tma_load_3d(dst + 3 * Lay::ARR, &rmap, u.x0, u.pos * L, u.b, bar, pol);
+        tma_load_4d(dst + NARR * Lay::ARR, &ckmap, u.x0, u.b, 0, u.pos * NB, bar, pol);
         next(ic[w]);
       };
       int issued[kChainWarps];
@@ -506,7 +536,7 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
         const int s = j % S;
         for (int w = 0; w < kChainWarps; ++w) {
           if (j >= tot[w]) continue;
-          if (!mbar_wait(done(w, s), (uint32_t)(j / S) & 1u, budget, nullptr)) {
+          if (!mbar_wait_sleepy(done(w, s), (uint32_t)(j / S) & 1u, budget)) {
             raise_timeout(p.hdr, epoch);
             failed = true;
             break;
@@ -514,6 +544,7 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
           const uint32_t src = smem_addr(stage(w, s));
           tma_store_3d(&gkmap, sc[w].x0, sc[w].pos * L, sc[w].b, src);
           tma_store_3d(&gvmap, sc[w].x0, sc[w].pos * L, sc[w].b, src + Lay::ARR);
+          if constexpr (GATE) tma_store_3d(&grmap, sc[w].x0, sc[w].pos * L, sc[w].b, src + 3 * Lay::ARR);
           next(sc[w]);
         }
         bulk_commit();
@@ -580,17 +611,26 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
     const E *kt = reinterpret_cast<const E *>(wbuf + (size_t)s * Lay::STAGE) + lane;
     const E *vt = kt + L * 32;
     const E *gt = kt + 2 * L * 32;
-    auto load_batch = [&](int bt, float(&K)[RB], float(&V)[RB], float(&Gy)[RB]) {
+    E *rt = const_cast<E *>(kt) + 3 * L * 32;  // gate input, then dL/dr (GATE only)
+    // a batch's inputs; with the gate, Gy becomes grad_o sigma(r) and Gd
+    // grad_o sigma'(r) (times y once the recompute has formed it)
+    auto load_batch = [&](int bt, float(&K)[RB], float(&V)[RB], float(&Gy)[RB], float(&Gd)[RB]) {
 #pragma unroll
       for (int q = 0; q < RB; ++q) {
         K[q] = to_f32(kt[(bt * RB + q) * 32]) * kLog2e;
         V[q] = to_f32(vt[(bt * RB + q) * 32]);
         Gy[q] = to_f32(gt[(bt * RB + q) * 32]);
+        if constexpr (GATE) {
+          float sg, ds;
+          gate_sigmoid_slope(to_f32(rt[(bt * RB + q) * 32]), sg, ds);
+          Gd[q] = Gy[q] * ds;
+          Gy[q] *= sg;
+        }
       }
     };
 
     // the batch-start states: the unit's checkpoints ([NB][3][32] floats)
-    const float *sts = reinterpret_cast<const float *>(wbuf + (size_t)s * Lay::STAGE + 3 * Lay::ARR);
+    const float *sts = reinterpret_cast<const float *>(wbuf + (size_t)s * Lay::STAGE + NARR * Lay::ARR);
 
     // ---- batches last to first, recompute then reverse sweep; dL/dk and
     // dL/dv overwrite k and v of the stage (a batch's k and v are in
@@ -602,11 +642,18 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
     for (int bi = 0; bi < NB; ++bi) {
       const int bt = NB - 1 - bi;
       if (n - bt * RB <= 0) continue;  // only padding past T: nothing to sweep
-      float K[RB], V[RB], Gy[RB];
-      load_batch(bt, K, V, Gy);
+      float K[RB], V[RB], Gy[RB], Gd[RB];
+      load_batch(bt, K, V, Gy, Gd);
       float qv[RB], gam[RB], eta[RB], e2v[RB], Mb;
-      const bool fast = chain_recompute<RB>(K, V, Gy, w2, u2, fc, sts[bt * 96 + lane], sts[bt * 96 + 32 + lane],
-                                            sts[bt * 96 + 64 + lane], qv, gam, eta, e2v, Mb);
+      const bool fast = chain_recompute<RB, GATE>(K, V, Gy, w2, u2, fc, sts[bt * 96 + lane],
+                                                  sts[bt * 96 + 32 + lane], sts[bt * 96 + 64 + lane], qv, gam,
+                                                  eta, e2v, Mb, Gd);
+      if constexpr (GATE) {
+        // dL/dr over r (this batch's r is in registers already)
+#pragma unroll
+        for (int q = 0; q < RB; q += 2)
+          store2<E>(rt + (bt * RB + q) * 32, rt + (bt * RB + q + 1) * 32, Gd[q], Gd[q + 1]);
+      }
       E *gkp = okp + bt * RB * 32;
       E *gvp = ovp + bt * RB * 32;
       // the reverse sweep of the tile backward (wkv_tile_bwd.cu): fast in the
@@ -726,20 +773,23 @@ cudaError_t launch_forward_chain(const FwdArgs &f, int dtype, cudaStream_t st) {
                     : launch_fwd_chain_t<uint16_t, WKV_CHAIN_LF, WKV_CHAIN_FRB, false>(f, dtype, st);
 }
 
-template <typename E, int L, int RB>
+template <typename E, int L, int RB, int S, bool GATE>
 static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *chain_sum,
                                       int num_sms, cudaStream_t st) {
-  CUtensorMap km, vm, gm, ckm, gkm, gvm;
+  CUtensorMap km, vm, gm, rm, ckm, gkm, gvm, grm;
   constexpr int NB = L / RB;
   if (!encode_btc(&km, p.k, dtype, p.B, p.T, p.C, L) || !encode_btc(&vm, p.v, dtype, p.B, p.T, p.C, L) ||
       !encode_btc(&gm, p.gy, dtype, p.B, p.T, p.C, L) || !encode_btc(&gkm, p.gk, dtype, p.B, p.T, p.C, L) ||
       !encode_btc(&gvm, p.gv, dtype, p.B, p.T, p.C, L) ||
       !encode_ckpt(&ckm, p.ckpt, p.B, p.C, (p.T + kCkpt - 1) / kCkpt, NB))
     return cudaErrorInvalidValue;
-  constexpr int S = WKV_CHAIN_SB;
+  rm = gm;  // placeholders without the gate
+  grm = gkm;
+  if (GATE && (!encode_btc(&rm, p.r, dtype, p.B, p.T, p.C, L) || !encode_btc(&grm, p.gr, dtype, p.B, p.T, p.C, L)))
+    return cudaErrorInvalidValue;
   // the compute warps' stages, then two barriers per stage and warp
-  constexpr int smem = kChainWarps * (ChainLayout<E, L, 3, 0, S, 0, NB * 96 * 4>::WARP + 16 * S);
-  auto kern = bwd_chain_kernel<E, L, RB, S>;
+  constexpr int smem = kChainWarps * (ChainLayout<E, L, GATE ? 4 : 3, 0, S, 0, NB * 96 * 4>::WARP + 16 * S);
+  auto kern = bwd_chain_kernel<E, L, RB, S, GATE>;
   int occ = 0;
   cudaError_t e = blocks_per_sm((const void *)kern, (kChainWarps + 1) * 32, smem, &occ);
   if (e != cudaSuccess) return e;
@@ -756,16 +806,22 @@ static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, fl
   a.gw = gw;
   a.gu = gu;
   a.chain_sum = chain_sum;
-  void *args[] = {&km, &vm, &gm, &ckm, &gkm, &gvm, &a};
+  void *args[] = {&km, &vm, &gm, &rm, &ckm, &gkm, &gvm, &grm, &a};
   return cudaLaunchCooperativeKernel((const void *)kern, dim3((unsigned)grid), dim3((kChainWarps + 1) * 32), args,
                                      (size_t)smem, st);
 }
 
 cudaError_t launch_backward_chain(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *chain_sum, int num_sms,
                                   cudaStream_t st) {
-  if (p.r || p.gs_out || p.gs_in) return cudaErrorInvalidValue;  // plain backward only
-  return dtype == 0 ? launch_bwd_chain_t<float, kTileLF32, kCkpt>(p, dtype, gw, gu, chain_sum, num_sms, st)
-                    : launch_bwd_chain_t<uint16_t, WKV_CHAIN_LB, kCkpt>(p, dtype, gw, gu, chain_sum, num_sms, st);
+  if (p.gs_out || p.gs_in) return cudaErrorInvalidValue;  // no state terms
+  if (p.r)  // the gate's fourth tile per stage: 64-token units (32 fp32), three stages
+    return dtype == 0
+               ? launch_bwd_chain_t<float, kTileLF32, kCkpt, 3, true>(p, dtype, gw, gu, chain_sum, num_sms, st)
+               : launch_bwd_chain_t<uint16_t, kTileLBF16, kCkpt, 3, true>(p, dtype, gw, gu, chain_sum, num_sms, st);
+  return dtype == 0
+             ? launch_bwd_chain_t<float, kTileLF32, kCkpt, WKV_CHAIN_SB, false>(p, dtype, gw, gu, chain_sum, num_sms, st)
+             : launch_bwd_chain_t<uint16_t, WKV_CHAIN_LB, kCkpt, WKV_CHAIN_SB, false>(p, dtype, gw, gu, chain_sum,
+                                                                                     num_sms, st);
 }
 
 }  // namespace wkv
