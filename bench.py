@@ -101,8 +101,10 @@ KERNEL_SOURCES = {
 # (workload, kernel, gated, hash of the kernel's code).  A kernel whose code changed
 # since its capture has no entry: its traffic is reported as null.
 TRAFFIC = {
-    ("rwkv1b5_bf16", "bwd_chain_kernel", False, "3d1d96462ca9c9e8"): 453_308_160 + 211_563_520,
-    ("rwkv1b5_bf16", "fwd_chain_kernel", False, "537462e38304278c"): 268_545_536 + 130_038_528,
+    ("rwkv1b5_bf16", "bwd_chain_kernel", False, "1c43104e8adf4cfa"): 453_145_600 + 211_877_632,
+    ("rwkv1b5_bf16", "fwd_chain_kernel", False, "bbe24d138eb5a661"): 268_531_712 + 130_670_336,
+    ("rwkv1b5_bf16", "bwd_chain_kernel", True, "1c43104e8adf4cfa"): 587_395_840 + 345_566_464,
+    ("rwkv1b5_bf16", "fwd_chain_kernel", True, "bbe24d138eb5a661"): 402_737_920 + 130_629_120,
     ("rwkv169m", "bwd_seg_kernel", False, "f3ee2d2581da2ffd"): 77_673_472 + 485_376,
     ("rwkv169m", "fwd_seg_kernel", False, "fbcb48b606b747e2"): 50_391_552 + 1_572_608,
     ("longctx", "fwd_seg_kernel", False, "fbcb48b606b747e2"): 1_454_121_728 + 638_856_704,
