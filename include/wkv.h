@@ -32,9 +32,11 @@
  * - All tensor pointers are DEVICE pointers owned by the caller.  The library
  *   allocates and frees nothing; scratch lives in a caller-provided
  *   workspace.  One exception: wkv_backward_static keeps its scratch in a
- *   file-scope device array of the library (see there), and the library
- *   caches per device the occupancy of its kernels and that array's set-up;
- *   nothing else is kept between calls.
+ *   file-scope device array of the library (see there).  Between calls the
+ *   library caches, per device, the occupancy of its kernels, the TMA
+ *   tensor maps it encoded for recently used buffers (keyed by address,
+ *   shape and element type, so a buffer reused with another shape gets a
+ *   new map) and that array's set-up; nothing else is kept.
  * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *   NULL = legacy default stream).  The return value covers host-side
  *   argument checks and the launch itself; conditions detected on the device
