@@ -311,8 +311,11 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) fwd_chain_kernel(co
           const float e0 = ex2(fmaf(kj[j], kLog2e, -M));
           const float V = Vj[j];
           const float eu = e0 * fc.cu;
-          float yv = fmaf(eu, V, al) * rcp(be + eu);
-          if constexpr (GATE) yv *= gate_sigmoid(Rj[j]);
+          float yv;
+          if constexpr (GATE)  // sigma(r) y = num / (den (1 + 2^{-r log2 e})): one reciprocal for both
+            yv = fmaf(eu, V, al) * rcp((be + eu) * (1.f + ex2(-Rj[j] * kLog2e)));
+          else
+            yv = fmaf(eu, V, al) * rcp(be + eu);
           al = fmaf(al, fc.ewm, e0 * V);
           be = fmaf(be, fc.ewm, e0);
           if (j & 1)

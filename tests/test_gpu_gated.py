@@ -74,7 +74,7 @@ def test_forward_gated_small_shapes(kernel, shape):
     assert state_err(host(s), s_ref) <= F32_FWD_TOL
 
 
-@pytest.mark.parametrize("kernel", ["segment", "chunked"])
+@pytest.mark.parametrize("kernel", ["segment", "chunked", "chain"])
 def test_forward_gated_state_in_and_extreme_gate(kernel):
     B, T, C = 2, 300, 64
     w, u, k, v, r, _, st = gated_case(B, T, C, seed=6, rstd=30.0, state=True)
@@ -131,6 +131,26 @@ def test_backward_gated_state_in(kernel):
     got = W.backward_gated(dev(w), dev(u), dev(k), dev(v), dev(r), dev(g), dev(st),
                            kernel=BWD_KERNELS[kernel])
     assert_grads5(got, oracle.bwd_gated(w, u, k, v, r, g, st), F32_GRAD_TOL)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_gated_chain_kernels_over_more_chains_than_one_wave(dtype):
+    """The gated chain forward and backward with more chains than four warps
+    per SM hold at once (several waves of blocks forward; several chains per
+    warp backward, with the batch rows' dL/dw, dL/du sums meeting)."""
+    B, T, C = 50, 100, 416  # 650 chains, a ragged channel tile
+    w, u, k, v, r, g, _ = gated_case(B, T, C, seed=52, dtype=dtype)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    W_, U_ = dev(w), dev(u)
+    K_, V_, R_, G_ = (dev(x, tdt) for x in (k, v, r, g))
+    o, s, ck = W.forward_gated(W_, U_, K_, V_, R_, want_state=True, want_ckpt=True,
+                               kernel=W.WKV_KERNEL_CHAIN)
+    o_ref, s_ref = oracle.fwd_gated(w, u, k, v, r)
+    tol = BF16_TOL if dtype == "bf16" else F32_FWD_TOL
+    assert fwd_err(host(o), o_ref) <= tol
+    assert state_err(host(s), s_ref) <= F32_FWD_TOL * (10 if dtype == "bf16" else 1)
+    got = W.backward_gated(W_, U_, K_, V_, R_, G_, ckpt=ck, kernel=W.WKV_KERNEL_CHAIN)
+    assert_grads5(got, oracle.bwd_gated(w, u, k, v, r, g), BF16_TOL if dtype == "bf16" else F32_GRAD_TOL)
 
 
 def test_backward_gated_unaligned_gate_input():
