@@ -13,21 +13,24 @@
 // to run, and the joins of a time-parallel scan (summaries, look-backs, a
 // second pass over every token) more than double the instructions per token.
 // Here a chain's state, or its adjoint, is carried from one unit of L tokens
-// to the next in registers.  Per warp, S tile buffers form a TMA ring that
-// keeps S units of input in flight ahead of the arithmetic, and the outputs
-// leave through two staging buffers by TMA stores, so the copy engine, not
-// the warp, moves every byte.  Blocks hold four warps (one per scheduler of
-// an SM) and nothing else is resident beside them.
+// to the next in registers.  A block holds four such compute warps (one per
+// scheduler of an SM) and a fifth warp that issues every TMA copy of the
+// block: per compute warp, S stages of input stay in flight; the compute
+// warp writes its outputs over the inputs it has consumed and signals the
+// stage through an mbarrier; the TMA warp stores them and reloads the stage
+// once the store has read it.  No compute warp ever waits on a copy
+// instruction, and the copy engine, not the warps, moves every byte.
 //
 // Forward, per unit: the recurrence over the unit's tokens, in batches of
 // RB tokens on the batch fast path of wkv_math.cuh where the warp allows it;
 // y, the checkpoints every 16 tokens and the final state are written.
 // Backward, per unit, units last to first: batches of one checkpoint
 // interval, last to first, each from its checkpoint (loaded by TMA with the
-// unit's tiles): recompute, reverse sweep of the adjoint, dL/dk and dL/dv.  dL/dw and dL/du are summed per
-// chain (per unit in float, across units in float64), and the chain of the
-// last batch row of each channel tile adds the B chains in batch-row order:
-// the result is bit-reproducible.
+// unit's tiles): recompute, reverse sweep of the adjoint, dL/dk and dL/dv.
+// dL/dw and dL/du are summed per chain (per unit in float, across units in
+// float64), and the chain of the last batch row of each channel tile adds
+// the B chains in batch-row order: the result is bit-reproducible.
+// GATE variants fuse the output gate o = sigma(r) * y into both.
 #include <cuda.h>
 
 #include "wkv_bwd_math.cuh"
@@ -35,12 +38,15 @@
 #include "wkv_math.cuh"
 #include "wkv_tile.cuh"
 
-// Tokens per batch of the fast paths (build-time knobs).
+// Build-time knobs.  Tokens per batch of the forward's fast path (bf16,
+// ungated; fp32 and gated calls use at most 32):
 #ifndef WKV_CHAIN_FRB
 #define WKV_CHAIN_FRB 64
 #endif
-// Tokens per bf16 unit of the forward and backward, and TMA stages per warp
-// of the backward (the forward takes as many as 48 KB of input per warp hold).
+// tokens per bf16 unit of the forward and the backward, TMA stages per warp
+// of the backward (the forward takes as many stages as 48 KB of input per
+// warp hold), and nanoseconds the TMA warp sleeps between polls that find
+// nothing to do:
 #ifndef WKV_CHAIN_LF
 #define WKV_CHAIN_LF 128
 #endif
@@ -59,9 +65,9 @@ namespace wkv {
 bool encode_btc(CUtensorMap *m, const void *ptr, int dtype, int64_t B, int64_t T, int64_t C, int box_t);
 bool encode_ckpt(CUtensorMap *m, const float *ck, int64_t B, int64_t C, int64_t nck, int box_ck);
 
-constexpr int kChainWarps = 4;  // warps per block: one per scheduler
-// tokens per forward batch: at most a unit (32 tokens for fp32), and at
-// most 32 with the gate (its third input array in registers)
+constexpr int kChainWarps = 4;  // compute warps per block, one per scheduler (and the TMA warp)
+// tokens per forward batch of fp32 calls (a unit of 32 tokens) and of gated
+// calls (their third input array in registers)
 constexpr int kFrbF32 = WKV_CHAIN_FRB < kTileLF32 ? WKV_CHAIN_FRB : kTileLF32;
 constexpr int kChainFwdBytes = 48 * 1024;  // input stages per warp of the forward
 
