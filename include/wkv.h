@@ -124,8 +124,8 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
  *               units by a decoupled look-back over records that carry their
  *               own validity tags (no fences), and, in the forward, runs the
  *               next unit's first pass before the current unit's join.
- *               CHAIN (16-byte aligned rows; the backward without the
- *               state terms) gives each warp whole chains, run in
+ *               CHAIN (16-byte aligned rows) gives each warp whole chains,
+ *               run in
  *               time order from a ring of TMA tiles with the state (or the
  *               adjoint) carried in registers: no joins and a single pass
  *               over every token, for problems whose chains alone fill the

@@ -352,7 +352,7 @@ int backward_impl(int64_t B, int64_t T, int64_t C, int dtype, const float *w, co
   const int kernel = opt ? opt->kernel : WKV_KERNEL_AUTO;
   const bool bwd_tma = bwd_uses_seg(B, T, C, dtype, k, v, grad_y, nullptr) && aligned(grad_k, 16) &&
                        aligned(grad_v, 16);
-  if (!sg.gs_out && !sg.gs_in && (!r || (aligned(r, 16) && aligned(gr, 16))) && bwd_tma && aligned(ck, 16) &&
+  if ((!r || (aligned(r, 16) && aligned(gr, 16))) && bwd_tma && aligned(ck, 16) &&
       (kernel == WKV_KERNEL_CHAIN || (kernel == WKV_KERNEL_AUTO && chain_pays(L.nchains)))) {
     float4 *sums = reinterpret_cast<float4 *>(base + L.sums);
     return cuda_rc(launch_backward_chain(a, dtype, grad_w, grad_u, sums, num_sms(), st));

@@ -442,7 +442,12 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *map, int x
 // backward's gate, wkv_tile_bwd.cu): r arrives with k, v and grad_o, the
 // WKV gradient is grad_o sigma(r), and dL/dr = grad_o sigma'(r) y from the
 // recomputed y overwrites r and leaves with dL/dk and dL/dv.
-template <typename E, int L, int RB, int S, bool GATE>
+// STATE: the state terms of a sequence split across calls (as the tile
+// backward's): a chain's adjoint starts from the final state's gradient,
+// its last batch sweeps exactly to token T-1 (the zero-filled padding would
+// decay that adjoint), and its first unit writes the initial state's
+// gradient.
+template <typename E, int L, int RB, int S, bool GATE, bool STATE>
 __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                         const __grid_constant__ CUtensorMap vmap,
                                                                         const __grid_constant__ CUtensorMap gmap,
@@ -453,6 +458,7 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
                                                                         const __grid_constant__ CUtensorMap grmap,
                                                                         ChainBwdArgs a) {
   static_assert(L % kCkpt == 0 && RB == kCkpt, "batches are checkpoint intervals");
+  static_assert(!(STATE && GATE), "no entry point combines the state terms and the gate");
   constexpr int NB = L / RB;
   constexpr int NARR = GATE ? 4 : 3;  // k, v, grad_y (and r)
   constexpr int CKB = NB * 96 * 4;    // the unit's checkpoints
@@ -472,7 +478,7 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
   __syncthreads();
   const int G = (int)gridDim.x * kChainWarps;
   const int nchains = (int)p.nchains, nct = (int)p.nct;
-  const int64_t T = p.T, C = p.C;
+  const int64_t T = p.T, C = p.C, BC = p.B * p.C;
   const int nseg = (int)((T + L - 1) / L);
   const int64_t budget = p.spin_limit * 1000;
   unsigned epoch = 0;
@@ -609,6 +615,9 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
       Ranc = kEmptyR;
       m = 0.f;
       gw_d = gu_d = 0.0;
+      if constexpr (STATE) {
+        if (p.gs_out && cok) end_adjoint(p.gs_out[bc], p.gs_out[BC + bc], p.p_out[bc], rah, rhh, Ranc);
+      }
     }
     if (!__all_sync(0xffffffffu, mbar_wait(full(wl, s), (uint32_t)(j / S) & 1u, budget, nullptr))) {
       failed = true;
@@ -670,7 +679,8 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
       // token with the running anchor
       const float rn_end = fmaf(-m, w2, Ranc);
       const float xin = fmaf((float)RB, fc.w2e, Mb) - rn_end;
-      if (__all_sync(0xffffffffu, fast && xin < 100.f)) {
+      const int nv = n - bt * RB;  // rows of the batch inside T
+      if (__all_sync(0xffffffffu, fast && xin < 100.f && (!STATE || nv >= RB))) {
         const float F = ex2(xin);
         float ra = rah * F, rh = rhh * F, rap = rahp * F, rhp = rhhp * F;
         const float ckf = fc.cw * ex2(-u2);  // ek = e2 * ckf
@@ -701,6 +711,7 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
       }
 #pragma unroll
       for (int q = RB - 1; q >= 0; --q) {
+        if (STATE && q >= nv) continue;  // past T
         const float rn = fmaf(-m, w2, Ranc);  // scale of the adjoint after token t
         const float tn = ex2(K[q] - rn);      // e^{k_t} 2^{-r_{t+1}} (<= 1)
         const float gv = fmaf(gam[q], e2v[q], tn * rah);
@@ -727,6 +738,9 @@ __global__ void __launch_bounds__((kChainWarps + 1) * 32, 1) bwd_chain_kernel(co
       // checkpoint before token 0
       const float r0 = fmaf(-m, w2, Ranc);
       gw_acc = fmaf(ex2(sts[64 + lane] - r0), fmaf(sts[lane], rahp, -sts[32 + lane] * rhhp), gw_acc);
+      if constexpr (STATE) {
+        if (p.gs_in) store_state_grad(p.gs_in, p.state_in, bc, BC, rah, rhh, r0);
+      }
     }
     gw_d += (double)gw_acc;
     gu_d += (double)gu_acc;
@@ -782,7 +796,7 @@ cudaError_t launch_forward_chain(const FwdArgs &f, int dtype, cudaStream_t st) {
                     : launch_fwd_chain_t<uint16_t, WKV_CHAIN_LF, WKV_CHAIN_FRB, false>(f, dtype, st);
 }
 
-template <typename E, int L, int RB, int S, bool GATE>
+template <typename E, int L, int RB, int S, bool GATE, bool STATE>
 static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *chain_sum,
                                       int num_sms, cudaStream_t st) {
   CUtensorMap km, vm, gm, rm, ckm, gkm, gvm, grm;
@@ -798,7 +812,7 @@ static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, fl
     return cudaErrorInvalidValue;
   // the compute warps' stages, then two barriers per stage and warp
   constexpr int smem = kChainWarps * (ChainLayout<E, L, GATE ? 4 : 3, 0, S, 0, NB * 96 * 4>::WARP + 16 * S);
-  auto kern = bwd_chain_kernel<E, L, RB, S, GATE>;
+  auto kern = bwd_chain_kernel<E, L, RB, S, GATE, STATE>;
   int occ = 0;
   cudaError_t e = blocks_per_sm((const void *)kern, (kChainWarps + 1) * 32, smem, &occ);
   if (e != cudaSuccess) return e;
@@ -822,15 +836,21 @@ static cudaError_t launch_bwd_chain_t(const BwdArgs &p, int dtype, float *gw, fl
 
 cudaError_t launch_backward_chain(const BwdArgs &p, int dtype, float *gw, float *gu, float4 *chain_sum, int num_sms,
                                   cudaStream_t st) {
-  if (p.gs_out || p.gs_in) return cudaErrorInvalidValue;  // no state terms
+  if (p.r && (p.gs_out || p.gs_in)) return cudaErrorInvalidValue;  // no entry point asks for both
   if (p.r)  // the gate's fourth tile per stage: 64-token units (32 fp32), three stages
-    return dtype == 0
-               ? launch_bwd_chain_t<float, kTileLF32, kCkpt, 3, true>(p, dtype, gw, gu, chain_sum, num_sms, st)
-               : launch_bwd_chain_t<uint16_t, kTileLBF16, kCkpt, 3, true>(p, dtype, gw, gu, chain_sum, num_sms, st);
-  return dtype == 0
-             ? launch_bwd_chain_t<float, kTileLF32, kCkpt, WKV_CHAIN_SB, false>(p, dtype, gw, gu, chain_sum, num_sms, st)
-             : launch_bwd_chain_t<uint16_t, WKV_CHAIN_LB, kCkpt, WKV_CHAIN_SB, false>(p, dtype, gw, gu, chain_sum,
-                                                                                     num_sms, st);
+    return dtype == 0 ? launch_bwd_chain_t<float, kTileLF32, kCkpt, 3, true, false>(p, dtype, gw, gu, chain_sum,
+                                                                                      num_sms, st)
+                      : launch_bwd_chain_t<uint16_t, kTileLBF16, kCkpt, 3, true, false>(p, dtype, gw, gu, chain_sum,
+                                                                                         num_sms, st);
+  if (p.gs_out || p.gs_in)
+    return dtype == 0 ? launch_bwd_chain_t<float, kTileLF32, kCkpt, WKV_CHAIN_SB, false, true>(p, dtype, gw, gu,
+                                                                                                 chain_sum, num_sms, st)
+                      : launch_bwd_chain_t<uint16_t, WKV_CHAIN_LB, kCkpt, WKV_CHAIN_SB, false, true>(
+                            p, dtype, gw, gu, chain_sum, num_sms, st);
+  return dtype == 0 ? launch_bwd_chain_t<float, kTileLF32, kCkpt, WKV_CHAIN_SB, false, false>(p, dtype, gw, gu,
+                                                                                                chain_sum, num_sms, st)
+                    : launch_bwd_chain_t<uint16_t, WKV_CHAIN_LB, kCkpt, WKV_CHAIN_SB, false, false>(
+                          p, dtype, gw, gu, chain_sum, num_sms, st);
 }
 
 }  // namespace wkv

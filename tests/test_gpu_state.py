@@ -73,6 +73,22 @@ def test_backward_state_small_shapes(shape, use_ckpt, kernel):
     assert_grads_state(got, ref, F32_GRAD_TOL)
 
 
+@pytest.mark.parametrize("T", [100, 129])
+def test_chain_state_backward_over_more_chains_than_one_wave(T):
+    """The chain backward's state terms with more chains than four warps per
+    SM hold at once: warps run several chains, each starting from its own
+    final-state gradient; T = 129 ends in a one-token batch that must not
+    sweep the zero-filled rows after it."""
+    B, C = 50, 416  # 650 chains, a ragged channel tile
+    w, u, k, v, g, s_in, s_out, gso = state_case(B, T, C, seed=T + 3)
+    a = (dev(w), dev(u), dev(k), dev(v))
+    _, _, ck = W.forward(*a, dev(s_in), want_ckpt=True)
+    got = W.backward_state(*a, dev(g), dev(s_in), ck, state_out=dev(s_out), grad_state_out=dev(gso),
+                           kernel=W.WKV_KERNEL_CHAIN)
+    ref = oracle.bwd_state(w, u, k, v, g, s_in, s_out, gso)
+    assert_grads_state(got, ref, F32_GRAD_TOL)
+
+
 @pytest.mark.parametrize("kernel", sorted(BWD_KERNELS))
 def test_state_in_gradient_without_final_state_term(kernel):
     B, T, C = 2, 300, 64
