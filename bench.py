@@ -67,13 +67,13 @@ BWD_PLAN = {"tile": ("bwd_tile_kernel", 1), "segment": ("bwd_seg_kernel", 1), "c
 def auto_kernel(op: str, B: int, C: int, gate: bool, num_sms: int = 148) -> str:
     """The kernel the library's AUTO selector runs on 16-byte aligned rows of
     at least one tile unit (mirrors chain_pays and tile_pays in the C ABI):
-    the chain kernels when the chains (batch row, 32 channels) fill three
-    quarters or more of the warp schedulers in one wave; else the tile
+    the chain kernels when the chains (batch row, 32 channels) occupy 60 %
+    or more of the warp schedulers (in one wave or several); else the tile
     kernels when a chain has at most about four resident warps' units in
     flight; else the segment kernels."""
     nchains = B * ((C + 31) // 32)
     slots = 4 * num_sms
-    if nchains * 4 >= slots * 3 and nchains <= slots:
+    if nchains * 5 >= slots * 3:
         return "chain"
     warps = (6 if gate else 9) if op == "fwd" else (6 if gate else 8)
     return "tile" if nchains * 4 >= warps * num_sms else "segment"

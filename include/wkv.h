@@ -131,11 +131,10 @@ enum { WKV_KERNEL_AUTO = 0, WKV_KERNEL_SEQUENTIAL = 1, WKV_KERNEL_CHUNKED = 2,
  *               over every token, for problems whose chains alone fill the
  *               GPU's warp schedulers; where it does not apply, the call
  *               runs TILE.  AUTO runs CHAIN on 16-byte aligned rows when the
- *               chains (batch rows x 32-channel tiles) number from three
- *               quarters of to all the warp schedulers (4 per SM), else TILE
- *               when a chain has at most about four resident warps' units in
- *               flight, else SEGMENT, and the chunked kernels on unaligned
- *               rows.  Values 4 and 5 are retired and rejected with
+ *               chains (batch rows x 32-channel tiles) number 60 % or more
+ *               of the warp schedulers (4 per SM), else TILE when a chain
+ *               has at most about four resident warps' units in flight, else
+ *               SEGMENT, and the chunked kernels on unaligned rows.  Values 4 and 5 are retired and rejected with
  *               WKV_ERR_INVALID_ARG.
  *   spin_limit  bound on any one device-side wait (a predecessor's record,
  *               a shared-memory load, the grid barrier) in microseconds (the

@@ -146,13 +146,17 @@ int num_sms() {
 // amortise their joins better.  warps_per_sm: resident warps of the kernel.
 bool tile_pays(int64_t nchains, int warps_per_sm) { return nchains * 4 >= (int64_t)warps_per_sm * num_sms(); }
 
-// AUTO picks the chain kernels when the chains alone come close to filling
-// the warp schedulers (four per SM, one chain each) in one wave: from three
-// quarters of them up.  With fewer, the idle schedulers cost more than the
-// time-parallel kernels' joins.
+// AUTO picks the chain kernels when the chains (one per warp scheduler, four
+// per SM) occupy at least 60 % of the schedulers; with more chains than one
+// wave holds they run in waves.  Measured on B200 (bf16, T 4096, forward /
+// backward): 384 chains 128 / 227 us against the tile kernels' 165 / 293;
+// 640 chains 222 / 410 against 239 / 439; 1024 chains 222 / 413 against
+// 375 / 625.  With fewer chains the idle schedulers cost more than the
+// time-parallel kernels' joins (192 chains, fp32 T 1024: 41 / 91 us against
+// the segment kernels' 29 / 52).
 bool chain_pays(int64_t nchains) {
   const int64_t slots = 4 * (int64_t)num_sms();
-  return nchains * 4 >= slots * 3 && nchains <= slots;
+  return nchains * 5 >= slots * 3;
 }
 
 bool pick_chunked(const wkv_options *opt, int64_t B, int64_t T, int64_t C) {

@@ -12,23 +12,24 @@ from rwkv_linear_rnn_b200 import workloads
 @pytest.mark.parametrize("op", ["fwd", "bwd"])
 @pytest.mark.parametrize("gate", [False, True])
 def test_auto_kernel_on_the_workload_shapes(op, gate):
-    """The 1.5B-shaped layer (512 chains) fills three quarters or more of the
-    148 x 4 warp schedulers: chain kernels.  The 169M-shaped layer (192
+    """The 1.5B-shaped layer (512 chains) occupies 60 % or more of the 148 x 4
+    warp schedulers: chain kernels.  The 169M-shaped layer (192
     chains) and the long sequence (80 chains) do not."""
     assert bench.auto_kernel(op, 8, 2048, gate) == "chain"
     assert bench.auto_kernel(op, 8, 768, gate) in ("tile", "segment")
     assert bench.auto_kernel(op, 1, 2560, gate) == "segment"
 
 
-def test_auto_kernel_chain_window():
-    """444..592 chains on 148 SMs run the chain kernels; one more chain than
-    a wave of one warp per scheduler does not."""
+def test_auto_kernel_chain_threshold():
+    """From 60 % of the 148 x 4 warp schedulers up (356 chains), in one wave
+    or several, the chain kernels run; below it, the time-parallel ones."""
     slots = 4 * 148
-    lo = (3 * slots + 3) // 4  # the fewest chains with chains * 4 >= 3 * slots
+    lo = (3 * slots + 4) // 5  # the fewest chains with chains * 5 >= 3 * slots
+    assert lo == 356
     assert bench.auto_kernel("fwd", lo, 32, False) == "chain"
     assert bench.auto_kernel("fwd", lo - 1, 32, False) != "chain"
     assert bench.auto_kernel("fwd", slots, 32, False) == "chain"
-    assert bench.auto_kernel("fwd", slots + 1, 32, False) != "chain"
+    assert bench.auto_kernel("bwd", 3 * slots + 7, 32, True) == "chain"
     # a ragged channel tile counts as a chain
     assert bench.auto_kernel("bwd", 1, 32 * lo - 31, False) == "chain"
 
