@@ -101,10 +101,10 @@ KERNEL_SOURCES = {
 # (workload, kernel, gated, hash of the kernel's code).  A kernel whose code changed
 # since its capture has no entry: its traffic is reported as null.
 TRAFFIC = {
-    ("rwkv1b5_bf16", "bwd_chain_kernel", False, "9cf1c472d134bfbe"): 453_355_776 + 212_812_800,
-    ("rwkv1b5_bf16", "fwd_chain_kernel", False, "827012a8fd427e8f"): 268_525_056 + 131_096_576,
-    ("rwkv1b5_bf16", "bwd_chain_kernel", True, "9cf1c472d134bfbe"): 587_434_752 + 345_717_504,
-    ("rwkv1b5_bf16", "fwd_chain_kernel", True, "827012a8fd427e8f"): 402_733_824 + 132_948_224,
+    ("rwkv1b5_bf16", "bwd_chain_kernel", False, "dd3bb205f2bafacc"): 453_355_776 + 212_812_800,
+    ("rwkv1b5_bf16", "fwd_chain_kernel", False, "f67c813868e39fed"): 268_525_056 + 131_096_576,
+    ("rwkv1b5_bf16", "bwd_chain_kernel", True, "dd3bb205f2bafacc"): 587_434_752 + 345_717_504,
+    ("rwkv1b5_bf16", "fwd_chain_kernel", True, "f67c813868e39fed"): 402_733_824 + 132_948_224,
     ("rwkv169m", "bwd_seg_kernel", False, "f3ee2d2581da2ffd"): 77_673_472 + 485_376,
     ("rwkv169m", "fwd_seg_kernel", False, "fbcb48b606b747e2"): 50_391_552 + 1_572_608,
     ("longctx", "fwd_seg_kernel", False, "fbcb48b606b747e2"): 1_454_121_728 + 638_856_704,

@@ -143,9 +143,6 @@ __device__ __forceinline__ bool mbar_wait_sleepy(uint32_t bar, uint32_t parity, 
 #endif
 }
 
-// Wait until at most one bulk store group of this thread still reads its
-// shared memory (the most recent one).
-__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 
 // Per warp: S input stages of NARR tiles [L][32] (and XST bytes more),
 // NOUT output tiles twice (double-buffered staging), STS bytes of scratch;
